@@ -1,0 +1,202 @@
+"""CSA2 decode step with the Hierarchical Sparse Indexer, in float64.
+
+Test infrastructure: see the package docstring for who may import this.
+
+What the pages fix, and the readings taken where they are silent:
+
+* Layer modes [readance summary of the DeepSeek-V4.1-Flash report, section 4.2;
+  4sapi blog, section 二 CSA2 (mode table)]: Full computes its own main KV and
+  indexer K and picks its own Top-K; Reindex reuses that KV and indexer K but
+  re-scores with its own indexer Q; Reuse takes main KV and Top-K indices as
+  they are.
+* Indexer shape [4sapi blog, section 四 Hierarchical Sparse Indexer]: 32 query
+  heads of dim 128, Top-512 per query.
+* Hierarchical pool [same section; alphalab analysis, section 2 CSA2]: the first
+  Full layer scans the whole visible context and keeps 2048 blocks of 8
+  positions (16,384 candidates); Reindex layers choose their Top-512 inside it.
+* Score function (reading, unpinned against DeepSeek's model):
+  s_t = sigma_t * sum_h w_h * ReLU(sigma^q_h * <q_h, k_t>) over FP8 codes.
+* Block score (reading, unpinned): the max of the <= 8 visible scores of the
+  block.  Ties in every selection go to the lower index (reading).
+* Selections are returned sorted ascending, padded with -1.
+* Attention (reading of "sparse attention over the gathered Top-K" with the
+  512-d shared K=V latent): o_h = sum_i softmax_i(q_h . v_i * scale) v_i over the
+  dequantised rows of the valid indices; no valid index gives o = 0.
+
+Every inner product of two FP8 values is exact in float64 (each product has at
+most 8 significant bits and every partial sum is a multiple of 2^-18 below
+2^25), so the dot products below are exact whatever the summation order.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+from .formats import (dequantize_main_kv, e4m3_value, indexer_sigma,
+                      quantize_indexer)
+
+INDEX_HEADS = 32
+BLOCK = 8            # positions per pool block
+POOL_BLOCKS = 2048   # blocks kept by the first Full layer
+TOPK = 512
+
+
+# ------------------------------------------------------------------ scores ---
+
+def quantize_index_query(q):
+    """Indexer query q[32,128] (fp32) -> (codes [32,128], sigma^q [32]) with the
+    same per-row power-of-two FP8 rule as the cached indexer K."""
+    codes, exp = quantize_indexer(q)
+    return codes, indexer_sigma(exp)
+
+
+def indexer_scores(q, w, ik_codes, ik_exp, chunk: int = 1 << 16) -> np.ndarray:
+    """Full-mode score of every given row for one query.
+
+    q: [32,128] fp32 indexer query; w: [32] head weights;
+    ik_codes: [N,128] uint8 E4M3; ik_exp: [N] uint8 exponent bytes.
+    Returns s[N] float64 with s_t = sigma_t * sum_h w_h ReLU(sigma^q_h <q^_h, k^_t>).
+    """
+    qc, sq = quantize_index_query(q)
+    qv = e4m3_value(qc)                        # [32,128]
+    w = np.asarray(w, dtype=np.float32).astype(np.float64)
+    n = len(ik_codes)
+    out = np.empty(n, dtype=np.float64)
+    for a in range(0, n, chunk):
+        kv = e4m3_value(ik_codes[a:a + chunk])     # [c,128]
+        dots = kv @ qv.T                           # [c,32], exact
+        relu = np.maximum(dots * sq, 0.0)
+        out[a:a + chunk] = indexer_sigma(ik_exp[a:a + chunk]) * (relu @ w)
+    return out
+
+
+def block_max(scores, n: int | None = None) -> np.ndarray:
+    """m_j = max of the visible scores of block j (positions 8j..8j+7, < n)."""
+    s = np.asarray(scores, dtype=np.float64)
+    n = len(s) if n is None else n
+    nb = -(-n // BLOCK)
+    pad = np.full(nb * BLOCK, -np.inf)
+    pad[:n] = s[:n]
+    return pad.reshape(nb, BLOCK).max(axis=1)
+
+
+# ------------------------------------------------------------- selections ---
+
+def top_k_ascending(cand_ids, cand_scores, k: int) -> np.ndarray:
+    """The k candidates with the largest score (ties: lower id first), returned
+    sorted ascending and padded with -1 to length k."""
+    cand_ids = np.asarray(cand_ids, dtype=np.int64)
+    cand_scores = np.asarray(cand_scores, dtype=np.float64)
+    order = np.lexsort((cand_ids, -cand_scores))   # by -score, then by id
+    sel = np.sort(cand_ids[order[:k]])
+    out = np.full(k, -1, dtype=np.int64)
+    out[:len(sel)] = sel
+    return out
+
+
+def pool_select(blockmax, pool_blocks: int = POOL_BLOCKS) -> np.ndarray:
+    """Top-`pool_blocks` block ids by block max, ascending, -1 padded.  With at
+    most `pool_blocks` blocks the pool is every block."""
+    m = np.asarray(blockmax, dtype=np.float64)
+    return top_k_ascending(np.arange(len(m)), m, pool_blocks)
+
+
+def pool_positions(pool, n: int) -> np.ndarray:
+    """Expand pool block ids into the visible positions they cover (ascending)."""
+    pool = np.asarray(pool, dtype=np.int64)
+    blocks = pool[pool >= 0]
+    pos = (blocks[:, None] * BLOCK + np.arange(BLOCK)[None, :]).reshape(-1)
+    return pos[pos < n]
+
+
+def full_topk(scores, pool, n: int, k: int = TOPK) -> np.ndarray:
+    """Full-mode Top-k: the best k of the Full scan's scores among the
+    candidates (the pool's positions, or all n positions when pool is None)."""
+    scores = np.asarray(scores, dtype=np.float64)
+    cand = np.arange(n) if pool is None else pool_positions(pool, n)
+    return top_k_ascending(cand, scores[cand], k)
+
+
+def reindex_topk(q, w, ik_codes, ik_exp, pool, n: int, k: int = TOPK) -> np.ndarray:
+    """Reindex-mode Top-k: re-score only the candidates (pool positions, or all
+    n positions when pool is None) with this layer's own q, w."""
+    cand = np.arange(n) if pool is None else pool_positions(pool, n)
+    s = indexer_scores(q, w, ik_codes[cand], ik_exp[cand])
+    return top_k_ascending(cand, s, k)
+
+
+def reuse_topk(prev_topk) -> np.ndarray:
+    """Reuse mode: the previous layer's Top-k indices, unchanged."""
+    return np.array(prev_topk, copy=True)
+
+
+# --------------------------------------------------------------- attention --
+
+def sparse_attention(q_main, kv_codes, kv_scales, idx, scale: float) -> np.ndarray:
+    """Sparse MQA attention for one query over the rows `idx` (-1 = skip).
+
+    q_main: [H,512] (bf16 values); kv_codes/kv_scales: the whole request's main
+    KV ([N,256] / [N,32]); K = V = the dequantised row.  Returns float64 [H,512].
+    """
+    q = np.asarray(q_main, dtype=np.float64)
+    idx = np.asarray(idx, dtype=np.int64)
+    idx = idx[idx >= 0]
+    if len(idx) == 0:
+        return np.zeros_like(q)
+    rows = dequantize_main_kv(kv_codes[idx], kv_scales[idx])   # [n,512]
+    logits = (q @ rows.T) * scale
+    logits -= logits.max(axis=1, keepdims=True)
+    p = np.exp(logits)
+    p /= p.sum(axis=1, keepdims=True)
+    return p @ rows
+
+
+# ------------------------------------------------------------ decode group ---
+
+def decode_group(modes, q_idx, w_idx, ik_codes, ik_exp, n: int,
+                 pool_blocks: int | None = POOL_BLOCKS, k: int = TOPK):
+    """Index selection of one decode query through a CSA2 layer group.
+
+    modes: sequence of "F", "Ri", "Ru" (the first must be "F");
+    q_idx / w_idx: per-layer indexer query and head weights (ignored for "Ru");
+    ik_codes / ik_exp: the request's cached indexer K for positions [0, n).
+    pool_blocks None means no hierarchical pool (Top-k over the whole context).
+
+    Returns dict(scores, blockmax, pool, topk=[per layer]).  The pool is built
+    by the first Full layer; a later Full layer would start a new pool.
+    """
+    out = {"topk": []}
+    pool = None
+    prev = None
+    for layer, mode in enumerate(modes):
+        if mode == "F":
+            s = indexer_scores(q_idx[layer], w_idx[layer], ik_codes[:n], ik_exp[:n])
+            bm = block_max(s, n)
+            pool = None if pool_blocks is None else pool_select(bm, pool_blocks)
+            t = full_topk(s, pool, n, k)
+            out.setdefault("scores", s)
+            out.setdefault("blockmax", bm)
+            out.setdefault("pool", pool)
+        elif mode == "Ri":
+            t = reindex_topk(q_idx[layer], w_idx[layer], ik_codes, ik_exp, pool, n, k)
+        elif mode == "Ru":
+            t = reuse_topk(prev)
+        else:
+            raise ValueError(f"unknown mode {mode!r}")
+        out["topk"].append(t)
+        prev = t
+    return out
+
+
+# ----------------------------------------------------------- causal prefill --
+
+def prefill_visible(p: int) -> int:
+    """Entries visible to the query at token p when entry e covers tokens 2e
+    and 2e+1 (m = 2): e is visible iff 2e + 1 <= p, i.e. floor((p + 1) / 2)."""
+    return (p + 1) // 2
+
+
+def prefill_topk(q, w, ik_codes, ik_exp, p: int, k: int = TOPK) -> np.ndarray:
+    """Top-k of one prefill query at token p over its visible entries (no pool)."""
+    v = min(prefill_visible(p), len(ik_codes))
+    s = indexer_scores(q, w, ik_codes[:v], ik_exp[:v])
+    return top_k_ascending(np.arange(v), s, k)

@@ -1,0 +1,251 @@
+"""Pins of the oracle's CSA2 step: closed forms and special cases of the score,
+brute-force selection on tiny inputs, the invariants the pages fix
+(hierarchical pool == flat Top-k while the context fits the pool; Reindex and
+Full Top-k inside the pool; Reuse == the previous indices), and sparse
+attention against torch's dense scaled-dot-product attention."""
+import json
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import csa2 as C
+from oracle import formats as F
+
+
+def _idx_rows(rng, n):
+    k = rng.standard_normal((n, 128)).astype(np.float32)
+    return F.quantize_indexer(k)
+
+
+def _query(rng):
+    return rng.standard_normal((32, 128)).astype(np.float32), rng.random(32).astype(np.float32)
+
+
+# ------------------------------------------------------------------- score --
+
+def test_score_reduces_to_plain_formula_when_quantisation_is_identity():
+    """Rows already on the E4M3 grid with amax exactly 448 quantise to
+    themselves with sigma = 1: the score is then the plain float64 formula
+    sum_h w_h ReLU(q_h . k_t), evaluated here with torch (library)."""
+    rng = np.random.default_rng(0)
+    grid = F.e4m3_value(rng.integers(0, 127, (64, 128)) | (rng.integers(0, 2, (64, 128)) << 7))
+    grid[:, 0] = 448.0
+    k = grid[:40].astype(np.float32)
+    q = grid[40:72 - 8].astype(np.float32)
+    q = np.concatenate([q, grid[:8]]).astype(np.float32)
+    w = rng.random(32).astype(np.float32)
+    codes, byte = F.quantize_indexer(k)
+    assert np.all(byte == 127)
+    ours = C.indexer_scores(q, w, codes, byte)
+    ref = torch.relu(torch.from_numpy(k).double() @ torch.from_numpy(q).double().T) @ torch.from_numpy(w).double()
+    np.testing.assert_allclose(ours, ref.numpy(), rtol=1e-15)
+
+
+def test_score_one_hot_closed_form():
+    """q = one-hot at (head h, dim d), w = e_h: s_t = ReLU(k~_{t,d}) * 448 * sigma^q
+    with q's element quantised to 448."""
+    rng = np.random.default_rng(1)
+    codes, byte = _idx_rows(rng, 50)
+    kd = F.dequantize_indexer(codes, byte)
+    for h, d in [(0, 0), (7, 99), (31, 127)]:
+        q = np.zeros((32, 128), np.float32)
+        q[h, d] = 3.0                       # sigma^q = 2^-7, q^ = 384 -> q~ = 3
+        w = np.zeros(32, np.float32)
+        w[h] = 1.0
+        np.testing.assert_array_equal(C.indexer_scores(q, w, codes, byte), np.maximum(kd[:, d], 0) * 3.0)
+
+
+def test_score_structure():
+    rng = np.random.default_rng(2)
+    codes, byte = _idx_rows(rng, 300)
+    q, w = _query(rng)
+    s = C.indexer_scores(q, w, codes, byte)
+    assert np.all(s >= 0)
+    # linear in w
+    w2 = rng.random(32).astype(np.float32)
+    np.testing.assert_allclose(C.indexer_scores(q, w + w2, codes, byte),
+                               s + C.indexer_scores(q, w2, codes, byte), rtol=1e-6)
+    # power-of-two scaling of q keeps the codes and scales the score
+    np.testing.assert_allclose(C.indexer_scores(q * 4, w, codes, byte), 4 * s, rtol=1e-15)
+    # ReLU: s(q) + s(-q) = sum_h w_h |q~_h . k~_t| (closed form of the two halves)
+    qc, sq = C.quantize_index_query(q)
+    kd = F.dequantize_indexer(codes, byte)
+    absdot = np.abs(kd @ (F.e4m3_value(qc) * sq[:, None]).T) @ w.astype(np.float64)
+    np.testing.assert_allclose(s + C.indexer_scores(-q, w, codes, byte), absdot, rtol=1e-12)
+    # each row scored on its own: permuting rows permutes scores
+    perm = rng.permutation(300)
+    np.testing.assert_array_equal(C.indexer_scores(q, w, codes[perm], byte[perm]), s[perm])
+
+
+def test_block_max_bruteforce():
+    rng = np.random.default_rng(3)
+    for n in [1, 7, 8, 9, 63, 64, 100]:
+        s = rng.random(n + 5)
+        bm = C.block_max(s, n)
+        ref = [max(s[j * 8:min(j * 8 + 8, n)]) for j in range(-(-n // 8))]
+        assert list(bm) == ref
+
+
+# -------------------------------------------------------------- selections --
+
+def _brute_topk(ids, scores, k):
+    """Repeatedly take the best remaining candidate (highest score, then lowest id)."""
+    left = list(zip(ids, scores))
+    taken = []
+    while left and len(taken) < k:
+        best = max(left, key=lambda t: (t[1], -t[0]))
+        taken.append(best[0])
+        left.remove(best)
+    return sorted(taken) + [-1] * (k - len(taken))
+
+
+def test_topk_bruteforce_with_ties():
+    rng = np.random.default_rng(4)
+    for n, k in [(10, 3), (40, 16), (64, 64), (20, 30), (0, 4)]:
+        ids = np.sort(rng.choice(1000, n, replace=False))
+        scores = rng.integers(0, 6, n).astype(np.float64)      # many ties
+        assert list(C.top_k_ascending(ids, scores, k)) == _brute_topk(list(ids), list(scores), k)
+    # ties straddling the cut: equal scores everywhere, and a two-level case
+    ids = np.arange(10) * 3
+    assert list(C.top_k_ascending(ids, np.ones(10), 4)) == [0, 3, 6, 9]
+    sc = np.array([1, 2, 2, 1, 2, 1, 2, 2, 1, 1], dtype=np.float64)
+    assert list(C.top_k_ascending(ids, sc, 3)) == _brute_topk(list(ids), list(sc), 3) == [3, 6, 12]
+
+
+def test_pool_bruteforce_tiny():
+    rng = np.random.default_rng(5)
+    s = rng.integers(0, 3, 64).astype(np.float64)           # block maxima tie across the cut
+    bm = C.block_max(s, 64)
+    pool = C.pool_select(bm, 4)
+    blocks = sorted(range(8), key=lambda j: (-max(s[8 * j:8 * j + 8]), j))[:4]
+    assert list(pool) == sorted(blocks)
+    pos = C.pool_positions(pool, 64)
+    assert list(pos) == [8 * j + i for j in sorted(blocks) for i in range(8)]
+
+
+def test_pool_is_every_block_when_context_fits():
+    rng = np.random.default_rng(6)
+    for n in [1, 4095, 16384]:
+        pool = C.pool_select(C.block_max(rng.random(n), n))
+        nb = -(-n // 8)
+        assert list(pool[:nb]) == list(range(nb)) and np.all(pool[nb:] == -1)
+
+
+def test_hierarchical_equals_flat_up_to_pool_size():
+    """ctx <= 16384: every block is in the pool, so the group with the pool
+    selects exactly what it would select with no pool at all."""
+    rng = np.random.default_rng(7)
+    n = 16384
+    codes, byte = _idx_rows(rng, n)
+    qs, ws = zip(*[_query(rng) for _ in range(3)])
+    modes = ("F", "Ri", "Ru")
+    a = C.decode_group(modes, qs, ws, codes, byte, n, pool_blocks=2048)
+    b = C.decode_group(modes, qs, ws, codes, byte, n, pool_blocks=None)
+    for ta, tb in zip(a["topk"], b["topk"]):
+        np.testing.assert_array_equal(ta, tb)
+
+
+def test_group_invariants_with_pool():
+    """Beyond the pool size: Full Top-k equals the flat Top-k (block max keeps
+    every Top-512 position's block), Reindex Top-k lies inside the pool, Reuse
+    repeats its predecessor."""
+    rng = np.random.default_rng(8)
+    n = 40000
+    codes, byte = _idx_rows(rng, n)
+    qs, ws = zip(*[_query(rng) for _ in range(6)])
+    modes = ("F", "Ri", "Ri", "Ru", "Ru", "Ru")
+    out = C.decode_group(modes, qs, ws, codes, byte, n, pool_blocks=256, k=64)
+    pool_pos = set(C.pool_positions(out["pool"], n))
+    flat = C.top_k_ascending(np.arange(n), out["scores"], 64)
+    np.testing.assert_array_equal(out["topk"][0], flat)
+    for t in out["topk"]:
+        assert set(t[t >= 0]) <= pool_pos
+    for l in (3, 4, 5):
+        np.testing.assert_array_equal(out["topk"][l], out["topk"][2])
+    # Reindex differs from a flat re-scan only through the pool restriction
+    flat1 = C.top_k_ascending(np.arange(n), C.indexer_scores(qs[1], ws[1], codes, byte), 64)
+    inside = np.isin(flat1, list(pool_pos))
+    assert set(flat1[inside]) <= set(out["topk"][1])
+
+
+def test_topk_pads_short_context():
+    rng = np.random.default_rng(9)
+    codes, byte = _idx_rows(rng, 100)
+    q, w = _query(rng)
+    t = C.decode_group(("F",), [q], [w], codes, byte, 100, pool_blocks=None)["topk"][0]
+    assert list(t[:100]) == list(range(100)) and np.all(t[100:] == -1)
+
+
+# --------------------------------------------------------------- attention --
+
+def _kv(rng, n):
+    x = (rng.standard_normal((n, 512)) * np.exp(0.5 * rng.standard_normal(512))).astype(np.float32)
+    return F.quantize_main_kv(x)
+
+
+def test_attention_dense_equivalence_vs_torch_sdpa():
+    """ctx <= 512: Top-512 keeps every position, so sparse attention is dense
+    attention over the whole context (torch SDPA in float64)."""
+    rng = np.random.default_rng(10)
+    n, H = 300, 16
+    codes, scales = _kv(rng, n)
+    q = torch.from_numpy(rng.standard_normal((H, 512)).astype(np.float32)).to(torch.bfloat16).double().numpy()
+    idx = np.concatenate([rng.permutation(n), -np.ones(212, dtype=np.int64)])
+    ours = C.sparse_attention(q, codes, scales, idx, 1 / np.sqrt(512))
+    kv = torch.from_numpy(F.dequantize_main_kv(codes, scales))
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(q)[None, :, None, :], kv[None, None].expand(1, H, n, 512),
+        kv[None, None].expand(1, H, n, 512), scale=1 / np.sqrt(512))[0, :, 0, :]
+    np.testing.assert_allclose(ours, ref.numpy(), rtol=1e-10, atol=1e-12)
+
+
+def test_attention_special_cases():
+    rng = np.random.default_rng(11)
+    codes, scales = _kv(rng, 20)
+    q = rng.standard_normal((4, 512))
+    rows = F.dequantize_main_kv(codes, scales)
+    one = C.sparse_attention(q, codes, scales, np.array([7, -1, -1]), 0.05)
+    np.testing.assert_array_equal(one, np.broadcast_to(rows[7], (4, 512)))
+    np.testing.assert_array_equal(C.sparse_attention(q, codes, scales, -np.ones(8, np.int64), 0.05), 0)
+    # q = 0: uniform weights -> mean of the rows
+    np.testing.assert_allclose(C.sparse_attention(np.zeros((2, 512)), codes, scales, np.arange(5), 1.0),
+                               np.broadcast_to(rows[:5].mean(0), (2, 512)), rtol=1e-12)
+    # order of the index list does not matter
+    a = C.sparse_attention(q, codes, scales, np.array([1, 5, 9, 13]), 0.05)
+    b = C.sparse_attention(q, codes, scales, np.array([13, 1, -1, 9, 5]), 0.05)
+    np.testing.assert_allclose(a, b, rtol=1e-12, atol=1e-15)
+
+
+# ----------------------------------------------------------------- prefill --
+
+def test_prefill_visibility():
+    # entry e covers tokens 2e, 2e+1 and is visible at token p iff 2e+1 <= p
+    for p in range(0, 40):
+        brute = sum(1 for e in range(100) if 2 * e + 1 <= p)
+        assert C.prefill_visible(p) == brute
+    assert C.prefill_visible(524288 - 8192) == 258048
+    assert C.prefill_visible(524287) == 262144
+
+
+def test_prefill_topk_is_causal():
+    rng = np.random.default_rng(12)
+    codes, byte = _idx_rows(rng, 2000)
+    q, w = _query(rng)
+    t = C.prefill_topk(q, w, codes, byte, p=1500, k=64)
+    assert t.max() < C.prefill_visible(1500)
+    s = C.indexer_scores(q, w, codes[:750], byte[:750])
+    np.testing.assert_array_equal(t, C.top_k_ascending(np.arange(750), s, 64))
+
+
+def test_pages_constants_match_oracle(golden_dir):
+    with open(os.path.join(golden_dir, "pages_constants.json")) as f:
+        g = json.load(f)
+    assert C.POOL_BLOCKS == g["pool_blocks"]["value"]
+    assert C.BLOCK == g["block_positions"]["value"]
+    assert C.POOL_BLOCKS * C.BLOCK == g["pool_positions"]["value"]
+    assert C.TOPK == g["topk"]["value"]
+    assert C.INDEX_HEADS == g["index_heads"]["value"]
+    assert F.INDEXER_DIM == g["index_head_dim"]["value"]
+    assert F.GROUP == g["scale_group_channels"]["value"]
