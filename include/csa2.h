@@ -1,0 +1,236 @@
+/*
+ * csa2.h -- C ABI of libcsa2.so: the CSA2 decode step (Compressed Sparse
+ * Attention 2) with its Hierarchical Sparse Indexer over an FP4 main-KV cache,
+ * as hand-written sm_100a (B200) CUDA kernels.
+ *
+ * Where each operation is defined (page title and section):
+ *   - Layer modes Full / Reindex / Reuse: readance summary of the
+ *     DeepSeek-V4.1-Flash report, section 4.2; 4sapi "DeepSeek V4.1 Flash
+ *     CED/CSA2" blog, section 二 (mode table).
+ *   - Indexer (32 heads x 128, Top-512) and the hierarchical pool (2048 blocks
+ *     x 8 positions kept by the first Full layer; Reindex layers choose inside
+ *     it): 4sapi blog, section 四; alphalab "DeepSeek-V4.1-Flash 深度分析",
+ *     section 2 CSA2; animattoys article, section 層與層之間拼車.
+ *   - Main KV in FP4 E2M1 with one E4M3 scale per 16 channels, no global
+ *     scale, quantised after RoPE: 4sapi blog, section 五 FP4 KV; animattoys
+ *     article, section 把精度降到4比特; alphalab analysis, section 3 FP4.
+ *   The pages leave open the indexer dtype, the score and block functions and
+ *   every tie rule; the readings implemented here are:
+ *     indexer K and Q: FP8 E4M3 codes with one power-of-two scale per row
+ *       (sigma = 2^e, e the smallest integer with 448 * 2^e >= max|row|,
+ *       e >= -126; stored byte e + 127);
+ *     score s_t = sigma_t * sum_h w_h * ReLU(sigma^q_h * <q^_h, k^_t>);
+ *     block score = max over the block's visible positions;
+ *     ties in every selection go to the lower index; selections are returned
+ *     sorted ascending and padded with -1.
+ *
+ * Conventions for every entry point:
+ *   - All pointers are DEVICE pointers owned by the caller unless marked
+ *     "host".  The library never allocates, frees or synchronises (except
+ *     csa2_get_error) and keeps no state between calls.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  All work is
+ *     enqueued asynchronously on it.
+ *   - Shapes and pointers are validated on the host before any launch; a
+ *     violation returns CSA2_ERR_ARG / CSA2_ERR_SHAPE / CSA2_ERR_UNSUPPORTED
+ *     and launches nothing.  csa2_last_error_message() then describes it.
+ *   - Data-dependent violations found on the device (a page id outside
+ *     [0, num_pages), a position outside the request's capacity, a Top-k
+ *     index outside the visible context) never trap: the kernel records the
+ *     first one in cache->err_word and skips or neutralises the offending
+ *     element; csa2_get_error() reads it back.
+ *   - Launch failures return CSA2_ERR_CUDA.
+ */
+#ifndef CSA2_H
+#define CSA2_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define CSA2_API __attribute__((visibility("default")))
+#else
+#define CSA2_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  CSA2_FULL = 0,     /* Top-k from this layer's own Full scan            */
+  CSA2_REINDEX = 1,  /* re-score the pool with this layer's own query    */
+  CSA2_REUSE = 2     /* take the previous layer's Top-k unchanged        */
+} csa2_mode;
+
+typedef enum {
+  CSA2_OK = 0,
+  CSA2_ERR_ARG = 1,            /* null / misaligned pointer, bad enum    */
+  CSA2_ERR_SHAPE = 2,          /* size outside the supported range        */
+  CSA2_ERR_CUDA = 3,           /* a CUDA runtime call failed              */
+  CSA2_ERR_DEVICE_BOUNDS = 4,  /* (err_word) out-of-range page/position   */
+  CSA2_ERR_TIMEOUT = 5,        /* (err_word) a pipeline wait gave up      */
+  CSA2_ERR_UNSUPPORTED = 6     /* device is not sm_100 / feature missing  */
+} csa2_status;
+
+/* Positions per pool block and cache row sizes (bytes). */
+#define CSA2_BLOCK 8
+#define CSA2_INDEX_HEADS 32
+#define CSA2_INDEX_DIM 128
+#define CSA2_KV_DIM 512
+#define CSA2_KV_CODE_BYTES 256   /* 512 E2M1 codes, 2 per byte            */
+#define CSA2_KV_SCALE_BYTES 32   /* one E4M3 scale per 16 channels         */
+
+/*
+ * The paged cache of one layer group.  A "row" is one cached position; rows
+ * live in pages of `page_size` consecutive rows.  Position t of request b is
+ * row  page_table[b * max_pages_per_req + t / page_size] * page_size
+ *      + t % page_size.
+ * Arrays (row-major, device memory, 16-byte aligned base pointers):
+ *   kv_codes   uint8 [num_pages * page_size][256]  E2M1 pairs: byte i holds
+ *              channel 2i in its low nibble, channel 2i+1 in its high nibble
+ *   kv_scales  uint8 [num_pages * page_size][32]   E4M3 scale of channels
+ *              16g..16g+15
+ *   ik_codes   uint8 [num_pages * page_size][128]  E4M3 indexer key
+ *   ik_exp     uint8 [num_pages * page_size]       sigma_t = 2^(byte - 127)
+ *   page_table int32 [batch][max_pages_per_req]
+ *   ctx_len    int32 [batch]  visible positions of each request
+ *   err_word   int32 [4]      {code, kernel, request, index} of the first
+ *              device-side error; the caller zeroes it once.
+ * page_size must be a positive multiple of 128.
+ */
+typedef struct csa2_cache {
+  uint8_t* kv_codes;
+  uint8_t* kv_scales;
+  uint8_t* ik_codes;
+  uint8_t* ik_exp;
+  const int32_t* page_table;
+  const int32_t* ctx_len;
+  int32_t num_pages;
+  int32_t page_size;
+  int32_t max_pages_per_req;
+  int32_t batch;
+  int32_t* err_word;
+} csa2_cache;
+
+/* Capacity of one request in positions: max_pages_per_req * page_size.  The
+ * per-request strides of the score and block-max buffers below derive from it:
+ *   scores   float [batch][capacity]
+ *   blockmax float [batch][capacity / 8]                                    */
+
+/*
+ * csa2_append_kv -- quantise-on-append (main KV to FP4, indexer K to FP8) and
+ * write n_rows rows into their page slots.
+ *   kv_new  float [n_rows][512]  main KV rows (already rotated: the pages
+ *                                state quantisation happens after RoPE)
+ *   ik_new  float [n_rows][128]  indexer keys
+ *   req     int32 [n_rows]       request of each row; NULL = row i -> request i
+ *   pos     int32 [n_rows]       position of each row inside its request
+ * Per 16 channels: s = E4M3 nearest (ties to even, saturating) of amax/6;
+ * codes = E2M1 nearest of x/s (ties to even code, saturating at 6, -0 -> +0).
+ * Indexer: sigma as above, codes = E4M3 nearest of k/sigma.
+ * ctx_len is not modified: the caller advances it.
+ * Device errors: req outside [0,batch), pos outside [0,capacity), page id
+ * outside [0,num_pages) -> CSA2_ERR_DEVICE_BOUNDS, row skipped.
+ */
+CSA2_API csa2_status csa2_append_kv(const csa2_cache* cache, int32_t n_rows, const float* kv_new,
+                           const float* ik_new, const int32_t* req, const int32_t* pos,
+                           void* stream);
+
+/*
+ * csa2_index_full -- Full-mode indexer scan of every visible position of every
+ * request (Hierarchical Sparse Indexer, first stage).
+ *   q        float [batch][32][128]  indexer query (quantised inside, FP8 rule)
+ *   w        float [batch][32]       head weights
+ *   blockmax float [batch][capacity/8]  out: m_j = max score of block j over
+ *            positions < ctx_len; entries past ceil(ctx_len/8) are untouched
+ *   scores   float [batch][capacity] or NULL  out: per-position scores s_t
+ * Runs on tcgen05 FP8 tensor cores (scores are fp32; the float64 reference
+ * differs by fp32 accumulation rounding only).
+ */
+CSA2_API csa2_status csa2_index_full(const csa2_cache* cache, const float* q, const float* w,
+                            float* blockmax, float* scores, void* stream);
+
+/*
+ * csa2_pool_select -- the hierarchical pool: the pool_blocks blocks with the
+ * largest block max (ties -> lower block id), sorted ascending, -1 padded.
+ * With ceil(ctx_len/8) <= pool_blocks the pool is every block.
+ *   blockmax float [batch][capacity/8]   (from csa2_index_full)
+ *   pool     int32 [batch][pool_blocks]  out
+ * pool_blocks in [1, 4096] (the pages use 2048); ceil(capacity/8) must not
+ * exceed 16 * 16384 blocks (2,097,152 positions per request).
+ */
+CSA2_API csa2_status csa2_pool_select(const csa2_cache* cache, const float* blockmax, int32_t pool_blocks,
+                             int32_t* pool, void* stream);
+
+/*
+ * csa2_reindex -- Top-k of one layer of the group, by mode:
+ *   CSA2_FULL    the k best positions of this layer's own Full scan among the
+ *                candidates.  Scores come from full_scores when it is not NULL,
+ *                else they are recomputed from (q, w) with the exact arithmetic
+ *                of csa2_index_full (bit-identical).
+ *   CSA2_REINDEX re-score only the candidates with this layer's own (q, w).
+ *   CSA2_REUSE   copy prev_topk into topk (nothing is done when they alias).
+ * Candidates: the positions of the pool's blocks (pool int32 [batch]
+ * [pool_blocks], ascending, -1 padded), or every visible position when pool is
+ * NULL (then ceil(ctx_len/8) must not exceed 131072 blocks).
+ *   q float [batch][32][128], w float [batch][32]  (FULL without full_scores,
+ *                                                   and REINDEX)
+ *   full_scores float [batch][capacity] or NULL
+ *   prev_topk int32 [batch][k]  (REUSE)
+ *   topk      int32 [batch][k]  out: positions ascending, -1 padded
+ * k in [1, 4096], pool_blocks in [1, 4096].
+ */
+CSA2_API csa2_status csa2_reindex(const csa2_cache* cache, csa2_mode mode, const int32_t* pool,
+                         int32_t pool_blocks, const float* q, const float* w,
+                         const float* full_scores, const int32_t* prev_topk, int32_t k,
+                         int32_t* topk, void* stream);
+
+/*
+ * csa2_sparse_attn -- sparse MQA attention over the gathered Top-k rows:
+ *   o_h = sum_i softmax_i(scale * q_h . v_i) v_i,  K = V = dequantised row,
+ * skipping -1 entries; a query with no valid entry gets o = 0.
+ *   n_queries  queries in this call
+ *   q_req      int32 [n_queries] request of each query, or NULL (query i ->
+ *              request i; then n_queries <= batch)
+ *   topk       int32 [n_queries][k]   positions in the query's request
+ *   q          bf16  [n_queries][H][512] (uint16 bit patterns)
+ *   out        bf16  [n_queries][H][512] out
+ * H in {16, 32, 64}; k in [1, 4096].  Dequantised rows are exact in fp16,
+ * logits and softmax are fp32, P.V uses fp16 probabilities with fp32 sums.
+ * Device errors: a Top-k entry >= ctx_len or < -1 -> CSA2_ERR_DEVICE_BOUNDS,
+ * entry skipped.
+ */
+CSA2_API csa2_status csa2_sparse_attn(const csa2_cache* cache, int32_t n_queries, const int32_t* q_req,
+                             const int32_t* topk, int32_t k, const uint16_t* q, int32_t H,
+                             float scale, uint16_t* out, void* stream);
+
+/*
+ * csa2_get_error -- synchronise `stream`, copy cache->err_word to the host
+ * array out[4] (host pointer) and return out[0] as a status (CSA2_OK when no
+ * device error was recorded).  Does not clear the word.
+ */
+CSA2_API csa2_status csa2_get_error(const csa2_cache* cache, int32_t* out, void* stream);
+
+/*
+ * csa2_set_wait_limit_ns -- process-wide bound, in nanoseconds, on every
+ * pipeline wait inside the tensor-core kernels (csa2_index_full and the
+ * re-scoring csa2_reindex); default 2e9.  A wait that runs out makes the
+ * kernel record CSA2_ERR_TIMEOUT in err_word, wait (with a fixed bound) for its
+ * own copies in flight, free its tensor memory and return; the call's outputs
+ * are then undefined.  0 gives up on the first wait that is not already
+ * satisfied (used by the tests of that path).  Not thread-safe with
+ * concurrent launches.
+ */
+CSA2_API void csa2_set_wait_limit_ns(uint64_t ns);
+
+/* Static description of a status code. */
+CSA2_API const char* csa2_status_string(csa2_status status);
+
+/* Thread-local description of the last host-side failure of this thread. */
+CSA2_API const char* csa2_last_error_message(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CSA2_H */

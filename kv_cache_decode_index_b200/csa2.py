@@ -1,0 +1,281 @@
+"""ctypes binding of libcsa2.so (include/csa2.h).
+
+Argument marshalling only: every step of the decode path runs in the library's
+CUDA kernels.  PyTorch supplies device memory and the current stream.  There is
+no fallback: importing this module raises if the library has not been built,
+and every call raises ``Csa2Error`` when the library reports a failure.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libcsa2.so")
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is missing: build it with `python -m kv_cache_decode_index_b200.build`")
+_lib = ctypes.CDLL(LIB_PATH)
+
+FULL, REINDEX, REUSE = 0, 1, 2
+MODE = {"F": FULL, "Ri": REINDEX, "Ru": REUSE}
+OK, ERR_ARG, ERR_SHAPE, ERR_CUDA, ERR_DEVICE_BOUNDS, ERR_TIMEOUT, ERR_UNSUPPORTED = range(7)
+BLOCK, INDEX_HEADS, INDEX_DIM, KV_DIM, KV_CODE_BYTES, KV_SCALE_BYTES = 8, 32, 128, 512, 256, 32
+
+
+class CacheStruct(ctypes.Structure):
+    _fields_ = [("kv_codes", ctypes.c_void_p), ("kv_scales", ctypes.c_void_p), ("ik_codes", ctypes.c_void_p),
+                ("ik_exp", ctypes.c_void_p), ("page_table", ctypes.c_void_p), ("ctx_len", ctypes.c_void_p),
+                ("num_pages", ctypes.c_int32), ("page_size", ctypes.c_int32),
+                ("max_pages_per_req", ctypes.c_int32), ("batch", ctypes.c_int32), ("err_word", ctypes.c_void_p)]
+
+
+_P = ctypes.c_void_p
+_I = ctypes.c_int32
+_CP = ctypes.POINTER(CacheStruct)
+_sig = {
+    "csa2_append_kv": [_CP, _I, _P, _P, _P, _P, _P],
+    "csa2_index_full": [_CP, _P, _P, _P, _P, _P],
+    "csa2_pool_select": [_CP, _P, _I, _P, _P],
+    "csa2_reindex": [_CP, _I, _P, _I, _P, _P, _P, _P, _I, _P, _P],
+    "csa2_sparse_attn": [_CP, _I, _P, _P, _I, _P, _I, ctypes.c_float, _P, _P],
+    "csa2_get_error": [_CP, ctypes.POINTER(ctypes.c_int32), _P],
+}
+for _name, _args in _sig.items():
+    getattr(_lib, _name).argtypes = _args
+    getattr(_lib, _name).restype = ctypes.c_int
+_lib.csa2_status_string.argtypes = [ctypes.c_int]
+_lib.csa2_status_string.restype = ctypes.c_char_p
+_lib.csa2_last_error_message.argtypes = []
+_lib.csa2_last_error_message.restype = ctypes.c_char_p
+_lib.csa2_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
+_lib.csa2_set_wait_limit_ns.restype = None
+
+
+class Csa2Error(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        msg = _lib.csa2_last_error_message().decode()
+        super().__init__(f"{where}: {_lib.csa2_status_string(status).decode()} ({status}): {msg}")
+
+
+def _check(status: int, where: str):
+    if status != OK:
+        raise Csa2Error(status, where)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(dev):
+    return ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
+
+
+def _need(t, dtype, shape, name):
+    if t.dtype != dtype or tuple(t.shape) != tuple(shape) or not t.is_contiguous() or t.device.type != "cuda":
+        raise ValueError(f"{name}: expected contiguous cuda {dtype} {tuple(shape)}, "
+                         f"got {t.device} {t.dtype} {tuple(t.shape)}")
+
+
+def set_wait_limit_ns(ns: int):
+    """Bound of every pipeline wait in the tensor-core kernels (default 2 s)."""
+    _lib.csa2_set_wait_limit_ns(int(ns))
+
+
+class Cache:
+    """The paged cache of one layer group (device memory owned by torch).
+
+    Rows: num_pages * page_size; request b's position t lives in row
+    page_table[b, t // page_size] * page_size + t % page_size.
+    """
+
+    def __init__(self, num_pages: int, page_size: int, page_table, ctx_len, device="cuda"):
+        self.device = torch.device(device)
+        rows = num_pages * page_size
+        self.num_pages, self.page_size = int(num_pages), int(page_size)
+        self.kv_codes = torch.zeros(rows, KV_CODE_BYTES, dtype=torch.uint8, device=self.device)
+        self.kv_scales = torch.zeros(rows, KV_SCALE_BYTES, dtype=torch.uint8, device=self.device)
+        self.ik_codes = torch.zeros(rows, INDEX_DIM, dtype=torch.uint8, device=self.device)
+        self.ik_exp = torch.zeros(rows, dtype=torch.uint8, device=self.device)
+        self.page_table = torch.as_tensor(page_table, dtype=torch.int32).to(self.device).contiguous()
+        self.ctx_len = torch.as_tensor(ctx_len, dtype=torch.int32).to(self.device).contiguous()
+        self.batch, self.max_pages_per_req = self.page_table.shape
+        self.err_word = torch.zeros(4, dtype=torch.int32, device=self.device)
+        self._struct = None
+
+    @property
+    def capacity(self) -> int:
+        return self.max_pages_per_req * self.page_size
+
+    @property
+    def struct(self) -> CacheStruct:
+        s = CacheStruct(self.kv_codes.data_ptr(), self.kv_scales.data_ptr(), self.ik_codes.data_ptr(),
+                        self.ik_exp.data_ptr(), self.page_table.data_ptr(), self.ctx_len.data_ptr(),
+                        self.num_pages, self.page_size, self.max_pages_per_req, self.batch,
+                        self.err_word.data_ptr())
+        self._struct = s   # keep alive while a call is in flight
+        return s
+
+    def rows_of(self, b: int, positions):
+        """Cache row numbers of request b's positions (host helper for tests)."""
+        pt = self.page_table[b].cpu()
+        positions = torch.as_tensor(positions, dtype=torch.int64)
+        return pt[positions // self.page_size].to(torch.int64) * self.page_size + positions % self.page_size
+
+
+def append_kv(cache: Cache, kv_new, ik_new, pos, req=None):
+    n = kv_new.shape[0]
+    _need(kv_new, torch.float32, (n, KV_DIM), "kv_new")
+    _need(ik_new, torch.float32, (n, INDEX_DIM), "ik_new")
+    _need(pos, torch.int32, (n,), "pos")
+    if req is not None:
+        _need(req, torch.int32, (n,), "req")
+    _check(_lib.csa2_append_kv(ctypes.byref(cache.struct), n, _ptr(kv_new), _ptr(ik_new), _ptr(req), _ptr(pos),
+                               _stream(cache.device)), "csa2_append_kv")
+
+
+def index_full(cache: Cache, q, w, blockmax=None, scores=None):
+    """Full scan: returns blockmax float32 [batch, capacity/8] (and fills scores if given)."""
+    B = cache.batch
+    _need(q, torch.float32, (B, INDEX_HEADS, INDEX_DIM), "q")
+    _need(w, torch.float32, (B, INDEX_HEADS), "w")
+    if blockmax is None:
+        blockmax = torch.empty(B, cache.capacity // BLOCK, dtype=torch.float32, device=cache.device)
+    _need(blockmax, torch.float32, (B, cache.capacity // BLOCK), "blockmax")
+    if scores is not None:
+        _need(scores, torch.float32, (B, cache.capacity), "scores")
+    _check(_lib.csa2_index_full(ctypes.byref(cache.struct), _ptr(q), _ptr(w), _ptr(blockmax), _ptr(scores),
+                                _stream(cache.device)), "csa2_index_full")
+    return blockmax
+
+
+def pool_select(cache: Cache, blockmax, pool_blocks: int = 2048, pool=None):
+    B = cache.batch
+    _need(blockmax, torch.float32, (B, cache.capacity // BLOCK), "blockmax")
+    if pool is None:
+        pool = torch.empty(B, pool_blocks, dtype=torch.int32, device=cache.device)
+    _need(pool, torch.int32, (B, pool_blocks), "pool")
+    _check(_lib.csa2_pool_select(ctypes.byref(cache.struct), _ptr(blockmax), pool_blocks, _ptr(pool),
+                                 _stream(cache.device)), "csa2_pool_select")
+    return pool
+
+
+def reindex(cache: Cache, mode: int, k: int = 512, pool=None, q=None, w=None, full_scores=None,
+            prev_topk=None, topk=None):
+    """Top-k of one layer (mode FULL / REINDEX / REUSE); returns topk int32 [batch, k]."""
+    B = cache.batch
+    P = 0
+    if pool is not None:
+        P = pool.shape[1]
+        _need(pool, torch.int32, (B, P), "pool")
+    if q is not None:
+        _need(q, torch.float32, (B, INDEX_HEADS, INDEX_DIM), "q")
+        _need(w, torch.float32, (B, INDEX_HEADS), "w")
+    if full_scores is not None:
+        _need(full_scores, torch.float32, (B, cache.capacity), "full_scores")
+    if prev_topk is not None:
+        _need(prev_topk, torch.int32, (B, k), "prev_topk")
+    if topk is None:
+        topk = torch.empty(B, k, dtype=torch.int32, device=cache.device)
+    _need(topk, torch.int32, (B, k), "topk")
+    _check(_lib.csa2_reindex(ctypes.byref(cache.struct), mode, _ptr(pool), P, _ptr(q), _ptr(w), _ptr(full_scores),
+                             _ptr(prev_topk), k, _ptr(topk), _stream(cache.device)), "csa2_reindex")
+    return topk
+
+
+def sparse_attn(cache: Cache, topk, q, scale: float | None = None, out=None, q_req=None):
+    """Sparse attention; q bf16 [n, H, 512] -> out bf16 [n, H, 512]."""
+    n, k = topk.shape
+    H = q.shape[1]
+    _need(topk, torch.int32, (n, k), "topk")
+    _need(q, torch.bfloat16, (n, H, KV_DIM), "q")
+    if q_req is not None:
+        _need(q_req, torch.int32, (n,), "q_req")
+    if out is None:
+        out = torch.empty_like(q)
+    _need(out, torch.bfloat16, (n, H, KV_DIM), "out")
+    scale = 1.0 / math.sqrt(KV_DIM) if scale is None else scale
+    _check(_lib.csa2_sparse_attn(ctypes.byref(cache.struct), n, _ptr(q_req), _ptr(topk), k, _ptr(q), H,
+                                 ctypes.c_float(scale), _ptr(out), _stream(cache.device)), "csa2_sparse_attn")
+    return out
+
+
+def get_error(cache: Cache):
+    """Synchronise the current stream and return (status, err_word list)."""
+    out = (ctypes.c_int32 * 4)()
+    st = _lib.csa2_get_error(ctypes.byref(cache.struct), out, _stream(cache.device))
+    return st, list(out)
+
+
+class DecodeGroup:
+    """One decode step of a CSA2 layer group over `cache`, through the C ABI.
+
+    modes: e.g. ("F", "Ri", "Ri", "Ru", "Ru", "Ru").  The first Full layer
+    scans the context and (with pool_blocks) builds the pool; Reindex layers
+    re-score the pool with their own query; Reuse layers take the previous
+    layer's Top-k.  Every layer attends with its own main query.
+    With `concurrent`, layers that only depend on the pool run on side streams
+    (the calls are stream-ordered, so the step can be captured in a CUDA graph).
+    """
+
+    def __init__(self, cache: Cache, modes, heads: int, k: int = 512, pool_blocks: int | None = 2048,
+                 scale: float | None = None, concurrent: bool = True):
+        if modes[0] != "F":
+            raise ValueError("a layer group starts with a Full layer")
+        self.cache, self.modes, self.heads, self.k = cache, tuple(modes), heads, k
+        self.pool_blocks = pool_blocks
+        self.scale = 1.0 / math.sqrt(KV_DIM) if scale is None else scale
+        dev, B = cache.device, cache.batch
+        self.blockmax = torch.empty(B, cache.capacity // BLOCK, dtype=torch.float32, device=dev)
+        self.pool = torch.empty(B, pool_blocks, dtype=torch.int32, device=dev) if pool_blocks else None
+        # Reuse layers alias the Top-k buffer of the layer they reuse
+        self.topk, src = [], None
+        for m in self.modes:
+            if m == "Ru":
+                self.topk.append(src)
+            else:
+                src = torch.empty(B, k, dtype=torch.int32, device=dev)
+                self.topk.append(src)
+        self.concurrent = concurrent
+        n_side = sum(1 for m in self.modes if m != "Ru")
+        self.streams = [torch.cuda.Stream(dev) for _ in range(n_side)] if concurrent else []
+        self.launches_per_step = 1 + (1 if pool_blocks else 0) + n_side + len(self.modes)
+
+    def step(self, q_idx, w_idx, q_main, out):
+        """q_idx / w_idx: per layer ([B,32,128] / [B,32], None for Reuse);
+        q_main / out: per layer bf16 [B, H, 512]."""
+        c = self.cache
+        index_full(c, q_idx[0], w_idx[0], self.blockmax)
+        if self.pool is not None:
+            pool_select(c, self.blockmax, self.pool_blocks, self.pool)
+        main = torch.cuda.current_stream(c.device)
+        side = 0
+        ev_ready = torch.cuda.Event()
+        ev_ready.record(main)
+        joins = []
+        src_stream = main
+        for layer, m in enumerate(self.modes):
+            if m != "Ru":
+                s = self.streams[side] if self.concurrent else main
+                side += 1
+                with torch.cuda.stream(s):
+                    if s is not main:
+                        s.wait_event(ev_ready)
+                    mode = FULL if m == "F" else REINDEX
+                    reindex(c, mode, self.k, self.pool, q_idx[layer], w_idx[layer], topk=self.topk[layer])
+                    sparse_attn(c, self.topk[layer], q_main[layer], self.scale, out[layer])
+                src_stream = s
+            else:
+                with torch.cuda.stream(src_stream):
+                    sparse_attn(c, self.topk[layer], q_main[layer], self.scale, out[layer])
+        if self.concurrent:
+            for s in self.streams:
+                e = torch.cuda.Event()
+                e.record(s)
+                joins.append(e)
+            for e in joins:
+                main.wait_event(e)
+        return out

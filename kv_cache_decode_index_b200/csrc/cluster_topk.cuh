@@ -1,0 +1,196 @@
+// Exact top-K over keys spread across the CTAs of one thread-block cluster.
+//
+// Each CTA holds its share of the candidates' keys in shared memory
+// (uint32, order-preserving; 0 = not a candidate).  Candidates are ordered by
+// (cluster rank, local index); that order is the ascending candidate-id order,
+// which decides ties (lower id first) and the output order (ascending).
+//
+// Radix select, 8 bits per pass from the top: every CTA builds the histogram
+// of its keys that match the prefix decided so far, the CTAs read each other's
+// histograms through distributed shared memory (one cluster barrier per pass,
+// two histogram buffers), and all of them derive the same next digit.  The
+// passes stop as soon as every key matching the prefix is needed.  Then each
+// CTA counts its keys above / on the threshold prefix, the counts are
+// exchanged once more, and every CTA writes its selected ids at their ranks.
+#pragma once
+
+#include <cooperative_groups.h>
+
+#include "common.cuh"
+
+namespace csa2 {
+
+namespace cg = cooperative_groups;
+
+constexpr int kMaxCluster = 16;
+
+struct SelectSmem {
+  uint32_t hist[2][256];
+  uint32_t ghist[256];
+  int gt_eq[2];              // this CTA's (above, on-threshold) counts, read remotely
+  int warp_tmp[32];
+  uint32_t prefix, mask;
+  int need;
+  int done;
+  int total;                 // valid candidates in the cluster
+};
+
+// Exclusive block-wide prefix sum of one int per thread (THREADS multiple of
+// 32, <= 1024).  Returns the thread's exclusive prefix; *sum gets the total.
+template <int THREADS>
+__device__ __forceinline__ int block_exclusive_sum(int v, int* warp_tmp, int* sum) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  __syncthreads();   // warp_tmp reuse guard
+  if (lane == 31) warp_tmp[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    int t = lane < THREADS / 32 ? warp_tmp[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, t, o);
+      if (lane >= o) t += y;
+    }
+    if (lane < THREADS / 32) warp_tmp[lane] = t;   // inclusive warp totals
+  }
+  __syncthreads();
+  *sum = warp_tmp[THREADS / 32 - 1];
+  return x - v + (warp > 0 ? warp_tmp[warp - 1] : 0);
+}
+
+// Select the K best of the cluster's candidates.  emit(i, r) is called for the
+// local candidate i that has output rank r (0 <= r < min(K, total)); pad(r) for
+// r in [total, K) by the cluster's rank-0 CTA.  Must be called by all THREADS
+// threads of every CTA of the cluster (it contains cluster barriers).
+template <int THREADS, class Emit, class Pad>
+__device__ void cluster_topk(const uint32_t* keys, int n_local, int K, SelectSmem& S, Emit emit, Pad pad) {
+  cg::cluster_group cluster = cg::this_cluster();
+  const int C = static_cast<int>(cluster.num_blocks());
+  const int rank = static_cast<int>(cluster.block_rank());
+  const int tid = threadIdx.x;
+  const int per = (n_local + THREADS - 1) / THREADS;
+  const int lo = min(tid * per, n_local), hi = min(lo + per, n_local);
+
+  if (tid == 0) {
+    S.prefix = 0;
+    S.mask = 0;
+    S.done = 0;
+  }
+  for (int i = tid; i < 256; i += THREADS) S.hist[0][i] = 0;
+  __syncthreads();
+
+#pragma unroll 1
+  for (int pass = 0; pass < 4; ++pass) {
+    const int shift = 24 - 8 * pass;
+    const int buf = pass & 1;
+    const uint32_t prefix = S.prefix, mask = S.mask;
+    for (int i = lo; i < hi; ++i) {
+      const uint32_t k = keys[i];
+      if (k != 0u && (k & mask) == prefix) atomicAdd(&S.hist[buf][(k >> shift) & 255u], 1u);
+    }
+    cluster.sync();   // every CTA's histogram of this pass is complete
+    for (int d = tid; d < 256; d += THREADS) {
+      uint32_t g = 0;
+      for (int r = 0; r < C; ++r) g += cluster.map_shared_rank(&S.hist[buf][0], r)[d];
+      S.ghist[d] = g;
+      S.hist[buf ^ 1][d] = 0;   // next pass's buffer (last read remotely before this barrier)
+    }
+    __syncthreads();
+    if (tid < 32) {
+      // lane l owns digits 255-8l .. 248-8l (descending)
+      uint32_t local[8];
+      uint32_t sum = 0;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        local[i] = S.ghist[255 - 8 * tid - i];
+        sum += local[i];
+      }
+      uint32_t incl = sum;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (tid >= o) incl += y;
+      }
+      const uint32_t total = __shfl_sync(0xffffffffu, incl, 31);
+      if (pass == 0 && tid == 0) {
+        S.total = static_cast<int>(total);
+        if (total <= static_cast<uint32_t>(K)) {   // everything valid is selected
+          S.need = static_cast<int>(total);
+          S.done = 1;
+        } else {
+          S.need = K;
+        }
+      }
+      __syncwarp();
+      if (!S.done) {
+        const uint32_t need = static_cast<uint32_t>(S.need);
+        uint32_t above = incl - sum;   // keys in digits above this lane's range
+        if (above < need && need <= incl) {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            if (above < need && need <= above + local[i]) {
+              const uint32_t d = 255u - 8u * tid - i;
+              S.prefix = prefix | (d << shift);
+              S.mask = mask | (255u << shift);
+              S.need = static_cast<int>(need - above);
+              if (local[i] == need - above) S.done = 1;   // all keys with this prefix are taken
+            }
+            above += local[i];
+          }
+        }
+      }
+    }
+    __syncthreads();
+    if (S.done) break;
+  }
+
+  // ---- final: above (prefix greater) and on-threshold (prefix equal) ----
+  const uint32_t prefix = S.prefix, mask = S.mask;
+  const int need = S.need;
+  int gt = 0, eq = 0;
+  for (int i = lo; i < hi; ++i) {
+    const uint32_t k = keys[i];
+    if (k == 0u) continue;
+    const uint32_t km = k & mask;
+    gt += km > prefix;
+    eq += km == prefix;
+  }
+  int local_gt, local_eq;
+  const int eq_before = block_exclusive_sum<THREADS>(eq, S.warp_tmp, &local_eq);
+  (void)block_exclusive_sum<THREADS>(gt, S.warp_tmp, &local_gt);
+  if (tid == 0) {
+    S.gt_eq[0] = local_gt;
+    S.gt_eq[1] = local_eq;
+  }
+  cluster.sync();   // counts visible cluster-wide
+  int out_base = 0, take_local = 0, sel_total = 0, ties_before = 0;
+  for (int r = 0; r < C; ++r) {
+    const int* ge = cluster.map_shared_rank(&S.gt_eq[0], r);
+    const int g = ge[0], e = ge[1];
+    const int take = max(0, min(need - ties_before, e));
+    if (r < rank) out_base += g + take;
+    if (r == rank) take_local = take;
+    sel_total += g + take;
+    ties_before += e;
+  }
+  const int take_t = max(0, min(take_local - eq_before, eq));
+  int dummy;
+  int off = out_base + block_exclusive_sum<THREADS>(gt + take_t, S.warp_tmp, &dummy);
+  int taken = 0;
+  for (int i = lo; i < hi; ++i) {
+    const uint32_t k = keys[i];
+    if (k == 0u) continue;
+    const uint32_t km = k & mask;
+    if (km > prefix || (km == prefix && taken++ < take_t)) emit(i, off++);
+  }
+  if (rank == 0)
+    for (int r = sel_total + tid; r < K; r += THREADS) pad(r);
+  cluster.sync();   // no CTA leaves while its shared memory may still be read
+}
+
+}  // namespace csa2

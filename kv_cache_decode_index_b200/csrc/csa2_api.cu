@@ -1,0 +1,262 @@
+// C ABI of libcsa2.so (declared in include/csa2.h): host-side validation,
+// TMA tensor maps, launches.  No allocation, no synchronisation except in
+// csa2_get_error.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdarg>
+#include <cstdio>
+#include <mutex>
+
+#include "common.cuh"
+#include "launch.h"
+
+namespace {
+
+thread_local char g_msg[512] = "";
+
+csa2_status fail(csa2_status s, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_msg, sizeof(g_msg), fmt, ap);
+  va_end(ap);
+  return s;
+}
+
+csa2_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(CSA2_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+constexpr int kMaxBatch = 1024;
+constexpr int kMaxK = 4096;
+constexpr int kMaxPool = 4096;
+constexpr long long kMaxFlatPositions = 131072;       // Top-k without a pool
+constexpr long long kMaxPoolSelectBlocks = 16LL * 16384;
+
+uint64_t g_wait_limit_ns = csa2::kWaitLimitNs;
+
+// Device properties, cached per device ordinal.
+struct DeviceInfo {
+  int sms = 0;
+  int major = 0;
+};
+std::mutex g_dev_mu;
+DeviceInfo g_dev[64];
+
+csa2_status device_info(DeviceInfo* out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= 64) return fail(CSA2_ERR_UNSUPPORTED, "device ordinal %d out of range", dev);
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  if (g_dev[dev].sms == 0) {
+    int sms = 0, major = 0;
+    e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
+    g_dev[dev].sms = sms;
+    g_dev[dev].major = major;
+  }
+  *out = g_dev[dev];
+  if (out->major != 10) return fail(CSA2_ERR_UNSUPPORTED, "needs an sm_100 (B200-class) device, found sm_%d", out->major * 10);
+  return CSA2_OK;
+}
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point.
+using EncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                              const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                              CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+csa2_status encode_ik_map(const csa2_cache* c, int box_rows, CUtensorMap* map) {
+  static EncodeFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeFn>(p);
+  });
+  if (fn == nullptr) return fail(CSA2_ERR_UNSUPPORTED, "cuTensorMapEncodeTiled is not available");
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(csa2::kIndexDim),
+                              static_cast<cuuint64_t>(c->num_pages) * static_cast<cuuint64_t>(c->page_size)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(csa2::kIndexDim)};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(csa2::kIndexDim), static_cast<cuuint32_t>(box_rows)};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, c->ik_codes, dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(CSA2_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+  return CSA2_OK;
+}
+
+long long capacity_of(const csa2_cache* c) {
+  return static_cast<long long>(c->max_pages_per_req) * c->page_size;
+}
+
+csa2_status check_cache(const csa2_cache* c, bool need_kv, bool need_ik) {
+  if (c == nullptr) return fail(CSA2_ERR_ARG, "cache is NULL");
+  if (c->page_table == nullptr || c->ctx_len == nullptr || c->err_word == nullptr)
+    return fail(CSA2_ERR_ARG, "cache.page_table, ctx_len and err_word must be set");
+  if (c->batch < 1 || c->batch > kMaxBatch) return fail(CSA2_ERR_SHAPE, "batch %d outside [1, %d]", c->batch, kMaxBatch);
+  if (c->page_size <= 0 || c->page_size % csa2::kTile != 0)
+    return fail(CSA2_ERR_SHAPE, "page_size %d must be a positive multiple of 128", c->page_size);
+  if (c->num_pages < 1 || c->max_pages_per_req < 1)
+    return fail(CSA2_ERR_SHAPE, "num_pages and max_pages_per_req must be >= 1");
+  if (static_cast<long long>(c->num_pages) * c->page_size >= (1LL << 31))
+    return fail(CSA2_ERR_SHAPE, "num_pages * page_size must stay below 2^31 rows");
+  if (capacity_of(c) >= (1LL << 31)) return fail(CSA2_ERR_SHAPE, "max_pages_per_req * page_size must stay below 2^31");
+  if (need_kv && (c->kv_codes == nullptr || c->kv_scales == nullptr || !aligned(c->kv_codes, 16) ||
+                  !aligned(c->kv_scales, 8)))
+    return fail(CSA2_ERR_ARG, "kv_codes (16-byte aligned) and kv_scales (8-byte aligned) must be set");
+  if (need_ik && (c->ik_codes == nullptr || c->ik_exp == nullptr || !aligned(c->ik_codes, 16)))
+    return fail(CSA2_ERR_ARG, "ik_codes (16-byte aligned) and ik_exp must be set");
+  return CSA2_OK;
+}
+
+#define CSA2_TRY(expr)                 \
+  do {                                 \
+    const csa2_status s_ = (expr);     \
+    if (s_ != CSA2_OK) return s_;      \
+  } while (0)
+
+}  // namespace
+
+extern "C" {
+
+csa2_status csa2_append_kv(const csa2_cache* cache, int32_t n_rows, const float* kv_new, const float* ik_new,
+                           const int32_t* req, const int32_t* pos, void* stream) {
+  CSA2_TRY(check_cache(cache, true, true));
+  if (n_rows < 0) return fail(CSA2_ERR_SHAPE, "n_rows %d < 0", n_rows);
+  if (n_rows == 0) return CSA2_OK;
+  if (kv_new == nullptr || ik_new == nullptr || pos == nullptr || !aligned(kv_new, 16) || !aligned(ik_new, 16))
+    return fail(CSA2_ERR_ARG, "kv_new, ik_new (16-byte aligned) and pos must be set");
+  if (req == nullptr && n_rows > cache->batch)
+    return fail(CSA2_ERR_SHAPE, "without req, n_rows (%d) must not exceed batch (%d)", n_rows, cache->batch);
+  DeviceInfo d;
+  CSA2_TRY(device_info(&d));
+  const cudaError_t e = csa2::launch_append(*cache, n_rows, kv_new, ik_new, req, pos, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? CSA2_OK : cuda_fail(e, "append_kv launch");
+}
+
+csa2_status csa2_index_full(const csa2_cache* cache, const float* q, const float* w, float* blockmax, float* scores,
+                            void* stream) {
+  CSA2_TRY(check_cache(cache, false, true));
+  if (q == nullptr || w == nullptr || blockmax == nullptr || !aligned(q, 16))
+    return fail(CSA2_ERR_ARG, "q (16-byte aligned), w and blockmax must be set");
+  DeviceInfo d;
+  CSA2_TRY(device_info(&d));
+  CUtensorMap map;
+  CSA2_TRY(encode_ik_map(cache, csa2::kTile, &map));
+  const cudaError_t e = csa2::launch_index_full(*cache, q, w, blockmax, scores, map, d.sms, g_wait_limit_ns,
+                                                static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? CSA2_OK : cuda_fail(e, "index_full launch");
+}
+
+csa2_status csa2_pool_select(const csa2_cache* cache, const float* blockmax, int32_t pool_blocks, int32_t* pool,
+                             void* stream) {
+  CSA2_TRY(check_cache(cache, false, false));
+  if (blockmax == nullptr || pool == nullptr) return fail(CSA2_ERR_ARG, "blockmax and pool must be set");
+  if (pool_blocks < 1 || pool_blocks > kMaxPool)
+    return fail(CSA2_ERR_SHAPE, "pool_blocks %d outside [1, %d]", pool_blocks, kMaxPool);
+  const long long nblk = (capacity_of(cache) + csa2::kBlock - 1) / csa2::kBlock;
+  if (nblk > kMaxPoolSelectBlocks)
+    return fail(CSA2_ERR_SHAPE, "request capacity %lld positions exceeds the pool-select limit of %lld",
+                capacity_of(cache), kMaxPoolSelectBlocks * csa2::kBlock);
+  DeviceInfo d;
+  CSA2_TRY(device_info(&d));
+  const int cluster = nblk <= 8LL * 16384 ? 8 : 16;
+  const cudaError_t e = csa2::launch_pool_select(*cache, blockmax, pool_blocks, pool, cluster,
+                                                 static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? CSA2_OK : cuda_fail(e, "pool_select launch");
+}
+
+csa2_status csa2_reindex(const csa2_cache* cache, csa2_mode mode, const int32_t* pool, int32_t pool_blocks,
+                         const float* q, const float* w, const float* full_scores, const int32_t* prev_topk,
+                         int32_t k, int32_t* topk, void* stream) {
+  CSA2_TRY(check_cache(cache, false, mode != CSA2_REUSE));
+  if (k < 1 || k > kMaxK) return fail(CSA2_ERR_SHAPE, "k %d outside [1, %d]", k, kMaxK);
+  if (topk == nullptr) return fail(CSA2_ERR_ARG, "topk must be set");
+  if (mode != CSA2_FULL && mode != CSA2_REINDEX && mode != CSA2_REUSE)
+    return fail(CSA2_ERR_ARG, "unknown mode %d", static_cast<int>(mode));
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (mode == CSA2_REUSE) {
+    if (prev_topk == nullptr) return fail(CSA2_ERR_ARG, "REUSE needs prev_topk");
+    if (prev_topk == topk) return CSA2_OK;
+    DeviceInfo d;
+    CSA2_TRY(device_info(&d));
+    const cudaError_t e = csa2::launch_copy_topk(prev_topk, topk, static_cast<long long>(cache->batch) * k, s);
+    return e == cudaSuccess ? CSA2_OK : cuda_fail(e, "reuse copy launch");
+  }
+  const float* stored = mode == CSA2_FULL ? full_scores : nullptr;
+  if (stored == nullptr && (q == nullptr || w == nullptr || !aligned(q, 16)))
+    return fail(CSA2_ERR_ARG, "re-scoring needs q (16-byte aligned) and w");
+  int max_blocks;
+  if (pool != nullptr) {
+    if (pool_blocks < 1 || pool_blocks > kMaxPool)
+      return fail(CSA2_ERR_SHAPE, "pool_blocks %d outside [1, %d]", pool_blocks, kMaxPool);
+    max_blocks = (pool_blocks + 7) / 8;
+  } else {
+    if (capacity_of(cache) > kMaxFlatPositions)
+      return fail(CSA2_ERR_SHAPE, "Top-k without a pool supports request capacity <= %lld positions (got %lld)",
+                  kMaxFlatPositions, capacity_of(cache));
+    const long long nblk = (capacity_of(cache) + csa2::kBlock - 1) / csa2::kBlock;
+    max_blocks = static_cast<int>((nblk + 7) / 8);
+  }
+  DeviceInfo d;
+  CSA2_TRY(device_info(&d));
+  CUtensorMap map;
+  CSA2_TRY(encode_ik_map(cache, csa2::kBlock, &map));
+  const cudaError_t e = csa2::launch_reindex(*cache, pool, pool_blocks, q, w, stored, k, topk, map, max_blocks,
+                                             g_wait_limit_ns, s);
+  return e == cudaSuccess ? CSA2_OK : cuda_fail(e, "reindex launch");
+}
+
+csa2_status csa2_sparse_attn(const csa2_cache* cache, int32_t n_queries, const int32_t* q_req, const int32_t* topk,
+                             int32_t k, const uint16_t* q, int32_t H, float scale, uint16_t* out, void* stream) {
+  CSA2_TRY(check_cache(cache, true, false));
+  if (n_queries < 0) return fail(CSA2_ERR_SHAPE, "n_queries %d < 0", n_queries);
+  if (n_queries == 0) return CSA2_OK;
+  if (q_req == nullptr && n_queries > cache->batch)
+    return fail(CSA2_ERR_SHAPE, "without q_req, n_queries (%d) must not exceed batch (%d)", n_queries, cache->batch);
+  if (H != 16 && H != 32 && H != 64) return fail(CSA2_ERR_SHAPE, "H %d not in {16, 32, 64}", H);
+  if (k < 1 || k > kMaxK) return fail(CSA2_ERR_SHAPE, "k %d outside [1, %d]", k, kMaxK);
+  if (topk == nullptr || q == nullptr || out == nullptr || !aligned(q, 16) || !aligned(out, 16))
+    return fail(CSA2_ERR_ARG, "topk, q and out (16-byte aligned) must be set");
+  DeviceInfo d;
+  CSA2_TRY(device_info(&d));
+  const cudaError_t e = csa2::launch_sparse_attn(*cache, n_queries, q_req, topk, k, q, H, scale, out,
+                                                 static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? CSA2_OK : cuda_fail(e, "sparse_attn launch");
+}
+
+csa2_status csa2_get_error(const csa2_cache* cache, int32_t* out, void* stream) {
+  if (cache == nullptr || cache->err_word == nullptr || out == nullptr)
+    return fail(CSA2_ERR_ARG, "cache, cache.err_word and out must be set");
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  e = cudaMemcpy(out, cache->err_word, 4 * sizeof(int32_t), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpy(err_word)");
+  return static_cast<csa2_status>(out[0]);
+}
+
+const char* csa2_status_string(csa2_status s) {
+  switch (s) {
+    case CSA2_OK: return "ok";
+    case CSA2_ERR_ARG: return "invalid argument";
+    case CSA2_ERR_SHAPE: return "unsupported shape";
+    case CSA2_ERR_CUDA: return "CUDA runtime error";
+    case CSA2_ERR_DEVICE_BOUNDS: return "out-of-range page or position found on the device";
+    case CSA2_ERR_TIMEOUT: return "a pipeline wait on the device gave up";
+    case CSA2_ERR_UNSUPPORTED: return "unsupported device or feature";
+  }
+  return "unknown status";
+}
+
+const char* csa2_last_error_message(void) { return g_msg; }
+
+void csa2_set_wait_limit_ns(uint64_t ns) { g_wait_limit_ns = ns; }
+
+}  // extern "C"

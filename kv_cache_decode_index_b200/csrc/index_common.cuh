@@ -1,0 +1,62 @@
+// Pieces shared by the Full scan (csa2_index_full) and the pool re-score
+// (csa2_reindex), so that both produce bit-identical fp32 scores:
+//   * quantisation of one request's indexer query into the swizzled B-operand
+//     tile (32 heads x 128 FP8 codes) plus w_h * sigma^q_h per head;
+//   * the score epilogue  s_t = sigma_t * sum_h (w_h sigma^q_h) * ReLU(acc_h)
+//     with a fixed summation order h = 0..31 (fp32 FMA).
+// Score reading (the pages give none): s_t = sigma_t * sum_h w_h *
+// ReLU(sigma^q_h <q^_h, k^_t>) [4sapi blog, section 四: 32 heads x 128].
+#pragma once
+
+#include "common.cuh"
+
+namespace csa2 {
+
+constexpr int kTileBytes = kTile * kIndexDim;          // 16 KB: 128 rows x 128 B
+constexpr int kQBytes = kIndexHeads * kIndexDim;       // 4 KB: 32 rows x 128 B
+constexpr int kAccCols = 32;                           // fp32 columns per accumulator (N = 32 heads)
+constexpr uint32_t kIdesc = idesc_e4m3_f32(kTile, kIndexHeads);
+
+// Byte offset of (row, byte c) in a 128-byte-swizzled tile of 128-byte rows.
+__device__ __forceinline__ uint32_t sw128_offset(uint32_t row, uint32_t c) {
+  return row * 128u + ((((c >> 4) ^ row) & 7u) << 4) + (c & 15u);
+}
+
+// Quantise heads 8*ew .. 8*ew+7 of query q[32][128] (fp32, row-major) into
+// `qtile` (swizzled FP8 codes).  One warp per call; four warps cover a query.
+__device__ __forceinline__ void prepare_query_codes(const float* __restrict__ q, uint8_t* qtile, int ew, int lane) {
+#pragma unroll 1
+  for (int hh = 0; hh < 8; ++hh) {
+    const int h = ew * 8 + hh;
+    const float4 v = reinterpret_cast<const float4*>(q + h * kIndexDim)[lane];
+    float m = fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w)));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    const float inv = exp2i(-indexer_exponent(m));
+    const uint32_t codes = e4m3x2(v.x * inv, v.y * inv) | (e4m3x2(v.z * inv, v.w * inv) << 16);
+    *reinterpret_cast<uint32_t*>(qtile + sw128_offset(h, 4u * lane)) = codes;
+  }
+}
+
+// ws[h] = w[h] * sigma^q_h for all 32 heads, in every lane of the calling warp.
+__device__ __forceinline__ void load_head_weights(const float* __restrict__ q, const float* __restrict__ w,
+                                                  float (&ws)[32], int lane) {
+#pragma unroll
+  for (int h = 0; h < 32; ++h) {
+    const float4 v = reinterpret_cast<const float4*>(q + h * kIndexDim)[lane];
+    float m = fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w)));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    ws[h] = w[h] * exp2i(indexer_exponent(m));
+  }
+}
+
+// Score of one position from its 32 fp32 head dot products.
+__device__ __forceinline__ float score_from_acc(const uint32_t (&acc)[32], const float (&ws)[32], uint32_t e_byte) {
+  float s = 0.0f;
+#pragma unroll
+  for (int h = 0; h < 32; ++h) s = fmaf(ws[h], fmaxf(__uint_as_float(acc[h]), 0.0f), s);
+  return s * exp2i(static_cast<int>(e_byte) - 127);
+}
+
+}  // namespace csa2

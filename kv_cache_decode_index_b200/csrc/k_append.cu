@@ -1,0 +1,82 @@
+// Quantise-on-append: one warp per new row.
+//
+// Main KV (512 fp32) -> 256 bytes of E2M1 pairs + 32 E4M3 scales; lane g owns
+// channel group g (16 channels): s = E4M3(amax / 6), codes = E2M1(x / s)
+// [FP4 main-KV format: 4sapi "DeepSeek V4.1 Flash CED/CSA2" blog, section 五;
+// animattoys article, section 把精度降到4比特].
+// Indexer K (128 fp32) -> 128 E4M3 bytes + one exponent byte, sigma = 2^e with
+// e the smallest integer such that 448 * 2^e >= amax (reading: the pages give
+// no indexer dtype).
+#include "fp4.cuh"
+#include "launch.h"
+
+namespace csa2 {
+
+__global__ void __launch_bounds__(256) append_kernel(csa2_cache cache, int n_rows, const float* __restrict__ kv_new,
+                                                     const float* __restrict__ ik_new,
+                                                     const int32_t* __restrict__ req,
+                                                     const int32_t* __restrict__ pos) {
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (warp >= n_rows) return;
+
+  const int b = req ? req[warp] : warp;
+  const int t = pos[warp];
+  const long long capacity = static_cast<long long>(cache.max_pages_per_req) * cache.page_size;
+  if (b < 0 || b >= cache.batch || t < 0 || t >= capacity) {
+    if (lane == 0) report_error(cache.err_word, CSA2_ERR_DEVICE_BOUNDS, kKAppend, b, t);
+    return;
+  }
+  const int page = cache.page_table[static_cast<long long>(b) * cache.max_pages_per_req + t / cache.page_size];
+  if (page < 0 || page >= cache.num_pages) {
+    if (lane == 0) report_error(cache.err_word, CSA2_ERR_DEVICE_BOUNDS, kKAppend, b, t);
+    return;
+  }
+  const long long row = static_cast<long long>(page) * cache.page_size + t % cache.page_size;
+
+  // ---- main KV: lane = channel group of 16 ----
+  const float4* src = reinterpret_cast<const float4*>(kv_new + static_cast<long long>(warp) * kKvDim) + lane * 4;
+  float x[16];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float4 v = src[i];
+    x[4 * i] = v.x; x[4 * i + 1] = v.y; x[4 * i + 2] = v.z; x[4 * i + 3] = v.w;
+  }
+  float amax = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(x[i]));
+  const uint32_t sc = e4m3_code_of_sixth(amax);
+  const float s = e4m3_value(sc);
+  uint32_t lo = 0, hi = 0;
+  if (s > 0.0f) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const uint32_t byte = e2m1_code(x[2 * i], s) | (e2m1_code(x[2 * i + 1], s) << 4);
+      if (i < 4) lo |= byte << (8 * i);
+      else hi |= byte << (8 * (i - 4));
+    }
+  }
+  reinterpret_cast<uint2*>(cache.kv_codes + row * kKvCodeBytes)[lane] = make_uint2(lo, hi);
+  cache.kv_scales[row * kKvScaleBytes + lane] = static_cast<uint8_t>(sc);
+
+  // ---- indexer K: lane = 4 consecutive elements ----
+  const float4 k = reinterpret_cast<const float4*>(ik_new + static_cast<long long>(warp) * kIndexDim)[lane];
+  float km = fmaxf(fmaxf(fabsf(k.x), fabsf(k.y)), fmaxf(fabsf(k.z), fabsf(k.w)));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) km = fmaxf(km, __shfl_xor_sync(0xffffffffu, km, o));
+  const int e = indexer_exponent(km);
+  const float inv = exp2i(-e);
+  const uint32_t codes = e4m3x2(k.x * inv, k.y * inv) | (e4m3x2(k.z * inv, k.w * inv) << 16);
+  reinterpret_cast<uint32_t*>(cache.ik_codes + row * kIndexDim)[lane] = codes;
+  if (lane == 0) cache.ik_exp[row] = static_cast<uint8_t>(e + 127);
+}
+
+cudaError_t launch_append(const csa2_cache& cache, int n_rows, const float* kv_new, const float* ik_new,
+                          const int32_t* req, const int32_t* pos, cudaStream_t stream) {
+  const int threads = 256;
+  const long long blocks = (static_cast<long long>(n_rows) * 32 + threads - 1) / threads;
+  append_kernel<<<static_cast<unsigned>(blocks), threads, 0, stream>>>(cache, n_rows, kv_new, ik_new, req, pos);
+  return cudaGetLastError();
+}
+
+}  // namespace csa2

@@ -1,0 +1,319 @@
+// Full-mode indexer scan (first stage of the Hierarchical Sparse Indexer):
+// every visible position of every request is scored against that request's
+// indexer query, and the max of each block of 8 positions is written out
+// [4sapi blog, section 四; alphalab analysis, section 2 CSA2: the first Full
+// layer scans the whole visible context].
+//
+// Design (sm_100a):
+//   * persistent grid, one CTA per SM; the concatenated tiles of all requests
+//     (128 positions each) are split into contiguous ranges, one per CTA;
+//   * warp 0 (one lane): TMA producer, 16 KB indexer-K tiles (128 rows x 128
+//     FP8 bytes, 128-byte swizzle) into a ring of kStages stages;
+//   * warp 1 (one lane): tcgen05.mma kind::f8f6f4, M = 128 positions, N = 32
+//     heads, K = 128 in 4 steps, fp32 accumulator in TMEM (two buffers);
+//   * warps 2..5: epilogue, one thread per position: tcgen05.ld of the 32
+//     head dot products, score, block max over 8 lanes, stores; they also
+//     quantise each request's query into the B-operand tile (two buffers).
+// Every mbarrier wait is bounded; a wait that runs out records
+// CSA2_ERR_TIMEOUT and the CTA leaves its loops, drains, frees TMEM, returns.
+#include <cub/block/block_scan.cuh>
+
+#include "index_common.cuh"
+#include "launch.h"
+
+namespace csa2 {
+
+namespace {
+
+constexpr int kStages = 8;
+constexpr int kThreads = 192;
+constexpr int kMaxBatchScan = 1024;
+constexpr int kScanItems = (kMaxBatchScan + kThreads - 1) / kThreads;
+constexpr uint32_t kTmemCols = 64;   // 2 accumulators x 32 columns
+
+struct __align__(1024) IndexSmem {
+  uint8_t tiles[kStages][kTileBytes];
+  uint8_t q[2][kQBytes];
+  int prefix[kMaxBatchScan + 1];       // tiles before request b
+  uint64_t full[kStages];
+  uint64_t empty[kStages];
+  uint64_t acc_full[2];
+  uint64_t acc_empty[2];
+  uint64_t q_full[2];
+  uint64_t drain;
+  uint32_t tmem_base;
+  volatile int abort_flag;
+};
+
+// Walks this CTA's tiles in order: request b, tile j inside it.
+struct TileIter {
+  const int* prefix;
+  int batch;
+  int b, j;
+  __device__ void init(const int* pre, int nb, int g) {
+    prefix = pre;
+    batch = nb;
+    int lo = 0, hi = nb - 1;   // last b with prefix[b] <= g
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (pre[mid] <= g) lo = mid;
+      else hi = mid - 1;
+    }
+    b = lo;
+    j = g - pre[lo];
+    skip_empty();
+  }
+  __device__ void skip_empty() {
+    while (b < batch && j >= prefix[b + 1] - prefix[b]) {
+      j = 0;
+      ++b;
+    }
+  }
+  __device__ void advance() {
+    ++j;
+    skip_empty();
+  }
+};
+
+__device__ __forceinline__ int next_request_with_tiles(const int* prefix, int batch, int b) {
+  ++b;
+  while (b < batch && prefix[b + 1] == prefix[b]) ++b;
+  return b;
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    index_full_kernel(const csa2_cache cache, const float* __restrict__ q, const float* __restrict__ w,
+                      float* __restrict__ blockmax, float* __restrict__ scores,
+                      const __grid_constant__ CUtensorMap ik_map, uint64_t wait_ns) {
+  extern __shared__ uint8_t smem_raw[];
+  IndexSmem& S = *reinterpret_cast<IndexSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31;
+  const int B = cache.batch;
+  const long long capacity = static_cast<long long>(cache.max_pages_per_req) * cache.page_size;
+
+  // ---- tiles per request, prefix sums ----
+  {
+    using Scan = cub::BlockScan<int, kThreads>;
+    __shared__ typename Scan::TempStorage scan_tmp;
+    int items[kScanItems];
+#pragma unroll
+    for (int i = 0; i < kScanItems; ++i) {
+      const int b = tid * kScanItems + i;
+      int n = 0;
+      if (b < B) {
+        n = cache.ctx_len[b];
+        n = n < 0 ? 0 : (n > capacity ? static_cast<int>(capacity) : n);
+      }
+      items[i] = (n + kTile - 1) / kTile;
+    }
+    int total;
+    Scan(scan_tmp).ExclusiveSum(items, items, total);
+#pragma unroll
+    for (int i = 0; i < kScanItems; ++i) {
+      const int b = tid * kScanItems + i;
+      if (b <= B) S.prefix[b] = items[i];
+    }
+    if (tid == 0) S.prefix[B] = total;
+  }
+  if (tid == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&S.full[s], 1);
+      mbar_init(&S.empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&S.acc_full[a], 1);
+      mbar_init(&S.acc_empty[a], 4);
+      mbar_init(&S.q_full[a], 4);   // one arrival per epilogue warp
+    }
+    mbar_init(&S.drain, 1);
+    S.abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&S.tmem_base, kTmemCols);
+    tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) tma_prefetch_map(&ik_map);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+
+  const int total = S.prefix[B];
+  const int G = gridDim.x;
+  const int t_begin = static_cast<int>((static_cast<long long>(total) * blockIdx.x) / G);
+  const int t_end = static_cast<int>((static_cast<long long>(total) * (blockIdx.x + 1)) / G);
+  const int n_tiles = t_end - t_begin;
+  const uint32_t tmem = S.tmem_base;
+
+  if (n_tiles > 0) {
+    if (warp == 0) {
+      // ================= TMA producer =================
+      if (lane == 0) {
+        const uint64_t policy = l2_policy_evict_first();
+        TileIter it;
+        it.init(S.prefix, B, t_begin);
+        int issued = 0;
+        for (int i = 0; i < n_tiles; ++i) {
+          const int s = i % kStages;
+          const uint32_t ph = (i / kStages) & 1;
+          if (!mbar_wait(&S.empty[s], ph ^ 1, wait_ns)) {
+            report_error(cache.err_word, CSA2_ERR_TIMEOUT, kKIndexFull, it.b, i);
+            S.abort_flag = 1;
+            break;
+          }
+          if (S.abort_flag) break;
+          const int p0 = it.j * kTile;
+          int page = cache.page_table[static_cast<long long>(it.b) * cache.max_pages_per_req + p0 / cache.page_size];
+          if (page < 0 || page >= cache.num_pages) {
+            report_error(cache.err_word, CSA2_ERR_DEVICE_BOUNDS, kKIndexFull, it.b, p0);
+            page = 0;   // load a valid page; the results of this tile are flagged invalid
+          }
+          const int row0 = page * cache.page_size + p0 % cache.page_size;
+          mbar_arrive_expect_tx(&S.full[s], kTileBytes);
+          tma_load_2d(S.tiles[s], &ik_map, &S.full[s], 0, row0, policy);
+          ++issued;
+          it.advance();
+        }
+        // loads still in flight (only after an abort): wait for the last one of each stage
+        for (int i = issued > kStages ? issued - kStages : 0; i < issued; ++i)
+          (void)mbar_wait(&S.full[i % kStages], (i / kStages) & 1, kWaitLimitNs / 2);
+      }
+    } else if (warp == 1) {
+      // ================= MMA issuer =================
+      if (lane == 0) {
+        TileIter it;
+        it.init(S.prefix, B, t_begin);
+        int seg = 0, cur_b = it.b;
+        bool ok = mbar_wait(&S.q_full[0], 0, wait_ns);
+        for (int i = 0; ok && i < n_tiles; ++i) {
+          if (it.b != cur_b) {
+            ++seg;
+            cur_b = it.b;
+            if (!mbar_wait(&S.q_full[seg & 1], (seg >> 1) & 1, wait_ns)) { ok = false; break; }
+          }
+          const int s = i % kStages;
+          const uint32_t ph = (i / kStages) & 1;
+          const int a = i & 1;
+          const uint32_t aph = (i >> 1) & 1;
+          if (!mbar_wait(&S.acc_empty[a], aph ^ 1, wait_ns)) { ok = false; break; }
+          if (!mbar_wait(&S.full[s], ph, wait_ns)) { ok = false; break; }
+          if (S.abort_flag) break;
+          tc_fence_after();
+          const uint64_t adesc = sw128_kmajor_desc(smem_u32(S.tiles[s]));
+          const uint64_t bdesc = sw128_kmajor_desc(smem_u32(S.q[seg & 1]));
+#pragma unroll
+          for (int k = 0; k < kIndexDim / 32; ++k)
+            umma_f8f6f4(tmem + a * kAccCols, adesc + 2 * k, bdesc + 2 * k, kIdesc, k > 0 ? 1u : 0u);
+          umma_commit(&S.empty[s]);
+          umma_commit(&S.acc_full[a]);
+          it.advance();
+        }
+        if (!ok) {
+          report_error(cache.err_word, CSA2_ERR_TIMEOUT, kKIndexFull, cur_b, -1);
+          S.abort_flag = 1;
+        }
+        umma_commit(&S.drain);                       // all MMAs issued above are complete
+        (void)mbar_wait(&S.drain, 0, kWaitLimitNs);
+      }
+    } else {
+      // ================= epilogue (warps 2..5) =================
+      const int ew = warp - 2;                 // 0..3: query-preparation share
+      const int quarter = warp & 3;            // TMEM lane quarter of this warp
+      const int toff = quarter * 32 + lane;    // position inside the tile
+      TileIter it;
+      it.init(S.prefix, B, t_begin);
+      int cur_b = it.b, seg = 0;
+      // queries of the first two segments
+      int prep_b = cur_b;
+      for (int k = 0; k < 2 && prep_b < B && S.prefix[prep_b] < t_end; ++k) {
+        prepare_query_codes(q + static_cast<long long>(prep_b) * kIndexHeads * kIndexDim, S.q[k], ew, lane);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&S.q_full[k]);
+        prep_b = next_request_with_tiles(S.prefix, B, prep_b);
+      }
+      float ws[32];
+      load_head_weights(q + static_cast<long long>(cur_b) * kIndexHeads * kIndexDim, w + cur_b * kIndexHeads, ws, lane);
+      int nb = cache.ctx_len[cur_b];
+
+      for (int i = 0; i < n_tiles; ++i) {
+        if (it.b != cur_b) {
+          // segment `seg` is fully consumed: its query buffer takes segment seg + 2
+          if (prep_b < B && S.prefix[prep_b] < t_end) {
+            prepare_query_codes(q + static_cast<long long>(prep_b) * kIndexHeads * kIndexDim, S.q[seg & 1], ew, lane);
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&S.q_full[seg & 1]);
+            prep_b = next_request_with_tiles(S.prefix, B, prep_b);
+          }
+          ++seg;
+          cur_b = it.b;
+          load_head_weights(q + static_cast<long long>(cur_b) * kIndexHeads * kIndexDim, w + cur_b * kIndexHeads, ws, lane);
+          nb = cache.ctx_len[cur_b];
+        }
+        const int a = i & 1;
+        const uint32_t aph = (i >> 1) & 1;
+        const int p0 = it.j * kTile;
+        const int p = p0 + toff;
+        const bool valid = p < nb;
+        int page = cache.page_table[static_cast<long long>(cur_b) * cache.max_pages_per_req + p0 / cache.page_size];
+        page = (page < 0 || page >= cache.num_pages) ? 0 : page;
+        const uint32_t e_byte = valid ? cache.ik_exp[static_cast<long long>(page) * cache.page_size + p0 % cache.page_size + toff] : 127u;
+
+        if (!mbar_wait_warp(&S.acc_full[a], aph, wait_ns)) {
+          if (lane == 0) {
+            report_error(cache.err_word, CSA2_ERR_TIMEOUT, kKIndexFull, cur_b, p0);
+            S.abort_flag = 1;
+          }
+          break;
+        }
+        tc_fence_after();
+        uint32_t acc[32];
+        tmem_ld_32x32b_x32(tmem + a * kAccCols + (static_cast<uint32_t>(quarter * 32) << 16), acc);
+        tmem_ld_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&S.acc_empty[a]);
+
+        const float sc = score_from_acc(acc, ws, e_byte);
+        float bm = valid ? sc : -INFINITY;
+        bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 1));
+        bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 2));
+        bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 4));
+        if ((lane & 7) == 0 && valid) blockmax[static_cast<long long>(cur_b) * (capacity / kBlock) + p / kBlock] = bm;
+        if (scores != nullptr && valid) scores[static_cast<long long>(cur_b) * capacity + p] = sc;
+        if (warp_flag(&S.abort_flag)) break;
+        it.advance();
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+}  // namespace
+
+size_t index_full_smem_bytes() { return sizeof(IndexSmem) + 1024; }
+
+cudaError_t launch_index_full(const csa2_cache& cache, const float* q, const float* w, float* blockmax,
+                              float* scores, const CUtensorMap& ik_map, int num_sms, uint64_t wait_ns,
+                              cudaStream_t stream) {
+  static bool configured = false;
+  const size_t smem = index_full_smem_bytes();
+  if (!configured) {
+    cudaError_t e = cudaFuncSetAttribute(index_full_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    configured = true;
+  }
+  index_full_kernel<<<num_sms, kThreads, smem, stream>>>(cache, q, w, blockmax, scores, ik_map, wait_ns);
+  return cudaGetLastError();
+}
+
+}  // namespace csa2

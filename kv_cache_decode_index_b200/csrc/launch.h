@@ -1,0 +1,35 @@
+// Host-side launchers of the CSA2 kernels (internal to libcsa2.so).  Each
+// returns the launch's cudaError_t; argument validation happens before, in
+// csa2_api.cu.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/csa2.h"
+
+namespace csa2 {
+
+cudaError_t launch_append(const csa2_cache& cache, int n_rows, const float* kv_new, const float* ik_new,
+                          const int32_t* req, const int32_t* pos, cudaStream_t stream);
+
+size_t index_full_smem_bytes();
+cudaError_t launch_index_full(const csa2_cache& cache, const float* q, const float* w, float* blockmax,
+                              float* scores, const CUtensorMap& ik_map, int num_sms, uint64_t wait_ns,
+                              cudaStream_t stream);
+
+cudaError_t launch_pool_select(const csa2_cache& cache, const float* blockmax, int pool_blocks, int32_t* pool,
+                               int cluster, cudaStream_t stream);
+
+cudaError_t launch_reindex(const csa2_cache& cache, const int32_t* pool, int pool_blocks, const float* q,
+                           const float* w, const float* full_scores, int k, int32_t* topk,
+                           const CUtensorMap& ik_blk_map, int cands_per_cta, uint64_t wait_ns, cudaStream_t stream);
+
+cudaError_t launch_copy_topk(const int32_t* src, int32_t* dst, long long n, cudaStream_t stream);
+
+cudaError_t launch_sparse_attn(const csa2_cache& cache, int n_queries, const int32_t* q_req, const int32_t* topk,
+                               int k, const uint16_t* q, int H, float scale, uint16_t* out, cudaStream_t stream);
+
+}  // namespace csa2

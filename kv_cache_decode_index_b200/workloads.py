@@ -109,9 +109,10 @@ def ctx_lengths(wl: Workload) -> np.ndarray:
     return np.floor(np.exp(np.log(lo) + u * (np.log(hi) - np.log(lo)))).astype(np.int64)
 
 
-def page_layout(wl: Workload):
-    """(page_table int32 [B, max_pages], num_pages).  Unused slots hold -1."""
-    n = ctx_lengths(wl)
+def page_layout(wl: Workload, lengths=None):
+    """(page_table int32 [B, max_pages], num_pages).  Unused slots hold -1.
+    `lengths` overrides the workload's context lengths."""
+    n = ctx_lengths(wl) if lengths is None else np.asarray(lengths, dtype=np.int64)
     per = -(-n // wl.page_size)
     max_pages = int(per.max())
     num_pages = int(per.sum())

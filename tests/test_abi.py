@@ -1,0 +1,74 @@
+"""The C-ABI library loads, exports every symbol include/csa2.h declares, and
+rejects bad arguments on the host before touching a GPU (no device needed)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "csa2.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from kv_cache_decode_index_b200 import build
+    build.build()
+    from kv_cache_decode_index_b200 import csa2
+    return csa2
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return re.findall(r"CSA2_API\s+[\w\s\*]+?\b(csa2_\w+)\s*\(", text)
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_symbols()
+    assert len(names) == 9, names
+    so = ctypes.CDLL(lib.LIB_PATH)
+    for n in names:
+        assert hasattr(so, n), f"{n} missing from libcsa2.so"
+
+
+def _cache(lib, **over):
+    buf = (ctypes.c_uint8 * 4096)()
+    base = (ctypes.addressof(buf) + 255) & ~255
+    f = dict(kv_codes=base, kv_scales=base, ik_codes=base, ik_exp=base, page_table=base, ctx_len=base,
+             num_pages=4, page_size=128, max_pages_per_req=2, batch=2, err_word=base)
+    f.update(over)
+    c = lib.CacheStruct(**f)
+    c._keep = buf
+    return c, base
+
+
+def test_host_side_validation(lib):
+    L = lib._lib
+    c, p = _cache(lib)
+    P = ctypes.c_void_p(p)
+    assert L.csa2_index_full(None, P, P, P, None, None) == lib.ERR_ARG
+    bad, _ = _cache(lib, batch=0)
+    assert L.csa2_index_full(ctypes.byref(bad), P, P, P, None, None) == lib.ERR_SHAPE
+    bad, _ = _cache(lib, page_size=100)
+    assert L.csa2_pool_select(ctypes.byref(bad), P, 2048, P, None) == lib.ERR_SHAPE
+    bad, _ = _cache(lib, ik_codes=p + 4)
+    assert L.csa2_index_full(ctypes.byref(bad), P, P, P, None, None) == lib.ERR_ARG
+    assert b"16-byte" in L.csa2_last_error_message()
+    assert L.csa2_pool_select(ctypes.byref(c), P, 0, P, None) == lib.ERR_SHAPE
+    assert L.csa2_reindex(ctypes.byref(c), lib.REINDEX, P, 2048, P, P, None, None, 0, P, None) == lib.ERR_SHAPE
+    assert L.csa2_reindex(ctypes.byref(c), 7, P, 2048, P, P, None, None, 512, P, None) == lib.ERR_ARG
+    assert L.csa2_reindex(ctypes.byref(c), lib.REUSE, None, 0, None, None, None, None, 512, P, None) == lib.ERR_ARG
+    assert L.csa2_sparse_attn(ctypes.byref(c), 2, None, P, 512, P, 48, ctypes.c_float(0.1), P, None) == lib.ERR_SHAPE
+    assert L.csa2_sparse_attn(ctypes.byref(c), 3, None, P, 512, P, 64, ctypes.c_float(0.1), P, None) == lib.ERR_SHAPE
+    assert L.csa2_append_kv(ctypes.byref(c), -1, P, P, None, P, None) == lib.ERR_SHAPE
+    assert L.csa2_append_kv(ctypes.byref(c), 0, P, P, None, P, None) == lib.OK   # nothing to do
+    big, _ = _cache(lib, max_pages_per_req=2048, page_size=4096)
+    assert L.csa2_reindex(ctypes.byref(big), lib.FULL, None, 0, P, P, None, None, 512, P, None) == lib.ERR_SHAPE
+    assert L.csa2_status_string(lib.ERR_TIMEOUT) == b"a pipeline wait on the device gave up"
+
+
+def test_binding_rejects_wrong_tensors(lib):
+    import torch
+    c = lib.Cache.__new__(lib.Cache)
+    with pytest.raises(ValueError):
+        lib._need(torch.zeros(3, dtype=torch.float32), torch.int32, (3,), "x")

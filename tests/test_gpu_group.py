@@ -1,0 +1,185 @@
+"""End-to-end parity of one CSA2 layer-group decode step (DecodeGroup through
+the C ABI) against the float64 oracle: pool, every layer's Top-k, and the
+attention outputs.  Needs a B200 and libcsa2.so."""
+import numpy as np
+import pytest
+import torch
+
+from kv_cache_decode_index_b200 import workloads as W
+from oracle import csa2 as C
+from tests import gpu_util as U
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def csa2():
+    from kv_cache_decode_index_b200 import csa2 as lib
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    return lib
+
+
+def _queries(wl, dev):
+    q_idx, w_idx, q_main = [], [], []
+    for layer, m in enumerate(wl.modes):
+        if m == "Ru":
+            q_idx.append(None)
+            w_idx.append(None)
+        else:
+            q, w = W.index_query(wl, layer)
+            q_idx.append(q)
+            w_idx.append(w)
+        q_main.append(W.main_query(wl, layer))
+    tq = [None if q is None else torch.from_numpy(q).to(dev) for q in q_idx]
+    tw = [None if w is None else torch.from_numpy(w).to(dev) for w in w_idx]
+    tm = [m.to(dev) for m in q_main]
+    return q_idx, w_idx, q_main, tq, tw, tm
+
+
+def _run_gpu(csa2, wl, cache, dev, append_rows=None):
+    q_idx, w_idx, q_main, tq, tw, tm = _queries(wl, dev)
+    group = csa2.DecodeGroup(cache, wl.modes, wl.heads, wl.topk, wl.pool_blocks, wl.scale)
+    out = [torch.empty_like(m) for m in tm]
+    if append_rows is not None:
+        kv, ik, pos = append_rows
+        csa2.append_kv(cache, kv, ik, pos)
+    group.step(tq, tw, tm, out)
+    torch.cuda.synchronize()
+    return group, q_idx, w_idx, q_main, out
+
+
+def _check_request(csa2, wl, cache, group, b, n, q_idx, w_idx, q_main, out, dev):
+    """Full oracle of request b and comparison under the parity rules."""
+    codes, exp = U.oracle_request(wl, b, n)
+    ora = C.decode_group(wl.modes, [None if q is None else q[b] for q in q_idx],
+                         [None if w is None else w[b] for w in w_idx], codes, exp, n, wl.pool_blocks, wl.topk)
+    s64 = ora["scores"]
+    excused = lambda t: False
+    if wl.pool_blocks:
+        gp = group.pool[b].cpu().numpy()
+        U.assert_sorted_padded(gp, f"pool b={b}")
+        bm64 = ora["blockmax"]
+        diff = U.assert_set_parity(gp, ora["pool"], lambda j: bm64[j], U.threshold(bm64, wl.pool_blocks),
+                                   what=f"pool b={b}")
+        pool_diff = set(gp[gp >= 0].tolist()) ^ set(ora["pool"][ora["pool"] >= 0].tolist())
+        excused = lambda t: (t // 8) in pool_diff
+        gpu_pool_pos = set(C.pool_positions(gp, n).tolist())
+    layer_scores = {}
+    for layer, m in enumerate(wl.modes):
+        gt = group.topk[layer][b].cpu().numpy()
+        U.assert_sorted_padded(gt, f"topk layer {layer} b={b}")
+        if m == "Ru":
+            np.testing.assert_array_equal(gt, group.topk[layer - 1][b].cpu().numpy())
+            layer_scores[layer] = layer_scores[layer - 1]
+            continue
+        if wl.pool_blocks:
+            assert set(gt[gt >= 0].tolist()) <= gpu_pool_pos, f"layer {layer} selects outside the pool"
+        if m == "F":
+            sc = s64
+        else:
+            sc = C.indexer_scores(q_idx[layer][b], w_idx[layer][b], codes, exp)
+        layer_scores[layer] = sc
+        ot = ora["topk"][layer]
+        cand = np.arange(n) if not wl.pool_blocks else C.pool_positions(ora["pool"], n)
+        U.assert_set_parity(gt, ot, lambda t: sc[t], U.threshold(sc[cand], wl.topk), excused,
+                            what=f"topk layer {layer} ({m}) b={b}")
+    # attention: GPU kernel fed the oracle's indices vs the oracle
+    sel = np.unique(np.concatenate([t[t >= 0] for t in ora["topk"]]))
+    kvc, kvs = U.oracle_kv_rows(wl, b, sel)
+    full_c = np.zeros((n, 256), np.uint8)
+    full_s = np.zeros((n, 32), np.uint8)
+    full_c[sel], full_s[sel] = kvc, kvs
+    worst = 0.0
+    for layer in range(len(wl.modes)):
+        ot = ora["topk"][layer].astype(np.int32)
+        ref = C.sparse_attention(q_main[layer][b].float().numpy(), full_c, full_s, ot, wl.scale)
+        qi = torch.tensor([b], dtype=torch.int32, device=dev)
+        g = csa2.sparse_attn(cache, torch.from_numpy(ot[None]).to(dev), q_main[layer][b:b + 1].to(dev), wl.scale,
+                             q_req=qi).float().cpu().numpy()[0]
+        worst = max(worst, U.assert_attention_close(g, ref, f"attention layer {layer} b={b}"))
+        if np.array_equal(group.topk[layer][b].cpu().numpy(), ot):
+            np.testing.assert_array_equal(out[layer][b].float().cpu().numpy(), g)
+    return ora, worst
+
+
+def test_group_full_4k_b1(csa2):
+    wl = W.WORKLOADS["full_4k_b1"]
+    cache = U.build_cache(wl, csa2)
+    dev = cache.device
+    group, q_idx, w_idx, q_main, out = _run_gpu(csa2, wl, cache, dev)
+    _, worst = _check_request(csa2, wl, cache, group, 0, 4096, q_idx, w_idx, q_main, out, dev)
+    print(f"max attention rel err {worst:.2e}")
+    assert csa2.get_error(cache)[0] == csa2.OK
+
+
+def test_group_64k_b8(csa2):
+    wl = W.WORKLOADS["group_64k_b8"]
+    cache = U.build_cache(wl, csa2)
+    dev = cache.device
+    group, q_idx, w_idx, q_main, out = _run_gpu(csa2, wl, cache, dev)
+    for b in range(wl.batch):
+        _check_request(csa2, wl, cache, group, b, 65536, q_idx, w_idx, q_main, out, dev)
+    assert csa2.get_error(cache)[0] == csa2.OK
+
+
+def test_group_ragged_paged_with_append(csa2):
+    """Ragged contexts behind a shuffled page table; one FP4 append per request
+    precedes the step (1 Full + 4 Reindex + 1 Reuse)."""
+    wl = W.scaled(W.WORKLOADS["ragged_b64"], batch=12, ctx_range=(4096, 300000))
+    n = W.ctx_lengths(wl)
+    cache = U.build_cache(wl, csa2, append_last=True)
+    dev = cache.device
+    last = n - 1
+    kv = np.stack([W.rows_at(wl, b, [last[b]], "kv")[0] for b in range(wl.batch)])
+    ik = np.stack([W.rows_at(wl, b, [last[b]], "ik")[0] for b in range(wl.batch)])
+    rows = (torch.from_numpy(kv).to(dev), torch.from_numpy(ik).to(dev),
+            torch.from_numpy(last.astype(np.int32)).to(dev))
+    group, q_idx, w_idx, q_main, out = _run_gpu(csa2, wl, cache, dev, append_rows=rows)
+    from oracle import formats as F
+    ikc, ike = F.quantize_indexer(ik)
+    for b in range(wl.batch):
+        row = int(cache.rows_of(b, [last[b]])[0])
+        np.testing.assert_array_equal(cache.ik_codes[row].cpu().numpy(), ikc[b])
+        assert int(cache.ik_exp[row]) == int(ike[b])
+        _check_request(csa2, wl, cache, group, b, int(n[b]), q_idx, w_idx, q_main, out, dev)
+    assert csa2.get_error(cache)[0] == csa2.OK
+
+
+def test_group_1m_b4_full_size(csa2):
+    """The 1M-context workload at full size, in the bench's launch configuration:
+    request 0 against the full oracle; requests 1..3 on sampled blocks and on
+    properties that hold at any size."""
+    wl = W.WORKLOADS["group_1m_b4"]
+    cache = U.build_cache(wl, csa2)
+    dev = cache.device
+    group, q_idx, w_idx, q_main, out = _run_gpu(csa2, wl, cache, dev)
+    n = wl.ctx
+    ora, worst = _check_request(csa2, wl, cache, group, 0, n, q_idx, w_idx, q_main, out, dev)
+    needles = W.needle_positions(wl, 0)
+    ora_recall = np.isin(needles // 8, ora["pool"]).sum()
+    gpu_recall = np.isin(needles // 8, group.pool[0].cpu().numpy()).sum()
+    print(f"needle pool recall: oracle {ora_recall}/64, gpu {gpu_recall}/64; attention rel err {worst:.2e}")
+    assert ora_recall == gpu_recall
+    bm_all = group.blockmax.cpu().numpy()
+    rng = np.random.default_rng(0)
+    for b in range(1, wl.batch):
+        bm = bm_all[b, :n // 8].astype(np.float64)
+        gp = group.pool[b].cpu().numpy()
+        # pool = exact top-2048 of the GPU's block maxima (ties -> lower id)
+        order = np.lexsort((np.arange(len(bm)), -bm))
+        np.testing.assert_array_equal(gp, np.sort(order[:2048]))
+        # sampled block maxima (including the needles' blocks) against the oracle
+        blocks = np.unique(np.concatenate([rng.choice(n // 8, 200, replace=False),
+                                           W.needle_positions(wl, b) // 8]))
+        pos = (blocks[:, None] * 8 + np.arange(8)).reshape(-1)
+        from oracle import formats as F
+        codes, exp = F.quantize_indexer(W.rows_at(wl, b, pos, "ik"))
+        s64 = C.indexer_scores(q_idx[0][b], w_idx[0][b], codes, exp)
+        bm64 = s64.reshape(-1, 8).max(axis=1)
+        assert np.all(np.abs(bm[blocks] - bm64) <= 1e-5 * np.abs(bm64))
+        pool_pos = set(C.pool_positions(gp, n).tolist())
+        for layer, m in enumerate(wl.modes):
+            t = group.topk[layer][b].cpu().numpy()
+            U.assert_sorted_padded(t)
+            assert (t >= 0).sum() == 512 and set(t.tolist()) <= pool_pos
+    assert csa2.get_error(cache)[0] == csa2.OK

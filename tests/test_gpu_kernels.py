@@ -1,0 +1,366 @@
+"""Stage-by-stage parity of the CUDA kernels (through the C ABI) against the
+float64 oracle, on the same seeded inputs.  Needs a B200 and libcsa2.so."""
+import json
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from kv_cache_decode_index_b200 import workloads as W
+from oracle import csa2 as C
+from oracle import formats as F
+from tests import gpu_util as U
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def csa2():
+    from kv_cache_decode_index_b200 import csa2 as lib
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    return lib
+
+
+def _flat_cache(csa2, rows, batch=1, page_size=512):
+    """One request (or `batch` requests) over contiguous pages, no data."""
+    per = -(-rows // page_size)
+    table = np.arange(batch * per, dtype=np.int32).reshape(batch, per)
+    return csa2.Cache(batch * per, page_size, table, [rows] * batch)
+
+
+# ------------------------------------------------------------ append (a1) --
+
+def _special_kv_rows(rng, golden_dir):
+    rows = []
+    with open(os.path.join(golden_dir, "fp4_hand_cases.json")) as f:
+        for g in json.load(f)["groups"]:
+            r = np.zeros(512, np.float32)
+            r[:16] = g["x"]
+            rows.append(r)
+    mids = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0, 0.5, 1, 1.5, 2, 3, 4, 6, 0, 7])
+    for _ in range(64):
+        r = np.zeros(512, np.float32)
+        for g in range(32):
+            c = rng.integers(1, 127)
+            s = F.e4m3_value(c)
+            v = rng.choice(mids, 16) * s * rng.choice([-1, 1], 16)
+            v[rng.integers(16)] = 6 * s                      # amax/6 = s exactly
+            if g % 4 == 0 and c < 126:                        # amax/6 on an E4M3 midpoint
+                v[0] = 3 * (s + F.e4m3_value(c + 1))
+            r[16 * g:16 * g + 16] = v
+        rows.append(r)
+    rows.append(np.zeros(512, np.float32))
+    rows.append(np.full(512, -0.0, np.float32))
+    return np.stack(rows).astype(np.float32)
+
+
+def _special_ik_rows(rng, golden_dir):
+    rows = []
+    with open(os.path.join(golden_dir, "fp8_indexer_hand_cases.json")) as f:
+        for g in json.load(f)["rows"]:
+            r = np.zeros(128, np.float32)
+            r[:len(g["k_head"])] = g["k_head"]
+            rows.append(r)
+    vals = np.unique(np.abs(F.e4m3_value(np.arange(127))))
+    mids = (vals[:-1] + vals[1:]) / 2
+    for _ in range(64):
+        e = rng.integers(-20, 20)
+        r = rng.choice(np.concatenate([vals, mids]), 128) * np.exp2(float(e)) * rng.choice([-1, 1], 128)
+        r[rng.integers(128)] = 448 * np.exp2(float(e))
+        rows.append(r)
+    rows += [np.zeros(128), np.full(128, 1e-40), np.full(128, 3e38)]
+    return np.stack(rows).astype(np.float32)
+
+
+def test_append_bitexact(csa2, golden_dir):
+    rng = np.random.default_rng(0)
+    kv_s = _special_kv_rows(rng, golden_dir)
+    ik_s = _special_ik_rows(rng, golden_dir)
+    n_rand = 700
+    kv = np.concatenate([kv_s, (rng.standard_normal((n_rand, 512)) *
+                                np.exp(rng.standard_normal(512) * 2)).astype(np.float32)])
+    ik = np.concatenate([ik_s, (rng.standard_normal((n_rand + len(kv_s) - len(ik_s), 128)) *
+                                np.exp(rng.uniform(-25, 25, (n_rand + len(kv_s) - len(ik_s), 1)))).astype(np.float32)])
+    n = len(kv)
+    cache = _flat_cache(csa2, n)
+    dev = cache.device
+    perm = rng.permutation(n).astype(np.int32)          # scattered positions
+    csa2.append_kv(cache, torch.from_numpy(kv).to(dev), torch.from_numpy(ik).to(dev),
+                   torch.from_numpy(perm).to(dev), torch.zeros(n, dtype=torch.int32, device=dev))
+    codes, scales = F.quantize_main_kv(kv)
+    ikc, ike = F.quantize_indexer(ik)
+    inv = np.argsort(perm)
+    g_codes = cache.kv_codes[:n].cpu().numpy()[perm]
+    g_scales = cache.kv_scales[:n].cpu().numpy()[perm]
+    g_ikc = cache.ik_codes[:n].cpu().numpy()[perm]
+    g_ike = cache.ik_exp[:n].cpu().numpy()[perm]
+    np.testing.assert_array_equal(g_scales, scales)
+    np.testing.assert_array_equal(g_codes, codes)
+    np.testing.assert_array_equal(g_ike, ike)
+    np.testing.assert_array_equal(g_ikc, ikc)
+    assert inv is not None
+    assert csa2.get_error(cache)[0] == csa2.OK
+
+
+def test_append_one_row_per_request(csa2):
+    """req = NULL: row i goes to request i (the decode-step append)."""
+    rng = np.random.default_rng(1)
+    B = 5
+    cache = _flat_cache(csa2, 256, batch=B, page_size=128)
+    kv = rng.standard_normal((B, 512)).astype(np.float32)
+    ik = rng.standard_normal((B, 128)).astype(np.float32)
+    pos = np.array([0, 255, 128, 7, 200], np.int32)
+    dev = cache.device
+    csa2.append_kv(cache, torch.from_numpy(kv).to(dev), torch.from_numpy(ik).to(dev), torch.from_numpy(pos).to(dev))
+    codes, scales = F.quantize_main_kv(kv)
+    ikc, ike = F.quantize_indexer(ik)
+    for b in range(B):
+        row = int(cache.rows_of(b, [pos[b]])[0])
+        np.testing.assert_array_equal(cache.kv_codes[row].cpu().numpy(), codes[b])
+        np.testing.assert_array_equal(cache.kv_scales[row].cpu().numpy(), scales[b])
+        np.testing.assert_array_equal(cache.ik_codes[row].cpu().numpy(), ikc[b])
+        assert int(cache.ik_exp[row]) == int(ike[b])
+
+
+# --------------------------------------------------------- index_full (a2) --
+
+def _score_bound(q, w, codes, exp):
+    """fp32 error bound of the tensor-core score: every head dot product within
+    2^-22 of its absolute sum, plus the 32-term fp32 sum (32 * 2^-24)."""
+    qc, sq = C.quantize_index_query(q)
+    qa = np.abs(F.e4m3_value(qc))
+    ka = np.abs(F.e4m3_value(codes))
+    absdot = ka @ qa.T * sq
+    sig = F.indexer_sigma(exp)
+    w64 = np.abs(w.astype(np.float64))
+    return sig * (absdot @ w64) * 2.0 ** -22 * 2, sig
+
+
+def test_index_full_scores_ragged(csa2):
+    wl = W.scaled(W.WORKLOADS["group_64k_b8"], batch=5, page_size=512, shuffle_pages=True)
+    lengths = [4096, 1, 1000, 9999, 128 * 37]
+    cache = U.build_cache(wl, csa2, lengths=lengths)
+    q, w = W.index_query(wl, 0)
+    dev = cache.device
+    bm = torch.full((5, cache.capacity // 8), float("nan"), device=dev)
+    sc = torch.full((5, cache.capacity), float("nan"), device=dev)
+    csa2.index_full(cache, torch.from_numpy(q).to(dev), torch.from_numpy(w).to(dev), bm, sc)
+    bm, sc = bm.cpu().numpy(), sc.cpu().numpy()
+    worst = 0.0
+    for b, n in enumerate(lengths):
+        codes, exp = U.oracle_request(wl, b, n)
+        s64 = C.indexer_scores(q[b], w[b], codes, exp)
+        bound, _ = _score_bound(q[b], w[b], codes, exp)
+        err = np.abs(sc[b, :n].astype(np.float64) - s64)
+        assert np.all(err <= bound + 1e-30), f"request {b}: score error beyond the fp32 bound"
+        worst = max(worst, float((err / np.maximum(s64, 1e-30)).max()))
+        assert np.all(np.isnan(sc[b, n:]))                          # nothing written past ctx
+        nb = -(-n // 8)
+        ref = C.block_max(sc[b, :n].astype(np.float64), n)
+        np.testing.assert_array_equal(bm[b, :nb].astype(np.float64), ref)   # GPU blockmax = max of GPU scores
+        assert np.all(np.isnan(bm[b, nb:]))
+        bm64 = C.block_max(s64, n)
+        assert np.all(np.abs(bm[b, :nb] - bm64) <= np.abs(bm64) * 1e-5)
+    print(f"max relative score error {worst:.3e}")
+    assert csa2.get_error(cache)[0] == csa2.OK
+
+
+# ------------------------------------------------------- pool_select (a3) --
+
+@pytest.mark.parametrize("lengths,P", [([1048576, 300000], 2048), ([16384, 16383, 8, 0], 2048),
+                                       ([200000, 5000], 64), ([1500000], 2048)])
+def test_pool_select_bitexact(csa2, lengths, P):
+    """Synthetic block maxima with many ties (and negative values), fed to both."""
+    rng = np.random.default_rng(len(lengths) * 1000 + P)
+    B = len(lengths)
+    page = 4096
+    per = max(-(-max(lengths) // page), 1)
+    table = np.arange(B * per, dtype=np.int32).reshape(B, per)
+    cache = csa2.Cache(B * per, page, table, lengths)
+    cap8 = cache.capacity // 8
+    vals = rng.standard_normal((B, cap8)).astype(np.float32)
+    vals[:, ::3] = np.round(vals[:, ::3] * 4) / 4                       # ties
+    vals[:, 5::7] = 2.0                                                  # a big tie group
+    dev = cache.device
+    pool = csa2.pool_select(cache, torch.from_numpy(vals).to(dev), P).cpu().numpy()
+    for b, n in enumerate(lengths):
+        nb = -(-n // 8)
+        ref = C.pool_select(vals[b, :nb].astype(np.float64), P)
+        np.testing.assert_array_equal(pool[b], ref, err_msg=f"request {b} (n={n})")
+
+
+# ---------------------------------------------------------- reindex (a4-a6) --
+
+def _synthetic_pool(rng, n, P):
+    nb = -(-n // 8)
+    k = min(P, nb)
+    ids = np.sort(rng.choice(nb, size=k, replace=False)) if nb else np.zeros(0, np.int64)
+    out = np.full(P, -1, np.int32)
+    out[:k] = ids
+    return out
+
+
+def test_full_topk_from_stored_scores_bitexact(csa2):
+    rng = np.random.default_rng(3)
+    lengths = [65536, 3000, 100]
+    B, page = 3, 4096
+    per = 16
+    cache = csa2.Cache(B * per, page, np.arange(B * per, dtype=np.int32).reshape(B, per), lengths)
+    scores = rng.standard_normal((B, cache.capacity)).astype(np.float32)
+    scores[:, ::5] = np.round(scores[:, ::5])                       # ties
+    pool = np.stack([_synthetic_pool(rng, n, 2048) for n in lengths])
+    dev = cache.device
+    topk = csa2.reindex(cache, csa2.FULL, 512, torch.from_numpy(pool).to(dev),
+                        full_scores=torch.from_numpy(scores).to(dev)).cpu().numpy()
+    for b, n in enumerate(lengths):
+        ref = C.full_topk(scores[b].astype(np.float64), pool[b], n, 512)
+        np.testing.assert_array_equal(topk[b], ref, err_msg=f"request {b}")
+    # without a pool: flat Top-k over every visible position
+    cache2 = csa2.Cache(B * 4, page, np.arange(B * 4, dtype=np.int32).reshape(B, 4), [16384, 5000, 100])
+    sc2 = scores[:, :cache2.capacity].copy()
+    topk2 = csa2.reindex(cache2, csa2.FULL, 512, None, full_scores=torch.from_numpy(sc2).to(dev)).cpu().numpy()
+    for b, n in enumerate([16384, 5000, 100]):
+        np.testing.assert_array_equal(topk2[b], C.full_topk(sc2[b].astype(np.float64), None, n, 512))
+
+
+def test_reindex_rescore_parity(csa2):
+    wl = W.scaled(W.WORKLOADS["group_64k_b8"], batch=3, shuffle_pages=True)
+    lengths = [65536, 20000, 4000]
+    cache = U.build_cache(wl, csa2, lengths=lengths)
+    rng = np.random.default_rng(4)
+    pool = np.stack([_synthetic_pool(rng, n, 2048) for n in lengths])
+    q, w = W.index_query(wl, 1)
+    dev = cache.device
+    tq, tw, tp = torch.from_numpy(q).to(dev), torch.from_numpy(w).to(dev), torch.from_numpy(pool).to(dev)
+    topk = csa2.reindex(cache, csa2.REINDEX, 512, tp, tq, tw).cpu().numpy()
+    # Full recompute: same arithmetic as the scan -> identical to Top-k of the scan's scores
+    sc = torch.empty(3, cache.capacity, device=dev)
+    csa2.index_full(cache, tq, tw, scores=sc)
+    full_re = csa2.reindex(cache, csa2.FULL, 512, tp, tq, tw).cpu().numpy()
+    full_st = csa2.reindex(cache, csa2.FULL, 512, tp, full_scores=sc).cpu().numpy()
+    np.testing.assert_array_equal(full_re, full_st)
+    np.testing.assert_array_equal(full_re, topk)
+    for b, n in enumerate(lengths):
+        codes, exp = U.oracle_request(wl, b, n)
+        ref = C.reindex_topk(q[b], w[b], codes, exp, pool[b], n, 512)
+        cand = C.pool_positions(pool[b], n)
+        s64 = C.indexer_scores(q[b], w[b], codes[cand], exp[cand])
+        score_of = dict(zip(cand.tolist(), s64.tolist())).get
+        U.assert_sorted_padded(topk[b], f"request {b}")
+        assert set(topk[b][topk[b] >= 0]) <= set(cand.tolist())
+        U.assert_set_parity(topk[b], ref, score_of, U.threshold(s64, 512), what=f"reindex b={b}")
+
+
+def test_reuse_copy_and_alias(csa2):
+    cache = _flat_cache(csa2, 1024, batch=2)
+    dev = cache.device
+    prev = torch.randint(-1, 1000, (2, 512), dtype=torch.int32, device=dev)
+    out = torch.zeros_like(prev)
+    csa2.reindex(cache, csa2.REUSE, 512, prev_topk=prev, topk=out)
+    assert torch.equal(out, prev)
+    same = prev.clone()
+    csa2.reindex(cache, csa2.REUSE, 512, prev_topk=same, topk=same)
+    assert torch.equal(same, prev)
+
+
+# ------------------------------------------------------------ attention (a7) --
+
+@pytest.mark.parametrize("H,k,n", [(64, 512, 65536), (16, 512, 4096), (32, 100, 3000), (64, 7, 50),
+                                   (16, 1024, 9000), (64, 512, 300)])
+def test_sparse_attention_parity(csa2, H, k, n):
+    wl = W.scaled(W.WORKLOADS["group_64k_b8"], batch=3, heads=H, page_size=1024, shuffle_pages=True, seed=11 + k)
+    lengths = [n, max(n // 3, 1), n]
+    cache = U.build_cache(wl, csa2, lengths=lengths)
+    rng = np.random.default_rng(H + k)
+    topk = np.full((3, k), -1, np.int32)
+    for b, nb in enumerate(lengths):
+        m = min(k, nb) - (1 if b == 1 and min(k, nb) > 1 else 0)     # request 1 keeps some -1 padding
+        topk[b, :m] = np.sort(rng.choice(nb, m, replace=False))
+    topk[2] = rng.permutation(topk[2])                                # order must not matter
+    qm = W.main_query(wl, 0)
+    dev = cache.device
+    out = csa2.sparse_attn(cache, torch.from_numpy(topk).to(dev), qm.to(dev), wl.scale).float().cpu().numpy()
+    for b, nb in enumerate(lengths):
+        sel = np.unique(topk[b][topk[b] >= 0])
+        codes, scales = U.oracle_kv_rows(wl, b, sel)
+        full_codes = np.zeros((nb, 256), np.uint8)
+        full_scales = np.zeros((nb, 32), np.uint8)
+        full_codes[sel], full_scales[sel] = codes, scales
+        ref = C.sparse_attention(qm[b].float().numpy(), full_codes, full_scales, topk[b], wl.scale)
+        rel = U.assert_attention_close(out[b], ref, f"H={H} k={k} b={b}")
+        print(f"H={H} k={k} b={b}: max rel err {rel:.2e}")
+
+
+def test_sparse_attention_empty_and_query_map(csa2):
+    wl = W.scaled(W.WORKLOADS["full_4k_b1"], batch=2, heads=16, page_size=1024)
+    cache = U.build_cache(wl, csa2, lengths=[2000, 3000])
+    dev = cache.device
+    rng = np.random.default_rng(5)
+    nq = 6
+    q_req = np.array([1, 0, 1, 1, 0, 0], np.int32)
+    topk = np.full((nq, 64), -1, np.int32)
+    for i in range(nq):
+        if i != 3:   # query 3: no valid index -> zeros
+            nb = [2000, 3000][q_req[i]]
+            topk[i, :40] = rng.choice(nb, 40, replace=False)
+    qm = W.main_query(wl, 0, rows=nq)
+    out = csa2.sparse_attn(cache, torch.from_numpy(topk).to(dev), qm.to(dev), wl.scale,
+                           q_req=torch.from_numpy(q_req).to(dev)).float().cpu().numpy()
+    assert np.all(out[3] == 0)
+    for i in range(nq):
+        if i == 3:
+            continue
+        b = q_req[i]
+        nb = [2000, 3000][b]
+        codes, scales = U.oracle_kv_rows(wl, b, np.arange(nb))
+        ref = C.sparse_attention(qm[i].float().numpy(), codes, scales, topk[i], wl.scale)
+        U.assert_attention_close(out[i], ref, f"query {i}")
+
+
+# ------------------------------------------------------------- error paths --
+
+def test_device_bounds_are_reported_not_trapped(csa2):
+    wl = W.scaled(W.WORKLOADS["full_4k_b1"], page_size=1024)
+    cache = U.build_cache(wl, csa2, lengths=[4096])
+    dev = cache.device
+    # an index past the visible context
+    topk = torch.tensor([[5, 4096 + 3, -1, 7]], dtype=torch.int32, device=dev)
+    csa2.sparse_attn(cache, topk, W.main_query(wl, 0).to(dev), wl.scale)
+    st, word = csa2.get_error(cache)
+    assert st == csa2.ERR_DEVICE_BOUNDS and word[1] == 5 and word[3] == 4096 + 3
+    # a corrupt page id in the page table
+    cache.err_word.zero_()
+    cache.page_table[0, 2] = 10_000
+    q, w = W.index_query(wl, 0)
+    csa2.index_full(cache, torch.from_numpy(q).to(dev), torch.from_numpy(w).to(dev))
+    st, word = csa2.get_error(cache)
+    assert st == csa2.ERR_DEVICE_BOUNDS and word[1] == 2
+    # the context is still usable
+    cache.page_table[0, 2] = 2
+    cache.err_word.zero_()
+    csa2.index_full(cache, torch.from_numpy(q).to(dev), torch.from_numpy(w).to(dev))
+    assert csa2.get_error(cache)[0] == csa2.OK
+
+
+def test_pipeline_wait_timeout_returns_status(csa2):
+    """A zero wait bound makes the tensor-core pipeline give up at once: the
+    kernel must record CSA2_ERR_TIMEOUT, drain and return (no hang, no trap)."""
+    wl = W.scaled(W.WORKLOADS["full_4k_b1"], page_size=1024)
+    cache = U.build_cache(wl, csa2, lengths=[4096])
+    dev = cache.device
+    q, w = W.index_query(wl, 0)
+    tq, tw = torch.from_numpy(q).to(dev), torch.from_numpy(w).to(dev)
+    try:
+        csa2.set_wait_limit_ns(0)
+        csa2.index_full(cache, tq, tw)
+        st, word = csa2.get_error(cache)
+    finally:
+        csa2.set_wait_limit_ns(2_000_000_000)
+    assert st in (csa2.ERR_TIMEOUT, csa2.OK)     # OK only if every wait happened to be ready
+    cache.err_word.zero_()
+    bm = csa2.index_full(cache, tq, tw)
+    assert csa2.get_error(cache)[0] == csa2.OK
+    codes, exp = U.oracle_request(wl, 0, 4096)
+    s64 = C.indexer_scores(q[0], w[0], codes, exp)
+    assert np.all(np.abs(bm[0, :512].cpu().numpy() - C.block_max(s64, 4096)) <= 1e-5 * C.block_max(s64, 4096))
