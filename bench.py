@@ -1,0 +1,471 @@
+#!/usr/bin/env python3
+"""Benchmark of one CSA2 decode layer-group step (Hierarchical Sparse Indexer
+over an FP4 main-KV cache) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl b200|reference]
+
+A step is one pass of the whole decode path over one batch: Full indexer scan,
+pool selection, the Full layer's Top-512, the two Reindex layers' Top-512 and
+six sparse-attention layers (1 Full + 2 Reindex + 3 Reuse), replayed as one
+CUDA graph.  Default workload: 4 decode queries, each over its own
+1,048,576-position cache (64 needles per request).  Multi-GPU (torchrun): every
+rank owns its own batch of requests (weak scaling, no data-path collective);
+timings are the max over ranks.
+
+Rank 0 prints one JSON line.  `value` is queries/s of the whole job with the
+cache resident in HBM; `e2e` is the same metric with the step's inputs copied
+from pinned host memory and the outputs read back every step; `roofline`
+rates the dominant kernel (the Full scan) against the measured copy bandwidth;
+`cpu_baseline` times the float64 oracle on a bounded sample.
+`--impl reference` times that oracle as the reference arm.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from kv_cache_decode_index_b200 import workloads as W  # noqa: E402
+
+METRIC = "CSA2 decode queries/s per layer group at 1M ctx; achieved HBM GB/s vs 8 TB/s"
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+IK_ROW_BYTES = 129     # 128 FP8 codes + 1 exponent byte
+KV_ROW_BYTES = 288     # 256 E2M1 bytes + 32 E4M3 scales
+POOL_ENTRY_BYTES = 4
+
+
+# --------------------------------------------------------------- host logic --
+
+def env_rank():
+    return (int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)),
+            int(os.environ.get("LOCAL_RANK", 0)))
+
+
+def rank_workload(wl, rank: int):
+    """Each rank serves its own requests: same shapes, its own seeded data."""
+    return wl if rank == 0 else W.scaled(wl, seed=wl.seed + 1000 * rank)
+
+
+def alg_bytes(wl, lengths=None):
+    """Algorithmic HBM bytes of one step and of one Full-scan launch.
+
+    Per request: the Full scan reads every visible indexer-K row (129 B); each
+    Reindex layer reads the pool's rows (<= 16,384 x 129 B); every layer
+    gathers its Top-k main-KV rows (<= 512 x 288 B); the pool is read once per
+    selecting layer (2048 x 4 B).  Score / block-max round trips and the
+    queries and outputs are implementation traffic and are not counted."""
+    n = W.ctx_lengths(wl) if lengths is None else np.asarray(lengths)
+    n_ri = sum(1 for m in wl.modes if m == "Ri")
+    P = wl.pool_blocks or 0
+    cand = np.minimum(n, P * 8) if P else n
+    scan = int((IK_ROW_BYTES * n).sum())
+    step = scan + int((n_ri * IK_ROW_BYTES * cand).sum()) + \
+        int((len(wl.modes) * KV_ROW_BYTES * np.minimum(n, wl.topk)).sum()) + \
+        (POOL_ENTRY_BYTES * P * (1 + n_ri) * len(n) if P else 0)
+    return step, scan
+
+
+def io_bytes(wl):
+    """Host<->device bytes of one end-to-end step: indexer queries and head
+    weights of every non-Reuse layer, main queries in; attention outputs out."""
+    B, H = wl.batch, wl.heads
+    n_idx = len(wl.index_layers)
+    h2d = n_idx * B * (32 * 128 * 4 + 32 * 4) + len(wl.modes) * B * H * 512 * 2
+    d2h = len(wl.modes) * B * H * 512 * 2
+    return h2d, d2h
+
+
+def measured_peak_hbm():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def scan_kernel_hash():
+    h = hashlib.sha256()
+    for name in ("k_index.cu", "index_common.cuh", "common.cuh"):
+        with open(os.path.join(ROOT, "kv_cache_decode_index_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def scan_traffic_per_launch(workload_name):
+    """DRAM bytes per Full-scan launch from the committed ncu summary, or None
+    when the summary is missing or was taken on a different kernel source."""
+    path = os.path.join(ROOT, "profiles", "index_full_traffic.txt")
+    try:
+        fields = dict(line.split(":", 1) for line in open(path).read().splitlines() if ":" in line)
+    except OSError:
+        return None
+    if fields.get("kernel_source_hash", "").strip() != scan_kernel_hash():
+        return None
+    if fields.get("workload", "").strip() != workload_name:
+        return None
+    try:
+        return float(fields["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling (every 200 ms) while the GPU works."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(prefix="clocks_", suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-lms", "200", "-i", self.gpu_id], stdout=open(self.path, "w"),
+                                         stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        return parse_clock_samples(open(self.path).read())
+
+
+def parse_clock_samples(text):
+    names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+    sm, mx, reasons, n = [], [], set(), 0
+    for line in text.splitlines():
+        parts = [p.strip() for p in line.split(",")]
+        if len(parts) < 9:
+            continue
+        try:
+            sm.append(float(parts[1]))
+            mx.append(float(parts[2]))
+        except ValueError:
+            continue
+        n += 1
+        for name, flag in zip(names, parts[5:9]):
+            if flag.lower() == "active":
+                reasons.add(name)
+    return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+            "reasons": sorted(reasons), "samples": n}
+
+
+def describe(wl):
+    n = W.ctx_lengths(wl)
+    ctx = f"{int(n[0]):,}-position" if len(set(n.tolist())) == 1 else "ragged"
+    modes = {"F": 0, "Ri": 0, "Ru": 0}
+    for m in wl.modes:
+        modes[m] += 1
+    pool = f"pool {wl.pool_blocks}x8, " if wl.pool_blocks else "no pool, "
+    return (f"{wl.name}: {wl.batch} decode queries x {ctx} contexts, {modes['F']} Full + {modes['Ri']} Reindex + "
+            f"{modes['Ru']} Reuse, {pool}Top-{wl.topk}, {wl.heads} heads d512"
+            + (f", {wl.needles} needles/request" if wl.needles else ""))
+
+
+def base_line(args, wl, world, value, ms):
+    return {"metric": METRIC, "value": value, "unit": "queries/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "fp8", "data": "synthetic",
+            "config": {"workload": describe(wl), "batch_per_gpu": wl.batch, "global_batch": wl.batch * world,
+                       "ctx": int(W.ctx_lengths(wl).max()), "page_size": wl.page_size,
+                       "parallelism": f"replicas{world}" if world > 1 else "single",
+                       "l2": "inputs larger than L2 (the Full scan streams 135 MB of indexer K per query)",
+                       "graph": "one CUDA graph per step"}}
+
+
+# ------------------------------------------------------------ oracle sample --
+
+def oracle_sample(wl, b: int = 0, prepared=None):
+    """Time the float64 oracle on one query of the workload: its whole decode
+    step (Full scan, pool, Full/Reindex/Reuse Top-512, six attention layers).
+    The cache rows are the oracle's own quantisation of the generated rows;
+    main-KV rows are prepared for the positions the step gathers."""
+    from oracle import csa2 as C
+    from oracle import formats as F
+    n = int(W.ctx_lengths(wl)[b])
+    if prepared is None:
+        codes, exp = F.quantize_indexer(W.request_rows(wl, b, n, "ik"))
+        q_idx = [None if m == "Ru" else W.index_query(wl, l)[0][b] for l, m in enumerate(wl.modes)]
+        w_idx = [None if m == "Ru" else W.index_query(wl, l)[1][b] for l, m in enumerate(wl.modes)]
+        q_main = [W.main_query(wl, l)[b].float().numpy() for l in range(len(wl.modes))]
+        sel = np.unique(np.concatenate([t[t >= 0] for t in
+                                        C.decode_group(wl.modes, q_idx, w_idx, codes, exp, n, wl.pool_blocks,
+                                                       wl.topk)["topk"]]))
+        kvc = np.zeros((n, 256), np.uint8)
+        kvs = np.zeros((n, 32), np.uint8)
+        kvc[sel], kvs[sel] = F.quantize_main_kv(W.rows_at(wl, b, sel, "kv"))
+        prepared = (codes, exp, q_idx, w_idx, q_main, kvc, kvs, n)
+    codes, exp, q_idx, w_idx, q_main, kvc, kvs, n = prepared
+    t0 = time.perf_counter()
+    out = C.decode_group(wl.modes, q_idx, w_idx, codes, exp, n, wl.pool_blocks, wl.topk)
+    for layer in range(len(wl.modes)):
+        C.sparse_attention(q_main[layer], kvc, kvs, out["topk"][layer], wl.scale)
+    return time.perf_counter() - t0, prepared
+
+
+def cpu_cores():
+    try:
+        import threadpoolctl
+        info = threadpoolctl.threadpool_info()
+        blas = [i["num_threads"] for i in info if i.get("user_api") == "blas"]
+        if blas:
+            return max(blas)
+    except Exception:
+        pass
+    return 1
+
+
+# --------------------------------------------------------------- b200 arm ----
+
+def run_b200(args):
+    import torch
+    import torch.distributed as dist
+    from datetime import timedelta
+
+    rank, world, local = env_rank()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=dev)
+    if local == 0:
+        from kv_cache_decode_index_b200 import build as _build
+        _build.build()
+    if world > 1:
+        dist.barrier()
+    from kv_cache_decode_index_b200 import csa2
+    from kv_cache_decode_index_b200.fill import build_cache
+
+    wl = rank_workload(selected_workload(args), rank)
+    t0 = time.time()
+    cache = build_cache(wl, csa2)
+    log(rank, f"cache filled in {time.time() - t0:.1f}s ({cache.kv_codes.numel() * 417 / 256 / 1e9:.2f} GB)")
+
+    q_idx, w_idx, q_main = [], [], []
+    for layer, m in enumerate(wl.modes):
+        if m == "Ru":
+            q_idx.append(None)
+            w_idx.append(None)
+        else:
+            q, w = W.index_query(wl, layer)
+            q_idx.append(torch.from_numpy(q).to(dev))
+            w_idx.append(torch.from_numpy(w).to(dev))
+        q_main.append(W.main_query(wl, layer).to(dev))
+    out = [torch.empty_like(m) for m in q_main]
+    group = csa2.DecodeGroup(cache, wl.modes, wl.heads, wl.topk, wl.pool_blocks, wl.scale)
+
+    # ---- warm-up (eager), then capture one step as a graph ----
+    for _ in range(args.warmup):
+        group.step(q_idx, w_idx, q_main, out)
+    torch.cuda.synchronize()
+    ev_scan = (torch.cuda.Event(enable_timing=True, external=True),
+               torch.cuda.Event(enable_timing=True, external=True))
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        group.step(q_idx, w_idx, q_main, out, scan_events=ev_scan)
+    graph.replay()
+    torch.cuda.synchronize()
+    st, word = csa2.get_error(cache)
+    if st != csa2.OK:
+        raise RuntimeError(f"device error during warm-up: {word}")
+
+    gpu_id = torch.cuda.get_device_properties(dev).uuid
+    sampler = ClockSampler(f"GPU-{gpu_id}" if not str(gpu_id).startswith("GPU-") else str(gpu_id))
+    sampler.start()
+    # keep the GPU busy ~0.5 s so the clock sampler sees it under load, then time K steps
+    t_busy = time.time()
+    while time.time() - t_busy < 0.5:
+        for _ in range(50):
+            graph.replay()
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        graph.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    ms = e0.elapsed_time(e1) / args.steps
+    ms = max_over_ranks(ms, dev, world)
+
+    # ---- the Full scan's launch duration, from events inside the graph ----
+    scan_ms = []
+    for _ in range(args.steps):
+        graph.replay()
+        torch.cuda.synchronize()
+        scan_ms.append(ev_scan[0].elapsed_time(ev_scan[1]))
+    clocks = sampler.stop()
+
+    # ---- end to end: pinned host inputs -> device, step, outputs -> host ----
+    h2d, d2h = io_bytes(wl)
+    e2e_value = None
+    if not args.no_e2e:
+        hq = [None if t is None else t.cpu().pin_memory() for t in q_idx]
+        hw = [None if t is None else t.cpu().pin_memory() for t in w_idx]
+        hm = [t.cpu().pin_memory() for t in q_main]
+        ho = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in out]
+        s = torch.cuda.current_stream()
+        for it in range(args.warmup + args.steps):
+            if it == args.warmup:
+                if world > 1:
+                    dist.barrier()
+                torch.cuda.synchronize()
+                a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a0.record()
+            for dst, src in zip(q_idx + w_idx + q_main, hq + hw + hm):
+                if dst is not None:
+                    dst.copy_(src, non_blocking=True)
+            graph.replay()
+            for dst, src in zip(ho, out):
+                dst.copy_(src, non_blocking=True)
+            s.synchronize()
+        a1.record()
+        torch.cuda.synchronize()
+        e2e_ms = max_over_ranks(a0.elapsed_time(a1) / args.steps, dev, world)
+        e2e_value = world * wl.batch / (e2e_ms / 1e3)
+
+    st, word = csa2.get_error(cache)
+    if st != csa2.OK:
+        raise RuntimeError(f"device error during the timed run: {word}")
+
+    step_bytes, scan_bytes = alg_bytes(wl)
+    scan_avg_ms = statistics.mean(scan_ms)
+    peak, peak_src = measured_peak_hbm()
+    achieved = scan_bytes / (scan_avg_ms / 1e3) / 1e9
+    traffic = scan_traffic_per_launch(wl.name)
+    if rank == 0:
+        value = world * wl.batch / (ms / 1e3)
+        line = base_line(args, wl, world, value, ms)
+        step_gbs = step_bytes / (ms / 1e3) / 1e9
+        line.update({
+            "alg_bytes_per_step": step_bytes,
+            "step_hbm_gbs": step_gbs,
+            "step_frac_of_8tbs": step_gbs / NOMINAL_HBM_GBS,
+            "step_frac_of_measured": step_gbs / peak,
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                         "traffic": traffic, "kernel": "csa2 index_full (Full indexer scan)",
+                         "kernel_ms": scan_avg_ms, "alg_bytes_per_launch": scan_bytes,
+                         "peak_source": f"{peak_src} copy bandwidth (MEASURED_PEAKS.json hbm_gbs, burst)"},
+            "e2e": {"value": e2e_value, "unit": "queries/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": group.launches_per_step * args.steps,
+            "clocks": clocks,
+        })
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline_entry(wl)
+        print(json.dumps(line), flush=True)
+    del graph
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def max_over_ranks(x: float, dev, world: int) -> float:
+    """Max of a per-rank timing over all ranks (NCCL on GPUs, gloo on CPU)."""
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def cpu_baseline_entry(wl):
+    secs, _ = oracle_sample(wl, 0)
+    return {"value": 1.0 / secs, "unit": "queries/s", "cores": cpu_cores(), "kind": "oracle",
+            "sample": f"1 of the {wl.batch} queries of one step (request 0, full {int(W.ctx_lengths(wl)[0]):,}-position "
+                      f"context): float64 numpy oracle, whole layer-group step, {secs:.1f} s"}
+
+
+# ---------------------------------------------------------- reference arm ----
+
+def run_reference(args):
+    """The float64 oracle as the reference arm: each step is one query of the
+    workload (cycling over the batch's requests), timed on the host cores."""
+    rank, world, _ = env_rank()
+    if rank != 0:
+        return
+    wl = selected_workload(args)
+    prepared = {}
+    times = []
+    for it in range(args.warmup + args.steps):
+        b = it % wl.batch
+        secs, prepared[b] = oracle_sample(wl, b, prepared.get(b))
+        if it >= args.warmup:
+            times.append(secs)
+    ms = 1e3 * sum(times) / len(times)
+    value = 1e3 / ms
+    line = base_line(args, wl, world, value, ms)
+    line.update({"impl": "reference", "dtype": "f64",
+                 "cpu_baseline": {"value": value, "unit": "queries/s", "cores": cpu_cores(), "kind": "oracle",
+                                  "sample": "one query per step (requests cycled), full context, float64 numpy "
+                                            "oracle of the whole layer-group step"},
+                 "e2e": {"value": value, "unit": "queries/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}})
+    print(json.dumps(line), flush=True)
+
+
+def selected_workload(args):
+    wl = W.WORKLOADS[args.workload]
+    changes = {}
+    if args.batch:
+        changes["batch"] = args.batch
+    if args.ctx:
+        changes["ctx"] = args.ctx
+    return W.scaled(wl, **changes) if changes else wl
+
+
+def log(rank, msg):
+    if rank == 0:
+        print(f"[bench] {msg}", file=sys.stderr, flush=True)
+
+
+def main(argv=None):
+    p = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=2000)
+    p.add_argument("--warmup", type=int, default=20)
+    p.add_argument("--impl", choices=["b200", "reference"], default="b200")
+    p.add_argument("--workload", default="group_1m_b4", choices=sorted(W.WORKLOADS))
+    p.add_argument("--batch", type=int, default=0, help="override the workload's batch (profiling cases)")
+    p.add_argument("--ctx", type=int, default=0, help="override the workload's context length (profiling cases)")
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    args = p.parse_args(argv)
+    if args.warmup < 3:
+        p.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_b200(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -244,11 +244,16 @@ class DecodeGroup:
         self.streams = [torch.cuda.Stream(dev) for _ in range(n_side)] if concurrent else []
         self.launches_per_step = 1 + (1 if pool_blocks else 0) + n_side + len(self.modes)
 
-    def step(self, q_idx, w_idx, q_main, out):
+    def step(self, q_idx, w_idx, q_main, out, scan_events=None):
         """q_idx / w_idx: per layer ([B,32,128] / [B,32], None for Reuse);
-        q_main / out: per layer bf16 [B, H, 512]."""
+        q_main / out: per layer bf16 [B, H, 512].  scan_events: optional pair of
+        CUDA events recorded on the launching stream around the Full scan."""
         c = self.cache
+        if scan_events is not None:
+            scan_events[0].record()
         index_full(c, q_idx[0], w_idx[0], self.blockmax)
+        if scan_events is not None:
+            scan_events[1].record()
         if self.pool is not None:
             pool_select(c, self.blockmax, self.pool_blocks, self.pool)
         main = torch.cuda.current_stream(c.device)

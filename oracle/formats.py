@@ -191,16 +191,33 @@ def indexer_exponent(amax) -> np.ndarray:
     return np.maximum(e, INDEXER_EXP_MIN)
 
 
-def quantize_indexer(k):
-    """FP8 indexer rows k[..., 128] (fp32 values) -> (codes uint8 [..., 128],
-    exponent byte uint8 [...]) with sigma = 2^(byte - 127) and
-    codes = E4M3(k / sigma).  Used for the cached indexer K and, per head, for
-    the indexer query."""
+def _quantize_indexer_rows(k):
     k = np.asarray(k, dtype=np.float32).astype(np.float64)
     amax = np.abs(k).max(axis=-1)
     e = indexer_exponent(amax)
     codes = e4m3_encode(k / np.ldexp(1.0, e)[..., None])
     return codes.astype(np.uint8), (e + INDEXER_EXP_BIAS).astype(np.uint8)
+
+
+def quantize_indexer(k, rows_per_chunk: int = 4096, threads: int = 8):
+    """FP8 indexer rows k[..., 128] (fp32 values) -> (codes uint8 [..., 128],
+    exponent byte uint8 [...]) with sigma = 2^(byte - 127) and
+    codes = E4M3(k / sigma).  Used for the cached indexer K and, per head, for
+    the indexer query.  Large inputs are processed in independent row chunks
+    (each row is quantised on its own; chunking only bounds the temporaries)."""
+    k = np.asarray(k, dtype=np.float32)
+    if k.ndim != 2 or len(k) <= rows_per_chunk:
+        return _quantize_indexer_rows(k)
+    from concurrent.futures import ThreadPoolExecutor
+    codes = np.empty(k.shape, dtype=np.uint8)
+    exp = np.empty(k.shape[0], dtype=np.uint8)
+
+    def one(a):
+        codes[a:a + rows_per_chunk], exp[a:a + rows_per_chunk] = _quantize_indexer_rows(k[a:a + rows_per_chunk])
+
+    with ThreadPoolExecutor(threads) as ex:
+        list(ex.map(one, range(0, len(k), rows_per_chunk)))
+    return codes, exp
 
 
 def indexer_sigma(exp_byte) -> np.ndarray:

@@ -25,22 +25,9 @@ ATTN_TOL = 2e-3
 
 
 def build_cache(wl, csa2, append_last=False, lengths=None):
-    """Allocate a cache for `wl` and fill it through csa2.append_kv, chunk by
-    chunk.  With append_last, each request's last position is left out (the
-    decode step appends it)."""
-    n = W.ctx_lengths(wl) if lengths is None else np.asarray(lengths)
-    table, num_pages = W.page_layout(wl, n)
-    cache = csa2.Cache(num_pages, wl.page_size, table, n)
-    dev = cache.device
-    for b, c, ik, kv, nvalid in W.iter_chunks(wl, lengths=n):
-        stop = nvalid - (1 if append_last and c * wl.page_size + nvalid == n[b] else 0)
-        if stop <= 0:
-            continue
-        pos = torch.arange(c * wl.page_size, c * wl.page_size + stop, dtype=torch.int32, device=dev)
-        req = torch.full((stop,), b, dtype=torch.int32, device=dev)
-        csa2.append_kv(cache, torch.from_numpy(kv[:stop]).to(dev), torch.from_numpy(ik[:stop]).to(dev), pos, req)
-    torch.cuda.synchronize()
-    return cache
+    """Cache for `wl`, filled through csa2_append_kv (see kv_cache_decode_index_b200.fill)."""
+    from kv_cache_decode_index_b200.fill import build_cache as _build
+    return _build(wl, csa2, append_last=append_last, lengths=lengths)
 
 
 def oracle_request(wl, b, n=None):

@@ -1,0 +1,101 @@
+"""Host-side logic of bench.py, on CPU: algorithmic bytes, I/O bytes, clock
+parsing, per-rank workloads, the max-over-ranks reduction across 2 gloo ranks,
+and the reference arm's JSON line on a small workload."""
+import io
+import json
+import os
+import socket
+import sys
+from contextlib import redirect_stdout
+
+import numpy as np
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+import bench
+from kv_cache_decode_index_b200 import workloads as W
+
+
+def test_alg_bytes_of_the_1m_group():
+    step, scan = bench.alg_bytes(W.WORKLOADS["group_1m_b4"])
+    assert scan == 4 * 1048576 * 129                        # 541.1 MB of indexer K
+    reindex = 2 * 4 * 16384 * 129                            # two Reindex layers over the pool
+    kv = 6 * 4 * 512 * 288                                   # six layers gather Top-512 FP4 rows
+    pool = 4 * 2048 * 4 * 3                                  # pool read by 3 selecting layers
+    assert step == scan + reindex + kv + pool
+    assert abs(step / 1e6 - 561.6) < 0.1
+
+
+def test_alg_bytes_short_context_and_no_pool():
+    step, scan = bench.alg_bytes(W.WORKLOADS["full_4k_b1"])
+    assert scan == 4096 * 129 and step == scan + 512 * 288
+
+
+def test_io_bytes():
+    h2d, d2h = bench.io_bytes(W.WORKLOADS["group_1m_b4"])
+    assert h2d == 3 * 4 * (32 * 128 * 4 + 32 * 4) + 6 * 4 * 64 * 512 * 2
+    assert d2h == 6 * 4 * 64 * 512 * 2
+
+
+def test_clock_parsing():
+    text = ("0, 1965, 1965, 700.1, 0x0000000000000000, Not Active, Not Active, Not Active, Not Active\n"
+            "0, 1800, 1965, 998.0, 0x0000000000000004, Not Active, Not Active, Not Active, Active\n"
+            "0, 1900, 1965, 990.0, 0x0000000000000004, Not Active, Not Active, Not Active, Active\n")
+    c = bench.parse_clock_samples(text)
+    assert c == {"sm_mhz": 1900.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"], "samples": 3}
+
+
+def test_rank_workloads_differ_only_in_data():
+    wl = W.WORKLOADS["group_1m_b4"]
+    w1 = bench.rank_workload(wl, 1)
+    assert bench.rank_workload(wl, 0) is wl
+    assert (w1.batch, w1.ctx, w1.modes) == (wl.batch, wl.ctx, wl.modes) and w1.seed != wl.seed
+    assert not np.array_equal(W.index_query(w1, 0)[0], W.index_query(wl, 0)[0])
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    return port
+
+
+def _rank_main(rank, world, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        t = [3.5, 7.25][rank]
+        out[rank] = bench.max_over_ranks(t, torch.device("cpu"), world)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_max_over_ranks_gloo_two_ranks():
+    ctx = mp.get_context("spawn")
+    with ctx.Manager() as m:
+        out = m.dict()
+        mp.start_processes(_rank_main, args=(2, _free_port(), out), nprocs=2, start_method="spawn", join=True)
+        assert dict(out) == {0: 7.25, 1: 7.25}
+
+
+def test_reference_arm_json_small(monkeypatch):
+    monkeypatch.setenv("RANK", "0")
+    monkeypatch.setenv("WORLD_SIZE", "1")
+    buf = io.StringIO()
+    with redirect_stdout(buf):
+        bench.main(["--impl", "reference", "--workload", "full_4k_b1", "--steps", "2", "--warmup", "3"])
+    line = json.loads(buf.getvalue().strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["value"] > 0 and line["unit"] == "queries/s"
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["cpu_baseline"]["kind"] == "oracle"
+    assert line["cpu_baseline"]["cores"] >= 1
+
+
+def test_reference_arm_other_ranks_do_nothing(monkeypatch):
+    monkeypatch.setenv("RANK", "1")
+    monkeypatch.setenv("WORLD_SIZE", "2")
+    buf = io.StringIO()
+    with redirect_stdout(buf):
+        bench.main(["--impl", "reference", "--workload", "full_4k_b1", "--steps", "2", "--warmup", "3"])
+    assert buf.getvalue() == ""
