@@ -69,12 +69,12 @@ __device__ __forceinline__ int block_exclusive_sum(int v, int* warp_tmp, int* su
 // threads of every CTA of the cluster (it contains cluster barriers).
 template <int THREADS, class Emit, class Pad>
 __device__ void cluster_topk(const uint32_t* keys, int n_local, int K, SelectSmem& S, Emit emit, Pad pad) {
+  constexpr int kWarps = THREADS / 32;
   cg::cluster_group cluster = cg::this_cluster();
   const int C = static_cast<int>(cluster.num_blocks());
   const int rank = static_cast<int>(cluster.block_rank());
-  const int tid = threadIdx.x;
-  const int per = (n_local + THREADS - 1) / THREADS;
-  const int lo = min(tid * per, n_local), hi = min(lo + per, n_local);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int rounds = (n_local + THREADS - 1) / THREADS;
 
   if (tid == 0) {
     S.prefix = 0;
@@ -89,9 +89,15 @@ __device__ void cluster_topk(const uint32_t* keys, int n_local, int K, SelectSme
     const int shift = 24 - 8 * pass;
     const int buf = pass & 1;
     const uint32_t prefix = S.prefix, mask = S.mask;
-    for (int i = lo; i < hi; ++i) {
-      const uint32_t k = keys[i];
-      if (k != 0u && (k & mask) == prefix) atomicAdd(&S.hist[buf][(k >> shift) & 255u], 1u);
+    // Keys of one request concentrate in a few bins in the first passes, so
+    // increments are aggregated per warp: one atomic per distinct bin.
+    for (int r = 0; r < rounds; ++r) {
+      const int i = r * THREADS + tid;
+      const uint32_t k = i < n_local ? keys[i] : 0u;
+      const bool counted = k != 0u && (k & mask) == prefix;
+      const uint32_t bin = counted ? ((k >> shift) & 255u) : 256u;
+      const uint32_t peers = __match_any_sync(0xffffffffu, bin);
+      if (counted && lane == __ffs(peers) - 1) atomicAdd(&S.hist[buf][bin], __popc(peers));
     }
     cluster.sync();   // every CTA's histogram of this pass is complete
     for (int d = tid; d < 256; d += THREADS) {
@@ -149,20 +155,27 @@ __device__ void cluster_topk(const uint32_t* keys, int n_local, int K, SelectSme
     if (S.done) break;
   }
 
-  // ---- final: above (prefix greater) and on-threshold (prefix equal) ----
+  // ---- final: keys above the threshold prefix, and keys on it (ties) ----
+  // Warp w owns the contiguous local range [wbeg, wend); lanes read it
+  // interleaved and rank their selections with ballots, so the output keeps
+  // the ascending candidate order.
   const uint32_t prefix = S.prefix, mask = S.mask;
   const int need = S.need;
-  int gt = 0, eq = 0;
-  for (int i = lo; i < hi; ++i) {
-    const uint32_t k = keys[i];
-    if (k == 0u) continue;
+  const int wper = (((n_local + kWarps - 1) / kWarps) + 31) & ~31;
+  const int wbeg = min(warp * wper, n_local), wend = min(wbeg + wper, n_local);
+  const uint32_t lt = (1u << lane) - 1u;
+  int gt_w = 0, eq_w = 0;
+  for (int base = wbeg; base < wend; base += 32) {
+    const int i = base + lane;
+    const uint32_t k = i < wend ? keys[i] : 0u;
     const uint32_t km = k & mask;
-    gt += km > prefix;
-    eq += km == prefix;
+    gt_w += __popc(__ballot_sync(0xffffffffu, k != 0u && km > prefix));
+    eq_w += __popc(__ballot_sync(0xffffffffu, k != 0u && km == prefix));
   }
+  // per-warp totals -> CTA totals and this warp's position among them
   int local_gt, local_eq;
-  const int eq_before = block_exclusive_sum<THREADS>(eq, S.warp_tmp, &local_eq);
-  (void)block_exclusive_sum<THREADS>(gt, S.warp_tmp, &local_gt);
+  const int eq_before_w = block_exclusive_sum<THREADS>(lane == 0 ? eq_w : 0, S.warp_tmp, &local_eq);
+  const int gt_before_w = block_exclusive_sum<THREADS>(lane == 0 ? gt_w : 0, S.warp_tmp, &local_gt);
   if (tid == 0) {
     S.gt_eq[0] = local_gt;
     S.gt_eq[1] = local_eq;
@@ -178,15 +191,25 @@ __device__ void cluster_topk(const uint32_t* keys, int n_local, int K, SelectSme
     sel_total += g + take;
     ties_before += e;
   }
-  const int take_t = max(0, min(take_local - eq_before, eq));
-  int dummy;
-  int off = out_base + block_exclusive_sum<THREADS>(gt + take_t, S.warp_tmp, &dummy);
-  int taken = 0;
-  for (int i = lo; i < hi; ++i) {
-    const uint32_t k = keys[i];
-    if (k == 0u) continue;
+  // ties taken by this warp, and the output rank of its first selection
+  const int eqb = __shfl_sync(0xffffffffu, eq_before_w, 0);
+  const int gtb = __shfl_sync(0xffffffffu, gt_before_w, 0);
+  const int take_w = max(0, min(take_local - eqb, eq_w));
+  const int ties_taken_before_w = max(0, min(take_local, eqb));
+  int sel_rank = out_base + gtb + ties_taken_before_w;
+  int ties_seen = 0;
+  for (int base = wbeg; base < wend; base += 32) {
+    const int i = base + lane;
+    const uint32_t k = i < wend ? keys[i] : 0u;
     const uint32_t km = k & mask;
-    if (km > prefix || (km == prefix && taken++ < take_t)) emit(i, off++);
+    const bool above = k != 0u && km > prefix;
+    const bool tie = k != 0u && km == prefix;
+    const uint32_t tie_bal = __ballot_sync(0xffffffffu, tie);
+    const bool take = above || (tie && ties_seen + __popc(tie_bal & lt) < take_w);
+    const uint32_t sel_bal = __ballot_sync(0xffffffffu, take);
+    if (take) emit(i, sel_rank + __popc(sel_bal & lt));
+    sel_rank += __popc(sel_bal);
+    ties_seen += __popc(tie_bal);
   }
   if (rank == 0)
     for (int r = sel_total + tid; r < K; r += THREADS) pad(r);

@@ -34,6 +34,7 @@ constexpr uint32_t kTmemCols = 64;   // 2 accumulators x 32 columns
 struct __align__(1024) IndexSmem {
   uint8_t tiles[kStages][kTileBytes];
   uint8_t q[2][kQBytes];
+  uint8_t exps[kStages][kTile];        // exponent bytes of the tile's 128 rows
   int prefix[kMaxBatchScan + 1];       // tiles before request b
   uint64_t full[kStages];
   uint64_t empty[kStages];
@@ -119,7 +120,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&S.full[s], 1);
-      mbar_init(&S.empty[s], 1);
+      mbar_init(&S.empty[s], 1 + 4);   // MMA commit + the 4 epilogue warps (exponents read)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&S.acc_full[a], 1);
@@ -154,24 +155,31 @@ __global__ void __launch_bounds__(kThreads, 1)
         TileIter it;
         it.init(S.prefix, B, t_begin);
         int issued = 0;
+        long long page_key = -1;   // page-table slot of the cached page id
+        int page = 0;
         for (int i = 0; i < n_tiles; ++i) {
           const int s = i % kStages;
           const uint32_t ph = (i / kStages) & 1;
+          const int p0 = it.j * kTile;
+          const long long key = static_cast<long long>(it.b) * cache.max_pages_per_req + p0 / cache.page_size;
+          if (key != page_key) {   // one page-table load per page (page_size / 128 tiles)
+            page_key = key;
+            page = cache.page_table[key];
+            if (page < 0 || page >= cache.num_pages) {
+              report_error(cache.err_word, CSA2_ERR_DEVICE_BOUNDS, kKIndexFull, it.b, p0);
+              page = 0;   // load a valid page; the results of this tile are flagged invalid
+            }
+          }
           if (!mbar_wait(&S.empty[s], ph ^ 1, wait_ns)) {
             report_error(cache.err_word, CSA2_ERR_TIMEOUT, kKIndexFull, it.b, i);
             S.abort_flag = 1;
             break;
           }
           if (S.abort_flag) break;
-          const int p0 = it.j * kTile;
-          int page = cache.page_table[static_cast<long long>(it.b) * cache.max_pages_per_req + p0 / cache.page_size];
-          if (page < 0 || page >= cache.num_pages) {
-            report_error(cache.err_word, CSA2_ERR_DEVICE_BOUNDS, kKIndexFull, it.b, p0);
-            page = 0;   // load a valid page; the results of this tile are flagged invalid
-          }
           const int row0 = page * cache.page_size + p0 % cache.page_size;
-          mbar_arrive_expect_tx(&S.full[s], kTileBytes);
+          mbar_arrive_expect_tx(&S.full[s], kTileBytes + kTile);
           tma_load_2d(S.tiles[s], &ik_map, &S.full[s], 0, row0, policy);
+          bulk_load_1d(S.exps[s], cache.ik_exp + row0, kTile, &S.full[s], policy);
           ++issued;
           it.advance();
         }
@@ -254,20 +262,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         const int a = i & 1;
         const uint32_t aph = (i >> 1) & 1;
+        const int s = i % kStages;
         const int p0 = it.j * kTile;
         const int p = p0 + toff;
         const bool valid = p < nb;
-        int page = cache.page_table[static_cast<long long>(cur_b) * cache.max_pages_per_req + p0 / cache.page_size];
-        page = (page < 0 || page >= cache.num_pages) ? 0 : page;
-        const uint32_t e_byte = valid ? cache.ik_exp[static_cast<long long>(page) * cache.page_size + p0 % cache.page_size + toff] : 127u;
 
-        if (!mbar_wait_warp(&S.acc_full[a], aph, wait_ns)) {
+        // accumulator ready; the stage's load (tile + exponents) completed before
+        // the MMA, and waiting on its barrier makes the exponent bytes visible here
+        if (!mbar_wait_warp(&S.acc_full[a], aph, wait_ns) ||
+            !mbar_wait_warp(&S.full[s], (i / kStages) & 1, wait_ns)) {
           if (lane == 0) {
             report_error(cache.err_word, CSA2_ERR_TIMEOUT, kKIndexFull, cur_b, p0);
             S.abort_flag = 1;
           }
           break;
         }
+        const uint32_t e_byte = valid ? S.exps[s][toff] : 127u;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&S.empty[s]);   // this warp is done with the stage
         tc_fence_after();
         uint32_t acc[32];
         tmem_ld_32x32b_x32(tmem + a * kAccCols + (static_cast<uint32_t>(quarter * 32) << 16), acc);

@@ -68,9 +68,9 @@ struct ReindexBarriers {
   volatile int abort_flag;
 };
 
-// Dynamic shared memory: [tiles][q tile][barriers][select][keys][blk_row][blk_id]
+// Dynamic shared memory: [tiles][q tile][barriers][select][keys][blk_exp][blk_row][blk_id]
 struct ReindexLayout {
-  uint32_t tiles, qtile, bars, sel, keys, blk_row, blk_id, total;
+  uint32_t tiles, qtile, bars, sel, keys, blk_exp, blk_row, blk_id, total;
   __host__ __device__ static ReindexLayout make(int max_blocks) {
     ReindexLayout L;
     L.tiles = 0;
@@ -78,7 +78,8 @@ struct ReindexLayout {
     L.bars = L.qtile + kQBytes;
     L.sel = (L.bars + sizeof(ReindexBarriers) + 15) & ~15u;
     L.keys = (L.sel + sizeof(SelectSmem) + 15) & ~15u;
-    L.blk_row = L.keys + max_blocks * kBlock * 4;
+    L.blk_exp = L.keys + max_blocks * kBlock * 4;
+    L.blk_row = L.blk_exp + max_blocks * 8;
     L.blk_id = L.blk_row + max_blocks * 4;
     L.total = L.blk_id + max_blocks * 4;
     return L;
@@ -98,6 +99,7 @@ __global__ void __launch_bounds__(kRThreads, 1)
   ReindexBarriers& R = *reinterpret_cast<ReindexBarriers*>(base + L.bars);
   SelectSmem& sel = *reinterpret_cast<SelectSmem*>(base + L.sel);
   uint32_t* keys = reinterpret_cast<uint32_t*>(base + L.keys);
+  uint64_t* blk_exp = reinterpret_cast<uint64_t*>(base + L.blk_exp);   // 8 exponent bytes per block
   int* blk_row = reinterpret_cast<int*>(base + L.blk_row);
   int* blk_id = reinterpret_cast<int*>(base + L.blk_id);
 
@@ -136,6 +138,8 @@ __global__ void __launch_bounds__(kRThreads, 1)
     }
     blk_row[i] = row;
     blk_id[i] = row >= 0 ? j : -1;
+    if (full_scores == nullptr)
+      blk_exp[i] = row >= 0 ? *reinterpret_cast<const uint64_t*>(cache.ik_exp + row) : 0x7F7F7F7F7F7F7F7Full;
   }
   const int n_tiles = (nloc + kBlocksPerTile - 1) / kBlocksPerTile;
   const bool recompute = full_scores == nullptr;
@@ -242,7 +246,7 @@ __global__ void __launch_bounds__(kRThreads, 1)
         const int o = m % kBlock;
         const int row = e < nloc ? blk_row[e] : -1;
         const bool valid = row >= 0 && blk_id[e] * kBlock + o < n;
-        const uint32_t e_byte = valid ? cache.ik_exp[static_cast<long long>(row) + o] : 127u;
+        const uint32_t e_byte = valid ? static_cast<uint32_t>((blk_exp[e] >> (8 * o)) & 0xFFu) : 127u;
         if (!mbar_wait_warp(&R.acc_full[a], aph, wait_ns)) {
           if (lane == 0) {
             report_error(cache.err_word, CSA2_ERR_TIMEOUT, kKReindex, b, t);
