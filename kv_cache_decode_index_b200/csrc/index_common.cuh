@@ -23,31 +23,26 @@ __device__ __forceinline__ uint32_t sw128_offset(uint32_t row, uint32_t c) {
 }
 
 // Quantise heads 8*ew .. 8*ew+7 of query q[32][128] (fp32, row-major) into
-// `qtile` (swizzled FP8 codes).  One warp per call; four warps cover a query.
-__device__ __forceinline__ void prepare_query_codes(const float* __restrict__ q, uint8_t* qtile, int ew, int lane) {
-#pragma unroll 1
+// `qtile` (swizzled FP8 codes) and store ws[h] = w[h] * sigma^q_h for those
+// heads into ws_sh.  One warp per call (four warps cover a query); the eight
+// heads' loads are issued together.
+__device__ __forceinline__ void prepare_query_part(const float* __restrict__ q, const float* __restrict__ w,
+                                                   uint8_t* qtile, float* ws_sh, int ew, int lane) {
+  float4 v[8];
+#pragma unroll
+  for (int hh = 0; hh < 8; ++hh) v[hh] = reinterpret_cast<const float4*>(q + (ew * 8 + hh) * kIndexDim)[lane];
+  const float wl = lane < 8 ? w[ew * 8 + lane] : 0.0f;
+#pragma unroll
   for (int hh = 0; hh < 8; ++hh) {
     const int h = ew * 8 + hh;
-    const float4 v = reinterpret_cast<const float4*>(q + h * kIndexDim)[lane];
-    float m = fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w)));
+    float m = fmaxf(fmaxf(fabsf(v[hh].x), fabsf(v[hh].y)), fmaxf(fabsf(v[hh].z), fabsf(v[hh].w)));
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    const float inv = exp2i(-indexer_exponent(m));
-    const uint32_t codes = e4m3x2(v.x * inv, v.y * inv) | (e4m3x2(v.z * inv, v.w * inv) << 16);
+    const int e = indexer_exponent(m);
+    const float inv = exp2i(-e);
+    const uint32_t codes = e4m3x2(v[hh].x * inv, v[hh].y * inv) | (e4m3x2(v[hh].z * inv, v[hh].w * inv) << 16);
     *reinterpret_cast<uint32_t*>(qtile + sw128_offset(h, 4u * lane)) = codes;
-  }
-}
-
-// ws[h] = w[h] * sigma^q_h for all 32 heads, in every lane of the calling warp.
-__device__ __forceinline__ void load_head_weights(const float* __restrict__ q, const float* __restrict__ w,
-                                                  float (&ws)[32], int lane) {
-#pragma unroll
-  for (int h = 0; h < 32; ++h) {
-    const float4 v = reinterpret_cast<const float4*>(q + h * kIndexDim)[lane];
-    float m = fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w)));
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    ws[h] = w[h] * exp2i(indexer_exponent(m));
+    if (lane == hh) ws_sh[h] = wl * exp2i(e);
   }
 }
 

@@ -121,9 +121,19 @@ __global__ void __launch_bounds__(kAThreads, 1)
   const int32_t* idx = topk + static_cast<long long>(qi) * K;
 
   // ---- query -> fp16 with a power-of-two scale per head ----
-  for (int h = warp; h < H; h += kAThreads / 32) {
-    const uint4* src = reinterpret_cast<const uint4*>(qg + (static_cast<long long>(qi) * H + h) * kKvDim) + lane * 2;
-    const uint4 v0 = src[0], v1 = src[1];
+  constexpr int kHpw = H / (kAThreads / 32);   // heads per warp; their loads are issued together
+  uint4 raw[kHpw][2];
+#pragma unroll
+  for (int hh = 0; hh < kHpw; ++hh) {
+    const uint4* src =
+        reinterpret_cast<const uint4*>(qg + (static_cast<long long>(qi) * H + warp * kHpw + hh) * kKvDim) + lane * 2;
+    raw[hh][0] = src[0];
+    raw[hh][1] = src[1];
+  }
+#pragma unroll
+  for (int hh = 0; hh < kHpw; ++hh) {
+    const int h = warp * kHpw + hh;
+    const uint4 v0 = raw[hh][0], v1 = raw[hh][1];
     const uint32_t wv[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
     float f[16];
     float amax = 0.0f;

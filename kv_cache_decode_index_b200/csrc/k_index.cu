@@ -5,15 +5,17 @@
 // layer scans the whole visible context].
 //
 // Design (sm_100a):
-//   * persistent grid, one CTA per SM; the concatenated tiles of all requests
+//   * persistent grid, two CTAs per SM; the concatenated tiles of all requests
 //     (128 positions each) are split into contiguous ranges, one per CTA;
 //   * warp 0 (one lane): TMA producer, 16 KB indexer-K tiles (128 rows x 128
-//     FP8 bytes, 128-byte swizzle) into a ring of kStages stages;
+//     FP8 bytes, 128-byte swizzle) plus the tile's 128 exponent bytes into a
+//     ring of kStages stages;
 //   * warp 1 (one lane): tcgen05.mma kind::f8f6f4, M = 128 positions, N = 32
 //     heads, K = 128 in 4 steps, fp32 accumulator in TMEM (two buffers);
 //   * warps 2..5: epilogue, one thread per position: tcgen05.ld of the 32
 //     head dot products, score, block max over 8 lanes, stores; they also
-//     quantise each request's query into the B-operand tile (two buffers).
+//     quantise each request's query into the B-operand tile (two buffers,
+//     handed over through the q_full / q_empty barriers).
 // Every mbarrier wait is bounded; a wait that runs out records
 // CSA2_ERR_TIMEOUT and the CTA leaves its loops, drains, frees TMEM, returns.
 #include <cub/block/block_scan.cuh>
@@ -25,7 +27,8 @@ namespace csa2 {
 
 namespace {
 
-constexpr int kStages = 8;
+constexpr int kStages = 6;
+constexpr int kCtasPerSm = 2;
 constexpr int kThreads = 192;
 constexpr int kMaxBatchScan = 1024;
 constexpr int kScanItems = (kMaxBatchScan + kThreads - 1) / kThreads;
@@ -35,12 +38,14 @@ struct __align__(1024) IndexSmem {
   uint8_t tiles[kStages][kTileBytes];
   uint8_t q[2][kQBytes];
   uint8_t exps[kStages][kTile];        // exponent bytes of the tile's 128 rows
+  float ws[2][kIndexHeads];            // w_h * sigma^q_h of the query in q[buf]
   int prefix[kMaxBatchScan + 1];       // tiles before request b
   uint64_t full[kStages];
   uint64_t empty[kStages];
   uint64_t acc_full[2];
   uint64_t acc_empty[2];
   uint64_t q_full[2];
+  uint64_t q_empty[2];
   uint64_t drain;
   uint32_t tmem_base;
   volatile int abort_flag;
@@ -82,7 +87,7 @@ __device__ __forceinline__ int next_request_with_tiles(const int* prefix, int ba
   return b;
 }
 
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, kCtasPerSm)
     index_full_kernel(const csa2_cache cache, const float* __restrict__ q, const float* __restrict__ w,
                       float* __restrict__ blockmax, float* __restrict__ scores,
                       const __grid_constant__ CUtensorMap ik_map, uint64_t wait_ns) {
@@ -125,7 +130,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int a = 0; a < 2; ++a) {
       mbar_init(&S.acc_full[a], 1);
       mbar_init(&S.acc_empty[a], 4);
-      mbar_init(&S.q_full[a], 4);   // one arrival per epilogue warp
+      mbar_init(&S.q_full[a], 4);    // one arrival per epilogue warp (its 8 heads written)
+      mbar_init(&S.q_empty[a], 4);   // one arrival per epilogue warp (head weights read)
     }
     mbar_init(&S.drain, 1);
     S.abort_flag = 0;
@@ -232,32 +238,51 @@ __global__ void __launch_bounds__(kThreads, 1)
       TileIter it;
       it.init(S.prefix, B, t_begin);
       int cur_b = it.b, seg = 0;
-      // queries of the first two segments
-      int prep_b = cur_b;
-      for (int k = 0; k < 2 && prep_b < B && S.prefix[prep_b] < t_end; ++k) {
-        prepare_query_codes(q + static_cast<long long>(prep_b) * kIndexHeads * kIndexDim, S.q[k], ew, lane);
+      // Query hand-over: segment x uses buffer x & 1.  A warp writes its part
+      // of segment x after every warp has read segment x - 2's head weights
+      // (q_empty), then arrives on q_full; the MMA of segment x - 2 is complete
+      // by then because this warp has seen an accumulator of a later segment.
+      int prep_b = cur_b, prep_x = 0;
+      auto timed_out = [&]() {
+        if (lane == 0) {
+          report_error(cache.err_word, CSA2_ERR_TIMEOUT, kKIndexFull, cur_b, -2);
+          S.abort_flag = 1;
+        }
+        return false;
+      };
+      auto prepare_next = [&]() -> bool {
+        const int buf = prep_x & 1;
+        if (!mbar_wait_warp(&S.q_empty[buf], ((prep_x >> 1) & 1) ^ 1, wait_ns)) return timed_out();
+        prepare_query_part(q + static_cast<long long>(prep_b) * kIndexHeads * kIndexDim, w + prep_b * kIndexHeads,
+                           S.q[buf], S.ws[buf], ew, lane);
         fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&S.q_full[k]);
+        if (lane == 0) mbar_arrive(&S.q_full[buf]);
         prep_b = next_request_with_tiles(S.prefix, B, prep_b);
-      }
+        ++prep_x;
+        return true;
+      };
+      auto read_weights = [&](int x, float (&ws)[32]) -> bool {
+        if (!mbar_wait_warp(&S.q_full[x & 1], (x >> 1) & 1, wait_ns)) return timed_out();
+#pragma unroll
+        for (int h = 0; h < 32; ++h) ws[h] = S.ws[x & 1][h];
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&S.q_empty[x & 1]);
+        return true;
+      };
+      bool ok = true;
+      for (int k = 0; ok && k < 2 && prep_b < B && S.prefix[prep_b] < t_end; ++k) ok = prepare_next();
       float ws[32];
-      load_head_weights(q + static_cast<long long>(cur_b) * kIndexHeads * kIndexDim, w + cur_b * kIndexHeads, ws, lane);
+      ok = ok && read_weights(0, ws);
       int nb = cache.ctx_len[cur_b];
 
-      for (int i = 0; i < n_tiles; ++i) {
+      for (int i = 0; ok && i < n_tiles; ++i) {
         if (it.b != cur_b) {
-          // segment `seg` is fully consumed: its query buffer takes segment seg + 2
-          if (prep_b < B && S.prefix[prep_b] < t_end) {
-            prepare_query_codes(q + static_cast<long long>(prep_b) * kIndexHeads * kIndexDim, S.q[seg & 1], ew, lane);
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&S.q_full[seg & 1]);
-            prep_b = next_request_with_tiles(S.prefix, B, prep_b);
-          }
+          // segment `seg` is fully consumed: its buffer takes segment seg + 2
+          if (prep_b < B && S.prefix[prep_b] < t_end && !prepare_next()) break;
           ++seg;
           cur_b = it.b;
-          load_head_weights(q + static_cast<long long>(cur_b) * kIndexHeads * kIndexDim, w + cur_b * kIndexHeads, ws, lane);
+          if (!read_weights(seg, ws)) break;
           nb = cache.ctx_len[cur_b];
         }
         const int a = i & 1;
@@ -316,15 +341,17 @@ size_t index_full_smem_bytes() { return sizeof(IndexSmem) + 1024; }
 cudaError_t launch_index_full(const csa2_cache& cache, const float* q, const float* w, float* blockmax,
                               float* scores, const CUtensorMap& ik_map, int num_sms, uint64_t wait_ns,
                               cudaStream_t stream) {
-  static bool configured = false;
+  static int per_sm = 0;   // resident CTAs per SM, so that the persistent grid is a single wave
   const size_t smem = index_full_smem_bytes();
-  if (!configured) {
+  if (per_sm == 0) {
     cudaError_t e = cudaFuncSetAttribute(index_full_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
+    if (e == cudaSuccess)
+      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, index_full_kernel, kThreads, smem);
     if (e != cudaSuccess) return e;
-    configured = true;
+    per_sm = per_sm < 1 ? 1 : (per_sm > kCtasPerSm ? kCtasPerSm : per_sm);
   }
-  index_full_kernel<<<num_sms, kThreads, smem, stream>>>(cache, q, w, blockmax, scores, ik_map, wait_ns);
+  index_full_kernel<<<num_sms * per_sm, kThreads, smem, stream>>>(cache, q, w, blockmax, scores, ik_map, wait_ns);
   return cudaGetLastError();
 }
 

@@ -43,7 +43,19 @@ __global__ void __launch_bounds__(kPoolThreads, 1)
   const int j0 = min(rank * per, nblk);
   const int nloc = min(per, nblk - j0);
   const float* src = blockmax + b * stride + j0;
-  for (int i = threadIdx.x; i < nloc; i += kPoolThreads) S.keys[i] = order_key(src[i]);
+  for (int base = 0; base < nloc; base += kPoolThreads * 8) {   // 8 independent loads per thread in flight
+    float v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int i = base + u * kPoolThreads + threadIdx.x;
+      v[u] = i < nloc ? src[i] : 0.0f;
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int i = base + u * kPoolThreads + threadIdx.x;
+      if (i < nloc) S.keys[i] = order_key(v[u]);
+    }
+  }
   __syncthreads();
   int32_t* out = pool + static_cast<long long>(b) * P;
   cluster_topk<kPoolThreads>(
@@ -66,6 +78,7 @@ struct ReindexBarriers {
   uint64_t drain;
   uint32_t tmem_base;
   volatile int abort_flag;
+  float ws[kIndexHeads];   // w_h * sigma^q_h of this layer's query
 };
 
 // Dynamic shared memory: [tiles][q tile][barriers][select][keys][blk_exp][blk_row][blk_id]
@@ -125,21 +138,52 @@ __global__ void __launch_bounds__(kRThreads, 1)
     nloc = min(per, nblk - e0);
   }
   if (nloc > max_blocks) nloc = max_blocks;   // host guarantees this never clips
-  for (int i = tid; i < nloc; i += kRThreads) {
-    const int j = pool != nullptr ? pool[static_cast<long long>(b) * P + e0 + i] : e0 + i;
-    int row = -1;
-    if (j >= 0 && static_cast<long long>(j) * kBlock < n) {
-      const int t = j * kBlock;
-      const int page = cache.page_table[static_cast<long long>(b) * cache.max_pages_per_req + t / cache.page_size];
-      if (page >= 0 && page < cache.num_pages) row = page * cache.page_size + t % cache.page_size;
-      else report_error(cache.err_word, CSA2_ERR_DEVICE_BOUNDS, kKReindex, b, t);
-    } else if (j >= 0 || j < -1) {
-      report_error(cache.err_word, CSA2_ERR_DEVICE_BOUNDS, kKReindex, b, j);
+  // block id -> page -> exponent bytes: each level's loads are issued together
+  constexpr int kU = 4;
+  for (int base = 0; base < nloc; base += kRThreads * kU) {
+    int j[kU], page[kU];
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      const int i = base + u * kRThreads + tid;
+      j[u] = i >= nloc ? -1 : (pool != nullptr ? pool[static_cast<long long>(b) * P + e0 + i] : e0 + i);
     }
-    blk_row[i] = row;
-    blk_id[i] = row >= 0 ? j : -1;
-    if (full_scores == nullptr)
-      blk_exp[i] = row >= 0 ? *reinterpret_cast<const uint64_t*>(cache.ik_exp + row) : 0x7F7F7F7F7F7F7F7Full;
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      const bool in = j[u] >= 0 && static_cast<long long>(j[u]) * kBlock < n;
+      page[u] = in ? cache.page_table[static_cast<long long>(b) * cache.max_pages_per_req +
+                                      j[u] * kBlock / cache.page_size]
+                   : -1;
+    }
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      const int i = base + u * kRThreads + tid;
+      if (i >= nloc) continue;
+      int row = -1;
+      if (j[u] >= 0 && static_cast<long long>(j[u]) * kBlock < n) {
+        const int t = j[u] * kBlock;
+        if (page[u] >= 0 && page[u] < cache.num_pages) row = page[u] * cache.page_size + t % cache.page_size;
+        else report_error(cache.err_word, CSA2_ERR_DEVICE_BOUNDS, kKReindex, b, t);
+      } else if (j[u] >= 0 || j[u] < -1) {
+        report_error(cache.err_word, CSA2_ERR_DEVICE_BOUNDS, kKReindex, b, j[u]);
+      }
+      blk_row[i] = row;
+      blk_id[i] = row >= 0 ? j[u] : -1;
+      page[u] = row;   // reuse as the row for the exponent load below
+    }
+    if (full_scores == nullptr) {
+      uint64_t ex[kU];
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        const int i = base + u * kRThreads + tid;
+        ex[u] = (i < nloc && page[u] >= 0) ? *reinterpret_cast<const uint64_t*>(cache.ik_exp + page[u])
+                                            : 0x7F7F7F7F7F7F7F7Full;
+      }
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        const int i = base + u * kRThreads + tid;
+        if (i < nloc) blk_exp[i] = ex[u];
+      }
+    }
   }
   const int n_tiles = (nloc + kBlocksPerTile - 1) / kBlocksPerTile;
   const bool recompute = full_scores == nullptr;
@@ -233,13 +277,19 @@ __global__ void __launch_bounds__(kRThreads, 1)
       // ---- epilogue: warps 2..5 ----
       const int ew = warp - 2, quarter = warp & 3, m = quarter * 32 + lane;
       const float* qb = q + static_cast<long long>(b) * kIndexHeads * kIndexDim;
-      prepare_query_codes(qb, qtile, ew, lane);
+      prepare_query_part(qb, w + b * kIndexHeads, qtile, R.ws, ew, lane);
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(&R.q_full);
       float ws[32];
-      load_head_weights(qb, w + b * kIndexHeads, ws, lane);
-      for (int t = 0; t < n_tiles; ++t) {
+      const bool q_ready = mbar_wait_warp(&R.q_full, 0, wait_ns);
+#pragma unroll
+      for (int h = 0; h < 32; ++h) ws[h] = R.ws[h];
+      if (!q_ready && lane == 0) {
+        report_error(cache.err_word, CSA2_ERR_TIMEOUT, kKReindex, b, -2);
+        R.abort_flag = 1;
+      }
+      for (int t = 0; q_ready && t < n_tiles; ++t) {
         const int a = t & 1;
         const uint32_t aph = (t >> 1) & 1;
         const int e = t * kBlocksPerTile + m / kBlock;
