@@ -282,11 +282,11 @@ def run_b200(args):
     for _ in range(args.warmup):
         group.step(q_idx, w_idx, q_main, out)
     torch.cuda.synchronize()
-    ev_scan = (torch.cuda.Event(enable_timing=True, external=True),
-               torch.cuda.Event(enable_timing=True, external=True))
+    timing = {name: (torch.cuda.Event(enable_timing=True, external=True),
+                     torch.cuda.Event(enable_timing=True, external=True)) for name in group.launch_names()}
     graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph):
-        group.step(q_idx, w_idx, q_main, out, scan_events=ev_scan)
+        group.step(q_idx, w_idx, q_main, out, timing=timing)
     graph.replay()
     torch.cuda.synchronize()
     st, word = csa2.get_error(cache)
@@ -316,12 +316,15 @@ def run_b200(args):
     ms = e0.elapsed_time(e1) / args.steps
     ms = max_over_ranks(ms, dev, world)
 
-    # ---- the Full scan's launch duration, from events inside the graph ----
-    scan_ms = []
+    # ---- launch durations, from events recorded inside the graph on each
+    # launch's own stream (one synchronised replay per sample) ----
+    per_launch = {name: [] for name in timing}
     for _ in range(args.steps):
         graph.replay()
         torch.cuda.synchronize()
-        scan_ms.append(ev_scan[0].elapsed_time(ev_scan[1]))
+        for name, (a, b) in timing.items():
+            per_launch[name].append(a.elapsed_time(b))
+    scan_ms = per_launch["scan"]
     clocks = sampler.stop()
 
     # ---- end to end: pinned host inputs -> device, step, outputs -> host ----
@@ -376,6 +379,7 @@ def run_b200(args):
                          "peak_source": f"{peak_src} copy bandwidth (MEASURED_PEAKS.json hbm_gbs, burst)"},
             "e2e": {"value": e2e_value, "unit": "queries/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "gpu_launches": group.launches_per_step * args.steps,
+            "launch_ms": {name: statistics.mean(v) for name, v in per_launch.items()},
             "clocks": clocks,
         })
         if world == 1 and not args.no_cpu_baseline:

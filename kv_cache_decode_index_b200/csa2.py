@@ -244,23 +244,29 @@ class DecodeGroup:
         self.streams = [torch.cuda.Stream(dev) for _ in range(n_side)] if concurrent else []
         self.launches_per_step = 1 + (1 if pool_blocks else 0) + n_side + len(self.modes)
 
-    def step(self, q_idx, w_idx, q_main, out, scan_events=None):
+    def step(self, q_idx, w_idx, q_main, out, timing=None):
         """q_idx / w_idx: per layer ([B,32,128] / [B,32], None for Reuse);
-        q_main / out: per layer bf16 [B, H, 512].  scan_events: optional pair of
-        CUDA events recorded on the launching stream around the Full scan."""
+        q_main / out: per layer bf16 [B, H, 512].  timing: optional dict
+        name -> (start, end) CUDA events, recorded on the launching stream
+        around the launch of that name ("scan", "pool", "topk<l>", "attn<l>")."""
         c = self.cache
-        if scan_events is not None:
-            scan_events[0].record()
-        index_full(c, q_idx[0], w_idx[0], self.blockmax)
-        if scan_events is not None:
-            scan_events[1].record()
+
+        def timed(name, fn):
+            ev = None if timing is None else timing.get(name)
+            if ev is not None:
+                ev[0].record()
+            r = fn()
+            if ev is not None:
+                ev[1].record()
+            return r
+
+        timed("scan", lambda: index_full(c, q_idx[0], w_idx[0], self.blockmax))
         if self.pool is not None:
-            pool_select(c, self.blockmax, self.pool_blocks, self.pool)
+            timed("pool", lambda: pool_select(c, self.blockmax, self.pool_blocks, self.pool))
         main = torch.cuda.current_stream(c.device)
         side = 0
         ev_ready = torch.cuda.Event()
         ev_ready.record(main)
-        joins = []
         src_stream = main
         for layer, m in enumerate(self.modes):
             if m != "Ru":
@@ -270,13 +276,17 @@ class DecodeGroup:
                     if s is not main:
                         s.wait_event(ev_ready)
                     mode = FULL if m == "F" else REINDEX
-                    reindex(c, mode, self.k, self.pool, q_idx[layer], w_idx[layer], topk=self.topk[layer])
-                    sparse_attn(c, self.topk[layer], q_main[layer], self.scale, out[layer])
+                    timed(f"topk{layer}", lambda: reindex(c, mode, self.k, self.pool, q_idx[layer], w_idx[layer],
+                                                          topk=self.topk[layer]))
+                    timed(f"attn{layer}", lambda: sparse_attn(c, self.topk[layer], q_main[layer], self.scale,
+                                                              out[layer]))
                 src_stream = s
             else:
                 with torch.cuda.stream(src_stream):
-                    sparse_attn(c, self.topk[layer], q_main[layer], self.scale, out[layer])
+                    timed(f"attn{layer}", lambda: sparse_attn(c, self.topk[layer], q_main[layer], self.scale,
+                                                              out[layer]))
         if self.concurrent:
+            joins = []
             for s in self.streams:
                 e = torch.cuda.Event()
                 e.record(s)
@@ -284,3 +294,11 @@ class DecodeGroup:
             for e in joins:
                 main.wait_event(e)
         return out
+
+    def launch_names(self):
+        names = ["scan"] + (["pool"] if self.pool is not None else [])
+        for layer, m in enumerate(self.modes):
+            if m != "Ru":
+                names.append(f"topk{layer}")
+            names.append(f"attn{layer}")
+        return names

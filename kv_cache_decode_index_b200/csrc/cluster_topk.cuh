@@ -101,8 +101,12 @@ __device__ void cluster_topk(const uint32_t* keys, int n_local, int K, SelectSme
     }
     cluster.sync();   // every CTA's histogram of this pass is complete
     for (int d = tid; d < 256; d += THREADS) {
+      uint32_t part[kMaxCluster];   // remote reads issued together
+#pragma unroll
+      for (int r = 0; r < kMaxCluster; ++r) part[r] = r < C ? cluster.map_shared_rank(&S.hist[buf][0], r)[d] : 0u;
       uint32_t g = 0;
-      for (int r = 0; r < C; ++r) g += cluster.map_shared_rank(&S.hist[buf][0], r)[d];
+#pragma unroll
+      for (int r = 0; r < kMaxCluster; ++r) g += part[r];
       S.ghist[d] = g;
       S.hist[buf ^ 1][d] = 0;   // next pass's buffer (last read remotely before this barrier)
     }
@@ -181,10 +185,17 @@ __device__ void cluster_topk(const uint32_t* keys, int n_local, int K, SelectSme
     S.gt_eq[1] = local_eq;
   }
   cluster.sync();   // counts visible cluster-wide
+  int rg[kMaxCluster], re[kMaxCluster];   // remote reads issued together
+#pragma unroll
+  for (int r = 0; r < kMaxCluster; ++r) {
+    rg[r] = r < C ? cluster.map_shared_rank(&S.gt_eq[0], r)[0] : 0;
+    re[r] = r < C ? cluster.map_shared_rank(&S.gt_eq[0], r)[1] : 0;
+  }
   int out_base = 0, take_local = 0, sel_total = 0, ties_before = 0;
-  for (int r = 0; r < C; ++r) {
-    const int* ge = cluster.map_shared_rank(&S.gt_eq[0], r);
-    const int g = ge[0], e = ge[1];
+#pragma unroll
+  for (int r = 0; r < kMaxCluster; ++r) {
+    if (r >= C) break;
+    const int g = rg[r], e = re[r];
     const int take = max(0, min(need - ties_before, e));
     if (r < rank) out_base += g + take;
     if (r == rank) take_local = take;

@@ -346,6 +346,8 @@ cudaError_t launch_index_full(const csa2_cache& cache, const float* q, const flo
   if (per_sm == 0) {
     cudaError_t e = cudaFuncSetAttribute(index_full_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
+    if (e == cudaSuccess)   // all of the unified L1 / shared storage as shared memory: two CTAs fit
+      e = cudaFuncSetAttribute(index_full_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
     if (e == cudaSuccess)
       e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, index_full_kernel, kThreads, smem);
     if (e != cudaSuccess) return e;
