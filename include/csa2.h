@@ -172,7 +172,7 @@ CSA2_API csa2_status csa2_pool_select(const csa2_cache* cache, const float* bloc
  *   CSA2_REUSE   copy prev_topk into topk (nothing is done when they alias).
  * Candidates: the positions of the pool's blocks (pool int32 [batch]
  * [pool_blocks], ascending, -1 padded), or every visible position when pool is
- * NULL (then ceil(ctx_len/8) must not exceed 131072 blocks).
+ * NULL (then the request capacity must not exceed 65,536 positions).
  *   q float [batch][32][128], w float [batch][32]  (FULL without full_scores,
  *                                                   and REINDEX)
  *   full_scores float [batch][capacity] or NULL

@@ -5,13 +5,17 @@
 // (cluster rank, local index); that order is the ascending candidate-id order,
 // which decides ties (lower id first) and the output order (ascending).
 //
-// Radix select, 8 bits per pass from the top: every CTA builds the histogram
-// of its keys that match the prefix decided so far, the CTAs read each other's
-// histograms through distributed shared memory (one cluster barrier per pass,
-// two histogram buffers), and all of them derive the same next digit.  The
-// passes stop as soon as every key matching the prefix is needed.  Then each
-// CTA counts its keys above / on the threshold prefix, the counts are
-// exchanged once more, and every CTA writes its selected ids at their ranks.
+// First the cluster-wide count, minimum and maximum of the valid keys: their
+// common leading bits need no pass (scores of one request share their sign and
+// most exponent bits), and K >= count selects everything.  Then radix select,
+// 8 bits per pass from the first differing bit: every CTA builds the
+// histogram of its keys that match the prefix decided so far, the CTAs read
+// each other's histograms through distributed shared memory (one cluster
+// barrier per pass, two histogram buffers), and all of them derive the same
+// next digit.  The passes stop as soon as every key matching the prefix is
+// needed.  Then each CTA counts its keys above / on the threshold prefix, the
+// counts are exchanged once more, and every CTA writes its selected ids at
+// their ranks.
 #pragma once
 
 #include <cooperative_groups.h>
@@ -28,10 +32,13 @@ struct SelectSmem {
   uint32_t hist[2][256];
   uint32_t ghist[256];
   int gt_eq[2];              // this CTA's (above, on-threshold) counts, read remotely
+  uint32_t stat[3];          // this CTA's (count, min, max) of valid keys, read remotely
+  uint32_t wstat[32][3];
   int warp_tmp[32];
   uint32_t prefix, mask;
   int need;
   int done;
+  int hi;                    // top bit of the next digit
   int total;                 // valid candidates in the cluster
 };
 
@@ -76,28 +83,86 @@ __device__ void cluster_topk(const uint32_t* keys, int n_local, int K, SelectSme
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int rounds = (n_local + THREADS - 1) / THREADS;
 
-  if (tid == 0) {
-    S.prefix = 0;
-    S.mask = 0;
-    S.done = 0;
-  }
-  for (int i = tid; i < 256; i += THREADS) S.hist[0][i] = 0;
-  __syncthreads();
-
-#pragma unroll 1
-  for (int pass = 0; pass < 4; ++pass) {
-    const int shift = 24 - 8 * pass;
-    const int buf = pass & 1;
-    const uint32_t prefix = S.prefix, mask = S.mask;
-    // Keys of one request concentrate in a few bins in the first passes, so
-    // increments are aggregated per warp: one atomic per distinct bin.
+  // ---- count, min and max of the valid keys ----
+  {
+    uint32_t cnt = 0, kmin = 0xFFFFFFFFu, kmax = 0u;
     for (int r = 0; r < rounds; ++r) {
       const int i = r * THREADS + tid;
       const uint32_t k = i < n_local ? keys[i] : 0u;
-      const bool counted = k != 0u && (k & mask) == prefix;
-      const uint32_t bin = counted ? ((k >> shift) & 255u) : 256u;
-      const uint32_t peers = __match_any_sync(0xffffffffu, bin);
-      if (counted && lane == __ffs(peers) - 1) atomicAdd(&S.hist[buf][bin], __popc(peers));
+      if (k != 0u) {
+        ++cnt;
+        kmin = min(kmin, k);
+        kmax = max(kmax, k);
+      }
+    }
+    cnt = __reduce_add_sync(0xffffffffu, cnt);
+    kmin = __reduce_min_sync(0xffffffffu, kmin);
+    kmax = __reduce_max_sync(0xffffffffu, kmax);
+    if (lane == 0) {
+      S.wstat[warp][0] = cnt;
+      S.wstat[warp][1] = kmin;
+      S.wstat[warp][2] = kmax;
+    }
+    for (int i = tid; i < 256; i += THREADS) S.hist[0][i] = 0;
+    __syncthreads();
+    if (warp == 0) {
+      cnt = lane < kWarps ? S.wstat[lane][0] : 0u;
+      kmin = lane < kWarps ? S.wstat[lane][1] : 0xFFFFFFFFu;
+      kmax = lane < kWarps ? S.wstat[lane][2] : 0u;
+      cnt = __reduce_add_sync(0xffffffffu, cnt);
+      kmin = __reduce_min_sync(0xffffffffu, kmin);
+      kmax = __reduce_max_sync(0xffffffffu, kmax);
+      if (lane == 0) {
+        S.stat[0] = cnt;
+        S.stat[1] = kmin;
+        S.stat[2] = kmax;
+      }
+    }
+    cluster.sync();   // every CTA's statistics are complete
+    if (warp == 0) {
+      const uint32_t* st = lane < C ? cluster.map_shared_rank(&S.stat[0], lane) : nullptr;
+      cnt = st ? st[0] : 0u;
+      kmin = st ? st[1] : 0xFFFFFFFFu;
+      kmax = st ? st[2] : 0u;
+      cnt = __reduce_add_sync(0xffffffffu, cnt);
+      kmin = __reduce_min_sync(0xffffffffu, kmin);
+      kmax = __reduce_max_sync(0xffffffffu, kmax);
+      if (lane == 0) {
+        S.total = static_cast<int>(cnt);
+        if (cnt <= static_cast<uint32_t>(K)) {   // everything valid is selected
+          S.prefix = 0u;
+          S.mask = 0u;
+          S.need = static_cast<int>(cnt);
+          S.done = 1;
+        } else if (kmin == kmax) {                 // all valid keys tie: the first K by id
+          S.prefix = kmin;
+          S.mask = 0xFFFFFFFFu;
+          S.need = K;
+          S.done = 1;
+        } else {
+          const int top = 31 - __clz(kmin ^ kmax);   // highest bit where the keys differ
+          S.mask = top == 31 ? 0u : (0xFFFFFFFFu << (top + 1));
+          S.prefix = kmin & S.mask;
+          S.need = K;
+          S.hi = top;
+          S.done = 0;
+        }
+      }
+    }
+    __syncthreads();
+  }
+
+#pragma unroll 1
+  for (int pass = 0; !S.done; ++pass) {
+    const int hi = S.hi;
+    const int lo = hi >= 7 ? hi - 7 : 0;
+    const uint32_t dmask = (hi - lo == 31) ? 0xFFFFFFFFu : (((1u << (hi - lo + 1)) - 1u) << lo);
+    const int buf = pass & 1;
+    const uint32_t prefix = S.prefix, mask = S.mask;
+    for (int r = 0; r < rounds; ++r) {
+      const int i = r * THREADS + tid;
+      const uint32_t k = i < n_local ? keys[i] : 0u;
+      if (k != 0u && (k & mask) == prefix) atomicAdd(&S.hist[buf][(k & dmask) >> lo], 1u);
     }
     cluster.sync();   // every CTA's histogram of this pass is complete
     for (int d = tid; d < 256; d += THREADS) {
@@ -126,37 +191,25 @@ __device__ void cluster_topk(const uint32_t* keys, int n_local, int K, SelectSme
         const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
         if (tid >= o) incl += y;
       }
-      const uint32_t total = __shfl_sync(0xffffffffu, incl, 31);
-      if (pass == 0 && tid == 0) {
-        S.total = static_cast<int>(total);
-        if (total <= static_cast<uint32_t>(K)) {   // everything valid is selected
-          S.need = static_cast<int>(total);
-          S.done = 1;
-        } else {
-          S.need = K;
-        }
-      }
-      __syncwarp();
-      if (!S.done) {
-        const uint32_t need = static_cast<uint32_t>(S.need);
-        uint32_t above = incl - sum;   // keys in digits above this lane's range
-        if (above < need && need <= incl) {
+      const uint32_t need = static_cast<uint32_t>(S.need);
+      uint32_t above = incl - sum;   // keys in digits above this lane's range
+      if (above < need && need <= incl) {
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            if (above < need && need <= above + local[i]) {
-              const uint32_t d = 255u - 8u * tid - i;
-              S.prefix = prefix | (d << shift);
-              S.mask = mask | (255u << shift);
-              S.need = static_cast<int>(need - above);
-              if (local[i] == need - above) S.done = 1;   // all keys with this prefix are taken
-            }
-            above += local[i];
+        for (int i = 0; i < 8; ++i) {
+          if (above < need && need <= above + local[i]) {
+            const uint32_t d = 255u - 8u * tid - i;
+            S.prefix = prefix | (d << lo);
+            S.mask = mask | dmask;
+            S.need = static_cast<int>(need - above);
+            S.hi = lo - 1;
+            // all keys with this prefix are taken, or no bit is left to split them
+            if (local[i] == need - above || lo == 0) S.done = 1;
           }
+          above += local[i];
         }
       }
     }
     __syncthreads();
-    if (S.done) break;
   }
 
   // ---- final: keys above the threshold prefix, and keys on it (ties) ----

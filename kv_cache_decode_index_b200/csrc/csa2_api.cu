@@ -32,7 +32,7 @@ bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) %
 constexpr int kMaxBatch = 1024;
 constexpr int kMaxK = 4096;
 constexpr int kMaxPool = 4096;
-constexpr long long kMaxFlatPositions = 131072;       // Top-k without a pool
+constexpr long long kMaxFlatPositions = 65536;        // Top-k without a pool
 constexpr long long kMaxPoolSelectBlocks = 16LL * 16384;
 
 uint64_t g_wait_limit_ns = csa2::kWaitLimitNs;

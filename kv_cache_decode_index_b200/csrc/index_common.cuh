@@ -46,6 +46,44 @@ __device__ __forceinline__ void prepare_query_part(const float* __restrict__ q, 
   }
 }
 
+// Quantise heads 8*ew .. 8*ew+7 of query q[32][128] into `qtile` (swizzled
+// FP8 codes) only.  One warp per call; the eight heads' loads are issued
+// together.
+__device__ __forceinline__ void prepare_query_codes(const float* __restrict__ q, uint8_t* qtile, int ew, int lane) {
+  float4 v[8];
+#pragma unroll
+  for (int hh = 0; hh < 8; ++hh) v[hh] = reinterpret_cast<const float4*>(q + (ew * 8 + hh) * kIndexDim)[lane];
+#pragma unroll
+  for (int hh = 0; hh < 8; ++hh) {
+    float m = fmaxf(fmaxf(fabsf(v[hh].x), fabsf(v[hh].y)), fmaxf(fabsf(v[hh].z), fabsf(v[hh].w)));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    const float inv = exp2i(-indexer_exponent(m));
+    const uint32_t codes = e4m3x2(v[hh].x * inv, v[hh].y * inv) | (e4m3x2(v[hh].z * inv, v[hh].w * inv) << 16);
+    *reinterpret_cast<uint32_t*>(qtile + sw128_offset(ew * 8 + hh, 4u * lane)) = codes;
+  }
+}
+
+// ws[h] = w[h] * sigma^q_h for all 32 heads, in every lane of the calling
+// warp; eight heads' loads are in flight at a time.
+__device__ __forceinline__ void load_head_weights(const float* __restrict__ q, const float* __restrict__ w,
+                                                  float (&ws)[32], int lane) {
+#pragma unroll
+  for (int g = 0; g < 4; ++g) {
+    float4 v[8];
+#pragma unroll
+    for (int hh = 0; hh < 8; ++hh) v[hh] = reinterpret_cast<const float4*>(q + (g * 8 + hh) * kIndexDim)[lane];
+    const float wl = lane < 8 ? w[g * 8 + lane] : 0.0f;
+#pragma unroll
+    for (int hh = 0; hh < 8; ++hh) {
+      float m = fmaxf(fmaxf(fabsf(v[hh].x), fabsf(v[hh].y)), fmaxf(fabsf(v[hh].z), fabsf(v[hh].w)));
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+      ws[g * 8 + hh] = __shfl_sync(0xffffffffu, wl, hh) * exp2i(indexer_exponent(m));
+    }
+  }
+}
+
 // Score of one position from its 32 fp32 head dot products.
 __device__ __forceinline__ float score_from_acc(const uint32_t (&acc)[32], const float (&ws)[32], uint32_t e_byte) {
   float s = 0.0f;

@@ -12,7 +12,8 @@
 //   * S = Q K^T and O = P V on mma.sync m16n8k16 (fp16 in, fp32 accumulate),
 //     online softmax in fp32 (exp2 domain), P rounded to fp16;
 // then the 8 partial (O, max, sum) triples are merged through distributed
-// shared memory: CTA r writes output dims [64r, 64r+64) of every head.
+// shared memory: every CTA pushes its slice of dims [64r, 64r+64) to CTA r,
+// which merges them locally and writes those dims of every head.
 #include <cooperative_groups.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -42,11 +43,12 @@ struct AttnLayout {
   static constexpr uint32_t kv_off = q_off + H * kRowBytes;          // fp16 [64][512]
   static constexpr uint32_t sred_off = kv_off + kChunk * kRowBytes;  // fp32 [DG][H][72]
   static constexpr uint32_t qscale_off = sred_off + DG * H * kSredStride * 4;
-  static constexpr uint32_t ml_off = qscale_off + H * 4;             // fp32 m[H], l[H]
-  static constexpr uint32_t fac_off = ml_off + 2 * H * 4;            // fp32 [8][H]
+  static constexpr uint32_t ml_off = qscale_off + H * 4;             // fp32 [8 ranks][2][H]: pushed m, l
+  static constexpr uint32_t fac_off = ml_off + kACluster * 2 * H * 4; // fp32 [8][H]
   static constexpr uint32_t kvalid_off = fac_off + kACluster * H * 4;
   static constexpr uint32_t total = kvalid_off + kChunk * 4;
-  static_assert(H * kKvDim * 4 <= sred_off, "O staging must fit in the Q + KV region");
+  // pushed partial O: [8 source ranks][H][64 dims] fp32, over the Q + KV region
+  static_assert(kACluster * H * 64 * 4 <= sred_off, "received partials must fit in the Q + KV region");
 };
 
 __device__ __forceinline__ uint32_t swz(uint32_t row, uint32_t chunk) {   // 16-byte chunk of a 1 KB row
@@ -104,8 +106,7 @@ __global__ void __launch_bounds__(kAThreads, 1)
   const uint32_t sbase = smem_u32(smem);
   float* sred = reinterpret_cast<float*>(smem + L::sred_off);
   float* qscale = reinterpret_cast<float*>(smem + L::qscale_off);
-  float* m_sh = reinterpret_cast<float*>(smem + L::ml_off);
-  float* l_sh = m_sh + H;
+  float* ml_sh = reinterpret_cast<float*>(smem + L::ml_off);
   float* fac = reinterpret_cast<float*>(smem + L::fac_off);
   int* kvalid = reinterpret_cast<int*>(smem + L::kvalid_off);
 
@@ -187,10 +188,13 @@ __global__ void __launch_bounds__(kAThreads, 1)
       if (src_row >= 0) {
         const uint4* cp = reinterpret_cast<const uint4*>(cache.kv_codes + src_row * kKvCodeBytes) + part * 4;
         const uint2 sp = *reinterpret_cast<const uint2*>(cache.kv_scales + src_row * kKvScaleBytes + part * 8);
+        uint4 cv[4];   // every load of the row part in flight before any shared-memory store
+#pragma unroll
+        for (int j = 0; j < 4; ++j) cv[j] = cp[j];
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           uint4 hv[4];
-          dequant16(cp[j], j < 2 ? (sp.x >> (16 * j)) : (sp.y >> (16 * (j - 2))), hv);
+          dequant16(cv[j], j < 2 ? (sp.x >> (16 * j)) : (sp.y >> (16 * (j - 2))), hv);
           const int chunk0 = part * 16 + j * 4;   // 8 fp16 per chunk
 #pragma unroll
           for (int c = 0; c < 4; ++c) *reinterpret_cast<uint4*>(smem + L::kv_off + swz(row, chunk0 + c)) = hv[c];
@@ -309,31 +313,38 @@ __global__ void __launch_bounds__(kAThreads, 1)
     }
   }
 
-  // ---- stage partial O, m, l for the cluster merge ----
-  __syncthreads();   // Q/KV region is reused as O staging
-  float* obuf = reinterpret_cast<float*>(smem);   // fp32 [H][512]
+  // ---- push the partial O slices, maxima and sums to their owners ----
+  // Output dims [64r, 64r + 64) belong to CTA r; it receives every rank's
+  // slice of them in recv[src][h][64].  Remote stores are fire-and-forget.
+  cluster.sync();   // every CTA is done reading its Q / KV region, which receives the partials
+  float* recv = reinterpret_cast<float*>(smem);
 #pragma unroll
   for (int i = 0; i < L::DW / 8; ++i) {
     const int col = dg * L::DW + i * 8 + 2 * (lane & 3);
-    *reinterpret_cast<float2*>(obuf + (ht * 16 + r0) * kKvDim + col) = make_float2(o_acc[i][0], o_acc[i][1]);
-    *reinterpret_cast<float2*>(obuf + (ht * 16 + r0 + 8) * kKvDim + col) = make_float2(o_acc[i][2], o_acc[i][3]);
+    const int owner = col >> 6, c64 = col & 63;
+    float* dst = cluster.map_shared_rank(recv, owner) + (rank * H + ht * 16 + r0) * 64 + c64;
+    *reinterpret_cast<float2*>(dst) = make_float2(o_acc[i][0], o_acc[i][1]);
+    *reinterpret_cast<float2*>(dst + 8 * 64) = make_float2(o_acc[i][2], o_acc[i][3]);
   }
   if (dg == 0 && (lane & 3) == 0) {
-    m_sh[ht * 16 + r0] = m_run[0];
-    m_sh[ht * 16 + r0 + 8] = m_run[1];
-    l_sh[ht * 16 + r0] = l_run[0];
-    l_sh[ht * 16 + r0 + 8] = l_run[1];
+    for (int r = 0; r < kACluster; ++r) {
+      float* dst = cluster.map_shared_rank(ml_sh, r) + rank * 2 * H;
+      dst[ht * 16 + r0] = m_run[0];
+      dst[ht * 16 + r0 + 8] = m_run[1];
+      dst[H + ht * 16 + r0] = l_run[0];
+      dst[H + ht * 16 + r0 + 8] = l_run[1];
+    }
   }
-  cluster.sync();
+  cluster.sync();   // all partials delivered
 
-  // merge factors per (rank, head): exp2(m_r - M) / L
+  // merge factors per (source rank, head): exp2(m_r - M) / L
   for (int h = tid; h < H; h += kAThreads) {
     float mr[kACluster], lr[kACluster];
     float M = -INFINITY;
 #pragma unroll
     for (int r = 0; r < kACluster; ++r) {
-      mr[r] = cluster.map_shared_rank(m_sh, r)[h];
-      lr[r] = cluster.map_shared_rank(l_sh, r)[h];
+      mr[r] = ml_sh[r * 2 * H + h];
+      lr[r] = ml_sh[r * 2 * H + H + h];
       M = fmaxf(M, mr[r]);
     }
     float Lsum = 0.0f;
@@ -349,11 +360,11 @@ __global__ void __launch_bounds__(kAThreads, 1)
   __syncthreads();
   // this CTA writes dims [64*rank, 64*rank + 64) of every head, 4 dims per item
   for (int item = tid; item < H * 16; item += kAThreads) {
-    const int h = item >> 4, d = rank * 64 + (item & 15) * 4;
+    const int h = item >> 4, d4 = (item & 15) * 4;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
     for (int r = 0; r < kACluster; ++r) {
-      const float4 v = *reinterpret_cast<const float4*>(cluster.map_shared_rank(obuf, r) + h * kKvDim + d);
+      const float4 v = *reinterpret_cast<const float4*>(recv + (r * H + h) * 64 + d4);
       const float f = fac[r * H + h];
       acc.x += v.x * f; acc.y += v.y * f; acc.z += v.z * f; acc.w += v.w * f;
     }
@@ -361,9 +372,8 @@ __global__ void __launch_bounds__(kAThreads, 1)
     uint2 pk;
     pk.x = *reinterpret_cast<uint32_t*>(&lo);
     pk.y = *reinterpret_cast<uint32_t*>(&hi);
-    *reinterpret_cast<uint2*>(out + (static_cast<long long>(qi) * H + h) * kKvDim + d) = pk;
+    *reinterpret_cast<uint2*>(out + (static_cast<long long>(qi) * H + h) * kKvDim + rank * 64 + d4) = pk;
   }
-  cluster.sync();   // keep shared memory alive until every CTA has read it
 }
 
 template <int H>

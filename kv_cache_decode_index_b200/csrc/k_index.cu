@@ -4,18 +4,18 @@
 // [4sapi blog, section 四; alphalab analysis, section 2 CSA2: the first Full
 // layer scans the whole visible context].
 //
-// Design (sm_100a):
-//   * persistent grid, two CTAs per SM; the concatenated tiles of all requests
-//     (128 positions each) are split into contiguous ranges, one per CTA;
-//   * warp 0 (one lane): TMA producer, 16 KB indexer-K tiles (128 rows x 128
-//     FP8 bytes, 128-byte swizzle) plus the tile's 128 exponent bytes into a
-//     ring of kStages stages;
+// Design (sm_100a), one persistent CTA per SM; the concatenated tiles of all
+// requests (128 positions each) are split into contiguous ranges, one per CTA:
+//   * warp 0 (one lane): producer.  TMA loads 16 KB indexer-K tiles (128 rows x
+//     128 FP8 bytes, 128-byte swizzle) into a ring of kStages stages, and the
+//     tile's 128 exponent bytes by bulk copy into a separate ring of kExp slots;
 //   * warp 1 (one lane): tcgen05.mma kind::f8f6f4, M = 128 positions, N = 32
-//     heads, K = 128 in 4 steps, fp32 accumulator in TMEM (two buffers);
-//   * warps 2..5: epilogue, one thread per position: tcgen05.ld of the 32
-//     head dot products, score, block max over 8 lanes, stores; they also
-//     quantise each request's query into the B-operand tile (two buffers,
-//     handed over through the q_full / q_empty barriers).
+//     heads, K = 128 in 4 steps, into one of kAcc fp32 accumulators in TMEM;
+//     the tile stage is released by the MMA's completion;
+//   * warps 2..9: two epilogue warpgroups taking alternate tiles, one thread per
+//     position: tcgen05.ld of the 32 head dot products, score, block max over 8
+//     lanes, stores.  Group 0 also quantises each request's query into the
+//     B-operand tile (three buffers) for the MMA.
 // Every mbarrier wait is bounded; a wait that runs out records
 // CSA2_ERR_TIMEOUT and the CTA leaves its loops, drains, frees TMEM, returns.
 #include <cub/block/block_scan.cuh>
@@ -27,25 +27,28 @@ namespace csa2 {
 
 namespace {
 
-constexpr int kStages = 6;
-constexpr int kCtasPerSm = 2;
-constexpr int kThreads = 192;
+constexpr int kStages = 12;                // indexer-K tile ring (16 KB each)
+constexpr int kExp = 16;                   // exponent ring (128 B each)
+constexpr int kAcc = 4;                    // TMEM accumulators (32 columns each)
+constexpr int kEpiGroups = 2;
+constexpr int kQBufs = 3;                  // query-code buffers (segments in flight)
+constexpr int kThreads = 64 + kEpiGroups * 128;
 constexpr int kMaxBatchScan = 1024;
 constexpr int kScanItems = (kMaxBatchScan + kThreads - 1) / kThreads;
-constexpr uint32_t kTmemCols = 64;   // 2 accumulators x 32 columns
+constexpr uint32_t kTmemCols = kAcc * kAccCols;   // 128
 
 struct __align__(1024) IndexSmem {
   uint8_t tiles[kStages][kTileBytes];
-  uint8_t q[2][kQBytes];
-  uint8_t exps[kStages][kTile];        // exponent bytes of the tile's 128 rows
-  float ws[2][kIndexHeads];            // w_h * sigma^q_h of the query in q[buf]
+  uint8_t q[kQBufs][kQBytes];
+  uint8_t exps[kExp][kTile];           // exponent bytes of a tile's 128 rows
   int prefix[kMaxBatchScan + 1];       // tiles before request b
   uint64_t full[kStages];
   uint64_t empty[kStages];
-  uint64_t acc_full[2];
-  uint64_t acc_empty[2];
-  uint64_t q_full[2];
-  uint64_t q_empty[2];
+  uint64_t xfull[kExp];
+  uint64_t xempty[kExp];
+  uint64_t acc_full[kAcc];
+  uint64_t acc_empty[kAcc];
+  uint64_t q_full[kQBufs];
   uint64_t drain;
   uint32_t tmem_base;
   volatile int abort_flag;
@@ -87,7 +90,7 @@ __device__ __forceinline__ int next_request_with_tiles(const int* prefix, int ba
   return b;
 }
 
-__global__ void __launch_bounds__(kThreads, kCtasPerSm)
+__global__ void __launch_bounds__(kThreads, 1)
     index_full_kernel(const csa2_cache cache, const float* __restrict__ q, const float* __restrict__ w,
                       float* __restrict__ blockmax, float* __restrict__ scores,
                       const __grid_constant__ CUtensorMap ik_map, uint64_t wait_ns) {
@@ -125,14 +128,17 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&S.full[s], 1);
-      mbar_init(&S.empty[s], 1 + 4);   // MMA commit + the 4 epilogue warps (exponents read)
+      mbar_init(&S.empty[s], 1);     // the MMA's completion
     }
-    for (int a = 0; a < 2; ++a) {
+    for (int e = 0; e < kExp; ++e) {
+      mbar_init(&S.xfull[e], 1);
+      mbar_init(&S.xempty[e], 4);    // the 4 warps of the epilogue group of that tile
+    }
+    for (int a = 0; a < kAcc; ++a) {
       mbar_init(&S.acc_full[a], 1);
       mbar_init(&S.acc_empty[a], 4);
-      mbar_init(&S.q_full[a], 4);    // one arrival per epilogue warp (its 8 heads written)
-      mbar_init(&S.q_empty[a], 4);   // one arrival per epilogue warp (head weights read)
     }
+    for (int k = 0; k < kQBufs; ++k) mbar_init(&S.q_full[k], 4);   // the 4 warps of epilogue group 0
     mbar_init(&S.drain, 1);
     S.abort_flag = 0;
     fence_barrier_init();
@@ -155,7 +161,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 
   if (n_tiles > 0) {
     if (warp == 0) {
-      // ================= TMA producer =================
+      // ================= producer =================
       if (lane == 0) {
         const uint64_t policy = l2_policy_evict_first();
         TileIter it;
@@ -164,8 +170,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         long long page_key = -1;   // page-table slot of the cached page id
         int page = 0;
         for (int i = 0; i < n_tiles; ++i) {
-          const int s = i % kStages;
-          const uint32_t ph = (i / kStages) & 1;
+          const int s = i % kStages, e = i % kExp;
           const int p0 = it.j * kTile;
           const long long key = static_cast<long long>(it.b) * cache.max_pages_per_req + p0 / cache.page_size;
           if (key != page_key) {   // one page-table load per page (page_size / 128 tiles)
@@ -176,22 +181,26 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
               page = 0;   // load a valid page; the results of this tile are flagged invalid
             }
           }
-          if (!mbar_wait(&S.empty[s], ph ^ 1, wait_ns)) {
+          if (!mbar_wait(&S.empty[s], ((i / kStages) & 1) ^ 1, wait_ns) ||
+              !mbar_wait(&S.xempty[e], ((i / kExp) & 1) ^ 1, wait_ns)) {
             report_error(cache.err_word, CSA2_ERR_TIMEOUT, kKIndexFull, it.b, i);
             S.abort_flag = 1;
             break;
           }
           if (S.abort_flag) break;
           const int row0 = page * cache.page_size + p0 % cache.page_size;
-          mbar_arrive_expect_tx(&S.full[s], kTileBytes + kTile);
+          mbar_arrive_expect_tx(&S.full[s], kTileBytes);
           tma_load_2d(S.tiles[s], &ik_map, &S.full[s], 0, row0, policy);
-          bulk_load_1d(S.exps[s], cache.ik_exp + row0, kTile, &S.full[s], policy);
+          mbar_arrive_expect_tx(&S.xfull[e], kTile);
+          bulk_load_1d(S.exps[e], cache.ik_exp + row0, kTile, &S.xfull[e], policy);
           ++issued;
           it.advance();
         }
-        // loads still in flight (only after an abort): wait for the last one of each stage
+        // copies still in flight (only after an abort): wait for the last one of each slot
         for (int i = issued > kStages ? issued - kStages : 0; i < issued; ++i)
           (void)mbar_wait(&S.full[i % kStages], (i / kStages) & 1, kWaitLimitNs / 2);
+        for (int i = issued > kExp ? issued - kExp : 0; i < issued; ++i)
+          (void)mbar_wait(&S.xfull[i % kExp], (i / kExp) & 1, kWaitLimitNs / 2);
       }
     } else if (warp == 1) {
       // ================= MMA issuer =================
@@ -204,18 +213,18 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
           if (it.b != cur_b) {
             ++seg;
             cur_b = it.b;
-            if (!mbar_wait(&S.q_full[seg & 1], (seg >> 1) & 1, wait_ns)) { ok = false; break; }
+            if (!mbar_wait(&S.q_full[seg % kQBufs], (seg / kQBufs) & 1, wait_ns)) { ok = false; break; }
           }
-          const int s = i % kStages;
-          const uint32_t ph = (i / kStages) & 1;
-          const int a = i & 1;
-          const uint32_t aph = (i >> 1) & 1;
-          if (!mbar_wait(&S.acc_empty[a], aph ^ 1, wait_ns)) { ok = false; break; }
-          if (!mbar_wait(&S.full[s], ph, wait_ns)) { ok = false; break; }
+          const int s = i % kStages, a = i % kAcc;
+          if (!mbar_wait(&S.acc_empty[a], ((i / kAcc) & 1) ^ 1, wait_ns) ||
+              !mbar_wait(&S.full[s], (i / kStages) & 1, wait_ns)) {
+            ok = false;
+            break;
+          }
           if (S.abort_flag) break;
           tc_fence_after();
           const uint64_t adesc = sw128_kmajor_desc(smem_u32(S.tiles[s]));
-          const uint64_t bdesc = sw128_kmajor_desc(smem_u32(S.q[seg & 1]));
+          const uint64_t bdesc = sw128_kmajor_desc(smem_u32(S.q[seg % kQBufs]));
 #pragma unroll
           for (int k = 0; k < kIndexDim / 32; ++k)
             umma_f8f6f4(tmem + a * kAccCols, adesc + 2 * k, bdesc + 2 * k, kIdesc, k > 0 ? 1u : 0u);
@@ -231,80 +240,73 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         (void)mbar_wait(&S.drain, 0, kWaitLimitNs);
       }
     } else {
-      // ================= epilogue (warps 2..5) =================
-      const int ew = warp - 2;                 // 0..3: query-preparation share
+      // ================= epilogue groups (warps 2..5, 6..9) =================
+      const int group = (warp - 2) >> 2;
+      const int ew = (warp - 2) & 3;           // 0..3: this warp's share of the query codes
       const int quarter = warp & 3;            // TMEM lane quarter of this warp
       const int toff = quarter * 32 + lane;    // position inside the tile
-      TileIter it;
-      it.init(S.prefix, B, t_begin);
-      int cur_b = it.b, seg = 0;
-      // Query hand-over: segment x uses buffer x & 1.  A warp writes its part
-      // of segment x after every warp has read segment x - 2's head weights
-      // (q_empty), then arrives on q_full; the MMA of segment x - 2 is complete
-      // by then because this warp has seen an accumulator of a later segment.
-      int prep_b = cur_b, prep_x = 0;
-      auto timed_out = [&]() {
+      auto timed_out = [&](int where) {
         if (lane == 0) {
-          report_error(cache.err_word, CSA2_ERR_TIMEOUT, kKIndexFull, cur_b, -2);
+          report_error(cache.err_word, CSA2_ERR_TIMEOUT, kKIndexFull, -1, where);
           S.abort_flag = 1;
         }
-        return false;
       };
-      auto prepare_next = [&]() -> bool {
-        const int buf = prep_x & 1;
-        if (!mbar_wait_warp(&S.q_empty[buf], ((prep_x >> 1) & 1) ^ 1, wait_ns)) return timed_out();
-        prepare_query_part(q + static_cast<long long>(prep_b) * kIndexHeads * kIndexDim, w + prep_b * kIndexHeads,
-                           S.q[buf], S.ws[buf], ew, lane);
+      // Query codes (group 0 only): segment x goes to buffer x % 3.  Writing
+      // segment x needs the MMAs of segment x - 3 complete, which holds once
+      // group 0 has seen an accumulator of segment x - 2 or later.  Group 0
+      // keeps the codes two segments ahead of its current one: between two of
+      // its tiles at most two segments begin, so the MMA never waits for codes
+      // that group 0 would write only after an accumulator it cannot get.
+      int prep_b = 0, prep_x = 0;
+      auto prepare = [&]() {
+        prepare_query_codes(q + static_cast<long long>(prep_b) * kIndexHeads * kIndexDim, S.q[prep_x % kQBufs], ew,
+                            lane);
         fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&S.q_full[buf]);
+        if (lane == 0) mbar_arrive(&S.q_full[prep_x % kQBufs]);
         prep_b = next_request_with_tiles(S.prefix, B, prep_b);
         ++prep_x;
-        return true;
       };
-      auto read_weights = [&](int x, float (&ws)[32]) -> bool {
-        if (!mbar_wait_warp(&S.q_full[x & 1], (x >> 1) & 1, wait_ns)) return timed_out();
-#pragma unroll
-        for (int h = 0; h < 32; ++h) ws[h] = S.ws[x & 1][h];
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&S.q_empty[x & 1]);
-        return true;
-      };
-      bool ok = true;
-      for (int k = 0; ok && k < 2 && prep_b < B && S.prefix[prep_b] < t_end; ++k) ok = prepare_next();
+      TileIter it;
+      it.init(S.prefix, B, t_begin);
+      int seg = 0, cur_b = it.b;
+      if (group == 0) {
+        prep_b = cur_b;
+        for (int k = 0; k < kQBufs && prep_b < B && S.prefix[prep_b] < t_end; ++k) prepare();
+      }
       float ws[32];
-      ok = ok && read_weights(0, ws);
+      load_head_weights(q + static_cast<long long>(cur_b) * kIndexHeads * kIndexDim, w + cur_b * kIndexHeads, ws,
+                        lane);
       int nb = cache.ctx_len[cur_b];
+      if (group == 1) it.advance();
 
-      for (int i = 0; ok && i < n_tiles; ++i) {
+      for (int i = group; i < n_tiles; i += kEpiGroups) {
         if (it.b != cur_b) {
-          // segment `seg` is fully consumed: its buffer takes segment seg + 2
-          if (prep_b < B && S.prefix[prep_b] < t_end && !prepare_next()) break;
-          ++seg;
+          // count the segments passed; group 0 keeps the codes two segments ahead
+          for (int b = cur_b; b != it.b; b = next_request_with_tiles(S.prefix, B, b)) ++seg;
           cur_b = it.b;
-          if (!read_weights(seg, ws)) break;
+          if (group == 0)
+            while (prep_x <= seg + 2 && prep_b < B && S.prefix[prep_b] < t_end) prepare();
+          load_head_weights(q + static_cast<long long>(cur_b) * kIndexHeads * kIndexDim, w + cur_b * kIndexHeads,
+                            ws, lane);
           nb = cache.ctx_len[cur_b];
         }
-        const int a = i & 1;
-        const uint32_t aph = (i >> 1) & 1;
-        const int s = i % kStages;
+        const int a = i % kAcc, e = i % kExp;
         const int p0 = it.j * kTile;
         const int p = p0 + toff;
         const bool valid = p < nb;
 
-        // accumulator ready; the stage's load (tile + exponents) completed before
-        // the MMA, and waiting on its barrier makes the exponent bytes visible here
-        if (!mbar_wait_warp(&S.acc_full[a], aph, wait_ns) ||
-            !mbar_wait_warp(&S.full[s], (i / kStages) & 1, wait_ns)) {
-          if (lane == 0) {
-            report_error(cache.err_word, CSA2_ERR_TIMEOUT, kKIndexFull, cur_b, p0);
-            S.abort_flag = 1;
-          }
+        if (!mbar_wait_warp(&S.xfull[e], (i / kExp) & 1, wait_ns)) {
+          timed_out(p0);
           break;
         }
-        const uint32_t e_byte = valid ? S.exps[s][toff] : 127u;
+        const uint32_t e_byte = valid ? S.exps[e][toff] : 127u;
         __syncwarp();
-        if (lane == 0) mbar_arrive(&S.empty[s]);   // this warp is done with the stage
+        if (lane == 0) mbar_arrive(&S.xempty[e]);
+        if (!mbar_wait_warp(&S.acc_full[a], (i / kAcc) & 1, wait_ns)) {
+          timed_out(p0);
+          break;
+        }
         tc_fence_after();
         uint32_t acc[32];
         tmem_ld_32x32b_x32(tmem + a * kAccCols + (static_cast<uint32_t>(quarter * 32) << 16), acc);
@@ -321,6 +323,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         if ((lane & 7) == 0 && valid) blockmax[static_cast<long long>(cur_b) * (capacity / kBlock) + p / kBlock] = bm;
         if (scores != nullptr && valid) scores[static_cast<long long>(cur_b) * capacity + p] = sc;
         if (warp_flag(&S.abort_flag)) break;
+        it.advance();
         it.advance();
       }
     }
@@ -341,19 +344,15 @@ size_t index_full_smem_bytes() { return sizeof(IndexSmem) + 1024; }
 cudaError_t launch_index_full(const csa2_cache& cache, const float* q, const float* w, float* blockmax,
                               float* scores, const CUtensorMap& ik_map, int num_sms, uint64_t wait_ns,
                               cudaStream_t stream) {
-  static int per_sm = 0;   // resident CTAs per SM, so that the persistent grid is a single wave
+  static bool configured = false;
   const size_t smem = index_full_smem_bytes();
-  if (per_sm == 0) {
-    cudaError_t e = cudaFuncSetAttribute(index_full_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
-    if (e == cudaSuccess)   // all of the unified L1 / shared storage as shared memory: two CTAs fit
-      e = cudaFuncSetAttribute(index_full_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
-    if (e == cudaSuccess)
-      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, index_full_kernel, kThreads, smem);
+  if (!configured) {
+    const cudaError_t e = cudaFuncSetAttribute(index_full_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               static_cast<int>(smem));
     if (e != cudaSuccess) return e;
-    per_sm = per_sm < 1 ? 1 : (per_sm > kCtasPerSm ? kCtasPerSm : per_sm);
+    configured = true;
   }
-  index_full_kernel<<<num_sms * per_sm, kThreads, smem, stream>>>(cache, q, w, blockmax, scores, ik_map, wait_ns);
+  index_full_kernel<<<num_sms, kThreads, smem, stream>>>(cache, q, w, blockmax, scores, ik_map, wait_ns);
   return cudaGetLastError();
 }
 

@@ -63,22 +63,23 @@ __global__ void __launch_bounds__(kPoolThreads, 1)
 }
 
 // --------------------------------------------------------------- reindex ----
-constexpr int kRThreads = 192;
-constexpr int kRStages = 4;
+constexpr int kRThreads = 320;          // producer, MMA, two epilogue warpgroups
+constexpr int kRStages = 8;
+constexpr int kRAcc = 4;
 constexpr int kBlkBytes = kBlock * kIndexDim;       // 1 KB: one block of 8 indexer-K rows
 constexpr int kBlocksPerTile = kTile / kBlock;      // 16
-constexpr uint32_t kRTmemCols = 64;
+constexpr uint32_t kRTmemCols = kRAcc * kAccCols;
+constexpr int kMaxReindexBlocks = 1024;   // candidate blocks per CTA (8 CTAs: 65,536 positions without a pool)
 
 struct ReindexBarriers {
   uint64_t full[kRStages];
   uint64_t empty[kRStages];
-  uint64_t acc_full[2];
-  uint64_t acc_empty[2];
+  uint64_t acc_full[kRAcc];
+  uint64_t acc_empty[kRAcc];
   uint64_t q_full;
   uint64_t drain;
   uint32_t tmem_base;
   volatile int abort_flag;
-  float ws[kIndexHeads];   // w_h * sigma^q_h of this layer's query
 };
 
 // Dynamic shared memory: [tiles][q tile][barriers][select][keys][blk_exp][blk_row][blk_id]
@@ -192,7 +193,7 @@ __global__ void __launch_bounds__(kRThreads, 1)
       mbar_init(&R.full[s], 1);
       mbar_init(&R.empty[s], 1);
     }
-    for (int a = 0; a < 2; ++a) {
+    for (int a = 0; a < kRAcc; ++a) {
       mbar_init(&R.acc_full[a], 1);
       mbar_init(&R.acc_empty[a], 4);
     }
@@ -220,38 +221,38 @@ __global__ void __launch_bounds__(kRThreads, 1)
   } else if (n_tiles > 0) {
     const uint32_t tmem = R.tmem_base;
     if (warp == 0) {
-      if (lane == 0) {   // ---- TMA producer: 16 gathered blocks per tile ----
-        const uint64_t policy = l2_policy_evict_normal();
-        int issued = 0;
-        for (int t = 0; t < n_tiles; ++t) {
-          const int s = t % kRStages;
-          const uint32_t ph = (t / kRStages) & 1;
-          if (!mbar_wait(&R.empty[s], ph ^ 1, wait_ns) || R.abort_flag) {
+      // ---- producer: lane l < 16 gathers block l of each tile ----
+      const uint64_t policy = l2_policy_evict_normal();
+      int issued = 0;
+      for (int t = 0; t < n_tiles; ++t) {
+        const int s = t % kRStages;
+        const uint32_t ph = (t / kRStages) & 1;
+        if (!mbar_wait_warp(&R.empty[s], ph ^ 1, wait_ns) || warp_flag(&R.abort_flag)) {
+          if (lane == 0) {
             report_error(cache.err_word, CSA2_ERR_TIMEOUT, kKReindex, b, t);
             R.abort_flag = 1;
-            break;
           }
-          const int eb = t * kBlocksPerTile;
-          const int ee = min(eb + kBlocksPerTile, nloc);
-          uint32_t bytes = 0;
-          for (int e = eb; e < ee; ++e) bytes += blk_row[e] >= 0 ? kBlkBytes : 0;
-          mbar_arrive_expect_tx(&R.full[s], bytes);
-          for (int e = eb; e < ee; ++e)
-            if (blk_row[e] >= 0)
-              tma_load_2d(tiles + s * kTileBytes + (e - eb) * kBlkBytes, &blk_map, &R.full[s], 0, blk_row[e], policy);
-          ++issued;
+          break;
         }
+        const int e = t * kBlocksPerTile + lane;
+        const int row = (lane < kBlocksPerTile && e < nloc) ? blk_row[e] : -1;
+        const uint32_t bytes = __popc(__ballot_sync(0xffffffffu, row >= 0)) * kBlkBytes;
+        if (lane == 0) mbar_arrive_expect_tx(&R.full[s], bytes);   // before any of the tile's copies
+        __syncwarp();
+        if (row >= 0) tma_load_2d(tiles + s * kTileBytes + lane * kBlkBytes, &blk_map, &R.full[s], 0, row, policy);
+        ++issued;
+      }
+      if (lane == 0)
         for (int i = issued > kRStages ? issued - kRStages : 0; i < issued; ++i)
           (void)mbar_wait(&R.full[i % kRStages], (i / kRStages) & 1, kWaitLimitNs / 2);
-      }
     } else if (warp == 1) {
       if (lane == 0) {   // ---- MMA issuer ----
         bool ok = mbar_wait(&R.q_full, 0, wait_ns);
         for (int t = 0; ok && t < n_tiles; ++t) {
           const int s = t % kRStages;
           const uint32_t ph = (t / kRStages) & 1;
-          const int a = t & 1;
-          const uint32_t aph = (t >> 1) & 1;
+          const int a = t % kRAcc;
+          const uint32_t aph = (t / kRAcc) & 1;
           if (!mbar_wait(&R.acc_empty[a], aph ^ 1, wait_ns) || !mbar_wait(&R.full[s], ph, wait_ns)) {
             ok = false;
             break;
@@ -274,24 +275,20 @@ __global__ void __launch_bounds__(kRThreads, 1)
         (void)mbar_wait(&R.drain, 0, kWaitLimitNs);
       }
     } else {
-      // ---- epilogue: warps 2..5 ----
-      const int ew = warp - 2, quarter = warp & 3, m = quarter * 32 + lane;
+      // ---- epilogue: warpgroups 2..5 and 6..9 take alternate tiles ----
+      const int group = (warp - 2) >> 2, ew = (warp - 2) & 3, quarter = warp & 3, m = quarter * 32 + lane;
       const float* qb = q + static_cast<long long>(b) * kIndexHeads * kIndexDim;
-      prepare_query_part(qb, w + b * kIndexHeads, qtile, R.ws, ew, lane);
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&R.q_full);
-      float ws[32];
-      const bool q_ready = mbar_wait_warp(&R.q_full, 0, wait_ns);
-#pragma unroll
-      for (int h = 0; h < 32; ++h) ws[h] = R.ws[h];
-      if (!q_ready && lane == 0) {
-        report_error(cache.err_word, CSA2_ERR_TIMEOUT, kKReindex, b, -2);
-        R.abort_flag = 1;
+      if (group == 0) {
+        prepare_query_codes(qb, qtile, ew, lane);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&R.q_full);
       }
-      for (int t = 0; q_ready && t < n_tiles; ++t) {
-        const int a = t & 1;
-        const uint32_t aph = (t >> 1) & 1;
+      float ws[32];
+      load_head_weights(qb, w + b * kIndexHeads, ws, lane);
+      for (int t = group; t < n_tiles; t += 2) {
+        const int a = t % kRAcc;
+        const uint32_t aph = (t / kRAcc) & 1;
         const int e = t * kBlocksPerTile + m / kBlock;
         const int o = m % kBlock;
         const int row = e < nloc ? blk_row[e] : -1;
@@ -382,7 +379,7 @@ cudaError_t launch_reindex(const csa2_cache& cache, const int32_t* pool, int poo
                            const CUtensorMap& blk_map, int max_blocks, uint64_t wait_ns, cudaStream_t stream) {
   static bool done = false;
   constexpr int kCluster = 8;
-  const size_t smem_max = reindex_smem_bytes(2048);
+  const size_t smem_max = reindex_smem_bytes(kMaxReindexBlocks);
   cudaError_t e = configure(reindex_kernel, smem_max, done);
   if (e != cudaSuccess) return e;
   return launch_cluster(reindex_kernel, cache.batch * kCluster, kRThreads, reindex_smem_bytes(max_blocks), kCluster,
