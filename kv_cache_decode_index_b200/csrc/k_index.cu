@@ -4,18 +4,22 @@
 // [4sapi blog, section 四; alphalab analysis, section 2 CSA2: the first Full
 // layer scans the whole visible context].
 //
-// Design (sm_100a), one persistent CTA per SM; the concatenated tiles of all
-// requests (128 positions each) are split into contiguous ranges, one per CTA:
-//   * warp 0 (one lane): producer.  TMA loads 16 KB indexer-K tiles (128 rows x
-//     128 FP8 bytes, 128-byte swizzle) into a ring of kStages stages, and the
-//     tile's 128 exponent bytes by bulk copy into a separate ring of kExp slots;
+// Design (sm_100a), one persistent CTA per SM; the concatenated work units of
+// all requests (256 positions each) are split into contiguous ranges, one per
+// CTA:
+//   * warp 0 (one lane): producer.  Per unit, two TMA loads of 128-row
+//     indexer-K sub-tiles (128 FP8 bytes per row, 128-byte swizzle) into one
+//     32 KB stage of a kStages ring;
 //   * warp 1 (one lane): tcgen05.mma kind::f8f6f4, M = 128 positions, N = 32
-//     heads, K = 128 in 4 steps, into one of kAcc fp32 accumulators in TMEM;
-//     the tile stage is released by the MMA's completion;
-//   * warps 2..9: two epilogue warpgroups taking alternate tiles, one thread per
-//     position: tcgen05.ld of the 32 head dot products, score, block max over 8
-//     lanes, stores.  Group 0 also quantises each request's query into the
-//     B-operand tile (three buffers) for the MMA.
+//     heads, K = 128 in 4 steps, per sub-tile, into an accumulator pair (one of
+//     kAcc) in TMEM; the stage is released by the MMAs' completion;
+//   * warps 2..9: two epilogue warpgroups taking alternate units, one thread
+//     per position of each sub-tile: tcgen05.ld of the 32 head dot products,
+//     score, block max over 8 lanes, stores.  The exponent bytes are read
+//     straight from global memory one unit ahead.  Group 0 also quantises each
+//     request's query into the B-operand tile (three buffers) for the MMA.
+// Per 256 positions the handshake is one stage and one accumulator pair: the
+// scan streams at the HBM rate instead of the rate of barrier round trips.
 // Every mbarrier wait is bounded; a wait that runs out records
 // CSA2_ERR_TIMEOUT and the CTA leaves its loops, drains, frees TMEM, returns.
 #include <cub/block/block_scan.cuh>
@@ -27,25 +31,22 @@ namespace csa2 {
 
 namespace {
 
-constexpr int kStages = 12;                // indexer-K tile ring (16 KB each)
-constexpr int kExp = 16;                   // exponent ring (128 B each)
-constexpr int kAcc = 4;                    // TMEM accumulators (32 columns each)
+constexpr int kUnit = 2 * kTile;           // positions per work unit (two MMA sub-tiles)
+constexpr int kStages = 6;                 // unit ring (32 KB each)
+constexpr int kAcc = 4;                    // TMEM accumulator pairs (2 x 32 columns each)
 constexpr int kEpiGroups = 2;
 constexpr int kQBufs = 3;                  // query-code buffers (segments in flight)
 constexpr int kThreads = 64 + kEpiGroups * 128;
 constexpr int kMaxBatchScan = 1024;
 constexpr int kScanItems = (kMaxBatchScan + kThreads - 1) / kThreads;
-constexpr uint32_t kTmemCols = kAcc * kAccCols;   // 128
+constexpr uint32_t kTmemCols = kAcc * 2 * kAccCols;   // 256
 
 struct __align__(1024) IndexSmem {
-  uint8_t tiles[kStages][kTileBytes];
+  uint8_t tiles[kStages][2][kTileBytes];
   uint8_t q[kQBufs][kQBytes];
-  uint8_t exps[kExp][kTile];           // exponent bytes of a tile's 128 rows
-  int prefix[kMaxBatchScan + 1];       // tiles before request b
+  int prefix[kMaxBatchScan + 1];       // units before request b
   uint64_t full[kStages];
   uint64_t empty[kStages];
-  uint64_t xfull[kExp];
-  uint64_t xempty[kExp];
   uint64_t acc_full[kAcc];
   uint64_t acc_empty[kAcc];
   uint64_t q_full[kQBufs];
@@ -54,7 +55,7 @@ struct __align__(1024) IndexSmem {
   volatile int abort_flag;
 };
 
-// Walks this CTA's tiles in order: request b, tile j inside it.
+// Walks this CTA's units in order: request b, unit j inside it.
 struct TileIter {
   const int* prefix;
   int batch;
@@ -114,7 +115,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         n = cache.ctx_len[b];
         n = n < 0 ? 0 : (n > capacity ? static_cast<int>(capacity) : n);
       }
-      items[i] = (n + kTile - 1) / kTile;
+      items[i] = (n + kUnit - 1) / kUnit;
     }
     int total;
     Scan(scan_tmp).ExclusiveSum(items, items, total);
@@ -129,10 +130,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&S.full[s], 1);
       mbar_init(&S.empty[s], 1);     // the MMA's completion
-    }
-    for (int e = 0; e < kExp; ++e) {
-      mbar_init(&S.xfull[e], 1);
-      mbar_init(&S.xempty[e], 4);    // the 4 warps of the epilogue group of that tile
     }
     for (int a = 0; a < kAcc; ++a) {
       mbar_init(&S.acc_full[a], 1);
@@ -170,37 +167,41 @@ __global__ void __launch_bounds__(kThreads, 1)
         long long page_key = -1;   // page-table slot of the cached page id
         int page = 0;
         for (int i = 0; i < n_tiles; ++i) {
-          const int s = i % kStages, e = i % kExp;
-          const int p0 = it.j * kTile;
-          const long long key = static_cast<long long>(it.b) * cache.max_pages_per_req + p0 / cache.page_size;
-          if (key != page_key) {   // one page-table load per page (page_size / 128 tiles)
-            page_key = key;
-            page = cache.page_table[key];
-            if (page < 0 || page >= cache.num_pages) {
-              report_error(cache.err_word, CSA2_ERR_DEVICE_BOUNDS, kKIndexFull, it.b, p0);
-              page = 0;   // load a valid page; the results of this tile are flagged invalid
-            }
-          }
-          if (!mbar_wait(&S.empty[s], ((i / kStages) & 1) ^ 1, wait_ns) ||
-              !mbar_wait(&S.xempty[e], ((i / kExp) & 1) ^ 1, wait_ns)) {
+          const int s = i % kStages;
+          if (!mbar_wait(&S.empty[s], ((i / kStages) & 1) ^ 1, wait_ns)) {
             report_error(cache.err_word, CSA2_ERR_TIMEOUT, kKIndexFull, it.b, i);
             S.abort_flag = 1;
             break;
           }
           if (S.abort_flag) break;
-          const int row0 = page * cache.page_size + p0 % cache.page_size;
-          mbar_arrive_expect_tx(&S.full[s], kTileBytes);
-          tma_load_2d(S.tiles[s], &ik_map, &S.full[s], 0, row0, policy);
-          mbar_arrive_expect_tx(&S.xfull[e], kTile);
-          bulk_load_1d(S.exps[e], cache.ik_exp + row0, kTile, &S.xfull[e], policy);
+          // sub-tiles of the unit that lie inside the request's capacity (page-table range)
+          int rows[2];
+          uint32_t bytes = 0;
+          for (int h = 0; h < 2; ++h) {
+            const long long p0 = static_cast<long long>(it.j) * kUnit + h * kTile;
+            rows[h] = -1;
+            if (p0 >= capacity) continue;
+            const long long key = static_cast<long long>(it.b) * cache.max_pages_per_req + p0 / cache.page_size;
+            if (key != page_key) {   // one page-table load per page
+              page_key = key;
+              page = cache.page_table[key];
+              if (page < 0 || page >= cache.num_pages) {
+                report_error(cache.err_word, CSA2_ERR_DEVICE_BOUNDS, kKIndexFull, it.b, static_cast<int>(p0));
+                page = 0;   // load a valid page; the results of this sub-tile are flagged invalid
+              }
+            }
+            rows[h] = page * cache.page_size + static_cast<int>(p0 % cache.page_size);
+            bytes += kTileBytes;
+          }
+          mbar_arrive_expect_tx(&S.full[s], bytes);
+          for (int h = 0; h < 2; ++h)
+            if (rows[h] >= 0) tma_load_2d(S.tiles[s][h], &ik_map, &S.full[s], 0, rows[h], policy);
           ++issued;
           it.advance();
         }
-        // copies still in flight (only after an abort): wait for the last one of each slot
+        // copies still in flight (only after an abort): wait for the last one of each stage
         for (int i = issued > kStages ? issued - kStages : 0; i < issued; ++i)
           (void)mbar_wait(&S.full[i % kStages], (i / kStages) & 1, kWaitLimitNs / 2);
-        for (int i = issued > kExp ? issued - kExp : 0; i < issued; ++i)
-          (void)mbar_wait(&S.xfull[i % kExp], (i / kExp) & 1, kWaitLimitNs / 2);
       }
     } else if (warp == 1) {
       // ================= MMA issuer =================
@@ -223,11 +224,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           if (S.abort_flag) break;
           tc_fence_after();
-          const uint64_t adesc = sw128_kmajor_desc(smem_u32(S.tiles[s]));
           const uint64_t bdesc = sw128_kmajor_desc(smem_u32(S.q[seg % kQBufs]));
 #pragma unroll
-          for (int k = 0; k < kIndexDim / 32; ++k)
-            umma_f8f6f4(tmem + a * kAccCols, adesc + 2 * k, bdesc + 2 * k, kIdesc, k > 0 ? 1u : 0u);
+          for (int h = 0; h < 2; ++h) {
+            const uint64_t adesc = sw128_kmajor_desc(smem_u32(S.tiles[s][h]));
+#pragma unroll
+            for (int k = 0; k < kIndexDim / 32; ++k)
+              umma_f8f6f4(tmem + (2 * a + h) * kAccCols, adesc + 2 * k, bdesc + 2 * k, kIdesc, k > 0 ? 1u : 0u);
+          }
           umma_commit(&S.empty[s]);
           umma_commit(&S.acc_full[a]);
           it.advance();
@@ -280,6 +284,27 @@ __global__ void __launch_bounds__(kThreads, 1)
       int nb = cache.ctx_len[cur_b];
       if (group == 1) it.advance();
 
+      // Exponent bytes of this thread's two positions in unit `u` (request b,
+      // unit j), read from global memory; issued one unit ahead of their use.
+      long long ex_key = -1;
+      int ex_page = 0;
+      auto exp_bytes = [&](int b, int j, uint32_t (&e)[2]) {
+        for (int h = 0; h < 2; ++h) {
+          const long long p = static_cast<long long>(j) * kUnit + h * kTile + toff;
+          e[h] = 127u;
+          if (b >= B || p >= capacity) continue;
+          const long long key = static_cast<long long>(b) * cache.max_pages_per_req + p / cache.page_size;
+          if (key != ex_key) {
+            ex_key = key;
+            ex_page = cache.page_table[key];
+            ex_page = (ex_page < 0 || ex_page >= cache.num_pages) ? 0 : ex_page;
+          }
+          e[h] = cache.ik_exp[static_cast<long long>(ex_page) * cache.page_size + p % cache.page_size];
+        }
+      };
+      uint32_t ex_cur[2], ex_next[2];
+      exp_bytes(it.b, it.j, ex_cur);
+
       for (int i = group; i < n_tiles; i += kEpiGroups) {
         if (it.b != cur_b) {
           // count the segments passed; group 0 keeps the codes two segments ahead
@@ -291,40 +316,44 @@ __global__ void __launch_bounds__(kThreads, 1)
                             ws, lane);
           nb = cache.ctx_len[cur_b];
         }
-        const int a = i % kAcc, e = i % kExp;
-        const int p0 = it.j * kTile;
-        const int p = p0 + toff;
-        const bool valid = p < nb;
+        const int a = i % kAcc;
+        const int j = it.j;
+        // prefetch the exponents of this group's next unit
+        TileIter nx = it;
+        nx.advance();
+        nx.advance();
+        if (i + kEpiGroups < n_tiles) exp_bytes(nx.b, nx.j, ex_next);
 
-        if (!mbar_wait_warp(&S.xfull[e], (i / kExp) & 1, wait_ns)) {
-          timed_out(p0);
-          break;
-        }
-        const uint32_t e_byte = valid ? S.exps[e][toff] : 127u;
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&S.xempty[e]);
         if (!mbar_wait_warp(&S.acc_full[a], (i / kAcc) & 1, wait_ns)) {
-          timed_out(p0);
+          timed_out(j);
           break;
         }
         tc_fence_after();
-        uint32_t acc[32];
-        tmem_ld_32x32b_x32(tmem + a * kAccCols + (static_cast<uint32_t>(quarter * 32) << 16), acc);
+        uint32_t acc0[32], acc1[32];
+        tmem_ld_32x32b_x32(tmem + (2 * a) * kAccCols + (static_cast<uint32_t>(quarter * 32) << 16), acc0);
+        tmem_ld_32x32b_x32(tmem + (2 * a + 1) * kAccCols + (static_cast<uint32_t>(quarter * 32) << 16), acc1);
         tmem_ld_wait();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&S.acc_empty[a]);
 
-        const float sc = score_from_acc(acc, ws, e_byte);
-        float bm = valid ? sc : -INFINITY;
-        bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 1));
-        bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 2));
-        bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 4));
-        if ((lane & 7) == 0 && valid) blockmax[static_cast<long long>(cur_b) * (capacity / kBlock) + p / kBlock] = bm;
-        if (scores != nullptr && valid) scores[static_cast<long long>(cur_b) * capacity + p] = sc;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int p = j * kUnit + h * kTile + toff;
+          const bool valid = p < nb;
+          const float sc = score_from_acc(h == 0 ? acc0 : acc1, ws, ex_cur[h]);
+          float bm = valid ? sc : -INFINITY;
+          bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 1));
+          bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 2));
+          bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 4));
+          if ((lane & 7) == 0 && valid)
+            blockmax[static_cast<long long>(cur_b) * (capacity / kBlock) + p / kBlock] = bm;
+          if (scores != nullptr && valid) scores[static_cast<long long>(cur_b) * capacity + p] = sc;
+        }
+        ex_cur[0] = ex_next[0];
+        ex_cur[1] = ex_next[1];
         if (warp_flag(&S.abort_flag)) break;
-        it.advance();
-        it.advance();
+        it = nx;
       }
     }
   }
