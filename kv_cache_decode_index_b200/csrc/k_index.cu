@@ -101,6 +101,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = tid >> 5, lane = tid & 31;
   const int B = cache.batch;
   const long long capacity = static_cast<long long>(cache.max_pages_per_req) * cache.page_size;
+  const uint32_t page_size = static_cast<uint32_t>(cache.page_size);
 
   // ---- tiles per request, prefix sums ----
   {
@@ -174,23 +175,25 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           if (S.abort_flag) break;
-          // sub-tiles of the unit that lie inside the request's capacity (page-table range)
+          // sub-tiles of the unit that lie inside the request's capacity (page-table range);
+          // positions are below 2^31 (checked on the host), so 32-bit arithmetic
           int rows[2];
           uint32_t bytes = 0;
           for (int h = 0; h < 2; ++h) {
-            const long long p0 = static_cast<long long>(it.j) * kUnit + h * kTile;
+            const int p0 = it.j * kUnit + h * kTile;
             rows[h] = -1;
             if (p0 >= capacity) continue;
-            const long long key = static_cast<long long>(it.b) * cache.max_pages_per_req + p0 / cache.page_size;
+            const int pidx = static_cast<int>(static_cast<uint32_t>(p0) / page_size);
+            const long long key = static_cast<long long>(it.b) * cache.max_pages_per_req + pidx;
             if (key != page_key) {   // one page-table load per page
               page_key = key;
               page = cache.page_table[key];
               if (page < 0 || page >= cache.num_pages) {
-                report_error(cache.err_word, CSA2_ERR_DEVICE_BOUNDS, kKIndexFull, it.b, static_cast<int>(p0));
+                report_error(cache.err_word, CSA2_ERR_DEVICE_BOUNDS, kKIndexFull, it.b, p0);
                 page = 0;   // load a valid page; the results of this sub-tile are flagged invalid
               }
             }
-            rows[h] = page * cache.page_size + static_cast<int>(p0 % cache.page_size);
+            rows[h] = page * cache.page_size + (p0 - pidx * cache.page_size);
             bytes += kTileBytes;
           }
           mbar_arrive_expect_tx(&S.full[s], bytes);
@@ -290,16 +293,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       int ex_page = 0;
       auto exp_bytes = [&](int b, int j, uint32_t (&e)[2]) {
         for (int h = 0; h < 2; ++h) {
-          const long long p = static_cast<long long>(j) * kUnit + h * kTile + toff;
+          const int p = j * kUnit + h * kTile + toff;
           e[h] = 127u;
           if (b >= B || p >= capacity) continue;
-          const long long key = static_cast<long long>(b) * cache.max_pages_per_req + p / cache.page_size;
+          const int pidx = static_cast<int>(static_cast<uint32_t>(p) / page_size);
+          const long long key = static_cast<long long>(b) * cache.max_pages_per_req + pidx;
           if (key != ex_key) {
             ex_key = key;
             ex_page = cache.page_table[key];
             ex_page = (ex_page < 0 || ex_page >= cache.num_pages) ? 0 : ex_page;
           }
-          e[h] = cache.ik_exp[static_cast<long long>(ex_page) * cache.page_size + p % cache.page_size];
+          e[h] = cache.ik_exp[static_cast<long long>(ex_page) * cache.page_size + (p - pidx * cache.page_size)];
         }
       };
       uint32_t ex_cur[2], ex_next[2];
