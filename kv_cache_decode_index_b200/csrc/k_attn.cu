@@ -3,20 +3,18 @@
 // blog, section 二: every layer attends over its Top-K, Reuse layers with
 // their own query; FP4 rows: 4sapi blog, section 五].
 //
-// One CTA per (query, tile of 16 heads); it walks the query's k rows in
-// chunks of 64:
-//   * the rows' cache addresses are resolved once (Top-k entry -> page);
-//   * the raw FP4 rows (256 code bytes + 32 scale bytes) of the next chunk are
-//     staged with cp.async while the current chunk is processed;
-//   * dequantisation: E2M1 code x E4M3 scale has <= 5 significant bits and lies
-//     in [2^-10, 2688], so the fp16 row is exact; codes become fp16 through a
-//     byte-permute table lookup;
+// One thread-block cluster of 8 CTAs per query.  CTA r takes Top-k entries
+// [r*kc, (r+1)*kc) (kc = ceil(k/8)) in chunks of 64 rows:
+//   * gather + dequantise: E2M1 code x E4M3 scale has <= 5 significant bits
+//     and lies in [2^-10, 2688], so the fp16 row is exact;
 //   * the query is moved to fp16 with a power-of-two scale per head (bf16 ->
 //     fp16 keeps every significant bit in the normal range);
-//   * S = Q K^T (each warp 8 keys) and O = P V (each warp 64 output dims) on
-//     mma.sync m16n8k16, fp16 in, fp32 accumulate; online softmax in fp32 in the
-//     exp2 domain, P rounded to fp16.
-// No cross-CTA reduction, no scratch memory.
+//   * S = Q K^T and O = P V on mma.sync m16n8k16 (fp16 in, fp32 accumulate),
+//     online softmax in fp32 (exp2 domain), P rounded to fp16;
+// then the 8 partial (O, max, sum) triples are merged through distributed
+// shared memory: every CTA pushes its slice of dims [64r, 64r+64) to CTA r,
+// which merges them locally and writes those dims of every head.
+#include <cooperative_groups.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -27,39 +25,40 @@ namespace csa2 {
 
 namespace {
 
+namespace cg = cooperative_groups;
+
 constexpr int kAThreads = 256;
-constexpr int kChunk = 64;                   // rows per chunk
-constexpr int kHT = 16;                      // heads per CTA
+constexpr int kACluster = 8;
+constexpr int kChunk = 64;                   // keys per chunk
 constexpr int kRowBytes = kKvDim * 2;        // fp16 row: 1024 B
-constexpr int kRawRow = kKvCodeBytes + kKvScaleBytes;   // 288 B
-constexpr int kSStride = kChunk + 4;         // fp32 row stride of S
+constexpr int kSredStride = kChunk + 8;      // fp32 row stride of the S reduction buffer
 constexpr float kLog2e = 1.4426950408889634f;
 
+template <int H>
 struct AttnLayout {
-  static constexpr uint32_t q_off = 0;                                  // fp16 [16][512], swizzled
-  static constexpr uint32_t kv_off = q_off + kHT * kRowBytes;           // fp16 [64][512], swizzled
-  static constexpr uint32_t raw_off = kv_off + kChunk * kRowBytes;      // u8 [2][64][288]
-  static constexpr uint32_t s_off = raw_off + 2 * kChunk * kRawRow;     // fp32 [16][68]
-  static constexpr uint32_t p_off = s_off + kHT * kSStride * 4;         // fp16 [16][64], swizzled (128 B rows)
-  static constexpr uint32_t st_off = p_off + kHT * kChunk * 2;          // fp32 qscale[16], m[16], l[16], corr[16]
-  static constexpr uint32_t rows_off = st_off + 4 * kHT * 4;            // int32 [k] cache row of each entry
-  __host__ __device__ static uint32_t total(int k) { return rows_off + 4u * static_cast<uint32_t>(k); }
+  static constexpr int HT = H / 16;            // head tiles of 16
+  static constexpr int DG = 8 / HT;            // dim groups (warps per head tile)
+  static constexpr int DW = kKvDim / DG;       // dims per warp
+  static constexpr uint32_t q_off = 0;                               // fp16 [H][512]
+  static constexpr uint32_t kv_off = q_off + H * kRowBytes;          // fp16 [64][512]
+  static constexpr uint32_t sred_off = kv_off + kChunk * kRowBytes;  // fp32 [DG][H][72]
+  static constexpr uint32_t qscale_off = sred_off + DG * H * kSredStride * 4;
+  static constexpr uint32_t ml_off = qscale_off + H * 4;             // fp32 [8 ranks][2][H]: pushed m, l
+  static constexpr uint32_t fac_off = ml_off + kACluster * 2 * H * 4; // fp32 [8][H]
+  static constexpr uint32_t kvalid_off = fac_off + kACluster * H * 4;
+  static constexpr uint32_t total = kvalid_off + kChunk * 4;
+  // pushed partial O: [8 source ranks][H][64 dims] fp32, over the Q + KV region
+  static_assert(kACluster * H * 64 * 4 <= sred_off, "received partials must fit in the Q + KV region");
 };
 
 __device__ __forceinline__ uint32_t swz(uint32_t row, uint32_t chunk) {   // 16-byte chunk of a 1 KB row
   return row * kRowBytes + ((chunk ^ (row & 7u)) << 4);
-}
-__device__ __forceinline__ uint32_t swz_p(uint32_t row, uint32_t chunk) {  // 16-byte chunk of a 128 B row
-  return row * (kChunk * 2) + ((chunk ^ (row & 7u)) << 4);
 }
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
                : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
                : "r"(addr));
-}
-__device__ __forceinline__ void ldsm_x2(uint32_t addr, uint32_t& r0, uint32_t& r1) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0,%1}, [%2];" : "=r"(r0), "=r"(r1) : "r"(addr));
 }
 __device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
@@ -78,298 +77,342 @@ __device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
   const __half2 h = __floats2half2_rn(lo, hi);
   return *reinterpret_cast<const uint32_t*>(&h);
 }
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void cp_async_wait_1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
 
-// Four E2M1 codes (two bytes, low nibble first) -> four fp16 values times the
-// fp16 scale s2 (two half2 words).  The magnitude bits index a byte table of
-// the fp16 high bytes of 0, 0.5, 1, 1.5, 2, 3, 4, 6; the sign bit of each code
-// becomes bit 15 of its fp16.
-__device__ __forceinline__ uint2 e2m1x4_to_half2(uint32_t two_bytes, __half2 s2) {
-  // the permute selects byte n by the low 3 bits of nibble n: code n's magnitude
-  const uint32_t hib = __byte_perm(0x3E3C3800u, 0x46444240u, two_bytes);            // table[code & 7] per byte
-  // code n spread to byte n, so that its sign bit (bit 3) moves to bit 7 of byte n
-  const uint32_t spread = (two_bytes & 0xFu) | ((two_bytes & 0xF0u) << 4) | ((two_bytes & 0xF00u) << 8) |
-                          ((two_bytes & 0xF000u) << 12);
-  const uint32_t sgn = (spread << 4) & 0x80808080u;
-  const uint32_t h = hib | sgn;
-  uint32_t w0 = __byte_perm(h, 0u, 0x1404u);   // [0, h0, 0, h1]: fp16 of codes 0, 1
-  uint32_t w1 = __byte_perm(h, 0u, 0x3424u);   // fp16 of codes 2, 3
-  __half2 v0 = __hmul2(*reinterpret_cast<__half2*>(&w0), s2);
-  __half2 v1 = __hmul2(*reinterpret_cast<__half2*>(&w1), s2);
-  return make_uint2(*reinterpret_cast<uint32_t*>(&v0), *reinterpret_cast<uint32_t*>(&v1));
+// Dequantise 16 code bytes (32 channels, 2 scale groups) into 4 fp16 chunks.
+__device__ __forceinline__ void dequant16(uint4 codes, uint32_t s01, uint4 (&out)[4]) {
+  const uint32_t sc0 = e4m3_half_bits(s01 & 0xFFu), sc1 = e4m3_half_bits((s01 >> 8) & 0xFFu);
+  const __half2 s0 = __halves2half2(__ushort_as_half(sc0), __ushort_as_half(sc0));
+  const __half2 s1 = __halves2half2(__ushort_as_half(sc1), __ushort_as_half(sc1));
+  const uint32_t w[4] = {codes.x, codes.y, codes.z, codes.w};
+  uint32_t h[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const uint32_t byte = (w[i >> 2] >> (8 * (i & 3))) & 0xFFu;
+    const uint32_t pair = e2m1_half_bits(byte & 0xFu) | (static_cast<uint32_t>(e2m1_half_bits(byte >> 4)) << 16);
+    __half2 v = *reinterpret_cast<const __half2*>(&pair);
+    v = __hmul2(v, i < 8 ? s0 : s1);   // exact: <= 5 significant bits, inside fp16's normal range
+    h[i] = *reinterpret_cast<const uint32_t*>(&v);
+  }
+#pragma unroll
+  for (int c = 0; c < 4; ++c) out[c] = make_uint4(h[4 * c], h[4 * c + 1], h[4 * c + 2], h[4 * c + 3]);
 }
 
+template <int H>
 __global__ void __launch_bounds__(kAThreads, 1)
     sparse_attn_kernel(const csa2_cache cache, const int32_t* __restrict__ q_req, const int32_t* __restrict__ topk,
-                       int K, int H, const __nv_bfloat16* __restrict__ qg, float softmax_scale,
-                       __nv_bfloat16* __restrict__ out) {
-  using L = AttnLayout;
+                       int K, const __nv_bfloat16* __restrict__ qg, float softmax_scale, __nv_bfloat16* __restrict__ out) {
+  using L = AttnLayout<H>;
   extern __shared__ __align__(1024) uint8_t smem[];
   const uint32_t sbase = smem_u32(smem);
-  float* s_sh = reinterpret_cast<float*>(smem + L::s_off);
-  float* qscale = reinterpret_cast<float*>(smem + L::st_off);
-  float* m_sh = qscale + kHT;
-  float* l_sh = m_sh + kHT;
-  float* corr_sh = l_sh + kHT;
-  int* rows = reinterpret_cast<int*>(smem + L::rows_off);
+  float* sred = reinterpret_cast<float*>(smem + L::sred_off);
+  float* qscale = reinterpret_cast<float*>(smem + L::qscale_off);
+  float* ml_sh = reinterpret_cast<float*>(smem + L::ml_off);
+  float* fac = reinterpret_cast<float*>(smem + L::fac_off);
+  int* kvalid = reinterpret_cast<int*>(smem + L::kvalid_off);
 
-  const int tiles_per_q = H / kHT;
-  const int qi = blockIdx.x / tiles_per_q, ht = blockIdx.x % tiles_per_q;
+  cg::cluster_group cluster = cg::this_cluster();
+  const int rank = static_cast<int>(cluster.block_rank());
+  const int qi = blockIdx.x / kACluster;
   const int b = q_req != nullptr ? q_req[qi] : qi;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int ht = warp % L::HT, dg = warp / L::HT;
   const long long capacity = static_cast<long long>(cache.max_pages_per_req) * cache.page_size;
   int n = (b >= 0 && b < cache.batch) ? cache.ctx_len[b] : 0;
   n = n < 0 ? 0 : (n > capacity ? static_cast<int>(capacity) : n);
   const int32_t* idx = topk + static_cast<long long>(qi) * K;
 
-  // ---- cache row of every Top-k entry (-1: skipped) ----
-  for (int base = 0; base < K; base += kAThreads * 4) {
-    int t[4], pg[4];
+  // ---- query -> fp16 with a power-of-two scale per head ----
+  constexpr int kHpw = H / (kAThreads / 32);   // heads per warp; their loads are issued together
+  uint4 raw[kHpw][2];
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int i = base + u * kAThreads + tid;
-      t[u] = i < K ? idx[i] : -1;
+  for (int hh = 0; hh < kHpw; ++hh) {
+    const uint4* src =
+        reinterpret_cast<const uint4*>(qg + (static_cast<long long>(qi) * H + warp * kHpw + hh) * kKvDim) + lane * 2;
+    raw[hh][0] = src[0];
+    raw[hh][1] = src[1];
+  }
+#pragma unroll
+  for (int hh = 0; hh < kHpw; ++hh) {
+    const int h = warp * kHpw + hh;
+    const uint4 v0 = raw[hh][0], v1 = raw[hh][1];
+    const uint32_t wv[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+    float f[16];
+    float amax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      f[2 * i] = __uint_as_float(wv[i] << 16);
+      f[2 * i + 1] = __uint_as_float(wv[i] & 0xFFFF0000u);
+      amax = fmaxf(amax, fmaxf(fabsf(f[2 * i]), fabsf(f[2 * i + 1])));
     }
 #pragma unroll
-    for (int u = 0; u < 4; ++u)
-      pg[u] = (t[u] >= 0 && t[u] < n)
-                  ? cache.page_table[static_cast<long long>(b) * cache.max_pages_per_req + t[u] / cache.page_size]
-                  : -1;
+    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    int E = static_cast<int>((__float_as_uint(amax) >> 23) & 0xFF) - 127;   // amax in [2^E, 2^(E+1))
+    if (amax == 0.0f) E = 14;
+    E = max(E, -100);
+    const float up = exp2i(14 - E), down = exp2i(E - 14);
+    uint32_t hv[8];
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int i = base + u * kAThreads + tid;
-      if (i >= K) continue;
-      int row = -1;
-      if (t[u] >= 0 && t[u] < n) {
-        if (pg[u] >= 0 && pg[u] < cache.num_pages) row = pg[u] * cache.page_size + t[u] % cache.page_size;
-        else if (ht == 0) report_error(cache.err_word, CSA2_ERR_DEVICE_BOUNDS, kKAttn, b, t[u]);
-      } else if (t[u] != -1 && ht == 0) {
-        report_error(cache.err_word, CSA2_ERR_DEVICE_BOUNDS, kKAttn, b, t[u]);
-      }
-      rows[i] = row;
-    }
+    for (int i = 0; i < 8; ++i) hv[i] = pack_half2(f[2 * i] * up, f[2 * i + 1] * up);
+    // lane holds dims [16*lane, 16*lane+16): chunks 2*lane, 2*lane+1
+    *reinterpret_cast<uint4*>(smem + swz(h, 2 * lane)) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
+    *reinterpret_cast<uint4*>(smem + swz(h, 2 * lane + 1)) = make_uint4(hv[4], hv[5], hv[6], hv[7]);
+    if (lane == 0) qscale[h] = softmax_scale * down * kLog2e;
   }
 
-  // ---- query heads [16 ht, 16 ht + 16) -> fp16 with a power-of-two scale per head ----
-  {
-    uint4 raw[2][2];
-#pragma unroll
-    for (int hh = 0; hh < 2; ++hh) {
-      const int h = ht * kHT + warp * 2 + hh;
-      const uint4* src = reinterpret_cast<const uint4*>(qg + (static_cast<long long>(qi) * H + h) * kKvDim) + lane * 2;
-      raw[hh][0] = src[0];
-      raw[hh][1] = src[1];
-    }
-#pragma unroll
-    for (int hh = 0; hh < 2; ++hh) {
-      const int hl = warp * 2 + hh;   // head inside the tile
-      const uint4 v0 = raw[hh][0], v1 = raw[hh][1];
-      const uint32_t wv[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-      float f[16];
-      float amax = 0.0f;
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        f[2 * i] = __uint_as_float(wv[i] << 16);
-        f[2 * i + 1] = __uint_as_float(wv[i] & 0xFFFF0000u);
-        amax = fmaxf(amax, fmaxf(fabsf(f[2 * i]), fabsf(f[2 * i + 1])));
-      }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-      int E = static_cast<int>((__float_as_uint(amax) >> 23) & 0xFF) - 127;   // amax in [2^E, 2^(E+1))
-      if (amax == 0.0f) E = 14;
-      E = max(E, -100);
-      const float up = exp2i(14 - E), down = exp2i(E - 14);
-      uint32_t hv[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) hv[i] = pack_half2(f[2 * i] * up, f[2 * i + 1] * up);
-      *reinterpret_cast<uint4*>(smem + L::q_off + swz(hl, 2 * lane)) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
-      *reinterpret_cast<uint4*>(smem + L::q_off + swz(hl, 2 * lane + 1)) = make_uint4(hv[4], hv[5], hv[6], hv[7]);
-      if (lane == 0) {
-        qscale[hl] = softmax_scale * down * kLog2e;
-        m_sh[hl] = -INFINITY;
-        l_sh[hl] = 0.0f;
-      }
-    }
-  }
-  __syncthreads();   // rows[] ready
+  // ---- this CTA's keys ----
+  const int kc = (K + kACluster - 1) / kACluster;
+  const int key_begin = min(rank * kc, K), key_end = min(key_begin + kc, K);
 
-  // ---- staging of a chunk's raw rows: 64 rows x 18 pieces of 16 bytes ----
-  const int nchunks = (K + kChunk - 1) / kChunk;
-  auto stage = [&](int c) {
-    const uint32_t dst0 = sbase + L::raw_off + (c & 1) * kChunk * kRawRow;
-    for (int p = tid; p < kChunk * (kRawRow / 16); p += kAThreads) {
-      const int r = p / (kRawRow / 16), u = p % (kRawRow / 16);
-      const int key = c * kChunk + r;
-      const int row = key < K ? rows[key] : -1;
-      if (row < 0) continue;
-      const uint8_t* src =
-          u < kKvCodeBytes / 16
-              ? cache.kv_codes + static_cast<long long>(row) * kKvCodeBytes + u * 16
-              : cache.kv_scales + static_cast<long long>(row) * kKvScaleBytes + (u - kKvCodeBytes / 16) * 16;
-      cp_async16(dst0 + r * kRawRow + u * 16, src);
-    }
-    cp_async_commit();
-  };
-  stage(0);
-
-  float o_acc[8][4];   // O[16 heads x 64 dims of this warp]
+  float o_acc[L::DW / 8][4];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) o_acc[i][0] = o_acc[i][1] = o_acc[i][2] = o_acc[i][3] = 0.0f;
-  const int r0 = lane >> 2;
+  for (int i = 0; i < L::DW / 8; ++i) o_acc[i][0] = o_acc[i][1] = o_acc[i][2] = o_acc[i][3] = 0.0f;
+  float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.0f, 0.0f};
+  const int r0 = lane >> 2;   // fragment row (and row + 8)
 
-  for (int c = 0; c < nchunks; ++c) {
-    if (c + 1 < nchunks) stage(c + 1);
-    else cp_async_commit();   // keep the group count uniform
-    cp_async_wait_1();        // chunk c has landed (this thread's copies)
-    __syncthreads();          // ... and everyone's
-
-    // ---- dequantise chunk c: thread = (row, quarter of 128 channels) ----
+  for (int c0 = key_begin; c0 < key_end; c0 += kChunk) {
+    const int nk = min(kChunk, key_end - c0);
+    __syncthreads();   // previous chunk's KV no longer read
     {
+      // gather + dequantise: 4 threads per row, 128 channels each
       const int row = tid >> 2, part = tid & 3;
-      const uint8_t* raw = smem + L::raw_off + (c & 1) * kChunk * kRawRow + row * kRawRow;
-      const int key = c * kChunk + row;
-      const bool valid = key < K && rows[key] >= 0;
-      const uint4* cw = reinterpret_cast<const uint4*>(raw + part * 64);
-      const uint2 sc = *reinterpret_cast<const uint2*>(raw + kKvCodeBytes + part * 8);
+      int t = row < nk ? idx[c0 + row] : -1;
+      long long src_row = -1;
+      if (t >= 0 && t < n) {
+        const int page = cache.page_table[static_cast<long long>(b) * cache.max_pages_per_req + t / cache.page_size];
+        if (page >= 0 && page < cache.num_pages) src_row = static_cast<long long>(page) * cache.page_size + t % cache.page_size;
+        else if (part == 0) report_error(cache.err_word, CSA2_ERR_DEVICE_BOUNDS, kKAttn, b, t);
+      } else if (row < nk && (t >= n || t < -1) && part == 0) {
+        report_error(cache.err_word, CSA2_ERR_DEVICE_BOUNDS, kKAttn, b, t);
+      }
+      if (part == 0) kvalid[row] = src_row >= 0;
+      if (src_row >= 0) {
+        const uint4* cp = reinterpret_cast<const uint4*>(cache.kv_codes + src_row * kKvCodeBytes) + part * 4;
+        const uint2 sp = *reinterpret_cast<const uint2*>(cache.kv_scales + src_row * kKvScaleBytes + part * 8);
+        uint4 cv[4];   // every load of the row part in flight before any shared-memory store
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {   // 16 code bytes = 32 channels = 2 scale groups
-        const uint4 v = valid ? cw[j] : make_uint4(0, 0, 0, 0);
-        const uint32_t sbytes = j < 2 ? (sc.x >> (16 * j)) : (sc.y >> (16 * (j - 2)));
-        const uint16_t s0b = valid ? e4m3_half_bits(sbytes & 0xFFu) : 0;
-        const uint16_t s1b = valid ? e4m3_half_bits((sbytes >> 8) & 0xFFu) : 0;
-        const __half2 s0 = __halves2half2(__ushort_as_half(s0b), __ushort_as_half(s0b));
-        const __half2 s1 = __halves2half2(__ushort_as_half(s1b), __ushort_as_half(s1b));
-        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-        uint32_t hv[16];
+        for (int j = 0; j < 4; ++j) cv[j] = cp[j];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {   // 4 code bytes = 8 channels per word
-          const uint2 lo = e2m1x4_to_half2(w[q] & 0xFFFFu, q < 2 ? s0 : s1);
-          const uint2 hi = e2m1x4_to_half2(w[q] >> 16, q < 2 ? s0 : s1);
-          hv[4 * q] = lo.x;
-          hv[4 * q + 1] = lo.y;
-          hv[4 * q + 2] = hi.x;
-          hv[4 * q + 3] = hi.y;
+        for (int j = 0; j < 4; ++j) {
+          uint4 hv[4];
+          dequant16(cv[j], j < 2 ? (sp.x >> (16 * j)) : (sp.y >> (16 * (j - 2))), hv);
+          const int chunk0 = part * 16 + j * 4;   // 8 fp16 per chunk
+#pragma unroll
+          for (int c = 0; c < 4; ++c) *reinterpret_cast<uint4*>(smem + L::kv_off + swz(row, chunk0 + c)) = hv[c];
         }
-        const int chunk0 = part * 16 + j * 4;   // 8 fp16 per 16-byte chunk
+      } else {
 #pragma unroll
-        for (int q = 0; q < 4; ++q)
-          *reinterpret_cast<uint4*>(smem + L::kv_off + swz(row, chunk0 + q)) =
-              make_uint4(hv[4 * q], hv[4 * q + 1], hv[4 * q + 2], hv[4 * q + 3]);
+        for (int c = 0; c < 16; ++c)
+          *reinterpret_cast<uint4*>(smem + L::kv_off + swz(row, part * 16 + c)) = make_uint4(0, 0, 0, 0);
       }
     }
     __syncthreads();
 
-    // ---- S = Q K^T: warp w scores keys [8w, 8w + 8) over all 512 dims ----
-    {
-      float s[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 8
-      for (int ks = 0; ks < kKvDim / 16; ++ks) {
-        uint32_t a0, a1, a2, a3, b0, b1;
-        ldsm_x4(sbase + L::q_off + swz(lane & 15, 2 * ks + (lane >> 4)), a0, a1, a2, a3);
-        ldsm_x2(sbase + L::kv_off + swz(warp * 8 + (lane & 7), 2 * ks + ((lane >> 3) & 1)), b0, b1);
-        mma_f16(s, a0, a1, a2, a3, b0, b1);
-      }
-      const int col = warp * 8 + 2 * (lane & 3);
-      const int k0 = c * kChunk + col;
-      const bool v0 = k0 < K && rows[k0] >= 0, v1 = k0 + 1 < K && rows[k0 + 1] >= 0;
-      const float sc0 = qscale[r0], sc1 = qscale[r0 + 8];
-      s_sh[r0 * kSStride + col] = v0 ? s[0] * sc0 : -INFINITY;
-      s_sh[r0 * kSStride + col + 1] = v1 ? s[1] * sc0 : -INFINITY;
-      s_sh[(r0 + 8) * kSStride + col] = v0 ? s[2] * sc1 : -INFINITY;
-      s_sh[(r0 + 8) * kSStride + col + 1] = v1 ? s[3] * sc1 : -INFINITY;
-    }
-    __syncthreads();
-
-    // ---- online softmax: warp w owns heads 2w, 2w+1 ----
+    // ---- S = Q K^T over this warp's dims ----
+    float s[8][4];
 #pragma unroll
-    for (int hh = 0; hh < 2; ++hh) {
-      const int h = warp * 2 + hh;
-      const float x0 = s_sh[h * kSStride + lane], x1 = s_sh[h * kSStride + lane + 32];
-      float mx = fmaxf(x0, x1);
+    for (int j = 0; j < 8; ++j) s[j][0] = s[j][1] = s[j][2] = s[j][3] = 0.0f;
+#pragma unroll 4
+    for (int ks = 0; ks < L::DW / 16; ++ks) {
+      const int kchunk = (dg * L::DW + ks * 16) / 8;
+      uint32_t a0, a1, a2, a3;
+      ldsm_x4(sbase + L::q_off + swz(ht * 16 + (lane & 15), kchunk + (lane >> 4)), a0, a1, a2, a3);
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-      const float m_old = m_sh[h];
-      const float m_new = fmaxf(m_old, mx);
-      const float ref = m_new == -INFINITY ? 0.0f : m_new;
-      const float p0 = exp2f(x0 - ref), p1 = exp2f(x1 - ref);
-      float sum = p0 + p1;
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-      // P[h][lane] and P[h][lane + 32] as fp16: 128-byte rows, swizzled 16-byte chunks
-      *reinterpret_cast<__half*>(smem + L::p_off + swz_p(h, lane >> 3) + (lane & 7) * 2) = __float2half_rn(p0);
-      *reinterpret_cast<__half*>(smem + L::p_off + swz_p(h, (lane + 32) >> 3) + (lane & 7) * 2) = __float2half_rn(p1);
-      __syncwarp();
-      if (lane == 0) {
-        const float cr = exp2f(m_old - ref);   // 0 when m_old = -inf
-        corr_sh[h] = cr;
-        l_sh[h] = l_sh[h] * cr + sum;
-        m_sh[h] = m_new;
+      for (int np = 0; np < 4; ++np) {   // pairs of 8-key tiles
+        const int mi = lane >> 3;
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4(sbase + L::kv_off + swz(np * 16 + (mi >> 1) * 8 + (lane & 7), kchunk + (mi & 1)), b0, b1, b2, b3);
+        mma_f16(s[2 * np], a0, a1, a2, a3, b0, b1);
+        mma_f16(s[2 * np + 1], a0, a1, a2, a3, b2, b3);
       }
     }
-    __syncthreads();
-
-    // ---- O = O * corr + P V: warp w owns output dims [64w, 64w + 64) ----
-    {
-      const float c0 = corr_sh[r0], c1 = corr_sh[r0 + 8];
+    if (L::DG > 1) {
+      float* mine = sred + (dg * H + ht * 16) * kSredStride;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        o_acc[i][0] *= c0;
-        o_acc[i][1] *= c0;
-        o_acc[i][2] *= c1;
-        o_acc[i][3] *= c1;
+      for (int j = 0; j < 8; ++j) {
+        const int col = j * 8 + 2 * (lane & 3);
+        *reinterpret_cast<float2*>(mine + r0 * kSredStride + col) = make_float2(s[j][0], s[j][1]);
+        *reinterpret_cast<float2*>(mine + (r0 + 8) * kSredStride + col) = make_float2(s[j][2], s[j][3]);
       }
+      __syncthreads();
 #pragma unroll
-      for (int kk = 0; kk < kChunk / 16; ++kk) {
-        uint32_t a0, a1, a2, a3;
-        ldsm_x4(sbase + L::p_off + swz_p(lane & 15, 2 * kk + (lane >> 4)), a0, a1, a2, a3);
+      for (int j = 0; j < 8; ++j) s[j][0] = s[j][1] = s[j][2] = s[j][3] = 0.0f;
+      for (int g = 0; g < L::DG; ++g) {
+        const float* part = sred + (g * H + ht * 16) * kSredStride;
 #pragma unroll
-        for (int np = 0; np < 4; ++np) {   // pairs of 8-dim tiles
-          const int mi = lane >> 3;
-          const int dchunk = warp * 8 + np * 2 + (mi >> 1);
-          uint32_t b0, b1, b2, b3;
-          ldsm_x4_t(sbase + L::kv_off + swz(kk * 16 + (mi & 1) * 8 + (lane & 7), dchunk), b0, b1, b2, b3);
-          mma_f16(o_acc[2 * np], a0, a1, a2, a3, b0, b1);
-          mma_f16(o_acc[2 * np + 1], a0, a1, a2, a3, b2, b3);
+        for (int j = 0; j < 8; ++j) {
+          const int col = j * 8 + 2 * (lane & 3);
+          const float2 u = *reinterpret_cast<const float2*>(part + r0 * kSredStride + col);
+          const float2 v = *reinterpret_cast<const float2*>(part + (r0 + 8) * kSredStride + col);
+          s[j][0] += u.x; s[j][1] += u.y; s[j][2] += v.x; s[j][3] += v.y;
         }
       }
     }
-    __syncthreads();   // kv, S and P are rewritten by the next chunk
+
+    // ---- online softmax (log2 domain) ----
+    const float sc0 = qscale[ht * 16 + r0], sc1 = qscale[ht * 16 + r0 + 8];
+    float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int col = j * 8 + 2 * (lane & 3);
+      const bool v0 = col < nk && kvalid[col], v1 = col + 1 < nk && kvalid[col + 1];
+      s[j][0] = v0 ? s[j][0] * sc0 : -INFINITY;
+      s[j][1] = v1 ? s[j][1] * sc0 : -INFINITY;
+      s[j][2] = v0 ? s[j][2] * sc1 : -INFINITY;
+      s[j][3] = v1 ? s[j][3] * sc1 : -INFINITY;
+      mx0 = fmaxf(mx0, fmaxf(s[j][0], s[j][1]));
+      mx1 = fmaxf(mx1, fmaxf(s[j][2], s[j][3]));
+    }
+#pragma unroll
+    for (int o = 1; o < 4; o <<= 1) {
+      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
+    }
+    const float mn0 = fmaxf(m_run[0], mx0), mn1 = fmaxf(m_run[1], mx1);
+    const float ref0 = mn0 == -INFINITY ? 0.0f : mn0, ref1 = mn1 == -INFINITY ? 0.0f : mn1;
+    const float corr0 = exp2f(m_run[0] - ref0), corr1 = exp2f(m_run[1] - ref1);
+    float sum0 = 0.0f, sum1 = 0.0f;
+    uint32_t pa[4][4];   // P as fp16 A fragments, one per 16-key step
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const float p0 = exp2f(s[j][0] - ref0), p1 = exp2f(s[j][1] - ref0);
+      const float p2 = exp2f(s[j][2] - ref1), p3 = exp2f(s[j][3] - ref1);
+      sum0 += p0 + p1;
+      sum1 += p2 + p3;
+      pa[j >> 1][(j & 1) * 2 + 0] = pack_half2(p0, p1);
+      pa[j >> 1][(j & 1) * 2 + 1] = pack_half2(p2, p3);
+    }
+#pragma unroll
+    for (int o = 1; o < 4; o <<= 1) {
+      sum0 += __shfl_xor_sync(0xffffffffu, sum0, o);
+      sum1 += __shfl_xor_sync(0xffffffffu, sum1, o);
+    }
+    l_run[0] = l_run[0] * corr0 + sum0;
+    l_run[1] = l_run[1] * corr1 + sum1;
+    m_run[0] = mn0;
+    m_run[1] = mn1;
+#pragma unroll
+    for (int i = 0; i < L::DW / 8; ++i) {
+      o_acc[i][0] *= corr0; o_acc[i][1] *= corr0;
+      o_acc[i][2] *= corr1; o_acc[i][3] *= corr1;
+    }
+
+    // ---- O += P V over this warp's dims ----
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk) {
+      // A fragment order: (row, k lo), (row+8, k lo), (row, k hi), (row+8, k hi)
+      const uint32_t a0 = pa[kk][0], a1 = pa[kk][1], a2 = pa[kk][2], a3 = pa[kk][3];
+#pragma unroll
+      for (int np = 0; np < L::DW / 16; ++np) {
+        const int mi = lane >> 3;
+        const int dchunk = (dg * L::DW) / 8 + np * 2 + (mi >> 1);
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4_t(sbase + L::kv_off + swz(kk * 16 + (mi & 1) * 8 + (lane & 7), dchunk), b0, b1, b2, b3);
+        mma_f16(o_acc[2 * np], a0, a1, a2, a3, b0, b1);
+        mma_f16(o_acc[2 * np + 1], a0, a1, a2, a3, b2, b3);
+      }
+    }
   }
 
-  // ---- normalise and write bf16 ----
-  const float l0 = l_sh[r0], l1 = l_sh[r0 + 8];
-  const float i0 = l0 > 0.0f ? 1.0f / l0 : 0.0f, i1 = l1 > 0.0f ? 1.0f / l1 : 0.0f;
-  const long long head0 = static_cast<long long>(qi) * H + ht * kHT;
+  // ---- push the partial O slices, maxima and sums to their owners ----
+  // Output dims [64r, 64r + 64) belong to CTA r; it receives every rank's
+  // slice of them in recv[src][h][64].  Remote stores are fire-and-forget.
+  cluster.sync();   // every CTA is done reading its Q / KV region, which receives the partials
+  float* recv = reinterpret_cast<float*>(smem);
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const int col = warp * 64 + i * 8 + 2 * (lane & 3);
-    const __nv_bfloat162 v0 = __floats2bfloat162_rn(o_acc[i][0] * i0, o_acc[i][1] * i0);
-    const __nv_bfloat162 v1 = __floats2bfloat162_rn(o_acc[i][2] * i1, o_acc[i][3] * i1);
-    *reinterpret_cast<__nv_bfloat162*>(out + (head0 + r0) * kKvDim + col) = v0;
-    *reinterpret_cast<__nv_bfloat162*>(out + (head0 + r0 + 8) * kKvDim + col) = v1;
+  for (int i = 0; i < L::DW / 8; ++i) {
+    const int col = dg * L::DW + i * 8 + 2 * (lane & 3);
+    const int owner = col >> 6, c64 = col & 63;
+    float* dst = cluster.map_shared_rank(recv, owner) + (rank * H + ht * 16 + r0) * 64 + c64;
+    *reinterpret_cast<float2*>(dst) = make_float2(o_acc[i][0], o_acc[i][1]);
+    *reinterpret_cast<float2*>(dst + 8 * 64) = make_float2(o_acc[i][2], o_acc[i][3]);
   }
+  if (dg == 0 && (lane & 3) == 0) {
+    for (int r = 0; r < kACluster; ++r) {
+      float* dst = cluster.map_shared_rank(ml_sh, r) + rank * 2 * H;
+      dst[ht * 16 + r0] = m_run[0];
+      dst[ht * 16 + r0 + 8] = m_run[1];
+      dst[H + ht * 16 + r0] = l_run[0];
+      dst[H + ht * 16 + r0 + 8] = l_run[1];
+    }
+  }
+  cluster.sync();   // all partials delivered
+
+  // merge factors per (source rank, head): exp2(m_r - M) / L
+  for (int h = tid; h < H; h += kAThreads) {
+    float mr[kACluster], lr[kACluster];
+    float M = -INFINITY;
+#pragma unroll
+    for (int r = 0; r < kACluster; ++r) {
+      mr[r] = ml_sh[r * 2 * H + h];
+      lr[r] = ml_sh[r * 2 * H + H + h];
+      M = fmaxf(M, mr[r]);
+    }
+    float Lsum = 0.0f;
+#pragma unroll
+    for (int r = 0; r < kACluster; ++r) {
+      mr[r] = (M == -INFINITY || mr[r] == -INFINITY) ? 0.0f : exp2f(mr[r] - M);
+      Lsum += lr[r] * mr[r];
+    }
+    const float inv = Lsum > 0.0f ? 1.0f / Lsum : 0.0f;
+#pragma unroll
+    for (int r = 0; r < kACluster; ++r) fac[r * H + h] = mr[r] * inv;
+  }
+  __syncthreads();
+  // this CTA writes dims [64*rank, 64*rank + 64) of every head, 4 dims per item
+  for (int item = tid; item < H * 16; item += kAThreads) {
+    const int h = item >> 4, d4 = (item & 15) * 4;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int r = 0; r < kACluster; ++r) {
+      const float4 v = *reinterpret_cast<const float4*>(recv + (r * H + h) * 64 + d4);
+      const float f = fac[r * H + h];
+      acc.x += v.x * f; acc.y += v.y * f; acc.z += v.z * f; acc.w += v.w * f;
+    }
+    __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y), hi = __floats2bfloat162_rn(acc.z, acc.w);
+    uint2 pk;
+    pk.x = *reinterpret_cast<uint32_t*>(&lo);
+    pk.y = *reinterpret_cast<uint32_t*>(&hi);
+    *reinterpret_cast<uint2*>(out + (static_cast<long long>(qi) * H + h) * kKvDim + rank * 64 + d4) = pk;
+  }
+}
+
+template <int H>
+cudaError_t launch_h(const csa2_cache& cache, int n_queries, const int32_t* q_req, const int32_t* topk, int k,
+                     const uint16_t* q, float scale, uint16_t* out, cudaStream_t stream) {
+  static bool done = false;
+  const size_t smem = AttnLayout<H>::total;
+  if (!done) {
+    cudaError_t e = cudaFuncSetAttribute(sparse_attn_kernel<H>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    done = true;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(n_queries * kACluster);
+  cfg.blockDim = dim3(kAThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = kACluster;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, sparse_attn_kernel<H>, cache, q_req, topk, k,
+                            reinterpret_cast<const __nv_bfloat16*>(q), scale, reinterpret_cast<__nv_bfloat16*>(out));
 }
 
 }  // namespace
 
 cudaError_t launch_sparse_attn(const csa2_cache& cache, int n_queries, const int32_t* q_req, const int32_t* topk,
                                int k, const uint16_t* q, int H, float scale, uint16_t* out, cudaStream_t stream) {
-  static bool done = false;
-  constexpr int kMaxK = 4096;
-  if (!done) {
-    const cudaError_t e = cudaFuncSetAttribute(sparse_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                               static_cast<int>(AttnLayout::total(kMaxK)));
-    if (e != cudaSuccess) return e;
-    done = true;
+  switch (H) {
+    case 16: return launch_h<16>(cache, n_queries, q_req, topk, k, q, scale, out, stream);
+    case 32: return launch_h<32>(cache, n_queries, q_req, topk, k, q, scale, out, stream);
+    case 64: return launch_h<64>(cache, n_queries, q_req, topk, k, q, scale, out, stream);
+    default: return cudaErrorInvalidValue;
   }
-  sparse_attn_kernel<<<n_queries * (H / kHT), kAThreads, AttnLayout::total(k), stream>>>(
-      cache, q_req, topk, k, H, reinterpret_cast<const __nv_bfloat16*>(q), scale,
-      reinterpret_cast<__nv_bfloat16*>(out));
-  return cudaGetLastError();
 }
 
 }  // namespace csa2
