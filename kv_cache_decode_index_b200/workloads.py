@@ -148,6 +148,17 @@ def main_query(wl: Workload, layer: int, rows: int | None = None):
     return torch.from_numpy(q).to(torch.bfloat16)
 
 
+def prefill_positions(wl: Workload) -> np.ndarray:
+    """Token positions (int32) of the prefill queries: the last
+    `prefill_queries` tokens of a `prefill_tokens`-token stream."""
+    return np.arange(wl.prefill_tokens - wl.prefill_queries, wl.prefill_tokens, dtype=np.int32)
+
+
+def prefill_ratio(wl: Workload) -> int:
+    """Tokens per compressed entry of a prefill workload (m = 2 on the pages)."""
+    return wl.prefill_tokens // wl.ctx
+
+
 # -------------------------------------------------------------- cache rows --
 
 def channel_scale(wl: Workload) -> np.ndarray:

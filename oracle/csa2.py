@@ -189,14 +189,16 @@ def decode_group(modes, q_idx, w_idx, ik_codes, ik_exp, n: int,
 
 # ----------------------------------------------------------- causal prefill --
 
-def prefill_visible(p: int) -> int:
-    """Entries visible to the query at token p when entry e covers tokens 2e
-    and 2e+1 (m = 2): e is visible iff 2e + 1 <= p, i.e. floor((p + 1) / 2)."""
-    return (p + 1) // 2
+def prefill_visible(p: int, m: int = 2) -> int:
+    """Entries visible to the query at token p when entry e covers the m tokens
+    m*e .. m*e + m - 1 (m = 2 on the pages' compressed prefill): e is visible
+    iff its last token is not after p, m*e + m - 1 <= p, i.e. floor((p + 1) / m).
+    A negative p sees nothing."""
+    return max(0, (p + 1) // m)
 
 
-def prefill_topk(q, w, ik_codes, ik_exp, p: int, k: int = TOPK) -> np.ndarray:
+def prefill_topk(q, w, ik_codes, ik_exp, p: int, k: int = TOPK, m: int = 2) -> np.ndarray:
     """Top-k of one prefill query at token p over its visible entries (no pool)."""
-    v = min(prefill_visible(p), len(ik_codes))
+    v = min(prefill_visible(p, m), len(ik_codes))
     s = indexer_scores(q, w, ik_codes[:v], ik_exp[:v])
     return top_k_ascending(np.arange(v), s, k)

@@ -227,6 +227,11 @@ def test_prefill_visibility():
         assert C.prefill_visible(p) == brute
     assert C.prefill_visible(524288 - 8192) == 258048
     assert C.prefill_visible(524287) == 262144
+    # other compression ratios: entry e covers tokens m*e .. m*e+m-1
+    for m in (1, 3, 4):
+        for p in range(-2, 30):
+            brute = sum(1 for e in range(100) if all(t <= p for t in range(m * e, m * e + m)))
+            assert C.prefill_visible(p, m) == brute
 
 
 def test_prefill_topk_is_causal():

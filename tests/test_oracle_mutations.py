@@ -141,5 +141,5 @@ def test_mutation_attention_softmax_over_heads(monkeypatch):
 
 
 def test_mutation_prefill_off_by_one(monkeypatch):
-    monkeypatch.setattr(C, "prefill_visible", lambda p: p // 2)
+    monkeypatch.setattr(C, "prefill_visible", lambda p, m=2: max(0, p // m))
     _fails(PC.test_prefill_visibility)
