@@ -18,6 +18,11 @@ from pinned host memory and the outputs read back every step; `roofline`
 rates the dominant kernel (the Full scan) against the measured copy bandwidth;
 `cpu_baseline` times the float64 oracle on a bounded sample.
 `--impl reference` times that oracle as the reference arm.
+
+`--workload prefill_256k_q8192` measures the encoder-style causal prefill
+chunk instead (8,192 queries over 262,144 m=2 entries: the causal prefill
+indexer, then six attention layers over its Top-512); its line rates the
+indexer against the FP8 tensor-core peak.
 """
 from __future__ import annotations
 
@@ -391,6 +396,147 @@ def run_b200(args):
         dist.destroy_process_group()
 
 
+PREFILL_METRIC = "CSA2 causal prefill chunk queries/s (indexer + 6 attention layers); indexer FP8 TFLOP/s"
+
+
+def prefill_flops(wl):
+    """Algorithmic FP8 MMA FLOPs of the prefill indexer: 2 * 32 heads * 128 per
+    visible (query, entry) pair."""
+    vis = np.minimum((W.prefill_positions(wl).astype(np.int64) + 1) // W.prefill_ratio(wl), wl.ctx)
+    return 2.0 * 32 * 128 * float(vis.sum())
+
+
+def measured_peak_fp8():
+    """Dense FP8 tensor peak: the measured cuBLAS bf16 burst x 2 (the nominal
+    FP8 : BF16 ratio), else the fallback bf16 figure x 2."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return 2.0 * float(json.load(f)["bf16_tflops"]), "measured bf16 burst x 2 (nominal FP8/BF16 ratio)"
+    except (OSError, KeyError, ValueError):
+        return 2.0 * 1590.0, "fallback bf16 x 2 (nominal FP8/BF16 ratio)"
+
+
+def prefill_oracle_sample(wl, n_q: int = 2):
+    """Float64 oracle of n_q prefill queries (Top-512 over all visible entries
+    plus six attention layers each); returns seconds per query."""
+    from oracle import csa2 as C
+    from oracle import formats as F
+    codes, exp = F.quantize_indexer(W.request_rows(wl, 0, wl.ctx, "ik"))
+    q, w = W.index_query(wl, 0, rows=n_q)
+    pos = W.prefill_positions(wl)[:n_q]
+    qm = [W.main_query(wl, l, rows=n_q).float().numpy() for l in range(len(wl.modes))]
+    t0 = time.perf_counter()
+    for j in range(n_q):
+        t = C.prefill_topk(q[j], w[j], codes, exp, int(pos[j]), wl.topk, W.prefill_ratio(wl))
+        kvc, kvs = F.quantize_main_kv(W.rows_at(wl, 0, t, "kv"))
+        for layer in range(len(wl.modes)):
+            C.sparse_attention(qm[layer][j], kvc, kvs, np.arange(len(t)), wl.scale)
+    return (time.perf_counter() - t0) / n_q
+
+
+def run_prefill(args):
+    """The causal prefill chunk: per step, the prefill indexer (FP8 GEMM with
+    streaming Top-512) and six attention layers over its Top-512."""
+    import torch
+    rank, world, local = env_rank()
+    if world > 1:
+        raise SystemExit("the prefill measurement runs on one GPU")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    from kv_cache_decode_index_b200 import build as _build
+    _build.build()
+    from kv_cache_decode_index_b200 import csa2
+    from kv_cache_decode_index_b200.fill import build_cache
+
+    wl = selected_workload(args)
+    cache = build_cache(wl, csa2)
+    n = wl.prefill_queries
+    pos = torch.from_numpy(W.prefill_positions(wl)).to(dev)
+    q, w = W.index_query(wl, 0)
+    tq = [torch.from_numpy(q).to(dev)] + [None] * (len(wl.modes) - 1)
+    tw = [torch.from_numpy(w).to(dev)] + [None] * (len(wl.modes) - 1)
+    qm = [W.main_query(wl, l).to(dev) for l in range(len(wl.modes))]
+    out = [torch.empty_like(m) for m in qm]
+    group = csa2.PrefillGroup(cache, 0, wl.modes, wl.heads, n, wl.topk, W.prefill_ratio(wl), wl.scale)
+    for _ in range(args.warmup):
+        group.step(pos, tq, tw, qm, out)
+    torch.cuda.synchronize()
+    st, word = csa2.get_error(cache)
+    if st != csa2.OK:
+        raise RuntimeError(f"device error during warm-up: {word}")
+    gpu_id = str(torch.cuda.get_device_properties(dev).uuid)
+    sampler = ClockSampler(gpu_id if gpu_id.startswith("GPU-") else f"GPU-{gpu_id}")
+    sampler.start()
+    names = [f"topk{l}" for l, m in enumerate(wl.modes) if m != "Ru"] + [f"attn{l}" for l in range(len(wl.modes))]
+    timing = {k: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for k in names}
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    per_launch = {k: [] for k in names}
+    step_ms = []
+    for _ in range(args.steps):
+        torch.cuda.synchronize()
+        e0.record()
+        group.step(pos, tq, tw, qm, out, timing=timing)
+        e1.record()
+        torch.cuda.synchronize()
+        step_ms.append(e0.elapsed_time(e1))
+        for k, (a, b) in timing.items():
+            per_launch[k].append(a.elapsed_time(b))
+    clocks = sampler.stop()
+    st, word = csa2.get_error(cache)
+    if st != csa2.OK:
+        raise RuntimeError(f"device error during the timed run: {word}")
+    ms = statistics.mean(step_ms)
+    idx_ms = statistics.mean(per_launch["topk0"])
+    flops = prefill_flops(wl)
+    peak, peak_src = measured_peak_fp8()
+    achieved = flops / (idx_ms / 1e3) / 1e12
+    e2e_value = None
+    h2d = pos.numel() * 4 + q.nbytes + w.nbytes + sum(t.numel() * 2 for t in qm)
+    d2h = n * wl.topk * 4 + sum(t.numel() * 2 for t in out)
+    if not args.no_e2e:
+        hp, hq, hw = pos.cpu().pin_memory(), tq[0].cpu().pin_memory(), tw[0].cpu().pin_memory()
+        hm = [t.cpu().pin_memory() for t in qm]
+        ho = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in out]
+        hk = torch.empty(n, wl.topk, dtype=torch.int32, pin_memory=True)
+        torch.cuda.synchronize()
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a0.record()
+        for _ in range(args.steps):
+            pos.copy_(hp, non_blocking=True)
+            tq[0].copy_(hq, non_blocking=True)
+            tw[0].copy_(hw, non_blocking=True)
+            for dst, src in zip(qm, hm):
+                dst.copy_(src, non_blocking=True)
+            group.step(pos, tq, tw, qm, out)
+            hk.copy_(group.topk[0], non_blocking=True)
+            for dst, src in zip(ho, out):
+                dst.copy_(src, non_blocking=True)
+        a1.record()
+        torch.cuda.synchronize()
+        e2e_value = n / (a0.elapsed_time(a1) / args.steps / 1e3)
+    line = {"metric": PREFILL_METRIC, "value": n / (ms / 1e3), "unit": "queries/s", "n_gpus": 1, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "fp8", "data": "synthetic",
+            "config": {"workload": f"{wl.name}: {n} causal prefill queries over {wl.ctx:,} m={W.prefill_ratio(wl)} "
+                                   f"entries, 1 Full + {len(wl.modes) - 1} Reuse, Top-{wl.topk}, {wl.heads} heads d512",
+                       "parallelism": "single", "l2": "indexer K (34 MB) is L2-resident by design; main KV rows "
+                                                     "gathered per query"},
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                         "frac": achieved / peak, "traffic": None, "kernel": "csa2 prefill_index (FP8 GEMM + "
+                         "streaming Top-512)", "kernel_ms": idx_ms, "flops_per_launch": flops,
+                         "peak_source": peak_src},
+            "e2e": {"value": e2e_value, "unit": "queries/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": group.launches_per_step * args.steps,
+            "launch_ms": {k: statistics.mean(v) for k, v in per_launch.items()},
+            "clocks": clocks}
+    if not args.no_cpu_baseline:
+        spq = prefill_oracle_sample(wl)
+        line["cpu_baseline"] = {"value": 1.0 / spq, "unit": "queries/s", "cores": cpu_cores(), "kind": "oracle",
+                                "sample": f"2 of the {n} queries: float64 oracle Top-512 over all visible entries "
+                                          f"and six attention layers, {spq:.1f} s per query"}
+    print(json.dumps(line), flush=True)
+
+
 def max_over_ranks(x: float, dev, world: int) -> float:
     """Max of a per-rank timing over all ranks (NCCL on GPUs, gloo on CPU)."""
     if world == 1:
@@ -418,6 +564,18 @@ def run_reference(args):
     if rank != 0:
         return
     wl = selected_workload(args)
+    if wl.prefill_queries:
+        times = [prefill_oracle_sample(wl, 1) for _ in range(args.steps)]
+        ms = 1e3 * sum(times) / len(times)
+        line = {"metric": PREFILL_METRIC, "value": 1e3 / ms, "unit": "queries/s", "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+                "config": {"workload": wl.name},
+                "cpu_baseline": {"value": 1e3 / ms, "unit": "queries/s", "cores": cpu_cores(), "kind": "oracle",
+                                 "sample": "one prefill query per step, float64 oracle"},
+                "e2e": {"value": 1e3 / ms, "unit": "queries/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return
     prepared = {}
     times = []
     for it in range(args.warmup + args.steps):
@@ -467,6 +625,8 @@ def main(argv=None):
         p.error("--warmup must be >= 3")
     if args.impl == "reference":
         run_reference(args)
+    elif W.WORKLOADS[args.workload].prefill_queries:
+        run_prefill(args)
     else:
         run_b200(args)
 

@@ -205,6 +205,46 @@ CSA2_API csa2_status csa2_sparse_attn(const csa2_cache* cache, int32_t n_queries
                              float scale, uint16_t* out, void* stream);
 
 /*
+ * csa2_prefill_index -- causal prefill indexer: for each of n_queries queries
+ * of request `req`, the Top-k visible entries by the score of
+ * csa2_index_full, with no pool.  This is the indexer of the pages' encoder
+ * group (1 Full + 5 Reuse layers over a sequence compressed m = 2, two tokens
+ * per cached entry) [4sapi blog, section 三; Top-512 and indexer shape, section
+ * 四].  Causal rule (a reading; the pages state none): entry e covers tokens
+ * ratio*e .. ratio*e + ratio - 1 and is visible to the query at token p iff
+ * ratio*e + ratio - 1 <= p, i.e. e < floor((p + 1) / ratio); entries at or past
+ * ctx_len[req] are never visible.
+ *   req        request holding the entries, 0 <= req < batch
+ *   n_queries  queries in this call (>= 0; 0 does nothing)
+ *   q_pos      int32 [n_queries] token position of each query (negative: sees
+ *              nothing)
+ *   ratio      tokens per entry, >= 1
+ *   q          float [n_queries][32][128] indexer queries (FP8 rule inside)
+ *   w          float [n_queries][32]      head weights
+ *   k          Top-k per query, in [1, CSA2_PREFILL_MAX_K]
+ *   topk       int32 [n_queries][k] out: entries ascending, -1 padded
+ *   workspace  device scratch of at least csa2_prefill_workspace_bytes(
+ *              n_queries) bytes, 16-byte aligned, owned by the caller; its
+ *              contents on entry do not matter and are undefined after.  Two
+ *              calls in flight at once must not share it.
+ *   workspace_bytes  its size
+ * The scores are an FP8 tensor-core GEMM (n_queries*32 x 128 by 128 x
+ * entries) reduced over the heads in fp32; each query keeps a list of at most
+ * CSA2_PREFILL_CANDIDATES candidates in the workspace, so the score matrix is
+ * never stored.  Ties go to the lower entry, as everywhere.  Launches two
+ * kernels.  Device errors: a page id outside [0, num_pages) ->
+ * CSA2_ERR_DEVICE_BOUNDS (outputs undefined); a pipeline wait that runs out
+ * -> CSA2_ERR_TIMEOUT (see csa2_set_wait_limit_ns).
+ */
+#define CSA2_PREFILL_MAX_K 1024
+#define CSA2_PREFILL_CANDIDATES 4096
+CSA2_API size_t csa2_prefill_workspace_bytes(int32_t n_queries);
+CSA2_API csa2_status csa2_prefill_index(const csa2_cache* cache, int32_t req, int32_t n_queries,
+                                        const int32_t* q_pos, int32_t ratio, const float* q, const float* w,
+                                        int32_t k, int32_t* topk, void* workspace, size_t workspace_bytes,
+                                        void* stream);
+
+/*
  * csa2_get_error -- synchronise `stream`, copy cache->err_word to the host
  * array out[4] (host pointer) and return out[0] as a status (CSA2_OK when no
  * device error was recorded).  Does not clear the word.
@@ -213,8 +253,8 @@ CSA2_API csa2_status csa2_get_error(const csa2_cache* cache, int32_t* out, void*
 
 /*
  * csa2_set_wait_limit_ns -- process-wide bound, in nanoseconds, on every
- * pipeline wait inside the tensor-core kernels (csa2_index_full and the
- * re-scoring csa2_reindex); default 2e9.  A wait that runs out makes the
+ * pipeline wait inside the tensor-core kernels (csa2_index_full, the
+ * re-scoring csa2_reindex and csa2_prefill_index); default 2e9.  A wait that runs out makes the
  * kernel record CSA2_ERR_TIMEOUT in err_word, wait (with a fixed bound) for its
  * own copies in flight, free its tensor memory and return; the call's outputs
  * are then undefined.  0 gives up on the first wait that is not already

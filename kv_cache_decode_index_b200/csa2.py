@@ -23,6 +23,7 @@ FULL, REINDEX, REUSE = 0, 1, 2
 MODE = {"F": FULL, "Ri": REINDEX, "Ru": REUSE}
 OK, ERR_ARG, ERR_SHAPE, ERR_CUDA, ERR_DEVICE_BOUNDS, ERR_TIMEOUT, ERR_UNSUPPORTED = range(7)
 BLOCK, INDEX_HEADS, INDEX_DIM, KV_DIM, KV_CODE_BYTES, KV_SCALE_BYTES = 8, 32, 128, 512, 256, 32
+PREFILL_MAX_K, PREFILL_CANDIDATES = 1024, 4096
 
 
 class CacheStruct(ctypes.Structure):
@@ -41,6 +42,7 @@ _sig = {
     "csa2_pool_select": [_CP, _P, _I, _P, _P],
     "csa2_reindex": [_CP, _I, _P, _I, _P, _P, _P, _P, _I, _P, _P],
     "csa2_sparse_attn": [_CP, _I, _P, _P, _I, _P, _I, ctypes.c_float, _P, _P],
+    "csa2_prefill_index": [_CP, _I, _I, _P, _I, _P, _P, _I, _P, _P, ctypes.c_size_t, _P],
     "csa2_get_error": [_CP, ctypes.POINTER(ctypes.c_int32), _P],
 }
 for _name, _args in _sig.items():
@@ -50,6 +52,8 @@ _lib.csa2_status_string.argtypes = [ctypes.c_int]
 _lib.csa2_status_string.restype = ctypes.c_char_p
 _lib.csa2_last_error_message.argtypes = []
 _lib.csa2_last_error_message.restype = ctypes.c_char_p
+_lib.csa2_prefill_workspace_bytes.argtypes = [_I]
+_lib.csa2_prefill_workspace_bytes.restype = ctypes.c_size_t
 _lib.csa2_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
 _lib.csa2_set_wait_limit_ns.restype = None
 
@@ -203,6 +207,31 @@ def sparse_attn(cache: Cache, topk, q, scale: float | None = None, out=None, q_r
     return out
 
 
+def prefill_workspace_bytes(n_queries: int) -> int:
+    return int(_lib.csa2_prefill_workspace_bytes(int(n_queries)))
+
+
+def prefill_index(cache: Cache, req: int, q_pos, q, w, k: int = 512, ratio: int = 2, topk=None, workspace=None):
+    """Causal prefill Top-k of n queries of request `req`: q_pos int32 [n]
+    (token positions), q float32 [n,32,128], w float32 [n,32]; returns topk
+    int32 [n, k] (entries ascending, -1 padded)."""
+    n = q_pos.shape[0]
+    _need(q_pos, torch.int32, (n,), "q_pos")
+    _need(q, torch.float32, (n, INDEX_HEADS, INDEX_DIM), "q")
+    _need(w, torch.float32, (n, INDEX_HEADS), "w")
+    if topk is None:
+        topk = torch.empty(n, k, dtype=torch.int32, device=cache.device)
+    _need(topk, torch.int32, (n, k), "topk")
+    if workspace is None:
+        workspace = torch.empty(max(prefill_workspace_bytes(n), 16), dtype=torch.uint8, device=cache.device)
+    if workspace.dtype != torch.uint8 or not workspace.is_contiguous() or workspace.device.type != "cuda":
+        raise ValueError("workspace: expected a contiguous cuda uint8 tensor")
+    _check(_lib.csa2_prefill_index(ctypes.byref(cache.struct), int(req), n, _ptr(q_pos), int(ratio), _ptr(q), _ptr(w),
+                                   int(k), _ptr(topk), _ptr(workspace), workspace.numel(), _stream(cache.device)),
+           "csa2_prefill_index")
+    return topk
+
+
 def get_error(cache: Cache):
     """Synchronise the current stream and return (status, err_word list)."""
     out = (ctypes.c_int32 * 4)()
@@ -302,3 +331,49 @@ class DecodeGroup:
                 names.append(f"topk{layer}")
             names.append(f"attn{layer}")
         return names
+
+
+class PrefillGroup:
+    """One encoder-style prefill chunk of a CSA2 layer group over request
+    `req` of `cache`: every Full (or Reindex) layer runs the causal prefill
+    indexer with its own query, Reuse layers take the previous layer's Top-k,
+    and every layer attends with its own main query (H heads of 512)."""
+
+    def __init__(self, cache: Cache, req: int, modes, heads: int, n_queries: int, k: int = 512, ratio: int = 2,
+                 scale: float | None = None):
+        if modes[0] == "Ru":
+            raise ValueError("a layer group starts with a Full layer")
+        self.cache, self.req, self.modes, self.heads, self.k, self.ratio = cache, req, tuple(modes), heads, k, ratio
+        self.scale = 1.0 / math.sqrt(KV_DIM) if scale is None else scale
+        dev = cache.device
+        self.n = n_queries
+        self.workspace = torch.empty(max(prefill_workspace_bytes(n_queries), 16), dtype=torch.uint8, device=dev)
+        self.q_req = torch.full((n_queries,), req, dtype=torch.int32, device=dev)
+        self.topk, src = [], None
+        for m in self.modes:
+            if m != "Ru":
+                src = torch.empty(n_queries, k, dtype=torch.int32, device=dev)
+            self.topk.append(src)
+        self.launches_per_step = sum(2 for m in self.modes if m != "Ru") + len(self.modes)
+
+    def step(self, q_pos, q_idx, w_idx, q_main, out, timing=None):
+        """q_pos int32 [n]; q_idx / w_idx per layer (None for Reuse); q_main /
+        out per layer bf16 [n, H, 512].  timing: optional dict name -> (start,
+        end) CUDA events around "topk<l>" and "attn<l>"."""
+        c = self.cache
+
+        def timed(name, fn):
+            ev = None if timing is None else timing.get(name)
+            if ev is not None:
+                ev[0].record()
+            fn()
+            if ev is not None:
+                ev[1].record()
+
+        for layer, m in enumerate(self.modes):
+            if m != "Ru":
+                timed(f"topk{layer}", lambda: prefill_index(c, self.req, q_pos, q_idx[layer], w_idx[layer], self.k,
+                                                            self.ratio, self.topk[layer], self.workspace))
+            timed(f"attn{layer}", lambda: sparse_attn(c, self.topk[layer], q_main[layer], self.scale, out[layer],
+                                                      q_req=self.q_req))
+        return out

@@ -21,7 +21,7 @@ constexpr int kBlock = CSA2_BLOCK;              // positions per pool block
 constexpr int kTile = 128;                      // positions per MMA tile (M)
 
 // kernel ids recorded in err_word[1]
-enum KernelId { kKAppend = 1, kKIndexFull = 2, kKPoolSelect = 3, kKReindex = 4, kKAttn = 5 };
+enum KernelId { kKAppend = 1, kKIndexFull = 2, kKPoolSelect = 3, kKReindex = 4, kKAttn = 5, kKPrefill = 6 };
 
 // Wait bound of the pipeline barriers (ns of %globaltimer).  Well above any
 // legitimate wait; a wait that runs out records CSA2_ERR_TIMEOUT and the CTA
@@ -106,6 +106,26 @@ __device__ __forceinline__ bool warp_flag(const volatile int* flag) {
   return __shfl_sync(0xffffffffu, v, 0) != 0;
 }
 
+// ------------------------------------------------------- named barriers ----
+// bar.sync on barrier `id` (1..15) for `count` threads (a multiple of 32).
+__device__ __forceinline__ void named_bar_sync(int id, int count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+// The same barrier, returning to every participant whether any of them passed
+// a true predicate.
+__device__ __forceinline__ bool named_bar_or(int id, int count, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.or.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"(pred ? 1u : 0u), "r"(id), "r"(count)
+      : "memory");
+  return r != 0;
+}
+
 // ------------------------------------------------------------------ TMA ----
 __device__ __forceinline__ void tma_prefetch_map(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(map) : "memory");
@@ -133,6 +153,11 @@ __device__ __forceinline__ void bulk_load_1d(void* dst, const void* src, uint32_
 __device__ __forceinline__ uint64_t l2_policy_evict_first() {
   uint64_t p;
   asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+__device__ __forceinline__ uint64_t l2_policy_evict_last() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
   return p;
 }
 __device__ __forceinline__ uint64_t l2_policy_evict_normal() {

@@ -34,6 +34,7 @@ constexpr int kMaxK = 4096;
 constexpr int kMaxPool = 4096;
 constexpr long long kMaxFlatPositions = 65536;        // Top-k without a pool
 constexpr long long kMaxPoolSelectBlocks = 16LL * 16384;
+constexpr int kMaxPrefillQueries = 1 << 20;
 
 uint64_t g_wait_limit_ns = csa2::kWaitLimitNs;
 
@@ -231,6 +232,34 @@ csa2_status csa2_sparse_attn(const csa2_cache* cache, int32_t n_queries, const i
   const cudaError_t e = csa2::launch_sparse_attn(*cache, n_queries, q_req, topk, k, q, H, scale, out,
                                                  static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? CSA2_OK : cuda_fail(e, "sparse_attn launch");
+}
+
+size_t csa2_prefill_workspace_bytes(int32_t n_queries) { return csa2::prefill_workspace_bytes(n_queries); }
+
+csa2_status csa2_prefill_index(const csa2_cache* cache, int32_t req, int32_t n_queries, const int32_t* q_pos,
+                               int32_t ratio, const float* q, const float* w, int32_t k, int32_t* topk,
+                               void* workspace, size_t workspace_bytes, void* stream) {
+  CSA2_TRY(check_cache(cache, false, true));
+  if (req < 0 || req >= cache->batch) return fail(CSA2_ERR_SHAPE, "req %d outside [0, %d)", req, cache->batch);
+  if (n_queries < 0 || n_queries > kMaxPrefillQueries)
+    return fail(CSA2_ERR_SHAPE, "n_queries %d outside [0, %d]", n_queries, kMaxPrefillQueries);
+  if (n_queries == 0) return CSA2_OK;
+  if (ratio < 1) return fail(CSA2_ERR_SHAPE, "ratio %d < 1", ratio);
+  if (k < 1 || k > CSA2_PREFILL_MAX_K) return fail(CSA2_ERR_SHAPE, "k %d outside [1, %d]", k, CSA2_PREFILL_MAX_K);
+  if (q_pos == nullptr || q == nullptr || w == nullptr || topk == nullptr || !aligned(q, 16))
+    return fail(CSA2_ERR_ARG, "q_pos, q (16-byte aligned), w and topk must be set");
+  if (workspace == nullptr || !aligned(workspace, 16))
+    return fail(CSA2_ERR_ARG, "workspace must be set and 16-byte aligned");
+  if (workspace_bytes < csa2::prefill_workspace_bytes(n_queries))
+    return fail(CSA2_ERR_SHAPE, "workspace of %zu bytes, %zu needed", workspace_bytes,
+                csa2::prefill_workspace_bytes(n_queries));
+  DeviceInfo d;
+  CSA2_TRY(device_info(&d));
+  CUtensorMap map;
+  CSA2_TRY(encode_ik_map(cache, csa2::kTile, &map));
+  const cudaError_t e = csa2::launch_prefill_index(*cache, req, n_queries, q_pos, ratio, q, w, k, topk, workspace,
+                                                   map, g_wait_limit_ns, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? CSA2_OK : cuda_fail(e, "prefill_index launch");
 }
 
 csa2_status csa2_get_error(const csa2_cache* cache, int32_t* out, void* stream) {

@@ -27,6 +27,11 @@ cudaError_t launch_reindex(const csa2_cache& cache, const int32_t* pool, int poo
                            const float* w, const float* full_scores, int k, int32_t* topk,
                            const CUtensorMap& ik_blk_map, int cands_per_cta, uint64_t wait_ns, cudaStream_t stream);
 
+size_t prefill_workspace_bytes(long long n_queries);
+cudaError_t launch_prefill_index(const csa2_cache& cache, int req, int n_queries, const int32_t* q_pos, int ratio,
+                                 const float* q, const float* w, int k, int32_t* topk, void* workspace,
+                                 const CUtensorMap& ik_map, uint64_t wait_ns, cudaStream_t stream);
+
 cudaError_t launch_copy_topk(const int32_t* src, int32_t* dst, long long n, cudaStream_t stream);
 
 cudaError_t launch_sparse_attn(const csa2_cache& cache, int n_queries, const int32_t* q_req, const int32_t* topk,

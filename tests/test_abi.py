@@ -25,7 +25,7 @@ def declared_symbols():
 
 def test_every_declared_symbol_is_exported(lib):
     names = declared_symbols()
-    assert len(names) == 9, names
+    assert len(names) == 11, names
     so = ctypes.CDLL(lib.LIB_PATH)
     for n in names:
         assert hasattr(so, n), f"{n} missing from libcsa2.so"
@@ -65,6 +65,18 @@ def test_host_side_validation(lib):
     big, _ = _cache(lib, max_pages_per_req=2048, page_size=4096)
     assert L.csa2_reindex(ctypes.byref(big), lib.FULL, None, 0, P, P, None, None, 512, P, None) == lib.ERR_SHAPE
     assert L.csa2_status_string(lib.ERR_TIMEOUT) == b"a pipeline wait on the device gave up"
+    # prefill: req, k, ratio, workspace size and alignment are checked on the host
+    need = L.csa2_prefill_workspace_bytes(8)
+    assert need == 8 * 4096 * 8 + 32 and L.csa2_prefill_workspace_bytes(0) == 0
+    pf = L.csa2_prefill_index
+    assert pf(ctypes.byref(c), 2, 8, P, 2, P, P, 512, P, P, need, None) == lib.ERR_SHAPE      # req >= batch
+    assert pf(ctypes.byref(c), 0, 8, P, 2, P, P, 1025, P, P, need, None) == lib.ERR_SHAPE     # k > 1024
+    assert pf(ctypes.byref(c), 0, 8, P, 0, P, P, 512, P, P, need, None) == lib.ERR_SHAPE      # ratio < 1
+    assert pf(ctypes.byref(c), 0, 8, P, 2, P, P, 512, P, P, need - 16, None) == lib.ERR_SHAPE
+    assert b"needed" in L.csa2_last_error_message()
+    assert pf(ctypes.byref(c), 0, 8, P, 2, P, P, 512, P, ctypes.c_void_p(p + 8), need, None) == lib.ERR_ARG
+    assert pf(ctypes.byref(c), 0, 8, None, 2, P, P, 512, P, P, need, None) == lib.ERR_ARG
+    assert pf(ctypes.byref(c), 0, 0, None, 2, None, None, 512, None, None, 0, None) == lib.OK   # nothing to do
 
 
 def test_binding_rejects_wrong_tensors(lib):

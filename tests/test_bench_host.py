@@ -99,3 +99,11 @@ def test_reference_arm_other_ranks_do_nothing(monkeypatch):
     with redirect_stdout(buf):
         bench.main(["--impl", "reference", "--workload", "full_4k_b1", "--steps", "2", "--warmup", "3"])
     assert buf.getvalue() == ""
+
+
+def test_prefill_flops_closed_form():
+    # queries at tokens 516096 + j (j < 8192) see 258048 + floor((j + 1) / 2)
+    # m=2 entries: sum = 8192 * 258048 + 4096 * 4096
+    import bench
+    wl = W.WORKLOADS["prefill_256k_q8192"]
+    assert bench.prefill_flops(wl) == 2 * 32 * 128 * (8192 * 258048 + 4096 * 4096)
