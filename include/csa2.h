@@ -245,6 +245,26 @@ CSA2_API csa2_status csa2_prefill_index(const csa2_cache* cache, int32_t req, in
                                         void* stream);
 
 /*
+ * csa2_prefill_index_static -- csa2_prefill_index without a workspace
+ * argument.  The pages have no counterpart: this entry point exists for
+ * callers that cannot hand the library scratch memory.  The candidate lists
+ * live in a file-scope static device array of the library sized for
+ * CSA2_PREFILL_STATIC_MAX_QUERIES queries (about 8.4 MB per device); a call
+ * with more queries returns CSA2_ERR_SHAPE and launches nothing.  Nothing in
+ * the array needs to start at zero (every list length is written before it is
+ * read).  The array's device address is looked up with cudaGetSymbolAddress
+ * on the first call on each device, so make that first call outside any
+ * stream capture.  Every call on a device uses the same array: two calls in
+ * flight at once on one device (other streams, other host threads) race and
+ * corrupt each other's results; serialise them.  Arguments, outputs and
+ * device errors are those of csa2_prefill_index.
+ */
+#define CSA2_PREFILL_STATIC_MAX_QUERIES 256
+CSA2_API csa2_status csa2_prefill_index_static(const csa2_cache* cache, int32_t req, int32_t n_queries,
+                                               const int32_t* q_pos, int32_t ratio, const float* q,
+                                               const float* w, int32_t k, int32_t* topk, void* stream);
+
+/*
  * csa2_get_error -- synchronise `stream`, copy cache->err_word to the host
  * array out[4] (host pointer) and return out[0] as a status (CSA2_OK when no
  * device error was recorded).  Does not clear the word.

@@ -23,7 +23,7 @@ FULL, REINDEX, REUSE = 0, 1, 2
 MODE = {"F": FULL, "Ri": REINDEX, "Ru": REUSE}
 OK, ERR_ARG, ERR_SHAPE, ERR_CUDA, ERR_DEVICE_BOUNDS, ERR_TIMEOUT, ERR_UNSUPPORTED = range(7)
 BLOCK, INDEX_HEADS, INDEX_DIM, KV_DIM, KV_CODE_BYTES, KV_SCALE_BYTES = 8, 32, 128, 512, 256, 32
-PREFILL_MAX_K, PREFILL_CANDIDATES = 1024, 4096
+PREFILL_MAX_K, PREFILL_CANDIDATES, PREFILL_STATIC_MAX_QUERIES = 1024, 4096, 256
 
 
 class CacheStruct(ctypes.Structure):
@@ -43,6 +43,7 @@ _sig = {
     "csa2_reindex": [_CP, _I, _P, _I, _P, _P, _P, _P, _I, _P, _P],
     "csa2_sparse_attn": [_CP, _I, _P, _P, _I, _P, _I, ctypes.c_float, _P, _P],
     "csa2_prefill_index": [_CP, _I, _I, _P, _I, _P, _P, _I, _P, _P, ctypes.c_size_t, _P],
+    "csa2_prefill_index_static": [_CP, _I, _I, _P, _I, _P, _P, _I, _P, _P],
     "csa2_get_error": [_CP, ctypes.POINTER(ctypes.c_int32), _P],
 }
 for _name, _args in _sig.items():
@@ -229,6 +230,23 @@ def prefill_index(cache: Cache, req: int, q_pos, q, w, k: int = 512, ratio: int 
     _check(_lib.csa2_prefill_index(ctypes.byref(cache.struct), int(req), n, _ptr(q_pos), int(ratio), _ptr(q), _ptr(w),
                                    int(k), _ptr(topk), _ptr(workspace), workspace.numel(), _stream(cache.device)),
            "csa2_prefill_index")
+    return topk
+
+
+def prefill_index_static(cache: Cache, req: int, q_pos, q, w, k: int = 512, ratio: int = 2, topk=None):
+    """csa2_prefill_index_static: prefill_index with the library's static
+    scratch instead of a workspace (at most 256 queries per call; calls on one
+    device must not overlap)."""
+    n = q_pos.shape[0]
+    _need(q_pos, torch.int32, (n,), "q_pos")
+    _need(q, torch.float32, (n, INDEX_HEADS, INDEX_DIM), "q")
+    _need(w, torch.float32, (n, INDEX_HEADS), "w")
+    if topk is None:
+        topk = torch.empty(n, k, dtype=torch.int32, device=cache.device)
+    _need(topk, torch.int32, (n, k), "topk")
+    _check(_lib.csa2_prefill_index_static(ctypes.byref(cache.struct), int(req), n, _ptr(q_pos), int(ratio), _ptr(q),
+                                          _ptr(w), int(k), _ptr(topk), _stream(cache.device)),
+           "csa2_prefill_index_static")
     return topk
 
 

@@ -262,6 +262,29 @@ csa2_status csa2_prefill_index(const csa2_cache* cache, int32_t req, int32_t n_q
   return e == cudaSuccess ? CSA2_OK : cuda_fail(e, "prefill_index launch");
 }
 
+csa2_status csa2_prefill_index_static(const csa2_cache* cache, int32_t req, int32_t n_queries,
+                                      const int32_t* q_pos, int32_t ratio, const float* q, const float* w,
+                                      int32_t k, int32_t* topk, void* stream) {
+  if (n_queries > CSA2_PREFILL_STATIC_MAX_QUERIES)
+    return fail(CSA2_ERR_SHAPE, "n_queries %d above the static scratch limit of %d", n_queries,
+                CSA2_PREFILL_STATIC_MAX_QUERIES);
+  if (n_queries <= 0) return csa2_prefill_index(cache, req, n_queries, q_pos, ratio, q, w, k, topk, nullptr, 0, stream);
+  // the host-side checks of csa2_prefill_index, before the device is touched
+  CSA2_TRY(check_cache(cache, false, true));
+  if (req < 0 || req >= cache->batch) return fail(CSA2_ERR_SHAPE, "req %d outside [0, %d)", req, cache->batch);
+  if (ratio < 1) return fail(CSA2_ERR_SHAPE, "ratio %d < 1", ratio);
+  if (k < 1 || k > CSA2_PREFILL_MAX_K) return fail(CSA2_ERR_SHAPE, "k %d outside [1, %d]", k, CSA2_PREFILL_MAX_K);
+  if (q_pos == nullptr || q == nullptr || w == nullptr || topk == nullptr || !aligned(q, 16))
+    return fail(CSA2_ERR_ARG, "q_pos, q (16-byte aligned), w and topk must be set");
+  DeviceInfo d;
+  CSA2_TRY(device_info(&d));
+  void* scratch = nullptr;
+  const cudaError_t e = csa2::static_prefill_scratch(&scratch);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(prefill scratch)");
+  return csa2_prefill_index(cache, req, n_queries, q_pos, ratio, q, w, k, topk, scratch,
+                            csa2::prefill_workspace_bytes(n_queries), stream);
+}
+
 csa2_status csa2_get_error(const csa2_cache* cache, int32_t* out, void* stream) {
   if (cache == nullptr || cache->err_word == nullptr || out == nullptr)
     return fail(CSA2_ERR_ARG, "cache, cache.err_word and out must be set");

@@ -32,6 +32,8 @@
 // CSA2_ERR_TIMEOUT and every role leaves its loop (the epilogue warps leave
 // together, decided at their per-tile barrier), drains, frees TMEM and
 // returns.
+#include <mutex>
+
 #include "index_common.cuh"
 #include "launch.h"
 #include "warp_select.cuh"
@@ -440,6 +442,33 @@ cudaError_t launch_prefill_index(const csa2_cache& cache, int req, int n_queries
   const int sgrid = (n_queries + kSelWarps - 1) / kSelWarps;
   prefill_select_kernel<<<sgrid, kSelWarps * 32, 0, stream>>>(n_queries, k, wsp, topk);
   return cudaGetLastError();
+}
+
+// ------------------------------------------------- static-scratch variant ----
+// Candidate lists of csa2_prefill_index_static: a file-scope device array
+// sized for kStaticPrefillMaxQueries queries, so the call needs no
+// caller-provided workspace.  Every call on a device uses the same array.
+namespace {
+constexpr long long kStaticPrefillBytes =
+    static_cast<long long>(kStaticPrefillMaxQueries) * kCand * 8 + kStaticPrefillMaxQueries * 4;
+__device__ __align__(256) uint8_t g_prefill_scratch[kStaticPrefillBytes];
+
+std::mutex g_scratch_mu;
+void* g_scratch_addr[64] = {};
+}  // namespace
+
+cudaError_t static_prefill_scratch(void** addr) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lk(g_scratch_mu);
+  if (g_scratch_addr[dev] == nullptr) {
+    e = cudaGetSymbolAddress(&g_scratch_addr[dev], g_prefill_scratch);
+    if (e != cudaSuccess) return e;
+  }
+  *addr = g_scratch_addr[dev];
+  return cudaSuccess;
 }
 
 }  // namespace csa2

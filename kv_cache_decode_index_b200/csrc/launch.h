@@ -28,6 +28,10 @@ cudaError_t launch_reindex(const csa2_cache& cache, const int32_t* pool, int poo
                            const CUtensorMap& ik_blk_map, int cands_per_cta, uint64_t wait_ns, cudaStream_t stream);
 
 size_t prefill_workspace_bytes(long long n_queries);
+constexpr int kStaticPrefillMaxQueries = CSA2_PREFILL_STATIC_MAX_QUERIES;
+// Device address (current device) of the static candidate-list array of
+// csa2_prefill_index_static; looked up once per device.
+cudaError_t static_prefill_scratch(void** addr);
 cudaError_t launch_prefill_index(const csa2_cache& cache, int req, int n_queries, const int32_t* q_pos, int ratio,
                                  const float* q, const float* w, int k, int32_t* topk, void* workspace,
                                  const CUtensorMap& ik_map, uint64_t wait_ns, cudaStream_t stream);
