@@ -288,7 +288,9 @@ class DecodeGroup:
                 self.topk.append(src)
         self.concurrent = concurrent
         n_side = sum(1 for m in self.modes if m != "Ru")
-        self.streams = [torch.cuda.Stream(dev) for _ in range(n_side)] if concurrent else []
+        # one stream per layer: every layer's Top-k waits for the pool only,
+        # and a Reuse layer's attention waits for its source's Top-k only
+        self.streams = [torch.cuda.Stream(dev) for _ in self.modes] if concurrent else []
         self.launches_per_step = 1 + (1 if pool_blocks else 0) + n_side + len(self.modes)
 
     def step(self, q_idx, w_idx, q_main, out, timing=None):
@@ -311,27 +313,27 @@ class DecodeGroup:
         if self.pool is not None:
             timed("pool", lambda: pool_select(c, self.blockmax, self.pool_blocks, self.pool))
         main = torch.cuda.current_stream(c.device)
-        side = 0
         ev_ready = torch.cuda.Event()
         ev_ready.record(main)
-        src_stream = main
+        ev_topk = {}
+        src = 0
         for layer, m in enumerate(self.modes):
-            if m != "Ru":
-                s = self.streams[side] if self.concurrent else main
-                side += 1
-                with torch.cuda.stream(s):
+            s = self.streams[layer] if self.concurrent else main
+            with torch.cuda.stream(s):
+                if m != "Ru":
                     if s is not main:
                         s.wait_event(ev_ready)
                     mode = FULL if m == "F" else REINDEX
                     timed(f"topk{layer}", lambda: reindex(c, mode, self.k, self.pool, q_idx[layer], w_idx[layer],
                                                           topk=self.topk[layer]))
-                    timed(f"attn{layer}", lambda: sparse_attn(c, self.topk[layer], q_main[layer], self.scale,
-                                                              out[layer]))
-                src_stream = s
-            else:
-                with torch.cuda.stream(src_stream):
-                    timed(f"attn{layer}", lambda: sparse_attn(c, self.topk[layer], q_main[layer], self.scale,
-                                                              out[layer]))
+                    src = layer
+                    if self.concurrent:
+                        ev_topk[layer] = torch.cuda.Event()
+                        ev_topk[layer].record(s)
+                elif s is not main:
+                    s.wait_event(ev_topk[src])
+                timed(f"attn{layer}", lambda: sparse_attn(c, self.topk[layer], q_main[layer], self.scale,
+                                                          out[layer]))
         if self.concurrent:
             joins = []
             for s in self.streams:

@@ -17,15 +17,15 @@
 //     with an L2 evict_last hint (every CTA reads the same keys);
 //   * warp 1 (one lane): tcgen05.mma kind::f8f6f4, M = 128 entries, N = 256,
 //     K = 128 in 4 steps, into one of two 256-column TMEM accumulators;
-//   * warps 2..9: epilogue.  Warp e reads TMEM lane quarter (warp % 4) for the
-//     four queries 4*(e/4) .. 4*(e/4)+3: 32 fp32 head dot products per (entry,
-//     query), all 128 columns loaded before the accumulator is handed back ->
+//   * warps 2..17: epilogue.  Warp e reads TMEM lane quarter (warp % 4) for
+//     the two queries 2*(e/4), 2*(e/4)+1: 32 fp32 head dot products per (entry,
+//     query), all 64 columns loaded before the accumulator is handed back ->
 //     score (ReLU split between the min/max and FMA units, packed fp32 FMA) ->
 //     filter against the query's running threshold theta.  Survivors are
 //     appended to the query's candidate list in the caller's workspace.  When
-//     any list nears its capacity, every warp compacts the list of the query
-//     it owns to the exact k best (warp radix select) and raises its theta, all
-//     at the same tile.  Entries arrive in increasing order, so an entry whose
+//     any list nears its capacity, epilogue warp j compacts the list of query
+//     j to the exact k best (warp radix select) and raises its theta, all at
+//     the same tile.  Entries arrive in increasing order, so an entry whose
 //     key does not exceed theta can never enter the Top-k.
 // A second kernel reduces every list to the exact Top-k, sorted ascending.
 // Every mbarrier wait is bounded; a wait that runs out records
@@ -47,8 +47,9 @@ constexpr int kPN = kPQ * kIndexHeads;                 // 256: MMA N
 constexpr int kPStages = 6;
 constexpr int kPExp = 8;                               // exponent-byte ring (slots of 128 B)
 constexpr int kPAcc = 2;                               // accumulators of kPN columns
-constexpr int kPEpiWarps = 8;
-constexpr int kPThreads = 64 + kPEpiWarps * 32;        // 320
+constexpr int kQPW = 2;                                // queries per epilogue warp and tile
+constexpr int kPEpiWarps = 4 * kPQ / kQPW;             // 16: four TMEM lane quarters per query group
+constexpr int kPThreads = 64 + kPEpiWarps * 32;        // 576
 constexpr uint32_t kPTmemCols = kPAcc * kPN;           // 512
 constexpr uint32_t kPIdesc = idesc_e4m3_f32(kTile, kPN);
 constexpr int kCand = CSA2_PREFILL_CANDIDATES;         // list capacity per query
@@ -63,7 +64,7 @@ struct __align__(1024) PrefillSmem {
   uint8_t q[kPN * kIndexDim];          // B operand: row 32*j + h = head h of query j
   uint8_t exps[kPExp][kTile];          // exponent bytes of the tiles in flight
   float ws[kPQ][kIndexHeads];          // w_h * sigma^q_h
-  uint32_t hist[kPEpiWarps][256];      // radix histograms of the compactions
+  uint32_t hist[kPQ][256];             // radix histograms of the compactions
   int vis[kPQ];                        // visible entries of each query
   int cnt[kPQ];                        // list lengths
   uint32_t theta[kPQ];                 // admission thresholds (order keys)
@@ -226,22 +227,27 @@ __global__ void __launch_bounds__(kPThreads, 1)
   } else {
     // ================= epilogue (warps 2..9) =================
     const int e = warp - 2;
-    const int half = e >> 2;
-    const int own = half * 4 + (e & 3);        // the query whose list this warp compacts
+    const int grp = e >> 2;                    // queries kQPW*grp .. kQPW*grp + kQPW - 1
+    const int own = e;                         // the query whose list this warp compacts (e < kPQ)
     const int quarter = warp & 3;              // TMEM lane quarter
     const int toff = quarter * 32 + lane;      // entry inside the tile
 
-    // This warp's query codes -> B operand rows 32*own .. 32*own + 31.
+    // Query codes -> B operand rows 32*j + h; each warp quantises
+    // 4*kPQ/kPEpiWarps groups of 8 heads.
     {
-      const int j = j0 + own;
-      uint8_t* qt = S.q + own * kIndexHeads * kIndexDim;
-      if (j < n_queries) {
-        for (int ew = 0; ew < 4; ++ew)
-          prepare_query_part(q + static_cast<long long>(j) * kIndexHeads * kIndexDim, w + static_cast<long long>(j) * kIndexHeads,
-                             qt, S.ws[own], ew, lane);
-      } else {
-        for (int r = 0; r < kIndexHeads; ++r) *reinterpret_cast<uint32_t*>(qt + r * kIndexDim + 4 * lane) = 0u;
-        S.ws[own][lane] = 0.0f;
+      constexpr int kParts = 4 * kPQ / kPEpiWarps;
+      for (int c = 0; c < kParts; ++c) {
+        const int part = e * kParts + c, jq = part >> 2, ew = part & 3;
+        const int j = j0 + jq;
+        uint8_t* qt = S.q + jq * kIndexHeads * kIndexDim;
+        if (j < n_queries) {
+          prepare_query_part(q + static_cast<long long>(j) * kIndexHeads * kIndexDim,
+                             w + static_cast<long long>(j) * kIndexHeads, qt, S.ws[jq], ew, lane);
+        } else {
+#pragma unroll
+          for (int hh = 0; hh < 8; ++hh) *reinterpret_cast<uint32_t*>(qt + sw128_offset(ew * 8 + hh, 4u * lane)) = 0u;
+          if (lane < 8) S.ws[jq][ew * 8 + lane] = 0.0f;
+        }
       }
       fence_proxy_async_smem();
       __syncwarp();
@@ -249,11 +255,11 @@ __global__ void __launch_bounds__(kPThreads, 1)
     }
     named_bar_sync(kBarAll, kPEpiWarps * 32);   // ws of all queries written
 
-    int vis_r[4];
-    uint32_t theta_r[4];
+    int vis_r[kQPW];
+    uint32_t theta_r[kQPW];
 #pragma unroll
-    for (int t = 0; t < 4; ++t) {
-      vis_r[t] = S.vis[half * 4 + t];
+    for (int t = 0; t < kQPW; ++t) {
+      vis_r[t] = S.vis[grp * kQPW + t];
       theta_r[t] = 0u;
     }
     const float kDown = exp2i(-25), kUp = exp2i(25);
@@ -271,10 +277,11 @@ __global__ void __launch_bounds__(kPThreads, 1)
         // All 128 columns of this warp's four queries at once; the
         // accumulator is handed back to the MMA before the arithmetic.
         tc_fence_after();
-        const uint32_t tbase = tmem + a * kPN + (static_cast<uint32_t>(quarter * 32) << 16) + half * 4 * kIndexHeads;
-        uint32_t acc[4][32];
+        const uint32_t tbase =
+            tmem + a * kPN + (static_cast<uint32_t>(quarter * 32) << 16) + grp * kQPW * kIndexHeads;
+        uint32_t acc[kQPW][32];
 #pragma unroll
-        for (int t = 0; t < 4; ++t) tmem_ld_32x32b_x32(tbase + t * kIndexHeads, acc[t]);
+        for (int t = 0; t < kQPW; ++t) tmem_ld_32x32b_x32(tbase + t * kIndexHeads, acc[t]);
         tmem_ld_wait();
         const uint32_t ex = S.exps[x][toff];
         tc_fence_before();
@@ -288,7 +295,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
         // Two queries at a time, each summed in two packed chains, so that
         // four independent FMA chains are in flight.
 #pragma unroll
-        for (int t0 = 0; t0 < 4; t0 += 2) {
+        for (int t0 = 0; t0 < kQPW; t0 += 2) {
           float2 sc[2][2];
 #pragma unroll
           for (int u = 0; u < 2; ++u) sc[u][0] = sc[u][1] = make_float2(0.0f, 0.0f);
@@ -301,7 +308,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
               // multiply by 2^-25 (|acc| < 2^25, so that is ReLU(acc) * 2^-25
               // exactly); the odd sums are scaled back by 2^25 at the end.
               const uint32_t(&ac)[32] = acc[t0 + u];
-              const float4 c = reinterpret_cast<const float4*>(S.ws[half * 4 + t0 + u])[h];
+              const float4 c = reinterpret_cast<const float4*>(S.ws[grp * kQPW + t0 + u])[h];
               float r1, r3;
               asm("mul.rn.sat.f32 %0, %1, %2;" : "=f"(r1) : "f"(__uint_as_float(ac[4 * h + 1])), "f"(kDown));
               asm("mul.rn.sat.f32 %0, %1, %2;" : "=f"(r3) : "f"(__uint_as_float(ac[4 * h + 3])), "f"(kDown));
@@ -314,7 +321,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
 #pragma unroll
           for (int u = 0; u < 2; ++u) {
             const int t = t0 + u;
-            const int jl = half * 4 + t;
+            const int jl = grp * kQPW + t;
             const float even = sc[u][0].x + sc[u][1].x, odd = sc[u][0].y + sc[u][1].y;
             const uint32_t key = order_key(fmaf(odd, kUp, even) * sigma);
             const bool admit = p < vis_r[t] && key > theta_r[t];
@@ -347,11 +354,11 @@ __global__ void __launch_bounds__(kPThreads, 1)
         continue;
       {
         if (*reinterpret_cast<volatile int*>(&S.epi_abort)) break;
-        const int n = *reinterpret_cast<volatile int*>(&S.cnt[own]);
+        const int n = own < kPQ ? *reinterpret_cast<volatile int*>(&S.cnt[own]) : 0;
         if (n > k) {
           const size_t at = static_cast<size_t>(j0 + own) * kCand;
           uint32_t th = 0u;
-          const int kept = warp_compact_topk(wsp.key + at, wsp.pos + at, n, k, S.hist[e], lane, &th);
+          const int kept = warp_compact_topk(wsp.key + at, wsp.pos + at, n, k, S.hist[own], lane, &th);
           if (lane == 0) {
             S.cnt[own] = kept;
             S.theta[own] = max(S.theta[own], th);
@@ -359,11 +366,12 @@ __global__ void __launch_bounds__(kPThreads, 1)
         }
         named_bar_sync(kBarTile, kPEpiWarps * 32);
 #pragma unroll
-        for (int t = 0; t < 4; ++t) theta_r[t] = *reinterpret_cast<volatile uint32_t*>(&S.theta[half * 4 + t]);
+        for (int t = 0; t < kQPW; ++t) theta_r[t] = *reinterpret_cast<volatile uint32_t*>(&S.theta[grp * kQPW + t]);
         crossed = false;
       }
     }
-    if (lane == 0 && j0 + own < n_queries) wsp.cnt[j0 + own] = *reinterpret_cast<volatile int*>(&S.cnt[own]);
+    if (lane == 0 && own < kPQ && j0 + own < n_queries)
+      wsp.cnt[j0 + own] = *reinterpret_cast<volatile int*>(&S.cnt[own]);
   }
 
   tc_fence_before();
