@@ -46,10 +46,36 @@ struct AttnLayout {
   static constexpr uint32_t ml_off = qscale_off + H * 4;             // fp32 [8 ranks][2][H]: pushed m, l
   static constexpr uint32_t fac_off = ml_off + kACluster * 2 * H * 4; // fp32 [8][H]
   static constexpr uint32_t kvalid_off = fac_off + kACluster * H * 4;
-  static constexpr uint32_t total = kvalid_off + kChunk * 4;
+  static constexpr uint32_t bar_off = (kvalid_off + kChunk * 4 + 7) & ~7u;   // receive mbarrier
+  static constexpr uint32_t total = bar_off + 8;
+  // partial-O slice sent to one owner: [H][64 dims] fp32
+  static constexpr uint32_t slice_bytes = H * 64 * 4;
+  static constexpr uint32_t ml_bytes = 2 * H * 4;
+  // staging of two slices and of (m, l), in the S reduction buffer
+  static_assert(2 * slice_bytes + ml_bytes <= DG * H * kSredStride * 4, "staging must fit in the S reduction buffer");
   // pushed partial O: [8 source ranks][H][64 dims] fp32, over the Q + KV region
   static_assert(kACluster * H * 64 * 4 <= sred_off, "received partials must fit in the Q + KV region");
 };
+
+// Address of the same shared-memory offset in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t mapa_rank(uint32_t addr, int rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+  return r;
+}
+// Bulk copy of `bytes` from this CTA's shared memory to another CTA's (no
+// multicast); completion is counted on that CTA's mbarrier.
+__device__ __forceinline__ void bulk_copy_to_rank(uint32_t dst_cluster, uint32_t src_cta, uint32_t bytes,
+                                                  uint32_t bar_cluster) {
+  asm volatile("cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   dst_cluster),
+               "r"(src_cta), "r"(bytes), "r"(bar_cluster)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit_and_wait_read() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
 
 __device__ __forceinline__ uint32_t swz(uint32_t row, uint32_t chunk) {   // 16-byte chunk of a 1 KB row
   return row * kRowBytes + ((chunk ^ (row & 7u)) << 4);
@@ -120,6 +146,13 @@ __global__ void __launch_bounds__(kAThreads, 1)
   int n = (b >= 0 && b < cache.batch) ? cache.ctx_len[b] : 0;
   n = n < 0 ? 0 : (n > capacity ? static_cast<int>(capacity) : n);
   const int32_t* idx = topk + static_cast<long long>(qi) * K;
+  uint64_t* recv_bar = reinterpret_cast<uint64_t*>(smem + L::bar_off);
+  if (tid == 0) {
+    // every rank (this one included) sends this CTA one slice and one (m, l) pair
+    mbar_init(recv_bar, 1);
+    fence_barrier_init();
+    mbar_arrive_expect_tx(recv_bar, kACluster * (L::slice_bytes + L::ml_bytes));
+  }
 
   // ---- query -> fp16 with a power-of-two scale per head ----
   constexpr int kHpw = H / (kAThreads / 32);   // heads per warp; their loads are issued together
@@ -313,29 +346,60 @@ __global__ void __launch_bounds__(kAThreads, 1)
     }
   }
 
-  // ---- push the partial O slices, maxima and sums to their owners ----
+  // ---- send the partial O slices, maxima and sums to their owners ----
   // Output dims [64r, 64r + 64) belong to CTA r; it receives every rank's
-  // slice of them in recv[src][h][64].  Remote stores are fire-and-forget.
+  // slice of them in recv[src][h][64] and every rank's (m, l) in ml_sh[src],
+  // by bulk copies between the cluster's shared memories, two owners' slices
+  // staged at a time.
   cluster.sync();   // every CTA is done reading its Q / KV region, which receives the partials
   float* recv = reinterpret_cast<float*>(smem);
-#pragma unroll
-  for (int i = 0; i < L::DW / 8; ++i) {
-    const int col = dg * L::DW + i * 8 + 2 * (lane & 3);
-    const int owner = col >> 6, c64 = col & 63;
-    float* dst = cluster.map_shared_rank(recv, owner) + (rank * H + ht * 16 + r0) * 64 + c64;
-    *reinterpret_cast<float2*>(dst) = make_float2(o_acc[i][0], o_acc[i][1]);
-    *reinterpret_cast<float2*>(dst + 8 * 64) = make_float2(o_acc[i][2], o_acc[i][3]);
-  }
+  float* stage = sred;                                              // [2][H][64]
+  float* stage_ml = sred + 2 * H * 64;                              // [2][H]: m, l
   if (dg == 0 && (lane & 3) == 0) {
-    for (int r = 0; r < kACluster; ++r) {
-      float* dst = cluster.map_shared_rank(ml_sh, r) + rank * 2 * H;
-      dst[ht * 16 + r0] = m_run[0];
-      dst[ht * 16 + r0 + 8] = m_run[1];
-      dst[H + ht * 16 + r0] = l_run[0];
-      dst[H + ht * 16 + r0 + 8] = l_run[1];
+    stage_ml[ht * 16 + r0] = m_run[0];
+    stage_ml[ht * 16 + r0 + 8] = m_run[1];
+    stage_ml[H + ht * 16 + r0] = l_run[0];
+    stage_ml[H + ht * 16 + r0 + 8] = l_run[1];
+  }
+  for (int pair = 0; pair < kACluster / 2; ++pair) {
+#pragma unroll
+    for (int i = 0; i < L::DW / 8; ++i) {
+      const int col = dg * L::DW + i * 8 + 2 * (lane & 3);
+      const int owner = col >> 6, c64 = col & 63;
+      if ((owner >> 1) != pair) continue;
+      float* dst = stage + ((owner & 1) * H + ht * 16 + r0) * 64 + c64;
+      *reinterpret_cast<float2*>(dst) = make_float2(o_acc[i][0], o_acc[i][1]);
+      *reinterpret_cast<float2*>(dst + 8 * 64) = make_float2(o_acc[i][2], o_acc[i][3]);
+    }
+    fence_proxy_async_smem();
+    __syncthreads();
+    if (tid == 0) {
+      const uint32_t bar = smem_u32(recv_bar);
+      for (int o = 2 * pair; o < 2 * pair + 2; ++o)
+        bulk_copy_to_rank(mapa_rank(smem_u32(recv + rank * H * 64), o), smem_u32(stage + (o & 1) * H * 64),
+                          L::slice_bytes, mapa_rank(bar, o));
+      if (pair == 0)
+        for (int o = 0; o < kACluster; ++o)
+          bulk_copy_to_rank(mapa_rank(smem_u32(ml_sh + rank * 2 * H), o), smem_u32(stage_ml), L::ml_bytes,
+                            mapa_rank(bar, o));
+      bulk_commit_and_wait_read();   // the staging area may be written again
+    }
+    __syncthreads();
+  }
+  // Every copy into this CTA has landed once the barrier completes, and every
+  // copy out of it has been read: after that the CTA may exit without a
+  // cluster-wide barrier.  If the wait runs out, the error is recorded, the
+  // CTA waits once more (bounded) for copies still in flight and leaves
+  // without writing its output.
+  bool received = true;
+  if (tid == 0) {
+    received = mbar_wait(recv_bar, 0, kWaitLimitNs);
+    if (!received) {
+      report_error(cache.err_word, CSA2_ERR_TIMEOUT, kKAttn, b, -1);
+      (void)mbar_wait(recv_bar, 0, kWaitLimitNs);
     }
   }
-  cluster.sync();   // all partials delivered
+  if (!__syncthreads_and(received)) return;
 
   // merge factors per (source rank, head): exp2(m_r - M) / L
   for (int h = tid; h < H; h += kAThreads) {
