@@ -601,6 +601,8 @@ def selected_workload(args):
         changes["batch"] = args.batch
     if args.ctx:
         changes["ctx"] = args.ctx
+    if args.prefill_queries:
+        changes["prefill_queries"] = args.prefill_queries
     return W.scaled(wl, **changes) if changes else wl
 
 
@@ -618,6 +620,8 @@ def main(argv=None):
     p.add_argument("--workload", default="group_1m_b4", choices=sorted(W.WORKLOADS))
     p.add_argument("--batch", type=int, default=0, help="override the workload's batch (profiling cases)")
     p.add_argument("--ctx", type=int, default=0, help="override the workload's context length (profiling cases)")
+    p.add_argument("--prefill-queries", type=int, default=0,
+                   help="override the number of prefill queries (profiling cases)")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
     args = p.parse_args(argv)

@@ -92,11 +92,34 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64
   }
 }
 
+// The same wait with a sleeping back-off between polls (32 ns doubling to
+// 128 ns).  Every poll is a shared-memory operation; many warps polling at
+// once take shared-memory bandwidth from the tensor cores' operand reads, so
+// waits that are expected to last (an epilogue waiting for the next
+// accumulator) use this form.
+__device__ __forceinline__ bool mbar_wait_backoff(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer();
+  uint32_t ns = 32;
+  while (true) {
+    __nanosleep(ns);
+    if (mbar_try_wait(bar, parity)) return true;
+    if (globaltimer() - t0 > limit_ns) return false;
+    if (ns < 128) ns <<= 1;
+  }
+}
+
 // Warp-uniform wait: lane 0 polls, the outcome is broadcast, so the whole warp
 // leaves together (the tcgen05 loads that follow need a converged warp).
 __device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
   bool ok = true;
   if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, limit_ns);
+  return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+}
+// Warp-uniform form of mbar_wait_backoff.
+__device__ __forceinline__ bool mbar_wait_warp_backoff(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
+  bool ok = true;
+  if ((threadIdx.x & 31) == 0) ok = mbar_wait_backoff(bar, parity, limit_ns);
   return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
 }
 // Warp-uniform read of a shared flag.

@@ -20,7 +20,8 @@
 //   * warps 2..17: epilogue.  Warp e reads TMEM lane quarter (warp % 4) for
 //     the two queries 2*(e/4), 2*(e/4)+1: 32 fp32 head dot products per (entry,
 //     query), all 64 columns loaded before the accumulator is handed back ->
-//     score (ReLU split between the min/max and FMA units, packed fp32 FMA) ->
+//     score (ReLU split between the min/max and FMA units, four fp32 FMA
+//     chains per query) ->
 //     filter against the query's running threshold theta.  Survivors are
 //     appended to the query's candidate list in the caller's workspace.  When
 //     any list nears its capacity, epilogue warp j compacts the list of query
@@ -268,7 +269,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
     for (int i = 0; i < n_tiles; ++i) {
       const int a = i % kPAcc, x = i % kPExp;
       if (!failed) failed = warp_flag(&S.abort_flag);
-      if (!failed && (!mbar_wait_warp(&S.acc_full[a], (i / kPAcc) & 1, wait_ns) ||
+      if (!failed && (!mbar_wait_warp_backoff(&S.acc_full[a], (i / kPAcc) & 1, wait_ns) ||
                       !mbar_wait_warp(&S.exp_full[x], (i / kPExp) & 1, wait_ns))) {
         failed = true;
         if (lane == 0) report_error(cache.err_word, CSA2_ERR_TIMEOUT, kKPrefill, req, i);
@@ -292,13 +293,12 @@ __global__ void __launch_bounds__(kPThreads, 1)
         }
         const float sigma = exp2i(static_cast<int>(ex) - 127);
         const int p = i * kTile + toff;
-        // Two queries at a time, each summed in two packed chains, so that
-        // four independent FMA chains are in flight.
+        // Two queries at a time, each summed in four scalar FMA chains.
 #pragma unroll
         for (int t0 = 0; t0 < kQPW; t0 += 2) {
-          float2 sc[2][2];
+          float sc[2][4];
 #pragma unroll
-          for (int u = 0; u < 2; ++u) sc[u][0] = sc[u][1] = make_float2(0.0f, 0.0f);
+          for (int u = 0; u < 2; ++u) sc[u][0] = sc[u][1] = sc[u][2] = sc[u][3] = 0.0f;
 #pragma unroll
           for (int h = 0; h < 8; ++h) {
 #pragma unroll
@@ -312,17 +312,17 @@ __global__ void __launch_bounds__(kPThreads, 1)
               float r1, r3;
               asm("mul.rn.sat.f32 %0, %1, %2;" : "=f"(r1) : "f"(__uint_as_float(ac[4 * h + 1])), "f"(kDown));
               asm("mul.rn.sat.f32 %0, %1, %2;" : "=f"(r3) : "f"(__uint_as_float(ac[4 * h + 3])), "f"(kDown));
-              sc[u][0] = __ffma2_rn(make_float2(c.x, c.y), make_float2(fmaxf(__uint_as_float(ac[4 * h]), 0.0f), r1),
-                                    sc[u][0]);
-              sc[u][1] = __ffma2_rn(make_float2(c.z, c.w),
-                                    make_float2(fmaxf(__uint_as_float(ac[4 * h + 2]), 0.0f), r3), sc[u][1]);
+              sc[u][0] = fmaf(c.x, fmaxf(__uint_as_float(ac[4 * h]), 0.0f), sc[u][0]);
+              sc[u][1] = fmaf(c.y, r1, sc[u][1]);
+              sc[u][2] = fmaf(c.z, fmaxf(__uint_as_float(ac[4 * h + 2]), 0.0f), sc[u][2]);
+              sc[u][3] = fmaf(c.w, r3, sc[u][3]);
             }
           }
 #pragma unroll
           for (int u = 0; u < 2; ++u) {
             const int t = t0 + u;
             const int jl = grp * kQPW + t;
-            const float even = sc[u][0].x + sc[u][1].x, odd = sc[u][0].y + sc[u][1].y;
+            const float even = sc[u][0] + sc[u][2], odd = sc[u][1] + sc[u][3];
             const uint32_t key = order_key(fmaf(odd, kUp, even) * sigma);
             const bool admit = p < vis_r[t] && key > theta_r[t];
             const uint32_t m = __ballot_sync(0xffffffffu, admit);
