@@ -202,3 +202,30 @@ def prefill_topk(q, w, ik_codes, ik_exp, p: int, k: int = TOPK, m: int = 2) -> n
     v = min(prefill_visible(p, m), len(ik_codes))
     s = indexer_scores(q, w, ik_codes[:v], ik_exp[:v])
     return top_k_ascending(np.arange(v), s, k)
+
+
+# ------------------------------------------------------ sequence compressor --
+
+COMPRESS_RATIOS = (1, 2, 4, 8)
+
+
+def compress_tokens(x, m: int) -> np.ndarray:
+    """Sequence compressor of the encoder groups [4sapi blog, section 三: the
+    encoder's Full + 5 Reuse groups compress the sequence with m = 2].
+
+    x: [n*m, d] fp32 token rows; returns [n, d] fp32 entries, entry i the mean of
+    tokens m*i .. m*i + m - 1.  Reading (the pages name m only): a plain mean,
+    summed in float64 in token order, scaled by 1/m and rounded once to fp32;
+    m is a power of two up to 8, so the scaling is exact and the only rounding
+    is the final one (the double sum of at most 8 fp32 values of similar size
+    is exact).  The entries are then quantised on append like any cache row."""
+    if m not in COMPRESS_RATIOS:
+        raise ValueError(f"m must be one of {COMPRESS_RATIOS}")
+    x = np.asarray(x, dtype=np.float32)
+    if x.shape[0] % m:
+        raise ValueError("the token count must be a multiple of m")
+    g = x.reshape(x.shape[0] // m, m, x.shape[1]).astype(np.float64)
+    acc = g[:, 0, :].copy()
+    for j in range(1, m):
+        acc += g[:, j, :]
+    return (acc / m).astype(np.float32)

@@ -254,3 +254,25 @@ def test_pages_constants_match_oracle(golden_dir):
     assert C.INDEX_HEADS == g["index_heads"]["value"]
     assert F.INDEXER_DIM == g["index_head_dim"]["value"]
     assert F.GROUP == g["scale_group_channels"]["value"]
+
+
+# ----------------------------------------------------- sequence compressor --
+
+def test_compress_tokens_is_the_exact_mean_rounded_once():
+    # pinned against exact rational arithmetic: the mean of the m tokens as a
+    # Fraction, rounded once to fp32
+    from fractions import Fraction
+    rng = np.random.default_rng(31)
+    for m in (2, 4, 8):
+        x = (rng.standard_normal((3 * m, 8)) * np.exp(rng.normal(0, 2, (3 * m, 8)))).astype(np.float32)
+        got = C.compress_tokens(x, m)
+        for i in range(3):
+            for d in range(8):
+                exact = sum(Fraction(float(x[m * i + j, d])) for j in range(m)) / m
+                assert got[i, d] == np.float32(float(exact)), (m, i, d)
+    x = rng.standard_normal((5, 16)).astype(np.float32)
+    np.testing.assert_array_equal(C.compress_tokens(x, 1), x)            # m = 1: identity
+    rep = np.repeat(x, 4, axis=0)
+    np.testing.assert_array_equal(C.compress_tokens(rep, 4), x)          # identical tokens
+    with pytest.raises(ValueError):
+        C.compress_tokens(np.zeros((6, 4), np.float32), 3)

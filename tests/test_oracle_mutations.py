@@ -143,3 +143,12 @@ def test_mutation_attention_softmax_over_heads(monkeypatch):
 def test_mutation_prefill_off_by_one(monkeypatch):
     monkeypatch.setattr(C, "prefill_visible", lambda p, m=2: max(0, p // m))
     _fails(PC.test_prefill_visibility)
+
+
+def test_mutation_compressor_drops_a_token(monkeypatch):
+    def wrong(x, m):
+        x = np.asarray(x, dtype=np.float32)
+        g = x.reshape(x.shape[0] // m, m, x.shape[1]).astype(np.float64)
+        return (g[:, : max(m - 1, 1), :].sum(axis=1) / m).astype(np.float32)
+    monkeypatch.setattr(C, "compress_tokens", wrong)
+    _fails(PC.test_compress_tokens_is_the_exact_mean_rounded_once)
