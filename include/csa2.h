@@ -137,6 +137,28 @@ CSA2_API csa2_status csa2_append_kv(const csa2_cache* cache, int32_t n_rows, con
                            void* stream);
 
 /*
+ * csa2_compress_append -- the sequence compressor of the encoder groups,
+ * then quantise-on-append: entry i is the mean of the m token rows
+ * m*i .. m*i + m - 1 and is stored, quantised exactly as by csa2_append_kv,
+ * at position pos[i] of request req[i] [4sapi blog, section 三: the
+ * encoder's 1 Full + 5 Reuse groups compress the sequence with m = 2].
+ * Reading (the pages name m only): a plain mean, summed in float64 in token
+ * order, scaled by 1/m and rounded once to fp32; m in {1, 2, 4, 8}.  Rotary
+ * position encoding, which the pages place before quantisation, is the
+ * caller's: the token rows arrive rotated.
+ *   n_entries  entries to write (>= 0; 0 does nothing)
+ *   m          tokens per entry
+ *   kv_tok     float [n_entries * m][512]  main-KV token rows
+ *   ik_tok     float [n_entries * m][128]  indexer-K token rows
+ *   req        int32 [n_entries] request of each entry, or NULL (request 0)
+ *   pos        int32 [n_entries] entry position inside its request
+ * Device errors as csa2_append_kv.
+ */
+CSA2_API csa2_status csa2_compress_append(const csa2_cache* cache, int32_t n_entries, int32_t m,
+                                          const float* kv_tok, const float* ik_tok, const int32_t* req,
+                                          const int32_t* pos, void* stream);
+
+/*
  * csa2_index_full -- Full-mode indexer scan of every visible position of every
  * request (Hierarchical Sparse Indexer, first stage).
  *   q        float [batch][32][128]  indexer query (quantised inside, FP8 rule)

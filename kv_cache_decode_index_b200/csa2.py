@@ -38,6 +38,7 @@ _I = ctypes.c_int32
 _CP = ctypes.POINTER(CacheStruct)
 _sig = {
     "csa2_append_kv": [_CP, _I, _P, _P, _P, _P, _P],
+    "csa2_compress_append": [_CP, _I, _I, _P, _P, _P, _P, _P],
     "csa2_index_full": [_CP, _P, _P, _P, _P, _P],
     "csa2_pool_select": [_CP, _P, _I, _P, _P],
     "csa2_reindex": [_CP, _I, _P, _I, _P, _P, _P, _P, _I, _P, _P],
@@ -140,6 +141,19 @@ def append_kv(cache: Cache, kv_new, ik_new, pos, req=None):
         _need(req, torch.int32, (n,), "req")
     _check(_lib.csa2_append_kv(ctypes.byref(cache.struct), n, _ptr(kv_new), _ptr(ik_new), _ptr(req), _ptr(pos),
                                _stream(cache.device)), "csa2_append_kv")
+
+
+def compress_append(cache: Cache, kv_tok, ik_tok, pos, m: int = 2, req=None):
+    """Sequence compressor + quantise-on-append: entry i = mean of token rows
+    m*i .. m*i+m-1 of kv_tok [n*m,512] / ik_tok [n*m,128], stored at pos[i]."""
+    n = pos.shape[0]
+    _need(kv_tok, torch.float32, (n * m, KV_DIM), "kv_tok")
+    _need(ik_tok, torch.float32, (n * m, INDEX_DIM), "ik_tok")
+    _need(pos, torch.int32, (n,), "pos")
+    if req is not None:
+        _need(req, torch.int32, (n,), "req")
+    _check(_lib.csa2_compress_append(ctypes.byref(cache.struct), n, int(m), _ptr(kv_tok), _ptr(ik_tok), _ptr(req),
+                                     _ptr(pos), _stream(cache.device)), "csa2_compress_append")
 
 
 def index_full(cache: Cache, q, w, blockmax=None, scores=None):

@@ -143,6 +143,23 @@ csa2_status csa2_append_kv(const csa2_cache* cache, int32_t n_rows, const float*
   return e == cudaSuccess ? CSA2_OK : cuda_fail(e, "append_kv launch");
 }
 
+csa2_status csa2_compress_append(const csa2_cache* cache, int32_t n_entries, int32_t m, const float* kv_tok,
+                                 const float* ik_tok, const int32_t* req, const int32_t* pos, void* stream) {
+  CSA2_TRY(check_cache(cache, true, true));
+  if (n_entries < 0) return fail(CSA2_ERR_SHAPE, "n_entries %d < 0", n_entries);
+  if (m != 1 && m != 2 && m != 4 && m != 8) return fail(CSA2_ERR_SHAPE, "m %d not in {1, 2, 4, 8}", m);
+  if (n_entries == 0) return CSA2_OK;
+  if (kv_tok == nullptr || ik_tok == nullptr || pos == nullptr || !aligned(kv_tok, 16) || !aligned(ik_tok, 16))
+    return fail(CSA2_ERR_ARG, "kv_tok, ik_tok (16-byte aligned) and pos must be set");
+  if (static_cast<long long>(n_entries) * m >= (1LL << 31))
+    return fail(CSA2_ERR_SHAPE, "n_entries * m must stay below 2^31");
+  DeviceInfo d;
+  CSA2_TRY(device_info(&d));
+  const cudaError_t e = csa2::launch_compress_append(*cache, n_entries, m, kv_tok, ik_tok, req, pos,
+                                                     static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? CSA2_OK : cuda_fail(e, "compress_append launch");
+}
+
 csa2_status csa2_index_full(const csa2_cache* cache, const float* q, const float* w, float* blockmax, float* scores,
                             void* stream) {
   CSA2_TRY(check_cache(cache, false, true));

@@ -15,6 +15,9 @@ namespace csa2 {
 cudaError_t launch_append(const csa2_cache& cache, int n_rows, const float* kv_new, const float* ik_new,
                           const int32_t* req, const int32_t* pos, cudaStream_t stream);
 
+cudaError_t launch_compress_append(const csa2_cache& cache, int n_entries, int m, const float* kv_tok,
+                                   const float* ik_tok, const int32_t* req, const int32_t* pos, cudaStream_t stream);
+
 size_t index_full_smem_bytes();
 cudaError_t launch_index_full(const csa2_cache& cache, const float* q, const float* w, float* blockmax,
                               float* scores, const CUtensorMap& ik_map, int num_sms, uint64_t wait_ns,

@@ -25,7 +25,7 @@ def declared_symbols():
 
 def test_every_declared_symbol_is_exported(lib):
     names = declared_symbols()
-    assert len(names) == 12, names
+    assert len(names) == 13, names
     so = ctypes.CDLL(lib.LIB_PATH)
     for n in names:
         assert hasattr(so, n), f"{n} missing from libcsa2.so"
@@ -77,6 +77,11 @@ def test_host_side_validation(lib):
     assert pf(ctypes.byref(c), 0, 8, P, 2, P, P, 512, P, ctypes.c_void_p(p + 8), need, None) == lib.ERR_ARG
     assert pf(ctypes.byref(c), 0, 8, None, 2, P, P, 512, P, P, need, None) == lib.ERR_ARG
     assert pf(ctypes.byref(c), 0, 0, None, 2, None, None, 512, None, None, 0, None) == lib.OK   # nothing to do
+    ca = L.csa2_compress_append
+    assert ca(ctypes.byref(c), 4, 3, P, P, None, P, None) == lib.ERR_SHAPE      # m not a power of two <= 8
+    assert ca(ctypes.byref(c), -1, 2, P, P, None, P, None) == lib.ERR_SHAPE
+    assert ca(ctypes.byref(c), 4, 2, None, P, None, P, None) == lib.ERR_ARG
+    assert ca(ctypes.byref(c), 0, 2, None, None, None, None, None) == lib.OK
     ps = L.csa2_prefill_index_static
     assert ps(ctypes.byref(c), 0, 257, P, 2, P, P, 512, P, None) == lib.ERR_SHAPE   # above the static limit
     assert b"static scratch" in L.csa2_last_error_message()

@@ -103,6 +103,56 @@ def test_append_bitexact(csa2, golden_dir):
     assert csa2.get_error(cache)[0] == csa2.OK
 
 
+@pytest.mark.parametrize("m", [1, 2, 4, 8])
+def test_compress_append_bitexact(csa2, golden_dir, m):
+    """Sequence compressor + quantise-on-append against the oracle's mean and
+    quantisation: codes, scales, indexer codes and exponents bit-exact.  The
+    first entries are the special rows of the append test written as m equal
+    tokens (their mean is the row itself), then pairs of tokens whose mean
+    lands exactly on E2M1 midpoints, then log-normal random tokens."""
+    rng = np.random.default_rng(40 + m)
+    kv_s = _special_kv_rows(rng, golden_dir)
+    ik_s = _special_ik_rows(rng, golden_dir)
+    n_s = min(len(kv_s), len(ik_s))
+    kv_tok = [np.repeat(kv_s[:n_s], m, axis=0)]
+    ik_tok = [np.repeat(ik_s[:n_s], m, axis=0)]
+    if m >= 2:
+        # mean exactly on a midpoint of the E2M1 grid (scale s = 1 by a 6 in the group)
+        mids = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0], np.float32)
+        for _ in range(16):
+            base = np.zeros((m, 512), np.float32)
+            base[:, ::16] = 6.0
+            target = rng.choice(mids, (512,)) * rng.choice([-1.0, 1.0], (512,))
+            d = rng.integers(-8, 9, 512).astype(np.float32) * np.float32(0.0625)   # target +- d exact in fp32
+            base[0] += target + d
+            base[1] += target - d
+            base[2:] += target
+            base[:, ::16] = 6.0
+            kv_tok.append(base)
+            ik_tok.append(np.repeat(rng.standard_normal((1, 128)).astype(np.float32), m, axis=0))
+    n_rand = 300
+    kv_tok.append((rng.standard_normal((n_rand * m, 512)) * np.exp(rng.standard_normal(512) * 2)).astype(np.float32))
+    ik_tok.append((rng.standard_normal((n_rand * m, 128)) *
+                   np.exp(rng.uniform(-20, 20, (n_rand * m, 1)))).astype(np.float32))
+    kv_tok = np.concatenate(kv_tok)
+    ik_tok = np.concatenate(ik_tok)
+    n = kv_tok.shape[0] // m
+    cache = _flat_cache(csa2, n)
+    dev = cache.device
+    perm = rng.permutation(n).astype(np.int32)
+    csa2.compress_append(cache, torch.from_numpy(kv_tok).to(dev), torch.from_numpy(ik_tok).to(dev),
+                         torch.from_numpy(perm).to(dev), m=m)
+    kv_e = C.compress_tokens(kv_tok, m)
+    ik_e = C.compress_tokens(ik_tok, m)
+    codes, scales = F.quantize_main_kv(kv_e)
+    ikc, ike = F.quantize_indexer(ik_e)
+    np.testing.assert_array_equal(cache.kv_scales[:n].cpu().numpy()[perm], scales)
+    np.testing.assert_array_equal(cache.kv_codes[:n].cpu().numpy()[perm], codes)
+    np.testing.assert_array_equal(cache.ik_exp[:n].cpu().numpy()[perm], ike)
+    np.testing.assert_array_equal(cache.ik_codes[:n].cpu().numpy()[perm], ikc)
+    assert csa2.get_error(cache)[0] == csa2.OK
+
+
 def test_append_one_row_per_request(csa2):
     """req = NULL: row i goes to request i (the decode-step append)."""
     rng = np.random.default_rng(1)
