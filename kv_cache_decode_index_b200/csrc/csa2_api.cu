@@ -186,7 +186,7 @@ csa2_status csa2_pool_select(const csa2_cache* cache, const float* blockmax, int
                 capacity_of(cache), kMaxPoolSelectBlocks * csa2::kBlock);
   DeviceInfo d;
   CSA2_TRY(device_info(&d));
-  const int cluster = nblk <= 8LL * 16384 ? 8 : 16;
+  const int cluster = nblk <= 4LL * 16384 ? 8 : 16;   // 16 CTAs above 524,288 positions: half the keys per CTA
   const cudaError_t e = csa2::launch_pool_select(*cache, blockmax, pool_blocks, pool, cluster,
                                                  static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? CSA2_OK : cuda_fail(e, "pool_select launch");
