@@ -3,17 +3,19 @@
 // blog, section 二: every layer attends over its Top-K, Reuse layers with
 // their own query; FP4 rows: 4sapi blog, section 五].
 //
-// One thread-block cluster of 8 CTAs per query.  CTA r takes Top-k entries
-// [r*kc, (r+1)*kc) (kc = ceil(k/8)) in chunks of 64 rows:
+// One thread-block cluster of kACluster (4) CTAs per query.  CTA r takes
+// Top-k entries [r*kc, (r+1)*kc) (kc = ceil(k/4)) in chunks of 64 rows:
 //   * gather + dequantise: E2M1 code x E4M3 scale has <= 5 significant bits
 //     and lies in [2^-10, 2688], so the fp16 row is exact;
 //   * the query is moved to fp16 with a power-of-two scale per head (bf16 ->
 //     fp16 keeps every significant bit in the normal range);
 //   * S = Q K^T and O = P V on mma.sync m16n8k16 (fp16 in, fp32 accumulate),
 //     online softmax in fp32 (exp2 domain), P rounded to fp16;
-// then the 8 partial (O, max, sum) triples are merged through distributed
-// shared memory: every CTA pushes its slice of dims [64r, 64r+64) to CTA r,
-// which merges them locally and writes those dims of every head.
+// then the partial (O, max, sum) triples are merged through distributed
+// shared memory: every CTA sends its slice of dims [128r, 128r+128) to CTA r
+// (bulk copies), which merges them locally and writes those dims of every
+// head.  Four CTAs per query keep all six layers' attention of a decode step
+// within one wave of the GPU's SMs.
 #include <cooperative_groups.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -28,7 +30,8 @@ namespace {
 namespace cg = cooperative_groups;
 
 constexpr int kAThreads = 256;
-constexpr int kACluster = 8;
+constexpr int kACluster = 4;                 // CTAs (key splits) per query
+constexpr int kODims = kKvDim / kACluster;   // output dims owned by one CTA of the cluster
 constexpr int kChunk = 64;                   // keys per chunk
 constexpr int kRowBytes = kKvDim * 2;        // fp16 row: 1024 B
 constexpr int kSredStride = kChunk + 8;      // fp32 row stride of the S reduction buffer
@@ -48,13 +51,15 @@ struct AttnLayout {
   static constexpr uint32_t kvalid_off = fac_off + kACluster * H * 4;
   static constexpr uint32_t bar_off = (kvalid_off + kChunk * 4 + 7) & ~7u;   // receive mbarrier
   static constexpr uint32_t total = bar_off + 8;
-  // partial-O slice sent to one owner: [H][64 dims] fp32
-  static constexpr uint32_t slice_bytes = H * 64 * 4;
+  // partial-O slice sent to one owner: [H][kODims dims] fp32
+  static constexpr uint32_t slice_bytes = H * kODims * 4;
   static constexpr uint32_t ml_bytes = 2 * H * 4;
-  // staging of two slices and of (m, l), in the S reduction buffer
-  static_assert(2 * slice_bytes + ml_bytes <= DG * H * kSredStride * 4, "staging must fit in the S reduction buffer");
-  // pushed partial O: [8 source ranks][H][64 dims] fp32, over the Q + KV region
-  static_assert(kACluster * H * 64 * 4 <= sred_off, "received partials must fit in the Q + KV region");
+  // staging of the slices sent in one round and of (m, l), in the S reduction buffer
+  static constexpr int per_round = (DG * H * kSredStride * 4 - ml_bytes) / slice_bytes >= 2 ? 2 : 1;
+  static_assert(per_round * slice_bytes + ml_bytes <= DG * H * kSredStride * 4, "staging must fit");
+  static_assert(kACluster % per_round == 0, "owners per round must divide the cluster");
+  // received partial O: [kACluster source ranks][H][kODims dims] fp32, over the Q + KV region
+  static_assert(kACluster * H * kODims * 4 <= sred_off, "received partials must fit in the Q + KV region");
 };
 
 // Address of the same shared-memory offset in CTA `rank` of the cluster.
@@ -347,38 +352,38 @@ __global__ void __launch_bounds__(kAThreads, 1)
   }
 
   // ---- send the partial O slices, maxima and sums to their owners ----
-  // Output dims [64r, 64r + 64) belong to CTA r; it receives every rank's
-  // slice of them in recv[src][h][64] and every rank's (m, l) in ml_sh[src],
-  // by bulk copies between the cluster's shared memories, two owners' slices
-  // staged at a time.
+  // Output dims [kODims*r, kODims*(r+1)) belong to CTA r; it receives every
+  // rank's slice of them in recv[src][h][kODims] and every rank's (m, l) in
+  // ml_sh[src], by bulk copies between the cluster's shared memories,
+  // L::per_round owners' slices staged at a time.
   cluster.sync();   // every CTA is done reading its Q / KV region, which receives the partials
   float* recv = reinterpret_cast<float*>(smem);
-  float* stage = sred;                                              // [2][H][64]
-  float* stage_ml = sred + 2 * H * 64;                              // [2][H]: m, l
+  float* stage = sred;                                              // [per_round][H][kODims]
+  float* stage_ml = sred + L::per_round * H * kODims;               // [2][H]: m, l
   if (dg == 0 && (lane & 3) == 0) {
     stage_ml[ht * 16 + r0] = m_run[0];
     stage_ml[ht * 16 + r0 + 8] = m_run[1];
     stage_ml[H + ht * 16 + r0] = l_run[0];
     stage_ml[H + ht * 16 + r0 + 8] = l_run[1];
   }
-  for (int pair = 0; pair < kACluster / 2; ++pair) {
+  for (int round = 0; round < kACluster / L::per_round; ++round) {
 #pragma unroll
     for (int i = 0; i < L::DW / 8; ++i) {
       const int col = dg * L::DW + i * 8 + 2 * (lane & 3);
-      const int owner = col >> 6, c64 = col & 63;
-      if ((owner >> 1) != pair) continue;
-      float* dst = stage + ((owner & 1) * H + ht * 16 + r0) * 64 + c64;
+      const int owner = col / kODims, cd = col % kODims;
+      if (owner / L::per_round != round) continue;
+      float* dst = stage + ((owner % L::per_round) * H + ht * 16 + r0) * kODims + cd;
       *reinterpret_cast<float2*>(dst) = make_float2(o_acc[i][0], o_acc[i][1]);
-      *reinterpret_cast<float2*>(dst + 8 * 64) = make_float2(o_acc[i][2], o_acc[i][3]);
+      *reinterpret_cast<float2*>(dst + 8 * kODims) = make_float2(o_acc[i][2], o_acc[i][3]);
     }
     fence_proxy_async_smem();
     __syncthreads();
     if (tid == 0) {
       const uint32_t bar = smem_u32(recv_bar);
-      for (int o = 2 * pair; o < 2 * pair + 2; ++o)
-        bulk_copy_to_rank(mapa_rank(smem_u32(recv + rank * H * 64), o), smem_u32(stage + (o & 1) * H * 64),
-                          L::slice_bytes, mapa_rank(bar, o));
-      if (pair == 0)
+      for (int o = round * L::per_round; o < (round + 1) * L::per_round; ++o)
+        bulk_copy_to_rank(mapa_rank(smem_u32(recv + rank * H * kODims), o),
+                          smem_u32(stage + (o % L::per_round) * H * kODims), L::slice_bytes, mapa_rank(bar, o));
+      if (round == 0)
         for (int o = 0; o < kACluster; ++o)
           bulk_copy_to_rank(mapa_rank(smem_u32(ml_sh + rank * 2 * H), o), smem_u32(stage_ml), L::ml_bytes,
                             mapa_rank(bar, o));
@@ -422,13 +427,13 @@ __global__ void __launch_bounds__(kAThreads, 1)
     for (int r = 0; r < kACluster; ++r) fac[r * H + h] = mr[r] * inv;
   }
   __syncthreads();
-  // this CTA writes dims [64*rank, 64*rank + 64) of every head, 4 dims per item
-  for (int item = tid; item < H * 16; item += kAThreads) {
-    const int h = item >> 4, d4 = (item & 15) * 4;
+  // this CTA writes dims [kODims*rank, kODims*(rank+1)) of every head, 4 dims per item
+  for (int item = tid; item < H * (kODims / 4); item += kAThreads) {
+    const int h = item / (kODims / 4), d4 = (item % (kODims / 4)) * 4;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
     for (int r = 0; r < kACluster; ++r) {
-      const float4 v = *reinterpret_cast<const float4*>(recv + (r * H + h) * 64 + d4);
+      const float4 v = *reinterpret_cast<const float4*>(recv + (r * H + h) * kODims + d4);
       const float f = fac[r * H + h];
       acc.x += v.x * f; acc.y += v.y * f; acc.z += v.z * f; acc.w += v.w * f;
     }
@@ -436,7 +441,7 @@ __global__ void __launch_bounds__(kAThreads, 1)
     uint2 pk;
     pk.x = *reinterpret_cast<uint32_t*>(&lo);
     pk.y = *reinterpret_cast<uint32_t*>(&hi);
-    *reinterpret_cast<uint2*>(out + (static_cast<long long>(qi) * H + h) * kKvDim + rank * 64 + d4) = pk;
+    *reinterpret_cast<uint2*>(out + (static_cast<long long>(qi) * H + h) * kKvDim + rank * kODims + d4) = pk;
   }
 }
 
