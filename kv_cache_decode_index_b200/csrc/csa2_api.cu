@@ -216,7 +216,7 @@ csa2_status csa2_reindex(const csa2_cache* cache, csa2_mode mode, const int32_t*
   if (pool != nullptr) {
     if (pool_blocks < 1 || pool_blocks > kMaxPool)
       return fail(CSA2_ERR_SHAPE, "pool_blocks %d outside [1, %d]", pool_blocks, kMaxPool);
-    max_blocks = (pool_blocks + 7) / 8;
+    max_blocks = (pool_blocks + csa2::kReindexPoolCluster - 1) / csa2::kReindexPoolCluster;
   } else {
     if (capacity_of(cache) > kMaxFlatPositions)
       return fail(CSA2_ERR_SHAPE, "Top-k without a pool supports request capacity <= %lld positions (got %lld)",

@@ -64,7 +64,7 @@ __global__ void __launch_bounds__(kPoolThreads, 1)
 
 // --------------------------------------------------------------- reindex ----
 constexpr int kRThreads = 320;          // producer, MMA, two epilogue warpgroups
-constexpr int kRStages = 8;
+constexpr int kRStages = 4;
 constexpr int kRAcc = 4;
 constexpr int kBlkBytes = kBlock * kIndexDim;       // 1 KB: one block of 8 indexer-K rows
 constexpr int kBlocksPerTile = kTile / kBlock;      // 16
@@ -100,7 +100,7 @@ struct ReindexLayout {
   }
 };
 
-__global__ void __launch_bounds__(kRThreads, 1)
+__global__ void __launch_bounds__(kRThreads, 2)
     reindex_kernel(const csa2_cache cache, const int32_t* __restrict__ pool, int P, const float* __restrict__ q,
                    const float* __restrict__ w, const float* __restrict__ full_scores, int K,
                    int32_t* __restrict__ topk, const __grid_constant__ CUtensorMap blk_map, int max_blocks,
@@ -356,6 +356,7 @@ cudaError_t configure(Kernel kernel, size_t smem, bool& done) {
   if (done) return cudaSuccess;
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e == cudaSuccess) e = cudaFuncSetAttribute(kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  if (e == cudaSuccess) e = cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
   if (e == cudaSuccess) done = true;
   return e;
 }
@@ -378,11 +379,13 @@ cudaError_t launch_reindex(const csa2_cache& cache, const int32_t* pool, int poo
                            const float* w, const float* full_scores, int k, int32_t* topk,
                            const CUtensorMap& blk_map, int max_blocks, uint64_t wait_ns, cudaStream_t stream) {
   static bool done = false;
-  constexpr int kCluster = 8;
+  // 16 CTAs per request over a pool (a few tiles each, several CTAs per SM),
+  // 8 over a whole context of up to 65,536 positions
+  const int cluster = pool != nullptr ? kReindexPoolCluster : 8;
   const size_t smem_max = reindex_smem_bytes(kMaxReindexBlocks);
   cudaError_t e = configure(reindex_kernel, smem_max, done);
   if (e != cudaSuccess) return e;
-  return launch_cluster(reindex_kernel, cache.batch * kCluster, kRThreads, reindex_smem_bytes(max_blocks), kCluster,
+  return launch_cluster(reindex_kernel, cache.batch * cluster, kRThreads, reindex_smem_bytes(max_blocks), cluster,
                         stream, cache, pool, pool_blocks, q, w, full_scores, k, topk, blk_map, max_blocks, wait_ns);
 }
 

@@ -26,6 +26,7 @@ cudaError_t launch_index_full(const csa2_cache& cache, const float* q, const flo
 cudaError_t launch_pool_select(const csa2_cache& cache, const float* blockmax, int pool_blocks, int32_t* pool,
                                int cluster, cudaStream_t stream);
 
+constexpr int kReindexPoolCluster = 16;   // CTAs per request when re-scoring a pool
 cudaError_t launch_reindex(const csa2_cache& cache, const int32_t* pool, int pool_blocks, const float* q,
                            const float* w, const float* full_scores, int k, int32_t* topk,
                            const CUtensorMap& ik_blk_map, int cands_per_cta, uint64_t wait_ns, cudaStream_t stream);
