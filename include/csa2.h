@@ -287,6 +287,21 @@ CSA2_API csa2_status csa2_prefill_index_static(const csa2_cache* cache, int32_t 
                                                const float* w, int32_t k, int32_t* topk, void* stream);
 
 /*
+ * csa2_sparse_attn_layers -- csa2_sparse_attn for n_layers layers that attend
+ * over the same Top-k (a Full or Reindex layer and the Reuse layers that take
+ * its indices [readance summary, section 4.2: a Reuse layer keeps its own main
+ * query]), in one launch.
+ *   q    host array [n_layers] of device pointers, each bf16 [n_queries][H][512]
+ *   out  host array [n_layers] of device pointers, each bf16 [n_queries][H][512]
+ * n_layers in [1, CSA2_ATTN_MAX_LAYERS]; everything else as csa2_sparse_attn.
+ */
+#define CSA2_ATTN_MAX_LAYERS 8
+CSA2_API csa2_status csa2_sparse_attn_layers(const csa2_cache* cache, int32_t n_layers, int32_t n_queries,
+                                             const int32_t* q_req, const int32_t* topk, int32_t k,
+                                             const uint16_t* const* q, int32_t H, float scale,
+                                             uint16_t* const* out, void* stream);
+
+/*
  * csa2_get_error -- synchronise `stream`, copy cache->err_word to the host
  * array out[4] (host pointer) and return out[0] as a status (CSA2_OK when no
  * device error was recorded).  Does not clear the word.

@@ -43,6 +43,7 @@ _sig = {
     "csa2_pool_select": [_CP, _P, _I, _P, _P],
     "csa2_reindex": [_CP, _I, _P, _I, _P, _P, _P, _P, _I, _P, _P],
     "csa2_sparse_attn": [_CP, _I, _P, _P, _I, _P, _I, ctypes.c_float, _P, _P],
+    "csa2_sparse_attn_layers": [_CP, _I, _I, _P, _P, _I, _P, _I, ctypes.c_float, _P, _P],
     "csa2_prefill_index": [_CP, _I, _I, _P, _I, _P, _P, _I, _P, _P, ctypes.c_size_t, _P],
     "csa2_prefill_index_static": [_CP, _I, _I, _P, _I, _P, _P, _I, _P, _P],
     "csa2_get_error": [_CP, ctypes.POINTER(ctypes.c_int32), _P],
@@ -264,6 +265,29 @@ def prefill_index_static(cache: Cache, req: int, q_pos, q, w, k: int = 512, rati
     return topk
 
 
+def sparse_attn_layers(cache: Cache, topk, q_layers, scale: float | None = None, out_layers=None, q_req=None):
+    """Sparse attention of several layers over the same Top-k in one launch;
+    q_layers: list of bf16 [n, H, 512] -> list of outputs of the same shape."""
+    n, k = topk.shape
+    L = len(q_layers)
+    H = q_layers[0].shape[1]
+    _need(topk, torch.int32, (n, k), "topk")
+    for i, q in enumerate(q_layers):
+        _need(q, torch.bfloat16, (n, H, KV_DIM), f"q_layers[{i}]")
+    if q_req is not None:
+        _need(q_req, torch.int32, (n,), "q_req")
+    if out_layers is None:
+        out_layers = [torch.empty_like(q) for q in q_layers]
+    for i, o in enumerate(out_layers):
+        _need(o, torch.bfloat16, (n, H, KV_DIM), f"out_layers[{i}]")
+    scale = 1.0 / math.sqrt(KV_DIM) if scale is None else scale
+    qa = (ctypes.c_void_p * L)(*[q.data_ptr() for q in q_layers])
+    oa = (ctypes.c_void_p * L)(*[o.data_ptr() for o in out_layers])
+    _check(_lib.csa2_sparse_attn_layers(ctypes.byref(cache.struct), L, n, _ptr(q_req), _ptr(topk), k, qa, H,
+                                        ctypes.c_float(scale), oa, _stream(cache.device)), "csa2_sparse_attn_layers")
+    return out_layers
+
+
 def get_error(cache: Cache):
     """Synchronise the current stream and return (status, err_word list)."""
     out = (ctypes.c_int32 * 4)()
@@ -301,17 +325,25 @@ class DecodeGroup:
                 src = torch.empty(B, k, dtype=torch.int32, device=dev)
                 self.topk.append(src)
         self.concurrent = concurrent
-        n_side = sum(1 for m in self.modes if m != "Ru")
-        # one stream per layer: every layer's Top-k waits for the pool only,
-        # and a Reuse layer's attention waits for its source's Top-k only
-        self.streams = [torch.cuda.Stream(dev) for _ in self.modes] if concurrent else []
-        self.launches_per_step = 1 + (1 if pool_blocks else 0) + n_side + len(self.modes)
+        # attention launches: each Full/Reindex layer with the Reuse layers that follow it
+        self.sources = []
+        for layer, m in enumerate(self.modes):
+            if m != "Ru":
+                self.sources.append([layer])
+            else:
+                self.sources[-1].append(layer)
+        # the last source's chain (pool -> Top-k -> attention) runs on the
+        # calling stream, linked by programmatic dependent launch; the other
+        # sources run on streams of their own, after the pool
+        self.streams = [torch.cuda.Stream(dev) for _ in self.sources[:-1]] if concurrent else []
+        self.launches_per_step = 1 + (1 if pool_blocks else 0) + 2 * len(self.sources)
 
     def step(self, q_idx, w_idx, q_main, out, timing=None):
         """q_idx / w_idx: per layer ([B,32,128] / [B,32], None for Reuse);
         q_main / out: per layer bf16 [B, H, 512].  timing: optional dict
         name -> (start, end) CUDA events, recorded on the launching stream
-        around the launch of that name ("scan", "pool", "topk<l>", "attn<l>")."""
+        around the launch of that name ("scan", "pool", "topk<l>", and
+        "attn<l>" for source layer l with its Reuse layers)."""
         c = self.cache
 
         def timed(name, fn):
@@ -327,27 +359,22 @@ class DecodeGroup:
         if self.pool is not None:
             timed("pool", lambda: pool_select(c, self.blockmax, self.pool_blocks, self.pool))
         main = torch.cuda.current_stream(c.device)
-        ev_ready = torch.cuda.Event()
-        ev_ready.record(main)
-        ev_topk = {}
-        src = 0
-        for layer, m in enumerate(self.modes):
-            s = self.streams[layer] if self.concurrent else main
+        ev_ready = None
+        if self.concurrent and len(self.sources) > 1:
+            ev_ready = torch.cuda.Event()
+            ev_ready.record(main)
+        for si in range(len(self.sources)):   # side streams first, the calling stream's chain last
+            layers = self.sources[si]
+            src = layers[0]
+            s = main if (si == len(self.sources) - 1 or not self.concurrent) else self.streams[si]
             with torch.cuda.stream(s):
-                if m != "Ru":
-                    if s is not main:
-                        s.wait_event(ev_ready)
-                    mode = FULL if m == "F" else REINDEX
-                    timed(f"topk{layer}", lambda: reindex(c, mode, self.k, self.pool, q_idx[layer], w_idx[layer],
-                                                          topk=self.topk[layer]))
-                    src = layer
-                    if self.concurrent:
-                        ev_topk[layer] = torch.cuda.Event()
-                        ev_topk[layer].record(s)
-                elif s is not main:
-                    s.wait_event(ev_topk[src])
-                timed(f"attn{layer}", lambda: sparse_attn(c, self.topk[layer], q_main[layer], self.scale,
-                                                          out[layer]))
+                if s is not main:
+                    s.wait_event(ev_ready)
+                mode = FULL if self.modes[src] == "F" else REINDEX
+                timed(f"topk{src}", lambda: reindex(c, mode, self.k, self.pool, q_idx[src], w_idx[src],
+                                                    topk=self.topk[src]))
+                timed(f"attn{src}", lambda: sparse_attn_layers(c, self.topk[src], [q_main[l] for l in layers],
+                                                               self.scale, [out[l] for l in layers]))
         if self.concurrent:
             joins = []
             for s in self.streams:
@@ -360,10 +387,8 @@ class DecodeGroup:
 
     def launch_names(self):
         names = ["scan"] + (["pool"] if self.pool is not None else [])
-        for layer, m in enumerate(self.modes):
-            if m != "Ru":
-                names.append(f"topk{layer}")
-            names.append(f"attn{layer}")
+        for layers in self.sources:
+            names += [f"topk{layers[0]}", f"attn{layers[0]}"]
         return names
 
 
@@ -384,16 +409,21 @@ class PrefillGroup:
         self.workspace = torch.empty(max(prefill_workspace_bytes(n_queries), 16), dtype=torch.uint8, device=dev)
         self.q_req = torch.full((n_queries,), req, dtype=torch.int32, device=dev)
         self.topk, src = [], None
-        for m in self.modes:
+        self.sources = []
+        for layer, m in enumerate(self.modes):
             if m != "Ru":
                 src = torch.empty(n_queries, k, dtype=torch.int32, device=dev)
+                self.sources.append([layer])
+            else:
+                self.sources[-1].append(layer)
             self.topk.append(src)
-        self.launches_per_step = sum(2 for m in self.modes if m != "Ru") + len(self.modes)
+        self.launches_per_step = 3 * len(self.sources)   # indexer (2 kernels) + one attention launch per source
 
     def step(self, q_pos, q_idx, w_idx, q_main, out, timing=None):
         """q_pos int32 [n]; q_idx / w_idx per layer (None for Reuse); q_main /
         out per layer bf16 [n, H, 512].  timing: optional dict name -> (start,
-        end) CUDA events around "topk<l>" and "attn<l>"."""
+        end) CUDA events around "topk<l>" and "attn<l>" (l a Full/Reindex
+        layer; its attention launch covers the Reuse layers that follow it)."""
         c = self.cache
 
         def timed(name, fn):
@@ -404,10 +434,10 @@ class PrefillGroup:
             if ev is not None:
                 ev[1].record()
 
-        for layer, m in enumerate(self.modes):
-            if m != "Ru":
-                timed(f"topk{layer}", lambda: prefill_index(c, self.req, q_pos, q_idx[layer], w_idx[layer], self.k,
-                                                            self.ratio, self.topk[layer], self.workspace))
-            timed(f"attn{layer}", lambda: sparse_attn(c, self.topk[layer], q_main[layer], self.scale, out[layer],
-                                                      q_req=self.q_req))
+        for layers in self.sources:
+            src = layers[0]
+            timed(f"topk{src}", lambda: prefill_index(c, self.req, q_pos, q_idx[src], w_idx[src], self.k,
+                                                      self.ratio, self.topk[src], self.workspace))
+            timed(f"attn{src}", lambda: sparse_attn_layers(c, self.topk[src], [q_main[l] for l in layers],
+                                                           self.scale, [out[l] for l in layers], q_req=self.q_req))
         return out

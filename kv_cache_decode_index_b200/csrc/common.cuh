@@ -129,6 +129,15 @@ __device__ __forceinline__ bool warp_flag(const volatile int* flag) {
   return __shfl_sync(0xffffffffu, v, 0) != 0;
 }
 
+// ------------------------------------------- programmatic dependent launch ----
+// A kernel launched with programmatic stream serialization may start while
+// its predecessor in the stream is still running: it must call pdl_wait()
+// before reading anything the predecessor writes.  pdl_launch_dependents()
+// lets the next kernel in the stream be launched early.  Both are no-ops
+// without a programmatic dependency.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ------------------------------------------------------- named barriers ----
 // bar.sync on barrier `id` (1..15) for `count` threads (a multiple of 32).
 __device__ __forceinline__ void named_bar_sync(int id, int count) {

@@ -124,6 +124,31 @@ csa2_status check_cache(const csa2_cache* c, bool need_kv, bool need_ik) {
     if (s_ != CSA2_OK) return s_;      \
   } while (0)
 
+csa2_status sparse_attn_impl(const csa2_cache* cache, int32_t n_layers, int32_t n_queries, const int32_t* q_req,
+                             const int32_t* topk, int32_t k, const uint16_t* const* q, int32_t H, float scale,
+                             uint16_t* const* out, void* stream) {
+  CSA2_TRY(check_cache(cache, true, false));
+  if (n_layers < 1 || n_layers > CSA2_ATTN_MAX_LAYERS)
+    return fail(CSA2_ERR_SHAPE, "n_layers %d outside [1, %d]", n_layers, CSA2_ATTN_MAX_LAYERS);
+  if (n_queries < 0) return fail(CSA2_ERR_SHAPE, "n_queries %d < 0", n_queries);
+  if (n_queries == 0) return CSA2_OK;
+  if (q_req == nullptr && n_queries > cache->batch)
+    return fail(CSA2_ERR_SHAPE, "without q_req, n_queries (%d) must not exceed batch (%d)", n_queries, cache->batch);
+  if (H != 16 && H != 32 && H != 64) return fail(CSA2_ERR_SHAPE, "H %d not in {16, 32, 64}", H);
+  if (k < 1 || k > kMaxK) return fail(CSA2_ERR_SHAPE, "k %d outside [1, %d]", k, kMaxK);
+  if (static_cast<long long>(n_layers) * n_queries * 4 >= (1LL << 31))
+    return fail(CSA2_ERR_SHAPE, "n_layers * n_queries too large");
+  if (topk == nullptr || q == nullptr || out == nullptr) return fail(CSA2_ERR_ARG, "topk, q and out must be set");
+  for (int l = 0; l < n_layers; ++l)
+    if (q[l] == nullptr || out[l] == nullptr || !aligned(q[l], 16) || !aligned(out[l], 16))
+      return fail(CSA2_ERR_ARG, "layer %d: q and out (16-byte aligned) must be set", l);
+  DeviceInfo d;
+  CSA2_TRY(device_info(&d));
+  const cudaError_t e = csa2::launch_sparse_attn(*cache, n_layers, n_queries, q_req, topk, k, q, H, scale, out,
+                                                 static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? CSA2_OK : cuda_fail(e, "sparse_attn launch");
+}
+
 }  // namespace
 
 extern "C" {
@@ -233,22 +258,19 @@ csa2_status csa2_reindex(const csa2_cache* cache, csa2_mode mode, const int32_t*
   return e == cudaSuccess ? CSA2_OK : cuda_fail(e, "reindex launch");
 }
 
+
 csa2_status csa2_sparse_attn(const csa2_cache* cache, int32_t n_queries, const int32_t* q_req, const int32_t* topk,
                              int32_t k, const uint16_t* q, int32_t H, float scale, uint16_t* out, void* stream) {
-  CSA2_TRY(check_cache(cache, true, false));
-  if (n_queries < 0) return fail(CSA2_ERR_SHAPE, "n_queries %d < 0", n_queries);
-  if (n_queries == 0) return CSA2_OK;
-  if (q_req == nullptr && n_queries > cache->batch)
-    return fail(CSA2_ERR_SHAPE, "without q_req, n_queries (%d) must not exceed batch (%d)", n_queries, cache->batch);
-  if (H != 16 && H != 32 && H != 64) return fail(CSA2_ERR_SHAPE, "H %d not in {16, 32, 64}", H);
-  if (k < 1 || k > kMaxK) return fail(CSA2_ERR_SHAPE, "k %d outside [1, %d]", k, kMaxK);
-  if (topk == nullptr || q == nullptr || out == nullptr || !aligned(q, 16) || !aligned(out, 16))
-    return fail(CSA2_ERR_ARG, "topk, q and out (16-byte aligned) must be set");
-  DeviceInfo d;
-  CSA2_TRY(device_info(&d));
-  const cudaError_t e = csa2::launch_sparse_attn(*cache, n_queries, q_req, topk, k, q, H, scale, out,
-                                                 static_cast<cudaStream_t>(stream));
-  return e == cudaSuccess ? CSA2_OK : cuda_fail(e, "sparse_attn launch");
+  const uint16_t* qs[1] = {q};
+  uint16_t* os[1] = {out};
+  if (q == nullptr || out == nullptr) return fail(CSA2_ERR_ARG, "topk, q and out (16-byte aligned) must be set");
+  return sparse_attn_impl(cache, 1, n_queries, q_req, topk, k, qs, H, scale, os, stream);
+}
+
+csa2_status csa2_sparse_attn_layers(const csa2_cache* cache, int32_t n_layers, int32_t n_queries,
+                                    const int32_t* q_req, const int32_t* topk, int32_t k, const uint16_t* const* q,
+                                    int32_t H, float scale, uint16_t* const* out, void* stream) {
+  return sparse_attn_impl(cache, n_layers, n_queries, q_req, topk, k, q, H, scale, out, stream);
 }
 
 size_t csa2_prefill_workspace_bytes(int32_t n_queries) { return csa2::prefill_workspace_bytes(n_queries); }

@@ -128,10 +128,17 @@ __device__ __forceinline__ void dequant16(uint4 codes, uint32_t s01, uint4 (&out
   for (int c = 0; c < 4; ++c) out[c] = make_uint4(h[4 * c], h[4 * c + 1], h[4 * c + 2], h[4 * c + 3]);
 }
 
+// Query and output of each layer attending over the same Top-k (a Full or
+// Reindex layer and the Reuse layers that take its indices).
+struct AttnLayers {
+  const __nv_bfloat16* q[CSA2_ATTN_MAX_LAYERS];
+  __nv_bfloat16* out[CSA2_ATTN_MAX_LAYERS];
+};
+
 template <int H>
 __global__ void __launch_bounds__(kAThreads, 1)
-    sparse_attn_kernel(const csa2_cache cache, const int32_t* __restrict__ q_req, const int32_t* __restrict__ topk,
-                       int K, const __nv_bfloat16* __restrict__ qg, float softmax_scale, __nv_bfloat16* __restrict__ out) {
+    sparse_attn_kernel(const csa2_cache cache, int n_queries, const int32_t* __restrict__ q_req,
+                       const int32_t* __restrict__ topk, int K, const AttnLayers io, float softmax_scale) {
   using L = AttnLayout<H>;
   extern __shared__ __align__(1024) uint8_t smem[];
   const uint32_t sbase = smem_u32(smem);
@@ -143,7 +150,12 @@ __global__ void __launch_bounds__(kAThreads, 1)
 
   cg::cluster_group cluster = cg::this_cluster();
   const int rank = static_cast<int>(cluster.block_rank());
-  const int qi = blockIdx.x / kACluster;
+  pdl_wait();                 // everything the preceding launch wrote (the Top-k) is visible
+  pdl_launch_dependents();
+  const int layer = static_cast<int>(blockIdx.x / kACluster) / n_queries;
+  const int qi = static_cast<int>(blockIdx.x / kACluster) % n_queries;
+  const __nv_bfloat16* __restrict__ qg = io.q[layer];
+  __nv_bfloat16* __restrict__ out = io.out[layer];
   const int b = q_req != nullptr ? q_req[qi] : qi;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int ht = warp % L::HT, dg = warp / L::HT;
@@ -446,8 +458,8 @@ __global__ void __launch_bounds__(kAThreads, 1)
 }
 
 template <int H>
-cudaError_t launch_h(const csa2_cache& cache, int n_queries, const int32_t* q_req, const int32_t* topk, int k,
-                     const uint16_t* q, float scale, uint16_t* out, cudaStream_t stream) {
+cudaError_t launch_h(const csa2_cache& cache, int n_layers, int n_queries, const int32_t* q_req, const int32_t* topk,
+                     int k, const AttnLayers& io, float scale, cudaStream_t stream) {
   static bool done = false;
   const size_t smem = AttnLayout<H>::total;
   if (!done) {
@@ -457,29 +469,36 @@ cudaError_t launch_h(const csa2_cache& cache, int n_queries, const int32_t* q_re
     done = true;
   }
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(n_queries * kACluster);
+  cfg.gridDim = dim3(n_layers * n_queries * kACluster);
   cfg.blockDim = dim3(kAThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = kACluster;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;   // the kernel calls pdl_wait() first
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, sparse_attn_kernel<H>, cache, q_req, topk, k,
-                            reinterpret_cast<const __nv_bfloat16*>(q), scale, reinterpret_cast<__nv_bfloat16*>(out));
+  cfg.numAttrs = 2;
+  return cudaLaunchKernelEx(&cfg, sparse_attn_kernel<H>, cache, n_queries, q_req, topk, k, io, scale);
 }
 
 }  // namespace
 
-cudaError_t launch_sparse_attn(const csa2_cache& cache, int n_queries, const int32_t* q_req, const int32_t* topk,
-                               int k, const uint16_t* q, int H, float scale, uint16_t* out, cudaStream_t stream) {
+cudaError_t launch_sparse_attn(const csa2_cache& cache, int n_layers, int n_queries, const int32_t* q_req,
+                               const int32_t* topk, int k, const uint16_t* const* q, int H, float scale,
+                               uint16_t* const* out, cudaStream_t stream) {
+  AttnLayers io = {};
+  for (int l = 0; l < n_layers; ++l) {
+    io.q[l] = reinterpret_cast<const __nv_bfloat16*>(q[l]);
+    io.out[l] = reinterpret_cast<__nv_bfloat16*>(out[l]);
+  }
   switch (H) {
-    case 16: return launch_h<16>(cache, n_queries, q_req, topk, k, q, scale, out, stream);
-    case 32: return launch_h<32>(cache, n_queries, q_req, topk, k, q, scale, out, stream);
-    case 64: return launch_h<64>(cache, n_queries, q_req, topk, k, q, scale, out, stream);
+    case 16: return launch_h<16>(cache, n_layers, n_queries, q_req, topk, k, io, scale, stream);
+    case 32: return launch_h<32>(cache, n_layers, n_queries, q_req, topk, k, io, scale, stream);
+    case 64: return launch_h<64>(cache, n_layers, n_queries, q_req, topk, k, io, scale, stream);
     default: return cudaErrorInvalidValue;
   }
 }

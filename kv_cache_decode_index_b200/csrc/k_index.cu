@@ -103,6 +103,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const long long capacity = static_cast<long long>(cache.max_pages_per_req) * cache.page_size;
   const uint32_t page_size = static_cast<uint32_t>(cache.page_size);
 
+  pdl_wait();                 // the cache rows of a preceding append are complete
+  pdl_launch_dependents();    // the pool selection may be launched (it waits for this grid)
+
   // ---- tiles per request, prefix sums ----
   {
     using Scan = cub::BlockScan<int, kThreads>;
@@ -385,8 +388,17 @@ cudaError_t launch_index_full(const csa2_cache& cache, const float* q, const flo
     if (e != cudaSuccess) return e;
     configured = true;
   }
-  index_full_kernel<<<num_sms, kThreads, smem, stream>>>(cache, q, w, blockmax, scores, ik_map, wait_ns);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(num_sms);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, index_full_kernel, cache, q, w, blockmax, scores, ik_map, wait_ns);
 }
 
 }  // namespace csa2

@@ -30,6 +30,8 @@ __global__ void __launch_bounds__(kPoolThreads, 1)
     pool_select_kernel(const csa2_cache cache, const float* __restrict__ blockmax, int P, int32_t* __restrict__ pool) {
   extern __shared__ uint8_t smem_raw[];
   PoolSmem& S = *reinterpret_cast<PoolSmem*>(smem_raw);
+  pdl_wait();                 // the block maxima of the scan are complete
+  pdl_launch_dependents();
   cg::cluster_group cluster = cg::this_cluster();
   const int C = static_cast<int>(cluster.num_blocks());
   const int rank = static_cast<int>(cluster.block_rank());
@@ -123,6 +125,8 @@ __global__ void __launch_bounds__(kRThreads, 2)
   const int b = blockIdx.x / C;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const long long capacity = static_cast<long long>(cache.max_pages_per_req) * cache.page_size;
+  pdl_wait();                 // the pool (or the stored scores) of the preceding launch are complete
+  pdl_launch_dependents();
   int n = cache.ctx_len[b];
   n = n < 0 ? 0 : (n > capacity ? static_cast<int>(capacity) : n);
 
@@ -341,13 +345,15 @@ cudaError_t launch_cluster(Kernel kernel, int grid, int threads, size_t smem, in
   cfg.blockDim = dim3(threads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = cluster;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;   // the kernels call pdl_wait()
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   return cudaLaunchKernelEx(&cfg, kernel, args...);
 }
 

@@ -42,7 +42,10 @@ cudaError_t launch_prefill_index(const csa2_cache& cache, int req, int n_queries
 
 cudaError_t launch_copy_topk(const int32_t* src, int32_t* dst, long long n, cudaStream_t stream);
 
-cudaError_t launch_sparse_attn(const csa2_cache& cache, int n_queries, const int32_t* q_req, const int32_t* topk,
-                               int k, const uint16_t* q, int H, float scale, uint16_t* out, cudaStream_t stream);
+// q[l] / out[l] (host array of device pointers): query and output of layer l
+// of n_layers layers sharing the Top-k.
+cudaError_t launch_sparse_attn(const csa2_cache& cache, int n_layers, int n_queries, const int32_t* q_req,
+                               const int32_t* topk, int k, const uint16_t* const* q, int H, float scale,
+                               uint16_t* const* out, cudaStream_t stream);
 
 }  // namespace csa2

@@ -342,6 +342,23 @@ def test_sparse_attention_parity(csa2, H, k, n):
         print(f"H={H} k={k} b={b}: max rel err {rel:.2e}")
 
 
+def test_sparse_attention_layers_equal_single_layer_launches(csa2):
+    """One launch over four layers sharing the Top-k (a Reindex layer and its
+    Reuse layers) gives, per layer, exactly the single-layer launch's output."""
+    wl = W.scaled(W.WORKLOADS["group_64k_b8"], batch=3, ctx=4000, heads=32)
+    cache = U.build_cache(wl, csa2)
+    dev = cache.device
+    rng = np.random.default_rng(17)
+    topk = torch.from_numpy(np.stack([np.sort(rng.choice(4000, 300, replace=False)) for _ in range(3)])
+                            .astype(np.int32)).to(dev)
+    qs = [W.main_query(wl, layer).to(dev) for layer in range(4)]
+    multi = csa2.sparse_attn_layers(cache, topk, qs, wl.scale)
+    for layer in range(4):
+        single = csa2.sparse_attn(cache, topk, qs[layer], wl.scale)
+        assert torch.equal(multi[layer], single), f"layer {layer}"
+    assert csa2.get_error(cache)[0] == csa2.OK
+
+
 def test_sparse_attention_empty_and_query_map(csa2):
     wl = W.scaled(W.WORKLOADS["full_4k_b1"], batch=2, heads=16, page_size=1024)
     cache = U.build_cache(wl, csa2, lengths=[2000, 3000])
