@@ -341,31 +341,11 @@ def run_b200(args):
 
     # ---- end to end: pinned host inputs -> device, step, outputs -> host ----
     h2d, d2h = io_bytes(wl)
-    e2e_value = None
+    e2e_value = e2e_serial = None
     if not args.no_e2e:
-        hq = [None if t is None else t.cpu().pin_memory() for t in q_idx]
-        hw = [None if t is None else t.cpu().pin_memory() for t in w_idx]
-        hm = [t.cpu().pin_memory() for t in q_main]
-        ho = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in out]
-        s = torch.cuda.current_stream()
-        for it in range(args.warmup + args.steps):
-            if it == args.warmup:
-                if world > 1:
-                    dist.barrier()
-                torch.cuda.synchronize()
-                a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                a0.record()
-            for dst, src in zip(q_idx + w_idx + q_main, hq + hw + hm):
-                if dst is not None:
-                    dst.copy_(src, non_blocking=True)
-            graph.replay()
-            for dst, src in zip(ho, out):
-                dst.copy_(src, non_blocking=True)
-            s.synchronize()
-        a1.record()
-        torch.cuda.synchronize()
-        e2e_ms = max_over_ranks(a0.elapsed_time(a1) / args.steps, dev, world)
-        e2e_value = world * wl.batch / (e2e_ms / 1e3)
+        piped_ms, serial_ms = e2e_step_ms(args, group, q_idx, w_idx, q_main, out, dev, world)
+        e2e_value = world * wl.batch / (max_over_ranks(piped_ms, dev, world) / 1e3)
+        e2e_serial = world * wl.batch / (max_over_ranks(serial_ms, dev, world) / 1e3)
 
     st, word = csa2.get_error(cache)
     if st != csa2.OK:
@@ -389,7 +369,12 @@ def run_b200(args):
                          "traffic": traffic, "kernel": "csa2 index_full (Full indexer scan)",
                          "kernel_ms": scan_avg_ms, "alg_bytes_per_launch": scan_bytes,
                          "peak_source": f"{peak_src} copy bandwidth (MEASURED_PEAKS.json hbm_gbs, burst)"},
-            "e2e": {"value": e2e_value, "unit": "queries/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "e2e": {"value": e2e_value, "unit": "queries/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "how": "DecodeGroup.step per step; one packed pinned host-to-device copy of all the step's inputs "
+                           "and one device-to-host copy of all its outputs every step, inside the timed region; two "
+                           "buffer slots and one copy stream per direction overlap step i+1's upload and step i-1's "
+                           "download with step i",
+                    "serial_value": e2e_serial},
             "gpu_launches": group.launches_per_step * args.steps,
             "launch_ms": {name: statistics.mean(v) for name, v in per_launch.items()},
             "clocks": clocks,
@@ -532,7 +517,12 @@ def run_prefill(args):
                          "frac": achieved / peak, "traffic": None, "kernel": "csa2 prefill_index (FP8 GEMM + "
                          "streaming Top-512)", "kernel_ms": idx_ms, "flops_per_launch": flops,
                          "peak_source": peak_src},
-            "e2e": {"value": e2e_value, "unit": "queries/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "e2e": {"value": e2e_value, "unit": "queries/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "how": "DecodeGroup.step per step; one packed pinned host-to-device copy of all the step's inputs "
+                           "and one device-to-host copy of all its outputs every step, inside the timed region; two "
+                           "buffer slots and one copy stream per direction overlap step i+1's upload and step i-1's "
+                           "download with step i",
+                    "serial_value": e2e_serial},
             "gpu_launches": group.launches_per_step * args.steps,
             "launch_ms": {k: statistics.mean(v) for k, v in per_launch.items()},
             "clocks": clocks}
@@ -542,6 +532,99 @@ def run_prefill(args):
                                 "sample": f"2 of the {n} queries: float64 oracle Top-512 over all visible entries "
                                           f"and six attention layers, {spq:.1f} s per query"}
     print(json.dumps(line), flush=True)
+
+
+def e2e_step_ms(args, group, q_idx, w_idx, q_main, out, dev, world):
+    """Milliseconds per step end to end through DecodeGroup.step with host
+    buffers.  Every step copies all of its inputs from pinned host memory
+    (packed: one host-to-device copy) and all of its outputs back (one
+    device-to-host copy), inside the timed region.  Two slots of device
+    buffers, each with its own captured step, and one copy stream per
+    direction let step i+1's upload and step i-1's download overlap step i."""
+    import torch
+    import torch.distributed as dist
+    ins = [t for t in q_idx + w_idx + q_main if t is not None]
+    nbytes = lambda t: t.numel() * t.element_size()
+    in_bytes, out_bytes = sum(nbytes(t) for t in ins), sum(nbytes(t) for t in out)
+    h_in = torch.empty(in_bytes, dtype=torch.uint8, pin_memory=True)
+    off = 0
+    for t in ins:
+        h_in[off:off + nbytes(t)].copy_(t.reshape(-1).view(torch.uint8).cpu())
+        off += nbytes(t)
+    h_out = [torch.empty(out_bytes, dtype=torch.uint8, pin_memory=True) for _ in range(2)]
+
+    def carve(buf, like):
+        views, off = [], 0
+        for t in like:
+            views.append(buf[off:off + nbytes(t)].view(t.dtype).view(t.shape))
+            off += nbytes(t)
+        return views
+
+    slots = []
+    for _ in range(2):
+        d_in = torch.empty(in_bytes, dtype=torch.uint8, device=dev)
+        d_out = torch.empty(out_bytes, dtype=torch.uint8, device=dev)
+        it_in = iter(carve(d_in, ins))
+        sq = [None if t is None else next(it_in) for t in q_idx]
+        sw = [None if t is None else next(it_in) for t in w_idx]
+        sm = [next(it_in) for _ in q_main]
+        so = carve(d_out, out)
+        d_in.copy_(h_in)
+        group.step(sq, sw, sm, so)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            group.step(sq, sw, sm, so)
+        slots.append((d_in, d_out, g))
+    comp = torch.cuda.current_stream(dev)
+    up, down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    in_ready = [torch.cuda.Event() for _ in range(2)]
+    done = [torch.cuda.Event() for _ in range(2)]
+    out_read = [torch.cuda.Event() for _ in range(2)]
+    a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for it in range(args.warmup + args.steps):
+        sl = it % 2
+        if it == args.warmup:
+            torch.cuda.synchronize()
+            if world > 1:
+                dist.barrier()
+            a0.record(comp)
+            up.wait_event(a0)
+        d_in, d_out, g = slots[sl]
+        with torch.cuda.stream(up):
+            if it >= 2:
+                up.wait_event(done[sl])          # step it-2 is done with this slot's inputs
+            d_in.copy_(h_in, non_blocking=True)
+            in_ready[sl].record(up)
+        comp.wait_event(in_ready[sl])
+        if it >= 2:
+            comp.wait_event(out_read[sl])        # step it-2's outputs have been read back
+        g.replay()
+        done[sl].record(comp)
+        with torch.cuda.stream(down):
+            down.wait_event(done[sl])
+            h_out[sl].copy_(d_out, non_blocking=True)
+            out_read[sl].record(down)
+    comp.wait_stream(down)
+    a1.record(comp)
+    torch.cuda.synchronize()
+    pipelined = a0.elapsed_time(a1) / args.steps
+    # the same copies and step back to back, with a host synchronisation per
+    # step (no overlap): reported beside the pipelined figure
+    d_in, d_out, g = slots[0]
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    a0.record(comp)
+    for _ in range(args.steps):
+        d_in.copy_(h_in, non_blocking=True)
+        g.replay()
+        h_out[0].copy_(d_out, non_blocking=True)
+        comp.synchronize()
+    a1.record(comp)
+    torch.cuda.synchronize()
+    del slots
+    return pipelined, a0.elapsed_time(a1) / args.steps
 
 
 def max_over_ranks(x: float, dev, world: int) -> float:
