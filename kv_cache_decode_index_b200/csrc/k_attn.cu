@@ -82,6 +82,10 @@ __device__ __forceinline__ void bulk_commit_and_wait_read() {
   asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
 }
 
+// Column (float index) of dim c of head h in a swizzled [H][kODims] fp32
+// slice: the 16-byte granule index is XORed with h % 8.
+__device__ __forceinline__ int attn_swz(int h, int c) { return (((c >> 2) ^ (h & 7)) << 2) | (c & 3); }
+
 __device__ __forceinline__ uint32_t swz(uint32_t row, uint32_t chunk) {   // 16-byte chunk of a 1 KB row
   return row * kRowBytes + ((chunk ^ (row & 7u)) << 4);
 }
@@ -384,9 +388,13 @@ __global__ void __launch_bounds__(kAThreads, 1)
       const int col = dg * L::DW + i * 8 + 2 * (lane & 3);
       const int owner = col / kODims, cd = col % kODims;
       if (owner / L::per_round != round) continue;
-      float* dst = stage + ((owner % L::per_round) * H + ht * 16 + r0) * kODims + cd;
-      *reinterpret_cast<float2*>(dst) = make_float2(o_acc[i][0], o_acc[i][1]);
-      *reinterpret_cast<float2*>(dst + 8 * kODims) = make_float2(o_acc[i][2], o_acc[i][3]);
+      // 16-byte granules of a head's row XOR-swizzled by the head (the same
+      // layout is read back by the owner), so the 8 rows a warp writes at once
+      // fall in different banks
+      const int h0 = ht * 16 + r0, h1 = h0 + 8;
+      float* row = stage + (owner % L::per_round) * H * kODims;
+      *reinterpret_cast<float2*>(row + h0 * kODims + attn_swz(h0, cd)) = make_float2(o_acc[i][0], o_acc[i][1]);
+      *reinterpret_cast<float2*>(row + h1 * kODims + attn_swz(h1, cd)) = make_float2(o_acc[i][2], o_acc[i][3]);
     }
     fence_proxy_async_smem();
     __syncthreads();
@@ -445,7 +453,7 @@ __global__ void __launch_bounds__(kAThreads, 1)
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
     for (int r = 0; r < kACluster; ++r) {
-      const float4 v = *reinterpret_cast<const float4*>(recv + (r * H + h) * kODims + d4);
+      const float4 v = *reinterpret_cast<const float4*>(recv + (r * H + h) * kODims + attn_swz(h, d4));
       const float f = fac[r * H + h];
       acc.x += v.x * f; acc.y += v.y * f; acc.z += v.z * f; acc.w += v.w * f;
     }
