@@ -183,3 +183,34 @@ def test_group_1m_b4_full_size(csa2):
             U.assert_sorted_padded(t)
             assert (t >= 0).sum() == 512 and set(t.tolist()) <= pool_pos
     assert csa2.get_error(cache)[0] == csa2.OK
+
+
+def test_group_graph_replay_matches_eager(csa2):
+    """The bench times CUDA-graph replays of the step (side streams and
+    programmatic dependent launch inside the graph); a replay must give the
+    eager step's indices and outputs exactly, twice in a row."""
+    wl = W.WORKLOADS["group_64k_b8"]
+    cache = U.build_cache(wl, csa2)
+    dev = cache.device
+    group, q_idx, w_idx, q_main, out = _run_gpu(csa2, wl, cache, dev)
+    ref_topk = [t.clone() for t in group.topk]
+    ref_pool = group.pool.clone()
+    ref_out = [o.clone() for o in out]
+    _, _, _, tq, tw, tm = _queries(wl, dev)
+    g_out = [torch.empty_like(m) for m in tm]
+    group.step(tq, tw, tm, g_out)   # warm-up outside capture
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        group.step(tq, tw, tm, g_out)
+    for _ in range(2):
+        for t in g_out:
+            t.zero_()
+        graph.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(group.pool, ref_pool)
+        for layer in range(len(wl.modes)):
+            assert torch.equal(group.topk[layer], ref_topk[layer]), f"topk layer {layer}"
+            assert torch.equal(g_out[layer], ref_out[layer]), f"attention layer {layer}"
+    del graph
+    assert csa2.get_error(cache)[0] == csa2.OK
