@@ -31,8 +31,8 @@ from __future__ import annotations
 
 import numpy as np
 
-from .formats import (dequantize_main_kv, e4m3_value, indexer_sigma,
-                      quantize_indexer)
+from .formats import (dequantize_indexer, dequantize_main_kv, e4m3_value,
+                      indexer_sigma, quantize_indexer)
 
 INDEX_HEADS = 32
 BLOCK = 8            # positions per pool block
@@ -229,3 +229,44 @@ def compress_tokens(x, m: int) -> np.ndarray:
     for j in range(1, m):
         acc += g[:, j, :]
     return (acc / m).astype(np.float32)
+
+
+# ------------------------------------------------------- sliding window (SWA) --
+
+def swa_tokens(p: int, window: int) -> np.ndarray:
+    """Tokens of the local window of the query at token p: the last `window`
+    tokens up to and including p (reading: the pages say every layer, Reuse
+    layers included, keeps its own local SWA state [4sapi blog, section 二],
+    but give no window size)."""
+    return np.arange(max(0, p - window + 1), p + 1, dtype=np.int64)
+
+
+def swa_quantize(x):
+    """SWA KV rows x[..., 512] (fp32) -> FP8 E4M3 codes and one power-of-two
+    scale byte per row.  The pages keep the precision-sensitive local SWA KV in
+    FP8 [4sapi blog, section 五]; reading: the indexer's per-row rule."""
+    return quantize_indexer(x)
+
+
+def sparse_attention_swa(q_main, kv_codes, kv_scales, idx, swa_codes, swa_exp, scale: float) -> np.ndarray:
+    """Sparse attention over the Top-k rows merged with the local window:
+    reading (the pages state no merge rule) -- one softmax over the union of the
+    dequantised Top-k rows (FP4 main KV, rows idx >= 0) and the window rows
+    (FP8 SWA KV, swa_codes / swa_exp [n_window, 512] / [n_window]); K = V for
+    both.  Returns float64 [H, 512]; no key at all gives o = 0."""
+    q = np.asarray(q_main, dtype=np.float64)
+    idx = np.asarray(idx, dtype=np.int64)
+    idx = idx[idx >= 0]
+    parts = []
+    if len(idx):
+        parts.append(dequantize_main_kv(kv_codes[idx], kv_scales[idx]))
+    if len(swa_exp):
+        parts.append(dequantize_indexer(swa_codes, swa_exp))
+    if not parts:
+        return np.zeros_like(q)
+    rows = np.concatenate(parts)
+    logits = (q @ rows.T) * scale
+    logits -= logits.max(axis=1, keepdims=True)
+    p = np.exp(logits)
+    p /= p.sum(axis=1, keepdims=True)
+    return p @ rows

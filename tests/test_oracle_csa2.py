@@ -276,3 +276,64 @@ def test_compress_tokens_is_the_exact_mean_rounded_once():
     np.testing.assert_array_equal(C.compress_tokens(rep, 4), x)          # identical tokens
     with pytest.raises(ValueError):
         C.compress_tokens(np.zeros((6, 4), np.float32), 3)
+
+
+# ------------------------------------------------------- sliding window ------
+
+def _swa_case(rng, n_main=40, n_win=9, H=4):
+    x = (rng.standard_normal((n_main, 512)) * 2).astype(np.float32)
+    codes, scales = F.quantize_main_kv(x)
+    y = rng.standard_normal((n_win, 512)).astype(np.float32)
+    sc, se = C.swa_quantize(y)
+    q = rng.standard_normal((H, 512))
+    return codes, scales, sc, se, q
+
+
+def test_swa_window_tokens():
+    np.testing.assert_array_equal(C.swa_tokens(10, 4), [7, 8, 9, 10])
+    np.testing.assert_array_equal(C.swa_tokens(2, 8), [0, 1, 2])        # the window starts at token 0
+    assert len(C.swa_tokens(1000, 128)) == 128
+
+
+def test_swa_attention_is_the_softmax_merge_of_its_two_parts():
+    # pinned by the identity of a softmax over a union of two key sets:
+    # o = (L1 o1 + L2 o2) / (L1 + L2) with L_i = sum_j exp(logit_j) of part i,
+    # where o1 is the (separately pinned) sparse attention over the Top-k rows
+    # and o2 a plain softmax attention over the window rows
+    rng = np.random.default_rng(8)
+    codes, scales, sc, se, q = _swa_case(rng)
+    idx = np.array([3, 17, -1, 25, 0, 39])
+    scale = 0.04
+    got = C.sparse_attention_swa(q, codes, scales, idx, sc, se, scale)
+    k1 = F.dequantize_main_kv(codes[[3, 17, 25, 0, 39]], scales[[3, 17, 25, 0, 39]])
+    k2 = F.e4m3_value(sc) * np.ldexp(1.0, se.astype(np.int64) - 127)[:, None]
+    l1, l2 = q @ k1.T * scale, q @ k2.T * scale
+    m = np.maximum(l1.max(1), l2.max(1))[:, None]
+    L1, L2 = np.exp(l1 - m).sum(1)[:, None], np.exp(l2 - m).sum(1)[:, None]
+    o1 = C.sparse_attention(q, codes, scales, idx, scale)
+    o2 = (np.exp(l2 - m) @ k2) / L2
+    np.testing.assert_allclose(got, (L1 * o1 + L2 * o2) / (L1 + L2), rtol=1e-12, atol=1e-12)
+    # special cases: no window -> the sparse attention; no Top-k -> the window alone
+    np.testing.assert_allclose(C.sparse_attention_swa(q, codes, scales, idx, sc[:0], se[:0], scale),
+                               C.sparse_attention(q, codes, scales, idx, scale), rtol=1e-14, atol=1e-15)
+    np.testing.assert_allclose(C.sparse_attention_swa(q, codes, scales, np.array([-1]), sc, se, scale), o2,
+                               rtol=1e-12, atol=1e-12)
+    # one key in all: o = that key
+    np.testing.assert_allclose(C.sparse_attention_swa(q, codes, scales, np.array([-1]), sc[:1], se[:1], scale),
+                               np.repeat(k2[:1], len(q), 0), rtol=1e-14)
+
+
+def test_swa_quantize_is_the_per_row_fp8_rule():
+    # the same per-row power-of-two FP8 rule as the indexer rows, on 512-d rows:
+    # every code decodes within half an E4M3 step of x / sigma, and sigma is the
+    # smallest power of two with 448 * sigma >= max |row|
+    rng = np.random.default_rng(3)
+    y = (rng.standard_normal((20, 512)) * np.exp(rng.normal(0, 3, (20, 1)))).astype(np.float32)
+    sc, se = C.swa_quantize(y)
+    sigma = np.ldexp(1.0, se.astype(np.int64) - 127)
+    amax = np.abs(y.astype(np.float64)).max(1)
+    assert np.all(448 * sigma >= amax) and np.all(448 * sigma / 2 < amax)
+    v = F.e4m3_value(sc)
+    r = y / sigma[:, None]
+    step = np.ldexp(1.0, np.floor(np.log2(np.maximum(np.abs(r), 2.0 ** -6))).astype(np.int64) - 3)
+    assert np.all(np.abs(v - r) <= step / 2 + 1e-12)

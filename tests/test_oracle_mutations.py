@@ -152,3 +152,15 @@ def test_mutation_compressor_drops_a_token(monkeypatch):
         return (g[:, : max(m - 1, 1), :].sum(axis=1) / m).astype(np.float32)
     monkeypatch.setattr(C, "compress_tokens", wrong)
     _fails(PC.test_compress_tokens_is_the_exact_mean_rounded_once)
+
+
+def test_mutation_swa_merge_by_halves(monkeypatch):
+    # a plausible wrong merge rule: the average of the two separate attentions
+    def wrong(q_main, kv_codes, kv_scales, idx, swa_codes, swa_exp, scale):
+        o1 = C.sparse_attention(q_main, kv_codes, kv_scales, idx, scale)
+        k2 = F.e4m3_value(swa_codes) * np.ldexp(1.0, np.asarray(swa_exp, np.int64) - 127)[:, None]
+        lg = np.asarray(q_main, np.float64) @ k2.T * scale
+        p = np.exp(lg - lg.max(1, keepdims=True))
+        return 0.5 * o1 + 0.5 * (p / p.sum(1, keepdims=True)) @ k2
+    monkeypatch.setattr(C, "sparse_attention_swa", wrong)
+    _fails(PC.test_swa_attention_is_the_softmax_merge_of_its_two_parts)
