@@ -302,6 +302,39 @@ CSA2_API csa2_status csa2_sparse_attn_layers(const csa2_cache* cache, int32_t n_
                                              uint16_t* const* out, void* stream);
 
 /*
+ * Sliding-window (SWA) branch.  Every layer, Reuse layers included, keeps its
+ * own local KV of the most recent tokens, in FP8 where the global KV is FP4
+ * [4sapi blog, section 二 (Reuse layers keep their own SWA state) and section
+ * 五 (the local SWA KV stays FP8)].  The window size and the way the window
+ * is merged with the sparse attention are not on the pages; the readings:
+ * the window is the last `window` tokens up to and including the query's
+ * own; its rows are FP8 E4M3 with one power-of-two scale per row (the
+ * indexer's rule); attention takes one softmax over the union of the Top-k
+ * rows and the window rows (K = V for both).
+ * Layout (one layer): swa_codes uint8 [batch][window][512], swa_exp uint8
+ * [batch][window]; token t of request b lives in slot t % window.
+ *
+ * csa2_swa_append -- quantise n_rows SWA rows and store them in their slots.
+ *   x    float [n_rows][512];  req int32 [n_rows] or NULL (row i -> request i);
+ *   pos  int32 [n_rows] token positions.
+ * Device errors: req outside [0, batch) or pos < 0 -> CSA2_ERR_DEVICE_BOUNDS.
+ *
+ * csa2_sparse_attn_swa -- csa2_sparse_attn of one layer with its window merged
+ * in: query i attends over its Top-k rows and the window tokens
+ * max(0, q_pos[i] - window + 1) .. q_pos[i] of its request (q_pos int32
+ * [n_queries], device).  window in [1, CSA2_SWA_MAX_WINDOW].
+ */
+#define CSA2_SWA_MAX_WINDOW 4096
+CSA2_API csa2_status csa2_swa_append(const csa2_cache* cache, int32_t window, uint8_t* swa_codes,
+                                     uint8_t* swa_exp, int32_t n_rows, const float* x, const int32_t* req,
+                                     const int32_t* pos, void* stream);
+CSA2_API csa2_status csa2_sparse_attn_swa(const csa2_cache* cache, int32_t n_queries, const int32_t* q_req,
+                                          const int32_t* topk, int32_t k, const uint8_t* swa_codes,
+                                          const uint8_t* swa_exp, int32_t window, const int32_t* q_pos,
+                                          const uint16_t* q, int32_t H, float scale, uint16_t* out,
+                                          void* stream);
+
+/*
  * csa2_get_error -- synchronise `stream`, copy cache->err_word to the host
  * array out[4] (host pointer) and return out[0] as a status (CSA2_OK when no
  * device error was recorded).  Does not clear the word.

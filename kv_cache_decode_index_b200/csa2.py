@@ -44,6 +44,8 @@ _sig = {
     "csa2_reindex": [_CP, _I, _P, _I, _P, _P, _P, _P, _I, _P, _P],
     "csa2_sparse_attn": [_CP, _I, _P, _P, _I, _P, _I, ctypes.c_float, _P, _P],
     "csa2_sparse_attn_layers": [_CP, _I, _I, _P, _P, _I, _P, _I, ctypes.c_float, _P, _P],
+    "csa2_swa_append": [_CP, _I, _P, _P, _I, _P, _P, _P, _P],
+    "csa2_sparse_attn_swa": [_CP, _I, _P, _P, _I, _P, _P, _I, _P, _P, _I, ctypes.c_float, _P, _P],
     "csa2_prefill_index": [_CP, _I, _I, _P, _I, _P, _P, _I, _P, _P, ctypes.c_size_t, _P],
     "csa2_prefill_index_static": [_CP, _I, _I, _P, _I, _P, _P, _I, _P, _P],
     "csa2_get_error": [_CP, ctypes.POINTER(ctypes.c_int32), _P],
@@ -286,6 +288,46 @@ def sparse_attn_layers(cache: Cache, topk, q_layers, scale: float | None = None,
     _check(_lib.csa2_sparse_attn_layers(ctypes.byref(cache.struct), L, n, _ptr(q_req), _ptr(topk), k, qa, H,
                                         ctypes.c_float(scale), oa, _stream(cache.device)), "csa2_sparse_attn_layers")
     return out_layers
+
+
+class SwaKV:
+    """One layer's sliding-window KV: FP8 rows in a ring of `window` slots per
+    request (codes uint8 [batch, window, 512], exponent bytes [batch, window])."""
+
+    def __init__(self, cache: Cache, window: int):
+        self.window = int(window)
+        self.codes = torch.zeros(cache.batch, self.window, KV_DIM, dtype=torch.uint8, device=cache.device)
+        self.exp = torch.zeros(cache.batch, self.window, dtype=torch.uint8, device=cache.device)
+
+
+def swa_append(cache: Cache, swa: SwaKV, x, pos, req=None):
+    """Quantise SWA rows x float32 [n, 512] and store token pos[i] in slot pos[i] % window."""
+    n = pos.shape[0]
+    _need(x, torch.float32, (n, KV_DIM), "x")
+    _need(pos, torch.int32, (n,), "pos")
+    if req is not None:
+        _need(req, torch.int32, (n,), "req")
+    _check(_lib.csa2_swa_append(ctypes.byref(cache.struct), swa.window, _ptr(swa.codes), _ptr(swa.exp), n, _ptr(x),
+                                _ptr(req), _ptr(pos), _stream(cache.device)), "csa2_swa_append")
+
+
+def sparse_attn_swa(cache: Cache, topk, swa: SwaKV, q_pos, q, scale: float | None = None, out=None, q_req=None):
+    """Sparse attention with the query's window (tokens q_pos-window+1 .. q_pos) merged in."""
+    n, k = topk.shape
+    H = q.shape[1]
+    _need(topk, torch.int32, (n, k), "topk")
+    _need(q_pos, torch.int32, (n,), "q_pos")
+    _need(q, torch.bfloat16, (n, H, KV_DIM), "q")
+    if q_req is not None:
+        _need(q_req, torch.int32, (n,), "q_req")
+    if out is None:
+        out = torch.empty_like(q)
+    _need(out, torch.bfloat16, (n, H, KV_DIM), "out")
+    scale = 1.0 / math.sqrt(KV_DIM) if scale is None else scale
+    _check(_lib.csa2_sparse_attn_swa(ctypes.byref(cache.struct), n, _ptr(q_req), _ptr(topk), k, _ptr(swa.codes),
+                                     _ptr(swa.exp), swa.window, _ptr(q_pos), _ptr(q), H, ctypes.c_float(scale),
+                                     _ptr(out), _stream(cache.device)), "csa2_sparse_attn_swa")
+    return out
 
 
 def get_error(cache: Cache):

@@ -267,6 +267,52 @@ csa2_status csa2_sparse_attn(const csa2_cache* cache, int32_t n_queries, const i
   return sparse_attn_impl(cache, 1, n_queries, q_req, topk, k, qs, H, scale, os, stream);
 }
 
+csa2_status csa2_swa_append(const csa2_cache* cache, int32_t window, uint8_t* swa_codes, uint8_t* swa_exp,
+                            int32_t n_rows, const float* x, const int32_t* req, const int32_t* pos, void* stream) {
+  CSA2_TRY(check_cache(cache, false, false));
+  if (window < 1 || window > CSA2_SWA_MAX_WINDOW)
+    return fail(CSA2_ERR_SHAPE, "window %d outside [1, %d]", window, CSA2_SWA_MAX_WINDOW);
+  if (n_rows < 0) return fail(CSA2_ERR_SHAPE, "n_rows %d < 0", n_rows);
+  if (n_rows == 0) return CSA2_OK;
+  if (swa_codes == nullptr || swa_exp == nullptr || x == nullptr || pos == nullptr || !aligned(swa_codes, 16) ||
+      !aligned(x, 16))
+    return fail(CSA2_ERR_ARG, "swa_codes (16-byte aligned), swa_exp, x (16-byte aligned) and pos must be set");
+  if (req == nullptr && n_rows > cache->batch)
+    return fail(CSA2_ERR_SHAPE, "without req, n_rows (%d) must not exceed batch (%d)", n_rows, cache->batch);
+  DeviceInfo d;
+  CSA2_TRY(device_info(&d));
+  const cudaError_t e = csa2::launch_swa_append(*cache, window, swa_codes, swa_exp, n_rows, x, req, pos,
+                                                static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? CSA2_OK : cuda_fail(e, "swa_append launch");
+}
+
+csa2_status csa2_sparse_attn_swa(const csa2_cache* cache, int32_t n_queries, const int32_t* q_req,
+                                 const int32_t* topk, int32_t k, const uint8_t* swa_codes, const uint8_t* swa_exp,
+                                 int32_t window, const int32_t* q_pos, const uint16_t* q, int32_t H, float scale,
+                                 uint16_t* out, void* stream) {
+  CSA2_TRY(check_cache(cache, true, false));
+  if (window < 1 || window > CSA2_SWA_MAX_WINDOW)
+    return fail(CSA2_ERR_SHAPE, "window %d outside [1, %d]", window, CSA2_SWA_MAX_WINDOW);
+  if (swa_codes == nullptr || swa_exp == nullptr || q_pos == nullptr || !aligned(swa_codes, 16))
+    return fail(CSA2_ERR_ARG, "swa_codes (16-byte aligned), swa_exp and q_pos must be set");
+  if (n_queries < 0) return fail(CSA2_ERR_SHAPE, "n_queries %d < 0", n_queries);
+  if (n_queries == 0) return CSA2_OK;
+  if (q_req == nullptr && n_queries > cache->batch)
+    return fail(CSA2_ERR_SHAPE, "without q_req, n_queries (%d) must not exceed batch (%d)", n_queries, cache->batch);
+  if (H != 16 && H != 32 && H != 64) return fail(CSA2_ERR_SHAPE, "H %d not in {16, 32, 64}", H);
+  if (k < 1 || k > kMaxK) return fail(CSA2_ERR_SHAPE, "k %d outside [1, %d]", k, kMaxK);
+  if (topk == nullptr || q == nullptr || out == nullptr || !aligned(q, 16) || !aligned(out, 16))
+    return fail(CSA2_ERR_ARG, "topk, q and out (16-byte aligned) must be set");
+  DeviceInfo d;
+  CSA2_TRY(device_info(&d));
+  const uint16_t* qs[1] = {q};
+  uint16_t* os[1] = {out};
+  const cudaError_t e = csa2::launch_sparse_attn(*cache, 1, n_queries, q_req, topk, k, qs, H, scale, os,
+                                                 static_cast<cudaStream_t>(stream), swa_codes, swa_exp, q_pos,
+                                                 window);
+  return e == cudaSuccess ? CSA2_OK : cuda_fail(e, "sparse_attn_swa launch");
+}
+
 csa2_status csa2_sparse_attn_layers(const csa2_cache* cache, int32_t n_layers, int32_t n_queries,
                                     const int32_t* q_req, const int32_t* topk, int32_t k, const uint16_t* const* q,
                                     int32_t H, float scale, uint16_t* const* out, void* stream) {

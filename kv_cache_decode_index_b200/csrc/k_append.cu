@@ -121,7 +121,56 @@ __global__ void __launch_bounds__(256) compress_append_kernel(csa2_cache cache, 
   quantize_store(cache, row, x, k, lane);
 }
 
+// Sliding-window (SWA) KV append: one warp per row; the 512-d row is stored
+// in FP8 E4M3 with one power-of-two scale, by the indexer's per-row rule, in
+// ring slot pos % window of its request [4sapi blog, section 五: the local
+// SWA KV stays in FP8].
+__global__ void __launch_bounds__(256) swa_append_kernel(csa2_cache cache, int window, uint8_t* __restrict__ codes,
+                                                         uint8_t* __restrict__ exps, int n_rows,
+                                                         const float* __restrict__ x, const int32_t* __restrict__ req,
+                                                         const int32_t* __restrict__ pos) {
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (warp >= n_rows) return;
+  const int b = req ? req[warp] : warp;
+  const int t = pos[warp];
+  if (b < 0 || b >= cache.batch || t < 0) {
+    if (lane == 0) report_error(cache.err_word, CSA2_ERR_DEVICE_BOUNDS, kKAppend, b, t);
+    return;
+  }
+  const float4* src = reinterpret_cast<const float4*>(x + static_cast<long long>(warp) * kKvDim) + lane * 4;
+  float v[16];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float4 f = src[i];
+    v[4 * i] = f.x; v[4 * i + 1] = f.y; v[4 * i + 2] = f.z; v[4 * i + 3] = f.w;
+  }
+  float m = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) m = fmaxf(m, fabsf(v[i]));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  const int e = indexer_exponent(m);
+  const float inv = exp2i(-e);
+  uint32_t w[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    w[i] = e4m3x2(v[4 * i] * inv, v[4 * i + 1] * inv) | (e4m3x2(v[4 * i + 2] * inv, v[4 * i + 3] * inv) << 16);
+  const long long slot = static_cast<long long>(b) * window + t % window;
+  reinterpret_cast<uint4*>(codes + slot * kKvDim)[lane] = make_uint4(w[0], w[1], w[2], w[3]);
+  if (lane == 0) exps[slot] = static_cast<uint8_t>(e + 127);
+}
+
 }  // namespace
+
+cudaError_t launch_swa_append(const csa2_cache& cache, int window, uint8_t* swa_codes, uint8_t* swa_exp, int n_rows,
+                              const float* x, const int32_t* req, const int32_t* pos, cudaStream_t stream) {
+  const int threads = 256;
+  const long long blocks = (static_cast<long long>(n_rows) * 32 + threads - 1) / threads;
+  swa_append_kernel<<<static_cast<unsigned>(blocks), threads, 0, stream>>>(cache, window, swa_codes, swa_exp, n_rows,
+                                                                          x, req, pos);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_compress_append(const csa2_cache& cache, int n_entries, int m, const float* kv_tok,
                                    const float* ik_tok, const int32_t* req, const int32_t* pos, cudaStream_t stream) {

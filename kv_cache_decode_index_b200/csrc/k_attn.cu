@@ -139,10 +139,21 @@ struct AttnLayers {
   __nv_bfloat16* out[CSA2_ATTN_MAX_LAYERS];
 };
 
+// The local sliding window (SWA) merged into the attention: FP8 E4M3 rows
+// with one power-of-two scale each, a ring of `window` slots per request
+// (token t in slot t % window); codes == nullptr: no window.
+struct SwaArgs {
+  const uint8_t* codes;      // [batch][window][512]
+  const uint8_t* exp;        // [batch][window]
+  const int32_t* q_pos;      // [n_queries] token position of each query
+  int window;
+};
+
 template <int H>
 __global__ void __launch_bounds__(kAThreads, 1)
     sparse_attn_kernel(const csa2_cache cache, int n_queries, const int32_t* __restrict__ q_req,
-                       const int32_t* __restrict__ topk, int K, const AttnLayers io, float softmax_scale) {
+                       const int32_t* __restrict__ topk, int K, const AttnLayers io, float softmax_scale,
+                       const SwaArgs swa) {
   using L = AttnLayout<H>;
   extern __shared__ __align__(1024) uint8_t smem[];
   const uint32_t sbase = smem_u32(smem);
@@ -213,9 +224,12 @@ __global__ void __launch_bounds__(kAThreads, 1)
     if (lane == 0) qscale[h] = softmax_scale * down * kLog2e;
   }
 
-  // ---- this CTA's keys ----
-  const int kc = (K + kACluster - 1) / kACluster;
-  const int key_begin = min(rank * kc, K), key_end = min(key_begin + kc, K);
+  // ---- this CTA's keys: the Top-k entries, then the window's tokens ----
+  const int n_win = swa.codes != nullptr ? swa.window : 0;
+  const int p_tok = n_win > 0 ? swa.q_pos[qi] : 0;
+  const int K_all = K + n_win;
+  const int kc = (K_all + kACluster - 1) / kACluster;
+  const int key_begin = min(rank * kc, K_all), key_end = min(key_begin + kc, K_all);
 
   float o_acc[L::DW / 8][4];
 #pragma unroll
@@ -229,6 +243,41 @@ __global__ void __launch_bounds__(kAThreads, 1)
     {
       // gather + dequantise: 4 threads per row, 128 channels each
       const int row = tid >> 2, part = tid & 3;
+      if (row < nk && c0 + row >= K) {
+        // window entry j: token p - window + 1 + j (none before token 0)
+        const int tw = p_tok - n_win + 1 + (c0 + row - K);
+        const bool ok = tw >= 0 && b >= 0 && b < cache.batch;
+        if (part == 0) kvalid[row] = ok;
+        if (ok) {
+          const long long slot = static_cast<long long>(b) * n_win + tw % n_win;
+          const uint4* cp = reinterpret_cast<const uint4*>(swa.codes + slot * kKvDim) + part * 8;
+          const float sigma = exp2i(static_cast<int>(swa.exp[slot]) - 127);
+          uint4 cv[8];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) cv[j] = cp[j];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            // 16 E4M3 codes -> 16 fp16 values (exact while sigma keeps them in fp16's range)
+            const uint32_t w4[4] = {cv[j].x, cv[j].y, cv[j].z, cv[j].w};
+            uint32_t hv[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const uint32_t two = (w4[i >> 1] >> (16 * (i & 1))) & 0xFFFFu;
+              const uint32_t c_lo = two & 0xFFu, c_hi = two >> 8;
+              const float v_lo = (c_lo & 0x80u ? -1.0f : 1.0f) * e4m3_value(c_lo & 0x7Fu) * sigma;
+              const float v_hi = (c_hi & 0x80u ? -1.0f : 1.0f) * e4m3_value(c_hi & 0x7Fu) * sigma;
+              hv[i] = pack_half2(v_lo, v_hi);
+            }
+            const int chunk0 = part * 16 + j * 2;
+            *reinterpret_cast<uint4*>(smem + L::kv_off + swz(row, chunk0)) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
+            *reinterpret_cast<uint4*>(smem + L::kv_off + swz(row, chunk0 + 1)) = make_uint4(hv[4], hv[5], hv[6], hv[7]);
+          }
+        } else {
+#pragma unroll
+          for (int c = 0; c < 16; ++c)
+            *reinterpret_cast<uint4*>(smem + L::kv_off + swz(row, part * 16 + c)) = make_uint4(0, 0, 0, 0);
+        }
+      } else {
       int t = row < nk ? idx[c0 + row] : -1;
       long long src_row = -1;
       if (t >= 0 && t < n) {
@@ -257,6 +306,7 @@ __global__ void __launch_bounds__(kAThreads, 1)
 #pragma unroll
         for (int c = 0; c < 16; ++c)
           *reinterpret_cast<uint4*>(smem + L::kv_off + swz(row, part * 16 + c)) = make_uint4(0, 0, 0, 0);
+      }
       }
     }
     __syncthreads();
@@ -467,7 +517,7 @@ __global__ void __launch_bounds__(kAThreads, 1)
 
 template <int H>
 cudaError_t launch_h(const csa2_cache& cache, int n_layers, int n_queries, const int32_t* q_req, const int32_t* topk,
-                     int k, const AttnLayers& io, float scale, cudaStream_t stream) {
+                     int k, const AttnLayers& io, float scale, const SwaArgs& swa, cudaStream_t stream) {
   static bool done = false;
   const size_t smem = AttnLayout<H>::total;
   if (!done) {
@@ -490,23 +540,25 @@ cudaError_t launch_h(const csa2_cache& cache, int n_layers, int n_queries, const
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  return cudaLaunchKernelEx(&cfg, sparse_attn_kernel<H>, cache, n_queries, q_req, topk, k, io, scale);
+  return cudaLaunchKernelEx(&cfg, sparse_attn_kernel<H>, cache, n_queries, q_req, topk, k, io, scale, swa);
 }
 
 }  // namespace
 
 cudaError_t launch_sparse_attn(const csa2_cache& cache, int n_layers, int n_queries, const int32_t* q_req,
                                const int32_t* topk, int k, const uint16_t* const* q, int H, float scale,
-                               uint16_t* const* out, cudaStream_t stream) {
+                               uint16_t* const* out, cudaStream_t stream, const uint8_t* swa_codes,
+                               const uint8_t* swa_exp, const int32_t* q_pos, int window) {
   AttnLayers io = {};
   for (int l = 0; l < n_layers; ++l) {
     io.q[l] = reinterpret_cast<const __nv_bfloat16*>(q[l]);
     io.out[l] = reinterpret_cast<__nv_bfloat16*>(out[l]);
   }
+  const SwaArgs swa = {swa_codes, swa_exp, q_pos, window};
   switch (H) {
-    case 16: return launch_h<16>(cache, n_layers, n_queries, q_req, topk, k, io, scale, stream);
-    case 32: return launch_h<32>(cache, n_layers, n_queries, q_req, topk, k, io, scale, stream);
-    case 64: return launch_h<64>(cache, n_layers, n_queries, q_req, topk, k, io, scale, stream);
+    case 16: return launch_h<16>(cache, n_layers, n_queries, q_req, topk, k, io, scale, swa, stream);
+    case 32: return launch_h<32>(cache, n_layers, n_queries, q_req, topk, k, io, scale, swa, stream);
+    case 64: return launch_h<64>(cache, n_layers, n_queries, q_req, topk, k, io, scale, swa, stream);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -44,8 +44,13 @@ cudaError_t launch_copy_topk(const int32_t* src, int32_t* dst, long long n, cuda
 
 // q[l] / out[l] (host array of device pointers): query and output of layer l
 // of n_layers layers sharing the Top-k.
+// swa_codes == nullptr: no sliding window; else the window of `window`
+// tokens ending at q_pos[i] is merged into query i's softmax.
 cudaError_t launch_sparse_attn(const csa2_cache& cache, int n_layers, int n_queries, const int32_t* q_req,
                                const int32_t* topk, int k, const uint16_t* const* q, int H, float scale,
-                               uint16_t* const* out, cudaStream_t stream);
+                               uint16_t* const* out, cudaStream_t stream, const uint8_t* swa_codes = nullptr,
+                               const uint8_t* swa_exp = nullptr, const int32_t* q_pos = nullptr, int window = 0);
+cudaError_t launch_swa_append(const csa2_cache& cache, int window, uint8_t* swa_codes, uint8_t* swa_exp, int n_rows,
+                              const float* x, const int32_t* req, const int32_t* pos, cudaStream_t stream);
 
 }  // namespace csa2

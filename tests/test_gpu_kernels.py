@@ -431,3 +431,70 @@ def test_pipeline_wait_timeout_returns_status(csa2):
     codes, exp = U.oracle_request(wl, 0, 4096)
     s64 = C.indexer_scores(q[0], w[0], codes, exp)
     assert np.all(np.abs(bm[0, :512].cpu().numpy() - C.block_max(s64, 4096)) <= 1e-5 * C.block_max(s64, 4096))
+
+
+# ------------------------------------------------------ sliding window (SWA) --
+
+def test_swa_append_bitexact(csa2):
+    rng = np.random.default_rng(61)
+    B, Wn = 3, 96
+    cache = _flat_cache(csa2, 256, batch=B, page_size=128)
+    swa = csa2.SwaKV(cache, Wn)
+    n = 250
+    x = (rng.standard_normal((n, 512)) * np.exp(rng.normal(0, 3, (n, 1)))).astype(np.float32)
+    x[5] = 0.0
+    req = rng.integers(0, B, n).astype(np.int32)
+    pos = rng.permutation(10_000)[:n].astype(np.int32)
+    # one row per (request, slot): the last writer would otherwise be ambiguous
+    _, keep = np.unique(req.astype(np.int64) * Wn + pos % Wn, return_index=True)
+    keep = np.sort(keep)
+    dev = cache.device
+    csa2.swa_append(cache, swa, torch.from_numpy(x[keep]).to(dev), torch.from_numpy(pos[keep]).to(dev),
+                    torch.from_numpy(req[keep]).to(dev))
+    codes, exp = C.swa_quantize(x[keep])
+    gc = swa.codes.cpu().numpy()[req[keep], pos[keep] % Wn]
+    ge = swa.exp.cpu().numpy()[req[keep], pos[keep] % Wn]
+    np.testing.assert_array_equal(ge, exp)
+    np.testing.assert_array_equal(gc, codes)
+    assert csa2.get_error(cache)[0] == csa2.OK
+
+
+@pytest.mark.parametrize("H,k,window", [(64, 512, 128), (16, 100, 40), (32, 512, 1)])
+def test_sparse_attention_swa_parity(csa2, H, k, window):
+    """Top-k rows of the FP4 cache merged with the query's window of FP8 SWA
+    rows, one softmax (the oracle's reading); windows that are full, cut at
+    token 0, and wrapped around the ring."""
+    rng = np.random.default_rng(70 + H + window)
+    wl = W.scaled(W.WORKLOADS["group_64k_b8"], batch=3, ctx=3000, heads=H)
+    cache = U.build_cache(wl, csa2)
+    dev = cache.device
+    swa = csa2.SwaKV(cache, window)
+    q_pos = np.array([2999, window // 3, 5 * window + 7], dtype=np.int32)   # full, partial, wrapped
+    rows = {}
+    for b in range(3):
+        # older tokens first (their slots collide with each other), then the
+        # window's tokens, which overwrite them in a later, stream-ordered call
+        p = int(q_pos[b])
+        older = np.arange(max(0, p - 3 * window), max(0, p - window + 1))
+        recent = np.arange(max(0, p - window + 1), p + 1)
+        rows[b] = {}
+        for toks in (older, recent):
+            if len(toks) == 0:
+                continue
+            y = rng.standard_normal((len(toks), 512)).astype(np.float32)
+            rows[b].update(zip(toks.tolist(), y))
+            csa2.swa_append(cache, swa, torch.from_numpy(y).to(dev), torch.from_numpy(toks.astype(np.int32)).to(dev),
+                            torch.full((len(toks),), b, dtype=torch.int32, device=dev))
+    topk = np.stack([np.sort(rng.choice(3000, k, replace=False)) for _ in range(3)]).astype(np.int32)
+    topk[1, k // 2:] = -1                                                    # a short Top-k
+    qm = W.main_query(wl, 0)
+    got = csa2.sparse_attn_swa(cache, torch.from_numpy(topk).to(dev), swa, torch.from_numpy(q_pos).to(dev),
+                               qm.to(dev), wl.scale)
+    for b in range(3):
+        sel = topk[b][topk[b] >= 0]
+        kvc, kvs = U.oracle_kv_rows(wl, b, sel)
+        toks = C.swa_tokens(int(q_pos[b]), window)
+        sc, se = C.swa_quantize(np.stack([rows[b][int(t)] for t in toks]))
+        ref = C.sparse_attention_swa(qm[b].float().numpy(), kvc, kvs, np.arange(len(sel)), sc, se, wl.scale)
+        U.assert_attention_close(got[b].float().cpu().numpy(), ref, f"swa attention b={b}")
+    assert csa2.get_error(cache)[0] == csa2.OK
