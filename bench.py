@@ -459,7 +459,7 @@ def run_prefill(args):
     gpu_id = str(torch.cuda.get_device_properties(dev).uuid)
     sampler = ClockSampler(gpu_id if gpu_id.startswith("GPU-") else f"GPU-{gpu_id}")
     sampler.start()
-    names = [f"topk{l}" for l, m in enumerate(wl.modes) if m != "Ru"] + [f"attn{l}" for l in range(len(wl.modes))]
+    names = group.launch_names()
     timing = {k: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for k in names}
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     per_launch = {k: [] for k in names}
@@ -518,11 +518,10 @@ def run_prefill(args):
                          "streaming Top-512)", "kernel_ms": idx_ms, "flops_per_launch": flops,
                          "peak_source": peak_src},
             "e2e": {"value": e2e_value, "unit": "queries/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                    "how": "DecodeGroup.step per step; one packed pinned host-to-device copy of all the step's inputs "
-                           "and one device-to-host copy of all its outputs every step, inside the timed region; two "
-                           "buffer slots and one copy stream per direction overlap step i+1's upload and step i-1's "
-                           "download with step i",
-                    "serial_value": e2e_serial},
+                    "how": "PrefillGroup.step per step; every step copies its inputs (positions, the Full layer's "
+                           "indexer query and weights, every layer's main query) from pinned host memory and its "
+                           "outputs (the Top-k and every layer's attention output) back, inside the timed region, "
+                           "in order on the calling stream"},
             "gpu_launches": group.launches_per_step * args.steps,
             "launch_ms": {k: statistics.mean(v) for k, v in per_launch.items()},
             "clocks": clocks}

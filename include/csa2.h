@@ -39,6 +39,13 @@
  *     first one in cache->err_word and skips or neutralises the offending
  *     element; csa2_get_error() reads it back.
  *   - Launch failures return CSA2_ERR_CUDA.
+ *   - Kernels are launched with programmatic dependent launch: each one waits
+ *     for the kernel before it on the stream before reading anything that
+ *     kernel may write, and lets its own successor start early.  The
+ *     attention entry points load their query rows `q` before that wait, so
+ *     q must not be written by an immediately preceding kernel that itself
+ *     signals early completion (griddepcontrol.launch_dependents); ordinary
+ *     kernels, copies and events before the call are safe.
  */
 #ifndef CSA2_H
 #define CSA2_H

@@ -483,3 +483,9 @@ class PrefillGroup:
             timed(f"attn{src}", lambda: sparse_attn_layers(c, self.topk[src], [q_main[l] for l in layers],
                                                            self.scale, [out[l] for l in layers], q_req=self.q_req))
         return out
+
+    def launch_names(self):
+        names = []
+        for layers in self.sources:
+            names += [f"topk{layers[0]}", f"attn{layers[0]}"]
+        return names

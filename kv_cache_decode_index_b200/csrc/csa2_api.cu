@@ -110,8 +110,8 @@ csa2_status check_cache(const csa2_cache* c, bool need_kv, bool need_ik) {
     return fail(CSA2_ERR_SHAPE, "num_pages * page_size must stay below 2^31 rows");
   if (capacity_of(c) >= (1LL << 31)) return fail(CSA2_ERR_SHAPE, "max_pages_per_req * page_size must stay below 2^31");
   if (need_kv && (c->kv_codes == nullptr || c->kv_scales == nullptr || !aligned(c->kv_codes, 16) ||
-                  !aligned(c->kv_scales, 8)))
-    return fail(CSA2_ERR_ARG, "kv_codes (16-byte aligned) and kv_scales (8-byte aligned) must be set");
+                  !aligned(c->kv_scales, 16)))
+    return fail(CSA2_ERR_ARG, "kv_codes and kv_scales must be set and 16-byte aligned");
   if (need_ik && (c->ik_codes == nullptr || c->ik_exp == nullptr || !aligned(c->ik_codes, 16) ||
                   !aligned(c->ik_exp, 16)))
     return fail(CSA2_ERR_ARG, "ik_codes and ik_exp must be set and 16-byte aligned");

@@ -3,22 +3,31 @@
 // blog, section 二: every layer attends over its Top-K, Reuse layers with
 // their own query; FP4 rows: 4sapi blog, section 五].
 //
-// One thread-block cluster of kACluster (4) CTAs per query.  CTA r takes
-// Top-k entries [r*kc, (r+1)*kc) (kc = ceil(k/4)) in chunks of 64 rows:
-//   * gather + dequantise: E2M1 code x E4M3 scale has <= 5 significant bits
-//     and lies in [2^-10, 2688], so the fp16 row is exact;
+// One thread-block cluster of kACluster (4) CTAs per (layer, query).  CTA r
+// takes entries [r*kc, (r+1)*kc) (kc = ceil(k/4)) in chunks of 64 rows:
+//   * prologue: the query's bf16 rows are loaded while the CTA turns its
+//     Top-k entries into cache rows (page table) once, into shared memory;
+//   * the packed rows (256 code bytes + 32 scale bytes each) are copied into
+//     a staging buffer by cp.async one chunk ahead of their use and
+//     dequantised shared -> shared with the E2M1 -> f16x2 conversion: E2M1
+//     code x E4M3 scale has <= 5 significant bits and lies in [2^-10, 2688],
+//     so the fp16 row is exact;
 //   * the query is moved to fp16 with a power-of-two scale per head (bf16 ->
 //     fp16 keeps every significant bit in the normal range);
-//   * S = Q K^T and O = P V on mma.sync m16n8k16 (fp16 in, fp32 accumulate),
-//     online softmax in fp32 (exp2 domain), P rounded to fp16;
-// then the partial (O, max, sum) triples are merged through distributed
-// shared memory: every CTA sends its slice of dims [128r, 128r+128) to CTA r
-// (bulk copies), which merges them locally and writes those dims of every
-// head.  Four CTAs per query keep all six layers' attention of a decode step
-// within one wave of the GPU's SMs.
+//   * S = Q K^T on mma.sync m16n8k16 (fp16 in, fp32 accumulate) with the
+//     chunk's keys split over the warps, an online softmax in fp32 (exp2
+//     domain) whose row maxima and sums are combined through shared memory,
+//     P rounded to fp16 in shared memory, O += P V with the 512 output dims
+//     split over the warps;
+// then every CTA stores its partial O slice of dims [128r, 128r+128) straight
+// into CTA r's shared memory (distributed shared memory) together with its
+// (max, sum) pairs, and after a cluster barrier CTA r merges the four
+// partials and writes those dims of every head.  Four CTAs per query keep all
+// six layers' attention of a decode step within one wave of the GPU's SMs.
 #include <cooperative_groups.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
+#include <cuda_fp4.h>
 
 #include "fp4.cuh"
 #include "launch.h"
@@ -30,57 +39,42 @@ namespace {
 namespace cg = cooperative_groups;
 
 constexpr int kAThreads = 256;
+constexpr int kAWarps = kAThreads / 32;
 constexpr int kACluster = 4;                 // CTAs (key splits) per query
 constexpr int kODims = kKvDim / kACluster;   // output dims owned by one CTA of the cluster
 constexpr int kChunk = 64;                   // keys per chunk
 constexpr int kRowBytes = kKvDim * 2;        // fp16 row: 1024 B
-constexpr int kSredStride = kChunk + 8;      // fp32 row stride of the S reduction buffer
+constexpr int kPRowBytes = kChunk * 2;       // fp16 row of P: 128 B
+constexpr int kCodeGran = kKvCodeBytes / 16;                    // 16-byte granules of a packed row's codes
+constexpr int kRowGran = (kKvCodeBytes + kKvScaleBytes) / 16;   // ... of codes + scales
+// Top-k entries one CTA resolves: k <= 4096 and a window <= 4096 give at most
+// ceil((4096 + 4096) / 4) entries per CTA.
+constexpr int kMaxTop = (4096 + CSA2_SWA_MAX_WINDOW + kACluster - 1) / kACluster;
 constexpr float kLog2e = 1.4426950408889634f;
 
 template <int H>
 struct AttnLayout {
-  static constexpr int HT = H / 16;            // head tiles of 16
-  static constexpr int DG = 8 / HT;            // dim groups (warps per head tile)
-  static constexpr int DW = kKvDim / DG;       // dims per warp
-  static constexpr uint32_t q_off = 0;                               // fp16 [H][512]
-  static constexpr uint32_t kv_off = q_off + H * kRowBytes;          // fp16 [64][512]
-  static constexpr uint32_t sred_off = kv_off + kChunk * kRowBytes;  // fp32 [DG][H][72]
-  static constexpr uint32_t qscale_off = sred_off + DG * H * kSredStride * 4;
-  static constexpr uint32_t ml_off = qscale_off + H * 4;             // fp32 [8 ranks][2][H]: pushed m, l
-  static constexpr uint32_t fac_off = ml_off + kACluster * 2 * H * 4; // fp32 [8][H]
-  static constexpr uint32_t kvalid_off = fac_off + kACluster * H * 4;
-  static constexpr uint32_t bar_off = (kvalid_off + kChunk * 4 + 7) & ~7u;   // receive mbarrier
-  static constexpr uint32_t total = bar_off + 8;
-  // partial-O slice sent to one owner: [H][kODims dims] fp32
-  static constexpr uint32_t slice_bytes = H * kODims * 4;
-  static constexpr uint32_t ml_bytes = 2 * H * 4;
-  // staging of the slices sent in one round and of (m, l), in the S reduction buffer
-  static constexpr int per_round = (DG * H * kSredStride * 4 - ml_bytes) / slice_bytes >= 2 ? 2 : 1;
-  static_assert(per_round * slice_bytes + ml_bytes <= DG * H * kSredStride * 4, "staging must fit");
-  static_assert(kACluster % per_round == 0, "owners per round must divide the cluster");
+  static constexpr int HT = H / 16;            // head tiles of 16 query rows
+  static constexpr int KG = kAWarps / HT;      // key groups in S = dim groups in P V
+  static constexpr int KW = kChunk / KG;       // keys per warp in S
+  static constexpr int NT = KW / 8;            // 8-key tiles per warp in S
+  static constexpr int DW = kKvDim / KG;       // output dims per warp in P V
+  static constexpr uint32_t q_off = 0;                                     // fp16 [H][512]
+  static constexpr uint32_t kv_off = q_off + H * kRowBytes;                // fp16 [64][512]
+  static constexpr uint32_t raw_off = kv_off + kChunk * kRowBytes;         // u8 [64][256] codes
+  static constexpr uint32_t raw_scale_off = raw_off + kChunk * kKvCodeBytes;   // u8 [64][32] scales
+  static constexpr uint32_t p_off = raw_scale_off + kChunk * kKvScaleBytes;    // fp16 [H][64]
+  static constexpr uint32_t red_off = p_off + H * kPRowBytes;              // fp32 [2][KG][H]: row max, row sum
+  static constexpr uint32_t qscale_off = red_off + 2 * KG * H * 4;
+  static constexpr uint32_t kvalid_off = qscale_off + H * 4;               // int [64]
+  static constexpr uint32_t srow_off = kvalid_off + kChunk * 4;            // int32 [kMaxTop] cache rows
+  static constexpr uint32_t ml_off = srow_off + kMaxTop * 4;               // fp32 [kACluster][2][H]: m, l
+  static constexpr uint32_t fac_off = ml_off + kACluster * 2 * H * 4;      // fp32 [kACluster][H]
+  static constexpr uint32_t total = fac_off + kACluster * H * 4;
   // received partial O: [kACluster source ranks][H][kODims dims] fp32, over the Q + KV region
-  static_assert(kACluster * H * kODims * 4 <= sred_off, "received partials must fit in the Q + KV region");
+  static_assert(kACluster * H * kODims * 4 <= raw_off, "received partials must fit in the Q + KV region");
+  static_assert(KW % 8 == 0 && (NT == 1 || NT % 2 == 0), "whole 8-key tiles per warp");
 };
-
-// Address of the same shared-memory offset in CTA `rank` of the cluster.
-__device__ __forceinline__ uint32_t mapa_rank(uint32_t addr, int rank) {
-  uint32_t r;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
-  return r;
-}
-// Bulk copy of `bytes` from this CTA's shared memory to another CTA's (no
-// multicast); completion is counted on that CTA's mbarrier.
-__device__ __forceinline__ void bulk_copy_to_rank(uint32_t dst_cluster, uint32_t src_cta, uint32_t bytes,
-                                                  uint32_t bar_cluster) {
-  asm volatile("cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-                   dst_cluster),
-               "r"(src_cta), "r"(bytes), "r"(bar_cluster)
-               : "memory");
-}
-__device__ __forceinline__ void bulk_commit_and_wait_read() {
-  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
-}
 
 // Column (float index) of dim c of head h in a swizzled [H][kODims] fp32
 // slice: the 16-byte granule index is XORed with h % 8.
@@ -89,11 +83,17 @@ __device__ __forceinline__ int attn_swz(int h, int c) { return (((c >> 2) ^ (h &
 __device__ __forceinline__ uint32_t swz(uint32_t row, uint32_t chunk) {   // 16-byte chunk of a 1 KB row
   return row * kRowBytes + ((chunk ^ (row & 7u)) << 4);
 }
+__device__ __forceinline__ uint32_t pswz(uint32_t row, uint32_t chunk) {  // 16-byte chunk of a 128 B row of P
+  return row * kPRowBytes + ((chunk ^ (row & 7u)) << 4);
+}
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
                : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
                : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x2(uint32_t addr, uint32_t& r0, uint32_t& r1) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0,%1}, [%2];" : "=r"(r0), "=r"(r1) : "r"(addr));
 }
 __device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
@@ -112,6 +112,17 @@ __device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
   const __half2 h = __floats2half2_rn(lo, hi);
   return *reinterpret_cast<const uint32_t*>(&h);
 }
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
+// Two E2M1 codes (low nibble = even channel) -> f16x2, low half = even channel.
+__device__ __forceinline__ uint32_t e2m1x2_half2(uint32_t byte) {
+  const __half2_raw r = __nv_cvt_fp4x2_to_halfraw2(static_cast<__nv_fp4x2_storage_t>(byte & 0xFFu), __NV_E2M1);
+  return static_cast<uint32_t>(r.x) | (static_cast<uint32_t>(r.y) << 16);
+}
 
 // Dequantise 16 code bytes (32 channels, 2 scale groups) into 4 fp16 chunks.
 __device__ __forceinline__ void dequant16(uint4 codes, uint32_t s01, uint4 (&out)[4]) {
@@ -122,8 +133,7 @@ __device__ __forceinline__ void dequant16(uint4 codes, uint32_t s01, uint4 (&out
   uint32_t h[16];
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
-    const uint32_t byte = (w[i >> 2] >> (8 * (i & 3))) & 0xFFu;
-    const uint32_t pair = e2m1_half_bits(byte & 0xFu) | (static_cast<uint32_t>(e2m1_half_bits(byte >> 4)) << 16);
+    const uint32_t pair = e2m1x2_half2(w[i >> 2] >> (8 * (i & 3)));
     __half2 v = *reinterpret_cast<const __half2*>(&pair);
     v = __hmul2(v, i < 8 ? s0 : s1);   // exact: <= 5 significant bits, inside fp16's normal range
     h[i] = *reinterpret_cast<const uint32_t*>(&v);
@@ -150,44 +160,33 @@ struct SwaArgs {
 };
 
 template <int H>
-__global__ void __launch_bounds__(kAThreads, 1)
+__global__ void __launch_bounds__(kAThreads, H == 16 ? 2 : 1)
     sparse_attn_kernel(const csa2_cache cache, int n_queries, const int32_t* __restrict__ q_req,
-                       const int32_t* __restrict__ topk, int K, const AttnLayers io, float softmax_scale,
+                       const int32_t* __restrict__ topk, int K, const __grid_constant__ AttnLayers io, float softmax_scale,
                        const SwaArgs swa) {
   using L = AttnLayout<H>;
   extern __shared__ __align__(1024) uint8_t smem[];
   const uint32_t sbase = smem_u32(smem);
-  float* sred = reinterpret_cast<float*>(smem + L::sred_off);
+  float* red_max = reinterpret_cast<float*>(smem + L::red_off);   // [KG][H]
+  float* red_sum = red_max + L::KG * H;                            // [KG][H]
   float* qscale = reinterpret_cast<float*>(smem + L::qscale_off);
+  int* kvalid = reinterpret_cast<int*>(smem + L::kvalid_off);
+  int32_t* srow = reinterpret_cast<int32_t*>(smem + L::srow_off);
   float* ml_sh = reinterpret_cast<float*>(smem + L::ml_off);
   float* fac = reinterpret_cast<float*>(smem + L::fac_off);
-  int* kvalid = reinterpret_cast<int*>(smem + L::kvalid_off);
 
   cg::cluster_group cluster = cg::this_cluster();
   const int rank = static_cast<int>(cluster.block_rank());
-  pdl_wait();                 // everything the preceding launch wrote (the Top-k) is visible
-  pdl_launch_dependents();
   const int layer = static_cast<int>(blockIdx.x / kACluster) / n_queries;
   const int qi = static_cast<int>(blockIdx.x / kACluster) % n_queries;
   const __nv_bfloat16* __restrict__ qg = io.q[layer];
   __nv_bfloat16* __restrict__ out = io.out[layer];
-  const int b = q_req != nullptr ? q_req[qi] : qi;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int ht = warp % L::HT, dg = warp / L::HT;
-  const long long capacity = static_cast<long long>(cache.max_pages_per_req) * cache.page_size;
-  int n = (b >= 0 && b < cache.batch) ? cache.ctx_len[b] : 0;
-  n = n < 0 ? 0 : (n > capacity ? static_cast<int>(capacity) : n);
-  const int32_t* idx = topk + static_cast<long long>(qi) * K;
-  uint64_t* recv_bar = reinterpret_cast<uint64_t*>(smem + L::bar_off);
-  if (tid == 0) {
-    // every rank (this one included) sends this CTA one slice and one (m, l) pair
-    mbar_init(recv_bar, 1);
-    fence_barrier_init();
-    mbar_arrive_expect_tx(recv_bar, kACluster * (L::slice_bytes + L::ml_bytes));
-  }
+  const int ht = warp % L::HT, kg = warp / L::HT;
 
-  // ---- query -> fp16 with a power-of-two scale per head ----
-  constexpr int kHpw = H / (kAThreads / 32);   // heads per warp; their loads are issued together
+  // ---- query rows: loads issued before the wait on the preceding launch
+  // (which does not write them), converted once the rows are resolved ----
+  constexpr int kHpw = H / kAWarps;   // heads per warp
   uint4 raw[kHpw][2];
 #pragma unroll
   for (int hh = 0; hh < kHpw; ++hh) {
@@ -196,6 +195,58 @@ __global__ void __launch_bounds__(kAThreads, 1)
     raw[hh][0] = src[0];
     raw[hh][1] = src[1];
   }
+
+  pdl_wait();                 // everything the preceding launch wrote (the Top-k) is visible
+  pdl_launch_dependents();
+  const int b = q_req != nullptr ? q_req[qi] : qi;
+  const long long capacity = static_cast<long long>(cache.max_pages_per_req) * cache.page_size;
+  int n = (b >= 0 && b < cache.batch) ? cache.ctx_len[b] : 0;
+  n = n < 0 ? 0 : (n > capacity ? static_cast<int>(capacity) : n);
+  const int32_t* idx = topk + static_cast<long long>(qi) * K;
+
+  // ---- this CTA's entries: the Top-k entries, then the window's tokens ----
+  const int n_win = swa.codes != nullptr ? swa.window : 0;
+  const int p_tok = n_win > 0 ? swa.q_pos[qi] : 0;
+  const int K_all = K + n_win;
+  const int kc = (K_all + kACluster - 1) / kACluster;
+  const int key_begin = min(rank * kc, K_all), key_end = min(key_begin + kc, K_all);
+  const int n_top = min(max(0, min(key_end, K) - key_begin), kMaxTop);
+  for (int i = tid; i < n_top; i += kAThreads) {
+    const int t = idx[key_begin + i];
+    int r = -1;
+    if (t >= 0 && t < n) {
+      const int page = cache.page_table[static_cast<long long>(b) * cache.max_pages_per_req + t / cache.page_size];
+      if (page >= 0 && page < cache.num_pages) r = page * cache.page_size + t % cache.page_size;
+      else report_error(cache.err_word, CSA2_ERR_DEVICE_BOUNDS, kKAttn, b, t);
+    } else if (t >= n || t < -1) {
+      report_error(cache.err_word, CSA2_ERR_DEVICE_BOUNDS, kKAttn, b, t);
+    }
+    srow[i] = r;
+  }
+  __syncthreads();
+
+  // cp.async of the packed rows of the chunk starting at entry c into the
+  // staging buffer (code granules XOR-swizzled by row % 8)
+  auto issue_chunk = [&](int c) {
+    const int nk = min(kChunk, key_end - c);
+    for (int g = tid; g < nk * kRowGran; g += kAThreads) {
+      const int row = g / kRowGran, part = g - row * kRowGran;
+      const int i = c + row - key_begin;
+      if (c + row >= K || i >= n_top) continue;
+      const int r = srow[i];
+      if (r < 0) continue;
+      if (part < kCodeGran)
+        cp_async16(sbase + L::raw_off + row * kKvCodeBytes + ((part ^ (row & 7)) << 4),
+                   cache.kv_codes + static_cast<long long>(r) * kKvCodeBytes + part * 16);
+      else
+        cp_async16(sbase + L::raw_scale_off + row * kKvScaleBytes + (part - kCodeGran) * 16,
+                   cache.kv_scales + static_cast<long long>(r) * kKvScaleBytes + (part - kCodeGran) * 16);
+    }
+    cp_async_commit();
+  };
+  if (key_begin < key_end) issue_chunk(key_begin);
+
+  // ---- query -> fp16 with a power-of-two scale per head ----
 #pragma unroll
   for (int hh = 0; hh < kHpw; ++hh) {
     const int h = warp * kHpw + hh;
@@ -224,28 +275,24 @@ __global__ void __launch_bounds__(kAThreads, 1)
     if (lane == 0) qscale[h] = softmax_scale * down * kLog2e;
   }
 
-  // ---- this CTA's keys: the Top-k entries, then the window's tokens ----
-  const int n_win = swa.codes != nullptr ? swa.window : 0;
-  const int p_tok = n_win > 0 ? swa.q_pos[qi] : 0;
-  const int K_all = K + n_win;
-  const int kc = (K_all + kACluster - 1) / kACluster;
-  const int key_begin = min(rank * kc, K_all), key_end = min(key_begin + kc, K_all);
-
   float o_acc[L::DW / 8][4];
 #pragma unroll
   for (int i = 0; i < L::DW / 8; ++i) o_acc[i][0] = o_acc[i][1] = o_acc[i][2] = o_acc[i][3] = 0.0f;
   float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.0f, 0.0f};
   const int r0 = lane >> 2;   // fragment row (and row + 8)
+  const int h0 = ht * 16 + r0, h1 = h0 + 8;
 
   for (int c0 = key_begin; c0 < key_end; c0 += kChunk) {
     const int nk = min(kChunk, key_end - c0);
-    __syncthreads();   // previous chunk's KV no longer read
+    cp_async_wait_all();
+    __syncthreads();   // staged rows visible; the previous chunk's S and P V are done
     {
-      // gather + dequantise: 4 threads per row, 128 channels each
-      const int row = tid >> 2, part = tid & 3;
-      if (row < nk && c0 + row >= K) {
+      // dequantise: thread (row, part) writes channels [128*part, 128*part + 128) of the row
+      const int row = tid & (kChunk - 1), part = tid / kChunk;
+      const int e = c0 + row;
+      if (row < nk && e >= K) {
         // window entry j: token p - window + 1 + j (none before token 0)
-        const int tw = p_tok - n_win + 1 + (c0 + row - K);
+        const int tw = p_tok - n_win + 1 + (e - K);
         const bool ok = tw >= 0 && b >= 0 && b < cache.batch;
         if (part == 0) kvalid[row] = ok;
         if (ok) {
@@ -278,86 +325,63 @@ __global__ void __launch_bounds__(kAThreads, 1)
             *reinterpret_cast<uint4*>(smem + L::kv_off + swz(row, part * 16 + c)) = make_uint4(0, 0, 0, 0);
         }
       } else {
-      int t = row < nk ? idx[c0 + row] : -1;
-      long long src_row = -1;
-      if (t >= 0 && t < n) {
-        const int page = cache.page_table[static_cast<long long>(b) * cache.max_pages_per_req + t / cache.page_size];
-        if (page >= 0 && page < cache.num_pages) src_row = static_cast<long long>(page) * cache.page_size + t % cache.page_size;
-        else if (part == 0) report_error(cache.err_word, CSA2_ERR_DEVICE_BOUNDS, kKAttn, b, t);
-      } else if (row < nk && (t >= n || t < -1) && part == 0) {
-        report_error(cache.err_word, CSA2_ERR_DEVICE_BOUNDS, kKAttn, b, t);
-      }
-      if (part == 0) kvalid[row] = src_row >= 0;
-      if (src_row >= 0) {
-        const uint4* cp = reinterpret_cast<const uint4*>(cache.kv_codes + src_row * kKvCodeBytes) + part * 4;
-        const uint2 sp = *reinterpret_cast<const uint2*>(cache.kv_scales + src_row * kKvScaleBytes + part * 8);
-        uint4 cv[4];   // every load of the row part in flight before any shared-memory store
+        const int i = e - key_begin;
+        const bool ok = row < nk && i < n_top && srow[i] >= 0;
+        if (part == 0) kvalid[row] = ok;
+        if (ok) {
+          const uint8_t* rc = smem + L::raw_off + row * kKvCodeBytes;
+          const uint2 sp = *reinterpret_cast<const uint2*>(smem + L::raw_scale_off + row * kKvScaleBytes + part * 8);
 #pragma unroll
-        for (int j = 0; j < 4; ++j) cv[j] = cp[j];
+          for (int j = 0; j < 4; ++j) {
+            const uint4 cv = *reinterpret_cast<const uint4*>(rc + (((4 * part + j) ^ (row & 7)) << 4));
+            uint4 hv[4];
+            dequant16(cv, j < 2 ? (sp.x >> (16 * j)) : (sp.y >> (16 * (j - 2))), hv);
+            const int chunk0 = part * 16 + j * 4;   // 8 fp16 per chunk
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          uint4 hv[4];
-          dequant16(cv[j], j < 2 ? (sp.x >> (16 * j)) : (sp.y >> (16 * (j - 2))), hv);
-          const int chunk0 = part * 16 + j * 4;   // 8 fp16 per chunk
+            for (int c = 0; c < 4; ++c) *reinterpret_cast<uint4*>(smem + L::kv_off + swz(row, chunk0 + c)) = hv[c];
+          }
+        } else {
 #pragma unroll
-          for (int c = 0; c < 4; ++c) *reinterpret_cast<uint4*>(smem + L::kv_off + swz(row, chunk0 + c)) = hv[c];
+          for (int c = 0; c < 16; ++c)
+            *reinterpret_cast<uint4*>(smem + L::kv_off + swz(row, part * 16 + c)) = make_uint4(0, 0, 0, 0);
         }
+      }
+    }
+    __syncthreads();   // the chunk's fp16 rows are visible; the staging buffer is free
+    if (c0 + kChunk < key_end) issue_chunk(c0 + kChunk);
+
+    // ---- S = Q K^T: this warp's 16 heads x KW keys over all 512 dims ----
+    float s[L::NT][4];
+#pragma unroll
+    for (int j = 0; j < L::NT; ++j) s[j][0] = s[j][1] = s[j][2] = s[j][3] = 0.0f;
+    const int key0 = kg * L::KW;
+#pragma unroll 4
+    for (int ks = 0; ks < kKvDim / 16; ++ks) {
+      uint32_t a0, a1, a2, a3;
+      ldsm_x4(sbase + L::q_off + swz(ht * 16 + (lane & 15), ks * 2 + (lane >> 4)), a0, a1, a2, a3);
+      if constexpr (L::NT == 1) {
+        uint32_t b0, b1;
+        ldsm_x2(sbase + L::kv_off + swz(key0 + (lane & 7), ks * 2 + ((lane >> 3) & 1)), b0, b1);
+        mma_f16(s[0], a0, a1, a2, a3, b0, b1);
       } else {
 #pragma unroll
-        for (int c = 0; c < 16; ++c)
-          *reinterpret_cast<uint4*>(smem + L::kv_off + swz(row, part * 16 + c)) = make_uint4(0, 0, 0, 0);
-      }
-      }
-    }
-    __syncthreads();
-
-    // ---- S = Q K^T over this warp's dims ----
-    float s[8][4];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) s[j][0] = s[j][1] = s[j][2] = s[j][3] = 0.0f;
-#pragma unroll 4
-    for (int ks = 0; ks < L::DW / 16; ++ks) {
-      const int kchunk = (dg * L::DW + ks * 16) / 8;
-      uint32_t a0, a1, a2, a3;
-      ldsm_x4(sbase + L::q_off + swz(ht * 16 + (lane & 15), kchunk + (lane >> 4)), a0, a1, a2, a3);
-#pragma unroll
-      for (int np = 0; np < 4; ++np) {   // pairs of 8-key tiles
-        const int mi = lane >> 3;
-        uint32_t b0, b1, b2, b3;
-        ldsm_x4(sbase + L::kv_off + swz(np * 16 + (mi >> 1) * 8 + (lane & 7), kchunk + (mi & 1)), b0, b1, b2, b3);
-        mma_f16(s[2 * np], a0, a1, a2, a3, b0, b1);
-        mma_f16(s[2 * np + 1], a0, a1, a2, a3, b2, b3);
-      }
-    }
-    if (L::DG > 1) {
-      float* mine = sred + (dg * H + ht * 16) * kSredStride;
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const int col = j * 8 + 2 * (lane & 3);
-        *reinterpret_cast<float2*>(mine + r0 * kSredStride + col) = make_float2(s[j][0], s[j][1]);
-        *reinterpret_cast<float2*>(mine + (r0 + 8) * kSredStride + col) = make_float2(s[j][2], s[j][3]);
-      }
-      __syncthreads();
-#pragma unroll
-      for (int j = 0; j < 8; ++j) s[j][0] = s[j][1] = s[j][2] = s[j][3] = 0.0f;
-      for (int g = 0; g < L::DG; ++g) {
-        const float* part = sred + (g * H + ht * 16) * kSredStride;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const int col = j * 8 + 2 * (lane & 3);
-          const float2 u = *reinterpret_cast<const float2*>(part + r0 * kSredStride + col);
-          const float2 v = *reinterpret_cast<const float2*>(part + (r0 + 8) * kSredStride + col);
-          s[j][0] += u.x; s[j][1] += u.y; s[j][2] += v.x; s[j][3] += v.y;
+        for (int np = 0; np < L::NT / 2; ++np) {   // pairs of 8-key tiles
+          const int mi = lane >> 3;
+          uint32_t b0, b1, b2, b3;
+          ldsm_x4(sbase + L::kv_off + swz(key0 + np * 16 + (mi >> 1) * 8 + (lane & 7), ks * 2 + (mi & 1)), b0, b1,
+                  b2, b3);
+          mma_f16(s[2 * np], a0, a1, a2, a3, b0, b1);
+          mma_f16(s[2 * np + 1], a0, a1, a2, a3, b2, b3);
         }
       }
     }
 
-    // ---- online softmax (log2 domain) ----
-    const float sc0 = qscale[ht * 16 + r0], sc1 = qscale[ht * 16 + r0 + 8];
+    // ---- online softmax (log2 domain), maxima and sums combined over the key groups ----
+    const float sc0 = qscale[h0], sc1 = qscale[h1];
     float mx0 = -INFINITY, mx1 = -INFINITY;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const int col = j * 8 + 2 * (lane & 3);
+    for (int j = 0; j < L::NT; ++j) {
+      const int col = key0 + j * 8 + 2 * (lane & 3);
       const bool v0 = col < nk && kvalid[col], v1 = col + 1 < nk && kvalid[col + 1];
       s[j][0] = v0 ? s[j][0] * sc0 : -INFINITY;
       s[j][1] = v1 ? s[j][1] * sc0 : -INFINITY;
@@ -371,27 +395,49 @@ __global__ void __launch_bounds__(kAThreads, 1)
       mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
       mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
     }
-    const float mn0 = fmaxf(m_run[0], mx0), mn1 = fmaxf(m_run[1], mx1);
+    if ((lane & 3) == 0) {
+      red_max[kg * H + h0] = mx0;
+      red_max[kg * H + h1] = mx1;
+    }
+    __syncthreads();   // every key group's row maxima
+    float mn0 = m_run[0], mn1 = m_run[1];
+#pragma unroll
+    for (int g = 0; g < L::KG; ++g) {
+      mn0 = fmaxf(mn0, red_max[g * H + h0]);
+      mn1 = fmaxf(mn1, red_max[g * H + h1]);
+    }
     const float ref0 = mn0 == -INFINITY ? 0.0f : mn0, ref1 = mn1 == -INFINITY ? 0.0f : mn1;
     const float corr0 = exp2f(m_run[0] - ref0), corr1 = exp2f(m_run[1] - ref1);
     float sum0 = 0.0f, sum1 = 0.0f;
-    uint32_t pa[4][4];   // P as fp16 A fragments, one per 16-key step
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
+    for (int j = 0; j < L::NT; ++j) {
       const float p0 = exp2f(s[j][0] - ref0), p1 = exp2f(s[j][1] - ref0);
       const float p2 = exp2f(s[j][2] - ref1), p3 = exp2f(s[j][3] - ref1);
       sum0 += p0 + p1;
       sum1 += p2 + p3;
-      pa[j >> 1][(j & 1) * 2 + 0] = pack_half2(p0, p1);
-      pa[j >> 1][(j & 1) * 2 + 1] = pack_half2(p2, p3);
+      const int col = key0 + j * 8 + 2 * (lane & 3);
+      const uint32_t within = (col & 7) * 2;
+      *reinterpret_cast<uint32_t*>(smem + L::p_off + pswz(h0, col >> 3) + within) = pack_half2(p0, p1);
+      *reinterpret_cast<uint32_t*>(smem + L::p_off + pswz(h1, col >> 3) + within) = pack_half2(p2, p3);
     }
 #pragma unroll
     for (int o = 1; o < 4; o <<= 1) {
       sum0 += __shfl_xor_sync(0xffffffffu, sum0, o);
       sum1 += __shfl_xor_sync(0xffffffffu, sum1, o);
     }
-    l_run[0] = l_run[0] * corr0 + sum0;
-    l_run[1] = l_run[1] * corr1 + sum1;
+    if ((lane & 3) == 0) {
+      red_sum[kg * H + h0] = sum0;
+      red_sum[kg * H + h1] = sum1;
+    }
+    __syncthreads();   // P and every key group's row sums
+    float tot0 = 0.0f, tot1 = 0.0f;
+#pragma unroll
+    for (int g = 0; g < L::KG; ++g) {
+      tot0 += red_sum[g * H + h0];
+      tot1 += red_sum[g * H + h1];
+    }
+    l_run[0] = l_run[0] * corr0 + tot0;
+    l_run[1] = l_run[1] * corr1 + tot1;
     m_run[0] = mn0;
     m_run[1] = mn1;
 #pragma unroll
@@ -400,15 +446,15 @@ __global__ void __launch_bounds__(kAThreads, 1)
       o_acc[i][2] *= corr1; o_acc[i][3] *= corr1;
     }
 
-    // ---- O += P V over this warp's dims ----
+    // ---- O += P V: this warp's 16 heads x DW dims over the chunk's 64 keys ----
 #pragma unroll
-    for (int kk = 0; kk < 4; ++kk) {
-      // A fragment order: (row, k lo), (row+8, k lo), (row, k hi), (row+8, k hi)
-      const uint32_t a0 = pa[kk][0], a1 = pa[kk][1], a2 = pa[kk][2], a3 = pa[kk][3];
+    for (int kk = 0; kk < kChunk / 16; ++kk) {
+      uint32_t a0, a1, a2, a3;
+      ldsm_x4(sbase + L::p_off + pswz(ht * 16 + (lane & 15), kk * 2 + (lane >> 4)), a0, a1, a2, a3);
 #pragma unroll
       for (int np = 0; np < L::DW / 16; ++np) {
         const int mi = lane >> 3;
-        const int dchunk = (dg * L::DW) / 8 + np * 2 + (mi >> 1);
+        const int dchunk = (kg * L::DW) / 8 + np * 2 + (mi >> 1);
         uint32_t b0, b1, b2, b3;
         ldsm_x4_t(sbase + L::kv_off + swz(kk * 16 + (mi & 1) * 8 + (lane & 7), dchunk), b0, b1, b2, b3);
         mma_f16(o_acc[2 * np], a0, a1, a2, a3, b0, b1);
@@ -417,64 +463,32 @@ __global__ void __launch_bounds__(kAThreads, 1)
     }
   }
 
-  // ---- send the partial O slices, maxima and sums to their owners ----
+  // ---- partial O slices, maxima and sums into their owners' shared memory ----
   // Output dims [kODims*r, kODims*(r+1)) belong to CTA r; it receives every
-  // rank's slice of them in recv[src][h][kODims] and every rank's (m, l) in
-  // ml_sh[src], by bulk copies between the cluster's shared memories,
-  // L::per_round owners' slices staged at a time.
+  // rank's slice of them in recv[src][h][kODims] (16-byte granules of a
+  // head's row XOR-swizzled by the head) and every rank's (m, l) in
+  // ml_sh[src].  Every CTA of the cluster passes both barriers.
   cluster.sync();   // every CTA is done reading its Q / KV region, which receives the partials
   float* recv = reinterpret_cast<float*>(smem);
-  float* stage = sred;                                              // [per_round][H][kODims]
-  float* stage_ml = sred + L::per_round * H * kODims;               // [2][H]: m, l
-  if (dg == 0 && (lane & 3) == 0) {
-    stage_ml[ht * 16 + r0] = m_run[0];
-    stage_ml[ht * 16 + r0 + 8] = m_run[1];
-    stage_ml[H + ht * 16 + r0] = l_run[0];
-    stage_ml[H + ht * 16 + r0 + 8] = l_run[1];
-  }
-  for (int round = 0; round < kACluster / L::per_round; ++round) {
 #pragma unroll
-    for (int i = 0; i < L::DW / 8; ++i) {
-      const int col = dg * L::DW + i * 8 + 2 * (lane & 3);
-      const int owner = col / kODims, cd = col % kODims;
-      if (owner / L::per_round != round) continue;
-      // 16-byte granules of a head's row XOR-swizzled by the head (the same
-      // layout is read back by the owner), so the 8 rows a warp writes at once
-      // fall in different banks
-      const int h0 = ht * 16 + r0, h1 = h0 + 8;
-      float* row = stage + (owner % L::per_round) * H * kODims;
-      *reinterpret_cast<float2*>(row + h0 * kODims + attn_swz(h0, cd)) = make_float2(o_acc[i][0], o_acc[i][1]);
-      *reinterpret_cast<float2*>(row + h1 * kODims + attn_swz(h1, cd)) = make_float2(o_acc[i][2], o_acc[i][3]);
-    }
-    fence_proxy_async_smem();
-    __syncthreads();
-    if (tid == 0) {
-      const uint32_t bar = smem_u32(recv_bar);
-      for (int o = round * L::per_round; o < (round + 1) * L::per_round; ++o)
-        bulk_copy_to_rank(mapa_rank(smem_u32(recv + rank * H * kODims), o),
-                          smem_u32(stage + (o % L::per_round) * H * kODims), L::slice_bytes, mapa_rank(bar, o));
-      if (round == 0)
-        for (int o = 0; o < kACluster; ++o)
-          bulk_copy_to_rank(mapa_rank(smem_u32(ml_sh + rank * 2 * H), o), smem_u32(stage_ml), L::ml_bytes,
-                            mapa_rank(bar, o));
-      bulk_commit_and_wait_read();   // the staging area may be written again
-    }
-    __syncthreads();
+  for (int i = 0; i < L::DW / 8; ++i) {
+    const int col = kg * L::DW + i * 8 + 2 * (lane & 3);
+    const int owner = col / kODims, cd = col % kODims;
+    float* dst = cluster.map_shared_rank(recv, owner) + rank * H * kODims;
+    *reinterpret_cast<float2*>(dst + h0 * kODims + attn_swz(h0, cd)) = make_float2(o_acc[i][0], o_acc[i][1]);
+    *reinterpret_cast<float2*>(dst + h1 * kODims + attn_swz(h1, cd)) = make_float2(o_acc[i][2], o_acc[i][3]);
   }
-  // Every copy into this CTA has landed once the barrier completes, and every
-  // copy out of it has been read: after that the CTA may exit without a
-  // cluster-wide barrier.  If the wait runs out, the error is recorded, the
-  // CTA waits once more (bounded) for copies still in flight and leaves
-  // without writing its output.
-  bool received = true;
-  if (tid == 0) {
-    received = mbar_wait(recv_bar, 0, kWaitLimitNs);
-    if (!received) {
-      report_error(cache.err_word, CSA2_ERR_TIMEOUT, kKAttn, b, -1);
-      (void)mbar_wait(recv_bar, 0, kWaitLimitNs);
+  if (kg == 0 && (lane & 3) == 0) {
+#pragma unroll
+    for (int o = 0; o < kACluster; ++o) {
+      float* ml = cluster.map_shared_rank(ml_sh, o) + rank * 2 * H;
+      ml[h0] = m_run[0];
+      ml[h1] = m_run[1];
+      ml[H + h0] = l_run[0];
+      ml[H + h1] = l_run[1];
     }
   }
-  if (!__syncthreads_and(received)) return;
+  cluster.sync();   // every partial has landed; no CTA touches another's memory after this
 
   // merge factors per (source rank, head): exp2(m_r - M) / L
   for (int h = tid; h < H; h += kAThreads) {
@@ -536,7 +550,7 @@ cudaError_t launch_h(const csa2_cache& cache, int n_layers, int n_queries, const
   attr[0].val.clusterDim.x = kACluster;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
-  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;   // the kernel calls pdl_wait() first
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;   // the kernel calls pdl_wait() before reading the Top-k
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
