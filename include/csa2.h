@@ -300,13 +300,28 @@ CSA2_API csa2_status csa2_prefill_index_static(const csa2_cache* cache, int32_t 
  * query]), in one launch.
  *   q    host array [n_layers] of device pointers, each bf16 [n_queries][H][512]
  *   out  host array [n_layers] of device pointers, each bf16 [n_queries][H][512]
+ *   workspace  NULL, or caller-owned device memory of at least
+ *              csa2_attn_workspace_bytes(n_layers, n_queries, H) bytes,
+ *              16-byte aligned, used as scratch by this call only (contents
+ *              need no initialisation; no two calls in flight may share it).
+ *              Each (layer, query) is split over four CTAs by Top-k entries;
+ *              with a workspace they merge their partial outputs through it
+ *              (L2), without one through each other's shared memory.  Both
+ *              give bit-identical results; the workspace is faster when few
+ *              queries are in flight (decode).
  * n_layers in [1, CSA2_ATTN_MAX_LAYERS]; everything else as csa2_sparse_attn.
+ * A workspace that is misaligned or smaller than required -> CSA2_ERR_ARG /
+ * CSA2_ERR_SHAPE, nothing launched.
  */
 #define CSA2_ATTN_MAX_LAYERS 8
 CSA2_API csa2_status csa2_sparse_attn_layers(const csa2_cache* cache, int32_t n_layers, int32_t n_queries,
                                              const int32_t* q_req, const int32_t* topk, int32_t k,
                                              const uint16_t* const* q, int32_t H, float scale,
-                                             uint16_t* const* out, void* stream);
+                                             uint16_t* const* out, void* workspace, size_t workspace_bytes,
+                                             void* stream);
+/* Workspace bytes of csa2_sparse_attn_layers: n_layers * n_queries * 4 splits
+ * * (H * 512 + 2 * H) floats (0 for negative arguments). */
+CSA2_API size_t csa2_attn_workspace_bytes(int32_t n_layers, int32_t n_queries, int32_t H);
 
 /*
  * Sliding-window (SWA) branch.  Every layer, Reuse layers included, keeps its

@@ -43,7 +43,7 @@ _sig = {
     "csa2_pool_select": [_CP, _P, _I, _P, _P],
     "csa2_reindex": [_CP, _I, _P, _I, _P, _P, _P, _P, _I, _P, _P],
     "csa2_sparse_attn": [_CP, _I, _P, _P, _I, _P, _I, ctypes.c_float, _P, _P],
-    "csa2_sparse_attn_layers": [_CP, _I, _I, _P, _P, _I, _P, _I, ctypes.c_float, _P, _P],
+    "csa2_sparse_attn_layers": [_CP, _I, _I, _P, _P, _I, _P, _I, ctypes.c_float, _P, _P, ctypes.c_size_t, _P],
     "csa2_swa_append": [_CP, _I, _P, _P, _I, _P, _P, _P, _P],
     "csa2_sparse_attn_swa": [_CP, _I, _P, _P, _I, _P, _P, _I, _P, _P, _I, ctypes.c_float, _P, _P],
     "csa2_prefill_index": [_CP, _I, _I, _P, _I, _P, _P, _I, _P, _P, ctypes.c_size_t, _P],
@@ -59,6 +59,8 @@ _lib.csa2_last_error_message.argtypes = []
 _lib.csa2_last_error_message.restype = ctypes.c_char_p
 _lib.csa2_prefill_workspace_bytes.argtypes = [_I]
 _lib.csa2_prefill_workspace_bytes.restype = ctypes.c_size_t
+_lib.csa2_attn_workspace_bytes.argtypes = [_I, _I, _I]
+_lib.csa2_attn_workspace_bytes.restype = ctypes.c_size_t
 _lib.csa2_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
 _lib.csa2_set_wait_limit_ns.restype = None
 
@@ -267,9 +269,16 @@ def prefill_index_static(cache: Cache, req: int, q_pos, q, w, k: int = 512, rati
     return topk
 
 
-def sparse_attn_layers(cache: Cache, topk, q_layers, scale: float | None = None, out_layers=None, q_req=None):
+def attn_workspace_bytes(n_layers: int, n_queries: int, heads: int) -> int:
+    return int(_lib.csa2_attn_workspace_bytes(int(n_layers), int(n_queries), int(heads)))
+
+
+def sparse_attn_layers(cache: Cache, topk, q_layers, scale: float | None = None, out_layers=None, q_req=None,
+                       workspace=None):
     """Sparse attention of several layers over the same Top-k in one launch;
-    q_layers: list of bf16 [n, H, 512] -> list of outputs of the same shape."""
+    q_layers: list of bf16 [n, H, 512] -> list of outputs of the same shape.
+    workspace: optional uint8 device tensor of attn_workspace_bytes(...) bytes
+    (the key splits then merge through it instead of shared memory)."""
     n, k = topk.shape
     L = len(q_layers)
     H = q_layers[0].shape[1]
@@ -285,8 +294,10 @@ def sparse_attn_layers(cache: Cache, topk, q_layers, scale: float | None = None,
     scale = 1.0 / math.sqrt(KV_DIM) if scale is None else scale
     qa = (ctypes.c_void_p * L)(*[q.data_ptr() for q in q_layers])
     oa = (ctypes.c_void_p * L)(*[o.data_ptr() for o in out_layers])
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(_lib.csa2_sparse_attn_layers(ctypes.byref(cache.struct), L, n, _ptr(q_req), _ptr(topk), k, qa, H,
-                                        ctypes.c_float(scale), oa, _stream(cache.device)), "csa2_sparse_attn_layers")
+                                        ctypes.c_float(scale), oa, _ptr(workspace), ws_bytes,
+                                        _stream(cache.device)), "csa2_sparse_attn_layers")
     return out_layers
 
 
@@ -378,6 +389,9 @@ class DecodeGroup:
         # calling stream, linked by programmatic dependent launch; the other
         # sources run on streams of their own, after the pool
         self.streams = [torch.cuda.Stream(dev) for _ in self.sources[:-1]] if concurrent else []
+        # one attention exchange workspace per source (the sources may run at once)
+        self.attn_ws = [torch.empty(attn_workspace_bytes(len(layers), B, heads), dtype=torch.uint8, device=dev)
+                        for layers in self.sources]
         self.launches_per_step = 1 + (1 if pool_blocks else 0) + 2 * len(self.sources)
 
     def step(self, q_idx, w_idx, q_main, out, timing=None):
@@ -416,7 +430,8 @@ class DecodeGroup:
                 timed(f"topk{src}", lambda: reindex(c, mode, self.k, self.pool, q_idx[src], w_idx[src],
                                                     topk=self.topk[src]))
                 timed(f"attn{src}", lambda: sparse_attn_layers(c, self.topk[src], [q_main[l] for l in layers],
-                                                               self.scale, [out[l] for l in layers]))
+                                                               self.scale, [out[l] for l in layers],
+                                                               workspace=self.attn_ws[si]))
         if self.concurrent:
             joins = []
             for s in self.streams:

@@ -126,7 +126,8 @@ csa2_status check_cache(const csa2_cache* c, bool need_kv, bool need_ik) {
 
 csa2_status sparse_attn_impl(const csa2_cache* cache, int32_t n_layers, int32_t n_queries, const int32_t* q_req,
                              const int32_t* topk, int32_t k, const uint16_t* const* q, int32_t H, float scale,
-                             uint16_t* const* out, void* stream) {
+                             uint16_t* const* out, void* stream, void* workspace = nullptr,
+                             size_t workspace_bytes = 0) {
   CSA2_TRY(check_cache(cache, true, false));
   if (n_layers < 1 || n_layers > CSA2_ATTN_MAX_LAYERS)
     return fail(CSA2_ERR_SHAPE, "n_layers %d outside [1, %d]", n_layers, CSA2_ATTN_MAX_LAYERS);
@@ -142,10 +143,17 @@ csa2_status sparse_attn_impl(const csa2_cache* cache, int32_t n_layers, int32_t 
   for (int l = 0; l < n_layers; ++l)
     if (q[l] == nullptr || out[l] == nullptr || !aligned(q[l], 16) || !aligned(out[l], 16))
       return fail(CSA2_ERR_ARG, "layer %d: q and out (16-byte aligned) must be set", l);
+  if (workspace != nullptr) {
+    if (!aligned(workspace, 16)) return fail(CSA2_ERR_ARG, "workspace must be 16-byte aligned");
+    const size_t need = csa2::attn_workspace_bytes(n_layers, n_queries, H);
+    if (workspace_bytes < need)
+      return fail(CSA2_ERR_SHAPE, "workspace_bytes %zu < %zu (csa2_attn_workspace_bytes)", workspace_bytes, need);
+  }
   DeviceInfo d;
   CSA2_TRY(device_info(&d));
   const cudaError_t e = csa2::launch_sparse_attn(*cache, n_layers, n_queries, q_req, topk, k, q, H, scale, out,
-                                                 static_cast<cudaStream_t>(stream));
+                                                 static_cast<cudaStream_t>(stream), nullptr, nullptr, nullptr, 0,
+                                                 workspace);
   return e == cudaSuccess ? CSA2_OK : cuda_fail(e, "sparse_attn launch");
 }
 
@@ -315,8 +323,15 @@ csa2_status csa2_sparse_attn_swa(const csa2_cache* cache, int32_t n_queries, con
 
 csa2_status csa2_sparse_attn_layers(const csa2_cache* cache, int32_t n_layers, int32_t n_queries,
                                     const int32_t* q_req, const int32_t* topk, int32_t k, const uint16_t* const* q,
-                                    int32_t H, float scale, uint16_t* const* out, void* stream) {
-  return sparse_attn_impl(cache, n_layers, n_queries, q_req, topk, k, q, H, scale, out, stream);
+                                    int32_t H, float scale, uint16_t* const* out, void* workspace,
+                                    size_t workspace_bytes, void* stream) {
+  return sparse_attn_impl(cache, n_layers, n_queries, q_req, topk, k, q, H, scale, out, stream, workspace,
+                          workspace_bytes);
+}
+
+size_t csa2_attn_workspace_bytes(int32_t n_layers, int32_t n_queries, int32_t H) {
+  if (n_layers < 0 || n_queries < 0 || H < 0) return 0;
+  return csa2::attn_workspace_bytes(n_layers, n_queries, H);
 }
 
 size_t csa2_prefill_workspace_bytes(int32_t n_queries) { return csa2::prefill_workspace_bytes(n_queries); }

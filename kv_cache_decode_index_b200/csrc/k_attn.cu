@@ -45,6 +45,7 @@ constexpr int kODims = kKvDim / kACluster;   // output dims owned by one CTA of 
 constexpr int kChunk = 64;                   // keys per chunk
 constexpr int kRowBytes = kKvDim * 2;        // fp16 row: 1024 B
 constexpr int kPRowBytes = kChunk * 2;       // fp16 row of P: 128 B
+constexpr int kPVDims = kKvDim / kAWarps;    // output dims per warp in P V: 64
 constexpr int kCodeGran = kKvCodeBytes / 16;                    // 16-byte granules of a packed row's codes
 constexpr int kRowGran = (kKvCodeBytes + kKvScaleBytes) / 16;   // ... of codes + scales
 // Top-k entries one CTA resolves: k <= 4096 and a window <= 4096 give at most
@@ -55,10 +56,9 @@ constexpr float kLog2e = 1.4426950408889634f;
 template <int H>
 struct AttnLayout {
   static constexpr int HT = H / 16;            // head tiles of 16 query rows
-  static constexpr int KG = kAWarps / HT;      // key groups in S = dim groups in P V
+  static constexpr int KG = kAWarps / HT;      // key groups in S
   static constexpr int KW = kChunk / KG;       // keys per warp in S
   static constexpr int NT = KW / 8;            // 8-key tiles per warp in S
-  static constexpr int DW = kKvDim / KG;       // output dims per warp in P V
   static constexpr uint32_t q_off = 0;                                     // fp16 [H][512]
   static constexpr uint32_t kv_off = q_off + H * kRowBytes;                // fp16 [64][512]
   static constexpr uint32_t raw_off = kv_off + kChunk * kRowBytes;         // u8 [64][256] codes
@@ -112,11 +112,6 @@ __device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
   const __half2 h = __floats2half2_rn(lo, hi);
   return *reinterpret_cast<const uint32_t*>(&h);
 }
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
 
 // Two E2M1 codes (low nibble = even channel) -> f16x2, low half = even channel.
 __device__ __forceinline__ uint32_t e2m1x2_half2(uint32_t byte) {
@@ -163,7 +158,7 @@ template <int H>
 __global__ void __launch_bounds__(kAThreads, H == 16 ? 2 : 1)
     sparse_attn_kernel(const csa2_cache cache, int n_queries, const int32_t* __restrict__ q_req,
                        const int32_t* __restrict__ topk, int K, const __grid_constant__ AttnLayers io, float softmax_scale,
-                       const SwaArgs swa) {
+                       const SwaArgs swa, float* __restrict__ xchg) {
   using L = AttnLayout<H>;
   extern __shared__ __align__(1024) uint8_t smem[];
   const uint32_t sbase = smem_u32(smem);
@@ -184,8 +179,8 @@ __global__ void __launch_bounds__(kAThreads, H == 16 ? 2 : 1)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int ht = warp % L::HT, kg = warp / L::HT;
 
-  // ---- query rows: loads issued before the wait on the preceding launch
-  // (which does not write them), converted once the rows are resolved ----
+  // ---- query rows, loaded and converted before the wait on the preceding
+  // launch (which does not write them) ----
   constexpr int kHpw = H / kAWarps;   // heads per warp
   uint4 raw[kHpw][2];
 #pragma unroll
@@ -194,6 +189,35 @@ __global__ void __launch_bounds__(kAThreads, H == 16 ? 2 : 1)
         reinterpret_cast<const uint4*>(qg + (static_cast<long long>(qi) * H + warp * kHpw + hh) * kKvDim) + lane * 2;
     raw[hh][0] = src[0];
     raw[hh][1] = src[1];
+  }
+
+  // ---- query -> fp16 with a power-of-two scale per head ----
+#pragma unroll
+  for (int hh = 0; hh < kHpw; ++hh) {
+    const int h = warp * kHpw + hh;
+    const uint4 v0 = raw[hh][0], v1 = raw[hh][1];
+    const uint32_t wv[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+    float f[16];
+    float amax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      f[2 * i] = __uint_as_float(wv[i] << 16);
+      f[2 * i + 1] = __uint_as_float(wv[i] & 0xFFFF0000u);
+      amax = fmaxf(amax, fmaxf(fabsf(f[2 * i]), fabsf(f[2 * i + 1])));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    int E = static_cast<int>((__float_as_uint(amax) >> 23) & 0xFF) - 127;   // amax in [2^E, 2^(E+1))
+    if (amax == 0.0f) E = 14;
+    E = max(E, -100);
+    const float up = exp2i(14 - E), down = exp2i(E - 14);
+    uint32_t hv[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) hv[i] = pack_half2(f[2 * i] * up, f[2 * i + 1] * up);
+    // lane holds dims [16*lane, 16*lane+16): chunks 2*lane, 2*lane+1
+    *reinterpret_cast<uint4*>(smem + swz(h, 2 * lane)) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
+    *reinterpret_cast<uint4*>(smem + swz(h, 2 * lane + 1)) = make_uint4(hv[4], hv[5], hv[6], hv[7]);
+    if (lane == 0) qscale[h] = softmax_scale * down * kLog2e;
   }
 
   pdl_wait();                 // everything the preceding launch wrote (the Top-k) is visible
@@ -246,41 +270,19 @@ __global__ void __launch_bounds__(kAThreads, H == 16 ? 2 : 1)
   };
   if (key_begin < key_end) issue_chunk(key_begin);
 
-  // ---- query -> fp16 with a power-of-two scale per head ----
+  // P V: warp w owns output dims [64w, 64w + 64) of every head; the running
+  // max / sum of rows t*16 + r0 and t*16 + r0 + 8 of every head tile t are
+  // kept in every warp (identical values)
+  float o_acc[L::HT][kPVDims / 8][4];
 #pragma unroll
-  for (int hh = 0; hh < kHpw; ++hh) {
-    const int h = warp * kHpw + hh;
-    const uint4 v0 = raw[hh][0], v1 = raw[hh][1];
-    const uint32_t wv[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-    float f[16];
-    float amax = 0.0f;
+  for (int t = 0; t < L::HT; ++t)
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      f[2 * i] = __uint_as_float(wv[i] << 16);
-      f[2 * i + 1] = __uint_as_float(wv[i] & 0xFFFF0000u);
-      amax = fmaxf(amax, fmaxf(fabsf(f[2 * i]), fabsf(f[2 * i + 1])));
-    }
+    for (int i = 0; i < kPVDims / 8; ++i) o_acc[t][i][0] = o_acc[t][i][1] = o_acc[t][i][2] = o_acc[t][i][3] = 0.0f;
+  float m_run[L::HT][2], l_run[L::HT][2];
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-    int E = static_cast<int>((__float_as_uint(amax) >> 23) & 0xFF) - 127;   // amax in [2^E, 2^(E+1))
-    if (amax == 0.0f) E = 14;
-    E = max(E, -100);
-    const float up = exp2i(14 - E), down = exp2i(E - 14);
-    uint32_t hv[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) hv[i] = pack_half2(f[2 * i] * up, f[2 * i + 1] * up);
-    // lane holds dims [16*lane, 16*lane+16): chunks 2*lane, 2*lane+1
-    *reinterpret_cast<uint4*>(smem + swz(h, 2 * lane)) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
-    *reinterpret_cast<uint4*>(smem + swz(h, 2 * lane + 1)) = make_uint4(hv[4], hv[5], hv[6], hv[7]);
-    if (lane == 0) qscale[h] = softmax_scale * down * kLog2e;
-  }
-
-  float o_acc[L::DW / 8][4];
-#pragma unroll
-  for (int i = 0; i < L::DW / 8; ++i) o_acc[i][0] = o_acc[i][1] = o_acc[i][2] = o_acc[i][3] = 0.0f;
-  float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.0f, 0.0f};
+  for (int t = 0; t < L::HT; ++t) m_run[t][0] = m_run[t][1] = -INFINITY, l_run[t][0] = l_run[t][1] = 0.0f;
   const int r0 = lane >> 2;   // fragment row (and row + 8)
-  const int h0 = ht * 16 + r0, h1 = h0 + 8;
+  const int h0 = ht * 16 + r0, h1 = h0 + 8;   // rows of this warp's S tile
 
   for (int c0 = key_begin; c0 < key_end; c0 += kChunk) {
     const int nk = min(kChunk, key_end - c0);
@@ -400,14 +402,18 @@ __global__ void __launch_bounds__(kAThreads, H == 16 ? 2 : 1)
       red_max[kg * H + h1] = mx1;
     }
     __syncthreads();   // every key group's row maxima
-    float mn0 = m_run[0], mn1 = m_run[1];
+    // this warp's S rows: the new running max (the same value every warp
+    // derives for those rows below) and P
+    float mn0 = m_run[0][0], mn1 = m_run[0][1];
+#pragma unroll
+    for (int t = 1; t < L::HT; ++t)   // select head tile ht without indexing registers by a variable
+      if (t == ht) mn0 = m_run[t][0], mn1 = m_run[t][1];
 #pragma unroll
     for (int g = 0; g < L::KG; ++g) {
       mn0 = fmaxf(mn0, red_max[g * H + h0]);
       mn1 = fmaxf(mn1, red_max[g * H + h1]);
     }
     const float ref0 = mn0 == -INFINITY ? 0.0f : mn0, ref1 = mn1 == -INFINITY ? 0.0f : mn1;
-    const float corr0 = exp2f(m_run[0] - ref0), corr1 = exp2f(m_run[1] - ref1);
     float sum0 = 0.0f, sum1 = 0.0f;
 #pragma unroll
     for (int j = 0; j < L::NT; ++j) {
@@ -430,65 +436,130 @@ __global__ void __launch_bounds__(kAThreads, H == 16 ? 2 : 1)
       red_sum[kg * H + h1] = sum1;
     }
     __syncthreads();   // P and every key group's row sums
-    float tot0 = 0.0f, tot1 = 0.0f;
+    // every head tile's rows: running max, sum and the rescaling of O
 #pragma unroll
-    for (int g = 0; g < L::KG; ++g) {
-      tot0 += red_sum[g * H + h0];
-      tot1 += red_sum[g * H + h1];
-    }
-    l_run[0] = l_run[0] * corr0 + tot0;
-    l_run[1] = l_run[1] * corr1 + tot1;
-    m_run[0] = mn0;
-    m_run[1] = mn1;
+    for (int t = 0; t < L::HT; ++t) {
 #pragma unroll
-    for (int i = 0; i < L::DW / 8; ++i) {
-      o_acc[i][0] *= corr0; o_acc[i][1] *= corr0;
-      o_acc[i][2] *= corr1; o_acc[i][3] *= corr1;
+      for (int hf = 0; hf < 2; ++hf) {
+        const int row = t * 16 + r0 + 8 * hf;
+        float mn = m_run[t][hf], tot = 0.0f;
+#pragma unroll
+        for (int g = 0; g < L::KG; ++g) {
+          mn = fmaxf(mn, red_max[g * H + row]);
+          tot += red_sum[g * H + row];
+        }
+        const float ref = mn == -INFINITY ? 0.0f : mn;
+        const float corr = exp2f(m_run[t][hf] - ref);
+        l_run[t][hf] = l_run[t][hf] * corr + tot;
+        m_run[t][hf] = mn;
+#pragma unroll
+        for (int i = 0; i < kPVDims / 8; ++i) {
+          o_acc[t][i][2 * hf] *= corr;
+          o_acc[t][i][2 * hf + 1] *= corr;
+        }
+      }
     }
 
-    // ---- O += P V: this warp's 16 heads x DW dims over the chunk's 64 keys ----
+    // ---- O += P V: every head x this warp's 64 dims over the chunk's 64 keys ----
 #pragma unroll
     for (int kk = 0; kk < kChunk / 16; ++kk) {
-      uint32_t a0, a1, a2, a3;
-      ldsm_x4(sbase + L::p_off + pswz(ht * 16 + (lane & 15), kk * 2 + (lane >> 4)), a0, a1, a2, a3);
+      uint32_t a[L::HT][4];
 #pragma unroll
-      for (int np = 0; np < L::DW / 16; ++np) {
+      for (int t = 0; t < L::HT; ++t)
+        ldsm_x4(sbase + L::p_off + pswz(t * 16 + (lane & 15), kk * 2 + (lane >> 4)), a[t][0], a[t][1], a[t][2],
+                a[t][3]);
+#pragma unroll
+      for (int np = 0; np < kPVDims / 16; ++np) {
         const int mi = lane >> 3;
-        const int dchunk = (kg * L::DW) / 8 + np * 2 + (mi >> 1);
+        const int dchunk = (warp * kPVDims) / 8 + np * 2 + (mi >> 1);
         uint32_t b0, b1, b2, b3;
         ldsm_x4_t(sbase + L::kv_off + swz(kk * 16 + (mi & 1) * 8 + (lane & 7), dchunk), b0, b1, b2, b3);
-        mma_f16(o_acc[2 * np], a0, a1, a2, a3, b0, b1);
-        mma_f16(o_acc[2 * np + 1], a0, a1, a2, a3, b2, b3);
+#pragma unroll
+        for (int t = 0; t < L::HT; ++t) {
+          mma_f16(o_acc[t][2 * np], a[t][0], a[t][1], a[t][2], a[t][3], b0, b1);
+          mma_f16(o_acc[t][2 * np + 1], a[t][0], a[t][1], a[t][2], a[t][3], b2, b3);
+        }
       }
     }
   }
 
-  // ---- partial O slices, maxima and sums into their owners' shared memory ----
-  // Output dims [kODims*r, kODims*(r+1)) belong to CTA r; it receives every
-  // rank's slice of them in recv[src][h][kODims] (16-byte granules of a
-  // head's row XOR-swizzled by the head) and every rank's (m, l) in
-  // ml_sh[src].  Every CTA of the cluster passes both barriers.
-  cluster.sync();   // every CTA is done reading its Q / KV region, which receives the partials
+  // ---- partial O slices, maxima and sums to their owners ----
+  // Output dims [kODims*r, kODims*(r+1)) belong to CTA r.  With a workspace
+  // (xchg) every CTA writes its partial O as [owner][H][kODims] fp32 plus its
+  // (m, l) into its own region of global memory (L2) and the owner reads the
+  // four slices back after one cluster barrier; without one, the slices go
+  // straight into the owner's shared memory (distributed shared memory,
+  // recv[src][h][kODims] with 16-byte granules XOR-swizzled by the head, and
+  // ml_sh[src]) between two cluster barriers.  Every CTA of the cluster
+  // passes the same barriers.
+  constexpr long long kRegion = static_cast<long long>(H) * kKvDim + 2 * H;   // floats per CTA in xchg
   float* recv = reinterpret_cast<float*>(smem);
+  const float* src_slice[kACluster];      // where the owner reads source r's slice of its dims
+  const float* src_ml[kACluster];         // ... and source r's (m[H], l[H])
+  int slice_swz;                          // 1: swizzled shared-memory slices
+  const int owner = (warp * kPVDims) / kODims, cd0 = (warp * kPVDims) % kODims;   // this warp's dims
+  if (xchg != nullptr) {
+    float* mine = xchg + static_cast<long long>(blockIdx.x) * kRegion;
+    float* dst = mine + owner * H * kODims;
 #pragma unroll
-  for (int i = 0; i < L::DW / 8; ++i) {
-    const int col = kg * L::DW + i * 8 + 2 * (lane & 3);
-    const int owner = col / kODims, cd = col % kODims;
-    float* dst = cluster.map_shared_rank(recv, owner) + rank * H * kODims;
-    *reinterpret_cast<float2*>(dst + h0 * kODims + attn_swz(h0, cd)) = make_float2(o_acc[i][0], o_acc[i][1]);
-    *reinterpret_cast<float2*>(dst + h1 * kODims + attn_swz(h1, cd)) = make_float2(o_acc[i][2], o_acc[i][3]);
-  }
-  if (kg == 0 && (lane & 3) == 0) {
+    for (int t = 0; t < L::HT; ++t)
 #pragma unroll
-    for (int o = 0; o < kACluster; ++o) {
-      float* ml = cluster.map_shared_rank(ml_sh, o) + rank * 2 * H;
-      ml[h0] = m_run[0];
-      ml[h1] = m_run[1];
-      ml[H + h0] = l_run[0];
-      ml[H + h1] = l_run[1];
+      for (int i = 0; i < kPVDims / 8; ++i) {
+        const int cd = cd0 + i * 8 + 2 * (lane & 3), row = t * 16 + r0;
+        *reinterpret_cast<float2*>(dst + row * kODims + cd) = make_float2(o_acc[t][i][0], o_acc[t][i][1]);
+        *reinterpret_cast<float2*>(dst + (row + 8) * kODims + cd) = make_float2(o_acc[t][i][2], o_acc[t][i][3]);
+      }
+    if (warp == 0 && (lane & 3) == 0) {
+#pragma unroll
+      for (int t = 0; t < L::HT; ++t)
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+          mine[H * kKvDim + t * 16 + r0 + 8 * hf] = m_run[t][hf];
+          mine[H * kKvDim + H + t * 16 + r0 + 8 * hf] = l_run[t][hf];
+        }
     }
+    cluster.sync();   // every CTA's partials are in the workspace (cluster-scope release / acquire)
+    const float* first = xchg + static_cast<long long>(blockIdx.x - rank) * kRegion;
+#pragma unroll
+    for (int r = 0; r < kACluster; ++r) {
+      src_slice[r] = first + r * kRegion + rank * H * kODims;
+      src_ml[r] = first + r * kRegion + H * kKvDim;
+    }
+    slice_swz = 0;
+  } else {
+    cluster.sync();   // every CTA is done reading its Q / KV region, which receives the partials
+    float* dst = cluster.map_shared_rank(recv, owner) + rank * H * kODims;
+#pragma unroll
+    for (int t = 0; t < L::HT; ++t)
+#pragma unroll
+      for (int i = 0; i < kPVDims / 8; ++i) {
+        const int cd = cd0 + i * 8 + 2 * (lane & 3), row = t * 16 + r0;
+        *reinterpret_cast<float2*>(dst + row * kODims + attn_swz(row, cd)) =
+            make_float2(o_acc[t][i][0], o_acc[t][i][1]);
+        *reinterpret_cast<float2*>(dst + (row + 8) * kODims + attn_swz(row + 8, cd)) =
+            make_float2(o_acc[t][i][2], o_acc[t][i][3]);
+      }
+    if (warp == 0 && (lane & 3) == 0) {
+#pragma unroll
+      for (int o = 0; o < kACluster; ++o) {
+        float* ml = cluster.map_shared_rank(ml_sh, o) + rank * 2 * H;
+#pragma unroll
+        for (int t = 0; t < L::HT; ++t)
+#pragma unroll
+          for (int hf = 0; hf < 2; ++hf) {
+            ml[t * 16 + r0 + 8 * hf] = m_run[t][hf];
+            ml[H + t * 16 + r0 + 8 * hf] = l_run[t][hf];
+          }
+      }
+    }
+    cluster.sync();   // every partial has landed; no CTA touches another's memory after this
+#pragma unroll
+    for (int r = 0; r < kACluster; ++r) {
+      src_slice[r] = recv + r * H * kODims;
+      src_ml[r] = ml_sh + r * 2 * H;
+    }
+    slice_swz = 1;
   }
-  cluster.sync();   // every partial has landed; no CTA touches another's memory after this
 
   // merge factors per (source rank, head): exp2(m_r - M) / L
   for (int h = tid; h < H; h += kAThreads) {
@@ -496,8 +567,8 @@ __global__ void __launch_bounds__(kAThreads, H == 16 ? 2 : 1)
     float M = -INFINITY;
 #pragma unroll
     for (int r = 0; r < kACluster; ++r) {
-      mr[r] = ml_sh[r * 2 * H + h];
-      lr[r] = ml_sh[r * 2 * H + H + h];
+      mr[r] = src_ml[r][h];
+      lr[r] = src_ml[r][H + h];
       M = fmaxf(M, mr[r]);
     }
     float Lsum = 0.0f;
@@ -511,13 +582,27 @@ __global__ void __launch_bounds__(kAThreads, H == 16 ? 2 : 1)
     for (int r = 0; r < kACluster; ++r) fac[r * H + h] = mr[r] * inv;
   }
   __syncthreads();
-  // this CTA writes dims [kODims*rank, kODims*(rank+1)) of every head, 4 dims per item
-  for (int item = tid; item < H * (kODims / 4); item += kAThreads) {
+  // this CTA writes dims [kODims*rank, kODims*(rank+1)) of every head, 4 dims
+  // per item; every item's partial slices are loaded before any is used
+  constexpr int kItems = H * (kODims / 4) / kAThreads;
+  static_assert(H * (kODims / 4) % kAThreads == 0, "whole items per thread");
+  float4 part[kItems][kACluster];
+#pragma unroll
+  for (int it = 0; it < kItems; ++it) {
+    const int item = it * kAThreads + tid;
+    const int h = item / (kODims / 4), d4 = (item % (kODims / 4)) * 4;
+    const int c = slice_swz ? attn_swz(h, d4) : d4;
+#pragma unroll
+    for (int r = 0; r < kACluster; ++r) part[it][r] = *reinterpret_cast<const float4*>(src_slice[r] + h * kODims + c);
+  }
+#pragma unroll
+  for (int it = 0; it < kItems; ++it) {
+    const int item = it * kAThreads + tid;
     const int h = item / (kODims / 4), d4 = (item % (kODims / 4)) * 4;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
     for (int r = 0; r < kACluster; ++r) {
-      const float4 v = *reinterpret_cast<const float4*>(recv + (r * H + h) * kODims + attn_swz(h, d4));
+      const float4 v = part[it][r];
       const float f = fac[r * H + h];
       acc.x += v.x * f; acc.y += v.y * f; acc.z += v.z * f; acc.w += v.w * f;
     }
@@ -531,7 +616,7 @@ __global__ void __launch_bounds__(kAThreads, H == 16 ? 2 : 1)
 
 template <int H>
 cudaError_t launch_h(const csa2_cache& cache, int n_layers, int n_queries, const int32_t* q_req, const int32_t* topk,
-                     int k, const AttnLayers& io, float scale, const SwaArgs& swa, cudaStream_t stream) {
+                     int k, const AttnLayers& io, float scale, const SwaArgs& swa, float* xchg, cudaStream_t stream) {
   static bool done = false;
   const size_t smem = AttnLayout<H>::total;
   if (!done) {
@@ -554,25 +639,30 @@ cudaError_t launch_h(const csa2_cache& cache, int n_layers, int n_queries, const
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  return cudaLaunchKernelEx(&cfg, sparse_attn_kernel<H>, cache, n_queries, q_req, topk, k, io, scale, swa);
+  return cudaLaunchKernelEx(&cfg, sparse_attn_kernel<H>, cache, n_queries, q_req, topk, k, io, scale, swa, xchg);
 }
 
 }  // namespace
 
+size_t attn_workspace_bytes(long long n_layers, long long n_queries, int H) {
+  return static_cast<size_t>(n_layers * n_queries * kACluster) * (static_cast<size_t>(H) * kKvDim + 2 * H) * 4;
+}
+
 cudaError_t launch_sparse_attn(const csa2_cache& cache, int n_layers, int n_queries, const int32_t* q_req,
                                const int32_t* topk, int k, const uint16_t* const* q, int H, float scale,
                                uint16_t* const* out, cudaStream_t stream, const uint8_t* swa_codes,
-                               const uint8_t* swa_exp, const int32_t* q_pos, int window) {
+                               const uint8_t* swa_exp, const int32_t* q_pos, int window, void* xchg) {
   AttnLayers io = {};
   for (int l = 0; l < n_layers; ++l) {
     io.q[l] = reinterpret_cast<const __nv_bfloat16*>(q[l]);
     io.out[l] = reinterpret_cast<__nv_bfloat16*>(out[l]);
   }
   const SwaArgs swa = {swa_codes, swa_exp, q_pos, window};
+  float* xf = static_cast<float*>(xchg);
   switch (H) {
-    case 16: return launch_h<16>(cache, n_layers, n_queries, q_req, topk, k, io, scale, swa, stream);
-    case 32: return launch_h<32>(cache, n_layers, n_queries, q_req, topk, k, io, scale, swa, stream);
-    case 64: return launch_h<64>(cache, n_layers, n_queries, q_req, topk, k, io, scale, swa, stream);
+    case 16: return launch_h<16>(cache, n_layers, n_queries, q_req, topk, k, io, scale, swa, xf, stream);
+    case 32: return launch_h<32>(cache, n_layers, n_queries, q_req, topk, k, io, scale, swa, xf, stream);
+    case 64: return launch_h<64>(cache, n_layers, n_queries, q_req, topk, k, io, scale, swa, xf, stream);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -49,7 +49,9 @@ cudaError_t launch_copy_topk(const int32_t* src, int32_t* dst, long long n, cuda
 cudaError_t launch_sparse_attn(const csa2_cache& cache, int n_layers, int n_queries, const int32_t* q_req,
                                const int32_t* topk, int k, const uint16_t* const* q, int H, float scale,
                                uint16_t* const* out, cudaStream_t stream, const uint8_t* swa_codes = nullptr,
-                               const uint8_t* swa_exp = nullptr, const int32_t* q_pos = nullptr, int window = 0);
+                               const uint8_t* swa_exp = nullptr, const int32_t* q_pos = nullptr, int window = 0,
+                               void* xchg = nullptr);
+size_t attn_workspace_bytes(long long n_layers, long long n_queries, int H);
 cudaError_t launch_swa_append(const csa2_cache& cache, int window, uint8_t* swa_codes, uint8_t* swa_exp, int n_rows,
                               const float* x, const int32_t* req, const int32_t* pos, cudaStream_t stream);
 

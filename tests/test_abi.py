@@ -25,7 +25,7 @@ def declared_symbols():
 
 def test_every_declared_symbol_is_exported(lib):
     names = declared_symbols()
-    assert len(names) == 16, names
+    assert len(names) == 17, names
     so = ctypes.CDLL(lib.LIB_PATH)
     for n in names:
         assert hasattr(so, n), f"{n} missing from libcsa2.so"
@@ -82,6 +82,17 @@ def test_host_side_validation(lib):
     assert ca(ctypes.byref(c), -1, 2, P, P, None, P, None) == lib.ERR_SHAPE
     assert ca(ctypes.byref(c), 4, 2, None, P, None, P, None) == lib.ERR_ARG
     assert ca(ctypes.byref(c), 0, 2, None, None, None, None, None) == lib.OK
+    # multi-layer attention: the optional exchange workspace is checked on the host
+    aw = L.csa2_attn_workspace_bytes
+    assert aw(2, 3, 64) == 2 * 3 * 4 * (64 * 512 + 2 * 64) * 4 and aw(-1, 3, 64) == 0
+    al = L.csa2_sparse_attn_layers
+    qa = (ctypes.c_void_p * 2)(p, p)
+    wneed = aw(2, 2, 64)
+    assert al(ctypes.byref(c), 2, 2, None, P, 512, qa, 64, ctypes.c_float(0.1), qa, P, wneed - 4, None) == lib.ERR_SHAPE
+    assert b"csa2_attn_workspace_bytes" in L.csa2_last_error_message()
+    assert al(ctypes.byref(c), 2, 2, None, P, 512, qa, 64, ctypes.c_float(0.1), qa, ctypes.c_void_p(p + 4), wneed,
+              None) == lib.ERR_ARG
+    assert al(ctypes.byref(c), 9, 2, None, P, 512, qa, 64, ctypes.c_float(0.1), qa, None, 0, None) == lib.ERR_SHAPE
     ps = L.csa2_prefill_index_static
     assert ps(ctypes.byref(c), 0, 257, P, 2, P, P, 512, P, None) == lib.ERR_SHAPE   # above the static limit
     assert b"static scratch" in L.csa2_last_error_message()

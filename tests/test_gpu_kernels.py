@@ -359,6 +359,29 @@ def test_sparse_attention_layers_equal_single_layer_launches(csa2):
     assert csa2.get_error(cache)[0] == csa2.OK
 
 
+@pytest.mark.parametrize("H,k,n_layers", [(64, 512, 4), (16, 300, 2), (32, 77, 1)])
+def test_sparse_attention_workspace_exchange_is_bit_identical(csa2, H, k, n_layers):
+    """The key splits merging through the caller's workspace (L2) give exactly
+    the output of the merge through distributed shared memory; ragged Top-k
+    with -1 padding, a query with no valid entry."""
+    wl = W.scaled(W.WORKLOADS["group_64k_b8"], batch=3, ctx=5000, heads=H)
+    cache = U.build_cache(wl, csa2)
+    dev = cache.device
+    rng = np.random.default_rng(23 + H)
+    topk = np.stack([np.sort(rng.choice(5000, k, replace=False)) for _ in range(3)]).astype(np.int32)
+    topk[1, k // 3:] = -1
+    topk[2, :] = -1
+    topk = torch.from_numpy(topk).to(dev)
+    qs = [W.main_query(wl, layer).to(dev) for layer in range(n_layers)]
+    ws = torch.full((csa2.attn_workspace_bytes(n_layers, 3, H),), 0xFF, dtype=torch.uint8, device=dev)
+    via_smem = csa2.sparse_attn_layers(cache, topk, qs, wl.scale)
+    via_ws = csa2.sparse_attn_layers(cache, topk, qs, wl.scale, workspace=ws)
+    for layer in range(n_layers):
+        assert torch.equal(via_ws[layer], via_smem[layer]), f"layer {layer}"
+        assert torch.all(via_ws[layer][2] == 0), "a query with no valid entry attends to nothing"
+    assert csa2.get_error(cache)[0] == csa2.OK
+
+
 def test_sparse_attention_empty_and_query_map(csa2):
     wl = W.scaled(W.WORKLOADS["full_4k_b1"], batch=2, heads=16, page_size=1024)
     cache = U.build_cache(wl, csa2, lengths=[2000, 3000])
