@@ -90,6 +90,22 @@ def test_reference_arm_json_small(monkeypatch):
     assert line["impl"] == "reference" and line["value"] > 0 and line["unit"] == "queries/s"
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["cpu_baseline"]["kind"] == "oracle"
     assert line["cpu_baseline"]["cores"] >= 1
+    assert line["timed_steps"] == 2
+
+
+def test_reference_arm_is_time_boxed(monkeypatch):
+    """Past the time box the reference arm stops after the query in progress,
+    so a large --steps still ends within minutes; the line says how many
+    steps it timed."""
+    monkeypatch.setenv("RANK", "0")
+    monkeypatch.setenv("WORLD_SIZE", "1")
+    monkeypatch.setattr(bench, "REFERENCE_TIME_BOX_S", 0)
+    buf = io.StringIO()
+    with redirect_stdout(buf):
+        bench.main(["--impl", "reference", "--workload", "full_4k_b1", "--steps", "500", "--warmup", "20"])
+    line = json.loads(buf.getvalue().strip().splitlines()[-1])
+    assert line["timed_steps"] == 1 and line["steps"] == 500 and line["value"] > 0
+    assert "1 of the 500 steps" in line["cpu_baseline"]["sample"]
 
 
 def test_reference_arm_other_ranks_do_nothing(monkeypatch):
