@@ -31,8 +31,8 @@ from __future__ import annotations
 
 import numpy as np
 
-from .formats import (dequantize_indexer, dequantize_main_kv, e4m3_value,
-                      indexer_sigma, quantize_indexer)
+from .formats import (dequantize_indexer, dequantize_indexer_fp4, dequantize_main_kv, e4m3_value,
+                      indexer_sigma, quantize_indexer, quantize_indexer_fp4)
 
 INDEX_HEADS = 32
 BLOCK = 8            # positions per pool block
@@ -67,6 +67,23 @@ def indexer_scores(q, w, ik_codes, ik_exp, chunk: int = 1 << 16) -> np.ndarray:
         relu = np.maximum(dots * sq, 0.0)
         out[a:a + chunk] = indexer_sigma(ik_exp[a:a + chunk]) * (relu @ w)
     return out
+
+
+def indexer_scores_fp4(q, w, k_packed, k_scales) -> np.ndarray:
+    """Full-mode score of every given row for one query, FP4 indexer variant
+    (reading: q per head and k both in the FP4 format of
+    formats.quantize_indexer_fp4; the pages give V4's indexer Q/K as FP4 but no
+    score function).  s_t = sum_h w_h ReLU(<q~_h, k~_t>) with q~, k~ the
+    dequantised values.  Each product of two dequantised values is a multiple
+    of 2^-20 below 2^23, so every dot product is exact in float64.
+
+    q: [32,128] fp32; w: [32]; k_packed: [N,64] uint8; k_scales: [N,8] uint8.
+    """
+    qc, qs = quantize_indexer_fp4(q)
+    qv = dequantize_indexer_fp4(qc, qs)                      # [32,128]
+    kv = dequantize_indexer_fp4(k_packed, k_scales)          # [N,128]
+    w = np.asarray(w, dtype=np.float32).astype(np.float64)
+    return np.maximum(kv @ qv.T, 0.0) @ w
 
 
 def block_max(scores, n: int | None = None) -> np.ndarray:

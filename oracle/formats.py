@@ -176,6 +176,39 @@ def dequantize_main_kv(packed, scale_code) -> np.ndarray:
     return (vals * s).reshape(*lead, MAIN_KV_DIM)
 
 
+# ------------------------------------------------ indexer K / Q (FP4 variant) -
+
+def quantize_indexer_fp4(k):
+    """FP4 indexer rows k[..., 128] (fp32 values) -> (packed E2M1 codes uint8
+    [..., 64], E4M3 scales uint8 [..., 8]).
+
+    The indexer variant the pages describe for V4, whose indexer Q and K were
+    FP4 [animattoys article, section 把精度降到4比特].  Reading: the main-KV
+    format applied to the 128-element row, one E4M3 scale per 16 elements,
+    s = E4M3(amax / 6), codes = E2M1(x / s), byte i = element 2i (low nibble)
+    and 2i + 1 (high nibble); no per-row or global scale.
+    """
+    x = np.asarray(k, dtype=np.float32).astype(np.float64)
+    assert x.shape[-1] == INDEXER_DIM
+    lead = x.shape[:-1]
+    groups = x.reshape(*lead, INDEXER_DIM // GROUP, GROUP)
+    scale_code = e4m3_encode(np.abs(groups).max(axis=-1) / 6.0)
+    codes = e2m1_encode(groups, e4m3_value(scale_code)[..., None]).reshape(*lead, INDEXER_DIM)
+    packed = codes[..., 0::2] | (codes[..., 1::2] << 4)
+    return packed.astype(np.uint8), scale_code.astype(np.uint8)
+
+
+def dequantize_indexer_fp4(packed, scale_code) -> np.ndarray:
+    """FP4 indexer rows [..., 128] in float64 from packed codes and scales."""
+    packed = np.asarray(packed, dtype=np.uint8)
+    lead = packed.shape[:-1]
+    codes = np.empty((*lead, INDEXER_DIM), dtype=np.uint8)
+    codes[..., 0::2] = packed & 0xF
+    codes[..., 1::2] = packed >> 4
+    vals = e2m1_value(codes).reshape(*lead, INDEXER_DIM // GROUP, GROUP)
+    return (vals * e4m3_value(scale_code)[..., None]).reshape(*lead, INDEXER_DIM)
+
+
 # ------------------------------------------------------- indexer K / Q (FP8) -
 
 def indexer_exponent(amax) -> np.ndarray:

@@ -57,6 +57,63 @@ def test_score_one_hot_closed_form():
         np.testing.assert_array_equal(C.indexer_scores(q, w, codes, byte), np.maximum(kd[:, d], 0) * 3.0)
 
 
+# ------------------------------------------------ score, FP4 indexer variant --
+
+def _fp4_exact_rows(rng, n):
+    """Rows whose every 16-element group is (E2M1 grid value) x s with the
+    group's largest magnitude exactly 6 s and s an E4M3 value: the FP4 format
+    holds them exactly."""
+    grid = F.e2m1_value(rng.integers(0, 16, (n, 128)))
+    grid = grid.reshape(n, 8, 16)
+    grid[:, :, 0] = 6.0 * np.where(rng.random((n, 8)) < 0.5, -1.0, 1.0)
+    s = F.e4m3_value(rng.integers(1, 127, (n, 8)))            # positive scales, subnormals included
+    return (grid * s[..., None]).reshape(n, 128).astype(np.float32)
+
+
+def test_fp4_score_reduces_to_plain_formula_on_exact_inputs():
+    """Inputs the FP4 format holds exactly quantise to themselves, so the FP4
+    score is the plain float64 sum_h w_h ReLU(q_h . k_t), evaluated here with
+    torch (library); the stored codes dequantise to the inputs bit for bit."""
+    rng = np.random.default_rng(11)
+    k = _fp4_exact_rows(rng, 60)
+    q = _fp4_exact_rows(rng, 32)
+    w = rng.random(32).astype(np.float32)
+    kp, ks = F.quantize_indexer_fp4(k)
+    np.testing.assert_array_equal(F.dequantize_indexer_fp4(kp, ks), k.astype(np.float64))
+    ours = C.indexer_scores_fp4(q, w, kp, ks)
+    ref = torch.relu(torch.from_numpy(k).double() @ torch.from_numpy(q).double().T) @ torch.from_numpy(w).double()
+    np.testing.assert_allclose(ours, ref.numpy(), rtol=1e-15, atol=0)
+    dots = k.astype(np.float64) @ q.astype(np.float64).T
+    assert (dots < 0).mean() > 0.2                          # the ReLU drops a good share of the head terms
+
+
+def test_fp4_indexer_format_is_the_main_kv_format():
+    """The FP4 indexer row is the main-KV format on 128 elements: four indexer
+    rows laid end to end quantise exactly like one 512-channel main-KV row
+    (an independent implementation of the same rule)."""
+    rng = np.random.default_rng(12)
+    k = (rng.standard_normal((40, 128)) * np.exp(rng.normal(0, 2, (40, 1)))).astype(np.float32)
+    k[3] = 0.0
+    kp, ks = F.quantize_indexer_fp4(k)
+    mp, ms = F.quantize_main_kv(k.reshape(10, 512))
+    np.testing.assert_array_equal(kp.reshape(10, 256), mp)
+    np.testing.assert_array_equal(ks.reshape(10, 32), ms)
+
+
+def test_fp4_score_power_of_two_scaling_and_head_permutation():
+    """Scaling the query by 2^j moves every E4M3 scale by j exponents and
+    leaves the codes alone (inside the normal range), so scores scale by 2^j
+    exactly; permuting the heads together with their weights changes nothing."""
+    rng = np.random.default_rng(13)
+    k = rng.standard_normal((50, 128)).astype(np.float32)
+    q, w = _query(rng)
+    kp, ks = F.quantize_indexer_fp4(k)
+    base = C.indexer_scores_fp4(q, w, kp, ks)
+    np.testing.assert_array_equal(C.indexer_scores_fp4(q * np.float32(4.0), w, kp, ks), base * 4.0)
+    perm = rng.permutation(32)
+    np.testing.assert_array_equal(C.indexer_scores_fp4(q[perm], w[perm], kp, ks), base)
+
+
 def test_score_structure():
     rng = np.random.default_rng(2)
     codes, byte = _idx_rows(rng, 300)

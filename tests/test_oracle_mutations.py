@@ -164,3 +164,38 @@ def test_mutation_swa_merge_by_halves(monkeypatch):
         return 0.5 * o1 + 0.5 * (p / p.sum(1, keepdims=True)) @ k2
     monkeypatch.setattr(C, "sparse_attention_swa", wrong)
     _fails(PC.test_swa_attention_is_the_softmax_merge_of_its_two_parts)
+
+
+def test_mutation_fp4_indexer_nibble_order(monkeypatch):
+    orig = F.quantize_indexer_fp4
+
+    def bad(k):
+        p, s = orig(k)
+        return ((p >> 4) | (p << 4)).astype(np.uint8), s
+    monkeypatch.setattr(F, "quantize_indexer_fp4", bad)
+    monkeypatch.setattr(C, "quantize_indexer_fp4", bad)
+    _fails(PC.test_fp4_indexer_format_is_the_main_kv_format)
+    _fails(PC.test_fp4_score_reduces_to_plain_formula_on_exact_inputs)
+
+
+def test_mutation_fp4_indexer_group_of_32(monkeypatch):
+    def bad(k):
+        x = np.asarray(k, dtype=np.float32).astype(np.float64)
+        lead = x.shape[:-1]
+        g = x.reshape(*lead, 4, 32)
+        sc = F.e4m3_encode(np.abs(g).max(axis=-1) / 6.0)
+        codes = F.e2m1_encode(g, F.e4m3_value(sc)[..., None]).reshape(*lead, 128)
+        return (codes[..., 0::2] | (codes[..., 1::2] << 4)).astype(np.uint8), np.repeat(sc, 2, axis=-1).astype(np.uint8)
+    monkeypatch.setattr(F, "quantize_indexer_fp4", bad)
+    monkeypatch.setattr(C, "quantize_indexer_fp4", bad)
+    _fails(PC.test_fp4_indexer_format_is_the_main_kv_format)
+    _fails(PC.test_fp4_score_reduces_to_plain_formula_on_exact_inputs)
+
+
+def test_mutation_fp4_score_drops_relu(monkeypatch):
+    def bad(q, w, kp, ks):
+        qv = F.dequantize_indexer_fp4(*F.quantize_indexer_fp4(q))
+        kv = F.dequantize_indexer_fp4(kp, ks)
+        return (kv @ qv.T) @ np.asarray(w, dtype=np.float64)
+    monkeypatch.setattr(C, "indexer_scores_fp4", bad)
+    _fails(PC.test_fp4_score_reduces_to_plain_formula_on_exact_inputs)
