@@ -344,7 +344,11 @@ CSA2_API size_t csa2_attn_workspace_bytes(int32_t n_layers, int32_t n_queries, i
  * csa2_sparse_attn_swa -- csa2_sparse_attn of one layer with its window merged
  * in: query i attends over its Top-k rows and the window tokens
  * max(0, q_pos[i] - window + 1) .. q_pos[i] of its request (q_pos int32
- * [n_queries], device).  window in [1, CSA2_SWA_MAX_WINDOW].
+ * [n_queries], device).  window in [1, CSA2_SWA_MAX_WINDOW].  Window rows are
+ * decoded to fp16 like the Top-k rows: exact while the row's largest
+ * magnitude stays below 2^15 (a larger row overflows fp16 and the query's
+ * output is undefined); rows below about 2^-14 lose low bits to fp16
+ * subnormals.
  */
 #define CSA2_SWA_MAX_WINDOW 4096
 CSA2_API csa2_status csa2_swa_append(const csa2_cache* cache, int32_t window, uint8_t* swa_codes,
