@@ -185,6 +185,62 @@ def test_group_1m_b4_full_size(csa2):
     assert csa2.get_error(cache)[0] == csa2.OK
 
 
+def test_group_ragged_b64_full_size(csa2):
+    """The 64-request ragged workload at full size (log-uniform contexts from
+    4,096 to 1,048,576 positions behind a shuffled page table, one append per
+    request, 1 Full + 4 Reindex + 1 Reuse): every appended row bit-exact; the
+    two shortest requests against the full oracle; every request on sampled
+    block maxima and on properties that hold at any size."""
+    wl = W.WORKLOADS["ragged_b64"]
+    n = W.ctx_lengths(wl)
+    cache = U.build_cache(wl, csa2, append_last=True)
+    dev = cache.device
+    last = n - 1
+    kv = np.stack([W.rows_at(wl, b, [last[b]], "kv")[0] for b in range(wl.batch)])
+    ik = np.stack([W.rows_at(wl, b, [last[b]], "ik")[0] for b in range(wl.batch)])
+    rows = (torch.from_numpy(kv).to(dev), torch.from_numpy(ik).to(dev),
+            torch.from_numpy(last.astype(np.int32)).to(dev))
+    group, q_idx, w_idx, q_main, out = _run_gpu(csa2, wl, cache, dev, append_rows=rows)
+    assert csa2.get_error(cache)[0] == csa2.OK
+    from oracle import formats as F
+    ikc, ike = F.quantize_indexer(ik)
+    kvc, kvs = F.quantize_main_kv(kv)
+    for b in range(wl.batch):
+        row = int(cache.rows_of(b, [last[b]])[0])
+        np.testing.assert_array_equal(cache.ik_codes[row].cpu().numpy(), ikc[b])
+        assert int(cache.ik_exp[row]) == int(ike[b])
+        np.testing.assert_array_equal(cache.kv_codes[row].cpu().numpy(), kvc[b])
+        np.testing.assert_array_equal(cache.kv_scales[row].cpu().numpy(), kvs[b])
+    for b in np.argsort(n)[:2]:
+        _check_request(csa2, wl, cache, group, int(b), int(n[b]), q_idx, w_idx, q_main, out, dev)
+    rng = np.random.default_rng(1)
+    bm_all = group.blockmax.cpu().numpy()
+    pools = group.pool.cpu().numpy()
+    for b in range(wl.batch):
+        nb = -(-int(n[b]) // 8)
+        bm = bm_all[b, :nb].astype(np.float64)
+        gp = pools[b]
+        order = np.lexsort((np.arange(nb), -bm))
+        want = np.full(wl.pool_blocks, -1, np.int64)
+        want[:min(nb, wl.pool_blocks)] = np.sort(order[:wl.pool_blocks])
+        np.testing.assert_array_equal(gp, want, err_msg=f"pool b={b}: not the top blocks of the GPU's maxima")
+        blocks = rng.choice(nb, min(nb, 64), replace=False)
+        pos = (blocks[:, None] * 8 + np.arange(8)).reshape(-1)
+        keep = pos < n[b]
+        codes, exp = F.quantize_indexer(W.rows_at(wl, b, pos[keep], "ik"))
+        s64 = np.full(len(pos), -np.inf)
+        s64[keep] = C.indexer_scores(q_idx[0][b], w_idx[0][b], codes, exp)
+        bm64 = s64.reshape(-1, 8).max(axis=1)
+        assert np.all(np.abs(bm[blocks] - bm64) <= 1e-5 * np.abs(bm64)), f"block maxima b={b}"
+        pool_pos = set(C.pool_positions(gp, int(n[b])).tolist())
+        for layer, m in enumerate(wl.modes):
+            t = group.topk[layer][b].cpu().numpy()
+            U.assert_sorted_padded(t, f"topk layer {layer} b={b}")
+            assert (t >= 0).sum() == min(wl.topk, int(n[b])) and set(t[t >= 0].tolist()) <= pool_pos
+            if m == "Ru":
+                np.testing.assert_array_equal(t, group.topk[layer - 1][b].cpu().numpy())
+
+
 def test_group_graph_replay_matches_eager(csa2):
     """The bench times CUDA-graph replays of the step (side streams and
     programmatic dependent launch inside the graph); a replay must give the
