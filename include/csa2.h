@@ -39,6 +39,10 @@
  *     first one in cache->err_word and skips or neutralises the offending
  *     element; csa2_get_error() reads it back.
  *   - Launch failures return CSA2_ERR_CUDA.
+ *   - One device per process: each kernel's launch attributes (dynamic shared
+ *     memory size, cluster size) are set on its first launch in the process,
+ *     on the device current then.  Use one process per GPU (the intended
+ *     deployment: data parallel over requests).
  *   - Kernels are launched with programmatic dependent launch: each one waits
  *     for the kernel before it on the stream before reading anything that
  *     kernel may write, and lets its own successor start early.  The
