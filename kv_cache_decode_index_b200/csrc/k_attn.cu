@@ -5,8 +5,9 @@
 //
 // One thread-block cluster of kACluster (4) CTAs per (layer, query).  CTA r
 // takes entries [r*kc, (r+1)*kc) (kc = ceil(k/4)) in chunks of 64 rows:
-//   * prologue: the query's bf16 rows are loaded while the CTA turns its
-//     Top-k entries into cache rows (page table) once, into shared memory;
+//   * prologue: the query's bf16 rows are loaded and converted before the
+//     wait on the preceding launch, then the CTA turns its Top-k entries into
+//     cache rows (page table) once, into shared memory;
 //   * the packed rows (256 code bytes + 32 scale bytes each) are copied into
 //     a staging buffer by cp.async one chunk ahead of their use and
 //     dequantised shared -> shared with the E2M1 -> f16x2 conversion: E2M1
@@ -17,12 +18,13 @@
 //   * S = Q K^T on mma.sync m16n8k16 (fp16 in, fp32 accumulate) with the
 //     chunk's keys split over the warps, an online softmax in fp32 (exp2
 //     domain) whose row maxima and sums are combined through shared memory,
-//     P rounded to fp16 in shared memory, O += P V with the 512 output dims
-//     split over the warps;
-// then every CTA stores its partial O slice of dims [128r, 128r+128) straight
-// into CTA r's shared memory (distributed shared memory) together with its
-// (max, sum) pairs, and after a cluster barrier CTA r merges the four
-// partials and writes those dims of every head.  Four CTAs per query keep all
+//     P rounded to fp16 in shared memory, O += P V with each warp on 64 of
+//     the 512 output dims of every head;
+// then CTA r merges the four partial (O, max, sum) sets for output dims
+// [128r, 128r+128) and writes those dims of every head.  The partials reach
+// it through a caller workspace in global memory (L2) when one is given,
+// else by stores into its shared memory from the other CTAs (distributed
+// shared memory), between cluster barriers.  Four CTAs per query keep all
 // six layers' attention of a decode step within one wave of the GPU's SMs.
 #include <cooperative_groups.h>
 #include <cuda_bf16.h>
