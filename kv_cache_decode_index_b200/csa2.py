@@ -348,6 +348,26 @@ def get_error(cache: Cache):
     return st, list(out)
 
 
+def layer_sources(modes):
+    """Group the layers of a layer group by the Top-k they attend over: each
+    Full or Reindex layer starts a group, and the Reuse layers that follow it
+    join that group (a Reuse layer takes the most recent Full/Reindex layer's
+    indices).  Returns a list of lists of layer indices."""
+    modes = tuple(modes)
+    if not modes or modes[0] == "Ru":
+        raise ValueError("a layer group starts with a Full or Reindex layer")
+    bad = [m for m in modes if m not in ("F", "Ri", "Ru")]
+    if bad:
+        raise ValueError(f"unknown layer modes {bad}")
+    sources = []
+    for layer, m in enumerate(modes):
+        if m != "Ru":
+            sources.append([layer])
+        else:
+            sources[-1].append(layer)
+    return sources
+
+
 class DecodeGroup:
     """One decode step of a CSA2 layer group over `cache`, through the C ABI.
 
@@ -379,12 +399,7 @@ class DecodeGroup:
                 self.topk.append(src)
         self.concurrent = concurrent
         # attention launches: each Full/Reindex layer with the Reuse layers that follow it
-        self.sources = []
-        for layer, m in enumerate(self.modes):
-            if m != "Ru":
-                self.sources.append([layer])
-            else:
-                self.sources[-1].append(layer)
+        self.sources = layer_sources(self.modes)
         # the last source's chain (pool -> Top-k -> attention) runs on the
         # calling stream, linked by programmatic dependent launch; the other
         # sources run on streams of their own, after the pool
@@ -465,15 +480,12 @@ class PrefillGroup:
         self.n = n_queries
         self.workspace = torch.empty(max(prefill_workspace_bytes(n_queries), 16), dtype=torch.uint8, device=dev)
         self.q_req = torch.full((n_queries,), req, dtype=torch.int32, device=dev)
-        self.topk, src = [], None
-        self.sources = []
-        for layer, m in enumerate(self.modes):
-            if m != "Ru":
-                src = torch.empty(n_queries, k, dtype=torch.int32, device=dev)
-                self.sources.append([layer])
-            else:
-                self.sources[-1].append(layer)
-            self.topk.append(src)
+        self.sources = layer_sources(self.modes)
+        self.topk = [None] * len(self.modes)
+        for layers in self.sources:
+            src = torch.empty(n_queries, k, dtype=torch.int32, device=dev)
+            for layer in layers:
+                self.topk[layer] = src
         self.launches_per_step = 3 * len(self.sources)   # indexer (2 kernels) + one attention launch per source
 
     def step(self, q_pos, q_idx, w_idx, q_main, out, timing=None):
