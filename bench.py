@@ -234,6 +234,8 @@ def oracle_sample(wl, b: int = 0, prepared=None):
 
 
 def cpu_cores():
+    """Threads the oracle's numpy BLAS calls use (the rest of the oracle is
+    single-threaded numpy)."""
     try:
         import threadpoolctl
         info = threadpoolctl.threadpool_info()
@@ -243,6 +245,20 @@ def cpu_cores():
     except Exception:
         pass
     return 1
+
+
+def cpu_host():
+    """The host the CPU baseline ran on: logical CPUs and the CPU model."""
+    model = None
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return {"nproc": os.cpu_count(), "cpu_model": model}
 
 
 # --------------------------------------------------------------- b200 arm ----
@@ -527,7 +543,7 @@ def run_prefill(args):
             "clocks": clocks}
     if not args.no_cpu_baseline:
         spq = prefill_oracle_sample(wl)
-        line["cpu_baseline"] = {"value": 1.0 / spq, "unit": "queries/s", "cores": cpu_cores(), "kind": "oracle",
+        line["cpu_baseline"] = {"value": 1.0 / spq, "unit": "queries/s", "cores": cpu_cores(), **cpu_host(), "kind": "oracle",
                                 "sample": f"2 of the {n} queries: float64 oracle Top-512 over all visible entries "
                                           f"and six attention layers, {spq:.1f} s per query"}
     print(json.dumps(line), flush=True)
@@ -639,7 +655,7 @@ def max_over_ranks(x: float, dev, world: int) -> float:
 
 def cpu_baseline_entry(wl):
     secs, _ = oracle_sample(wl, 0)
-    return {"value": 1.0 / secs, "unit": "queries/s", "cores": cpu_cores(), "kind": "oracle",
+    return {"value": 1.0 / secs, "unit": "queries/s", "cores": cpu_cores(), **cpu_host(), "kind": "oracle",
             "sample": f"1 of the {wl.batch} queries of one step (request 0, full {int(W.ctx_lengths(wl)[0]):,}-position "
                       f"context): float64 numpy oracle, whole layer-group step, {secs:.1f} s"}
 
@@ -668,7 +684,7 @@ def run_reference(args):
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
                 "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
                 "config": {"workload": wl.name},
-                "cpu_baseline": {"value": 1e3 / ms, "unit": "queries/s", "cores": cpu_cores(), "kind": "oracle",
+                "cpu_baseline": {"value": 1e3 / ms, "unit": "queries/s", "cores": cpu_cores(), **cpu_host(), "kind": "oracle",
                                  "sample": f"one prefill query per step, float64 oracle; {len(times)} of the "
                                            f"{args.steps} steps timed inside a {REFERENCE_TIME_BOX_S} s box"},
                 "timed_steps": len(times),
@@ -692,7 +708,7 @@ def run_reference(args):
     value = 1e3 / ms
     line = base_line(args, wl, world, value, ms)
     line.update({"impl": "reference", "dtype": "f64",
-                 "cpu_baseline": {"value": value, "unit": "queries/s", "cores": cpu_cores(), "kind": "oracle",
+                 "cpu_baseline": {"value": value, "unit": "queries/s", "cores": cpu_cores(), **cpu_host(), "kind": "oracle",
                                   "sample": f"one query per step (requests cycled), full context, float64 numpy "
                                             f"oracle of the whole layer-group step; {len(times)} of the {args.steps} "
                                             f"steps timed inside a {REFERENCE_TIME_BOX_S} s box after {warm} "

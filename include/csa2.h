@@ -38,11 +38,16 @@
  *     index outside the visible context) never trap: the kernel records the
  *     first one in cache->err_word and skips or neutralises the offending
  *     element; csa2_get_error() reads it back.
+ *   - A ctx_len[b] outside [0, capacity] is such a violation too: every
+ *     kernel that reads it records CSA2_ERR_DEVICE_BOUNDS with index = the
+ *     length and treats request b as empty (no scan, an all -1 pool and
+ *     Top-k, zero attention output): a corrupt length never silently
+ *     truncates a request.
  *   - Launch failures return CSA2_ERR_CUDA.
- *   - One device per process: each kernel's launch attributes (dynamic shared
- *     memory size, cluster size) are set on its first launch in the process,
- *     on the device current then.  Use one process per GPU (the intended
- *     deployment: data parallel over requests).
+ *   - Each kernel's launch attributes (dynamic shared memory size, cluster
+ *     size) are set once per CUDA context, on its first launch there: one
+ *     process may drive several devices, and a context that is destroyed and
+ *     created again is set up anew.
  *   - Kernels are launched with programmatic dependent launch: each one waits
  *     for the kernel before it on the stream before reading anything that
  *     kernel may write, and lets its own successor start early.  The
@@ -231,7 +236,8 @@ CSA2_API csa2_status csa2_reindex(const csa2_cache* cache, csa2_mode mode, const
  * H in {16, 32, 64}; k in [1, 4096].  Dequantised rows are exact in fp16,
  * logits and softmax are fp32, P.V uses fp16 probabilities with fp32 sums.
  * Device errors: a Top-k entry >= ctx_len or < -1 -> CSA2_ERR_DEVICE_BOUNDS,
- * entry skipped.
+ * entry skipped; a q_req entry outside [0, batch) -> CSA2_ERR_DEVICE_BOUNDS
+ * (request = that value, index = -1), the query's output is 0.
  */
 CSA2_API csa2_status csa2_sparse_attn(const csa2_cache* cache, int32_t n_queries, const int32_t* q_req,
                              const int32_t* topk, int32_t k, const uint16_t* q, int32_t H,
@@ -286,8 +292,8 @@ CSA2_API csa2_status csa2_prefill_index(const csa2_cache* cache, int32_t req, in
  * with more queries returns CSA2_ERR_SHAPE and launches nothing.  Nothing in
  * the array needs to start at zero (every list length is written before it is
  * read).  The array's device address is looked up with cudaGetSymbolAddress
- * on the first call on each device, so make that first call outside any
- * stream capture.  Every call on a device uses the same array: two calls in
+ * on the first call in each CUDA context (each device, and again in a context
+ * created anew), so make that first call outside any stream capture.  Every call on a device uses the same array: two calls in
  * flight at once on one device (other streams, other host threads) race and
  * corrupt each other's results; serialise them.  Arguments, outputs and
  * device errors are those of csa2_prefill_index.

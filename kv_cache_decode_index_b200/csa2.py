@@ -421,7 +421,11 @@ class DecodeGroup:
             ev = None if timing is None else timing.get(name)
             if ev is not None:
                 ev[0].record()
-            r = fn()
+            torch.cuda.nvtx.range_push(f"csa2 {name}")   # profiler range around the launch
+            try:
+                r = fn()
+            finally:
+                torch.cuda.nvtx.range_pop()
             if ev is not None:
                 ev[1].record()
             return r
@@ -499,7 +503,11 @@ class PrefillGroup:
             ev = None if timing is None else timing.get(name)
             if ev is not None:
                 ev[0].record()
-            fn()
+            torch.cuda.nvtx.range_push(f"csa2 {name}")
+            try:
+                fn()
+            finally:
+                torch.cuda.nvtx.range_pop()
             if ev is not None:
                 ev[1].record()
 

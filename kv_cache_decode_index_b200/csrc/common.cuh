@@ -36,6 +36,21 @@ __device__ __forceinline__ void report_error(int32_t* err, int code, int kernel,
   }
 }
 
+// Visible positions of request b, or -1 for a length outside [0, capacity]
+// (a corrupt ctx_len), which the caller that passes `report` records as
+// CSA2_ERR_DEVICE_BOUNDS with the length as the index.  Callers treat such a
+// request as empty: its results are left unwritten or padded, never computed
+// over a truncated context, and none of its entries is checked or reported.
+__device__ __forceinline__ int checked_ctx_len(const csa2_cache& c, int b, long long capacity, int kernel,
+                                               bool report) {
+  const int n = c.ctx_len[b];
+  if (n < 0 || n > capacity) {
+    if (report) report_error(c.err_word, CSA2_ERR_DEVICE_BOUNDS, kernel, b, n);
+    return -1;
+  }
+  return n;
+}
+
 __device__ __forceinline__ uint64_t globaltimer() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));

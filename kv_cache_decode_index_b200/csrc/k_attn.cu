@@ -234,8 +234,10 @@ __global__ void __launch_bounds__(kAThreads, H == 16 ? 2 : 1)
   pdl_launch_dependents();
   const int b = q_req != nullptr ? q_req[qi] : qi;
   const long long capacity = static_cast<long long>(cache.max_pages_per_req) * cache.page_size;
-  int n = (b >= 0 && b < cache.batch) ? cache.ctx_len[b] : 0;
-  n = n < 0 ? 0 : (n > capacity ? static_cast<int>(capacity) : n);
+  const bool b_ok = b >= 0 && b < cache.batch;
+  if (!b_ok && rank == 0 && tid == 0) report_error(cache.err_word, CSA2_ERR_DEVICE_BOUNDS, kKAttn, b, -1);
+  const int n_raw = b_ok ? checked_ctx_len(cache, b, capacity, kKAttn, rank == 0 && tid == 0) : -1;
+  const int n = max(0, n_raw);   // n_raw < 0: no entry of this query is used (or checked)
   const int32_t* idx = topk + static_cast<long long>(qi) * K;
 
   // ---- this CTA's entries: the Top-k entries, then the window's tokens ----
@@ -244,7 +246,7 @@ __global__ void __launch_bounds__(kAThreads, H == 16 ? 2 : 1)
   const int K_all = K + n_win;
   const int kc = (K_all + kACluster - 1) / kACluster;
   const int key_begin = min(rank * kc, K_all), key_end = min(key_begin + kc, K_all);
-  const int n_top = min(max(0, min(key_end, K) - key_begin), kMaxTop);
+  const int n_top = n_raw < 0 ? 0 : min(max(0, min(key_end, K) - key_begin), kMaxTop);
   for (int i = tid; i < n_top; i += kAThreads) {
     const int t = idx[key_begin + i];
     int r = -1;
@@ -305,7 +307,7 @@ __global__ void __launch_bounds__(kAThreads, H == 16 ? 2 : 1)
       if (row < nk && e >= K) {
         // window entry j: token p - window + 1 + j (none before token 0)
         const int tw = p_tok - n_win + 1 + (e - K);
-        const bool ok = tw >= 0 && b >= 0 && b < cache.batch;
+        const bool ok = tw >= 0 && n_raw >= 0;
         if (part == 0) kvalid[row] = ok;
         if (ok) {
           const long long slot = static_cast<long long>(b) * n_win + tw % n_win;
@@ -627,14 +629,13 @@ __global__ void __launch_bounds__(kAThreads, H == 16 ? 2 : 1)
 template <int H>
 cudaError_t launch_h(const csa2_cache& cache, int n_layers, int n_queries, const int32_t* q_req, const int32_t* topk,
                      int k, const AttnLayers& io, float scale, const SwaArgs& swa, float* xchg, cudaStream_t stream) {
-  static bool done = false;
+  static ContextMemo attrs;
   const size_t smem = AttnLayout<H>::total;
-  if (!done) {
-    cudaError_t e = cudaFuncSetAttribute(sparse_attn_kernel<H>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
-    if (e != cudaSuccess) return e;
-    done = true;
-  }
+  const cudaError_t e = attrs.once([&] {
+    return cudaFuncSetAttribute(sparse_attn_kernel<H>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                static_cast<int>(smem));
+  });
+  if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(n_layers * n_queries * kACluster);
   cfg.blockDim = dim3(kAThreads);

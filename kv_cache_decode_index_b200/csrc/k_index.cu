@@ -115,10 +115,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; i < kScanItems; ++i) {
       const int b = tid * kScanItems + i;
       int n = 0;
-      if (b < B) {
-        n = cache.ctx_len[b];
-        n = n < 0 ? 0 : (n > capacity ? static_cast<int>(capacity) : n);
-      }
+      if (b < B) n = max(0, checked_ctx_len(cache, b, capacity, kKIndexFull, blockIdx.x == 0));
       items[i] = (n + kUnit - 1) / kUnit;
     }
     int total;
@@ -380,14 +377,12 @@ size_t index_full_smem_bytes() { return sizeof(IndexSmem) + 1024; }
 cudaError_t launch_index_full(const csa2_cache& cache, const float* q, const float* w, float* blockmax,
                               float* scores, const CUtensorMap& ik_map, int num_sms, uint64_t wait_ns,
                               cudaStream_t stream) {
-  static bool configured = false;
+  static ContextMemo attrs;
   const size_t smem = index_full_smem_bytes();
-  if (!configured) {
-    const cudaError_t e = cudaFuncSetAttribute(index_full_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                               static_cast<int>(smem));
-    if (e != cudaSuccess) return e;
-    configured = true;
-  }
+  const cudaError_t e = attrs.once([&] {
+    return cudaFuncSetAttribute(index_full_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  });
+  if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(num_sms);
   cfg.blockDim = dim3(kThreads);

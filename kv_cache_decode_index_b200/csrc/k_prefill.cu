@@ -117,8 +117,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
     if (j < n_queries) {
       const long long p = q_pos[j];
       v = p < 0 ? 0 : (p + 1) / ratio;
-      long long n = cache.ctx_len[req];
-      n = n < 0 ? 0 : (n > capacity ? capacity : n);
+      const long long n = max(0, checked_ctx_len(cache, req, capacity, kKPrefill, blockIdx.x == 0 && tid == 0));
       v = v < n ? v : n;
     }
     S.vis[tid] = static_cast<int>(v);
@@ -433,19 +432,18 @@ size_t prefill_workspace_bytes(long long n_queries) {
 cudaError_t launch_prefill_index(const csa2_cache& cache, int req, int n_queries, const int32_t* q_pos, int ratio,
                                  const float* q, const float* w, int k, int32_t* topk, void* workspace,
                                  const CUtensorMap& ik_map, uint64_t wait_ns, cudaStream_t stream) {
-  static bool configured = false;
+  static ContextMemo attrs;
   const size_t smem = sizeof(PrefillSmem) + 1024;
-  if (!configured) {
-    const cudaError_t e =
-        cudaFuncSetAttribute(prefill_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-    if (e != cudaSuccess) return e;
-    configured = true;
-  }
+  cudaError_t e = attrs.once([&] {
+    return cudaFuncSetAttribute(prefill_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                static_cast<int>(smem));
+  });
+  if (e != cudaSuccess) return e;
   const Workspace wsp = split_workspace(workspace, n_queries);
   const int grid = (n_queries + kPQ - 1) / kPQ;
   prefill_scan_kernel<<<grid, kPThreads, smem, stream>>>(cache, req, n_queries, q_pos, ratio, q, w, k, wsp, ik_map,
                                                          wait_ns);
-  cudaError_t e = cudaGetLastError();
+  e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int sgrid = (n_queries + kSelWarps - 1) / kSelWarps;
   prefill_select_kernel<<<sgrid, kSelWarps * 32, 0, stream>>>(n_queries, k, wsp, topk);
@@ -461,22 +459,13 @@ constexpr long long kStaticPrefillBytes =
     static_cast<long long>(kStaticPrefillMaxQueries) * kCand * 8 + kStaticPrefillMaxQueries * 4;
 __device__ __align__(256) uint8_t g_prefill_scratch[kStaticPrefillBytes];
 
-std::mutex g_scratch_mu;
-void* g_scratch_addr[64] = {};
+// Its device address, looked up once per CUDA context (the module, and the
+// array with it, is loaded again in a context that is created anew).
+ContextMemo g_scratch_addr;
 }  // namespace
 
 cudaError_t static_prefill_scratch(void** addr) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  std::lock_guard<std::mutex> lk(g_scratch_mu);
-  if (g_scratch_addr[dev] == nullptr) {
-    e = cudaGetSymbolAddress(&g_scratch_addr[dev], g_prefill_scratch);
-    if (e != cudaSuccess) return e;
-  }
-  *addr = g_scratch_addr[dev];
-  return cudaSuccess;
+  return g_scratch_addr.get(addr, [](void** out) { return cudaGetSymbolAddress(out, g_prefill_scratch); });
 }
 
 }  // namespace csa2

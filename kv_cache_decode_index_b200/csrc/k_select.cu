@@ -38,8 +38,7 @@ __global__ void __launch_bounds__(kPoolThreads, 1)
   const int b = blockIdx.x / C;
   const long long capacity = static_cast<long long>(cache.max_pages_per_req) * cache.page_size;
   const long long stride = capacity / kBlock;
-  int n = cache.ctx_len[b];
-  n = n < 0 ? 0 : (n > capacity ? static_cast<int>(capacity) : n);
+  const int n = max(0, checked_ctx_len(cache, b, capacity, kKPoolSelect, rank == 0 && threadIdx.x == 0));
   const int nblk = (n + kBlock - 1) / kBlock;
   const int per = (nblk + C - 1) / C;
   const int j0 = min(rank * per, nblk);
@@ -127,8 +126,8 @@ __global__ void __launch_bounds__(kRThreads, 2)
   const long long capacity = static_cast<long long>(cache.max_pages_per_req) * cache.page_size;
   pdl_wait();                 // the pool (or the stored scores) of the preceding launch are complete
   pdl_launch_dependents();
-  int n = cache.ctx_len[b];
-  n = n < 0 ? 0 : (n > capacity ? static_cast<int>(capacity) : n);
+  const int n_raw = checked_ctx_len(cache, b, capacity, kKReindex, rank == 0 && tid == 0);
+  const int n = max(0, n_raw);
 
   // ---- this CTA's candidate blocks ----
   int e0, nloc;
@@ -143,6 +142,7 @@ __global__ void __launch_bounds__(kRThreads, 2)
     nloc = min(per, nblk - e0);
   }
   if (nloc > max_blocks) nloc = max_blocks;   // host guarantees this never clips
+  if (n_raw < 0) nloc = 0;                     // corrupt length: no candidates
   // block id -> page -> exponent bytes: each level's loads are issued together
   constexpr int kU = 4;
   for (int base = 0; base < nloc; base += kRThreads * kU) {
@@ -357,21 +357,22 @@ cudaError_t launch_cluster(Kernel kernel, int grid, int threads, size_t smem, in
   return cudaLaunchKernelEx(&cfg, kernel, args...);
 }
 
+// Attributes of a cluster kernel, set once per CUDA context.
 template <class Kernel>
-cudaError_t configure(Kernel kernel, size_t smem, bool& done) {
-  if (done) return cudaSuccess;
-  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-  if (e == cudaSuccess) e = cudaFuncSetAttribute(kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-  if (e == cudaSuccess) e = cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
-  if (e == cudaSuccess) done = true;
-  return e;
+cudaError_t configure(Kernel kernel, size_t smem, ContextMemo& memo) {
+  return memo.once([&] {
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+    return e;
+  });
 }
 
 }  // namespace
 
 cudaError_t launch_pool_select(const csa2_cache& cache, const float* blockmax, int pool_blocks, int32_t* pool,
                                int cluster, cudaStream_t stream) {
-  static bool done = false;
+  static ContextMemo done;
   const size_t smem = sizeof(PoolSmem);
   cudaError_t e = configure(pool_select_kernel, smem, done);
   if (e != cudaSuccess) return e;
@@ -384,7 +385,7 @@ size_t reindex_smem_bytes(int max_blocks) { return ReindexLayout::make(max_block
 cudaError_t launch_reindex(const csa2_cache& cache, const int32_t* pool, int pool_blocks, const float* q,
                            const float* w, const float* full_scores, int k, int32_t* topk,
                            const CUtensorMap& blk_map, int max_blocks, uint64_t wait_ns, cudaStream_t stream) {
-  static bool done = false;
+  static ContextMemo done;
   // 16 CTAs per request over a pool (a few tiles each, several CTAs per SM),
   // 8 over a whole context of up to 65,536 positions
   const int cluster = pool != nullptr ? kReindexPoolCluster : 8;

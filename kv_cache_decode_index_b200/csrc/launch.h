@@ -8,9 +8,51 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <mutex>
+
 #include "../../include/csa2.h"
 
 namespace csa2 {
+
+// Unique id of the calling thread's current CUDA context (the current
+// device's primary context is made current first when none is).
+cudaError_t current_context_id(unsigned long long* id);
+
+// Set-up that belongs to one CUDA context (kernel attributes, the address of a
+// __device__ array), run once in each context the library is used in.
+class ContextMemo {
+ public:
+  // *value = the value stored for the current context; make(value) computes
+  // and stores it the first time.
+  template <class Make>
+  cudaError_t get(void** value, Make make) {
+    unsigned long long id = 0;
+    bool found = false;
+    cudaError_t e = lookup(&id, &found, value);
+    if (e != cudaSuccess || found) return e;
+    e = make(value);
+    if (e == cudaSuccess) store(id, *value);
+    return e;
+  }
+  // run() once per context (set-up without a value).
+  template <class Run>
+  cudaError_t once(Run run) {
+    void* v = nullptr;
+    return get(&v, [&](void** out) {
+      *out = nullptr;
+      return run();
+    });
+  }
+
+ private:
+  cudaError_t lookup(unsigned long long* id, bool* found, void** value);
+  void store(unsigned long long id, void* value);
+  static constexpr int kSlots = 64;
+  std::mutex mu_;
+  unsigned long long ids_[kSlots] = {};
+  void* vals_[kSlots] = {};
+  int n_ = 0, next_ = 0;
+};
 
 cudaError_t launch_append(const csa2_cache& cache, int n_rows, const float* kv_new, const float* ik_new,
                           const int32_t* req, const int32_t* pos, cudaStream_t stream);

@@ -433,6 +433,58 @@ def test_device_bounds_are_reported_not_trapped(csa2):
     assert csa2.get_error(cache)[0] == csa2.OK
 
 
+@pytest.mark.parametrize("bad_len", [4096 + 1, -5])
+def test_corrupt_length_is_reported_and_the_request_skipped(csa2, bad_len):
+    """A ctx_len outside [0, capacity] must not truncate the request silently:
+    every kernel that reads it records CSA2_ERR_DEVICE_BOUNDS (index = the
+    length) and treats the request as empty, while the other requests of the
+    call are computed normally."""
+    wl = W.scaled(W.WORKLOADS["full_4k_b1"], page_size=1024, batch=2)
+    cache = U.build_cache(wl, csa2, lengths=[4096, 4096])
+    dev = cache.device
+    q, w = W.index_query(wl, 0)
+    tq, tw = torch.from_numpy(q).to(dev), torch.from_numpy(w).to(dev)
+    good_bm = csa2.index_full(cache, tq, tw).clone()
+    good_pool = csa2.pool_select(cache, good_bm, 64).clone()
+    assert csa2.get_error(cache)[0] == csa2.OK
+    cache.ctx_len[1] = bad_len
+
+    def expect_bounds(kernel_id):
+        st, word = csa2.get_error(cache)
+        assert st == csa2.ERR_DEVICE_BOUNDS and word[1] == kernel_id and word[2] == 1 and word[3] == bad_len, word
+        cache.err_word.zero_()
+
+    bm = torch.full_like(good_bm, -7.0)
+    csa2.index_full(cache, tq, tw, bm)
+    expect_bounds(2)
+    assert torch.equal(bm[0], good_bm[0]) and bool((bm[1] == -7.0).all())   # request 1 not scanned
+    pool = csa2.pool_select(cache, good_bm, 64)
+    expect_bounds(3)
+    assert torch.equal(pool[0], good_pool[0]) and bool((pool[1] == -1).all())
+    topk = csa2.reindex(cache, csa2.REINDEX, 512, good_pool, tq, tw)
+    expect_bounds(4)
+    assert bool((topk[1] == -1).all()) and bool((topk[0] >= 0).all())
+    qm = W.main_query(wl, 0).to(dev)
+    ids = torch.arange(512, dtype=torch.int32, device=dev).repeat(2, 1)
+    out = csa2.sparse_attn(cache, ids, qm, wl.scale)
+    expect_bounds(5)
+    assert bool((out[1] == 0).all()) and bool((out[0] != 0).any())
+    pos = torch.tensor([8000, 8100], dtype=torch.int32, device=dev)
+    cache.ctx_len[0] = bad_len
+    cache.ctx_len[1] = 4096
+    tp = csa2.prefill_index(cache, 0, pos, tq, tw, k=64)
+    st, word = csa2.get_error(cache)
+    assert st == csa2.ERR_DEVICE_BOUNDS and word[1] == 6 and word[2] == 0 and word[3] == bad_len, word
+    assert bool((tp == -1).all())
+    # an out-of-range request index in the attention's query map
+    cache.ctx_len[0] = 4096
+    cache.err_word.zero_()
+    out = csa2.sparse_attn(cache, ids, qm, wl.scale, q_req=torch.tensor([0, 9], dtype=torch.int32, device=dev))
+    st, word = csa2.get_error(cache)
+    assert st == csa2.ERR_DEVICE_BOUNDS and word[1] == 5 and word[2] == 9 and word[3] == -1, word
+    assert bool((out[1] == 0).all())
+
+
 def test_pipeline_wait_timeout_returns_status(csa2):
     """A zero wait bound makes the tensor-core pipeline give up at once: the
     kernel must record CSA2_ERR_TIMEOUT, drain and return (no hang, no trap)."""
