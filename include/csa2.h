@@ -175,6 +175,20 @@ CSA2_API csa2_status csa2_compress_append(const csa2_cache* cache, int32_t n_ent
                                           const int32_t* pos, void* stream);
 
 /*
+ * Histogram of the block maxima passed from csa2_index_full to
+ * csa2_pool_select: uint32 [batch][CSA2_POOL_HIST_BINS], one count per
+ * visible block in the bin of its score's leading 14 order-key bits (the fp32
+ * bit pattern with the sign bit flipped, or all bits flipped when negative).
+ * The scan adds to it, so it must hold zeros when the scan starts;
+ * csa2_pool_select reads it and zeroes it again.  Zero it once (for instance
+ * cudaMemsetAsync) before its first use.  It only saves time: a histogram
+ * that does not hold exactly one count per block (not zeroed, shared by two
+ * scans, a scan that gave up) is detected and ignored by csa2_pool_select,
+ * which then selects without it, exactly, and still zeroes it.
+ */
+#define CSA2_POOL_HIST_BINS 16384
+
+/*
  * csa2_index_full -- Full-mode indexer scan of every visible position of every
  * request (Hierarchical Sparse Indexer, first stage).
  *   q        float [batch][32][128]  indexer query (quantised inside, FP8 rule)
@@ -182,23 +196,29 @@ CSA2_API csa2_status csa2_compress_append(const csa2_cache* cache, int32_t n_ent
  *   blockmax float [batch][capacity/8]  out: m_j = max score of block j over
  *            positions < ctx_len; entries past ceil(ctx_len/8) are untouched
  *   scores   float [batch][capacity] or NULL  out: per-position scores s_t
+ *   hist     uint32 [batch][CSA2_POOL_HIST_BINS] or NULL (16-byte aligned):
+ *            the block maxima's histogram for csa2_pool_select (see above)
  * Runs on tcgen05 FP8 tensor cores (scores are fp32; the float64 reference
  * differs by fp32 accumulation rounding only).
  */
 CSA2_API csa2_status csa2_index_full(const csa2_cache* cache, const float* q, const float* w,
-                            float* blockmax, float* scores, void* stream);
+                            float* blockmax, float* scores, uint32_t* hist, void* stream);
 
 /*
  * csa2_pool_select -- the hierarchical pool: the pool_blocks blocks with the
  * largest block max (ties -> lower block id), sorted ascending, -1 padded.
  * With ceil(ctx_len/8) <= pool_blocks the pool is every block.
  *   blockmax float [batch][capacity/8]   (from csa2_index_full)
+ *   hist     uint32 [batch][CSA2_POOL_HIST_BINS] from the same scan, or NULL:
+ *            with it the selection starts from the bin that holds the
+ *            threshold instead of radix passes over every block; it is left
+ *            zeroed.  The result is the same with or without it.
  *   pool     int32 [batch][pool_blocks]  out
  * pool_blocks in [1, 4096] (the pages use 2048); ceil(capacity/8) must not
  * exceed 16 * 16384 blocks (2,097,152 positions per request).
  */
-CSA2_API csa2_status csa2_pool_select(const csa2_cache* cache, const float* blockmax, int32_t pool_blocks,
-                             int32_t* pool, void* stream);
+CSA2_API csa2_status csa2_pool_select(const csa2_cache* cache, const float* blockmax, uint32_t* hist,
+                             int32_t pool_blocks, int32_t* pool, void* stream);
 
 /*
  * csa2_reindex -- Top-k of one layer of the group, by mode:
@@ -222,6 +242,42 @@ CSA2_API csa2_status csa2_reindex(const csa2_cache* cache, csa2_mode mode, const
                          int32_t pool_blocks, const float* q, const float* w,
                          const float* full_scores, const int32_t* prev_topk, int32_t k,
                          int32_t* topk, void* stream);
+
+/*
+ * csa2_reindex_layers -- csa2_reindex over a pool for n_layers layers at once:
+ * layer l's Top-k is the k best positions of the pool by the score of
+ * (q[l], w[l]), exactly as csa2_reindex in mode CSA2_REINDEX would return it;
+ * a Full layer passes its own (q, w) and gets the Top-k of its scan's scores
+ * (the arithmetic is bit-identical).  Reuse layers take no part: they alias
+ * the Top-k of the layer they follow.  Every pool block is gathered from the
+ * cache once for all layers, and all layers are scored in one tensor-core
+ * pass; one select launch then serves every (request, layer).
+ *   n_layers     in [1, CSA2_MAX_SCORE_LAYERS]
+ *   pool         int32 [batch][pool_blocks] (from csa2_pool_select)
+ *   q, w         host arrays [n_layers] of device pointers: float
+ *                [batch][32][128] (16-byte aligned) and float [batch][32]
+ *   k            in [1, 4096]
+ *   topk         host array [n_layers] of device pointers, int32 [batch][k]
+ *                out: positions ascending, -1 padded (ties -> lower position)
+ *   workspace    caller-owned device memory of at least
+ *                csa2_reindex_layers_workspace_bytes(batch, n_layers,
+ *                pool_blocks) bytes, 16-byte aligned: the layers' pool scores
+ *                and one histogram of their leading 12 bits per (request,
+ *                layer).  Zero it once before its first use; each call leaves
+ *                the histograms zeroed again.  As with the pool's histogram,
+ *                a histogram that is not zero at the start only costs time
+ *                (it is detected, ignored and zeroed).  Two calls in flight at
+ *                once must not share a workspace.
+ * Launches two kernels.  Device errors as csa2_reindex; on CSA2_ERR_TIMEOUT
+ * the outputs are undefined.
+ */
+#define CSA2_MAX_SCORE_LAYERS 8
+#define CSA2_RESCORE_HIST_BINS 4096
+CSA2_API size_t csa2_reindex_layers_workspace_bytes(int32_t batch, int32_t n_layers, int32_t pool_blocks);
+CSA2_API csa2_status csa2_reindex_layers(const csa2_cache* cache, int32_t n_layers, const int32_t* pool,
+                                         int32_t pool_blocks, const float* const* q, const float* const* w,
+                                         int32_t k, int32_t* const* topk, void* workspace,
+                                         size_t workspace_bytes, void* stream);
 
 /*
  * csa2_sparse_attn -- sparse MQA attention over the gathered Top-k rows:
@@ -304,10 +360,12 @@ CSA2_API csa2_status csa2_prefill_index_static(const csa2_cache* cache, int32_t 
                                                const float* w, int32_t k, int32_t* topk, void* stream);
 
 /*
- * csa2_sparse_attn_layers -- csa2_sparse_attn for n_layers layers that attend
- * over the same Top-k (a Full or Reindex layer and the Reuse layers that take
- * its indices [readance summary, section 4.2: a Reuse layer keeps its own main
- * query]), in one launch.
+ * csa2_sparse_attn_layers -- csa2_sparse_attn for n_layers layers in one
+ * launch, each layer over its own Top-k (a Reuse layer passes the Top-k of the
+ * layer it follows, and keeps its own main query [readance summary, section
+ * 4.2]).
+ *   topk host array [n_layers] of device pointers, each int32 [n_queries][k]
+ *        (layers may share one)
  *   q    host array [n_layers] of device pointers, each bf16 [n_queries][H][512]
  *   out  host array [n_layers] of device pointers, each bf16 [n_queries][H][512]
  *   workspace  NULL, or caller-owned device memory of at least
@@ -325,7 +383,7 @@ CSA2_API csa2_status csa2_prefill_index_static(const csa2_cache* cache, int32_t 
  */
 #define CSA2_ATTN_MAX_LAYERS 8
 CSA2_API csa2_status csa2_sparse_attn_layers(const csa2_cache* cache, int32_t n_layers, int32_t n_queries,
-                                             const int32_t* q_req, const int32_t* topk, int32_t k,
+                                             const int32_t* q_req, const int32_t* const* topk, int32_t k,
                                              const uint16_t* const* q, int32_t H, float scale,
                                              uint16_t* const* out, void* workspace, size_t workspace_bytes,
                                              void* stream);

@@ -24,6 +24,7 @@ MODE = {"F": FULL, "Ri": REINDEX, "Ru": REUSE}
 OK, ERR_ARG, ERR_SHAPE, ERR_CUDA, ERR_DEVICE_BOUNDS, ERR_TIMEOUT, ERR_UNSUPPORTED = range(7)
 BLOCK, INDEX_HEADS, INDEX_DIM, KV_DIM, KV_CODE_BYTES, KV_SCALE_BYTES = 8, 32, 128, 512, 256, 32
 PREFILL_MAX_K, PREFILL_CANDIDATES, PREFILL_STATIC_MAX_QUERIES = 1024, 4096, 256
+POOL_HIST_BINS, RESCORE_HIST_BINS, MAX_SCORE_LAYERS = 16384, 4096, 8
 
 
 class CacheStruct(ctypes.Structure):
@@ -39,9 +40,10 @@ _CP = ctypes.POINTER(CacheStruct)
 _sig = {
     "csa2_append_kv": [_CP, _I, _P, _P, _P, _P, _P],
     "csa2_compress_append": [_CP, _I, _I, _P, _P, _P, _P, _P],
-    "csa2_index_full": [_CP, _P, _P, _P, _P, _P],
-    "csa2_pool_select": [_CP, _P, _I, _P, _P],
+    "csa2_index_full": [_CP, _P, _P, _P, _P, _P, _P],
+    "csa2_pool_select": [_CP, _P, _P, _I, _P, _P],
     "csa2_reindex": [_CP, _I, _P, _I, _P, _P, _P, _P, _I, _P, _P],
+    "csa2_reindex_layers": [_CP, _I, _P, _I, _P, _P, _I, _P, _P, ctypes.c_size_t, _P],
     "csa2_sparse_attn": [_CP, _I, _P, _P, _I, _P, _I, ctypes.c_float, _P, _P],
     "csa2_sparse_attn_layers": [_CP, _I, _I, _P, _P, _I, _P, _I, ctypes.c_float, _P, _P, ctypes.c_size_t, _P],
     "csa2_swa_append": [_CP, _I, _P, _P, _I, _P, _P, _P, _P],
@@ -61,6 +63,8 @@ _lib.csa2_prefill_workspace_bytes.argtypes = [_I]
 _lib.csa2_prefill_workspace_bytes.restype = ctypes.c_size_t
 _lib.csa2_attn_workspace_bytes.argtypes = [_I, _I, _I]
 _lib.csa2_attn_workspace_bytes.restype = ctypes.c_size_t
+_lib.csa2_reindex_layers_workspace_bytes.argtypes = [_I, _I, _I]
+_lib.csa2_reindex_layers_workspace_bytes.restype = ctypes.c_size_t
 _lib.csa2_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
 _lib.csa2_set_wait_limit_ns.restype = None
 
@@ -161,8 +165,15 @@ def compress_append(cache: Cache, kv_tok, ik_tok, pos, m: int = 2, req=None):
                                      _ptr(pos), _stream(cache.device)), "csa2_compress_append")
 
 
-def index_full(cache: Cache, q, w, blockmax=None, scores=None):
-    """Full scan: returns blockmax float32 [batch, capacity/8] (and fills scores if given)."""
+def pool_hist(cache: Cache):
+    """A zeroed block-max histogram buffer (uint32 bit patterns in an int32
+    tensor [batch, POOL_HIST_BINS]) for index_full / pool_select."""
+    return torch.zeros(cache.batch, POOL_HIST_BINS, dtype=torch.int32, device=cache.device)
+
+
+def index_full(cache: Cache, q, w, blockmax=None, scores=None, hist=None):
+    """Full scan: returns blockmax float32 [batch, capacity/8] (and fills scores
+    if given; adds the block maxima's histogram into hist if given)."""
     B = cache.batch
     _need(q, torch.float32, (B, INDEX_HEADS, INDEX_DIM), "q")
     _need(w, torch.float32, (B, INDEX_HEADS), "w")
@@ -171,20 +182,59 @@ def index_full(cache: Cache, q, w, blockmax=None, scores=None):
     _need(blockmax, torch.float32, (B, cache.capacity // BLOCK), "blockmax")
     if scores is not None:
         _need(scores, torch.float32, (B, cache.capacity), "scores")
+    if hist is not None:
+        _need(hist, torch.int32, (B, POOL_HIST_BINS), "hist")
     _check(_lib.csa2_index_full(ctypes.byref(cache.struct), _ptr(q), _ptr(w), _ptr(blockmax), _ptr(scores),
-                                _stream(cache.device)), "csa2_index_full")
+                                _ptr(hist), _stream(cache.device)), "csa2_index_full")
     return blockmax
 
 
-def pool_select(cache: Cache, blockmax, pool_blocks: int = 2048, pool=None):
+def pool_select(cache: Cache, blockmax, pool_blocks: int = 2048, pool=None, hist=None):
+    """The pool (int32 [batch, pool_blocks]); hist: the scan's block-max
+    histogram (read, then zeroed), or None."""
     B = cache.batch
     _need(blockmax, torch.float32, (B, cache.capacity // BLOCK), "blockmax")
     if pool is None:
         pool = torch.empty(B, pool_blocks, dtype=torch.int32, device=cache.device)
     _need(pool, torch.int32, (B, pool_blocks), "pool")
-    _check(_lib.csa2_pool_select(ctypes.byref(cache.struct), _ptr(blockmax), pool_blocks, _ptr(pool),
+    if hist is not None:
+        _need(hist, torch.int32, (B, POOL_HIST_BINS), "hist")
+    _check(_lib.csa2_pool_select(ctypes.byref(cache.struct), _ptr(blockmax), _ptr(hist), pool_blocks, _ptr(pool),
                                  _stream(cache.device)), "csa2_pool_select")
     return pool
+
+
+def reindex_layers_workspace_bytes(batch: int, n_layers: int, pool_blocks: int) -> int:
+    return int(_lib.csa2_reindex_layers_workspace_bytes(int(batch), int(n_layers), int(pool_blocks)))
+
+
+def reindex_layers(cache: Cache, pool, q_layers, w_layers, k: int = 512, topk_layers=None, workspace=None):
+    """Top-k over the pool of several Full / Reindex layers in one pass
+    (csa2_reindex_layers); returns the list of int32 [batch, k] Top-k.
+    workspace: a zeroed uint8 device tensor of reindex_layers_workspace_bytes
+    bytes, kept between calls (allocated and zeroed here when None)."""
+    B, P = pool.shape
+    L = len(q_layers)
+    _need(pool, torch.int32, (B, P), "pool")
+    for i, (q, w) in enumerate(zip(q_layers, w_layers)):
+        _need(q, torch.float32, (B, INDEX_HEADS, INDEX_DIM), f"q_layers[{i}]")
+        _need(w, torch.float32, (B, INDEX_HEADS), f"w_layers[{i}]")
+    if topk_layers is None:
+        topk_layers = [torch.empty(B, k, dtype=torch.int32, device=cache.device) for _ in range(L)]
+    for i, t in enumerate(topk_layers):
+        _need(t, torch.int32, (B, k), f"topk_layers[{i}]")
+    need = reindex_layers_workspace_bytes(B, L, P)
+    if workspace is None:
+        workspace = torch.zeros(need, dtype=torch.uint8, device=cache.device)
+    if workspace.dtype != torch.uint8 or not workspace.is_contiguous() or workspace.device.type != "cuda":
+        raise ValueError("workspace: expected a contiguous cuda uint8 tensor")
+    qa = (ctypes.c_void_p * L)(*[q.data_ptr() for q in q_layers])
+    wa = (ctypes.c_void_p * L)(*[w.data_ptr() for w in w_layers])
+    ta = (ctypes.c_void_p * L)(*[t.data_ptr() for t in topk_layers])
+    _check(_lib.csa2_reindex_layers(ctypes.byref(cache.struct), L, _ptr(pool), P, qa, wa, int(k), ta,
+                                    _ptr(workspace), workspace.numel(), _stream(cache.device)),
+           "csa2_reindex_layers")
+    return topk_layers
 
 
 def reindex(cache: Cache, mode: int, k: int = 512, pool=None, q=None, w=None, full_scores=None,
@@ -275,14 +325,19 @@ def attn_workspace_bytes(n_layers: int, n_queries: int, heads: int) -> int:
 
 def sparse_attn_layers(cache: Cache, topk, q_layers, scale: float | None = None, out_layers=None, q_req=None,
                        workspace=None):
-    """Sparse attention of several layers over the same Top-k in one launch;
+    """Sparse attention of several layers in one launch; topk: one int32
+    [n, k] tensor shared by every layer, or a list with one per layer;
     q_layers: list of bf16 [n, H, 512] -> list of outputs of the same shape.
     workspace: optional uint8 device tensor of attn_workspace_bytes(...) bytes
     (the key splits then merge through it instead of shared memory)."""
-    n, k = topk.shape
     L = len(q_layers)
+    topk_layers = list(topk) if isinstance(topk, (list, tuple)) else [topk] * L
+    n, k = topk_layers[0].shape
     H = q_layers[0].shape[1]
-    _need(topk, torch.int32, (n, k), "topk")
+    if len(topk_layers) != L:
+        raise ValueError(f"{len(topk_layers)} Top-k tensors for {L} layers")
+    for i, t in enumerate(topk_layers):
+        _need(t, torch.int32, (n, k), f"topk[{i}]")
     for i, q in enumerate(q_layers):
         _need(q, torch.bfloat16, (n, H, KV_DIM), f"q_layers[{i}]")
     if q_req is not None:
@@ -294,8 +349,9 @@ def sparse_attn_layers(cache: Cache, topk, q_layers, scale: float | None = None,
     scale = 1.0 / math.sqrt(KV_DIM) if scale is None else scale
     qa = (ctypes.c_void_p * L)(*[q.data_ptr() for q in q_layers])
     oa = (ctypes.c_void_p * L)(*[o.data_ptr() for o in out_layers])
+    ta = (ctypes.c_void_p * L)(*[t.data_ptr() for t in topk_layers])
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    _check(_lib.csa2_sparse_attn_layers(ctypes.byref(cache.struct), L, n, _ptr(q_req), _ptr(topk), k, qa, H,
+    _check(_lib.csa2_sparse_attn_layers(ctypes.byref(cache.struct), L, n, _ptr(q_req), ta, k, qa, H,
                                         ctypes.c_float(scale), oa, _ptr(workspace), ws_bytes,
                                         _stream(cache.device)), "csa2_sparse_attn_layers")
     return out_layers
@@ -375,12 +431,19 @@ class DecodeGroup:
     scans the context and (with pool_blocks) builds the pool; Reindex layers
     re-score the pool with their own query; Reuse layers take the previous
     layer's Top-k.  Every layer attends with its own main query.
-    With `concurrent`, layers that only depend on the pool run on side streams
-    (the calls are stream-ordered, so the step can be captured in a CUDA graph).
+
+    With a pool the step is five kernels on the calling stream, each linked
+    to the one before by programmatic dependent launch (so it can be captured
+    in a CUDA graph): the scan (which also fills the block maxima's
+    histogram), the pool selection (which starts from that histogram), the
+    Top-k of every Full / Reindex layer (csa2_reindex_layers: one scoring and
+    one select launch for all of them), and one attention launch for all
+    layers.  Without a pool each Full / Reindex layer takes its flat Top-k
+    with csa2_reindex, then the same single attention launch follows.
     """
 
     def __init__(self, cache: Cache, modes, heads: int, k: int = 512, pool_blocks: int | None = 2048,
-                 scale: float | None = None, concurrent: bool = True):
+                 scale: float | None = None):
         if modes[0] != "F":
             raise ValueError("a layer group starts with a Full layer")
         self.cache, self.modes, self.heads, self.k = cache, tuple(modes), heads, k
@@ -389,6 +452,7 @@ class DecodeGroup:
         dev, B = cache.device, cache.batch
         self.blockmax = torch.empty(B, cache.capacity // BLOCK, dtype=torch.float32, device=dev)
         self.pool = torch.empty(B, pool_blocks, dtype=torch.int32, device=dev) if pool_blocks else None
+        self.hist = pool_hist(cache) if pool_blocks else None
         # Reuse layers alias the Top-k buffer of the layer they reuse
         self.topk, src = [], None
         for m in self.modes:
@@ -397,31 +461,30 @@ class DecodeGroup:
             else:
                 src = torch.empty(B, k, dtype=torch.int32, device=dev)
                 self.topk.append(src)
-        self.concurrent = concurrent
-        # attention launches: each Full/Reindex layer with the Reuse layers that follow it
         self.sources = layer_sources(self.modes)
-        # the last source's chain (pool -> Top-k -> attention) runs on the
-        # calling stream, linked by programmatic dependent launch; the other
-        # sources run on streams of their own, after the pool
-        self.streams = [torch.cuda.Stream(dev) for _ in self.sources[:-1]] if concurrent else []
-        # one attention exchange workspace per source (the sources may run at once)
-        self.attn_ws = [torch.empty(attn_workspace_bytes(len(layers), B, heads), dtype=torch.uint8, device=dev)
-                        for layers in self.sources]
-        self.launches_per_step = 1 + (1 if pool_blocks else 0) + 2 * len(self.sources)
+        self.index_layers = [layers[0] for layers in self.sources]
+        if pool_blocks:
+            self.rs_ws = torch.zeros(reindex_layers_workspace_bytes(B, len(self.index_layers), pool_blocks),
+                                     dtype=torch.uint8, device=dev)
+        self.attn_ws = torch.empty(attn_workspace_bytes(len(self.modes), B, heads), dtype=torch.uint8, device=dev)
+        # kernels per step: scan, pool, score + select, attention (with a
+        # pool); scan, one Top-k per index layer, attention (without)
+        self.launches_per_step = 5 if pool_blocks else 2 + len(self.index_layers)
 
     def step(self, q_idx, w_idx, q_main, out, timing=None):
         """q_idx / w_idx: per layer ([B,32,128] / [B,32], None for Reuse);
         q_main / out: per layer bf16 [B, H, 512].  timing: optional dict
-        name -> (start, end) CUDA events, recorded on the launching stream
-        around the launch of that name ("scan", "pool", "topk<l>", and
-        "attn<l>" for source layer l with its Reuse layers)."""
+        name -> (start, end) CUDA events, recorded on the calling stream
+        around the launches of that name ("scan", "pool", "topk", "attn"; an
+        event between two launches cuts their programmatic link, so time a
+        separate graph with it)."""
         c = self.cache
 
         def timed(name, fn):
             ev = None if timing is None else timing.get(name)
             if ev is not None:
                 ev[0].record()
-            torch.cuda.nvtx.range_push(f"csa2 {name}")   # profiler range around the launch
+            torch.cuda.nvtx.range_push(f"csa2 {name}")   # profiler range around the launches
             try:
                 r = fn()
             finally:
@@ -430,42 +493,23 @@ class DecodeGroup:
                 ev[1].record()
             return r
 
-        timed("scan", lambda: index_full(c, q_idx[0], w_idx[0], self.blockmax))
+        timed("scan", lambda: index_full(c, q_idx[0], w_idx[0], self.blockmax, hist=self.hist))
         if self.pool is not None:
-            timed("pool", lambda: pool_select(c, self.blockmax, self.pool_blocks, self.pool))
-        main = torch.cuda.current_stream(c.device)
-        ev_ready = None
-        if self.concurrent and len(self.sources) > 1:
-            ev_ready = torch.cuda.Event()
-            ev_ready.record(main)
-        for si in range(len(self.sources)):   # side streams first, the calling stream's chain last
-            layers = self.sources[si]
-            src = layers[0]
-            s = main if (si == len(self.sources) - 1 or not self.concurrent) else self.streams[si]
-            with torch.cuda.stream(s):
-                if s is not main:
-                    s.wait_event(ev_ready)
-                mode = FULL if self.modes[src] == "F" else REINDEX
-                timed(f"topk{src}", lambda: reindex(c, mode, self.k, self.pool, q_idx[src], w_idx[src],
-                                                    topk=self.topk[src]))
-                timed(f"attn{src}", lambda: sparse_attn_layers(c, self.topk[src], [q_main[l] for l in layers],
-                                                               self.scale, [out[l] for l in layers],
-                                                               workspace=self.attn_ws[si]))
-        if self.concurrent:
-            joins = []
-            for s in self.streams:
-                e = torch.cuda.Event()
-                e.record(s)
-                joins.append(e)
-            for e in joins:
-                main.wait_event(e)
+            timed("pool", lambda: pool_select(c, self.blockmax, self.pool_blocks, self.pool, hist=self.hist))
+            L = self.index_layers
+            timed("topk", lambda: reindex_layers(c, self.pool, [q_idx[l] for l in L], [w_idx[l] for l in L],
+                                                 self.k, [self.topk[l] for l in L], self.rs_ws))
+        else:
+            def flat():
+                for l in self.index_layers:
+                    mode = FULL if self.modes[l] == "F" else REINDEX
+                    reindex(c, mode, self.k, None, q_idx[l], w_idx[l], topk=self.topk[l])
+            timed("topk", flat)
+        timed("attn", lambda: sparse_attn_layers(c, self.topk, q_main, self.scale, out, workspace=self.attn_ws))
         return out
 
     def launch_names(self):
-        names = ["scan"] + (["pool"] if self.pool is not None else [])
-        for layers in self.sources:
-            names += [f"topk{layers[0]}", f"attn{layers[0]}"]
-        return names
+        return ["scan"] + (["pool"] if self.pool is not None else []) + ["topk", "attn"]
 
 
 class PrefillGroup:

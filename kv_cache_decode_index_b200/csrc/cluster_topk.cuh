@@ -7,7 +7,9 @@
 //
 // First the cluster-wide count, minimum and maximum of the valid keys: their
 // common leading bits need no pass (scores of one request share their sign and
-// most exponent bits), and K >= count selects everything.  Then radix select,
+// most exponent bits), and K >= count selects everything.  A caller that knows
+// the threshold's leading bits already (from a histogram of the keys) passes
+// them as a SelectStart instead, and that phase is skipped.  Then radix select,
 // 8 bits per pass from the first differing bit: every CTA builds the
 // histogram of its keys that match the prefix decided so far, the CTAs read
 // each other's histograms through distributed shared memory (one cluster
@@ -42,6 +44,18 @@ struct SelectSmem {
   int total;                 // valid candidates in the cluster
 };
 
+// Head start of a select: the threshold's leading bits (prefix under mask),
+// found elsewhere, and the number of keys still needed among the keys that
+// match them.  hi is the top bit of the next radix digit; done = 1 when the
+// selection is decided already (every matching key is needed, or no bit is
+// left).  All keys not matching the prefix are above it or below it.
+struct SelectStart {
+  uint32_t prefix, mask;
+  int need;
+  int hi;
+  int done;
+};
+
 // Exclusive block-wide prefix sum of one int per thread (THREADS multiple of
 // 32, <= 1024).  Returns the thread's exclusive prefix; *sum gets the total.
 template <int THREADS>
@@ -73,9 +87,11 @@ __device__ __forceinline__ int block_exclusive_sum(int v, int* warp_tmp, int* su
 // Select the K best of the cluster's candidates.  emit(i, r) is called for the
 // local candidate i that has output rank r (0 <= r < min(K, total)); pad(r) for
 // r in [total, K) by the cluster's rank-0 CTA.  Must be called by all THREADS
-// threads of every CTA of the cluster (it contains cluster barriers).
+// threads of every CTA of the cluster (it contains cluster barriers).  start:
+// an optional head start, the same in every CTA of the cluster.
 template <int THREADS, class Emit, class Pad>
-__device__ void cluster_topk(const uint32_t* keys, int n_local, int K, SelectSmem& S, Emit emit, Pad pad) {
+__device__ void cluster_topk(const uint32_t* keys, int n_local, int K, SelectSmem& S, Emit emit, Pad pad,
+                             const SelectStart* start = nullptr) {
   constexpr int kWarps = THREADS / 32;
   cg::cluster_group cluster = cg::this_cluster();
   const int C = static_cast<int>(cluster.num_blocks());
@@ -83,8 +99,18 @@ __device__ void cluster_topk(const uint32_t* keys, int n_local, int K, SelectSme
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int rounds = (n_local + THREADS - 1) / THREADS;
 
-  // ---- count, min and max of the valid keys ----
-  {
+  if (start != nullptr) {
+    for (int i = tid; i < 256; i += THREADS) S.hist[0][i] = 0;
+    if (tid == 0) {
+      S.prefix = start->prefix;
+      S.mask = start->mask;
+      S.need = start->need;
+      S.hi = start->hi;
+      S.done = start->done;
+    }
+    __syncthreads();
+  } else {
+    // ---- count, min and max of the valid keys ----
     uint32_t cnt = 0, kmin = 0xFFFFFFFFu, kmax = 0u;
     for (int r = 0; r < rounds; ++r) {
       const int i = r * THREADS + tid;

@@ -125,7 +125,7 @@ csa2_status check_cache(const csa2_cache* c, bool need_kv, bool need_ik) {
   } while (0)
 
 csa2_status sparse_attn_impl(const csa2_cache* cache, int32_t n_layers, int32_t n_queries, const int32_t* q_req,
-                             const int32_t* topk, int32_t k, const uint16_t* const* q, int32_t H, float scale,
+                             const int32_t* const* topk, int32_t k, const uint16_t* const* q, int32_t H, float scale,
                              uint16_t* const* out, void* stream, void* workspace = nullptr,
                              size_t workspace_bytes = 0) {
   CSA2_TRY(check_cache(cache, true, false));
@@ -141,8 +141,8 @@ csa2_status sparse_attn_impl(const csa2_cache* cache, int32_t n_layers, int32_t 
     return fail(CSA2_ERR_SHAPE, "n_layers * n_queries too large");
   if (topk == nullptr || q == nullptr || out == nullptr) return fail(CSA2_ERR_ARG, "topk, q and out must be set");
   for (int l = 0; l < n_layers; ++l)
-    if (q[l] == nullptr || out[l] == nullptr || !aligned(q[l], 16) || !aligned(out[l], 16))
-      return fail(CSA2_ERR_ARG, "layer %d: q and out (16-byte aligned) must be set", l);
+    if (topk[l] == nullptr || q[l] == nullptr || out[l] == nullptr || !aligned(q[l], 16) || !aligned(out[l], 16))
+      return fail(CSA2_ERR_ARG, "layer %d: topk, q and out (16-byte aligned) must be set", l);
   if (workspace != nullptr) {
     if (!aligned(workspace, 16)) return fail(CSA2_ERR_ARG, "workspace must be 16-byte aligned");
     const size_t need = csa2::attn_workspace_bytes(n_layers, n_queries, H);
@@ -194,23 +194,25 @@ csa2_status csa2_compress_append(const csa2_cache* cache, int32_t n_entries, int
 }
 
 csa2_status csa2_index_full(const csa2_cache* cache, const float* q, const float* w, float* blockmax, float* scores,
-                            void* stream) {
+                            uint32_t* hist, void* stream) {
   CSA2_TRY(check_cache(cache, false, true));
   if (q == nullptr || w == nullptr || blockmax == nullptr || !aligned(q, 16))
     return fail(CSA2_ERR_ARG, "q (16-byte aligned), w and blockmax must be set");
+  if (hist != nullptr && !aligned(hist, 16)) return fail(CSA2_ERR_ARG, "hist must be 16-byte aligned");
   DeviceInfo d;
   CSA2_TRY(device_info(&d));
   CUtensorMap map;
   CSA2_TRY(encode_ik_map(cache, csa2::kTile, &map));
-  const cudaError_t e = csa2::launch_index_full(*cache, q, w, blockmax, scores, map, d.sms, g_wait_limit_ns,
+  const cudaError_t e = csa2::launch_index_full(*cache, q, w, blockmax, scores, hist, map, d.sms, g_wait_limit_ns,
                                                 static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? CSA2_OK : cuda_fail(e, "index_full launch");
 }
 
-csa2_status csa2_pool_select(const csa2_cache* cache, const float* blockmax, int32_t pool_blocks, int32_t* pool,
-                             void* stream) {
+csa2_status csa2_pool_select(const csa2_cache* cache, const float* blockmax, uint32_t* hist, int32_t pool_blocks,
+                             int32_t* pool, void* stream) {
   CSA2_TRY(check_cache(cache, false, false));
   if (blockmax == nullptr || pool == nullptr) return fail(CSA2_ERR_ARG, "blockmax and pool must be set");
+  if (hist != nullptr && !aligned(hist, 16)) return fail(CSA2_ERR_ARG, "hist must be 16-byte aligned");
   if (pool_blocks < 1 || pool_blocks > kMaxPool)
     return fail(CSA2_ERR_SHAPE, "pool_blocks %d outside [1, %d]", pool_blocks, kMaxPool);
   const long long nblk = (capacity_of(cache) + csa2::kBlock - 1) / csa2::kBlock;
@@ -219,8 +221,13 @@ csa2_status csa2_pool_select(const csa2_cache* cache, const float* blockmax, int
                 capacity_of(cache), kMaxPoolSelectBlocks * csa2::kBlock);
   DeviceInfo d;
   CSA2_TRY(device_info(&d));
-  const int cluster = nblk <= 4LL * 16384 ? 8 : 16;   // 16 CTAs above 524,288 positions: half the keys per CTA
-  const cudaError_t e = csa2::launch_pool_select(*cache, blockmax, pool_blocks, pool, cluster,
+  // Without a histogram the radix passes scan every key: 16 CTAs above
+  // 524,288 positions halve the keys per CTA.  With one, the passes only
+  // touch the keys of the threshold's bin, and 8 CTAs (up to 16,384 keys
+  // each) halve the cost of each pass's exchange instead.
+  const long long per_cta = 16384;
+  const int cluster = (nblk <= 4LL * per_cta || (hist != nullptr && nblk <= 8LL * per_cta)) ? 8 : 16;
+  const cudaError_t e = csa2::launch_pool_select(*cache, blockmax, hist, pool_blocks, pool, cluster,
                                                  static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? CSA2_OK : cuda_fail(e, "pool_select launch");
 }
@@ -266,13 +273,45 @@ csa2_status csa2_reindex(const csa2_cache* cache, csa2_mode mode, const int32_t*
   return e == cudaSuccess ? CSA2_OK : cuda_fail(e, "reindex launch");
 }
 
+size_t csa2_reindex_layers_workspace_bytes(int32_t batch, int32_t n_layers, int32_t pool_blocks) {
+  return csa2::rescore_workspace_bytes(batch, n_layers, pool_blocks);
+}
+
+csa2_status csa2_reindex_layers(const csa2_cache* cache, int32_t n_layers, const int32_t* pool, int32_t pool_blocks,
+                                const float* const* q, const float* const* w, int32_t k, int32_t* const* topk,
+                                void* workspace, size_t workspace_bytes, void* stream) {
+  CSA2_TRY(check_cache(cache, false, true));
+  if (n_layers < 1 || n_layers > CSA2_MAX_SCORE_LAYERS)
+    return fail(CSA2_ERR_SHAPE, "n_layers %d outside [1, %d]", n_layers, CSA2_MAX_SCORE_LAYERS);
+  if (pool_blocks < 1 || pool_blocks > kMaxPool)
+    return fail(CSA2_ERR_SHAPE, "pool_blocks %d outside [1, %d]", pool_blocks, kMaxPool);
+  if (k < 1 || k > kMaxK) return fail(CSA2_ERR_SHAPE, "k %d outside [1, %d]", k, kMaxK);
+  if (pool == nullptr || q == nullptr || w == nullptr || topk == nullptr)
+    return fail(CSA2_ERR_ARG, "pool, q, w and topk must be set");
+  for (int l = 0; l < n_layers; ++l)
+    if (q[l] == nullptr || w[l] == nullptr || topk[l] == nullptr || !aligned(q[l], 16))
+      return fail(CSA2_ERR_ARG, "layer %d: q (16-byte aligned), w and topk must be set", l);
+  if (workspace == nullptr || !aligned(workspace, 16))
+    return fail(CSA2_ERR_ARG, "workspace must be set and 16-byte aligned");
+  const size_t need = csa2::rescore_workspace_bytes(cache->batch, n_layers, pool_blocks);
+  if (workspace_bytes < need)
+    return fail(CSA2_ERR_SHAPE, "workspace_bytes %zu < %zu (csa2_reindex_layers_workspace_bytes)", workspace_bytes,
+                need);
+  DeviceInfo d;
+  CSA2_TRY(device_info(&d));
+  CUtensorMap map;
+  CSA2_TRY(encode_ik_map(cache, csa2::kBlock, &map));
+  const cudaError_t e = csa2::launch_rescore_layers(*cache, n_layers, pool, pool_blocks, q, w, k, topk, workspace,
+                                                    map, d.sms, g_wait_limit_ns, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? CSA2_OK : cuda_fail(e, "reindex_layers launch");
+}
 
 csa2_status csa2_sparse_attn(const csa2_cache* cache, int32_t n_queries, const int32_t* q_req, const int32_t* topk,
                              int32_t k, const uint16_t* q, int32_t H, float scale, uint16_t* out, void* stream) {
   const uint16_t* qs[1] = {q};
   uint16_t* os[1] = {out};
-  if (q == nullptr || out == nullptr) return fail(CSA2_ERR_ARG, "topk, q and out (16-byte aligned) must be set");
-  return sparse_attn_impl(cache, 1, n_queries, q_req, topk, k, qs, H, scale, os, stream);
+  const int32_t* ts[1] = {topk};
+  return sparse_attn_impl(cache, 1, n_queries, q_req, ts, k, qs, H, scale, os, stream);
 }
 
 csa2_status csa2_swa_append(const csa2_cache* cache, int32_t window, uint8_t* swa_codes, uint8_t* swa_exp,
@@ -315,14 +354,15 @@ csa2_status csa2_sparse_attn_swa(const csa2_cache* cache, int32_t n_queries, con
   CSA2_TRY(device_info(&d));
   const uint16_t* qs[1] = {q};
   uint16_t* os[1] = {out};
-  const cudaError_t e = csa2::launch_sparse_attn(*cache, 1, n_queries, q_req, topk, k, qs, H, scale, os,
+  const int32_t* ts[1] = {topk};
+  const cudaError_t e = csa2::launch_sparse_attn(*cache, 1, n_queries, q_req, ts, k, qs, H, scale, os,
                                                  static_cast<cudaStream_t>(stream), swa_codes, swa_exp, q_pos,
                                                  window);
   return e == cudaSuccess ? CSA2_OK : cuda_fail(e, "sparse_attn_swa launch");
 }
 
 csa2_status csa2_sparse_attn_layers(const csa2_cache* cache, int32_t n_layers, int32_t n_queries,
-                                    const int32_t* q_req, const int32_t* topk, int32_t k, const uint16_t* const* q,
+                                    const int32_t* q_req, const int32_t* const* topk, int32_t k, const uint16_t* const* q,
                                     int32_t H, float scale, uint16_t* const* out, void* workspace,
                                     size_t workspace_bytes, void* stream) {
   return sparse_attn_impl(cache, n_layers, n_queries, q_req, topk, k, q, H, scale, out, stream, workspace,

@@ -147,9 +147,10 @@ __device__ __forceinline__ void dequant16(uint4 codes, uint32_t s01, uint4 (&out
   for (int c = 0; c < 4; ++c) out[c] = make_uint4(h[4 * c], h[4 * c + 1], h[4 * c + 2], h[4 * c + 3]);
 }
 
-// Query and output of each layer attending over the same Top-k (a Full or
-// Reindex layer and the Reuse layers that take its indices).
+// Top-k, query and output of each layer of one launch (layers may share a
+// Top-k: a Full or Reindex layer and the Reuse layers that take its indices).
 struct AttnLayers {
+  const int32_t* topk[CSA2_ATTN_MAX_LAYERS];
   const __nv_bfloat16* q[CSA2_ATTN_MAX_LAYERS];
   __nv_bfloat16* out[CSA2_ATTN_MAX_LAYERS];
 };
@@ -167,7 +168,7 @@ struct SwaArgs {
 template <int H>
 __global__ void __launch_bounds__(kAThreads, H == 16 ? 2 : 1)
     sparse_attn_kernel(const csa2_cache cache, int n_queries, const int32_t* __restrict__ q_req,
-                       const int32_t* __restrict__ topk, int K, const __grid_constant__ AttnLayers io, float softmax_scale,
+                       int K, const __grid_constant__ AttnLayers io, float softmax_scale,
                        const SwaArgs swa, float* __restrict__ xchg) {
   using L = AttnLayout<H>;
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -238,7 +239,7 @@ __global__ void __launch_bounds__(kAThreads, H == 16 ? 2 : 1)
   if (!b_ok && rank == 0 && tid == 0) report_error(cache.err_word, CSA2_ERR_DEVICE_BOUNDS, kKAttn, b, -1);
   const int n_raw = b_ok ? checked_ctx_len(cache, b, capacity, kKAttn, rank == 0 && tid == 0) : -1;
   const int n = max(0, n_raw);   // n_raw < 0: no entry of this query is used (or checked)
-  const int32_t* idx = topk + static_cast<long long>(qi) * K;
+  const int32_t* idx = io.topk[layer] + static_cast<long long>(qi) * K;
 
   // ---- this CTA's entries: the Top-k entries, then the window's tokens ----
   const int n_win = swa.codes != nullptr ? swa.window : 0;
@@ -627,8 +628,8 @@ __global__ void __launch_bounds__(kAThreads, H == 16 ? 2 : 1)
 }
 
 template <int H>
-cudaError_t launch_h(const csa2_cache& cache, int n_layers, int n_queries, const int32_t* q_req, const int32_t* topk,
-                     int k, const AttnLayers& io, float scale, const SwaArgs& swa, float* xchg, cudaStream_t stream) {
+cudaError_t launch_h(const csa2_cache& cache, int n_layers, int n_queries, const int32_t* q_req, int k,
+                     const AttnLayers& io, float scale, const SwaArgs& swa, float* xchg, cudaStream_t stream) {
   static ContextMemo attrs;
   const size_t smem = AttnLayout<H>::total;
   const cudaError_t e = attrs.once([&] {
@@ -650,7 +651,7 @@ cudaError_t launch_h(const csa2_cache& cache, int n_layers, int n_queries, const
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  return cudaLaunchKernelEx(&cfg, sparse_attn_kernel<H>, cache, n_queries, q_req, topk, k, io, scale, swa, xchg);
+  return cudaLaunchKernelEx(&cfg, sparse_attn_kernel<H>, cache, n_queries, q_req, k, io, scale, swa, xchg);
 }
 
 }  // namespace
@@ -660,20 +661,21 @@ size_t attn_workspace_bytes(long long n_layers, long long n_queries, int H) {
 }
 
 cudaError_t launch_sparse_attn(const csa2_cache& cache, int n_layers, int n_queries, const int32_t* q_req,
-                               const int32_t* topk, int k, const uint16_t* const* q, int H, float scale,
+                               const int32_t* const* topk, int k, const uint16_t* const* q, int H, float scale,
                                uint16_t* const* out, cudaStream_t stream, const uint8_t* swa_codes,
                                const uint8_t* swa_exp, const int32_t* q_pos, int window, void* xchg) {
   AttnLayers io = {};
   for (int l = 0; l < n_layers; ++l) {
+    io.topk[l] = topk[l];
     io.q[l] = reinterpret_cast<const __nv_bfloat16*>(q[l]);
     io.out[l] = reinterpret_cast<__nv_bfloat16*>(out[l]);
   }
   const SwaArgs swa = {swa_codes, swa_exp, q_pos, window};
   float* xf = static_cast<float*>(xchg);
   switch (H) {
-    case 16: return launch_h<16>(cache, n_layers, n_queries, q_req, topk, k, io, scale, swa, xf, stream);
-    case 32: return launch_h<32>(cache, n_layers, n_queries, q_req, topk, k, io, scale, swa, xf, stream);
-    case 64: return launch_h<64>(cache, n_layers, n_queries, q_req, topk, k, io, scale, swa, xf, stream);
+    case 16: return launch_h<16>(cache, n_layers, n_queries, q_req, k, io, scale, swa, xf, stream);
+    case 32: return launch_h<32>(cache, n_layers, n_queries, q_req, k, io, scale, swa, xf, stream);
+    case 64: return launch_h<64>(cache, n_layers, n_queries, q_req, k, io, scale, swa, xf, stream);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -18,6 +18,9 @@
 //     score, block max over 8 lanes, stores.  The exponent bytes are read
 //     straight from global memory one unit ahead.  Group 0 also quantises each
 //     request's query into the B-operand tile (three buffers) for the MMA.
+//     With a histogram buffer, each block max also adds one count to its
+//     request's histogram of leading order-key bits, from which the pool
+//     selection finds its threshold's leading bits without a pass.
 // Per 256 positions the handshake is one stage and one accumulator pair: the
 // scan streams at the HBM rate instead of the rate of barrier round trips.
 // Every mbarrier wait is bounded; a wait that runs out records
@@ -93,7 +96,7 @@ __device__ __forceinline__ int next_request_with_tiles(const int* prefix, int ba
 
 __global__ void __launch_bounds__(kThreads, 1)
     index_full_kernel(const csa2_cache cache, const float* __restrict__ q, const float* __restrict__ w,
-                      float* __restrict__ blockmax, float* __restrict__ scores,
+                      float* __restrict__ blockmax, float* __restrict__ scores, uint32_t* __restrict__ hist,
                       const __grid_constant__ CUtensorMap ik_map, uint64_t wait_ns) {
   extern __shared__ uint8_t smem_raw[];
   IndexSmem& S = *reinterpret_cast<IndexSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -350,8 +353,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 1));
           bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 2));
           bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 4));
-          if ((lane & 7) == 0 && valid)
+          if ((lane & 7) == 0 && valid) {
             blockmax[static_cast<long long>(cur_b) * (capacity / kBlock) + p / kBlock] = bm;
+            // one count per block in the request's histogram of leading key bits
+            if (hist != nullptr)
+              atomicAdd(&hist[static_cast<long long>(cur_b) * kPoolHistBins + (order_key(bm) >> (32 - kPoolHistBits))],
+                        1u);
+          }
           if (scores != nullptr && valid) scores[static_cast<long long>(cur_b) * capacity + p] = sc;
         }
         ex_cur[0] = ex_next[0];
@@ -375,7 +383,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 size_t index_full_smem_bytes() { return sizeof(IndexSmem) + 1024; }
 
 cudaError_t launch_index_full(const csa2_cache& cache, const float* q, const float* w, float* blockmax,
-                              float* scores, const CUtensorMap& ik_map, int num_sms, uint64_t wait_ns,
+                              float* scores, uint32_t* hist, const CUtensorMap& ik_map, int num_sms, uint64_t wait_ns,
                               cudaStream_t stream) {
   static ContextMemo attrs;
   const size_t smem = index_full_smem_bytes();
@@ -393,7 +401,7 @@ cudaError_t launch_index_full(const csa2_cache& cache, const float* q, const flo
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, index_full_kernel, cache, q, w, blockmax, scores, ik_map, wait_ns);
+  return cudaLaunchKernelEx(&cfg, index_full_kernel, cache, q, w, blockmax, scores, hist, ik_map, wait_ns);
 }
 
 }  // namespace csa2

@@ -9,6 +9,7 @@
 //     or recomputes them the same way [readance summary, section 4.2: modes];
 //   * copy_topk: Reuse mode, the previous layer's indices.
 // Ties go to the lower block id / position; outputs are ascending, -1 padded.
+#include "block_topk.cuh"
 #include "cluster_topk.cuh"
 #include "index_common.cuh"
 #include "launch.h"
@@ -24,10 +25,17 @@ constexpr int kPoolKeysPerCta = 16384;
 struct PoolSmem {
   uint32_t keys[kPoolKeysPerCta];
   SelectSmem sel;
+  SelectStart start;
 };
 
+// With `hist` (the scan's per-request histogram of the leading 14 bits of the
+// block-max order keys), every CTA of the cluster reads it, finds the bin that
+// holds the pool's threshold and starts the radix select below those 14 bits;
+// the CTAs then zero their slices of it for the next scan.  A histogram that
+// does not hold exactly one count per block is ignored (select from scratch).
 __global__ void __launch_bounds__(kPoolThreads, 1)
-    pool_select_kernel(const csa2_cache cache, const float* __restrict__ blockmax, int P, int32_t* __restrict__ pool) {
+    pool_select_kernel(const csa2_cache cache, const float* __restrict__ blockmax, uint32_t* __restrict__ hist, int P,
+                       int32_t* __restrict__ pool) {
   extern __shared__ uint8_t smem_raw[];
   PoolSmem& S = *reinterpret_cast<PoolSmem*>(smem_raw);
   pdl_wait();                 // the block maxima of the scan are complete
@@ -57,10 +65,33 @@ __global__ void __launch_bounds__(kPoolThreads, 1)
       if (i < nloc) S.keys[i] = order_key(v[u]);
     }
   }
-  __syncthreads();
+  const SelectStart* start = nullptr;
+  if (hist != nullptr) {
+    // this thread's 32 bins, highest first: thread order is descending bin order
+    constexpr int kNB = kPoolHistBins / kPoolThreads;   // 32
+    const int base = kNB * (kPoolThreads - 1 - static_cast<int>(threadIdx.x));
+    const uint4* hb = reinterpret_cast<const uint4*>(hist + static_cast<long long>(b) * kPoolHistBins + base);
+    uint32_t c[kNB];
+#pragma unroll
+    for (int i = 0; i < kNB / 4; ++i) {
+      const uint4 v = hb[i];
+      c[kNB - 1 - 4 * i] = v.x;
+      c[kNB - 2 - 4 * i] = v.y;
+      c[kNB - 3 - 4 * i] = v.z;
+      c[kNB - 4 - 4 * i] = v.w;
+    }
+    if (hist_head_start<kPoolThreads, kNB>(c, base + kNB - 1, kPoolHistBits, nblk, P, S.sel.warp_tmp, &S.start))
+      start = &S.start;
+  }
+  __syncthreads();   // the keys (and a head start) are in shared memory
   int32_t* out = pool + static_cast<long long>(b) * P;
   cluster_topk<kPoolThreads>(
-      S.keys, nloc, P, S.sel, [&](int i, int r) { out[r] = j0 + i; }, [&](int r) { out[r] = -1; });
+      S.keys, nloc, P, S.sel, [&](int i, int r) { out[r] = j0 + i; }, [&](int r) { out[r] = -1; }, start);
+  if (hist != nullptr) {   // every CTA has read the histogram before the select's last cluster barrier
+    const int per = kPoolHistBins / C;
+    uint4* hz = reinterpret_cast<uint4*>(hist + static_cast<long long>(b) * kPoolHistBins + rank * per);
+    for (int i = threadIdx.x; i < per / 4; i += kPoolThreads) hz[i] = make_uint4(0u, 0u, 0u, 0u);
+  }
 }
 
 // --------------------------------------------------------------- reindex ----
@@ -370,14 +401,14 @@ cudaError_t configure(Kernel kernel, size_t smem, ContextMemo& memo) {
 
 }  // namespace
 
-cudaError_t launch_pool_select(const csa2_cache& cache, const float* blockmax, int pool_blocks, int32_t* pool,
-                               int cluster, cudaStream_t stream) {
+cudaError_t launch_pool_select(const csa2_cache& cache, const float* blockmax, uint32_t* hist, int pool_blocks,
+                               int32_t* pool, int cluster, cudaStream_t stream) {
   static ContextMemo done;
   const size_t smem = sizeof(PoolSmem);
   cudaError_t e = configure(pool_select_kernel, smem, done);
   if (e != cudaSuccess) return e;
   return launch_cluster(pool_select_kernel, cache.batch * cluster, kPoolThreads, smem, cluster, stream, cache,
-                        blockmax, pool_blocks, pool);
+                        blockmax, hist, pool_blocks, pool);
 }
 
 size_t reindex_smem_bytes(int max_blocks) { return ReindexLayout::make(max_blocks).total + 1024; }

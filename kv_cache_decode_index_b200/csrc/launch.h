@@ -62,11 +62,19 @@ cudaError_t launch_compress_append(const csa2_cache& cache, int n_entries, int m
 
 size_t index_full_smem_bytes();
 cudaError_t launch_index_full(const csa2_cache& cache, const float* q, const float* w, float* blockmax,
-                              float* scores, const CUtensorMap& ik_map, int num_sms, uint64_t wait_ns,
+                              float* scores, uint32_t* hist, const CUtensorMap& ik_map, int num_sms, uint64_t wait_ns,
                               cudaStream_t stream);
 
-cudaError_t launch_pool_select(const csa2_cache& cache, const float* blockmax, int pool_blocks, int32_t* pool,
-                               int cluster, cudaStream_t stream);
+cudaError_t launch_pool_select(const csa2_cache& cache, const float* blockmax, uint32_t* hist, int pool_blocks,
+                               int32_t* pool, int cluster, cudaStream_t stream);
+
+// Top-k of n_layers layers over the pool: one scoring launch (every pool
+// block gathered once, all layers in one MMA) and one select launch.
+size_t rescore_workspace_bytes(long long batch, int n_layers, int pool_blocks);
+cudaError_t launch_rescore_layers(const csa2_cache& cache, int n_layers, const int32_t* pool, int pool_blocks,
+                                  const float* const* q, const float* const* w, int k, int32_t* const* topk,
+                                  void* workspace, const CUtensorMap& blk_map, int num_sms, uint64_t wait_ns,
+                                  cudaStream_t stream);
 
 constexpr int kReindexPoolCluster = 16;   // CTAs per request when re-scoring a pool
 cudaError_t launch_reindex(const csa2_cache& cache, const int32_t* pool, int pool_blocks, const float* q,
@@ -84,12 +92,12 @@ cudaError_t launch_prefill_index(const csa2_cache& cache, int req, int n_queries
 
 cudaError_t launch_copy_topk(const int32_t* src, int32_t* dst, long long n, cudaStream_t stream);
 
-// q[l] / out[l] (host array of device pointers): query and output of layer l
-// of n_layers layers sharing the Top-k.
+// topk[l] / q[l] / out[l] (host arrays of device pointers): Top-k, query and
+// output of layer l of n_layers layers (layers may share a Top-k).
 // swa_codes == nullptr: no sliding window; else the window of `window`
 // tokens ending at q_pos[i] is merged into query i's softmax.
 cudaError_t launch_sparse_attn(const csa2_cache& cache, int n_layers, int n_queries, const int32_t* q_req,
-                               const int32_t* topk, int k, const uint16_t* const* q, int H, float scale,
+                               const int32_t* const* topk, int k, const uint16_t* const* q, int H, float scale,
                                uint16_t* const* out, cudaStream_t stream, const uint8_t* swa_codes = nullptr,
                                const uint8_t* swa_exp = nullptr, const int32_t* q_pos = nullptr, int window = 0,
                                void* xchg = nullptr);

@@ -25,7 +25,7 @@ def declared_symbols():
 
 def test_every_declared_symbol_is_exported(lib):
     names = declared_symbols()
-    assert len(names) == 17, names
+    assert len(names) == 19, names
     so = ctypes.CDLL(lib.LIB_PATH)
     for n in names:
         assert hasattr(so, n), f"{n} missing from libcsa2.so"
@@ -46,15 +46,31 @@ def test_host_side_validation(lib):
     L = lib._lib
     c, p = _cache(lib)
     P = ctypes.c_void_p(p)
-    assert L.csa2_index_full(None, P, P, P, None, None) == lib.ERR_ARG
+    assert L.csa2_index_full(None, P, P, P, None, None, None) == lib.ERR_ARG
     bad, _ = _cache(lib, batch=0)
-    assert L.csa2_index_full(ctypes.byref(bad), P, P, P, None, None) == lib.ERR_SHAPE
+    assert L.csa2_index_full(ctypes.byref(bad), P, P, P, None, None, None) == lib.ERR_SHAPE
     bad, _ = _cache(lib, page_size=100)
-    assert L.csa2_pool_select(ctypes.byref(bad), P, 2048, P, None) == lib.ERR_SHAPE
+    assert L.csa2_pool_select(ctypes.byref(bad), P, None, 2048, P, None) == lib.ERR_SHAPE
     bad, _ = _cache(lib, ik_codes=p + 4)
-    assert L.csa2_index_full(ctypes.byref(bad), P, P, P, None, None) == lib.ERR_ARG
+    assert L.csa2_index_full(ctypes.byref(bad), P, P, P, None, None, None) == lib.ERR_ARG
     assert b"16-byte" in L.csa2_last_error_message()
-    assert L.csa2_pool_select(ctypes.byref(c), P, 0, P, None) == lib.ERR_SHAPE
+    assert L.csa2_pool_select(ctypes.byref(c), P, None, 0, P, None) == lib.ERR_SHAPE
+    assert L.csa2_pool_select(ctypes.byref(c), P, ctypes.c_void_p(p + 4), 2048, P, None) == lib.ERR_ARG
+    assert L.csa2_index_full(ctypes.byref(c), P, P, P, None, ctypes.c_void_p(p + 4), None) == lib.ERR_ARG
+    # multi-layer Top-k over a pool: layer count, k, pointers and workspace are checked on the host
+    rw = L.csa2_reindex_layers_workspace_bytes
+    assert rw(2, 3, 2048) == 2 * 3 * (2048 * 8 + 4096) * 4 and rw(0, 3, 2048) == 0
+    rl = L.csa2_reindex_layers
+    pa = (ctypes.c_void_p * 3)(p, p, p)
+    rneed = rw(2, 3, 2048)
+    assert rl(ctypes.byref(c), 9, P, 2048, pa, pa, 512, pa, P, rneed, None) == lib.ERR_SHAPE
+    assert rl(ctypes.byref(c), 3, P, 2048, pa, pa, 0, pa, P, rneed, None) == lib.ERR_SHAPE
+    assert rl(ctypes.byref(c), 3, None, 2048, pa, pa, 512, pa, P, rneed, None) == lib.ERR_ARG
+    assert rl(ctypes.byref(c), 3, P, 2048, pa, pa, 512, pa, P, rneed - 4, None) == lib.ERR_SHAPE
+    assert b"csa2_reindex_layers_workspace_bytes" in L.csa2_last_error_message()
+    assert rl(ctypes.byref(c), 3, P, 2048, pa, pa, 512, pa, None, rneed, None) == lib.ERR_ARG
+    pz = (ctypes.c_void_p * 3)(p, None, p)
+    assert rl(ctypes.byref(c), 3, P, 2048, pa, pz, 512, pa, P, rneed, None) == lib.ERR_ARG
     assert L.csa2_reindex(ctypes.byref(c), lib.REINDEX, P, 2048, P, P, None, None, 0, P, None) == lib.ERR_SHAPE
     assert L.csa2_reindex(ctypes.byref(c), 7, P, 2048, P, P, None, None, 512, P, None) == lib.ERR_ARG
     assert L.csa2_reindex(ctypes.byref(c), lib.REUSE, None, 0, None, None, None, None, 512, P, None) == lib.ERR_ARG
@@ -88,11 +104,13 @@ def test_host_side_validation(lib):
     al = L.csa2_sparse_attn_layers
     qa = (ctypes.c_void_p * 2)(p, p)
     wneed = aw(2, 2, 64)
-    assert al(ctypes.byref(c), 2, 2, None, P, 512, qa, 64, ctypes.c_float(0.1), qa, P, wneed - 4, None) == lib.ERR_SHAPE
+    assert al(ctypes.byref(c), 2, 2, None, qa, 512, qa, 64, ctypes.c_float(0.1), qa, P, wneed - 4, None) == lib.ERR_SHAPE
     assert b"csa2_attn_workspace_bytes" in L.csa2_last_error_message()
-    assert al(ctypes.byref(c), 2, 2, None, P, 512, qa, 64, ctypes.c_float(0.1), qa, ctypes.c_void_p(p + 4), wneed,
+    assert al(ctypes.byref(c), 2, 2, None, qa, 512, qa, 64, ctypes.c_float(0.1), qa, ctypes.c_void_p(p + 4), wneed,
               None) == lib.ERR_ARG
-    assert al(ctypes.byref(c), 9, 2, None, P, 512, qa, 64, ctypes.c_float(0.1), qa, None, 0, None) == lib.ERR_SHAPE
+    assert al(ctypes.byref(c), 9, 2, None, qa, 512, qa, 64, ctypes.c_float(0.1), qa, None, 0, None) == lib.ERR_SHAPE
+    tz = (ctypes.c_void_p * 2)(p, None)
+    assert al(ctypes.byref(c), 2, 2, None, tz, 512, qa, 64, ctypes.c_float(0.1), qa, None, 0, None) == lib.ERR_ARG
     ps = L.csa2_prefill_index_static
     assert ps(ctypes.byref(c), 0, 257, P, 2, P, P, 512, P, None) == lib.ERR_SHAPE   # above the static limit
     assert b"static scratch" in L.csa2_last_error_message()

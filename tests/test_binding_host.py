@@ -29,13 +29,21 @@ def _cpu_cache():
 
 def test_groups_alias_reuse_topk_and_count_launches():
     """Built on host tensors (no launch): Reuse layers share their source's
-    Top-k buffer, and the launch names / counts follow the grouping."""
-    g = csa2.DecodeGroup(_cpu_cache(), ("F", "Ri", "Ri", "Ru", "Ru", "Ru"), 64, 512, 2048, concurrent=False)
+    Top-k buffer; with a pool the step is scan, pool, one two-kernel Top-k of
+    every index layer and one attention launch; without one, one flat Top-k
+    per index layer."""
+    g = csa2.DecodeGroup(_cpu_cache(), ("F", "Ri", "Ri", "Ru", "Ru", "Ru"), 64, 512, 2048)
     assert all(g.topk[layer] is g.topk[2] for layer in (3, 4, 5))
     assert len({id(g.topk[layer]) for layer in (0, 1, 2)}) == 3
-    assert g.launch_names() == ["scan", "pool", "topk0", "attn0", "topk1", "attn1", "topk2", "attn2"]
-    assert g.launches_per_step == len(g.launch_names())
-    assert [w.numel() for w in g.attn_ws] == [csa2.attn_workspace_bytes(len(s), 1, 64) for s in g.sources]
+    assert g.index_layers == [0, 1, 2]
+    assert g.launch_names() == ["scan", "pool", "topk", "attn"] and g.launches_per_step == 5
+    assert g.attn_ws.numel() == csa2.attn_workspace_bytes(6, 1, 64)
+    assert g.rs_ws.numel() == csa2.reindex_layers_workspace_bytes(1, 3, 2048)
+    assert g.hist.shape == (1, csa2.POOL_HIST_BINS) and int(g.hist.abs().sum()) == 0
+    assert int(g.rs_ws.sum()) == 0    # the histograms start at zero
+    g2 = csa2.DecodeGroup(_cpu_cache(), ("F", "Ri", "Ri", "Ri", "Ri", "Ru"), 64, 512, None)
+    assert g2.launch_names() == ["scan", "topk", "attn"] and g2.launches_per_step == 2 + 5
+    assert g2.hist is None and g2.pool is None
     p = csa2.PrefillGroup(_cpu_cache(), 0, ("F", "Ru", "Ru", "Ru", "Ru", "Ru"), 16, 8, 64)
     assert all(t is p.topk[0] for t in p.topk)
     assert p.launch_names() == ["topk0", "attn0"] and p.launches_per_step == 3   # the indexer is two kernels

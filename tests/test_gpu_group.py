@@ -146,42 +146,35 @@ def test_group_ragged_paged_with_append(csa2):
 
 
 def test_group_1m_b4_full_size(csa2):
-    """The 1M-context workload at full size, in the bench's launch configuration:
-    request 0 against the full oracle; requests 1..3 on sampled blocks and on
-    properties that hold at any size."""
+    """The 1M-context workload at full size, in the bench's launch
+    configuration: every request against the full oracle (pool, every layer's
+    Top-k, attention), the pool also against the exact top blocks of the GPU's
+    own block maxima, and the planted needles' pool recall and score margin
+    reported per request."""
     wl = W.WORKLOADS["group_1m_b4"]
     cache = U.build_cache(wl, csa2)
     dev = cache.device
     group, q_idx, w_idx, q_main, out = _run_gpu(csa2, wl, cache, dev)
     n = wl.ctx
-    ora, worst = _check_request(csa2, wl, cache, group, 0, n, q_idx, w_idx, q_main, out, dev)
-    needles = W.needle_positions(wl, 0)
-    ora_recall = np.isin(needles // 8, ora["pool"]).sum()
-    gpu_recall = np.isin(needles // 8, group.pool[0].cpu().numpy()).sum()
-    print(f"needle pool recall: oracle {ora_recall}/64, gpu {gpu_recall}/64; attention rel err {worst:.2e}")
-    assert ora_recall == gpu_recall
     bm_all = group.blockmax.cpu().numpy()
-    rng = np.random.default_rng(0)
-    for b in range(1, wl.batch):
-        bm = bm_all[b, :n // 8].astype(np.float64)
+    for b in range(wl.batch):
+        ora, worst = _check_request(csa2, wl, cache, group, b, n, q_idx, w_idx, q_main, out, dev)
         gp = group.pool[b].cpu().numpy()
-        # pool = exact top-2048 of the GPU's block maxima (ties -> lower id)
+        bm = bm_all[b, :n // 8].astype(np.float64)
         order = np.lexsort((np.arange(len(bm)), -bm))
-        np.testing.assert_array_equal(gp, np.sort(order[:2048]))
-        # sampled block maxima (including the needles' blocks) against the oracle
-        blocks = np.unique(np.concatenate([rng.choice(n // 8, 200, replace=False),
-                                           W.needle_positions(wl, b) // 8]))
-        pos = (blocks[:, None] * 8 + np.arange(8)).reshape(-1)
-        from oracle import formats as F
-        codes, exp = F.quantize_indexer(W.rows_at(wl, b, pos, "ik"))
-        s64 = C.indexer_scores(q_idx[0][b], w_idx[0][b], codes, exp)
-        bm64 = s64.reshape(-1, 8).max(axis=1)
-        assert np.all(np.abs(bm[blocks] - bm64) <= 1e-5 * np.abs(bm64))
-        pool_pos = set(C.pool_positions(gp, n).tolist())
-        for layer, m in enumerate(wl.modes):
-            t = group.topk[layer][b].cpu().numpy()
-            U.assert_sorted_padded(t)
-            assert (t >= 0).sum() == 512 and set(t.tolist()) <= pool_pos
+        np.testing.assert_array_equal(gp, np.sort(order[:2048]), err_msg=f"pool b={b}")
+        needles = W.needle_positions(wl, b)
+        s64 = ora["scores"]
+        sd = s64.std()
+        theta = np.sort(ora["blockmax"])[::-1][wl.pool_blocks - 1]   # the pool's threshold block max
+        z = (s64[needles] - s64.mean()) / sd
+        margin = (s64[needles] - theta) / sd
+        ora_recall = int(np.isin(needles // 8, ora["pool"]).sum())
+        gpu_recall = int(np.isin(needles // 8, gp).sum())
+        print(f"request {b}: needle pool recall oracle {ora_recall}/64, gpu {gpu_recall}/64; needle score "
+              f"z = {np.median(z):.2f} median ({z.min():.2f} min) standard deviations above the mean score; "
+              f"{np.median(margin):+.2f} median sd from the pool threshold; attention rel err {worst:.2e}")
+        assert ora_recall == gpu_recall
     assert csa2.get_error(cache)[0] == csa2.OK
 
 
@@ -242,9 +235,9 @@ def test_group_ragged_b64_full_size(csa2):
 
 
 def test_group_graph_replay_matches_eager(csa2):
-    """The bench times CUDA-graph replays of the step (side streams and
-    programmatic dependent launch inside the graph); a replay must give the
-    eager step's indices and outputs exactly, twice in a row."""
+    """The bench times CUDA-graph replays of the step (programmatic dependent
+    launch inside the graph); a replay must give the eager step's indices and
+    outputs exactly, twice in a row."""
     wl = W.WORKLOADS["group_64k_b8"]
     cache = U.build_cache(wl, csa2)
     dev = cache.device

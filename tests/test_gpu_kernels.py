@@ -233,11 +233,58 @@ def test_pool_select_bitexact(csa2, lengths, P):
     vals[:, ::3] = np.round(vals[:, ::3] * 4) / 4                       # ties
     vals[:, 5::7] = 2.0                                                  # a big tie group
     dev = cache.device
-    pool = csa2.pool_select(cache, torch.from_numpy(vals).to(dev), P).cpu().numpy()
+    tv = torch.from_numpy(vals).to(dev)
+    pool = csa2.pool_select(cache, tv, P).cpu().numpy()
     for b, n in enumerate(lengths):
         nb = -(-n // 8)
         ref = C.pool_select(vals[b, :nb].astype(np.float64), P)
         np.testing.assert_array_equal(pool[b], ref, err_msg=f"request {b} (n={n})")
+    # with the block maxima's histogram (as the scan writes it): the same pool,
+    # and the histogram is left zeroed; a histogram that does not match the
+    # block maxima (stale) is ignored, with the same result
+    hist = np.zeros((B, csa2.POOL_HIST_BINS), np.int64)
+    for b, n in enumerate(lengths):
+        hist[b] = np.bincount(_order_keys(vals[b, :-(-n // 8)]) >> 18, minlength=csa2.POOL_HIST_BINS)
+    th = torch.from_numpy(hist.astype(np.int32)).to(dev)
+    pool_h = csa2.pool_select(cache, tv, P, hist=th).cpu().numpy()
+    np.testing.assert_array_equal(pool_h, pool)
+    assert int(th.abs().sum()) == 0
+    th = torch.from_numpy((hist + rng.integers(0, 3, hist.shape)).astype(np.int32)).to(dev)
+    np.testing.assert_array_equal(csa2.pool_select(cache, tv, P, hist=th).cpu().numpy(), pool)
+    assert int(th.abs().sum()) == 0
+    assert csa2.get_error(cache)[0] == csa2.OK
+
+
+def _order_keys(v):
+    """The kernels' order-preserving uint32 key of an fp32 score (sign bit
+    flipped for positive values, all bits for negative ones; 0 -> 1)."""
+    bits = np.asarray(v, np.float32).view(np.uint32).astype(np.uint64)
+    k = np.where(bits & 0x80000000, ~bits & 0xFFFFFFFF, bits | 0x80000000)
+    return np.where(k == 0, 1, k).astype(np.uint64)
+
+
+def test_scan_histogram_drives_the_pool(csa2):
+    """The scan's histogram holds one count per visible block in the bin of
+    its block max's leading 14 key bits; the pool selected from it equals the
+    pool selected without it, and the histogram is zero again afterwards."""
+    wl = W.scaled(W.WORKLOADS["group_64k_b8"], batch=3, page_size=512, shuffle_pages=True)
+    lengths = [65536, 40001, 777]
+    cache = U.build_cache(wl, csa2, lengths=lengths)
+    q, w = W.index_query(wl, 0)
+    dev = cache.device
+    tq, tw = torch.from_numpy(q).to(dev), torch.from_numpy(w).to(dev)
+    hist = csa2.pool_hist(cache)
+    bm = csa2.index_full(cache, tq, tw, hist=hist)
+    h = hist.cpu().numpy().astype(np.int64)
+    bmh = bm.cpu().numpy()
+    for b, n in enumerate(lengths):
+        want = np.bincount(_order_keys(bmh[b, :-(-n // 8)]) >> 18, minlength=csa2.POOL_HIST_BINS)
+        np.testing.assert_array_equal(h[b], want, err_msg=f"request {b}")
+    pool_h = csa2.pool_select(cache, bm, 512, hist=hist)
+    assert int(hist.abs().sum()) == 0
+    pool = csa2.pool_select(cache, bm, 512)
+    assert torch.equal(pool_h, pool)
+    assert csa2.get_error(cache)[0] == csa2.OK
 
 
 # ---------------------------------------------------------- reindex (a4-a6) --
@@ -302,6 +349,67 @@ def test_reindex_rescore_parity(csa2):
         U.assert_set_parity(topk[b], ref, score_of, U.threshold(s64, 512), what=f"reindex b={b}")
 
 
+@pytest.mark.parametrize("n_layers,lengths,P", [(3, [65536, 20000, 4000], 2048), (5, [65536, 3001], 2048),
+                                                 (8, [9000, 300], 64), (1, [65536], 1000)])
+def test_reindex_layers_equal_per_layer_reindex(csa2, n_layers, lengths, P):
+    """csa2_reindex_layers (all layers gathered and scored at once, histogram
+    select) returns for every layer exactly what csa2_reindex returns for that
+    layer alone, on two calls in a row with the same workspace (whose
+    histograms each call leaves zeroed) and with a workspace whose histograms
+    were not zero; the first layer is checked against the oracle too."""
+    wl = W.scaled(W.WORKLOADS["group_64k_b8"], batch=len(lengths), shuffle_pages=True)
+    cache = U.build_cache(wl, csa2, lengths=lengths)
+    rng = np.random.default_rng(40 + n_layers)
+    pool = np.stack([_synthetic_pool(rng, n, P) for n in lengths])
+    dev = cache.device
+    tp = torch.from_numpy(pool).to(dev)
+    qs, ws = [], []
+    for layer in range(n_layers):
+        q, w = W.index_query(wl, layer)
+        qs.append(torch.from_numpy(q).to(dev))
+        ws.append(torch.from_numpy(w).to(dev))
+    want = [csa2.reindex(cache, csa2.REINDEX, 512, tp, qs[l], ws[l]).cpu().numpy() for l in range(n_layers)]
+    B = len(lengths)
+    nbytes = csa2.reindex_layers_workspace_bytes(B, n_layers, P)
+    ws_buf = torch.zeros(nbytes, dtype=torch.uint8, device=dev)
+    hist_part = ws_buf[B * n_layers * P * 8 * 4:]
+    for attempt in range(3):
+        if attempt == 2:   # histograms that do not match the keys
+            hist_part.copy_(torch.randint(0, 255, hist_part.shape, dtype=torch.uint8, device=dev))
+        got = csa2.reindex_layers(cache, tp, qs, ws, 512, workspace=ws_buf)
+        for l in range(n_layers):
+            np.testing.assert_array_equal(got[l].cpu().numpy(), want[l], err_msg=f"layer {l}, call {attempt}")
+        assert int(hist_part.sum()) == 0
+    assert csa2.get_error(cache)[0] == csa2.OK
+    q0, w0 = W.index_query(wl, 0)
+    for b, n in enumerate(lengths):
+        codes, exp = U.oracle_request(wl, b, n)
+        cand = C.pool_positions(pool[b], n)
+        s64 = C.indexer_scores(q0[b], w0[b], codes[cand], exp[cand])
+        score_of = dict(zip(cand.tolist(), s64.tolist())).get
+        U.assert_sorted_padded(want[0][b], f"request {b}")
+        U.assert_set_parity(want[0][b], C.reindex_topk(q0[b], w0[b], codes, exp, pool[b], n, 512), score_of,
+                            U.threshold(s64, 512), what=f"reindex_layers b={b}")
+
+
+def test_reindex_layers_full_layer_equals_stored_scores(csa2):
+    """A Full layer's Top-k from csa2_reindex_layers equals the Top-k of its
+    own scan's stored scores (bit-identical scoring arithmetic)."""
+    wl = W.scaled(W.WORKLOADS["group_64k_b8"], batch=2, shuffle_pages=True)
+    lengths = [65536, 12345]
+    cache = U.build_cache(wl, csa2, lengths=lengths)
+    dev = cache.device
+    q, w = W.index_query(wl, 0)
+    q1, w1 = W.index_query(wl, 1)
+    tq, tw = torch.from_numpy(q).to(dev), torch.from_numpy(w).to(dev)
+    sc = torch.empty(2, cache.capacity, device=dev)
+    bm = csa2.index_full(cache, tq, tw, scores=sc)
+    pool = csa2.pool_select(cache, bm, 2048)
+    full_st = csa2.reindex(cache, csa2.FULL, 512, pool, full_scores=sc)
+    got = csa2.reindex_layers(cache, pool, [tq, torch.from_numpy(q1).to(dev)], [tw, torch.from_numpy(w1).to(dev)], 512)
+    assert torch.equal(got[0], full_st)
+
+
 def test_reuse_copy_and_alias(csa2):
     cache = _flat_cache(csa2, 1024, batch=2)
     dev = cache.device
@@ -340,6 +448,26 @@ def test_sparse_attention_parity(csa2, H, k, n):
         ref = C.sparse_attention(qm[b].float().numpy(), full_codes, full_scales, topk[b], wl.scale)
         rel = U.assert_attention_close(out[b], ref, f"H={H} k={k} b={b}")
         print(f"H={H} k={k} b={b}: max rel err {rel:.2e}")
+
+
+def test_sparse_attention_layers_with_their_own_topk(csa2):
+    """One launch over layers with different Top-k equals one launch per layer."""
+    wl = W.scaled(W.WORKLOADS["group_64k_b8"], batch=3)
+    cache = U.build_cache(wl, csa2, lengths=[65536, 4000, 700])
+    dev = cache.device
+    rng = np.random.default_rng(11)
+    tks, qs = [], []
+    for layer in range(5):
+        t = np.stack([np.sort(rng.choice(n, 512, replace=False)) for n in (65536, 4000, 700)]).astype(np.int32)
+        t[2, 300:] = -1
+        tks.append(torch.from_numpy(t).to(dev))
+        qs.append(W.main_query(wl, layer).to(dev))
+    ws = torch.empty(csa2.attn_workspace_bytes(5, 3, 64), dtype=torch.uint8, device=dev)
+    multi = csa2.sparse_attn_layers(cache, tks, qs, wl.scale, workspace=ws)
+    for layer in range(5):
+        single = csa2.sparse_attn(cache, tks[layer], qs[layer], wl.scale)
+        assert torch.equal(multi[layer], single), f"layer {layer}"
+    assert csa2.get_error(cache)[0] == csa2.OK
 
 
 def test_sparse_attention_layers_equal_single_layer_launches(csa2):
