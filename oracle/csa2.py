@@ -117,6 +117,34 @@ def pool_select(blockmax, pool_blocks: int = POOL_BLOCKS) -> np.ndarray:
     return top_k_ascending(np.arange(len(m)), m, pool_blocks)
 
 
+def slice_candidates(blockmax_slice, block_offset: int, pool_blocks: int = POOL_BLOCKS):
+    """One context slice's candidates for a sharded pool: its own top
+    `pool_blocks` blocks (pool_select over the slice's block maxima) as
+    (block max, global block id) pairs, global id = local id + block_offset;
+    empty entries have id -1 (value 0)."""
+    m = np.asarray(blockmax_slice, dtype=np.float64)
+    local = pool_select(m, pool_blocks)
+    ok = local >= 0
+    values = np.zeros(pool_blocks)
+    values[ok] = m[local[ok]]
+    return values, np.where(ok, local + block_offset, -1)
+
+
+def pool_merge(cand_values, cand_ids, pool_blocks: int = POOL_BLOCKS) -> np.ndarray:
+    """The pool of a request whose context is split into slices (one per
+    device), from each slice's candidates (slice_candidates): the top
+    `pool_blocks` of the union by block max, ties to the lower global block id,
+    ascending, -1 padded.  A reading of the pages' remark that a 1M context may
+    have to be sharded across machines (alphalab analysis, limits section):
+    the merge is exact, because a block among the whole request's top
+    pool_blocks has fewer than pool_blocks blocks ahead of it in the whole
+    request, hence in its own slice, so its slice kept it."""
+    v = np.concatenate([np.asarray(x, dtype=np.float64).reshape(-1) for x in cand_values])
+    i = np.concatenate([np.asarray(x, dtype=np.int64).reshape(-1) for x in cand_ids])
+    keep = i >= 0
+    return top_k_ascending(i[keep], v[keep], pool_blocks)
+
+
 def pool_positions(pool, n: int) -> np.ndarray:
     """Expand pool block ids into the visible positions they cover (ascending)."""
     pool = np.asarray(pool, dtype=np.int64)

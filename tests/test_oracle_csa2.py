@@ -394,3 +394,51 @@ def test_swa_quantize_is_the_per_row_fp8_rule():
     r = y / sigma[:, None]
     step = np.ldexp(1.0, np.floor(np.log2(np.maximum(np.abs(r), 2.0 ** -6))).astype(np.int64) - 3)
     assert np.all(np.abs(v - r) <= step / 2 + 1e-12)
+
+
+# ------------------------------------------------------- sharded pool merge --
+
+@pytest.mark.parametrize("n,G,P", [(100000, 2, 2048), (100000, 3, 2048), (65536, 8, 512), (5000, 4, 2048),
+                                   (1000, 5, 64), (64, 2, 4)])
+def test_pool_merge_of_slices_equals_the_whole_pool(n, G, P):
+    """The merged candidates of G consecutive slices give exactly the pool of
+    the whole request (block maxima with many ties across slices), for even
+    and uneven slices, and slices shorter than the pool."""
+    rng = np.random.default_rng(n + G + P)
+    nb = -(-n // 8)
+    bm = np.round(rng.standard_normal(nb) * 3) / 3          # heavy ties
+    bm[rng.choice(nb, nb // 10, replace=False)] = 1.0       # one big tie group spread over every slice
+    cuts = np.sort(rng.choice(np.arange(1, nb), G - 1, replace=False)) if G > 1 else []
+    bounds = [0, *cuts, nb]
+    vals, ids = [], []
+    for g in range(G):
+        v, i = C.slice_candidates(bm[bounds[g]:bounds[g + 1]], bounds[g], P)
+        vals.append(v)
+        ids.append(i)
+    np.testing.assert_array_equal(C.pool_merge(vals, ids, P), C.pool_select(bm, P))
+
+
+def test_pool_merge_bruteforce_tiny():
+    """Brute force: sort every (value, id) pair by value desc, id asc."""
+    rng = np.random.default_rng(9)
+    for _ in range(200):
+        G = int(rng.integers(1, 4))
+        P = int(rng.integers(1, 6))
+        vals = [rng.integers(0, 3, P).astype(float) for _ in range(G)]
+        ids = [rng.permutation(50)[:P] for _ in range(G)]
+        for g in range(G):
+            ids[g][rng.random(P) < 0.2] = -1
+        pairs = sorted((-v, i) for g in range(G) for v, i in zip(vals[g], ids[g]) if i >= 0)
+        want = sorted(i for _, i in pairs[:P])
+        got = C.pool_merge(vals, ids, P)
+        np.testing.assert_array_equal(got[:len(want)], want)
+        assert np.all(got[len(want):] == -1)
+
+
+def test_slice_candidates_carry_global_ids_and_values():
+    bm = np.array([0.5, 3.0, 2.0, 3.0, -1.0])
+    v, i = C.slice_candidates(bm, 1000, 3)
+    np.testing.assert_array_equal(i, [1001, 1002, 1003])
+    np.testing.assert_array_equal(v, [3.0, 2.0, 3.0])
+    v, i = C.slice_candidates(bm[:2], 8, 4)
+    np.testing.assert_array_equal(i, [8, 9, -1, -1])

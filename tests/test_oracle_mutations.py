@@ -199,3 +199,32 @@ def test_mutation_fp4_score_drops_relu(monkeypatch):
         return (kv @ qv.T) @ np.asarray(w, dtype=np.float64)
     monkeypatch.setattr(C, "indexer_scores_fp4", bad)
     _fails(PC.test_fp4_score_reduces_to_plain_formula_on_exact_inputs)
+
+
+def test_mutation_slice_candidates_keep_local_ids(monkeypatch):
+    """Forgetting the slice's block offset."""
+    orig = C.slice_candidates
+    monkeypatch.setattr(C, "slice_candidates", lambda m, off, P=C.POOL_BLOCKS: orig(m, 0, P))
+    _fails(PC.test_pool_merge_of_slices_equals_the_whole_pool, 100000, 3, 2048)
+    _fails(PC.test_slice_candidates_carry_global_ids_and_values)
+
+
+def test_mutation_pool_merge_ties_to_higher_id(monkeypatch):
+    def bad(vals, ids, P=C.POOL_BLOCKS):
+        v = np.concatenate([np.asarray(x, dtype=np.float64).reshape(-1) for x in vals])
+        i = np.concatenate([np.asarray(x, dtype=np.int64).reshape(-1) for x in ids])
+        keep = i >= 0
+        order = np.lexsort((-i[keep], -v[keep]))
+        out = np.full(P, -1, np.int64)
+        sel = np.sort(i[keep][order[:P]])
+        out[:len(sel)] = sel
+        return out
+    monkeypatch.setattr(C, "pool_merge", bad)
+    _fails(PC.test_pool_merge_of_slices_equals_the_whole_pool, 100000, 3, 2048)
+    _fails(PC.test_pool_merge_bruteforce_tiny)
+
+
+def test_mutation_pool_merge_drops_the_last_slice(monkeypatch):
+    orig = C.pool_merge
+    monkeypatch.setattr(C, "pool_merge", lambda vals, ids, P=C.POOL_BLOCKS: orig(vals[:-1], ids[:-1], P))
+    _fails(PC.test_pool_merge_of_slices_equals_the_whole_pool, 100000, 3, 2048)
