@@ -177,7 +177,7 @@ CSA2_API csa2_status csa2_compress_append(const csa2_cache* cache, int32_t n_ent
 /*
  * Histogram of the block maxima passed from csa2_index_full to
  * csa2_pool_select: uint32 [batch][CSA2_POOL_HIST_BINS], one count per
- * visible block in the bin of its score's leading 14 order-key bits (the fp32
+ * visible block in the bin of its score's leading 11 order-key bits (the fp32
  * bit pattern with the sign bit flipped, or all bits flipped when negative).
  * The scan adds to it, so it must hold zeros when the scan starts;
  * csa2_pool_select reads it and zeroes it again.  Zero it once (for instance
@@ -186,7 +186,7 @@ CSA2_API csa2_status csa2_compress_append(const csa2_cache* cache, int32_t n_ent
  * scans, a scan that gave up) is detected and ignored by csa2_pool_select,
  * which then selects without it, exactly, and still zeroes it.
  */
-#define CSA2_POOL_HIST_BINS 16384
+#define CSA2_POOL_HIST_BINS 2048
 
 /*
  * csa2_index_full -- Full-mode indexer scan of every visible position of every
@@ -219,6 +219,48 @@ CSA2_API csa2_status csa2_index_full(const csa2_cache* cache, const float* q, co
  */
 CSA2_API csa2_status csa2_pool_select(const csa2_cache* cache, const float* blockmax, uint32_t* hist,
                              int32_t pool_blocks, int32_t* pool, void* stream);
+
+/*
+ * Context-sharded pool.  One request's context split into consecutive slices,
+ * one per device (slice g holds positions [start_g, start_g + len_g), start_g
+ * a multiple of 8), each device holding its slice in a cache of its own whose
+ * positions count from the slice start [alphalab analysis, limits section: a
+ * 1M context may have to be sharded across machines, with the exchange as
+ * its cost].  Per device: csa2_index_full and csa2_pool_select on the slice,
+ * then csa2_pool_candidates; the devices exchange the candidates (an
+ * all-gather of pool_blocks * 8 bytes per request and device); every device
+ * (or the one that continues) calls csa2_pool_merge.  The merged pool is
+ * exactly the pool csa2_pool_select returns for the unsharded request: a
+ * block of that pool has fewer than pool_blocks blocks ahead of it in its own
+ * slice, so its slice kept it.
+ *
+ * csa2_pool_candidates -- a slice's local pool as (block max, global block id)
+ * pairs.
+ *   shard        the slice's cache (ctx_len = the slice's visible length)
+ *   blockmax     float [batch][capacity/8] of the slice's scan
+ *   pool         int32 [batch][pool_blocks] of the slice's csa2_pool_select
+ *   block_offset global block id of the slice's block 0 (start_g / 8)
+ *   values       float [batch][pool_blocks] out (0 where the pool is -1)
+ *   ids          int32 [batch][pool_blocks] out: pool + block_offset, or -1
+ * Device errors: a pool entry outside [-1, ceil(ctx_len/8)) ->
+ * CSA2_ERR_DEVICE_BOUNDS, entry emptied.
+ *
+ * csa2_pool_merge -- the request's pool from the G slices' candidates.
+ *   values float [n_shards][batch][pool_blocks], ids int32 [same], the slices
+ *          in ascending order of their start (as gathered by rank), each list
+ *          ascending with -1 last (as csa2_pool_candidates writes it): the
+ *          candidate order is then the global block order that decides ties
+ *   pool   int32 [batch][pool_blocks] out: the pool_blocks best (block max
+ *          desc, global id asc), ascending, -1 padded
+ * n_shards in [1, CSA2_MAX_SHARDS], n_shards * pool_blocks <= 32768.  One
+ * CTA per request; no workspace.
+ */
+#define CSA2_MAX_SHARDS 16
+CSA2_API csa2_status csa2_pool_candidates(const csa2_cache* shard, const float* blockmax, const int32_t* pool,
+                                          int32_t pool_blocks, int32_t block_offset, float* values,
+                                          int32_t* ids, void* stream);
+CSA2_API csa2_status csa2_pool_merge(int32_t n_shards, int32_t batch, int32_t pool_blocks, const float* values,
+                                     const int32_t* ids, int32_t* pool, void* stream);
 
 /*
  * csa2_reindex -- Top-k of one layer of the group, by mode:

@@ -24,7 +24,7 @@ MODE = {"F": FULL, "Ri": REINDEX, "Ru": REUSE}
 OK, ERR_ARG, ERR_SHAPE, ERR_CUDA, ERR_DEVICE_BOUNDS, ERR_TIMEOUT, ERR_UNSUPPORTED = range(7)
 BLOCK, INDEX_HEADS, INDEX_DIM, KV_DIM, KV_CODE_BYTES, KV_SCALE_BYTES = 8, 32, 128, 512, 256, 32
 PREFILL_MAX_K, PREFILL_CANDIDATES, PREFILL_STATIC_MAX_QUERIES = 1024, 4096, 256
-POOL_HIST_BINS, RESCORE_HIST_BINS, MAX_SCORE_LAYERS = 16384, 4096, 8
+POOL_HIST_BINS, RESCORE_HIST_BINS, MAX_SCORE_LAYERS = 2048, 4096, 8
 
 
 class CacheStruct(ctypes.Structure):
@@ -44,6 +44,8 @@ _sig = {
     "csa2_pool_select": [_CP, _P, _P, _I, _P, _P],
     "csa2_reindex": [_CP, _I, _P, _I, _P, _P, _P, _P, _I, _P, _P],
     "csa2_reindex_layers": [_CP, _I, _P, _I, _P, _P, _I, _P, _P, ctypes.c_size_t, _P],
+    "csa2_pool_candidates": [_CP, _P, _P, _I, _I, _P, _P, _P],
+    "csa2_pool_merge": [_I, _I, _I, _P, _P, _P, _P],
     "csa2_sparse_attn": [_CP, _I, _P, _P, _I, _P, _I, ctypes.c_float, _P, _P],
     "csa2_sparse_attn_layers": [_CP, _I, _I, _P, _P, _I, _P, _I, ctypes.c_float, _P, _P, ctypes.c_size_t, _P],
     "csa2_swa_append": [_CP, _I, _P, _P, _I, _P, _P, _P, _P],

@@ -19,8 +19,8 @@ constexpr int kKvCodeBytes = CSA2_KV_CODE_BYTES;
 constexpr int kKvScaleBytes = CSA2_KV_SCALE_BYTES;
 constexpr int kBlock = CSA2_BLOCK;              // positions per pool block
 constexpr int kTile = 128;                      // positions per MMA tile (M)
-constexpr int kPoolHistBins = CSA2_POOL_HIST_BINS;   // 16384: leading 14 bits of a block-max order key
-constexpr int kPoolHistBits = 14;
+constexpr int kPoolHistBins = CSA2_POOL_HIST_BINS;   // 2048: leading 11 bits of a block-max order key
+constexpr int kPoolHistBits = 11;
 
 // kernel ids recorded in err_word[1]
 enum KernelId { kKAppend = 1, kKIndexFull = 2, kKPoolSelect = 3, kKReindex = 4, kKAttn = 5, kKPrefill = 6 };

@@ -306,6 +306,43 @@ csa2_status csa2_reindex_layers(const csa2_cache* cache, int32_t n_layers, const
   return e == cudaSuccess ? CSA2_OK : cuda_fail(e, "reindex_layers launch");
 }
 
+csa2_status csa2_pool_candidates(const csa2_cache* shard, const float* blockmax, const int32_t* pool,
+                                 int32_t pool_blocks, int32_t block_offset, float* values, int32_t* ids,
+                                 void* stream) {
+  CSA2_TRY(check_cache(shard, false, false));
+  if (blockmax == nullptr || pool == nullptr || values == nullptr || ids == nullptr)
+    return fail(CSA2_ERR_ARG, "blockmax, pool, values and ids must be set");
+  if (pool_blocks < 1 || pool_blocks > kMaxPool)
+    return fail(CSA2_ERR_SHAPE, "pool_blocks %d outside [1, %d]", pool_blocks, kMaxPool);
+  if (block_offset < 0 ||
+      static_cast<long long>(block_offset) + (capacity_of(shard) + csa2::kBlock - 1) / csa2::kBlock >= (1LL << 31))
+    return fail(CSA2_ERR_SHAPE, "block_offset %d: global block ids must lie in [0, 2^31)", block_offset);
+  DeviceInfo d;
+  CSA2_TRY(device_info(&d));
+  const cudaError_t e = csa2::launch_pool_candidates(*shard, blockmax, pool, pool_blocks, block_offset, values, ids,
+                                                     static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? CSA2_OK : cuda_fail(e, "pool_candidates launch");
+}
+
+csa2_status csa2_pool_merge(int32_t n_shards, int32_t batch, int32_t pool_blocks, const float* values,
+                            const int32_t* ids, int32_t* pool, void* stream) {
+  if (n_shards < 1 || n_shards > CSA2_MAX_SHARDS)
+    return fail(CSA2_ERR_SHAPE, "n_shards %d outside [1, %d]", n_shards, CSA2_MAX_SHARDS);
+  if (batch < 1 || batch > kMaxBatch) return fail(CSA2_ERR_SHAPE, "batch %d outside [1, %d]", batch, kMaxBatch);
+  if (pool_blocks < 1 || pool_blocks > kMaxPool)
+    return fail(CSA2_ERR_SHAPE, "pool_blocks %d outside [1, %d]", pool_blocks, kMaxPool);
+  if (static_cast<long long>(n_shards) * pool_blocks > 32768)
+    return fail(CSA2_ERR_SHAPE, "n_shards * pool_blocks = %lld exceeds 32768 candidates",
+                static_cast<long long>(n_shards) * pool_blocks);
+  if (values == nullptr || ids == nullptr || pool == nullptr)
+    return fail(CSA2_ERR_ARG, "values, ids and pool must be set");
+  DeviceInfo d;
+  CSA2_TRY(device_info(&d));
+  const cudaError_t e =
+      csa2::launch_pool_merge(n_shards, batch, pool_blocks, values, ids, pool, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? CSA2_OK : cuda_fail(e, "pool_merge launch");
+}
+
 csa2_status csa2_sparse_attn(const csa2_cache* cache, int32_t n_queries, const int32_t* q_req, const int32_t* topk,
                              int32_t k, const uint16_t* q, int32_t H, float scale, uint16_t* out, void* stream) {
   const uint16_t* qs[1] = {q};

@@ -19,8 +19,10 @@
 //     straight from global memory one unit ahead.  Group 0 also quantises each
 //     request's query into the B-operand tile (three buffers) for the MMA.
 //     With a histogram buffer, each block max also adds one count to its
-//     request's histogram of leading order-key bits, from which the pool
-//     selection finds its threshold's leading bits without a pass.
+//     request's histogram of leading order-key bits (in shared memory, flushed
+//     once per CTA: the maxima crowd into few bins, and global atomics on them
+//     would serialise), from which the pool selection finds its threshold's
+//     leading bits without a pass.
 // Per 256 positions the handshake is one stage and one accumulator pair: the
 // scan streams at the HBM rate instead of the rate of barrier round trips.
 // Every mbarrier wait is bounded; a wait that runs out records
@@ -56,6 +58,9 @@ struct __align__(1024) IndexSmem {
   uint64_t drain;
   uint32_t tmem_base;
   volatile int abort_flag;
+  // block-max histogram of the CTA's first two requests (slot = request -
+  // first request), two 16-bit counts per word; flushed to global memory once
+  uint32_t hist[2][kPoolHistBins / 2];
 };
 
 // Walks this CTA's units in order: request b, unit j inside it.
@@ -149,6 +154,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_relinquish();
   }
   if (warp == 0 && lane == 0) tma_prefetch_map(&ik_map);
+  if (hist != nullptr)
+    for (int i = tid; i < kPoolHistBins; i += kThreads) (&S.hist[0][0])[i] = 0u;
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -159,6 +166,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int t_end = static_cast<int>((static_cast<long long>(total) * (blockIdx.x + 1)) / G);
   const int n_tiles = t_end - t_begin;
   const uint32_t tmem = S.tmem_base;
+  // The histogram counts of this CTA's first two requests go to shared
+  // memory (16-bit counts: at most 32 blocks per unit, so fewer than 2^16 per
+  // bin while the CTA has fewer than 2048 units); other requests', or all
+  // when the CTA has more units, straight to global memory.
+  int hist_b0 = 0;
+  {
+    TileIter first;
+    first.init(S.prefix, B, t_begin);
+    hist_b0 = first.b;
+  }
+  const bool hist_smem = n_tiles < 2048;
 
   if (n_tiles > 0) {
     if (warp == 0) {
@@ -356,9 +374,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           if ((lane & 7) == 0 && valid) {
             blockmax[static_cast<long long>(cur_b) * (capacity / kBlock) + p / kBlock] = bm;
             // one count per block in the request's histogram of leading key bits
-            if (hist != nullptr)
-              atomicAdd(&hist[static_cast<long long>(cur_b) * kPoolHistBins + (order_key(bm) >> (32 - kPoolHistBits))],
-                        1u);
+            if (hist != nullptr) {
+              const uint32_t bin = order_key(bm) >> (32 - kPoolHistBits);
+              const int slot = cur_b - hist_b0;
+              if (hist_smem && slot < 2) atomicAdd(&S.hist[slot][bin >> 1], 1u << (16 * (bin & 1)));
+              else atomicAdd(&hist[static_cast<long long>(cur_b) * kPoolHistBins + bin], 1u);
+            }
           }
           if (scores != nullptr && valid) scores[static_cast<long long>(cur_b) * capacity + p] = sc;
         }
@@ -375,6 +396,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
+  }
+  if (hist != nullptr && hist_smem) {   // flush the non-zero counts of the two slots
+    for (int i = tid; i < kPoolHistBins; i += kThreads) {
+      const int slot = i / (kPoolHistBins / 2), w2 = i % (kPoolHistBins / 2);
+      const int b = hist_b0 + slot;
+      const uint32_t v = S.hist[slot][w2];
+      if (v == 0u || b >= B) continue;
+      uint32_t* g = hist + static_cast<long long>(b) * kPoolHistBins + 2 * w2;
+      if (v & 0xFFFFu) atomicAdd(g, v & 0xFFFFu);
+      if (v >> 16) atomicAdd(g + 1, v >> 16);
+    }
   }
 }
 

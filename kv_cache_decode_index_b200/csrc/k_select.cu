@@ -28,9 +28,9 @@ struct PoolSmem {
   SelectStart start;
 };
 
-// With `hist` (the scan's per-request histogram of the leading 14 bits of the
+// With `hist` (the scan's per-request histogram of the leading 11 bits of the
 // block-max order keys), every CTA of the cluster reads it, finds the bin that
-// holds the pool's threshold and starts the radix select below those 14 bits;
+// holds the pool's threshold and starts the radix select below those 11 bits;
 // the CTAs then zero their slices of it for the next scan.  A histogram that
 // does not hold exactly one count per block is ignored (select from scratch).
 __global__ void __launch_bounds__(kPoolThreads, 1)
@@ -67,8 +67,8 @@ __global__ void __launch_bounds__(kPoolThreads, 1)
   }
   const SelectStart* start = nullptr;
   if (hist != nullptr) {
-    // this thread's 32 bins, highest first: thread order is descending bin order
-    constexpr int kNB = kPoolHistBins / kPoolThreads;   // 32
+    // this thread's 4 bins, highest first: thread order is descending bin order
+    constexpr int kNB = kPoolHistBins / kPoolThreads;   // 4
     const int base = kNB * (kPoolThreads - 1 - static_cast<int>(threadIdx.x));
     const uint4* hb = reinterpret_cast<const uint4*>(hist + static_cast<long long>(b) * kPoolHistBins + base);
     uint32_t c[kNB];

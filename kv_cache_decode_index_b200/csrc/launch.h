@@ -90,6 +90,13 @@ cudaError_t launch_prefill_index(const csa2_cache& cache, int req, int n_queries
                                  const float* q, const float* w, int k, int32_t* topk, void* workspace,
                                  const CUtensorMap& ik_map, uint64_t wait_ns, cudaStream_t stream);
 
+// Sharded pool: a slice's (block max, global id) candidates, and the exact
+// merge of G slices' candidates ([G][batch][P] each).
+cudaError_t launch_pool_candidates(const csa2_cache& cache, const float* blockmax, const int32_t* pool, int P,
+                                   int block_offset, float* values, int32_t* ids, cudaStream_t stream);
+cudaError_t launch_pool_merge(int n_shards, int batch, int P, const float* values, const int32_t* ids, int32_t* pool,
+                              cudaStream_t stream);
+
 cudaError_t launch_copy_topk(const int32_t* src, int32_t* dst, long long n, cudaStream_t stream);
 
 // topk[l] / q[l] / out[l] (host arrays of device pointers): Top-k, query and

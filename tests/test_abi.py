@@ -25,7 +25,7 @@ def declared_symbols():
 
 def test_every_declared_symbol_is_exported(lib):
     names = declared_symbols()
-    assert len(names) == 19, names
+    assert len(names) == 21, names
     so = ctypes.CDLL(lib.LIB_PATH)
     for n in names:
         assert hasattr(so, n), f"{n} missing from libcsa2.so"
@@ -111,6 +111,16 @@ def test_host_side_validation(lib):
     assert al(ctypes.byref(c), 9, 2, None, qa, 512, qa, 64, ctypes.c_float(0.1), qa, None, 0, None) == lib.ERR_SHAPE
     tz = (ctypes.c_void_p * 2)(p, None)
     assert al(ctypes.byref(c), 2, 2, None, tz, 512, qa, 64, ctypes.c_float(0.1), qa, None, 0, None) == lib.ERR_ARG
+    # sharded pool: shard count, sizes and pointers are checked on the host
+    pm = L.csa2_pool_merge
+    assert pm(0, 2, 2048, P, P, P, None) == lib.ERR_SHAPE
+    assert pm(17, 2, 2048, P, P, P, None) == lib.ERR_SHAPE
+    assert pm(16, 2, 4096, P, P, P, None) == lib.ERR_SHAPE        # more than 32768 candidates
+    assert pm(2, 2, 2048, None, P, P, None) == lib.ERR_ARG
+    pc = L.csa2_pool_candidates
+    assert pc(ctypes.byref(c), P, P, 0, 0, P, P, None) == lib.ERR_SHAPE
+    assert pc(ctypes.byref(c), P, P, 2048, -1, P, P, None) == lib.ERR_SHAPE
+    assert pc(ctypes.byref(c), P, None, 2048, 0, P, P, None) == lib.ERR_ARG
     ps = L.csa2_prefill_index_static
     assert ps(ctypes.byref(c), 0, 257, P, 2, P, P, 512, P, None) == lib.ERR_SHAPE   # above the static limit
     assert b"static scratch" in L.csa2_last_error_message()

@@ -123,3 +123,48 @@ def test_prefill_flops_closed_form():
     import bench
     wl = W.WORKLOADS["prefill_256k_q8192"]
     assert bench.prefill_flops(wl) == 2 * 32 * 128 * (8192 * 258048 + 4096 * 4096)
+
+
+def _shard_rank_main(rank, world, port, out):
+    """Rank g holds slice g of two requests' block maxima; the candidates are
+    exchanged with the product's all-gather and merged with the oracle."""
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        import numpy as np
+        from kv_cache_decode_index_b200 import sharded
+        from oracle import csa2 as C
+        rng = np.random.default_rng(5)
+        nb, P = 5000, 512
+        bm = np.round(rng.standard_normal((2, nb)) * 4) / 4          # ties across the slices
+        cut = [0, 2100, nb]
+        v = np.zeros((2, P), np.float32)
+        i = np.zeros((2, P), np.int32)
+        for b in range(2):
+            vb, ib = C.slice_candidates(bm[b, cut[rank]:cut[rank + 1]], cut[rank], P)
+            v[b], i[b] = vb, ib
+        all_v, all_i = sharded.exchange_candidates(torch.from_numpy(v), torch.from_numpy(i))
+        assert tuple(all_v.shape) == (world, 2, P) and tuple(all_i.shape) == (world, 2, P)
+        merged = [C.pool_merge(all_v[:, b].numpy(), all_i[:, b].numpy(), P) for b in range(2)]
+        whole = [C.pool_select(bm[b].astype(np.float32).astype(np.float64), P) for b in range(2)]
+        out[rank] = all(np.array_equal(m, w) for m, w in zip(merged, whole)) and \
+            bool((all_i[rank].numpy() == i).all())
+    finally:
+        dist.destroy_process_group()
+
+
+def test_sharded_pool_exchange_gloo_two_ranks():
+    ctx = mp.get_context("spawn")
+    with ctx.Manager() as m:
+        out = m.dict()
+        mp.start_processes(_shard_rank_main, args=(2, _free_port(), out), nprocs=2, start_method="spawn", join=True)
+        assert dict(out) == {0: True, 1: True}
+
+
+def test_slice_pages_cover_the_table():
+    from kv_cache_decode_index_b200 import sharded
+    for pages, g in [(256, 2), (256, 8), (10, 3), (7, 7), (5, 1)]:
+        s = sharded.slice_pages(pages, g)
+        assert len(s) == g and s[0][0] == 0 and sum(n for _, n in s) == pages
+        assert all(s[k][0] + s[k][1] == s[k + 1][0] for k in range(g - 1))
+        assert max(n for _, n in s) - min(n for _, n in s) <= 1

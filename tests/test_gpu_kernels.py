@@ -244,7 +244,7 @@ def test_pool_select_bitexact(csa2, lengths, P):
     # block maxima (stale) is ignored, with the same result
     hist = np.zeros((B, csa2.POOL_HIST_BINS), np.int64)
     for b, n in enumerate(lengths):
-        hist[b] = np.bincount(_order_keys(vals[b, :-(-n // 8)]) >> 18, minlength=csa2.POOL_HIST_BINS)
+        hist[b] = np.bincount(_order_keys(vals[b, :-(-n // 8)]) >> 21, minlength=csa2.POOL_HIST_BINS)
     th = torch.from_numpy(hist.astype(np.int32)).to(dev)
     pool_h = csa2.pool_select(cache, tv, P, hist=th).cpu().numpy()
     np.testing.assert_array_equal(pool_h, pool)
@@ -265,7 +265,7 @@ def _order_keys(v):
 
 def test_scan_histogram_drives_the_pool(csa2):
     """The scan's histogram holds one count per visible block in the bin of
-    its block max's leading 14 key bits; the pool selected from it equals the
+    its block max's leading 11 key bits; the pool selected from it equals the
     pool selected without it, and the histogram is zero again afterwards."""
     wl = W.scaled(W.WORKLOADS["group_64k_b8"], batch=3, page_size=512, shuffle_pages=True)
     lengths = [65536, 40001, 777]
@@ -278,7 +278,7 @@ def test_scan_histogram_drives_the_pool(csa2):
     h = hist.cpu().numpy().astype(np.int64)
     bmh = bm.cpu().numpy()
     for b, n in enumerate(lengths):
-        want = np.bincount(_order_keys(bmh[b, :-(-n // 8)]) >> 18, minlength=csa2.POOL_HIST_BINS)
+        want = np.bincount(_order_keys(bmh[b, :-(-n // 8)]) >> 21, minlength=csa2.POOL_HIST_BINS)
         np.testing.assert_array_equal(h[b], want, err_msg=f"request {b}")
     pool_h = csa2.pool_select(cache, bm, 512, hist=hist)
     assert int(hist.abs().sum()) == 0
