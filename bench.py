@@ -49,6 +49,7 @@ METRIC = "CSA2 decode queries/s per layer group at 1M ctx; achieved HBM GB/s vs 
 NOMINAL_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
 IK_ROW_BYTES = 129     # 128 FP8 codes + 1 exponent byte
+IK4_ROW_BYTES = 72     # FP4 indexer: 64 E2M1 code bytes + 8 E4M3 scales
 KV_ROW_BYTES = 288     # 256 E2M1 bytes + 32 E4M3 scales
 POOL_ENTRY_BYTES = 4
 
@@ -65,7 +66,7 @@ def rank_workload(wl, rank: int):
     return wl if rank == 0 else W.scaled(wl, seed=wl.seed + 1000 * rank)
 
 
-def alg_bytes(wl, lengths=None):
+def alg_bytes(wl, lengths=None, ik_row_bytes=IK_ROW_BYTES):
     """Algorithmic HBM bytes of one step and of one Full-scan launch.
 
     Per request: the Full scan reads every visible indexer-K row (129 B); each
@@ -77,19 +78,33 @@ def alg_bytes(wl, lengths=None):
     n_ri = sum(1 for m in wl.modes if m == "Ri")
     P = wl.pool_blocks or 0
     cand = np.minimum(n, P * 8) if P else n
-    scan = int((IK_ROW_BYTES * n).sum())
-    step = scan + int((n_ri * IK_ROW_BYTES * cand).sum()) + \
+    scan = int((ik_row_bytes * n).sum())
+    step = scan + int((n_ri * ik_row_bytes * cand).sum()) + \
         int((len(wl.modes) * KV_ROW_BYTES * np.minimum(n, wl.topk)).sum()) + \
         (POOL_ENTRY_BYTES * P * (1 + n_ri) * len(n) if P else 0)
     return step, scan
 
 
+def append_rows(wl, dev):
+    """(kv_new [B,512], ik_new [B,128], pos [B]) of each request's newest row:
+    its last visible position, regenerated from the workload's seeds."""
+    import torch
+    last = W.ctx_lengths(wl) - 1
+    kv = np.stack([W.rows_at(wl, b, [last[b]], "kv")[0] for b in range(wl.batch)]).astype(np.float32)
+    ik = np.stack([W.rows_at(wl, b, [last[b]], "ik")[0] for b in range(wl.batch)]).astype(np.float32)
+    return (torch.from_numpy(kv).to(dev), torch.from_numpy(ik).to(dev),
+            torch.from_numpy(last.astype(np.int32)).to(dev))
+
+
 def io_bytes(wl):
     """Host<->device bytes of one end-to-end step: indexer queries and head
-    weights of every non-Reuse layer, main queries in; attention outputs out."""
+    weights of every non-Reuse layer, main queries (and the appended rows with
+    their positions, for workloads with an append) in; attention outputs out."""
     B, H = wl.batch, wl.heads
     n_idx = len(wl.index_layers)
     h2d = n_idx * B * (32 * 128 * 4 + 32 * 4) + len(wl.modes) * B * H * 512 * 2
+    if wl.append:
+        h2d += B * (512 + 128 + 1) * 4
     d2h = len(wl.modes) * B * H * 512 * 2
     return h2d, d2h
 
@@ -102,23 +117,23 @@ def measured_peak_hbm():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def scan_kernel_hash():
+def scan_kernel_hash(fp4=False):
     h = hashlib.sha256()
-    for name in ("k_index.cu", "index_common.cuh", "common.cuh"):
+    for name in (("k_index_fp4.cu", "fp4.cuh", "common.cuh") if fp4 else ("k_index.cu", "index_common.cuh", "common.cuh")):
         with open(os.path.join(ROOT, "kv_cache_decode_index_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
 
 
-def scan_traffic_per_launch(workload_name):
+def scan_traffic_per_launch(workload_name, fp4=False):
     """DRAM bytes per Full-scan launch from the committed ncu summary, or None
     when the summary is missing or was taken on a different kernel source."""
-    path = os.path.join(ROOT, "profiles", "index_full_traffic.txt")
+    path = os.path.join(ROOT, "profiles", "index_full_fp4_traffic.txt" if fp4 else "index_full_traffic.txt")
     try:
         fields = dict(line.split(":", 1) for line in open(path).read().splitlines() if ":" in line)
     except OSError:
         return None
-    if fields.get("kernel_source_hash", "").strip() != scan_kernel_hash():
+    if fields.get("kernel_source_hash", "").strip() != scan_kernel_hash(fp4):
         return None
     if fields.get("workload", "").strip() != workload_name:
         return None
@@ -283,7 +298,8 @@ def run_b200(args):
 
     wl = rank_workload(selected_workload(args), rank)
     t0 = time.time()
-    cache = build_cache(wl, csa2)
+    fp4 = args.indexer == "fp4"
+    cache = build_cache(wl, csa2, fp4_indexer=fp4, append_last=wl.append)
     log(rank, f"cache filled in {time.time() - t0:.1f}s ({cache.kv_codes.numel() * 417 / 256 / 1e9:.2f} GB)")
 
     q_idx, w_idx, q_main = [], [], []
@@ -297,23 +313,29 @@ def run_b200(args):
             w_idx.append(torch.from_numpy(w).to(dev))
         q_main.append(W.main_query(wl, layer).to(dev))
     out = [torch.empty_like(m) for m in q_main]
-    group = csa2.DecodeGroup(cache, wl.modes, wl.heads, wl.topk, wl.pool_blocks, wl.scale)
+    group = csa2.DecodeGroup(cache, wl.modes, wl.heads, wl.topk, wl.pool_blocks, wl.scale,
+                             ik4=cache.ik4 if fp4 else None)
+    # workloads with an append: every step first appends each request's newest
+    # row (its last position, left out of the filled cache) through the
+    # quantise-on-append kernel
+    append = append_rows(wl, dev) if wl.append else None
 
     # ---- warm-up (eager), then capture one step as a graph ----
     for _ in range(args.warmup):
-        group.step(q_idx, w_idx, q_main, out)
+        group.step(q_idx, w_idx, q_main, out, append=append)
     torch.cuda.synchronize()
     # The timed graph has no events between launches (an event between two
     # kernels would cut their programmatic-dependent-launch link); a second
     # graph with events around every launch gives the per-launch durations.
     graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph):
-        group.step(q_idx, w_idx, q_main, out)
+        group.step(q_idx, w_idx, q_main, out, append=append)
     timing = {name: (torch.cuda.Event(enable_timing=True, external=True),
-                     torch.cuda.Event(enable_timing=True, external=True)) for name in group.launch_names()}
+                     torch.cuda.Event(enable_timing=True, external=True))
+              for name in group.launch_names(append is not None)}
     tgraph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(tgraph):
-        group.step(q_idx, w_idx, q_main, out, timing=timing)
+        group.step(q_idx, w_idx, q_main, out, timing=timing, append=append)
     graph.replay()
     tgraph.replay()
     torch.cuda.synchronize()
@@ -359,7 +381,7 @@ def run_b200(args):
     h2d, d2h = io_bytes(wl)
     e2e_value = e2e_serial = None
     if not args.no_e2e:
-        piped_ms, serial_ms = e2e_step_ms(args, group, q_idx, w_idx, q_main, out, dev, world)
+        piped_ms, serial_ms = e2e_step_ms(args, group, q_idx, w_idx, q_main, out, dev, world, append)
         e2e_value = world * wl.batch / (max_over_ranks(piped_ms, dev, world) / 1e3)
         e2e_serial = world * wl.batch / (max_over_ranks(serial_ms, dev, world) / 1e3)
 
@@ -367,14 +389,17 @@ def run_b200(args):
     if st != csa2.OK:
         raise RuntimeError(f"device error during the timed run: {word}")
 
-    step_bytes, scan_bytes = alg_bytes(wl)
+    step_bytes, scan_bytes = alg_bytes(wl, ik_row_bytes=IK4_ROW_BYTES if fp4 else IK_ROW_BYTES)
     scan_avg_ms = statistics.mean(scan_ms)
     peak, peak_src = measured_peak_hbm()
     achieved = scan_bytes / (scan_avg_ms / 1e3) / 1e9
-    traffic = scan_traffic_per_launch(wl.name)
+    traffic = scan_traffic_per_launch(wl.name, fp4)
     if rank == 0:
         value = world * wl.batch / (ms / 1e3)
         line = base_line(args, wl, world, value, ms)
+        if fp4:
+            line["dtype"] = "fp4"
+            line["config"]["indexer"] = "FP4 (E2M1 + E4M3 per 16) indexer K and Q, 72 B/position"
         step_gbs = step_bytes / (ms / 1e3) / 1e9
         line.update({
             "alg_bytes_per_step": step_bytes,
@@ -382,7 +407,9 @@ def run_b200(args):
             "step_frac_of_8tbs": step_gbs / NOMINAL_HBM_GBS,
             "step_frac_of_measured": step_gbs / peak,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-                         "traffic": traffic, "kernel": "csa2 index_full (Full indexer scan)",
+                         "traffic": traffic,
+                         "kernel": "csa2 index_full_fp4 (Full indexer scan, FP4 indexer K, 72 B/position)" if fp4
+                         else "csa2 index_full (Full indexer scan)",
                          "kernel_ms": scan_avg_ms, "alg_bytes_per_launch": scan_bytes,
                          "peak_source": f"{peak_src} copy bandwidth (MEASURED_PEAKS.json hbm_gbs, burst)"},
             "e2e": {"value": e2e_value, "unit": "queries/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
@@ -391,12 +418,12 @@ def run_b200(args):
                            "buffer slots and one copy stream per direction overlap step i+1's upload and step i-1's "
                            "download with step i",
                     "serial_value": e2e_serial},
-            "gpu_launches": group.launches_per_step * args.steps,
+            "gpu_launches": (group.launches_per_step + (0 if append is None else (2 if fp4 else 1))) * args.steps,
             "launch_ms": {name: statistics.mean(v) for name, v in per_launch.items()},
             "clocks": clocks,
         })
         if world == 1 and not args.no_cpu_baseline:
-            line["cpu_baseline"] = cpu_baseline_entry(wl)
+            line["cpu_baseline"] = cpu_baseline_entry(wl, fp4)
         print(json.dumps(line), flush=True)
     del graph, tgraph
     if world > 1:
@@ -549,7 +576,7 @@ def run_prefill(args):
     print(json.dumps(line), flush=True)
 
 
-def e2e_step_ms(args, group, q_idx, w_idx, q_main, out, dev, world):
+def e2e_step_ms(args, group, q_idx, w_idx, q_main, out, dev, world, append=None):
     """Milliseconds per step end to end through DecodeGroup.step with host
     buffers.  Every step copies all of its inputs from pinned host memory
     (packed: one host-to-device copy) and all of its outputs back (one
@@ -558,7 +585,8 @@ def e2e_step_ms(args, group, q_idx, w_idx, q_main, out, dev, world):
     direction let step i+1's upload and step i-1's download overlap step i."""
     import torch
     import torch.distributed as dist
-    ins = [t for t in q_idx + w_idx + q_main if t is not None]
+    app = list(append) if append is not None else []
+    ins = [t for t in q_idx + w_idx + q_main if t is not None] + app
     nbytes = lambda t: t.numel() * t.element_size()
     in_bytes, out_bytes = sum(nbytes(t) for t in ins), sum(nbytes(t) for t in out)
     h_in = torch.empty(in_bytes, dtype=torch.uint8, pin_memory=True)
@@ -583,13 +611,14 @@ def e2e_step_ms(args, group, q_idx, w_idx, q_main, out, dev, world):
         sq = [None if t is None else next(it_in) for t in q_idx]
         sw = [None if t is None else next(it_in) for t in w_idx]
         sm = [next(it_in) for _ in q_main]
+        sa = tuple(next(it_in) for _ in app) if app else None
         so = carve(d_out, out)
         d_in.copy_(h_in)
-        group.step(sq, sw, sm, so)
+        group.step(sq, sw, sm, so, append=sa)
         torch.cuda.synchronize()
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g):
-            group.step(sq, sw, sm, so)
+            group.step(sq, sw, sm, so, append=sa)
         slots.append((d_in, d_out, g))
     comp = torch.cuda.current_stream(dev)
     up, down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
@@ -653,7 +682,47 @@ def max_over_ranks(x: float, dev, world: int) -> float:
     return float(t.item())
 
 
-def cpu_baseline_entry(wl):
+def oracle_sample_fp4(wl, b: int = 0):
+    """Time the float64 oracle of the FP4 indexer variant on one query: FP4
+    scores of every position, pool, Full/Reindex/Reuse Top-k, six attention
+    layers (main-KV rows prepared for the gathered positions only)."""
+    from oracle import csa2 as C
+    from oracle import formats as F
+    n = int(W.ctx_lengths(wl)[b])
+    codes, scales = F.quantize_indexer_fp4(W.request_rows(wl, b, n, "ik"))
+    qw = [None if m == "Ru" else (W.index_query(wl, l)[0][b], W.index_query(wl, l)[1][b])
+          for l, m in enumerate(wl.modes)]
+    q_main = [W.main_query(wl, l)[b].float().numpy() for l in range(len(wl.modes))]
+    t0 = time.perf_counter()
+    s = C.indexer_scores_fp4(qw[0][0], qw[0][1], codes, scales)
+    pool = C.pool_select(C.block_max(s, n), wl.pool_blocks)
+    cand = C.pool_positions(pool, n)
+    topk, cur = [], None
+    for l, m in enumerate(wl.modes):
+        if m == "F":
+            cur = C.top_k_ascending(cand, s[cand], wl.topk)
+        elif m == "Ri":
+            cur = C.top_k_ascending(cand, C.indexer_scores_fp4(qw[l][0], qw[l][1], codes[cand], scales[cand]),
+                                    wl.topk)
+        topk.append(cur)
+    t_sel = time.perf_counter() - t0
+    sel = np.unique(np.concatenate([t[t >= 0] for t in topk]))
+    kvc = np.zeros((n, 256), np.uint8)
+    kvs = np.zeros((n, 32), np.uint8)
+    kvc[sel], kvs[sel] = F.quantize_main_kv(W.rows_at(wl, b, sel, "kv"))
+    t1 = time.perf_counter()
+    for layer in range(len(wl.modes)):
+        C.sparse_attention(q_main[layer], kvc, kvs, topk[layer], wl.scale)
+    return t_sel + time.perf_counter() - t1
+
+
+def cpu_baseline_entry(wl, fp4=False):
+    if fp4:
+        secs = oracle_sample_fp4(wl, 0)
+        return {"value": 1.0 / secs, "unit": "queries/s", "cores": cpu_cores(), **cpu_host(), "kind": "oracle",
+                "sample": f"1 of the {wl.batch} queries of one step (request 0, full "
+                          f"{int(W.ctx_lengths(wl)[0]):,}-position context): float64 numpy oracle of the FP4 "
+                          f"indexer variant, whole layer-group step, {secs:.1f} s"}
     secs, _ = oracle_sample(wl, 0)
     return {"value": 1.0 / secs, "unit": "queries/s", "cores": cpu_cores(), **cpu_host(), "kind": "oracle",
             "sample": f"1 of the {wl.batch} queries of one step (request 0, full {int(W.ctx_lengths(wl)[0]):,}-position "
@@ -748,6 +817,8 @@ def main(argv=None):
                    help="override the number of prefill queries (profiling cases)")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--indexer", choices=["fp8", "fp4"], default="fp8",
+                   help="indexer K format of the decode workloads (fp4: the FP4 indexer variant)")
     args = p.parse_args(argv)
     if args.warmup < 3:
         p.error("--warmup must be >= 3")

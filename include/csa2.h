@@ -263,6 +263,56 @@ CSA2_API csa2_status csa2_pool_merge(int32_t n_shards, int32_t batch, int32_t po
                                      const int32_t* ids, int32_t* pool, void* stream);
 
 /*
+ * FP4 indexer variant [animattoys article, section 把精度降到4比特: V4 kept
+ * the indexer's Q and K in FP4].  Reading (the pages give no format): the
+ * main-KV format on the indexer's 128-element row, E2M1 codes with one E4M3
+ * scale per 16 elements, s = E4M3(amax / 6) (nearest, ties to even,
+ * saturating), no row scale, for the cached keys and for each query head; the
+ * score is s_t = sum_h w_h * ReLU(<q~_h, k~_t>) over the dequantised values.
+ * 72 bytes per position instead of the FP8 indexer's 129.  The keys live next
+ * to the cache (same rows, same page table):
+ *   codes   uint8 [num_pages * page_size][64]: element 2i in the low nibble
+ *           of byte i, element 2i + 1 in the high nibble
+ *   scales  uint8 [num_pages * page_size / 128][1024]: the scales of each
+ *           128-row tile (rows r .. r + 127 with r a multiple of 128), the
+ *           scale of tile row m and element group g (elements 16g .. 16g+15)
+ *           at byte  (g / 4) * 512 + (m % 32) * 16 + (m / 32) * 4 + g % 4,
+ *           the order in which the tensor cores read block scales
+ * Both 16-byte aligned, caller-owned.
+ */
+#define CSA2_IK4_CODE_BYTES 64
+#define CSA2_IK4_TILE_SCALE_BYTES 1024
+typedef struct csa2_ik4 {
+  uint8_t* codes;
+  uint8_t* scales;
+} csa2_ik4;
+
+/*
+ * csa2_append_ik4 -- quantise n_rows indexer keys (float [n_rows][128]) to
+ * the FP4 indexer format and store them at (req[i], pos[i]) (req NULL: row i
+ * -> request i).  Device errors as csa2_append_kv.
+ *
+ * csa2_index_full_fp4 -- csa2_index_full over the FP4 indexer keys: q float
+ * [batch][32][128] is quantised per head to the same format inside; w, blockmax,
+ * scores and hist as csa2_index_full.  The contraction runs on the tensor
+ * cores as block-scaled FP4 (tcgen05 kind::mxf4nvf4, E4M3 scales per 16
+ * elements), fp32 accumulation.
+ *
+ * csa2_reindex_layers_fp4 -- csa2_reindex_layers over the FP4 indexer keys
+ * (every layer's query quantised per head to FP4); n_layers in [1, 4], other
+ * arguments and the workspace as csa2_reindex_layers.
+ */
+CSA2_API csa2_status csa2_append_ik4(const csa2_cache* cache, const csa2_ik4* ik4, int32_t n_rows,
+                                     const float* ik_new, const int32_t* req, const int32_t* pos, void* stream);
+CSA2_API csa2_status csa2_index_full_fp4(const csa2_cache* cache, const csa2_ik4* ik4, const float* q,
+                                         const float* w, float* blockmax, float* scores, uint32_t* hist,
+                                         void* stream);
+CSA2_API csa2_status csa2_reindex_layers_fp4(const csa2_cache* cache, const csa2_ik4* ik4, int32_t n_layers,
+                                             const int32_t* pool, int32_t pool_blocks, const float* const* q,
+                                             const float* const* w, int32_t k, int32_t* const* topk,
+                                             void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * csa2_reindex -- Top-k of one layer of the group, by mode:
  *   CSA2_FULL    the k best positions of this layer's own Full scan among the
  *                candidates.  Scores come from full_scores when it is not NULL,

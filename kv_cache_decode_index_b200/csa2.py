@@ -25,6 +25,7 @@ OK, ERR_ARG, ERR_SHAPE, ERR_CUDA, ERR_DEVICE_BOUNDS, ERR_TIMEOUT, ERR_UNSUPPORTE
 BLOCK, INDEX_HEADS, INDEX_DIM, KV_DIM, KV_CODE_BYTES, KV_SCALE_BYTES = 8, 32, 128, 512, 256, 32
 PREFILL_MAX_K, PREFILL_CANDIDATES, PREFILL_STATIC_MAX_QUERIES = 1024, 4096, 256
 POOL_HIST_BINS, RESCORE_HIST_BINS, MAX_SCORE_LAYERS = 2048, 4096, 8
+IK4_CODE_BYTES, IK4_TILE_SCALE_BYTES, MAX_FP4_SCORE_LAYERS = 64, 1024, 4
 
 
 class CacheStruct(ctypes.Structure):
@@ -34,9 +35,14 @@ class CacheStruct(ctypes.Structure):
                 ("max_pages_per_req", ctypes.c_int32), ("batch", ctypes.c_int32), ("err_word", ctypes.c_void_p)]
 
 
+class Ik4Struct(ctypes.Structure):
+    _fields_ = [("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p)]
+
+
 _P = ctypes.c_void_p
 _I = ctypes.c_int32
 _CP = ctypes.POINTER(CacheStruct)
+_KP = ctypes.POINTER(Ik4Struct)
 _sig = {
     "csa2_append_kv": [_CP, _I, _P, _P, _P, _P, _P],
     "csa2_compress_append": [_CP, _I, _I, _P, _P, _P, _P, _P],
@@ -45,6 +51,9 @@ _sig = {
     "csa2_reindex": [_CP, _I, _P, _I, _P, _P, _P, _P, _I, _P, _P],
     "csa2_reindex_layers": [_CP, _I, _P, _I, _P, _P, _I, _P, _P, ctypes.c_size_t, _P],
     "csa2_pool_candidates": [_CP, _P, _P, _I, _I, _P, _P, _P],
+    "csa2_append_ik4": [_CP, _KP, _I, _P, _P, _P, _P],
+    "csa2_index_full_fp4": [_CP, _KP, _P, _P, _P, _P, _P, _P],
+    "csa2_reindex_layers_fp4": [_CP, _KP, _I, _P, _I, _P, _P, _I, _P, _P, ctypes.c_size_t, _P],
     "csa2_pool_merge": [_I, _I, _I, _P, _P, _P, _P],
     "csa2_sparse_attn": [_CP, _I, _P, _P, _I, _P, _I, ctypes.c_float, _P, _P],
     "csa2_sparse_attn_layers": [_CP, _I, _I, _P, _P, _I, _P, _I, ctypes.c_float, _P, _P, ctypes.c_size_t, _P],
@@ -143,6 +152,60 @@ class Cache:
         return pt[positions // self.page_size].to(torch.int64) * self.page_size + positions % self.page_size
 
 
+class Ik4:
+    """FP4 indexer keys of a cache (same rows and page table as `cache`):
+    codes uint8 [rows, 64] (element 2i in the low nibble of byte i) and the
+    block scales uint8 [rows / 128, 1024] of every 128-row tile in the
+    tensor-core order (ik4_scale_offset)."""
+
+    def __init__(self, cache: Cache):
+        rows = cache.num_pages * cache.page_size
+        self.codes = torch.zeros(rows, IK4_CODE_BYTES, dtype=torch.uint8, device=cache.device)
+        self.scales = torch.zeros(rows // 128, IK4_TILE_SCALE_BYTES, dtype=torch.uint8, device=cache.device)
+        self._struct = None
+
+    @property
+    def struct(self) -> Ik4Struct:
+        s = Ik4Struct(self.codes.data_ptr(), self.scales.data_ptr())
+        self._struct = s
+        return s
+
+
+def ik4_scale_offset(m, g):
+    """Byte of the scale of tile row m (0..127), element group g (0..7) inside
+    a tile's 1 KB scale block (host helper)."""
+    return (g // 4) * 512 + (m % 32) * 16 + (m // 32) * 4 + g % 4
+
+
+def append_ik4(cache: Cache, ik4: Ik4, ik_new, pos, req=None):
+    """Quantise indexer keys ik_new float32 [n, 128] to the FP4 indexer format."""
+    n = ik_new.shape[0]
+    _need(ik_new, torch.float32, (n, INDEX_DIM), "ik_new")
+    _need(pos, torch.int32, (n,), "pos")
+    if req is not None:
+        _need(req, torch.int32, (n,), "req")
+    _check(_lib.csa2_append_ik4(ctypes.byref(cache.struct), ctypes.byref(ik4.struct), n, _ptr(ik_new), _ptr(req),
+                                _ptr(pos), _stream(cache.device)), "csa2_append_ik4")
+
+
+def index_full_fp4(cache: Cache, ik4: Ik4, q, w, blockmax=None, scores=None, hist=None):
+    """Full scan over the FP4 indexer keys (as index_full)."""
+    B = cache.batch
+    _need(q, torch.float32, (B, INDEX_HEADS, INDEX_DIM), "q")
+    _need(w, torch.float32, (B, INDEX_HEADS), "w")
+    if blockmax is None:
+        blockmax = torch.empty(B, cache.capacity // BLOCK, dtype=torch.float32, device=cache.device)
+    _need(blockmax, torch.float32, (B, cache.capacity // BLOCK), "blockmax")
+    if scores is not None:
+        _need(scores, torch.float32, (B, cache.capacity), "scores")
+    if hist is not None:
+        _need(hist, torch.int32, (B, POOL_HIST_BINS), "hist")
+    _check(_lib.csa2_index_full_fp4(ctypes.byref(cache.struct), ctypes.byref(ik4.struct), _ptr(q), _ptr(w),
+                                    _ptr(blockmax), _ptr(scores), _ptr(hist), _stream(cache.device)),
+           "csa2_index_full_fp4")
+    return blockmax
+
+
 def append_kv(cache: Cache, kv_new, ik_new, pos, req=None):
     n = kv_new.shape[0]
     _need(kv_new, torch.float32, (n, KV_DIM), "kv_new")
@@ -210,9 +273,11 @@ def reindex_layers_workspace_bytes(batch: int, n_layers: int, pool_blocks: int) 
     return int(_lib.csa2_reindex_layers_workspace_bytes(int(batch), int(n_layers), int(pool_blocks)))
 
 
-def reindex_layers(cache: Cache, pool, q_layers, w_layers, k: int = 512, topk_layers=None, workspace=None):
+def reindex_layers(cache: Cache, pool, q_layers, w_layers, k: int = 512, topk_layers=None, workspace=None,
+                   ik4: Ik4 | None = None):
     """Top-k over the pool of several Full / Reindex layers in one pass
-    (csa2_reindex_layers); returns the list of int32 [batch, k] Top-k.
+    (csa2_reindex_layers, or csa2_reindex_layers_fp4 over the FP4 indexer keys
+    `ik4`); returns the list of int32 [batch, k] Top-k.
     workspace: a zeroed uint8 device tensor of reindex_layers_workspace_bytes
     bytes, kept between calls (allocated and zeroed here when None)."""
     B, P = pool.shape
@@ -233,9 +298,14 @@ def reindex_layers(cache: Cache, pool, q_layers, w_layers, k: int = 512, topk_la
     qa = (ctypes.c_void_p * L)(*[q.data_ptr() for q in q_layers])
     wa = (ctypes.c_void_p * L)(*[w.data_ptr() for w in w_layers])
     ta = (ctypes.c_void_p * L)(*[t.data_ptr() for t in topk_layers])
-    _check(_lib.csa2_reindex_layers(ctypes.byref(cache.struct), L, _ptr(pool), P, qa, wa, int(k), ta,
-                                    _ptr(workspace), workspace.numel(), _stream(cache.device)),
-           "csa2_reindex_layers")
+    if ik4 is None:
+        _check(_lib.csa2_reindex_layers(ctypes.byref(cache.struct), L, _ptr(pool), P, qa, wa, int(k), ta,
+                                        _ptr(workspace), workspace.numel(), _stream(cache.device)),
+               "csa2_reindex_layers")
+    else:
+        _check(_lib.csa2_reindex_layers_fp4(ctypes.byref(cache.struct), ctypes.byref(ik4.struct), L, _ptr(pool), P,
+                                            qa, wa, int(k), ta, _ptr(workspace), workspace.numel(),
+                                            _stream(cache.device)), "csa2_reindex_layers_fp4")
     return topk_layers
 
 
@@ -445,9 +515,12 @@ class DecodeGroup:
     """
 
     def __init__(self, cache: Cache, modes, heads: int, k: int = 512, pool_blocks: int | None = 2048,
-                 scale: float | None = None):
+                 scale: float | None = None, ik4: Ik4 | None = None):
         if modes[0] != "F":
             raise ValueError("a layer group starts with a Full layer")
+        if ik4 is not None and not pool_blocks:
+            raise ValueError("the FP4 indexer path needs a pool")
+        self.ik4 = ik4
         self.cache, self.modes, self.heads, self.k = cache, tuple(modes), heads, k
         self.pool_blocks = pool_blocks
         self.scale = 1.0 / math.sqrt(KV_DIM) if scale is None else scale
@@ -468,18 +541,30 @@ class DecodeGroup:
         if pool_blocks:
             self.rs_ws = torch.zeros(reindex_layers_workspace_bytes(B, len(self.index_layers), pool_blocks),
                                      dtype=torch.uint8, device=dev)
+            # one workspace part per Top-k launch pair
+            step = MAX_FP4_SCORE_LAYERS if ik4 is not None else len(self.index_layers)
+            n_parts = -(-len(self.index_layers) // step)
+            self.rs_ws_parts, off = [], 0
+            for i in range(n_parts):
+                nl = min(step, len(self.index_layers) - i * step)
+                nb = reindex_layers_workspace_bytes(B, nl, pool_blocks)
+                self.rs_ws_parts.append(self.rs_ws[off:off + nb])
+                off += nb
         self.attn_ws = torch.empty(attn_workspace_bytes(len(self.modes), B, heads), dtype=torch.uint8, device=dev)
         # kernels per step: scan, pool, score + select, attention (with a
         # pool); scan, one Top-k per index layer, attention (without)
-        self.launches_per_step = 5 if pool_blocks else 2 + len(self.index_layers)
+        self.launches_per_step = (3 + 2 * len(self.rs_ws_parts)) if pool_blocks else 2 + len(self.index_layers)
 
-    def step(self, q_idx, w_idx, q_main, out, timing=None):
+    def step(self, q_idx, w_idx, q_main, out, timing=None, append=None):
         """q_idx / w_idx: per layer ([B,32,128] / [B,32], None for Reuse);
-        q_main / out: per layer bf16 [B, H, 512].  timing: optional dict
-        name -> (start, end) CUDA events, recorded on the calling stream
-        around the launches of that name ("scan", "pool", "topk", "attn"; an
-        event between two launches cuts their programmatic link, so time a
-        separate graph with it)."""
+        q_main / out: per layer bf16 [B, H, 512].  append: optional (kv_new
+        [B,512], ik_new [B,128], pos [B]) float32 / int32 rows that each
+        request appends (quantise-on-append) before the scan, one per request
+        (ctx_len already counts them).  timing: optional dict name -> (start,
+        end) CUDA events, recorded on the calling stream around the launches of
+        that name ("append", "scan", "pool", "topk", "attn"; an event between
+        two launches cuts their programmatic link, so time a separate graph
+        with it)."""
         c = self.cache
 
         def timed(name, fn):
@@ -495,12 +580,22 @@ class DecodeGroup:
                 ev[1].record()
             return r
 
-        timed("scan", lambda: index_full(c, q_idx[0], w_idx[0], self.blockmax, hist=self.hist))
+        if append is not None:
+            kv_new, ik_new, pos = append
+
+            def do_append():
+                append_kv(c, kv_new, ik_new, pos)
+                if self.ik4 is not None:
+                    append_ik4(c, self.ik4, ik_new, pos)
+            timed("append", do_append)
+        if self.ik4 is None:
+            timed("scan", lambda: index_full(c, q_idx[0], w_idx[0], self.blockmax, hist=self.hist))
+        else:
+            timed("scan", lambda: index_full_fp4(c, self.ik4, q_idx[0], w_idx[0], self.blockmax, hist=self.hist))
         if self.pool is not None:
             timed("pool", lambda: pool_select(c, self.blockmax, self.pool_blocks, self.pool, hist=self.hist))
             L = self.index_layers
-            timed("topk", lambda: reindex_layers(c, self.pool, [q_idx[l] for l in L], [w_idx[l] for l in L],
-                                                 self.k, [self.topk[l] for l in L], self.rs_ws))
+            timed("topk", lambda: self._pool_topk(q_idx, w_idx))
         else:
             def flat():
                 for l in self.index_layers:
@@ -510,8 +605,19 @@ class DecodeGroup:
         timed("attn", lambda: sparse_attn_layers(c, self.topk, q_main, self.scale, out, workspace=self.attn_ws))
         return out
 
-    def launch_names(self):
-        return ["scan"] + (["pool"] if self.pool is not None else []) + ["topk", "attn"]
+    def _pool_topk(self, q_idx, w_idx):
+        """Top-k of every index layer over the pool; the FP4 path scores at
+        most four layers per launch pair (one block of query scales)."""
+        L = self.index_layers
+        step = MAX_FP4_SCORE_LAYERS if self.ik4 is not None else len(L)
+        for i, ws in zip(range(0, len(L), step), self.rs_ws_parts):
+            part = L[i:i + step]
+            reindex_layers(self.cache, self.pool, [q_idx[l] for l in part], [w_idx[l] for l in part], self.k,
+                           [self.topk[l] for l in part], ws, ik4=self.ik4)
+
+    def launch_names(self, append: bool = False):
+        return (["append"] if append else []) + ["scan"] + (["pool"] if self.pool is not None else []) + \
+            ["topk", "attn"]
 
 
 class PrefillGroup:

@@ -42,6 +42,7 @@ struct SelectSmem {
   int done;
   int hi;                    // top bit of the next digit
   int total;                 // valid candidates in the cluster
+  int fin[3];                // this CTA's output base, ties taken, cluster total
 };
 
 // Head start of a select: the threshold's leading bits (prefix under mask),
@@ -264,23 +265,32 @@ __device__ void cluster_topk(const uint32_t* keys, int n_local, int K, SelectSme
     S.gt_eq[1] = local_eq;
   }
   cluster.sync();   // counts visible cluster-wide
-  int rg[kMaxCluster], re[kMaxCluster];   // remote reads issued together
+  // one warp reads the C ranks' counts (lane r: rank r) and derives this
+  // CTA's output base, its share of the ties and the total selected
+  if (warp == 0) {
+    const int g = lane < C ? cluster.map_shared_rank(&S.gt_eq[0], lane)[0] : 0;
+    const int e = lane < C ? cluster.map_shared_rank(&S.gt_eq[0], lane)[1] : 0;
+    int ties_incl = e;   // inclusive prefix of the tie counts over the ranks
 #pragma unroll
-  for (int r = 0; r < kMaxCluster; ++r) {
-    rg[r] = r < C ? cluster.map_shared_rank(&S.gt_eq[0], r)[0] : 0;
-    re[r] = r < C ? cluster.map_shared_rank(&S.gt_eq[0], r)[1] : 0;
-  }
-  int out_base = 0, take_local = 0, sel_total = 0, ties_before = 0;
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, ties_incl, o);
+      if (lane >= o) ties_incl += y;
+    }
+    const int take = max(0, min(need - (ties_incl - e), e));
+    int sel_incl = g + take;
 #pragma unroll
-  for (int r = 0; r < kMaxCluster; ++r) {
-    if (r >= C) break;
-    const int g = rg[r], e = re[r];
-    const int take = max(0, min(need - ties_before, e));
-    if (r < rank) out_base += g + take;
-    if (r == rank) take_local = take;
-    sel_total += g + take;
-    ties_before += e;
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, sel_incl, o);
+      if (lane >= o) sel_incl += y;
+    }
+    if (lane == rank) {
+      S.fin[0] = sel_incl - (g + take);   // selections of the lower ranks
+      S.fin[1] = take;
+    }
+    if (lane == 31) S.fin[2] = sel_incl;
   }
+  __syncthreads();
+  const int out_base = S.fin[0], take_local = S.fin[1], sel_total = S.fin[2];
   // ties taken by this warp, and the output rank of its first selection
   const int eqb = __shfl_sync(0xffffffffu, eq_before_w, 0);
   const int gtb = __shfl_sync(0xffffffffu, gt_before_w, 0);

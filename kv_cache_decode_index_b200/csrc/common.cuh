@@ -288,6 +288,74 @@ __device__ __forceinline__ uint64_t sw128_kmajor_desc(uint32_t smem_addr) {
   return d;
 }
 
+// Shared-memory matrix descriptor of a K-major operand stored as rows of 64
+// bytes with the 64-byte swizzle (16-byte chunk c of row r lives at chunk
+// c ^ ((r / 2) % 4)); 8-row groups are 512 bytes apart.  The base must be
+// 512-byte aligned; a 32-byte step along K adds 2 to the start-address field.
+__device__ __forceinline__ uint64_t sw64_kmajor_desc(uint32_t smem_addr) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((smem_addr >> 4) & 0x3FFFu);   // start address
+  d |= static_cast<uint64_t>(1) << 16;                        // LBO (unused here)
+  d |= static_cast<uint64_t>(512 >> 4) << 32;                 // SBO: 8 rows x 64 B
+  d |= static_cast<uint64_t>(1) << 46;                        // descriptor version
+  d |= static_cast<uint64_t>(4) << 61;                        // 64-byte swizzle
+  return d;
+}
+// Byte offset of (row, byte c) in a 64-byte-swizzled tile of 64-byte rows.
+__host__ __device__ __forceinline__ uint32_t sw64_offset(uint32_t row, uint32_t c) {
+  return row * 64u + ((((c >> 4) ^ (row >> 1)) & 3u) << 4) + (c & 15u);
+}
+// Descriptor of 32 rows x 16 bytes stored contiguously (the block-scale
+// layout below) for tcgen05.cp: 8-row core matrices 128 bytes apart.
+__device__ __forceinline__ uint64_t scale_rows_desc(uint32_t smem_addr) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((smem_addr >> 4) & 0x3FFFu);
+  d |= static_cast<uint64_t>(1) << 16;
+  d |= static_cast<uint64_t>(128 >> 4) << 32;
+  d |= static_cast<uint64_t>(1) << 46;
+  return d;
+}
+
+// Block scales of FP4 operands, in the order the tensor core reads them.  For
+// a tile of 128 rows and 8 groups of 16 elements (K = 128) they take 1 KB:
+// byte (g / 4) * 512 + (m % 32) * 16 + (m / 32) * 4 + g % 4 holds the scale of
+// row m, group g.  Each 512-byte half (one K = 64 MMA) is 32 lines of 16 bytes,
+// copied to tensor memory by one tcgen05.cp 32x128b.warpx4 (lines to lanes
+// 0..31, replicated in the four lane quarters); the MMA then reads the scales
+// of row m from lane m, column m / 32 of the copy.  An operand of N <= 128 rows
+// (the query heads) uses the same layout.
+__host__ __device__ constexpr uint32_t block_scale_offset(uint32_t m, uint32_t g) {
+  return (g >> 2) * 512u + (m & 31u) * 16u + (m >> 5) * 4u + (g & 3u);
+}
+
+// tcgen05.cp of 32 lines x 16 bytes from shared memory to tensor memory
+// columns taddr .. taddr + 3 of all four lane quarters.
+__device__ __forceinline__ void tmem_cp_scales(uint32_t taddr, uint32_t smem_addr) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(scale_rows_desc(smem_addr))
+               : "memory");
+}
+
+// D[tmem] (+)= (A * scale_A) x (B * scale_B)^T for FP4 (E2M1) operands with
+// one E4M3 scale per 16 elements along K (K = 64 per instruction), fp32 D.
+__device__ __forceinline__ void umma_mxf4nvf4(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                              uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
+
+// Instruction descriptor of kind::mxf4nvf4: A = B = E2M1, E4M3 block scales,
+// fp32 D, both K-major, shape M x N, K = 64.
+__host__ __device__ constexpr uint32_t idesc_mxf4nvf4(int M, int N) {
+  return (1u << 7) | (1u << 10)                       // A, B: E2M1
+         | (static_cast<uint32_t>(N >> 3) << 17)      // N / 8
+         | (0u << 23)                                 // scales: E4M3
+         | (static_cast<uint32_t>(M >> 4) << 24);     // M / 16
+}
+
 // Instruction descriptor of kind::f8f6f4: A = B = E4M3, D = fp32, both
 // K-major, shape M x N.
 __host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N) {

@@ -70,7 +70,18 @@ using EncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, voi
                               const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
                               CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
+csa2_status encode_rows_map(void* base, long long rows, int row_bytes, int box_rows, CUtensorMapSwizzle swizzle,
+                            CUtensorMap* map);
+
 csa2_status encode_ik_map(const csa2_cache* c, int box_rows, CUtensorMap* map) {
+  return encode_rows_map(c->ik_codes, static_cast<long long>(c->num_pages) * c->page_size, csa2::kIndexDim, box_rows,
+                         CU_TENSOR_MAP_SWIZZLE_128B, map);
+}
+
+// 2-D map over `rows` rows of `row_bytes` bytes (uint8), box of box_rows
+// full rows.
+csa2_status encode_rows_map(void* base, long long rows, int row_bytes, int box_rows, CUtensorMapSwizzle swizzle,
+                            CUtensorMap* map) {
   static EncodeFn fn = nullptr;
   static std::once_flag once;
   std::call_once(once, [] {
@@ -81,15 +92,21 @@ csa2_status encode_ik_map(const csa2_cache* c, int box_rows, CUtensorMap* map) {
       fn = reinterpret_cast<EncodeFn>(p);
   });
   if (fn == nullptr) return fail(CSA2_ERR_UNSUPPORTED, "cuTensorMapEncodeTiled is not available");
-  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(csa2::kIndexDim),
-                              static_cast<cuuint64_t>(c->num_pages) * static_cast<cuuint64_t>(c->page_size)};
-  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(csa2::kIndexDim)};
-  const cuuint32_t box[2] = {static_cast<cuuint32_t>(csa2::kIndexDim), static_cast<cuuint32_t>(box_rows)};
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(row_bytes), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(row_bytes)};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(row_bytes), static_cast<cuuint32_t>(box_rows)};
   const cuuint32_t estr[2] = {1, 1};
-  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, c->ik_codes, dims, strides, box, estr,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, base, dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(CSA2_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+  return CSA2_OK;
+}
+
+csa2_status check_ik4(const csa2_ik4* ik4) {
+  if (ik4 == nullptr || ik4->codes == nullptr || ik4->scales == nullptr || !aligned(ik4->codes, 16) ||
+      !aligned(ik4->scales, 16))
+    return fail(CSA2_ERR_ARG, "ik4, ik4.codes and ik4.scales must be set and 16-byte aligned");
   return CSA2_OK;
 }
 
@@ -208,6 +225,40 @@ csa2_status csa2_index_full(const csa2_cache* cache, const float* q, const float
   return e == cudaSuccess ? CSA2_OK : cuda_fail(e, "index_full launch");
 }
 
+csa2_status csa2_append_ik4(const csa2_cache* cache, const csa2_ik4* ik4, int32_t n_rows, const float* ik_new,
+                            const int32_t* req, const int32_t* pos, void* stream) {
+  CSA2_TRY(check_cache(cache, false, false));
+  CSA2_TRY(check_ik4(ik4));
+  if (n_rows < 0) return fail(CSA2_ERR_SHAPE, "n_rows %d < 0", n_rows);
+  if (n_rows == 0) return CSA2_OK;
+  if (ik_new == nullptr || pos == nullptr || !aligned(ik_new, 16))
+    return fail(CSA2_ERR_ARG, "ik_new (16-byte aligned) and pos must be set");
+  if (req == nullptr && n_rows > cache->batch)
+    return fail(CSA2_ERR_SHAPE, "without req, n_rows (%d) must not exceed batch (%d)", n_rows, cache->batch);
+  DeviceInfo d;
+  CSA2_TRY(device_info(&d));
+  const cudaError_t e = csa2::launch_append_ik4(*cache, ik4->codes, ik4->scales, n_rows, ik_new, req, pos,
+                                                static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? CSA2_OK : cuda_fail(e, "append_ik4 launch");
+}
+
+csa2_status csa2_index_full_fp4(const csa2_cache* cache, const csa2_ik4* ik4, const float* q, const float* w,
+                                float* blockmax, float* scores, uint32_t* hist, void* stream) {
+  CSA2_TRY(check_cache(cache, false, false));
+  CSA2_TRY(check_ik4(ik4));
+  if (q == nullptr || w == nullptr || blockmax == nullptr || !aligned(q, 16))
+    return fail(CSA2_ERR_ARG, "q (16-byte aligned), w and blockmax must be set");
+  if (hist != nullptr && !aligned(hist, 16)) return fail(CSA2_ERR_ARG, "hist must be 16-byte aligned");
+  DeviceInfo d;
+  CSA2_TRY(device_info(&d));
+  CUtensorMap map;
+  CSA2_TRY(encode_rows_map(ik4->codes, static_cast<long long>(cache->num_pages) * cache->page_size,
+                           CSA2_IK4_CODE_BYTES, csa2::kTile, CU_TENSOR_MAP_SWIZZLE_64B, &map));
+  const cudaError_t e = csa2::launch_index_full_fp4(*cache, ik4->scales, q, w, blockmax, scores, hist, map, d.sms,
+                                                    g_wait_limit_ns, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? CSA2_OK : cuda_fail(e, "index_full_fp4 launch");
+}
+
 csa2_status csa2_pool_select(const csa2_cache* cache, const float* blockmax, uint32_t* hist, int32_t pool_blocks,
                              int32_t* pool, void* stream) {
   CSA2_TRY(check_cache(cache, false, false));
@@ -277,12 +328,14 @@ size_t csa2_reindex_layers_workspace_bytes(int32_t batch, int32_t n_layers, int3
   return csa2::rescore_workspace_bytes(batch, n_layers, pool_blocks);
 }
 
-csa2_status csa2_reindex_layers(const csa2_cache* cache, int32_t n_layers, const int32_t* pool, int32_t pool_blocks,
-                                const float* const* q, const float* const* w, int32_t k, int32_t* const* topk,
-                                void* workspace, size_t workspace_bytes, void* stream) {
-  CSA2_TRY(check_cache(cache, false, true));
-  if (n_layers < 1 || n_layers > CSA2_MAX_SCORE_LAYERS)
-    return fail(CSA2_ERR_SHAPE, "n_layers %d outside [1, %d]", n_layers, CSA2_MAX_SCORE_LAYERS);
+static csa2_status reindex_layers_impl(const csa2_cache* cache, const csa2_ik4* ik4, int32_t n_layers, const int32_t* pool,
+                                int32_t pool_blocks, const float* const* q, const float* const* w, int32_t k,
+                                int32_t* const* topk, void* workspace, size_t workspace_bytes, void* stream) {
+  CSA2_TRY(check_cache(cache, false, ik4 == nullptr));
+  if (ik4 != nullptr) CSA2_TRY(check_ik4(ik4));
+  const int max_layers = ik4 != nullptr ? 4 : CSA2_MAX_SCORE_LAYERS;
+  if (n_layers < 1 || n_layers > max_layers)
+    return fail(CSA2_ERR_SHAPE, "n_layers %d outside [1, %d]", n_layers, max_layers);
   if (pool_blocks < 1 || pool_blocks > kMaxPool)
     return fail(CSA2_ERR_SHAPE, "pool_blocks %d outside [1, %d]", pool_blocks, kMaxPool);
   if (k < 1 || k > kMaxK) return fail(CSA2_ERR_SHAPE, "k %d outside [1, %d]", k, kMaxK);
@@ -300,10 +353,31 @@ csa2_status csa2_reindex_layers(const csa2_cache* cache, int32_t n_layers, const
   DeviceInfo d;
   CSA2_TRY(device_info(&d));
   CUtensorMap map;
-  CSA2_TRY(encode_ik_map(cache, csa2::kBlock, &map));
-  const cudaError_t e = csa2::launch_rescore_layers(*cache, n_layers, pool, pool_blocks, q, w, k, topk, workspace,
-                                                    map, d.sms, g_wait_limit_ns, static_cast<cudaStream_t>(stream));
+  if (ik4 != nullptr)
+    CSA2_TRY(encode_rows_map(ik4->codes, static_cast<long long>(cache->num_pages) * cache->page_size,
+                             CSA2_IK4_CODE_BYTES, csa2::kBlock, CU_TENSOR_MAP_SWIZZLE_64B, &map));
+  else
+    CSA2_TRY(encode_ik_map(cache, csa2::kBlock, &map));
+  const cudaError_t e =
+      csa2::launch_rescore_layers(*cache, ik4 != nullptr ? ik4->scales : nullptr, n_layers, pool, pool_blocks, q, w, k,
+                                  topk, workspace, map, d.sms, g_wait_limit_ns, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? CSA2_OK : cuda_fail(e, "reindex_layers launch");
+}
+
+csa2_status csa2_reindex_layers(const csa2_cache* cache, int32_t n_layers, const int32_t* pool, int32_t pool_blocks,
+                                const float* const* q, const float* const* w, int32_t k, int32_t* const* topk,
+                                void* workspace, size_t workspace_bytes, void* stream) {
+  return reindex_layers_impl(cache, nullptr, n_layers, pool, pool_blocks, q, w, k, topk, workspace, workspace_bytes,
+                             stream);
+}
+
+csa2_status csa2_reindex_layers_fp4(const csa2_cache* cache, const csa2_ik4* ik4, int32_t n_layers,
+                                    const int32_t* pool, int32_t pool_blocks, const float* const* q,
+                                    const float* const* w, int32_t k, int32_t* const* topk, void* workspace,
+                                    size_t workspace_bytes, void* stream) {
+  if (ik4 == nullptr) return fail(CSA2_ERR_ARG, "ik4 must be set");
+  return reindex_layers_impl(cache, ik4, n_layers, pool, pool_blocks, q, w, k, topk, workspace, workspace_bytes,
+                             stream);
 }
 
 csa2_status csa2_pool_candidates(const csa2_cache* shard, const float* blockmax, const int32_t* pool,

@@ -55,6 +55,41 @@ __device__ __forceinline__ uint32_t e2m1_code(float x, float s) {
   return c;
 }
 
+// FP4 indexer row (128 elements: E2M1 codes with one E4M3 scale per 16,
+// s = E4M3(amax / 6); the main-KV format on the indexer's row) held by a warp,
+// lane l owning elements 4l .. 4l+3 of group l / 4.  Returns the lane's two
+// code bytes (element 4l in the low nibble of the low byte) and the group's
+// scale code in *scale.
+__device__ __forceinline__ uint32_t fp4_row_lane(float4 v, uint32_t* scale) {
+  float m = fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w)));
+  m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
+  m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
+  const uint32_t sc = e4m3_code_of_sixth(m);
+  const float s = e4m3_value(sc);
+  *scale = sc;
+  if (!(s > 0.0f)) return 0u;
+  return e2m1_code(v.x, s) | (e2m1_code(v.y, s) << 4) | (e2m1_code(v.z, s) << 8) | (e2m1_code(v.w, s) << 12);
+}
+
+// FP4 codes and block scales of query heads 8*ew .. 8*ew+7 of q [32][128]
+// (one warp) as rows row0 + h of a tensor-core B operand: the codes into the
+// 64-byte-swizzled tile `qtile`, the scales into `qscale` in the tensor-core
+// order (row0 + 32 <= 128).
+__device__ __forceinline__ void prepare_query_fp4(const float* __restrict__ q, uint8_t* qtile, uint8_t* qscale,
+                                                  int row0, int ew, int lane) {
+  float4 v[8];
+#pragma unroll
+  for (int hh = 0; hh < 8; ++hh) v[hh] = reinterpret_cast<const float4*>(q + (ew * 8 + hh) * kIndexDim)[lane];
+#pragma unroll
+  for (int hh = 0; hh < 8; ++hh) {
+    const uint32_t r = static_cast<uint32_t>(row0 + ew * 8 + hh);
+    uint32_t sc;
+    const uint32_t codes = fp4_row_lane(v[hh], &sc);
+    *reinterpret_cast<uint16_t*>(qtile + sw64_offset(r, 2u * lane)) = static_cast<uint16_t>(codes);
+    if ((lane & 3) == 0) qscale[block_scale_offset(r, lane >> 2)] = static_cast<uint8_t>(sc);
+  }
+}
+
 // E2M1 magnitude (codes 0..7) as fp16 bit patterns: 0, 0.5, 1, 1.5, 2, 3, 4, 6.
 __device__ __forceinline__ uint16_t e2m1_half_bits(uint32_t c) {
   // fp16: sign(1) exp(5, bias 15) mant(10)

@@ -17,6 +17,7 @@
 // exact Top-k with 10-bit radix passes over the few keys in that bin, and
 // writes the positions ascending (ties to the lower position, -1 padding).
 #include "block_topk.cuh"
+#include "fp4.cuh"
 #include "index_common.cuh"
 #include "launch.h"
 
@@ -27,7 +28,6 @@ namespace {
 constexpr int kSThreads = 192;   // warp 0: TMA producer, warp 1: MMA, warps 2..5: epilogue
 constexpr int kSStages = 4;
 constexpr int kSMaxTiles = 8;    // tiles (16 pool blocks each) per CTA
-constexpr int kSBlkBytes = kBlock * kIndexDim;
 constexpr int kSBlocksPerTile = kTile / kBlock;   // 16
 constexpr uint32_t kSTmemCols = 256;
 constexpr int kSMaxAcc = 4;
@@ -42,10 +42,21 @@ struct TopkLayers {
   int32_t* topk[CSA2_MAX_SCORE_LAYERS];
 };
 
-struct __align__(1024) ScoreSmem {
-  uint8_t tiles[kSStages][kTileBytes];
-  uint8_t qtile[CSA2_MAX_SCORE_LAYERS][kQBytes];   // layer l: B-operand rows 32l .. 32l+31
-  float ws[CSA2_MAX_SCORE_LAYERS][kIndexHeads];    // w_h * sigma^q_h per layer
+constexpr int kMaxFp4ScoreLayers = 4;
+constexpr int kMaxPoolSlots = 4096;     // pool blocks (the host accepts up to 4096)   // N = 32 x layers <= 128: one block of query scales
+
+// Shared memory of the scoring kernel for the FP8 indexer (kFp4 = false: 128
+// code bytes and an exponent byte per row) or the FP4 one (64 code bytes and
+// the block scales of each row, gathered into the tensor-core order per tile).
+template <bool kFp4>
+struct __align__(1024) ScoreSmemT {
+  static constexpr int kRowBytes = kFp4 ? CSA2_IK4_CODE_BYTES : kIndexDim;
+  static constexpr int kLayers = kFp4 ? kMaxFp4ScoreLayers : CSA2_MAX_SCORE_LAYERS;
+  uint8_t tiles[kSStages][kTile * kRowBytes];
+  uint8_t qtile[kLayers][kIndexHeads * kRowBytes];          // layer l: B-operand rows 32l .. 32l+31
+  uint8_t qscale[kFp4 ? 1024 : 16];                         // FP4: the query heads' block scales
+  uint8_t tscale[kFp4 ? kSMaxTiles : 1][kFp4 ? 1024 : 16];  // FP4: each tile's block scales
+  float ws[kLayers][kIndexHeads];                           // w_h (FP4) or w_h * sigma^q_h (FP8) per layer
   uint64_t blk_exp[kSMaxTiles * kSBlocksPerTile];
   int blk_row[kSMaxTiles * kSBlocksPerTile];
   int blk_id[kSMaxTiles * kSBlocksPerTile];
@@ -59,13 +70,21 @@ struct __align__(1024) ScoreSmem {
   volatile int abort_flag;
 };
 
-// keys: uint32 [batch][L][P * 8]; hist: uint32 [batch][L][4096]
+// keys: uint32 [batch][L][P * 8]; hist: uint32 [batch][L][4096].  ik4_scales:
+// the FP4 keys' block scales (kFp4 only); blk_map: 8-row boxes of the index
+// codes (FP8: 128-byte rows, 128-byte swizzle; FP4: 64-byte rows, 64-byte
+// swizzle).
+template <bool kFp4>
 __global__ void __launch_bounds__(kSThreads, 2)
-    pool_score_kernel(const csa2_cache cache, const int32_t* __restrict__ pool, int P, int L, int tiles_per_cta,
-                      const __grid_constant__ ScoreLayers io, uint32_t* __restrict__ keys,
-                      uint32_t* __restrict__ hist, const __grid_constant__ CUtensorMap blk_map, uint64_t wait_ns) {
+    pool_score_kernel(const csa2_cache cache, const uint8_t* __restrict__ ik4_scales, const int32_t* __restrict__ pool,
+                      int P, int L, int tiles_per_cta, const __grid_constant__ ScoreLayers io,
+                      uint32_t* __restrict__ keys, uint32_t* __restrict__ hist,
+                      const __grid_constant__ CUtensorMap blk_map, uint64_t wait_ns) {
+  using Smem = ScoreSmemT<kFp4>;
+  constexpr int kBlkBytes = kBlock * Smem::kRowBytes;
+  constexpr int kTileB = kTile * Smem::kRowBytes;
   extern __shared__ uint8_t smem_raw[];
-  ScoreSmem& S = *reinterpret_cast<ScoreSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  Smem& S = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int tiles_per_req = (P + kSBlocksPerTile - 1) / kSBlocksPerTile;
   const int ctas_per_req = (tiles_per_req + tiles_per_cta - 1) / tiles_per_cta;
@@ -75,9 +94,14 @@ __global__ void __launch_bounds__(kSThreads, 2)
   const int nblk = max(0, min(tiles_per_cta * kSBlocksPerTile, P - slot0));   // pool slots of this CTA
   const int n_tiles = (nblk + kSBlocksPerTile - 1) / kSBlocksPerTile;
   const int ncols = kIndexHeads * L;                                     // accumulator columns per tile
-  // accumulators start at multiples of the next power of two >= ncols
+  // accumulators start at multiples of the next power of two >= ncols; with
+  // FP4, each accumulator also has 8 columns of its tile's block scales and the
+  // query scales take 8 more
   const int acc_stride = ncols <= 32 ? 32 : (ncols <= 64 ? 64 : (ncols <= 128 ? 128 : 256));
-  const int n_acc = min(kSMaxAcc, static_cast<int>(kSTmemCols) / acc_stride);
+  const int n_acc = kFp4 ? max(1, min(kSMaxAcc, static_cast<int>(kSTmemCols - 8) / (acc_stride + 8)))
+                         : min(kSMaxAcc, static_cast<int>(kSTmemCols) / acc_stride);
+  const uint32_t sfa_col = static_cast<uint32_t>(n_acc * acc_stride);   // FP4: tile scales of accumulator a at + 8a
+  const uint32_t sfb_col = sfa_col + 8u * n_acc;                        // FP4: query scales
   const long long key_stride = static_cast<long long>(P) * kBlock;
 
   pdl_wait();                 // the pool of the preceding launch is complete
@@ -101,7 +125,7 @@ __global__ void __launch_bounds__(kSThreads, 2)
       const int page = cache.page_table[static_cast<long long>(b) * cache.max_pages_per_req + t / cache.page_size];
       if (page >= 0 && page < cache.num_pages) {
         row = page * cache.page_size + t % cache.page_size;
-        ex = *reinterpret_cast<const uint64_t*>(cache.ik_exp + row);
+        if (!kFp4) ex = *reinterpret_cast<const uint64_t*>(cache.ik_exp + row);
       } else {
         report_error(cache.err_word, CSA2_ERR_DEVICE_BOUNDS, kKReindex, b, t);
       }
@@ -111,6 +135,25 @@ __global__ void __launch_bounds__(kSThreads, 2)
     S.blk_row[i] = row;
     S.blk_id[i] = row >= 0 ? j : -1;
     S.blk_exp[i] = ex;
+  }
+  if constexpr (kFp4) {
+    // block scales of the CTA's blocks, moved into each tile's tensor-core
+    // order: tile row m = 8 * (block % 16) + r takes the scales of the
+    // block's row r (4 bytes per half of the row's 8 scales)
+    __syncthreads();
+    for (int x = tid; x < n_tiles * kSBlocksPerTile * kBlock * 2; x += kSThreads) {
+      const int kh = x & 1, r = (x >> 1) & 7, i = x >> 4;
+      const int t = i / kSBlocksPerTile, m = kBlock * (i % kSBlocksPerTile) + r;
+      const int row = i < nblk ? S.blk_row[i] : -1;
+      uint32_t v = 0u;
+      if (row >= 0) {
+        const int sr = row % kTile + r;
+        v = *reinterpret_cast<const uint32_t*>(ik4_scales + static_cast<long long>(row / kTile) * 1024 +
+                                               block_scale_offset(sr, 4 * kh));
+      }
+      *reinterpret_cast<uint32_t*>(S.tscale[t] + block_scale_offset(m, 4 * kh)) = v;
+    }
+    fence_proxy_async_smem();
   }
   if (tid == 0) {
     for (int s = 0; s < kSStages; ++s) {
@@ -153,10 +196,10 @@ __global__ void __launch_bounds__(kSThreads, 2)
         }
         const int e = t * kSBlocksPerTile + lane;
         const int row = (lane < kSBlocksPerTile && e < nblk) ? S.blk_row[e] : -1;
-        const uint32_t bytes = __popc(__ballot_sync(0xffffffffu, row >= 0)) * kSBlkBytes;
+        const uint32_t bytes = __popc(__ballot_sync(0xffffffffu, row >= 0)) * kBlkBytes;
         if (lane == 0) mbar_arrive_expect_tx(&S.full[s], bytes);   // before any of the tile's copies
         __syncwarp();
-        if (row >= 0) tma_load_2d(S.tiles[s] + lane * kSBlkBytes, &blk_map, &S.full[s], 0, row, policy);
+        if (row >= 0) tma_load_2d(S.tiles[s] + lane * kBlkBytes, &blk_map, &S.full[s], 0, row, policy);
         ++issued;
       }
       if (lane == 0)
@@ -164,9 +207,15 @@ __global__ void __launch_bounds__(kSThreads, 2)
           (void)mbar_wait(&S.full[i % kSStages], (i / kSStages) & 1, kWaitLimitNs / 2);
     } else if (warp == 1) {
       if (lane == 0) {   // ---- MMA issuer: one N = 32L MMA chain per tile ----
-        const uint32_t idesc = idesc_e4m3_f32(kTile, ncols);
-        const uint64_t bdesc = sw128_kmajor_desc(smem_u32(S.qtile[0]));
+        const uint32_t idesc = kFp4 ? idesc_mxf4nvf4(kTile, ncols) : idesc_e4m3_f32(kTile, ncols);
+        const uint64_t bdesc = kFp4 ? sw64_kmajor_desc(smem_u32(S.qtile[0])) : sw128_kmajor_desc(smem_u32(S.qtile[0]));
         bool ok = mbar_wait(&S.q_full, 0, wait_ns);
+        if constexpr (kFp4) {
+          if (ok) {
+            tc_fence_after();
+            for (int kh = 0; kh < 2; ++kh) tmem_cp_scales(tmem + sfb_col + 4 * kh, smem_u32(S.qscale + 512 * kh));
+          }
+        }
         for (int t = 0; ok && t < n_tiles; ++t) {
           const int s = t % kSStages;
           const uint32_t ph = (t / kSStages) & 1;
@@ -178,10 +227,20 @@ __global__ void __launch_bounds__(kSThreads, 2)
           }
           if (S.abort_flag) break;
           tc_fence_after();
-          const uint64_t adesc = sw128_kmajor_desc(smem_u32(S.tiles[s]));
+          if constexpr (kFp4) {
+            const uint32_t sfa = tmem + sfa_col + 8 * a;
+            for (int kh = 0; kh < 2; ++kh) tmem_cp_scales(sfa + 4 * kh, smem_u32(S.tscale[t] + 512 * kh));
+            const uint64_t adesc = sw64_kmajor_desc(smem_u32(S.tiles[s]));
 #pragma unroll
-          for (int k = 0; k < kIndexDim / 32; ++k)
-            umma_f8f6f4(tmem + a * acc_stride, adesc + 2 * k, bdesc + 2 * k, idesc, k > 0 ? 1u : 0u);
+            for (int kh = 0; kh < 2; ++kh)
+              umma_mxf4nvf4(tmem + a * acc_stride, adesc + 2 * kh, bdesc + 2 * kh, idesc, sfa + 4 * kh,
+                            tmem + sfb_col + 4 * kh, kh > 0 ? 1u : 0u);
+          } else {
+            const uint64_t adesc = sw128_kmajor_desc(smem_u32(S.tiles[s]));
+#pragma unroll
+            for (int k = 0; k < kIndexDim / 32; ++k)
+              umma_f8f6f4(tmem + a * acc_stride, adesc + 2 * k, bdesc + 2 * k, idesc, k > 0 ? 1u : 0u);
+          }
           umma_commit(&S.empty[s]);
           umma_commit(&S.acc_full[a]);
         }
@@ -195,9 +254,16 @@ __global__ void __launch_bounds__(kSThreads, 2)
     } else {
       // ---- epilogue (warps 2..5): one position per thread, every layer ----
       const int ew = warp - 2, quarter = warp & 3, m = quarter * 32 + lane;
-      for (int l = 0; l < L; ++l)
-        prepare_query_part(io.q[l] + static_cast<long long>(b) * kIndexHeads * kIndexDim,
-                           io.w[l] + static_cast<long long>(b) * kIndexHeads, S.qtile[l], S.ws[l], ew, lane);
+      for (int l = 0; l < L; ++l) {
+        const float* ql = io.q[l] + static_cast<long long>(b) * kIndexHeads * kIndexDim;
+        const float* wl = io.w[l] + static_cast<long long>(b) * kIndexHeads;
+        if constexpr (kFp4) {
+          prepare_query_fp4(ql, S.qtile[0], S.qscale, kIndexHeads * l, ew, lane);
+          if (lane < 8) S.ws[l][ew * 8 + lane] = wl[ew * 8 + lane];
+        } else {
+          prepare_query_part(ql, wl, S.qtile[l], S.ws[l], ew, lane);
+        }
+      }
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(&S.q_full);
@@ -209,7 +275,7 @@ __global__ void __launch_bounds__(kSThreads, 2)
         const int o = m % kBlock;
         const bool in_range = e < nblk;
         const bool valid = in_range && S.blk_row[e] >= 0 && S.blk_id[e] * kBlock + o < n;
-        const uint32_t e_byte = valid ? static_cast<uint32_t>((S.blk_exp[e] >> (8 * o)) & 0xFFu) : 127u;
+        const uint32_t e_byte = (!kFp4 && valid) ? static_cast<uint32_t>((S.blk_exp[e] >> (8 * o)) & 0xFFu) : 127u;
         if (!mbar_wait_warp(&S.acc_full[a], aph, wait_ns)) {
           if (lane == 0) {
             report_error(cache.err_word, CSA2_ERR_TIMEOUT, kKReindex, b, t);
@@ -225,7 +291,15 @@ __global__ void __launch_bounds__(kSThreads, 2)
           float ws[32];
 #pragma unroll
           for (int h = 0; h < 32; ++h) ws[h] = S.ws[l][h];
-          const uint32_t key = valid ? order_key(score_from_acc(acc, ws, e_byte)) : 0u;
+          float sc;
+          if constexpr (kFp4) {
+            sc = 0.0f;
+#pragma unroll
+            for (int h = 0; h < 32; ++h) sc = fmaf(ws[h], fmaxf(__uint_as_float(acc[h]), 0.0f), sc);
+          } else {
+            sc = score_from_acc(acc, ws, e_byte);
+          }
+          const uint32_t key = valid ? order_key(sc) : 0u;
           const long long bl = static_cast<long long>(b) * L + l;
           if (in_range) keys[bl * key_stride + static_cast<long long>(slot0 + e) * kBlock + o] = key;
           if (valid) atomicAdd(&hist[bl * kRsHistBins + (key >> (32 - kRsHistBits))], 1u);
@@ -252,6 +326,7 @@ __global__ void __launch_bounds__(kBlockSelectThreads, 1)
     layer_select_kernel(const int32_t* __restrict__ pool, int P, int L, int K, const uint32_t* __restrict__ keys,
                         uint32_t* __restrict__ hist, const __grid_constant__ TopkLayers out) {
   __shared__ BlockSelectSmem S;
+  __shared__ int32_t pool_ids[kMaxPoolSlots];
   const int tid = threadIdx.x;
   const int b = blockIdx.x / L, l = blockIdx.x % L;
   const long long bl = static_cast<long long>(b) * L + l;
@@ -259,6 +334,9 @@ __global__ void __launch_bounds__(kBlockSelectThreads, 1)
   pdl_wait();                 // the keys and histograms of the scoring launch are complete
   pdl_launch_dependents();
 
+  // the request's pool (block ids of the key groups), read before the keys
+  // and used by the emits after the select's barriers
+  for (int i = tid; i < P; i += kBlockSelectThreads) pool_ids[i] = pool[static_cast<long long>(b) * P + i];
   // keys [tid*ITEMS, (tid+1)*ITEMS) in registers (groups of 4: n_keys is a multiple of 8)
   uint32_t k[ITEMS];
   const uint32_t* src = keys + bl * n_keys;
@@ -285,10 +363,9 @@ __global__ void __launch_bounds__(kBlockSelectThreads, 1)
   (void)block_exclusive_sum<kBlockSelectThreads>(valid, S.warp_tmp, &n_valid);
   const bool ok = hist_head_start<kBlockSelectThreads, 4>(c, 4 * (kBlockSelectThreads - 1 - tid) + 3, kRsHistBits,
                                                           n_valid, K, S.warp_tmp, &S.start);
-  const int32_t* pb = pool + static_cast<long long>(b) * P;
   int32_t* dst = out.topk[l] + static_cast<long long>(b) * K;
   block_topk<ITEMS>(
-      k, K, S, [&](int i, int r) { dst[r] = pb[i / kBlock] * kBlock + (i % kBlock); },
+      k, K, S, [&](int i, int r) { dst[r] = pool_ids[i / kBlock] * kBlock + (i % kBlock); },
       [&](int r) { dst[r] = -1; }, ok ? &S.start : nullptr);
 }
 
@@ -300,17 +377,22 @@ size_t rescore_workspace_bytes(long long batch, int n_layers, int pool_blocks) {
          (static_cast<size_t>(pool_blocks) * kBlock + kRsHistBins) * sizeof(uint32_t);
 }
 
-cudaError_t launch_rescore_layers(const csa2_cache& cache, int n_layers, const int32_t* pool, int pool_blocks,
-                                  const float* const* q, const float* const* w, int k, int32_t* const* topk,
-                                  void* workspace, const CUtensorMap& blk_map, int num_sms, uint64_t wait_ns,
-                                  cudaStream_t stream) {
-  static ContextMemo attrs;
-  const size_t smem = sizeof(ScoreSmem) + 1024;
-  cudaError_t e = attrs.once([&] {
-    cudaError_t r =
-        cudaFuncSetAttribute(pool_score_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-    return r;
-  });
+cudaError_t launch_rescore_layers(const csa2_cache& cache, const uint8_t* ik4_scales, int n_layers,
+                                  const int32_t* pool, int pool_blocks, const float* const* q, const float* const* w,
+                                  int k, int32_t* const* topk, void* workspace, const CUtensorMap& blk_map,
+                                  int num_sms, uint64_t wait_ns, cudaStream_t stream) {
+  const bool fp4 = ik4_scales != nullptr;
+  static ContextMemo attrs8, attrs4;
+  const size_t smem = (fp4 ? sizeof(ScoreSmemT<true>) : sizeof(ScoreSmemT<false>)) + 1024;
+  cudaError_t e = fp4 ? attrs4.once([&] {
+    return cudaFuncSetAttribute(pool_score_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                static_cast<int>(smem));
+  })
+                      : attrs8.once([&] {
+                          return cudaFuncSetAttribute(pool_score_kernel<false>,
+                                                      cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                      static_cast<int>(smem));
+                        });
   if (e != cudaSuccess) return e;
   ScoreLayers io = {};
   TopkLayers out = {};
@@ -338,8 +420,12 @@ cudaError_t launch_rescore_layers(const csa2_cache& cache, int n_layers, const i
   cfg.gridDim = dim3(cache.batch * ctas_per_req);
   cfg.blockDim = dim3(kSThreads);
   cfg.dynamicSmemBytes = smem;
-  e = cudaLaunchKernelEx(&cfg, pool_score_kernel, cache, pool, pool_blocks, n_layers, tpc, io, keys, hist, blk_map,
-                         wait_ns);
+  if (fp4)
+    e = cudaLaunchKernelEx(&cfg, pool_score_kernel<true>, cache, ik4_scales, pool, pool_blocks, n_layers, tpc, io, keys,
+                           hist, blk_map, wait_ns);
+  else
+    e = cudaLaunchKernelEx(&cfg, pool_score_kernel<false>, cache, ik4_scales, pool, pool_blocks, n_layers, tpc, io,
+                           keys, hist, blk_map, wait_ns);
   if (e != cudaSuccess) return e;
   cfg.gridDim = dim3(cache.batch * n_layers);
   cfg.blockDim = dim3(kBlockSelectThreads);

@@ -65,16 +65,25 @@ cudaError_t launch_index_full(const csa2_cache& cache, const float* q, const flo
                               float* scores, uint32_t* hist, const CUtensorMap& ik_map, int num_sms, uint64_t wait_ns,
                               cudaStream_t stream);
 
+// FP4 indexer: scan and quantise-on-append.
+size_t index_full_fp4_smem_bytes();
+cudaError_t launch_index_full_fp4(const csa2_cache& cache, const uint8_t* ik4_scales, const float* q, const float* w,
+                                  float* blockmax, float* scores, uint32_t* hist, const CUtensorMap& code_map,
+                                  int num_sms, uint64_t wait_ns, cudaStream_t stream);
+cudaError_t launch_append_ik4(const csa2_cache& cache, uint8_t* codes, uint8_t* scales, int n_rows,
+                              const float* ik_new, const int32_t* req, const int32_t* pos, cudaStream_t stream);
+
 cudaError_t launch_pool_select(const csa2_cache& cache, const float* blockmax, uint32_t* hist, int pool_blocks,
                                int32_t* pool, int cluster, cudaStream_t stream);
 
 // Top-k of n_layers layers over the pool: one scoring launch (every pool
 // block gathered once, all layers in one MMA) and one select launch.
 size_t rescore_workspace_bytes(long long batch, int n_layers, int pool_blocks);
-cudaError_t launch_rescore_layers(const csa2_cache& cache, int n_layers, const int32_t* pool, int pool_blocks,
-                                  const float* const* q, const float* const* w, int k, int32_t* const* topk,
-                                  void* workspace, const CUtensorMap& blk_map, int num_sms, uint64_t wait_ns,
-                                  cudaStream_t stream);
+// ik4_scales != nullptr: the FP4 indexer (blk_map over its codes, n_layers <= 4).
+cudaError_t launch_rescore_layers(const csa2_cache& cache, const uint8_t* ik4_scales, int n_layers,
+                                  const int32_t* pool, int pool_blocks, const float* const* q, const float* const* w,
+                                  int k, int32_t* const* topk, void* workspace, const CUtensorMap& blk_map,
+                                  int num_sms, uint64_t wait_ns, cudaStream_t stream);
 
 constexpr int kReindexPoolCluster = 16;   // CTAs per request when re-scoring a pool
 cudaError_t launch_reindex(const csa2_cache& cache, const int32_t* pool, int pool_blocks, const float* q,

@@ -168,3 +168,11 @@ def test_slice_pages_cover_the_table():
         assert len(s) == g and s[0][0] == 0 and sum(n for _, n in s) == pages
         assert all(s[k][0] + s[k][1] == s[k + 1][0] for k in range(g - 1))
         assert max(n for _, n in s) - min(n for _, n in s) <= 1
+
+
+def test_fp4_oracle_sample_runs_small():
+    from kv_cache_decode_index_b200 import workloads as W
+    wl = W.scaled(W.WORKLOADS["group_1m_b4"], ctx=8192, pool_blocks=64, needles=0)
+    assert bench.oracle_sample_fp4(wl, 0) > 0
+    step, scan = bench.alg_bytes(wl, ik_row_bytes=bench.IK4_ROW_BYTES)
+    assert scan == 72 * 8192 * wl.batch
