@@ -97,11 +97,16 @@ __global__ void __launch_bounds__(kSThreads, 2)
   // accumulators start at multiples of the next power of two >= ncols; with
   // FP4, each accumulator also has 8 columns of its tile's block scales and the
   // query scales take 8 more
+  // (in the columns an accumulator slot leaves unused when there are 16 of
+  // them: 3 layers, N = 96 in 128-column slots, keep two slots)
   const int acc_stride = ncols <= 32 ? 32 : (ncols <= 64 ? 64 : (ncols <= 128 ? 128 : 256));
-  const int n_acc = kFp4 ? max(1, min(kSMaxAcc, static_cast<int>(kSTmemCols - 8) / (acc_stride + 8)))
-                         : min(kSMaxAcc, static_cast<int>(kSTmemCols) / acc_stride);
-  const uint32_t sfa_col = static_cast<uint32_t>(n_acc * acc_stride);   // FP4: tile scales of accumulator a at + 8a
-  const uint32_t sfb_col = sfa_col + 8u * n_acc;                        // FP4: query scales
+  const bool sf_inside = kFp4 && acc_stride - ncols >= 16;
+  const int n_acc = !kFp4 || sf_inside ? min(kSMaxAcc, static_cast<int>(kSTmemCols) / acc_stride)
+                                       : max(1, min(kSMaxAcc, static_cast<int>(kSTmemCols - 8) / (acc_stride + 8)));
+  // FP4: tile scales of accumulator a at sfa_col + sfa_step * a, query scales at sfb_col
+  const uint32_t sfa_col = static_cast<uint32_t>(sf_inside ? ncols : n_acc * acc_stride);
+  const uint32_t sfa_step = static_cast<uint32_t>(sf_inside ? acc_stride : 8);
+  const uint32_t sfb_col = sf_inside ? static_cast<uint32_t>(ncols + 8) : sfa_col + 8u * n_acc;
   const long long key_stride = static_cast<long long>(P) * kBlock;
 
   pdl_wait();                 // the pool of the preceding launch is complete
@@ -141,17 +146,26 @@ __global__ void __launch_bounds__(kSThreads, 2)
     // order: tile row m = 8 * (block % 16) + r takes the scales of the
     // block's row r (4 bytes per half of the row's 8 scales)
     __syncthreads();
-    for (int x = tid; x < n_tiles * kSBlocksPerTile * kBlock * 2; x += kSThreads) {
+    // all of a thread's loads are issued before any is used
+    constexpr int kWords = (kSMaxTiles * kSBlocksPerTile * kBlock * 2 + kSThreads - 1) / kSThreads;
+    const int n_words = n_tiles * kSBlocksPerTile * kBlock * 2;
+    uint32_t v[kWords];
+#pragma unroll
+    for (int u = 0; u < kWords; ++u) {
+      const int x = tid + u * kSThreads;
+      const int kh = x & 1, r = (x >> 1) & 7, i = x >> 4;
+      const int row = (x < n_words && i < nblk) ? S.blk_row[i] : -1;
+      v[u] = row >= 0 ? *reinterpret_cast<const uint32_t*>(ik4_scales + static_cast<long long>(row / kTile) * 1024 +
+                                                           block_scale_offset(row % kTile + r, 4 * kh))
+                      : 0u;
+    }
+#pragma unroll
+    for (int u = 0; u < kWords; ++u) {
+      const int x = tid + u * kSThreads;
+      if (x >= n_words) continue;
       const int kh = x & 1, r = (x >> 1) & 7, i = x >> 4;
       const int t = i / kSBlocksPerTile, m = kBlock * (i % kSBlocksPerTile) + r;
-      const int row = i < nblk ? S.blk_row[i] : -1;
-      uint32_t v = 0u;
-      if (row >= 0) {
-        const int sr = row % kTile + r;
-        v = *reinterpret_cast<const uint32_t*>(ik4_scales + static_cast<long long>(row / kTile) * 1024 +
-                                               block_scale_offset(sr, 4 * kh));
-      }
-      *reinterpret_cast<uint32_t*>(S.tscale[t] + block_scale_offset(m, 4 * kh)) = v;
+      *reinterpret_cast<uint32_t*>(S.tscale[t] + block_scale_offset(m, 4 * kh)) = v[u];
     }
     fence_proxy_async_smem();
   }
@@ -228,7 +242,7 @@ __global__ void __launch_bounds__(kSThreads, 2)
           if (S.abort_flag) break;
           tc_fence_after();
           if constexpr (kFp4) {
-            const uint32_t sfa = tmem + sfa_col + 8 * a;
+            const uint32_t sfa = tmem + sfa_col + sfa_step * a;
             for (int kh = 0; kh < 2; ++kh) tmem_cp_scales(sfa + 4 * kh, smem_u32(S.tscale[t] + 512 * kh));
             const uint64_t adesc = sw64_kmajor_desc(smem_u32(S.tiles[s]));
 #pragma unroll

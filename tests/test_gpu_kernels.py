@@ -218,10 +218,16 @@ def test_index_full_scores_ragged(csa2):
 
 # ------------------------------------------------------- pool_select (a3) --
 
-@pytest.mark.parametrize("lengths,P", [([1048576, 300000], 2048), ([16384, 16383, 8, 0], 2048),
-                                       ([200000, 5000], 64), ([1500000], 2048)])
-def test_pool_select_bitexact(csa2, lengths, P):
-    """Synthetic block maxima with many ties (and negative values), fed to both."""
+@pytest.mark.parametrize("lengths,P,kind", [([1048576, 300000], 2048, "ties"), ([16384, 16383, 8, 0], 2048, "ties"),
+                                            ([200000, 5000], 64, "ties"), ([1500000], 2048, "ties"),
+                                            ([1048576, 700000], 2048, "on_sample_grid"),
+                                            ([1048576], 2048, "all_equal")])
+def test_pool_select_bitexact(csa2, lengths, P, kind):
+    """Synthetic block maxima with many ties (and negative values), fed to both.
+    "on_sample_grid": the largest maxima sit exactly on the evenly spaced
+    sample, so the sampled threshold admits fewer blocks than the pool needs
+    and the kernel must take its exact fallback; "all_equal": every block ties
+    (more candidates than the fast path holds)."""
     rng = np.random.default_rng(len(lengths) * 1000 + P)
     B = len(lengths)
     page = 4096
@@ -232,6 +238,13 @@ def test_pool_select_bitexact(csa2, lengths, P):
     vals = rng.standard_normal((B, cap8)).astype(np.float32)
     vals[:, ::3] = np.round(vals[:, ::3] * 4) / 4                       # ties
     vals[:, 5::7] = 2.0                                                  # a big tie group
+    if kind == "on_sample_grid":
+        for b, n in enumerate(lengths):
+            nb = -(-n // 8)
+            grid = (np.arange(4096, dtype=np.int64) * nb) // 4096
+            vals[b, grid] = 100.0 + rng.random(4096).astype(np.float32)
+    elif kind == "all_equal":
+        vals[:] = 3.5
     dev = cache.device
     tv = torch.from_numpy(vals).to(dev)
     pool = csa2.pool_select(cache, tv, P).cpu().numpy()
