@@ -218,9 +218,12 @@ csa2_status csa2_index_full(const csa2_cache* cache, const float* q, const float
   if (hist != nullptr && !aligned(hist, 16)) return fail(CSA2_ERR_ARG, "hist must be 16-byte aligned");
   DeviceInfo d;
   CSA2_TRY(device_info(&d));
+  // With pages of whole 256-position units, one TMA box covers a unit.
+  const int whole_units = cache->page_size % (2 * csa2::kTile) == 0;
   CUtensorMap map;
-  CSA2_TRY(encode_ik_map(cache, csa2::kTile, &map));
-  const cudaError_t e = csa2::launch_index_full(*cache, q, w, blockmax, scores, hist, map, d.sms, g_wait_limit_ns,
+  CSA2_TRY(encode_ik_map(cache, whole_units ? 2 * csa2::kTile : csa2::kTile, &map));
+  const cudaError_t e = csa2::launch_index_full(*cache, q, w, blockmax, scores, hist, map, whole_units, d.sms,
+                                                g_wait_limit_ns,
                                                 static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? CSA2_OK : cuda_fail(e, "index_full launch");
 }
@@ -251,11 +254,14 @@ csa2_status csa2_index_full_fp4(const csa2_cache* cache, const csa2_ik4* ik4, co
   if (hist != nullptr && !aligned(hist, 16)) return fail(CSA2_ERR_ARG, "hist must be 16-byte aligned");
   DeviceInfo d;
   CSA2_TRY(device_info(&d));
+  const int whole_units = cache->page_size % (2 * csa2::kTile) == 0;   // one TMA box per unit
   CUtensorMap map;
   CSA2_TRY(encode_rows_map(ik4->codes, static_cast<long long>(cache->num_pages) * cache->page_size,
-                           CSA2_IK4_CODE_BYTES, csa2::kTile, CU_TENSOR_MAP_SWIZZLE_64B, &map));
-  const cudaError_t e = csa2::launch_index_full_fp4(*cache, ik4->scales, q, w, blockmax, scores, hist, map, d.sms,
-                                                    g_wait_limit_ns, static_cast<cudaStream_t>(stream));
+                           CSA2_IK4_CODE_BYTES, whole_units ? 2 * csa2::kTile : csa2::kTile,
+                           CU_TENSOR_MAP_SWIZZLE_64B, &map));
+  const cudaError_t e = csa2::launch_index_full_fp4(*cache, ik4->scales, q, w, blockmax, scores, hist, map,
+                                                    whole_units, d.sms, g_wait_limit_ns,
+                                                    static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? CSA2_OK : cuda_fail(e, "index_full_fp4 launch");
 }
 

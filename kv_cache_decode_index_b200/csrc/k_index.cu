@@ -7,16 +7,27 @@
 // Design (sm_100a), one persistent CTA per SM; the concatenated work units of
 // all requests (256 positions each) are split into contiguous ranges, one per
 // CTA:
-//   * warp 0 (one lane): producer.  Per unit, two TMA loads of 128-row
-//     indexer-K sub-tiles (128 FP8 bytes per row, 128-byte swizzle) into one
-//     32 KB stage of a kStages ring;
+//   * warp 0: producer.  Every 32 units the warp finds their cache rows in
+//     parallel (one unit per lane: request, page-table entry, row; the
+//     page-table loads of the next 32 are in flight while lane 0 issues the
+//     current 32), so that the issuing lane does no address arithmetic and
+//     waits on no global load.  Per unit, lane 0 issues one TMA load of the
+//     256-row unit (128 FP8 bytes per row, 128-byte swizzle; two 128-row
+//     loads when a page holds an odd number of 128-row tiles) and one bulk
+//     copy of its 256 exponent bytes into one stage of a kStages ring.  The
+//     issuing lane is the scan's pacing resource: it shares its SM
+//     sub-partition with two epilogue warps, and every instruction it saves
+//     is time the copies spend in flight;
 //   * warp 1 (one lane): tcgen05.mma kind::f8f6f4, M = 128 positions, N = 32
 //     heads, K = 128 in 4 steps, per sub-tile, into an accumulator pair (one of
-//     kAcc) in TMEM; the stage is released by the MMAs' completion;
+//     kAcc) in TMEM; the stage is released by the MMAs' completion together
+//     with the epilogue warps' reads of its exponent bytes;
 //   * warps 2..9: two epilogue warpgroups taking alternate units, one thread
 //     per position of each sub-tile: tcgen05.ld of the 32 head dot products,
-//     score, block max over 8 lanes, stores.  The exponent bytes are read
-//     straight from global memory one unit ahead.  Group 0 also quantises each
+//     score, block max over 8 lanes, stores.  The exponent bytes come from
+//     the stage (per-thread byte loads from global memory put their latency
+//     and address arithmetic on the epilogue warps, which share issue slots
+//     with the producer).  Group 0 also quantises each
 //     request's query into the B-operand tile (three buffers) for the MMA.
 //     With a histogram buffer, each block max also adds one count to its
 //     request's histogram of leading order-key bits (in shared memory, flushed
@@ -31,12 +42,13 @@
 
 #include "index_common.cuh"
 #include "launch.h"
+#include "scan_units.cuh"
 
 namespace csa2 {
 
 namespace {
 
-constexpr int kUnit = 2 * kTile;           // positions per work unit (two MMA sub-tiles)
+constexpr int kUnit = kScanUnit;           // positions per work unit (two MMA sub-tiles)
 constexpr int kStages = 6;                 // unit ring (32 KB each)
 constexpr int kAcc = 4;                    // TMEM accumulator pairs (2 x 32 columns each)
 constexpr int kEpiGroups = 2;
@@ -49,9 +61,11 @@ constexpr uint32_t kTmemCols = kAcc * 2 * kAccCols;   // 256
 struct __align__(1024) IndexSmem {
   uint8_t tiles[kStages][2][kTileBytes];
   uint8_t q[kQBufs][kQBytes];
+  uint8_t exps[kStages][kUnit];        // exponent bytes of the stage's unit
+  int rowq[32][2];                     // cache rows of the producer's current 32 units (-1: none)
   int prefix[kMaxBatchScan + 1];       // units before request b
   uint64_t full[kStages];
-  uint64_t empty[kStages];
+  uint64_t empty[kStages];             // the MMAs' completion + the 4 epilogue warps of the unit
   uint64_t acc_full[kAcc];
   uint64_t acc_empty[kAcc];
   uint64_t q_full[kQBufs];
@@ -63,46 +77,10 @@ struct __align__(1024) IndexSmem {
   uint32_t hist[2][kPoolHistBins / 2];
 };
 
-// Walks this CTA's units in order: request b, unit j inside it.
-struct TileIter {
-  const int* prefix;
-  int batch;
-  int b, j;
-  __device__ void init(const int* pre, int nb, int g) {
-    prefix = pre;
-    batch = nb;
-    int lo = 0, hi = nb - 1;   // last b with prefix[b] <= g
-    while (lo < hi) {
-      const int mid = (lo + hi + 1) >> 1;
-      if (pre[mid] <= g) lo = mid;
-      else hi = mid - 1;
-    }
-    b = lo;
-    j = g - pre[lo];
-    skip_empty();
-  }
-  __device__ void skip_empty() {
-    while (b < batch && j >= prefix[b + 1] - prefix[b]) {
-      j = 0;
-      ++b;
-    }
-  }
-  __device__ void advance() {
-    ++j;
-    skip_empty();
-  }
-};
-
-__device__ __forceinline__ int next_request_with_tiles(const int* prefix, int batch, int b) {
-  ++b;
-  while (b < batch && prefix[b + 1] == prefix[b]) ++b;
-  return b;
-}
-
 __global__ void __launch_bounds__(kThreads, 1)
     index_full_kernel(const csa2_cache cache, const float* __restrict__ q, const float* __restrict__ w,
                       float* __restrict__ blockmax, float* __restrict__ scores, uint32_t* __restrict__ hist,
-                      const __grid_constant__ CUtensorMap ik_map, uint64_t wait_ns) {
+                      const __grid_constant__ CUtensorMap ik_map, int whole_units, uint64_t wait_ns) {
   extern __shared__ uint8_t smem_raw[];
   IndexSmem& S = *reinterpret_cast<IndexSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int tid = threadIdx.x;
@@ -138,7 +116,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&S.full[s], 1);
-      mbar_init(&S.empty[s], 1);     // the MMA's completion
+      mbar_init(&S.empty[s], 5);
     }
     for (int a = 0; a < kAcc; ++a) {
       mbar_init(&S.acc_full[a], 1);
@@ -181,48 +159,56 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (n_tiles > 0) {
     if (warp == 0) {
       // ================= producer =================
-      if (lane == 0) {
-        const uint64_t policy = l2_policy_evict_first();
-        TileIter it;
-        it.init(S.prefix, B, t_begin);
-        int issued = 0;
-        long long page_key = -1;   // page-table slot of the cached page id
-        int page = 0;
-        for (int i = 0; i < n_tiles; ++i) {
-          const int s = i % kStages;
-          if (!mbar_wait(&S.empty[s], ((i / kStages) & 1) ^ 1, wait_ns)) {
-            report_error(cache.err_word, CSA2_ERR_TIMEOUT, kKIndexFull, it.b, i);
-            S.abort_flag = 1;
-            break;
-          }
-          if (S.abort_flag) break;
-          // sub-tiles of the unit that lie inside the request's capacity (page-table range);
-          // positions are below 2^31 (checked on the host), so 32-bit arithmetic
-          int rows[2];
-          uint32_t bytes = 0;
-          for (int h = 0; h < 2; ++h) {
-            const int p0 = it.j * kUnit + h * kTile;
-            rows[h] = -1;
-            if (p0 >= capacity) continue;
-            const int pidx = static_cast<int>(static_cast<uint32_t>(p0) / page_size);
-            const long long key = static_cast<long long>(it.b) * cache.max_pages_per_req + pidx;
-            if (key != page_key) {   // one page-table load per page
-              page_key = key;
-              page = cache.page_table[key];
-              if (page < 0 || page >= cache.num_pages) {
-                report_error(cache.err_word, CSA2_ERR_DEVICE_BOUNDS, kKIndexFull, it.b, p0);
-                page = 0;   // load a valid page; the results of this sub-tile are flagged invalid
+      const uint64_t policy = l2_policy_evict_first();
+      const uint32_t full_mask = 0xffffffffu;
+      UnitRows next;   // this lane's unit of the next 32
+      next.fetch(cache, S.prefix, B, t_begin + lane, lane < n_tiles, capacity, page_size);
+      int issued = 0;   // lane 0
+      bool stop = false;
+      for (int i0 = 0; i0 < n_tiles && !stop; i0 += 32) {
+        int r[2];
+        next.rows(cache, capacity, kKIndexFull, r);
+        S.rowq[lane][0] = r[0];
+        S.rowq[lane][1] = r[1];
+        // the next 32 units' page-table loads are in flight while lane 0 issues
+        next.fetch(cache, S.prefix, B, t_begin + i0 + 32 + lane, i0 + 32 + lane < n_tiles, capacity, page_size);
+        __syncwarp();
+        if (lane == 0) {
+          const int n = min(32, n_tiles - i0);
+          for (int k = 0; k < n; ++k) {
+            const int i = i0 + k, s = i % kStages;
+            if (!mbar_wait(&S.empty[s], ((i / kStages) & 1) ^ 1, wait_ns)) {
+              report_error(cache.err_word, CSA2_ERR_TIMEOUT, kKIndexFull, -1, i);
+              S.abort_flag = 1;
+            }
+            if (S.abort_flag) {
+              stop = true;
+              break;
+            }
+            const int r0 = S.rowq[k][0], r1 = S.rowq[k][1];
+            // rows are multiples of 128, so the exponent copies start 16-byte aligned
+            if (whole_units && r0 >= 0) {   // the unit's 256 rows are consecutive
+              mbar_arrive_expect_tx(&S.full[s], 2 * kTileBytes + kUnit);
+              tma_load_2d(S.tiles[s][0], &ik_map, &S.full[s], 0, r0, policy);
+              bulk_load_1d(S.exps[s], cache.ik_exp + r0, kUnit, &S.full[s], policy);
+            } else {
+              mbar_arrive_expect_tx(&S.full[s], (r0 >= 0) * (kTileBytes + kTile) + (r1 >= 0) * (kTileBytes + kTile));
+              if (r0 >= 0) {
+                tma_load_2d(S.tiles[s][0], &ik_map, &S.full[s], 0, r0, policy);
+                bulk_load_1d(S.exps[s], cache.ik_exp + r0, kTile, &S.full[s], policy);
+              }
+              if (r1 >= 0) {
+                tma_load_2d(S.tiles[s][1], &ik_map, &S.full[s], 0, r1, policy);
+                bulk_load_1d(S.exps[s] + kTile, cache.ik_exp + r1, kTile, &S.full[s], policy);
               }
             }
-            rows[h] = page * cache.page_size + (p0 - pidx * cache.page_size);
-            bytes += kTileBytes;
+            ++issued;
           }
-          mbar_arrive_expect_tx(&S.full[s], bytes);
-          for (int h = 0; h < 2; ++h)
-            if (rows[h] >= 0) tma_load_2d(S.tiles[s][h], &ik_map, &S.full[s], 0, rows[h], policy);
-          ++issued;
-          it.advance();
         }
+        stop = __shfl_sync(full_mask, stop, 0);
+        __syncwarp();
+      }
+      if (lane == 0) {
         // copies still in flight (only after an abort): wait for the last one of each stage
         for (int i = issued > kStages ? issued - kStages : 0; i < issued; ++i)
           (void)mbar_wait(&S.full[i % kStages], (i / kStages) & 1, kWaitLimitNs / 2);
@@ -308,27 +294,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       int nb = cache.ctx_len[cur_b];
       if (group == 1) it.advance();
 
-      // Exponent bytes of this thread's two positions in unit `u` (request b,
-      // unit j), read from global memory; issued one unit ahead of their use.
-      long long ex_key = -1;
-      int ex_page = 0;
-      auto exp_bytes = [&](int b, int j, uint32_t (&e)[2]) {
-        for (int h = 0; h < 2; ++h) {
-          const int p = j * kUnit + h * kTile + toff;
-          e[h] = 127u;
-          if (b >= B || p >= capacity) continue;
-          const int pidx = static_cast<int>(static_cast<uint32_t>(p) / page_size);
-          const long long key = static_cast<long long>(b) * cache.max_pages_per_req + pidx;
-          if (key != ex_key) {
-            ex_key = key;
-            ex_page = cache.page_table[key];
-            ex_page = (ex_page < 0 || ex_page >= cache.num_pages) ? 0 : ex_page;
-          }
-          e[h] = cache.ik_exp[static_cast<long long>(ex_page) * cache.page_size + (p - pidx * cache.page_size)];
-        }
-      };
-      uint32_t ex_cur[2], ex_next[2];
-      exp_bytes(it.b, it.j, ex_cur);
 
       for (int i = group; i < n_tiles; i += kEpiGroups) {
         if (it.b != cur_b) {
@@ -341,15 +306,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                             ws, lane);
           nb = cache.ctx_len[cur_b];
         }
-        const int a = i % kAcc;
+        const int a = i % kAcc, s = i % kStages;
         const int j = it.j;
-        // prefetch the exponents of this group's next unit
         TileIter nx = it;
         nx.advance();
         nx.advance();
-        if (i + kEpiGroups < n_tiles) exp_bytes(nx.b, nx.j, ex_next);
 
-        if (!mbar_wait_warp(&S.acc_full[a], (i / kAcc) & 1, wait_ns)) {
+        // The stage's copies completed before the MMAs were issued; the wait
+        // on its full barrier (the phase of this unit: the stage is not
+        // refilled before this warp releases it) makes them visible here.
+        if (!mbar_wait_warp(&S.acc_full[a], (i / kAcc) & 1, wait_ns) ||
+            !mbar_wait_warp(&S.full[s], (i / kStages) & 1, wait_ns)) {
           timed_out(j);
           break;
         }
@@ -357,16 +324,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t acc0[32], acc1[32];
         tmem_ld_32x32b_x32(tmem + (2 * a) * kAccCols + (static_cast<uint32_t>(quarter * 32) << 16), acc0);
         tmem_ld_32x32b_x32(tmem + (2 * a + 1) * kAccCols + (static_cast<uint32_t>(quarter * 32) << 16), acc1);
+        const uint32_t ex[2] = {S.exps[s][toff], S.exps[s][kTile + toff]};
         tmem_ld_wait();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&S.acc_empty[a]);
+        if (lane == 0) {
+          mbar_arrive(&S.acc_empty[a]);
+          mbar_arrive(&S.empty[s]);
+        }
 
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
           const int p = j * kUnit + h * kTile + toff;
           const bool valid = p < nb;
-          const float sc = score_from_acc(h == 0 ? acc0 : acc1, ws, ex_cur[h]);
+          const float sc = score_from_acc(h == 0 ? acc0 : acc1, ws, ex[h]);
           float bm = valid ? sc : -INFINITY;
           bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 1));
           bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 2));
@@ -383,8 +354,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           if (scores != nullptr && valid) scores[static_cast<long long>(cur_b) * capacity + p] = sc;
         }
-        ex_cur[0] = ex_next[0];
-        ex_cur[1] = ex_next[1];
         if (warp_flag(&S.abort_flag)) break;
         it = nx;
       }
@@ -415,8 +384,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 size_t index_full_smem_bytes() { return sizeof(IndexSmem) + 1024; }
 
 cudaError_t launch_index_full(const csa2_cache& cache, const float* q, const float* w, float* blockmax,
-                              float* scores, uint32_t* hist, const CUtensorMap& ik_map, int num_sms, uint64_t wait_ns,
-                              cudaStream_t stream) {
+                              float* scores, uint32_t* hist, const CUtensorMap& ik_map, int whole_units, int num_sms,
+                              uint64_t wait_ns, cudaStream_t stream) {
   static ContextMemo attrs;
   const size_t smem = index_full_smem_bytes();
   const cudaError_t e = attrs.once([&] {
@@ -433,7 +402,7 @@ cudaError_t launch_index_full(const csa2_cache& cache, const float* q, const flo
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, index_full_kernel, cache, q, w, blockmax, scores, hist, ik_map, wait_ns);
+  return cudaLaunchKernelEx(&cfg, index_full_kernel, cache, q, w, blockmax, scores, hist, ik_map, whole_units, wait_ns);
 }
 
 }  // namespace csa2

@@ -16,7 +16,10 @@
 // 256-position units split into contiguous CTA ranges, TMA producer warp, MMA
 // warp, two epilogue warpgroups on alternate units), with:
 //   * stages of two 128-row code tiles (64-byte rows, 64-byte swizzle, 8 KB
-//     each) and their two 1 KB scale blocks (bulk copies);
+//     each) and their two 1 KB scale blocks: with pages of whole units, one
+//     256-row TMA load and one 2 KB bulk copy per unit (else one of each per
+//     tile), issued from cache rows the producer warp resolved 32 units at a
+//     time (UnitRows);
 //   * the MMA: per 128-row tile, tcgen05.cp of its scales to tensor memory,
 //     then two tcgen05.mma kind::mxf4nvf4 (K = 64 each, E4M3 block scales,
 //     M = 128 positions, N = 32 heads) into the tile's accumulator;
@@ -28,12 +31,13 @@
 
 #include "fp4.cuh"
 #include "launch.h"
+#include "scan_units.cuh"
 
 namespace csa2 {
 
 namespace {
 
-constexpr int kUnit = 2 * kTile;
+constexpr int kUnit = kScanUnit;
 constexpr int kStages = 8;
 constexpr int kAcc = 4;                    // accumulator pairs
 constexpr int kEpiGroups = 2;
@@ -57,6 +61,7 @@ struct __align__(1024) Fp4Smem {
   uint8_t q[kQBufs][kQCodeBytes];
   uint8_t qscales[kQBufs][kTileScaleBytes];
   uint32_t hist[2][kPoolHistBins / 2];
+  int rowq[32][2];                     // cache rows of the producer's current 32 units (-1: none)
   int prefix[kMaxBatchScan + 1];
   uint64_t full[kStages];
   uint64_t empty[kStages];
@@ -68,46 +73,11 @@ struct __align__(1024) Fp4Smem {
   volatile int abort_flag;
 };
 
-struct TileIter {
-  const int* prefix;
-  int batch;
-  int b, j;
-  __device__ void init(const int* pre, int nb, int g) {
-    prefix = pre;
-    batch = nb;
-    int lo = 0, hi = nb - 1;
-    while (lo < hi) {
-      const int mid = (lo + hi + 1) >> 1;
-      if (pre[mid] <= g) lo = mid;
-      else hi = mid - 1;
-    }
-    b = lo;
-    j = g - pre[lo];
-    skip_empty();
-  }
-  __device__ void skip_empty() {
-    while (b < batch && j >= prefix[b + 1] - prefix[b]) {
-      j = 0;
-      ++b;
-    }
-  }
-  __device__ void advance() {
-    ++j;
-    skip_empty();
-  }
-};
-
-__device__ __forceinline__ int next_request_with_tiles(const int* prefix, int batch, int b) {
-  ++b;
-  while (b < batch && prefix[b + 1] == prefix[b]) ++b;
-  return b;
-}
-
 __global__ void __launch_bounds__(kThreads, 1)
     index_full_fp4_kernel(const csa2_cache cache, const uint8_t* __restrict__ ik4_scales,
                           const float* __restrict__ q, const float* __restrict__ w, float* __restrict__ blockmax,
                           float* __restrict__ scores, uint32_t* __restrict__ hist,
-                          const __grid_constant__ CUtensorMap code_map, uint64_t wait_ns) {
+                          const __grid_constant__ CUtensorMap code_map, int whole_units, uint64_t wait_ns) {
   extern __shared__ uint8_t smem_raw[];
   Fp4Smem& S = *reinterpret_cast<Fp4Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int tid = threadIdx.x;
@@ -183,50 +153,56 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (n_tiles > 0) {
     if (warp == 0) {
       // ================= producer =================
-      if (lane == 0) {
-        const uint64_t policy = l2_policy_evict_first();
-        TileIter it;
-        it.init(S.prefix, B, t_begin);
-        int issued = 0;
-        long long page_key = -1;
-        int page = 0;
-        for (int i = 0; i < n_tiles; ++i) {
-          const int s = i % kStages;
-          if (!mbar_wait(&S.empty[s], ((i / kStages) & 1) ^ 1, wait_ns)) {
-            report_error(cache.err_word, CSA2_ERR_TIMEOUT, kKIndexFull, it.b, i);
-            S.abort_flag = 1;
-            break;
-          }
-          if (S.abort_flag) break;
-          int rows[2];
-          uint32_t bytes = 0;
-          for (int h = 0; h < 2; ++h) {
-            const int p0 = it.j * kUnit + h * kTile;
-            rows[h] = -1;
-            if (p0 >= capacity) continue;
-            const int pidx = static_cast<int>(static_cast<uint32_t>(p0) / page_size);
-            const long long key = static_cast<long long>(it.b) * cache.max_pages_per_req + pidx;
-            if (key != page_key) {
-              page_key = key;
-              page = cache.page_table[key];
-              if (page < 0 || page >= cache.num_pages) {
-                report_error(cache.err_word, CSA2_ERR_DEVICE_BOUNDS, kKIndexFull, it.b, p0);
-                page = 0;
+      const uint64_t policy = l2_policy_evict_first();
+      UnitRows next;   // this lane's unit of the next 32
+      next.fetch(cache, S.prefix, B, t_begin + lane, lane < n_tiles, capacity, page_size);
+      int issued = 0;   // lane 0
+      bool stop = false;
+      for (int i0 = 0; i0 < n_tiles && !stop; i0 += 32) {
+        int r[2];
+        next.rows(cache, capacity, kKIndexFull, r);
+        S.rowq[lane][0] = r[0];
+        S.rowq[lane][1] = r[1];
+        // the next 32 units' page-table loads are in flight while lane 0 issues
+        next.fetch(cache, S.prefix, B, t_begin + i0 + 32 + lane, i0 + 32 + lane < n_tiles, capacity, page_size);
+        __syncwarp();
+        if (lane == 0) {
+          const int n = min(32, n_tiles - i0);
+          for (int k = 0; k < n; ++k) {
+            const int i = i0 + k, s = i % kStages;
+            if (!mbar_wait(&S.empty[s], ((i / kStages) & 1) ^ 1, wait_ns)) {
+              report_error(cache.err_word, CSA2_ERR_TIMEOUT, kKIndexFull, -1, i);
+              S.abort_flag = 1;
+            }
+            if (S.abort_flag) {
+              stop = true;
+              break;
+            }
+            const int r0 = S.rowq[k][0], r1 = S.rowq[k][1];
+            // a tile's scale block is 1 KB at (row / 128) KB: 16-byte aligned
+            if (whole_units && r0 >= 0) {   // the unit's 256 rows and two scale blocks are consecutive
+              mbar_arrive_expect_tx(&S.full[s], 2 * (kTileCodeBytes + kTileScaleBytes));
+              tma_load_2d(S.tiles[s][0], &code_map, &S.full[s], 0, r0, policy);
+              bulk_load_1d(S.scales[s][0], ik4_scales + static_cast<long long>(r0 / kTile) * kTileScaleBytes,
+                           2 * kTileScaleBytes, &S.full[s], policy);
+            } else {
+              mbar_arrive_expect_tx(&S.full[s], ((r0 >= 0) + (r1 >= 0)) * (kTileCodeBytes + kTileScaleBytes));
+              for (int h = 0; h < 2; ++h) {
+                const int rh = h == 0 ? r0 : r1;
+                if (rh < 0) continue;
+                tma_load_2d(S.tiles[s][h], &code_map, &S.full[s], 0, rh, policy);
+                bulk_load_1d(S.scales[s][h], ik4_scales + static_cast<long long>(rh / kTile) * kTileScaleBytes,
+                             kTileScaleBytes, &S.full[s], policy);
               }
             }
-            rows[h] = page * cache.page_size + (p0 - pidx * cache.page_size);
-            bytes += kTileCodeBytes + kTileScaleBytes;
+            ++issued;
           }
-          mbar_arrive_expect_tx(&S.full[s], bytes);
-          for (int h = 0; h < 2; ++h)
-            if (rows[h] >= 0) {
-              tma_load_2d(S.tiles[s][h], &code_map, &S.full[s], 0, rows[h], policy);
-              bulk_load_1d(S.scales[s][h], ik4_scales + static_cast<long long>(rows[h] / kTile) * kTileScaleBytes,
-                           kTileScaleBytes, &S.full[s], policy);
-            }
-          ++issued;
-          it.advance();
         }
+        stop = __shfl_sync(0xffffffffu, stop, 0);
+        __syncwarp();
+      }
+      if (lane == 0) {
+        // copies still in flight (only after an abort): wait for the last one of each stage
         for (int i = issued > kStages ? issued - kStages : 0; i < issued; ++i)
           (void)mbar_wait(&S.full[i % kStages], (i / kStages) & 1, kWaitLimitNs / 2);
       }
@@ -435,7 +411,7 @@ size_t index_full_fp4_smem_bytes() { return sizeof(Fp4Smem) + 1024; }
 
 cudaError_t launch_index_full_fp4(const csa2_cache& cache, const uint8_t* ik4_scales, const float* q, const float* w,
                                   float* blockmax, float* scores, uint32_t* hist, const CUtensorMap& code_map,
-                                  int num_sms, uint64_t wait_ns, cudaStream_t stream) {
+                                  int whole_units, int num_sms, uint64_t wait_ns, cudaStream_t stream) {
   static ContextMemo attrs;
   const size_t smem = index_full_fp4_smem_bytes();
   const cudaError_t e = attrs.once([&] {
@@ -454,7 +430,7 @@ cudaError_t launch_index_full_fp4(const csa2_cache& cache, const uint8_t* ik4_sc
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, index_full_fp4_kernel, cache, ik4_scales, q, w, blockmax, scores, hist, code_map,
-                            wait_ns);
+                            whole_units, wait_ns);
 }
 
 cudaError_t launch_append_ik4(const csa2_cache& cache, uint8_t* codes, uint8_t* scales, int n_rows,

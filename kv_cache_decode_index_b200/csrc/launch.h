@@ -62,14 +62,14 @@ cudaError_t launch_compress_append(const csa2_cache& cache, int n_entries, int m
 
 size_t index_full_smem_bytes();
 cudaError_t launch_index_full(const csa2_cache& cache, const float* q, const float* w, float* blockmax,
-                              float* scores, uint32_t* hist, const CUtensorMap& ik_map, int num_sms, uint64_t wait_ns,
-                              cudaStream_t stream);
+                              float* scores, uint32_t* hist, const CUtensorMap& ik_map, int whole_units, int num_sms,
+                              uint64_t wait_ns, cudaStream_t stream);
 
 // FP4 indexer: scan and quantise-on-append.
 size_t index_full_fp4_smem_bytes();
 cudaError_t launch_index_full_fp4(const csa2_cache& cache, const uint8_t* ik4_scales, const float* q, const float* w,
                                   float* blockmax, float* scores, uint32_t* hist, const CUtensorMap& code_map,
-                                  int num_sms, uint64_t wait_ns, cudaStream_t stream);
+                                  int whole_units, int num_sms, uint64_t wait_ns, cudaStream_t stream);
 cudaError_t launch_append_ik4(const csa2_cache& cache, uint8_t* codes, uint8_t* scales, int n_rows,
                               const float* ik_new, const int32_t* req, const int32_t* pos, cudaStream_t stream);
 
