@@ -177,16 +177,19 @@ CSA2_API csa2_status csa2_compress_append(const csa2_cache* cache, int32_t n_ent
 /*
  * Histogram of the block maxima passed from csa2_index_full to
  * csa2_pool_select: uint32 [batch][CSA2_POOL_HIST_BINS], one count per
- * visible block in the bin of its score's leading 11 order-key bits (the fp32
- * bit pattern with the sign bit flipped, or all bits flipped when negative).
+ * visible block in the bin of its score's leading 12 order-key bits (the fp32
+ * bit pattern with the sign bit flipped, or all bits flipped when negative:
+ * sign, exponent and 3 mantissa bits, so that one bin spans an eighth of an
+ * octave; the block maxima of a request crowd into few octaves).
  * The scan adds to it, so it must hold zeros when the scan starts;
  * csa2_pool_select reads it and zeroes it again.  Zero it once (for instance
  * cudaMemsetAsync) before its first use.  It only saves time: a histogram
- * that does not hold exactly one count per block (not zeroed, shared by two
+ * that does not hold exactly one count per block, or whose threshold bin and
+ * the bins above it disagree with the block maxima (not zeroed, shared by two
  * scans, a scan that gave up) is detected and ignored by csa2_pool_select,
  * which then selects without it, exactly, and still zeroes it.
  */
-#define CSA2_POOL_HIST_BINS 2048
+#define CSA2_POOL_HIST_BINS 4096
 
 /*
  * csa2_index_full -- Full-mode indexer scan of every visible position of every

@@ -24,7 +24,7 @@ MODE = {"F": FULL, "Ri": REINDEX, "Ru": REUSE}
 OK, ERR_ARG, ERR_SHAPE, ERR_CUDA, ERR_DEVICE_BOUNDS, ERR_TIMEOUT, ERR_UNSUPPORTED = range(7)
 BLOCK, INDEX_HEADS, INDEX_DIM, KV_DIM, KV_CODE_BYTES, KV_SCALE_BYTES = 8, 32, 128, 512, 256, 32
 PREFILL_MAX_K, PREFILL_CANDIDATES, PREFILL_STATIC_MAX_QUERIES = 1024, 4096, 256
-POOL_HIST_BINS, RESCORE_HIST_BINS, MAX_SCORE_LAYERS = 2048, 4096, 8
+POOL_HIST_BINS, RESCORE_HIST_BINS, MAX_SCORE_LAYERS = 4096, 4096, 8
 IK4_CODE_BYTES, IK4_TILE_SCALE_BYTES, MAX_FP4_SCORE_LAYERS = 64, 1024, 4
 
 

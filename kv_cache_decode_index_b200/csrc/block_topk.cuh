@@ -35,9 +35,10 @@ struct BlockSelectSmem {
 // back to a select without head start, so it costs time, never correctness.
 // The start is written to *out by the thread that finds it (read it after a
 // barrier).
+// With bin_count, the count of the threshold's bin is stored there too.
 template <int THREADS, int NB>
 __device__ bool hist_head_start(const uint32_t (&c)[NB], int top_bin, int bits, int valid, int K, int* warp_tmp,
-                                SelectStart* out) {
+                                SelectStart* out, int* bin_count = nullptr) {
   int sum = 0;
 #pragma unroll
   for (int j = 0; j < NB; ++j) sum += static_cast<int>(c[j]);
@@ -56,6 +57,7 @@ __device__ bool hist_head_start(const uint32_t (&c)[NB], int top_bin, int bits, 
       if (a < K && K <= a + cj) {
         const uint32_t T = static_cast<uint32_t>(top_bin - j);
         *out = SelectStart{T << (32 - bits), 0xFFFFFFFFu << (32 - bits), K - a, 31 - bits, cj == K - a ? 1 : 0};
+        if (bin_count != nullptr) *bin_count = cj;
       }
       a += cj;
     }
@@ -63,13 +65,15 @@ __device__ bool hist_head_start(const uint32_t (&c)[NB], int top_bin, int bits, 
   return true;
 }
 
-// Select the K best keys of the CTA.  emit(i, r): key index i has output rank
-// r (0 <= r < min(K, valid keys)); pad(r) for the ranks past the valid keys.
-// start: optional head start (read after a barrier; may point into S.start).
-// Called by all 1024 threads.
-template <int ITEMS, class Emit, class Pad>
-__device__ void block_topk(const uint32_t (&keys)[ITEMS], int K, BlockSelectSmem& S, Emit emit, Pad pad,
-                           const SelectStart* start) {
+// The radix passes of block_topk.  On return (after a barrier) S.prefix,
+// S.mask and S.need describe the selection of the K best keys: every valid key
+// whose masked bits exceed S.prefix, and the first S.need keys (by index)
+// whose masked bits equal it.  start: optional head start (read after a
+// barrier; may point into S.start), whose need replaces K.  Called by all
+// 1024 threads.
+template <int ITEMS>
+__device__ void block_select_prefix(const uint32_t (&keys)[ITEMS], int K, BlockSelectSmem& S,
+                                    const SelectStart* start) {
   constexpr int THREADS = kBlockSelectThreads;
   constexpr int kWarps = THREADS / 32;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -154,6 +158,12 @@ __device__ void block_topk(const uint32_t (&keys)[ITEMS], int K, BlockSelectSmem
     const int c = static_cast<int>(S.hist[1023 - tid]);
     int total;
     const int above = block_exclusive_sum<THREADS>(c, S.warp_tmp, &total);
+    // fewer matching keys than needed (a head start that does not describe
+    // the keys): stop with what is above the prefix instead of passing forever
+    if (tid == 0 && total < need) {
+      S.need = 0;
+      S.done = 1;
+    }
     if (above < need && need <= above + c) {   // exactly one thread
       const uint32_t d = 1023u - static_cast<uint32_t>(tid);
       S.prefix = prefix | (d << lo);
@@ -164,6 +174,18 @@ __device__ void block_topk(const uint32_t (&keys)[ITEMS], int K, BlockSelectSmem
     }
     __syncthreads();
   }
+}
+
+// Select the K best keys of the CTA.  emit(i, r): key index i has output rank
+// r (0 <= r < min(K, valid keys)); pad(r) for the ranks past the valid keys.
+// start: optional head start (read after a barrier; may point into S.start).
+// Called by all 1024 threads.
+template <int ITEMS, class Emit, class Pad>
+__device__ void block_topk(const uint32_t (&keys)[ITEMS], int K, BlockSelectSmem& S, Emit emit, Pad pad,
+                           const SelectStart* start) {
+  constexpr int THREADS = kBlockSelectThreads;
+  const int tid = threadIdx.x;
+  block_select_prefix(keys, K, S, start);
 
   // ---- keys above the threshold prefix, and ties on it (lower index first) ----
   const uint32_t prefix = S.prefix, mask = S.mask;

@@ -220,6 +220,13 @@ __device__ void cluster_topk(const uint32_t* keys, int n_local, int K, SelectSme
       }
       const uint32_t need = static_cast<uint32_t>(S.need);
       uint32_t above = incl - sum;   // keys in digits above this lane's range
+      // fewer matching keys than needed: only a head start that does not
+      // describe the keys does that; stop with what is above the prefix
+      // rather than pass forever (the caller's start is verified)
+      if (__shfl_sync(0xffffffffu, incl, 31) < need && tid == 0) {
+        S.need = 0;
+        S.done = 1;
+      }
       if (above < need && need <= incl) {
 #pragma unroll
         for (int i = 0; i < 8; ++i) {

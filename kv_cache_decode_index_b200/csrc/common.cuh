@@ -19,8 +19,9 @@ constexpr int kKvCodeBytes = CSA2_KV_CODE_BYTES;
 constexpr int kKvScaleBytes = CSA2_KV_SCALE_BYTES;
 constexpr int kBlock = CSA2_BLOCK;              // positions per pool block
 constexpr int kTile = 128;                      // positions per MMA tile (M)
-constexpr int kPoolHistBins = CSA2_POOL_HIST_BINS;   // 2048: leading 11 bits of a block-max order key
-constexpr int kPoolHistBits = 11;
+constexpr int kPoolHistBins = CSA2_POOL_HIST_BINS;   // 4096: leading 12 bits of a block-max order key
+constexpr int kPoolHistBits = 12;
+static_assert(kPoolHistBins == 1 << kPoolHistBits, "one bin per leading-bit pattern");
 
 // kernel ids recorded in err_word[1]
 enum KernelId { kKAppend = 1, kKIndexFull = 2, kKPoolSelect = 3, kKReindex = 4, kKAttn = 5, kKPrefill = 6 };

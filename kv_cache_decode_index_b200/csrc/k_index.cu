@@ -61,8 +61,13 @@ constexpr uint32_t kTmemCols = kAcc * 2 * kAccCols;   // 256
 struct __align__(1024) IndexSmem {
   uint8_t tiles[kStages][2][kTileBytes];
   uint8_t q[kQBufs][kQBytes];
-  uint8_t exps[kStages][kUnit];        // exponent bytes of the stage's unit
-  int rowq[32][2];                     // cache rows of the producer's current 32 units (-1: none)
+  union {
+    struct {
+      uint8_t exps[kStages][kUnit];    // exponent bytes of the stage's unit
+      int rowq[32][2];                 // cache rows of the producer's current 32 units (-1: none)
+    };
+    cub::BlockScan<int, kThreads>::TempStorage scan_tmp;   // the prologue's prefix sum only
+  };
   int prefix[kMaxBatchScan + 1];       // units before request b
   uint64_t full[kStages];
   uint64_t empty[kStages];             // the MMAs' completion + the 4 epilogue warps of the unit
@@ -95,7 +100,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   // ---- tiles per request, prefix sums ----
   {
     using Scan = cub::BlockScan<int, kThreads>;
-    __shared__ typename Scan::TempStorage scan_tmp;
     int items[kScanItems];
 #pragma unroll
     for (int i = 0; i < kScanItems; ++i) {
@@ -105,7 +109,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       items[i] = (n + kUnit - 1) / kUnit;
     }
     int total;
-    Scan(scan_tmp).ExclusiveSum(items, items, total);
+    Scan(S.scan_tmp).ExclusiveSum(items, items, total);
 #pragma unroll
     for (int i = 0; i < kScanItems; ++i) {
       const int b = tid * kScanItems + i;
@@ -215,36 +219,54 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     } else if (warp == 1) {
       // ================= MMA issuer =================
+      // The issuing lane is on the scan's critical path (its instructions share
+      // an SM sub-partition with two epilogue warps): descriptors come from
+      // one base by adding stage offsets, the query's only when the request
+      // changes, and a count of the request's remaining units replaces the
+      // unit walker.
       if (lane == 0) {
         TileIter it;
         it.init(S.prefix, B, t_begin);
         int seg = 0, cur_b = it.b;
+        int left = S.prefix[cur_b + 1] - S.prefix[cur_b] - it.j;   // units of this request from here
         bool ok = mbar_wait(&S.q_full[0], 0, wait_ns);
+        const uint64_t adesc0 = sw128_kmajor_desc(smem_u32(S.tiles[0][0]));
+        uint64_t bdesc = sw128_kmajor_desc(smem_u32(S.q[0]));
+        int s = 0, a = 0;                  // i % kStages, i % kAcc
+        uint32_t ph_s = 0, ph_a = 0;       // (i / kStages) & 1, (i / kAcc) & 1
         for (int i = 0; ok && i < n_tiles; ++i) {
-          if (it.b != cur_b) {
+          if (left == 0) {   // the next request with units: the next query buffer
+            cur_b = next_request_with_tiles(S.prefix, B, cur_b);
+            left = S.prefix[cur_b + 1] - S.prefix[cur_b];
             ++seg;
-            cur_b = it.b;
             if (!mbar_wait(&S.q_full[seg % kQBufs], (seg / kQBufs) & 1, wait_ns)) { ok = false; break; }
+            bdesc = sw128_kmajor_desc(smem_u32(S.q[seg % kQBufs]));
           }
-          const int s = i % kStages, a = i % kAcc;
-          if (!mbar_wait(&S.acc_empty[a], ((i / kAcc) & 1) ^ 1, wait_ns) ||
-              !mbar_wait(&S.full[s], (i / kStages) & 1, wait_ns)) {
+          --left;
+          if (!mbar_wait(&S.acc_empty[a], ph_a ^ 1, wait_ns) || !mbar_wait(&S.full[s], ph_s, wait_ns)) {
             ok = false;
             break;
           }
           if (S.abort_flag) break;
           tc_fence_after();
-          const uint64_t bdesc = sw128_kmajor_desc(smem_u32(S.q[seg % kQBufs]));
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
-            const uint64_t adesc = sw128_kmajor_desc(smem_u32(S.tiles[s][h]));
+            // start-address field: bits 0..13 of the descriptor (address / 16)
+            const uint64_t adesc = adesc0 + static_cast<uint64_t>(((2 * s + h) * kTileBytes) >> 4);
 #pragma unroll
             for (int k = 0; k < kIndexDim / 32; ++k)
               umma_f8f6f4(tmem + (2 * a + h) * kAccCols, adesc + 2 * k, bdesc + 2 * k, kIdesc, k > 0 ? 1u : 0u);
           }
           umma_commit(&S.empty[s]);
           umma_commit(&S.acc_full[a]);
-          it.advance();
+          if (++s == kStages) {
+            s = 0;
+            ph_s ^= 1u;
+          }
+          if (++a == kAcc) {
+            a = 0;
+            ph_a ^= 1u;
+          }
         }
         if (!ok) {
           report_error(cache.err_word, CSA2_ERR_TIMEOUT, kKIndexFull, cur_b, -1);
@@ -381,6 +403,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 }  // namespace
 
+// 227 KB per block with no static shared memory (the prefix sum's scratch is
+// in the union above), 1 KB of it for aligning the struct
+static_assert(sizeof(IndexSmem) + 1024 <= 227 * 1024, "the scan's shared memory exceeds one SM");
 size_t index_full_smem_bytes() { return sizeof(IndexSmem) + 1024; }
 
 cudaError_t launch_index_full(const csa2_cache& cache, const float* q, const float* w, float* blockmax,

@@ -208,41 +208,54 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     } else if (warp == 1) {
       // ================= MMA issuer =================
+      // (the FP8 scan's issue loop: descriptors from one base, the query's
+      // only when the request changes, a unit count instead of the walker)
       if (lane == 0) {
         TileIter it;
         it.init(S.prefix, B, t_begin);
         int seg = 0, cur_b = it.b;
+        int left = S.prefix[cur_b + 1] - S.prefix[cur_b] - it.j;
         bool ok = mbar_wait(&S.q_full[0], 0, wait_ns);
         if (ok) {
           tc_fence_after();
+#pragma unroll
           for (int kh = 0; kh < 2; ++kh)
             tmem_cp_scales(tmem + kSfbCol + kh * 4, smem_u32(S.qscales[0] + kh * 512));
         }
+        const uint64_t adesc0 = sw64_kmajor_desc(smem_u32(S.tiles[0][0]));
+        const uint32_t scales0 = smem_u32(S.scales[0][0]);
+        uint64_t bdesc = sw64_kmajor_desc(smem_u32(S.q[0]));
+        uint32_t sfb = tmem + kSfbCol;
+        int s = 0, a = 0;
+        uint32_t ph_s = 0, ph_a = 0;
         for (int i = 0; ok && i < n_tiles; ++i) {
-          if (it.b != cur_b) {
+          if (left == 0) {
+            cur_b = next_request_with_tiles(S.prefix, B, cur_b);
+            left = S.prefix[cur_b + 1] - S.prefix[cur_b];
             ++seg;
-            cur_b = it.b;
             if (!mbar_wait(&S.q_full[seg % kQBufs], (seg / kQBufs) & 1, wait_ns)) { ok = false; break; }
             tc_fence_after();
+            sfb = tmem + kSfbCol + (seg % kQBufs) * 8;
+#pragma unroll
             for (int kh = 0; kh < 2; ++kh)
-              tmem_cp_scales(tmem + kSfbCol + (seg % kQBufs) * 8 + kh * 4,
-                             smem_u32(S.qscales[seg % kQBufs] + kh * 512));
+              tmem_cp_scales(sfb + kh * 4, smem_u32(S.qscales[seg % kQBufs] + kh * 512));
+            bdesc = sw64_kmajor_desc(smem_u32(S.q[seg % kQBufs]));
           }
-          const int s = i % kStages, a = i % kAcc;
-          if (!mbar_wait(&S.acc_empty[a], ((i / kAcc) & 1) ^ 1, wait_ns) ||
-              !mbar_wait(&S.full[s], (i / kStages) & 1, wait_ns)) {
+          --left;
+          if (!mbar_wait(&S.acc_empty[a], ph_a ^ 1, wait_ns) || !mbar_wait(&S.full[s], ph_s, wait_ns)) {
             ok = false;
             break;
           }
           if (S.abort_flag) break;
           tc_fence_after();
-          const uint64_t bdesc = sw64_kmajor_desc(smem_u32(S.q[seg % kQBufs]));
-          const uint32_t sfb = tmem + kSfbCol + (seg % kQBufs) * 8;
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
             const uint32_t sfa = tmem + kSfaCol + (2 * a + h) * 8;
-            for (int kh = 0; kh < 2; ++kh) tmem_cp_scales(sfa + kh * 4, smem_u32(S.scales[s][h] + kh * 512));
-            const uint64_t adesc = sw64_kmajor_desc(smem_u32(S.tiles[s][h]));
+            const uint32_t sc = scales0 + static_cast<uint32_t>((2 * s + h) * kTileScaleBytes);
+#pragma unroll
+            for (int kh = 0; kh < 2; ++kh) tmem_cp_scales(sfa + kh * 4, sc + kh * 512);
+            // start-address field: bits 0..13 of the descriptor (address / 16)
+            const uint64_t adesc = adesc0 + static_cast<uint64_t>(((2 * s + h) * kTileCodeBytes) >> 4);
 #pragma unroll
             for (int kh = 0; kh < 2; ++kh)
               umma_mxf4nvf4(tmem + (2 * a + h) * kAccCols, adesc + 2 * kh, bdesc + 2 * kh, kIdesc, sfa + kh * 4,
@@ -250,7 +263,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           umma_commit(&S.empty[s]);
           umma_commit(&S.acc_full[a]);
-          it.advance();
+          if (++s == kStages) {
+            s = 0;
+            ph_s ^= 1u;
+          }
+          if (++a == kAcc) {
+            a = 0;
+            ph_a ^= 1u;
+          }
         }
         if (!ok) {
           report_error(cache.err_word, CSA2_ERR_TIMEOUT, kKIndexFull, cur_b, -1);

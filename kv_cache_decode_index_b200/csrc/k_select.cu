@@ -19,20 +19,59 @@ namespace csa2 {
 namespace {
 
 // ------------------------------------------------------------------ pool ----
-constexpr int kPoolThreads = 512;
+constexpr int kPoolThreads = 1024;
 constexpr int kPoolKeysPerCta = 16384;
+constexpr int kPoolKpt = kPoolKeysPerCta / kPoolThreads;   // 16 consecutive keys per thread
+constexpr int kPoolGather = 8192;                          // threshold-bin keys rank 0 gathers
+constexpr int kPoolGpt = kPoolGather / kPoolThreads;       // 8 per thread (two 16-byte loads)
 
-struct PoolSmem {
-  uint32_t keys[kPoolKeysPerCta];
-  SelectSmem sel;
-  SelectStart start;
+struct PoolFinal {
+  uint32_t prefix, mask;   // the selection: masked bits above prefix, ties on it
+  int base;                // output rank of this CTA's first selection
+  int quota;               // ties this CTA takes (lowest block ids first)
+  int total;               // selections of the cluster
 };
 
-// With `hist` (the scan's per-request histogram of the leading 11 bits of the
-// block-max order keys), every CTA of the cluster reads it, finds the bin that
-// holds the pool's threshold and starts the radix select below those 11 bits;
-// the CTAs then zero their slices of it for the next scan.  A histogram that
-// does not hold exactly one count per block is ignored (select from scratch).
+struct PoolSmem {
+  union {
+    uint32_t keys[kPoolKeysPerCta];   // general path: the cluster select's keys
+    uint32_t cand[kPoolKeysPerCta];   // this CTA's keys in the threshold's bin, padded with zeros to 4
+  };
+  SelectSmem sel;
+  BlockSelectSmem bsel;               // rank 0: the select inside the bin
+  SelectStart start;
+  int bin_count;                      // keys in the threshold's bin (histogram)
+  int n_cand, n_gt;                   // this CTA's keys in / above the bin, read remotely
+  int hist_ok;                        // the counts agree with the histogram
+  int cbase[kMaxCluster + 1];         // rank 0: first gathered slot of each rank (padded lists)
+  int gt_above[kMaxCluster];          // rank 0: per rank, keys above the bin
+  int gt_bin[kMaxCluster], eq_bin[kMaxCluster];   // rank 0: per rank, bin keys above / on the final prefix
+  PoolFinal fin;                      // written by rank 0
+  uint32_t wsum[32];                  // per warp: selections (low 16 bits) and ties (high)
+};
+
+// One cluster per request; CTA `rank` holds block maxima [j0, j0 + nloc) as
+// order keys, 16 consecutive ones per thread.
+//
+// With `hist` (the scan's per-request histogram of the leading 12 bits of the
+// block-max order keys), every CTA reads it and finds the bin T that holds
+// the pool's threshold, the keys above it (all selected) and how many of T's
+// keys are still needed.  Every CTA counts its keys above T and in T; when T
+// holds at most ~8,100 keys (the maxima crowd into few bins: 2-6 % of a
+// request's blocks fall in the threshold's bin on the bench workload) it also
+// compacts its keys in T into shared memory.  After one cluster barrier every
+// CTA checks all ranks' counts against the histogram; the rank-0 CTA gathers
+// T's keys through distributed shared memory (16-byte loads), finds the exact
+// threshold among them with the block radix select (10-bit digits, block
+// barriers only), counts per rank the keys above it and on it, and writes
+// every CTA its output base and its share of the ties; after a second barrier
+// every CTA writes its selections in block order (one block prefix sum of
+// packed selection and tie counts).  Without a histogram, or with one that
+// does not describe these keys (stale, foreign), the general cluster radix
+// select runs over every key; with a larger bin it starts from the verified
+// bin.  The CTAs zero their slices of the histogram for the next scan.
+// Every step costs instructions in all 32 warps, so each is a handful of
+// instructions per thread: warp-aggregated atomics, 16-byte loads, one scan.
 __global__ void __launch_bounds__(kPoolThreads, 1)
     pool_select_kernel(const csa2_cache cache, const float* __restrict__ blockmax, uint32_t* __restrict__ hist, int P,
                        int32_t* __restrict__ pool) {
@@ -44,54 +83,294 @@ __global__ void __launch_bounds__(kPoolThreads, 1)
   const int C = static_cast<int>(cluster.num_blocks());
   const int rank = static_cast<int>(cluster.block_rank());
   const int b = blockIdx.x / C;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const uint32_t lt = (1u << lane) - 1u;
+
+  // this thread's 4 histogram bins, highest first (thread order is descending
+  // bin order); loaded before the length, which the keys' loads wait for
+  constexpr int kNB = kPoolHistBins / kPoolThreads;   // 4
+  static_assert(kNB == 4, "one 16-byte load of bins per thread");
+  const int hbase = kNB * (kPoolThreads - 1 - tid);
+  uint4 hv = make_uint4(0u, 0u, 0u, 0u);
+  if (hist != nullptr) hv = *reinterpret_cast<const uint4*>(hist + static_cast<long long>(b) * kPoolHistBins + hbase);
+
   const long long capacity = static_cast<long long>(cache.max_pages_per_req) * cache.page_size;
   const long long stride = capacity / kBlock;
-  const int n = max(0, checked_ctx_len(cache, b, capacity, kKPoolSelect, rank == 0 && threadIdx.x == 0));
+  const int n = max(0, checked_ctx_len(cache, b, capacity, kKPoolSelect, rank == 0 && tid == 0));
   const int nblk = (n + kBlock - 1) / kBlock;
-  const int per = (nblk + C - 1) / C;
+  // slices of a multiple of 4 blocks: each starts 16-byte aligned when the row does
+  const int per = (((nblk + C - 1) / C) + 3) & ~3;
   const int j0 = min(rank * per, nblk);
   const int nloc = min(per, nblk - j0);
-  const float* src = blockmax + b * stride + j0;
-  for (int base = 0; base < nloc; base += kPoolThreads * 8) {   // 8 independent loads per thread in flight
-    float v[8];
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int i = base + u * kPoolThreads + threadIdx.x;
-      v[u] = i < nloc ? src[i] : 0.0f;
-    }
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int i = base + u * kPoolThreads + threadIdx.x;
-      if (i < nloc) S.keys[i] = order_key(v[u]);
-    }
-  }
-  const SelectStart* start = nullptr;
-  if (hist != nullptr) {
-    // this thread's 4 bins, highest first: thread order is descending bin order
-    constexpr int kNB = kPoolHistBins / kPoolThreads;   // 4
-    const int base = kNB * (kPoolThreads - 1 - static_cast<int>(threadIdx.x));
-    const uint4* hb = reinterpret_cast<const uint4*>(hist + static_cast<long long>(b) * kPoolHistBins + base);
-    uint32_t c[kNB];
-#pragma unroll
-    for (int i = 0; i < kNB / 4; ++i) {
-      const uint4 v = hb[i];
-      c[kNB - 1 - 4 * i] = v.x;
-      c[kNB - 2 - 4 * i] = v.y;
-      c[kNB - 3 - 4 * i] = v.z;
-      c[kNB - 4 - 4 * i] = v.w;
-    }
-    if (hist_head_start<kPoolThreads, kNB>(c, base + kNB - 1, kPoolHistBits, nblk, P, S.sel.warp_tmp, &S.start))
-      start = &S.start;
-  }
-  __syncthreads();   // the keys (and a head start) are in shared memory
   int32_t* out = pool + static_cast<long long>(b) * P;
-  cluster_topk<kPoolThreads>(
-      S.keys, nloc, P, S.sel, [&](int i, int r) { out[r] = j0 + i; }, [&](int r) { out[r] = -1; }, start);
-  if (hist != nullptr) {   // every CTA has read the histogram before the select's last cluster barrier
-    const int per = kPoolHistBins / C;
-    uint4* hz = reinterpret_cast<uint4*>(hist + static_cast<long long>(b) * kPoolHistBins + rank * per);
-    for (int i = threadIdx.x; i < per / 4; i += kPoolThreads) hz[i] = make_uint4(0u, 0u, 0u, 0u);
+
+  // ---- keys [16 tid, 16 tid + 16): all loads in flight at once ----
+  uint32_t key[kPoolKpt];
+  {
+    const float* src = blockmax + b * stride + j0;
+    const bool vec = (reinterpret_cast<uintptr_t>(src) & 15u) == 0u;
+    const int i0 = kPoolKpt * tid;
+    float f[kPoolKpt];
+    if (vec && i0 + kPoolKpt <= nloc) {
+#pragma unroll
+      for (int u = 0; u < kPoolKpt / 4; ++u) {
+        const float4 v = *reinterpret_cast<const float4*>(src + i0 + 4 * u);
+        f[4 * u] = v.x;
+        f[4 * u + 1] = v.y;
+        f[4 * u + 2] = v.z;
+        f[4 * u + 3] = v.w;
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < kPoolKpt; ++j) f[j] = i0 + j < nloc ? src[i0 + j] : 0.0f;
+    }
+#pragma unroll
+    for (int j = 0; j < kPoolKpt; ++j) key[j] = i0 + j < nloc ? order_key(f[j]) : 0u;
   }
+
+  // ---- head start from the histogram (the same in every CTA) ----
+  bool head = false;
+  if (hist != nullptr) {
+    const uint32_t c[kNB] = {hv.w, hv.z, hv.y, hv.x};
+    if (tid == 0) S.bin_count = kPoolGather + 1;
+    head = hist_head_start<kPoolThreads, kNB>(c, hbase + kNB - 1, kPoolHistBits, nblk, P, S.sel.warp_tmp, &S.start,
+                                              &S.bin_count);
+  }
+  if (tid == 0) {
+    S.n_cand = 0;
+    S.n_gt = 0;
+  }
+  __syncthreads();   // the head start, the counters
+  const bool all_selected = head && S.start.done && S.start.mask == 0u;   // nblk <= P
+  const bool counted = head && !all_selected;
+  // the padded lists of all ranks fit the gather (each pads at most 3 zeros)
+  const bool compact = counted && S.bin_count <= kPoolGather - 3 * C;
+  const uint32_t t_prefix = S.start.prefix, t_mask = S.start.mask;
+
+  if (counted) {
+    // this CTA's keys above the bin and in it: one atomic per warp each
+    int gt = 0, nc = 0;
+#pragma unroll
+    for (int j = 0; j < kPoolKpt; ++j) {
+      const uint32_t km = key[j] & t_mask;
+      gt += (key[j] != 0u && km > t_prefix) ? 1 : 0;
+      nc += (key[j] != 0u && km == t_prefix) ? 1 : 0;
+    }
+    int incl = nc;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    int wbase = 0;
+    if (lane == 31 && incl != 0) wbase = atomicAdd(&S.n_cand, incl);
+    wbase = __shfl_sync(0xffffffffu, wbase, 31);
+    gt = __reduce_add_sync(0xffffffffu, gt);
+    if (lane == 0 && gt != 0) atomicAdd(&S.n_gt, gt);
+    if (compact && nc != 0) {   // slots < 16384: at most one per key of this CTA
+      int slot = wbase + incl - nc;
+#pragma unroll
+      for (int j = 0; j < kPoolKpt; ++j)
+        if (key[j] != 0u && (key[j] & t_mask) == t_prefix) S.cand[slot++] = key[j];
+    }
+    __syncthreads();
+    if (compact && tid < 3) {   // zeros up to a multiple of 4 (no key is 0)
+      const int nc_all = S.n_cand;
+      const int pad = (nc_all + 3) & ~3;
+      if (nc_all + tid < pad) S.cand[nc_all + tid] = 0u;
+    }
+  }
+  cluster.sync();   // #1: every CTA's counts and bin keys; every CTA has read the histogram
+
+  if (hist != nullptr) {   // zero this CTA's slice of the histogram for the next scan
+    const int hper = kPoolHistBins / C;
+    uint4* hz = reinterpret_cast<uint4*>(hist + static_cast<long long>(b) * kPoolHistBins + rank * hper);
+    for (int i = tid; i < hper / 4; i += kPoolThreads) hz[i] = make_uint4(0u, 0u, 0u, 0u);
+  }
+
+  if (all_selected) {   // every block is in the pool, in block order
+#pragma unroll
+    for (int j = 0; j < kPoolKpt; ++j) {
+      const int i = kPoolKpt * tid + j;
+      if (i < nloc) out[j0 + i] = j0 + i;
+    }
+    if (rank == 0)
+      for (int r = nblk + tid; r < P; r += kPoolThreads) out[r] = -1;
+    return;   // no shared memory of this CTA is read remotely on this path
+  }
+
+  bool hist_ok = false;
+  if (counted) {
+    // the counts of all ranks against the histogram (every CTA reads them)
+    if (warp == 0) {
+      const int nc = lane < C ? cluster.map_shared_rank(&S.n_cand, lane)[0] : 0;
+      const int ng = lane < C ? cluster.map_shared_rank(&S.n_gt, lane)[0] : 0;
+      const int ncp = (nc + 3) & ~3;   // padded list
+      int incl = ncp;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      const int sum_c = __reduce_add_sync(0xffffffffu, nc);
+      const int sum_g = __reduce_add_sync(0xffffffffu, ng);
+      if (lane < C) {
+        S.cbase[lane] = incl - ncp;
+        S.gt_above[lane] = ng;
+        S.gt_bin[lane] = 0;
+        S.eq_bin[lane] = 0;
+      }
+      if (lane == C - 1) S.cbase[C] = incl;
+      if (lane == 0) S.hist_ok = (sum_c == S.bin_count && sum_g == P - S.start.need) ? 1 : 0;
+    }
+    __syncthreads();
+    hist_ok = S.hist_ok != 0;
+  }
+
+  if (!(hist_ok && compact)) {
+    // ---- general path: cluster radix select over every key ----
+#pragma unroll
+    for (int u = 0; u < kPoolKpt / 4; ++u)
+      *reinterpret_cast<uint4*>(&S.keys[kPoolKpt * tid + 4 * u]) =
+          make_uint4(key[4 * u], key[4 * u + 1], key[4 * u + 2], key[4 * u + 3]);
+    __syncthreads();
+    // the head start only from a histogram whose threshold bin and the bins
+    // above it hold exactly the keys it says (a start from a bin without the
+    // keys it claims would leave the radix passes nothing to select)
+    const SelectStart* start = hist_ok ? &S.start : nullptr;
+    cluster_topk<kPoolThreads>(
+        S.keys, nloc, P, S.sel, [&](int i, int r) { out[r] = j0 + i; }, [&](int r) { out[r] = -1; }, start);
+    return;
+  }
+
+  // ---- rank 0: the threshold inside the bin, and every rank's share ----
+  if (rank == 0) {
+    const int M = S.cbase[C];   // padded total <= kPoolGather
+    constexpr int kQ = kPoolGpt / 4;   // 16-byte loads per thread
+    uint32_t g[kPoolGpt];
+    int rq[kQ];
+    {
+      int p[kQ];
+#pragma unroll
+      for (int q = 0; q < kQ; ++q) {
+        p[q] = kPoolGpt * tid + 4 * q;
+        rq[q] = 0;
+      }
+      for (int r = 1; r < C; ++r) {   // rank of each load: independent shared-memory reads
+        const int cb = S.cbase[r];
+#pragma unroll
+        for (int q = 0; q < kQ; ++q) rq[q] = cb <= p[q] ? r : rq[q];
+      }
+      uint4 v[kQ];
+#pragma unroll
+      for (int q = 0; q < kQ; ++q)
+        v[q] = (!S.start.done && p[q] < M)
+                   ? *reinterpret_cast<const uint4*>(cluster.map_shared_rank(&S.cand[0], rq[q]) + (p[q] - S.cbase[rq[q]]))
+                   : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+      for (int q = 0; q < kQ; ++q) {
+        g[4 * q] = v[q].x;
+        g[4 * q + 1] = v[q].y;
+        g[4 * q + 2] = v[q].z;
+        g[4 * q + 3] = v[q].w;
+      }
+    }
+    block_select_prefix(g, S.start.need, S.bsel, &S.start);   // ends with a barrier
+    const uint32_t f_prefix = S.bsel.prefix, f_mask = S.bsel.mask;
+    const int f_need = S.bsel.need;
+    if (!S.start.done) {
+      // per rank: the bin's keys above the final prefix and on it (one atomic
+      // per group of lanes whose loads came from the same rank)
+#pragma unroll
+      for (int q = 0; q < kQ; ++q) {
+        int ga = 0, eq = 0;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const uint32_t k = g[4 * q + e], km = k & f_mask;
+          ga += (k != 0u && km > f_prefix) ? 1 : 0;
+          eq += (k != 0u && km == f_prefix) ? 1 : 0;
+        }
+        const uint32_t same = __match_any_sync(0xffffffffu, rq[q]);
+        ga = __reduce_add_sync(same, ga);
+        eq = __reduce_add_sync(same, eq);
+        if ((same & lt) == 0u) {   // the group's lowest lane
+          if (ga != 0) atomicAdd(&S.gt_bin[rq[q]], ga);
+          if (eq != 0) atomicAdd(&S.eq_bin[rq[q]], eq);
+        }
+      }
+    }
+    __syncthreads();
+    if (warp == 0) {
+      // whole bin taken: every bin key ties on the bin's prefix
+      const int eq = lane < C ? (S.start.done ? cluster.map_shared_rank(&S.n_cand, lane)[0] : S.eq_bin[lane]) : 0;
+      const int above = lane < C ? S.gt_above[lane] + S.gt_bin[lane] : 0;
+      int eq_incl = eq;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, eq_incl, o);
+        if (lane >= o) eq_incl += y;
+      }
+      const int quota = max(0, min(f_need - (eq_incl - eq), eq));
+      const int sel = above + quota;
+      int sel_incl = sel;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, sel_incl, o);
+        if (lane >= o) sel_incl += y;
+      }
+      const int total = __shfl_sync(0xffffffffu, sel_incl, 31);
+      if (lane < C)
+        *cluster.map_shared_rank(&S.fin, lane) = PoolFinal{f_prefix, f_mask, sel_incl - sel, quota, total};
+    }
+  }
+  cluster.sync();   // #2: every CTA's share is written; no remote reads after this
+
+  // ---- this CTA's selections, in block order (thread order) ----
+  const PoolFinal fin = S.fin;
+  uint32_t c = 0;   // selections (low 16 bits) and ties (high 16 bits) of this thread's keys
+#pragma unroll
+  for (int j = 0; j < kPoolKpt; ++j) {
+    const uint32_t km = key[j] & fin.mask;
+    c += (key[j] != 0u && km > fin.prefix) ? 1u : 0u;
+    c += (key[j] != 0u && km == fin.prefix) ? 0x10000u : 0u;
+  }
+  uint32_t incl = c;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) S.wsum[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    const uint32_t v = S.wsum[lane];
+    uint32_t x = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    S.wsum[lane] = x - v;
+  }
+  __syncthreads();
+  if (c != 0u) {
+    const uint32_t run = S.wsum[warp] + incl - c;
+    int sel_b = static_cast<int>(run & 0xFFFFu), tie_b = static_cast<int>(run >> 16);
+#pragma unroll
+    for (int j = 0; j < kPoolKpt; ++j) {
+      const uint32_t km = key[j] & fin.mask;
+      const int i = kPoolKpt * tid + j;
+      if (key[j] != 0u && km > fin.prefix) {
+        out[fin.base + sel_b + min(tie_b, fin.quota)] = j0 + i;
+        ++sel_b;
+      } else if (key[j] != 0u && km == fin.prefix) {
+        if (tie_b < fin.quota) out[fin.base + sel_b + tie_b] = j0 + i;
+        ++tie_b;
+      }
+    }
+  }
+  if (rank == 0)
+    for (int r = fin.total + tid; r < P; r += kPoolThreads) out[r] = -1;
 }
 
 // --------------------------------------------------------------- reindex ----

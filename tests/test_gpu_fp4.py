@@ -11,6 +11,9 @@ from oracle import csa2 as C
 from oracle import formats as F
 from tests import gpu_util as U
 
+# the pool histogram bins the leading 12 bits of a block max's order key
+HIST_SHIFT = 20
+
 pytestmark = pytest.mark.gpu
 
 
@@ -102,7 +105,7 @@ def test_index_full_fp4_scores_ragged(csa2):
         assert np.all(np.isnan(bm[b, nb:]))
         keys = bm[b, :nb].view(np.uint32).astype(np.uint64)
         keys = np.where(keys & 0x80000000, ~keys & 0xFFFFFFFF, keys | 0x80000000)
-        np.testing.assert_array_equal(h[b], np.bincount(keys >> 21, minlength=csa2.POOL_HIST_BINS))
+        np.testing.assert_array_equal(h[b], np.bincount(keys >> HIST_SHIFT, minlength=1 << (32 - HIST_SHIFT)))
     print(f"FP4 scan: max relative score error {worst:.3e}")
 
 

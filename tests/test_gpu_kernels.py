@@ -12,6 +12,9 @@ from oracle import csa2 as C
 from oracle import formats as F
 from tests import gpu_util as U
 
+# the pool histogram bins the leading 12 bits of a block max's order key
+HIST_SHIFT = 20
+
 pytestmark = pytest.mark.gpu
 
 
@@ -224,10 +227,10 @@ def test_index_full_scores_ragged(csa2):
                                             ([1048576], 2048, "all_equal")])
 def test_pool_select_bitexact(csa2, lengths, P, kind):
     """Synthetic block maxima with many ties (and negative values), fed to both.
-    "on_sample_grid": the largest maxima sit exactly on the evenly spaced
-    sample, so the sampled threshold admits fewer blocks than the pool needs
-    and the kernel must take its exact fallback; "all_equal": every block ties
-    (more candidates than the fast path holds)."""
+    "on_sample_grid": 4096 evenly spaced blocks far above the rest, in a few
+    histogram bins; "all_equal": every block ties (the threshold's bin holds
+    every block: more keys than the kernel gathers in one CTA, so it takes
+    the general cluster select)."""
     rng = np.random.default_rng(len(lengths) * 1000 + P)
     B = len(lengths)
     page = 4096
@@ -257,12 +260,19 @@ def test_pool_select_bitexact(csa2, lengths, P, kind):
     # block maxima (stale) is ignored, with the same result
     hist = np.zeros((B, csa2.POOL_HIST_BINS), np.int64)
     for b, n in enumerate(lengths):
-        hist[b] = np.bincount(_order_keys(vals[b, :-(-n // 8)]) >> 21, minlength=csa2.POOL_HIST_BINS)
+        hist[b] = np.bincount(_order_keys(vals[b, :-(-n // 8)]) >> HIST_SHIFT, minlength=1 << (32 - HIST_SHIFT))
     th = torch.from_numpy(hist.astype(np.int32)).to(dev)
     pool_h = csa2.pool_select(cache, tv, P, hist=th).cpu().numpy()
     np.testing.assert_array_equal(pool_h, pool)
     assert int(th.abs().sum()) == 0
     th = torch.from_numpy((hist + rng.integers(0, 3, hist.shape)).astype(np.int32)).to(dev)
+    np.testing.assert_array_equal(csa2.pool_select(cache, tv, P, hist=th).cpu().numpy(), pool)
+    assert int(th.abs().sum()) == 0
+    # the right total in the wrong bin (every count in the top bin): the
+    # per-CTA counts of the bin's keys contradict it, and the result is exact
+    wrong = np.zeros_like(hist)
+    wrong[:, -1] = hist.sum(axis=1)
+    th = torch.from_numpy(wrong.astype(np.int32)).to(dev)
     np.testing.assert_array_equal(csa2.pool_select(cache, tv, P, hist=th).cpu().numpy(), pool)
     assert int(th.abs().sum()) == 0
     assert csa2.get_error(cache)[0] == csa2.OK
@@ -278,7 +288,7 @@ def _order_keys(v):
 
 def test_scan_histogram_drives_the_pool(csa2):
     """The scan's histogram holds one count per visible block in the bin of
-    its block max's leading 11 key bits; the pool selected from it equals the
+    its block max's leading 12 key bits; the pool selected from it equals the
     pool selected without it, and the histogram is zero again afterwards."""
     wl = W.scaled(W.WORKLOADS["group_64k_b8"], batch=3, page_size=512, shuffle_pages=True)
     lengths = [65536, 40001, 777]
@@ -291,7 +301,7 @@ def test_scan_histogram_drives_the_pool(csa2):
     h = hist.cpu().numpy().astype(np.int64)
     bmh = bm.cpu().numpy()
     for b, n in enumerate(lengths):
-        want = np.bincount(_order_keys(bmh[b, :-(-n // 8)]) >> 21, minlength=csa2.POOL_HIST_BINS)
+        want = np.bincount(_order_keys(bmh[b, :-(-n // 8)]) >> HIST_SHIFT, minlength=1 << (32 - HIST_SHIFT))
         np.testing.assert_array_equal(h[b], want, err_msg=f"request {b}")
     pool_h = csa2.pool_select(cache, bm, 512, hist=hist)
     assert int(hist.abs().sum()) == 0
