@@ -119,7 +119,8 @@ def measured_peak_hbm():
 
 def scan_kernel_hash(fp4=False):
     h = hashlib.sha256()
-    for name in (("k_index_fp4.cu", "fp4.cuh", "common.cuh") if fp4 else ("k_index.cu", "index_common.cuh", "common.cuh")):
+    names = ("k_index_fp4.cu", "fp4.cuh") if fp4 else ("k_index.cu", "index_common.cuh")
+    for name in names + ("scan_units.cuh", "common.cuh"):
         with open(os.path.join(ROOT, "kv_cache_decode_index_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
