@@ -19,7 +19,7 @@ constexpr int kBlockSelectThreads = 1024;
 
 struct BlockSelectSmem {
   uint32_t hist[1024];
-  int warp_tmp[32];
+  int warp_tmp[64];
   uint32_t wstat[32][3];
   SelectStart start;   // a head start staged by the caller (optional)
   uint32_t prefix, mask;
@@ -36,14 +36,22 @@ struct BlockSelectSmem {
 // The start is written to *out by the thread that finds it (read it after a
 // barrier).
 // With bin_count, the count of the threshold's bin is stored there too.
-template <int THREADS, int NB>
+// With kLocalValid, `valid` is this thread's count of valid keys, summed over
+// the block in the same prefix sum as the bins (warp_tmp: 2 * THREADS / 32).
+template <int THREADS, int NB, bool kLocalValid = false>
 __device__ bool hist_head_start(const uint32_t (&c)[NB], int top_bin, int bits, int valid, int K, int* warp_tmp,
                                 SelectStart* out, int* bin_count = nullptr) {
   int sum = 0;
 #pragma unroll
   for (int j = 0; j < NB; ++j) sum += static_cast<int>(c[j]);
-  int total;
-  const int above = block_exclusive_sum<THREADS>(sum, warp_tmp, &total);
+  int total, above;
+  if constexpr (kLocalValid) {
+    int valid_total;
+    above = block_exclusive_sum2<THREADS>(sum, valid, warp_tmp, &total, &valid_total).x;
+    valid = valid_total;
+  } else {
+    above = block_exclusive_sum<THREADS>(sum, warp_tmp, &total);
+  }
   if (total != valid) return false;
   if (valid <= K) {   // everything valid is selected
     if (threadIdx.x == 0) *out = SelectStart{0u, 0u, valid, -1, 1};
@@ -198,8 +206,8 @@ __device__ void block_topk(const uint32_t (&keys)[ITEMS], int K, BlockSelectSmem
     eq += (k != 0u && km == prefix) ? 1 : 0;
   }
   int gt_total, eq_total;
-  const int gt_before = block_exclusive_sum<THREADS>(gt, S.warp_tmp, &gt_total);
-  const int eq_before = block_exclusive_sum<THREADS>(eq, S.warp_tmp, &eq_total);
+  const int2 before = block_exclusive_sum2<THREADS>(gt, eq, S.warp_tmp, &gt_total, &eq_total);
+  const int gt_before = before.x, eq_before = before.y;
   int take = max(0, min(need - eq_before, eq));   // ties this thread takes
   int r = gt_before + min(eq_before, need);
 #pragma unroll

@@ -85,6 +85,50 @@ __device__ __forceinline__ int block_exclusive_sum(int v, int* warp_tmp, int* su
   return x - v + (warp > 0 ? warp_tmp[warp - 1] : 0);
 }
 
+// Two exclusive block-wide prefix sums at once, sharing the barriers of one
+// (warp_tmp holds 2 * THREADS / 32 ints).  *sa, *sb get the totals.
+template <int THREADS>
+__device__ __forceinline__ int2 block_exclusive_sum2(int a, int b, int* warp_tmp, int* sa, int* sb) {
+  constexpr int kW = THREADS / 32;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int x = a, y = b;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int xa = __shfl_up_sync(0xffffffffu, x, o);
+    const int yb = __shfl_up_sync(0xffffffffu, y, o);
+    if (lane >= o) {
+      x += xa;
+      y += yb;
+    }
+  }
+  __syncthreads();   // warp_tmp reuse guard
+  if (lane == 31) {
+    warp_tmp[warp] = x;
+    warp_tmp[kW + warp] = y;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    int t = lane < kW ? warp_tmp[lane] : 0, u = lane < kW ? warp_tmp[kW + lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int ta = __shfl_up_sync(0xffffffffu, t, o);
+      const int ub = __shfl_up_sync(0xffffffffu, u, o);
+      if (lane >= o) {
+        t += ta;
+        u += ub;
+      }
+    }
+    if (lane < kW) {   // inclusive warp totals
+      warp_tmp[lane] = t;
+      warp_tmp[kW + lane] = u;
+    }
+  }
+  __syncthreads();
+  *sa = warp_tmp[kW - 1];
+  *sb = warp_tmp[2 * kW - 1];
+  return make_int2(x - a + (warp > 0 ? warp_tmp[warp - 1] : 0), y - b + (warp > 0 ? warp_tmp[kW + warp - 1] : 0));
+}
+
 // Select the K best of the cluster's candidates.  emit(i, r) is called for the
 // local candidate i that has output rank r (0 <= r < min(K, total)); pad(r) for
 // r in [total, K) by the cluster's rank-0 CTA.  Must be called by all THREADS

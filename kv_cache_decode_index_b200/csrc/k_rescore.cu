@@ -373,10 +373,8 @@ __global__ void __launch_bounds__(kBlockSelectThreads, 1)
   int valid = 0;
 #pragma unroll
   for (int i = 0; i < ITEMS; ++i) valid += k[i] != 0u ? 1 : 0;
-  int n_valid;
-  (void)block_exclusive_sum<kBlockSelectThreads>(valid, S.warp_tmp, &n_valid);
-  const bool ok = hist_head_start<kBlockSelectThreads, 4>(c, 4 * (kBlockSelectThreads - 1 - tid) + 3, kRsHistBits,
-                                                          n_valid, K, S.warp_tmp, &S.start);
+  const bool ok = hist_head_start<kBlockSelectThreads, 4, true>(c, 4 * (kBlockSelectThreads - 1 - tid) + 3,
+                                                                kRsHistBits, valid, K, S.warp_tmp, &S.start);
   int32_t* dst = out.topk[l] + static_cast<long long>(b) * K;
   block_topk<ITEMS>(
       k, K, S, [&](int i, int r) { dst[r] = pool_ids[i / kBlock] * kBlock + (i % kBlock); },

@@ -87,31 +87,33 @@ __global__ void __launch_bounds__(kPoolThreads, 1)
   const uint32_t lt = (1u << lane) - 1u;
 
   // this thread's 4 histogram bins, highest first (thread order is descending
-  // bin order); loaded before the length, which the keys' loads wait for
+  // bin order)
   constexpr int kNB = kPoolHistBins / kPoolThreads;   // 4
   static_assert(kNB == 4, "one 16-byte load of bins per thread");
   const int hbase = kNB * (kPoolThreads - 1 - tid);
   uint4 hv = make_uint4(0u, 0u, 0u, 0u);
   if (hist != nullptr) hv = *reinterpret_cast<const uint4*>(hist + static_cast<long long>(b) * kPoolHistBins + hbase);
 
+  // Slices of the request's block-max row by its capacity (a multiple of 4
+  // blocks each: every slice starts 16-byte aligned when the row does), so
+  // that the keys' loads need not wait for the length; keys past the length
+  // are masked once it arrives.
   const long long capacity = static_cast<long long>(cache.max_pages_per_req) * cache.page_size;
-  const long long stride = capacity / kBlock;
-  const int n = max(0, checked_ctx_len(cache, b, capacity, kKPoolSelect, rank == 0 && tid == 0));
-  const int nblk = (n + kBlock - 1) / kBlock;
-  // slices of a multiple of 4 blocks: each starts 16-byte aligned when the row does
-  const int per = (((nblk + C - 1) / C) + 3) & ~3;
-  const int j0 = min(rank * per, nblk);
-  const int nloc = min(per, nblk - j0);
+  const int stride = static_cast<int>(capacity / kBlock);   // <= 16 x 16,384 (checked on the host)
+  const int per = (((stride + C - 1) / C) + 3) & ~3;
+  const int j0 = min(rank * per, stride);
+  const int ncap = min(per, stride - j0);
   int32_t* out = pool + static_cast<long long>(b) * P;
 
   // ---- keys [16 tid, 16 tid + 16): all loads in flight at once ----
   uint32_t key[kPoolKpt];
+  const int i0 = kPoolKpt * tid;
+  int n;
   {
-    const float* src = blockmax + b * stride + j0;
+    const float* src = blockmax + static_cast<long long>(b) * stride + j0;
     const bool vec = (reinterpret_cast<uintptr_t>(src) & 15u) == 0u;
-    const int i0 = kPoolKpt * tid;
     float f[kPoolKpt];
-    if (vec && i0 + kPoolKpt <= nloc) {
+    if (vec && i0 + kPoolKpt <= ncap) {
 #pragma unroll
       for (int u = 0; u < kPoolKpt / 4; ++u) {
         const float4 v = *reinterpret_cast<const float4*>(src + i0 + 4 * u);
@@ -122,11 +124,16 @@ __global__ void __launch_bounds__(kPoolThreads, 1)
       }
     } else {
 #pragma unroll
-      for (int j = 0; j < kPoolKpt; ++j) f[j] = i0 + j < nloc ? src[i0 + j] : 0.0f;
+      for (int j = 0; j < kPoolKpt; ++j) f[j] = i0 + j < ncap ? src[i0 + j] : 0.0f;
     }
+    n = max(0, checked_ctx_len(cache, b, capacity, kKPoolSelect, rank == 0 && tid == 0));
 #pragma unroll
-    for (int j = 0; j < kPoolKpt; ++j) key[j] = i0 + j < nloc ? order_key(f[j]) : 0u;
+    for (int j = 0; j < kPoolKpt; ++j) key[j] = order_key(f[j]);
   }
+  const int nblk = (n + kBlock - 1) / kBlock;
+  const int nloc = max(0, min(ncap, nblk - j0));   // valid keys of this CTA
+#pragma unroll
+  for (int j = 0; j < kPoolKpt; ++j) key[j] = i0 + j < nloc ? key[j] : 0u;
 
   // ---- head start from the histogram (the same in every CTA) ----
   bool head = false;
