@@ -16,26 +16,20 @@ __device__ __forceinline__ float e4m3_value(uint32_t c) {
   return E ? __uint_as_float(((E + 120u) << 23) | (M << 20)) : static_cast<float>(M) * 0.001953125f;
 }
 
-// E4M3 code nearest to amax / 6 (ties to the even code, saturating at 448).
-// Found as the largest code c with 6 * value(c) <= amax, then moved up when
-// amax lies above the midpoint 3 * (value(c) + value(c + 1)) (or on it with
-// c odd).
+// E4M3 code nearest to amax / 6 (ties to the even code, saturating at 448),
+// from the correctly rounded fp32 quotient and the hardware conversion (round
+// to nearest even, saturating).  The rounded quotient lies on the same side
+// of every E4M3 midpoint as the exact one: a midpoint m has at most 5
+// significant bits, so 6m is an fp32 value; amax either equals 6m (and the
+// quotient is m exactly) or differs from it by at least one ulp of 6m's
+// binade, which is more than 6 times the quotient's rounding error (half an
+// ulp of m's binade, a quarter to an eighth of 6m's).  NaN gives code 0.
 __device__ __forceinline__ uint32_t e4m3_code_of_sixth(float amax) {
-  int lo = 0, hi = 126;
-#pragma unroll
-  for (int it = 0; it < 7; ++it) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (lo < hi) {
-      if (6.0f * e4m3_value(static_cast<uint32_t>(mid)) <= amax) lo = mid;
-      else hi = mid - 1;
-    }
-  }
-  uint32_t c = static_cast<uint32_t>(lo);
-  if (c < 126u) {
-    const float mid6 = 3.0f * (e4m3_value(c) + e4m3_value(c + 1u));
-    if (amax > mid6 || (amax == mid6 && (c & 1u))) c += 1u;
-  }
-  return c;
+  if (!(amax >= 0.0f)) return 0u;
+  const float x = amax / 6.0f;
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(0.0f), "f"(x));   // low byte: x
+  return r & 0xFFu;
 }
 
 // E2M1 code (0..15) of x under scale s > 0: nearest grid value of |x| / s,
