@@ -109,6 +109,48 @@ __global__ void __launch_bounds__(kSThreads, 2)
   const uint32_t sfb_col = sf_inside ? static_cast<uint32_t>(ncols + 8) : sfa_col + 8u * n_acc;
   const long long key_stride = static_cast<long long>(P) * kBlock;
 
+  // ---- independent of the preceding launch (it selects the pool): the
+  // barriers, tensor memory and the layers' queries, overlapping its tail ----
+  if (tid == 0) {
+    for (int s = 0; s < kSStages; ++s) {
+      mbar_init(&S.full[s], 1);
+      mbar_init(&S.empty[s], 1);
+    }
+    for (int a = 0; a < kSMaxAcc; ++a) {
+      mbar_init(&S.acc_full[a], 1);
+      mbar_init(&S.acc_empty[a], 4);
+    }
+    mbar_init(&S.q_full, 4);
+    mbar_init(&S.drain, 1);
+    S.abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&S.tmem_base, kSTmemCols);
+    tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) tma_prefetch_map(&blk_map);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = S.tmem_base;
+  if (warp >= 2) {   // the epilogue warps: every layer's query codes and head weights
+    const int ew = warp - 2;
+    for (int l = 0; l < L; ++l) {
+      const float* ql = io.q[l] + static_cast<long long>(b) * kIndexHeads * kIndexDim;
+      const float* wl = io.w[l] + static_cast<long long>(b) * kIndexHeads;
+      if constexpr (kFp4) {
+        prepare_query_fp4(ql, S.qtile[0], S.qscale, kIndexHeads * l, ew, lane);
+        if (lane < 8) S.ws[l][ew * 8 + lane] = wl[ew * 8 + lane];
+      } else {
+        prepare_query_part(ql, wl, S.qtile[l], S.ws[l], ew, lane);
+      }
+    }
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&S.q_full);
+  }
+
   pdl_wait();                 // the pool of the preceding launch is complete
   pdl_launch_dependents();
   const int n_raw = checked_ctx_len(cache, b, capacity, kKReindex, c == 0 && tid == 0);
@@ -116,12 +158,12 @@ __global__ void __launch_bounds__(kSThreads, 2)
     for (int l = 0; l < L; ++l)
       for (int i = tid; i < nblk * kBlock; i += kSThreads)
         keys[(static_cast<long long>(b) * L + l) * key_stride + slot0 * kBlock + i] = 0u;
-    return;
   }
-  const int n = n_raw;
+  const int n = max(n_raw, 0);
+  const int n_work = n_raw < 0 ? 0 : n_tiles;   // tiles this CTA scores
 
   // ---- this CTA's pool blocks: block id -> page -> row and exponent bytes ----
-  for (int i = tid; i < nblk; i += kSThreads) {
+  for (int i = tid; i < (n_raw < 0 ? 0 : nblk); i += kSThreads) {
     const int j = pool[static_cast<long long>(b) * P + slot0 + i];
     int row = -1;
     uint64_t ex = 0x7F7F7F7F7F7F7F7Full;
@@ -148,7 +190,7 @@ __global__ void __launch_bounds__(kSThreads, 2)
     __syncthreads();
     // all of a thread's loads are issued before any is used
     constexpr int kWords = (kSMaxTiles * kSBlocksPerTile * kBlock * 2 + kSThreads - 1) / kSThreads;
-    const int n_words = n_tiles * kSBlocksPerTile * kBlock * 2;
+    const int n_words = n_work * kSBlocksPerTile * kBlock * 2;   // none after a corrupt length
     uint32_t v[kWords];
 #pragma unroll
     for (int u = 0; u < kWords; ++u) {
@@ -169,31 +211,9 @@ __global__ void __launch_bounds__(kSThreads, 2)
     }
     fence_proxy_async_smem();
   }
-  if (tid == 0) {
-    for (int s = 0; s < kSStages; ++s) {
-      mbar_init(&S.full[s], 1);
-      mbar_init(&S.empty[s], 1);
-    }
-    for (int a = 0; a < kSMaxAcc; ++a) {
-      mbar_init(&S.acc_full[a], 1);
-      mbar_init(&S.acc_empty[a], 4);
-    }
-    mbar_init(&S.q_full, 4);
-    mbar_init(&S.drain, 1);
-    S.abort_flag = 0;
-    fence_barrier_init();
-  }
-  if (warp == 1) {
-    tmem_alloc(&S.tmem_base, kSTmemCols);
-    tmem_relinquish();
-  }
-  if (warp == 0 && lane == 0) tma_prefetch_map(&blk_map);
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = S.tmem_base;
+  __syncthreads();   // the blocks' rows, ids and exponents; every layer's head weights
 
-  if (n_tiles > 0) {
+  if (n_work > 0) {
     if (warp == 0) {
       // ---- producer: lane l < 16 gathers block l of each tile ----
       const uint64_t policy = l2_policy_evict_normal();
@@ -267,21 +287,7 @@ __global__ void __launch_bounds__(kSThreads, 2)
       }
     } else {
       // ---- epilogue (warps 2..5): one position per thread, every layer ----
-      const int ew = warp - 2, quarter = warp & 3, m = quarter * 32 + lane;
-      for (int l = 0; l < L; ++l) {
-        const float* ql = io.q[l] + static_cast<long long>(b) * kIndexHeads * kIndexDim;
-        const float* wl = io.w[l] + static_cast<long long>(b) * kIndexHeads;
-        if constexpr (kFp4) {
-          prepare_query_fp4(ql, S.qtile[0], S.qscale, kIndexHeads * l, ew, lane);
-          if (lane < 8) S.ws[l][ew * 8 + lane] = wl[ew * 8 + lane];
-        } else {
-          prepare_query_part(ql, wl, S.qtile[l], S.ws[l], ew, lane);
-        }
-      }
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&S.q_full);
-      named_bar_sync(1, 128);   // every layer's ws is in shared memory
+      const int quarter = warp & 3, m = quarter * 32 + lane;
       for (int t = 0; t < n_tiles; ++t) {
         const int a = t % n_acc;
         const uint32_t aph = (t / n_acc) & 1;
@@ -316,7 +322,13 @@ __global__ void __launch_bounds__(kSThreads, 2)
           const uint32_t key = valid ? order_key(sc) : 0u;
           const long long bl = static_cast<long long>(b) * L + l;
           if (in_range) keys[bl * key_stride + static_cast<long long>(slot0 + e) * kBlock + o] = key;
-          if (valid) atomicAdd(&hist[bl * kRsHistBins + (key >> (32 - kRsHistBits))], 1u);
+          // one count per distinct bin of the warp's keys: the keys crowd into few bins
+          const uint32_t vm = __ballot_sync(0xffffffffu, valid);
+          if (valid) {
+            const uint32_t bin = key >> (32 - kRsHistBits);
+            const uint32_t peers = __match_any_sync(vm, bin);
+            if ((peers & ((1u << lane) - 1u)) == 0u) atomicAdd(&hist[bl * kRsHistBins + bin], __popc(peers));
+          }
         }
         tc_fence_before();
         __syncwarp();
