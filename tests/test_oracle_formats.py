@@ -182,3 +182,28 @@ def test_indexer_quantize_roundtrip():
     assert np.all(err <= np.maximum(np.abs(k) * 2.0 ** -4, 2.0 ** -10 * sig))
     # the largest element of each row lands in the top binade [256, 448]
     assert np.all(np.abs(F.e4m3_value(codes)).max(axis=1) >= 224)
+
+
+def test_e4m3_scale_from_the_fp32_quotient_is_the_exact_code():
+    """The kernels take a group's E4M3 scale as the round-to-nearest-even
+    conversion of the fp32 quotient amax / 6 (one division, one conversion)
+    instead of deciding against the exact quotient.  The two agree: every
+    E4M3 midpoint times 6 is an fp32 value, so the fp32 quotient lies on the
+    same side of every midpoint as the exact one.  Checked on the amax values
+    closest to 6 x each midpoint (the only place a rounding could flip a
+    decision), on 6 x each code value, and on random values over the whole
+    range, against the oracle's exact rule."""
+    vals = F.e4m3_value(np.arange(127))
+    mids = (vals[:-1] + vals[1:]) / 2.0
+    six = (6.0 * mids).astype(np.float32)
+    near = [six, (6.0 * vals).astype(np.float32)]
+    for k in range(1, 33):
+        near.append((six.view(np.uint32) + k).view(np.float32))
+        near.append((six.view(np.uint32) - k).view(np.float32))
+    rng = np.random.default_rng(11)
+    rand = [np.exp(rng.uniform(-35.0, 9.0, 200_000)).astype(np.float32),
+            (rng.random(200_000) * 3000.0).astype(np.float32)]
+    amax = np.abs(np.concatenate(near + rand))
+    exact = F.e4m3_encode(amax.astype(np.float64) / 6.0)
+    via_fp32 = F.e4m3_encode((amax / np.float32(6.0)).astype(np.float64))
+    np.testing.assert_array_equal(via_fp32, exact)
