@@ -386,6 +386,11 @@ CSA2_API csa2_status csa2_reindex_layers(const csa2_cache* cache, int32_t n_laye
  *   out        bf16  [n_queries][H][512] out
  * H in {16, 32, 64}; k in [1, 4096].  Dequantised rows are exact in fp16,
  * logits and softmax are fp32, P.V uses fp16 probabilities with fp32 sums.
+ * A query's rows are split over 4, 2 or 1 CTAs (H = 16: always 4) by the
+ * number of queries in the call (up to 6, up to 12, more), and the partial
+ * results are merged in fp32: a query's output is bit-identical across calls
+ * with the same number of queries, whatever the number of layers, and may
+ * differ in the last bits between calls with different numbers.
  * Device errors: a Top-k entry >= ctx_len or < -1 -> CSA2_ERR_DEVICE_BOUNDS,
  * entry skipped; a q_req entry outside [0, batch) -> CSA2_ERR_DEVICE_BOUNDS
  * (request = that value, index = -1), the query's output is 0.

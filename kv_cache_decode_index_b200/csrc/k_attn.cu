@@ -3,8 +3,10 @@
 // blog, section 二: every layer attends over its Top-K, Reuse layers with
 // their own query; FP4 rows: 4sapi blog, section 五].
 //
-// One thread-block cluster of kACluster (4) CTAs per (layer, query).  CTA r
-// takes entries [r*kc, (r+1)*kc) (kc = ceil(k/4)) in chunks of 64 rows:
+// One thread-block cluster of CL CTAs (key splits) per (layer, query): 4 for
+// up to 6 queries (a decode group's six layers of them fill one wave of the
+// GPU's SMs), 2 for up to 12, else 1 (16 heads: always 4).  CTA r takes
+// entries [r*kc, (r+1)*kc) (kc = ceil(k/CL)) in chunks of 64 rows:
 //   * prologue: the query's bf16 rows are loaded and converted before the
 //     wait on the preceding launch, then the CTA turns its Top-k entries into
 //     cache rows (page table) once, into shared memory;
@@ -20,12 +22,11 @@
 //     domain) whose row maxima and sums are combined through shared memory,
 //     P rounded to fp16 in shared memory, O += P V with each warp on 64 of
 //     the 512 output dims of every head;
-// then CTA r merges the four partial (O, max, sum) sets for output dims
-// [128r, 128r+128) and writes those dims of every head.  The partials reach
-// it through a caller workspace in global memory (L2) when one is given,
-// else by stores into its shared memory from the other CTAs (distributed
-// shared memory), between cluster barriers.  Four CTAs per query keep all
-// six layers' attention of a decode step within one wave of the GPU's SMs.
+// then CTA r merges the CL partial (O, max, sum) sets for output dims
+// [512r/CL, 512(r+1)/CL) and writes those dims of every head.  The partials
+// reach it through a caller workspace in global memory (L2) when one is
+// given, else by stores into its shared memory from the other CTAs
+// (distributed shared memory), between cluster barriers.
 #include <cooperative_groups.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -42,21 +43,22 @@ namespace cg = cooperative_groups;
 
 constexpr int kAThreads = 256;
 constexpr int kAWarps = kAThreads / 32;
-constexpr int kACluster = 4;                 // CTAs (key splits) per query
-constexpr int kODims = kKvDim / kACluster;   // output dims owned by one CTA of the cluster
+constexpr int kAMaxCluster = 4;             // CTAs (key splits) per query, at most
 constexpr int kChunk = 64;                   // keys per chunk
 constexpr int kRowBytes = kKvDim * 2;        // fp16 row: 1024 B
 constexpr int kPRowBytes = kChunk * 2;       // fp16 row of P: 128 B
 constexpr int kPVDims = kKvDim / kAWarps;    // output dims per warp in P V: 64
 constexpr int kCodeGran = kKvCodeBytes / 16;                    // 16-byte granules of a packed row's codes
 constexpr int kRowGran = (kKvCodeBytes + kKvScaleBytes) / 16;   // ... of codes + scales
-// Top-k entries one CTA resolves: k <= 4096 and a window <= 4096 give at most
-// ceil((4096 + 4096) / 4) entries per CTA.
-constexpr int kMaxTop = (4096 + CSA2_SWA_MAX_WINDOW + kACluster - 1) / kACluster;
 constexpr float kLog2e = 1.4426950408889634f;
 
-template <int H>
+// CL: CTAs (key splits) per query.
+template <int H, int CL>
 struct AttnLayout {
+  static constexpr int kODims = kKvDim / CL;   // output dims owned by one CTA of the cluster
+  // Top-k entries one CTA resolves: k <= 4096 and a window <= 4096 give at
+  // most ceil((4096 + 4096) / CL) entries per CTA.
+  static constexpr int kMaxTop = (4096 + CSA2_SWA_MAX_WINDOW + CL - 1) / CL;
   static constexpr int HT = H / 16;            // head tiles of 16 query rows
   static constexpr int KG = kAWarps / HT;      // key groups in S
   static constexpr int KW = kChunk / KG;       // keys per warp in S
@@ -70,15 +72,15 @@ struct AttnLayout {
   static constexpr uint32_t qscale_off = red_off + 2 * KG * H * 4;
   static constexpr uint32_t kvalid_off = qscale_off + H * 4;               // int [64]
   static constexpr uint32_t srow_off = kvalid_off + kChunk * 4;            // int32 [kMaxTop] cache rows
-  static constexpr uint32_t ml_off = srow_off + kMaxTop * 4;               // fp32 [kACluster][2][H]: m, l
-  static constexpr uint32_t fac_off = ml_off + kACluster * 2 * H * 4;      // fp32 [kACluster][H]
-  static constexpr uint32_t total = fac_off + kACluster * H * 4;
-  // received partial O: [kACluster source ranks][H][kODims dims] fp32, over the Q + KV region
-  static_assert(kACluster * H * kODims * 4 <= raw_off, "received partials must fit in the Q + KV region");
+  static constexpr uint32_t ml_off = srow_off + kMaxTop * 4;               // fp32 [CL][2][H]: m, l
+  static constexpr uint32_t fac_off = ml_off + CL * 2 * H * 4;             // fp32 [CL][H]
+  static constexpr uint32_t total = fac_off + CL * H * 4;
+  // received partial O: [CL source ranks][H][kODims dims] fp32, over the Q + KV region
+  static_assert(CL * H * kODims * 4 <= raw_off, "received partials must fit in the Q + KV region");
   static_assert(KW % 8 == 0 && (NT == 1 || NT % 2 == 0), "whole 8-key tiles per warp");
 };
 
-// Column (float index) of dim c of head h in a swizzled [H][kODims] fp32
+// Column (float index) of dim c of head h in a swizzled [H][dims] fp32
 // slice: the 16-byte granule index is XORed with h % 8.
 __device__ __forceinline__ int attn_swz(int h, int c) { return (((c >> 2) ^ (h & 7)) << 2) | (c & 3); }
 
@@ -165,12 +167,14 @@ struct SwaArgs {
   int window;
 };
 
-template <int H>
+template <int H, int CL>
 __global__ void __launch_bounds__(kAThreads, H == 16 ? 2 : 1)
     sparse_attn_kernel(const csa2_cache cache, int n_queries, const int32_t* __restrict__ q_req,
                        int K, const __grid_constant__ AttnLayers io, float softmax_scale,
                        const SwaArgs swa, float* __restrict__ xchg) {
-  using L = AttnLayout<H>;
+  using L = AttnLayout<H, CL>;
+  constexpr int kODims = L::kODims;
+  constexpr int kMaxTop = L::kMaxTop;
   extern __shared__ __align__(1024) uint8_t smem[];
   const uint32_t sbase = smem_u32(smem);
   float* red_max = reinterpret_cast<float*>(smem + L::red_off);   // [KG][H]
@@ -183,8 +187,8 @@ __global__ void __launch_bounds__(kAThreads, H == 16 ? 2 : 1)
 
   cg::cluster_group cluster = cg::this_cluster();
   const int rank = static_cast<int>(cluster.block_rank());
-  const int layer = static_cast<int>(blockIdx.x / kACluster) / n_queries;
-  const int qi = static_cast<int>(blockIdx.x / kACluster) % n_queries;
+  const int layer = static_cast<int>(blockIdx.x / CL) / n_queries;
+  const int qi = static_cast<int>(blockIdx.x / CL) % n_queries;
   const __nv_bfloat16* __restrict__ qg = io.q[layer];
   __nv_bfloat16* __restrict__ out = io.out[layer];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -245,7 +249,7 @@ __global__ void __launch_bounds__(kAThreads, H == 16 ? 2 : 1)
   const int n_win = swa.codes != nullptr ? swa.window : 0;
   const int p_tok = n_win > 0 ? swa.q_pos[qi] : 0;
   const int K_all = K + n_win;
-  const int kc = (K_all + kACluster - 1) / kACluster;
+  const int kc = (K_all + CL - 1) / CL;
   const int key_begin = min(rank * kc, K_all), key_end = min(key_begin + kc, K_all);
   const int n_top = n_raw < 0 ? 0 : min(max(0, min(key_end, K) - key_begin), kMaxTop);
   for (int i = tid; i < n_top; i += kAThreads) {
@@ -507,8 +511,8 @@ __global__ void __launch_bounds__(kAThreads, H == 16 ? 2 : 1)
   // passes the same barriers.
   constexpr long long kRegion = static_cast<long long>(H) * kKvDim + 2 * H;   // floats per CTA in xchg
   float* recv = reinterpret_cast<float*>(smem);
-  const float* src_slice[kACluster];      // where the owner reads source r's slice of its dims
-  const float* src_ml[kACluster];         // ... and source r's (m[H], l[H])
+  const float* src_slice[CL];      // where the owner reads source r's slice of its dims
+  const float* src_ml[CL];         // ... and source r's (m[H], l[H])
   int slice_swz;                          // 1: swizzled shared-memory slices
   const int owner = (warp * kPVDims) / kODims, cd0 = (warp * kPVDims) % kODims;   // this warp's dims
   if (xchg != nullptr) {
@@ -534,7 +538,7 @@ __global__ void __launch_bounds__(kAThreads, H == 16 ? 2 : 1)
     cluster.sync();   // every CTA's partials are in the workspace (cluster-scope release / acquire)
     const float* first = xchg + static_cast<long long>(blockIdx.x - rank) * kRegion;
 #pragma unroll
-    for (int r = 0; r < kACluster; ++r) {
+    for (int r = 0; r < CL; ++r) {
       src_slice[r] = first + r * kRegion + rank * H * kODims;
       src_ml[r] = first + r * kRegion + H * kKvDim;
     }
@@ -554,7 +558,7 @@ __global__ void __launch_bounds__(kAThreads, H == 16 ? 2 : 1)
       }
     if (warp == 0 && (lane & 3) == 0) {
 #pragma unroll
-      for (int o = 0; o < kACluster; ++o) {
+      for (int o = 0; o < CL; ++o) {
         float* ml = cluster.map_shared_rank(ml_sh, o) + rank * 2 * H;
 #pragma unroll
         for (int t = 0; t < L::HT; ++t)
@@ -567,7 +571,7 @@ __global__ void __launch_bounds__(kAThreads, H == 16 ? 2 : 1)
     }
     cluster.sync();   // every partial has landed; no CTA touches another's memory after this
 #pragma unroll
-    for (int r = 0; r < kACluster; ++r) {
+    for (int r = 0; r < CL; ++r) {
       src_slice[r] = recv + r * H * kODims;
       src_ml[r] = ml_sh + r * 2 * H;
     }
@@ -576,37 +580,37 @@ __global__ void __launch_bounds__(kAThreads, H == 16 ? 2 : 1)
 
   // merge factors per (source rank, head): exp2(m_r - M) / L
   for (int h = tid; h < H; h += kAThreads) {
-    float mr[kACluster], lr[kACluster];
+    float mr[CL], lr[CL];
     float M = -INFINITY;
 #pragma unroll
-    for (int r = 0; r < kACluster; ++r) {
+    for (int r = 0; r < CL; ++r) {
       mr[r] = src_ml[r][h];
       lr[r] = src_ml[r][H + h];
       M = fmaxf(M, mr[r]);
     }
     float Lsum = 0.0f;
 #pragma unroll
-    for (int r = 0; r < kACluster; ++r) {
+    for (int r = 0; r < CL; ++r) {
       mr[r] = (M == -INFINITY || mr[r] == -INFINITY) ? 0.0f : exp2f(mr[r] - M);
       Lsum += lr[r] * mr[r];
     }
     const float inv = Lsum > 0.0f ? 1.0f / Lsum : 0.0f;
 #pragma unroll
-    for (int r = 0; r < kACluster; ++r) fac[r * H + h] = mr[r] * inv;
+    for (int r = 0; r < CL; ++r) fac[r * H + h] = mr[r] * inv;
   }
   __syncthreads();
   // this CTA writes dims [kODims*rank, kODims*(rank+1)) of every head, 4 dims
   // per item; every item's partial slices are loaded before any is used
   constexpr int kItems = H * (kODims / 4) / kAThreads;
   static_assert(H * (kODims / 4) % kAThreads == 0, "whole items per thread");
-  float4 part[kItems][kACluster];
+  float4 part[kItems][CL];
 #pragma unroll
   for (int it = 0; it < kItems; ++it) {
     const int item = it * kAThreads + tid;
     const int h = item / (kODims / 4), d4 = (item % (kODims / 4)) * 4;
     const int c = slice_swz ? attn_swz(h, d4) : d4;
 #pragma unroll
-    for (int r = 0; r < kACluster; ++r) part[it][r] = *reinterpret_cast<const float4*>(src_slice[r] + h * kODims + c);
+    for (int r = 0; r < CL; ++r) part[it][r] = *reinterpret_cast<const float4*>(src_slice[r] + h * kODims + c);
   }
 #pragma unroll
   for (int it = 0; it < kItems; ++it) {
@@ -614,7 +618,7 @@ __global__ void __launch_bounds__(kAThreads, H == 16 ? 2 : 1)
     const int h = item / (kODims / 4), d4 = (item % (kODims / 4)) * 4;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-    for (int r = 0; r < kACluster; ++r) {
+    for (int r = 0; r < CL; ++r) {
       const float4 v = part[it][r];
       const float f = fac[r * H + h];
       acc.x += v.x * f; acc.y += v.y * f; acc.z += v.z * f; acc.w += v.w * f;
@@ -627,37 +631,63 @@ __global__ void __launch_bounds__(kAThreads, H == 16 ? 2 : 1)
   }
 }
 
-template <int H>
-cudaError_t launch_h(const csa2_cache& cache, int n_layers, int n_queries, const int32_t* q_req, int k,
-                     const AttnLayers& io, float scale, const SwaArgs& swa, float* xchg, cudaStream_t stream) {
+template <int H, int CL>
+cudaError_t launch_hc(const csa2_cache& cache, int n_layers, int n_queries, const int32_t* q_req, int k,
+                      const AttnLayers& io, float scale, const SwaArgs& swa, float* xchg, cudaStream_t stream) {
   static ContextMemo attrs;
-  const size_t smem = AttnLayout<H>::total;
+  const size_t smem = AttnLayout<H, CL>::total;
   const cudaError_t e = attrs.once([&] {
-    return cudaFuncSetAttribute(sparse_attn_kernel<H>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    return cudaFuncSetAttribute(sparse_attn_kernel<H, CL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 static_cast<int>(smem));
   });
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(n_layers * n_queries * kACluster);
+  cfg.gridDim = dim3(n_layers * n_queries * CL);
   cfg.blockDim = dim3(kAThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = kACluster;
+  attr[0].val.clusterDim.x = CL;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
   attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;   // the kernel calls pdl_wait() before reading the Top-k
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  return cudaLaunchKernelEx(&cfg, sparse_attn_kernel<H>, cache, n_queries, q_req, k, io, scale, swa, xchg);
+  return cudaLaunchKernelEx(&cfg, sparse_attn_kernel<H, CL>, cache, n_queries, q_req, k, io, scale, swa, xchg);
+}
+
+// Key splits per query, from the number of queries alone (so that one query's
+// result does not depend on how many layers a launch covers): 4 while a
+// decode group's six layers of all queries fit one wave of the GPU's SMs at
+// 4 CTAs per query, then 2, then 1 (more queries fill the GPU by themselves,
+// and one CTA per query merges no partial outputs).  16 heads keep 4: their
+// CTAs fit two per SM, which the larger entry table of fewer splits would
+// prevent.
+int key_splits(int n_queries, int H) {
+  if (H == 16) return 4;
+  return n_queries <= 6 ? 4 : (n_queries <= 12 ? 2 : 1);
+}
+
+template <int H>
+cudaError_t launch_h(const csa2_cache& cache, int n_layers, int n_queries, const int32_t* q_req, int k,
+                     const AttnLayers& io, float scale, const SwaArgs& swa, float* xchg, cudaStream_t stream) {
+  if constexpr (H == 16) {
+    return launch_hc<H, 4>(cache, n_layers, n_queries, q_req, k, io, scale, swa, xchg, stream);
+  } else {
+    switch (key_splits(n_queries, H)) {
+      case 4: return launch_hc<H, 4>(cache, n_layers, n_queries, q_req, k, io, scale, swa, xchg, stream);
+      case 2: return launch_hc<H, 2>(cache, n_layers, n_queries, q_req, k, io, scale, swa, xchg, stream);
+      default: return launch_hc<H, 1>(cache, n_layers, n_queries, q_req, k, io, scale, swa, xchg, stream);
+    }
+  }
 }
 
 }  // namespace
 
 size_t attn_workspace_bytes(long long n_layers, long long n_queries, int H) {
-  return static_cast<size_t>(n_layers * n_queries * kACluster) * (static_cast<size_t>(H) * kKvDim + 2 * H) * 4;
+  return static_cast<size_t>(n_layers * n_queries * kAMaxCluster) * (static_cast<size_t>(H) * kKvDim + 2 * H) * 4;
 }
 
 cudaError_t launch_sparse_attn(const csa2_cache& cache, int n_layers, int n_queries, const int32_t* q_req,

@@ -54,11 +54,14 @@ constexpr int kPThreads = 64 + kPEpiWarps * 32;        // 576
 constexpr uint32_t kPTmemCols = kPAcc * kPN;           // 512
 constexpr uint32_t kPIdesc = idesc_e4m3_f32(kTile, kPN);
 constexpr int kCand = CSA2_PREFILL_CANDIDATES;         // list capacity per query
-constexpr int kBarEvery = 2;                           // tiles between the epilogue's barriers
+constexpr int kBarEvery = 8;                           // tiles between the epilogue's barriers
 constexpr int kHigh = kCand - kBarEvery * kTile;       // compaction trigger
 constexpr int kBarAll = 1;                             // named barrier: all epilogue warps
 constexpr int kBarTile = 2;                            // per-tile barrier of the epilogue warps
 static_assert(kCand % 4 == 0 && kCand >= 2 * CSA2_PREFILL_MAX_K + 2 * kTile, "candidate capacity");
+// a list compacted to k is below the trigger, and one below the trigger has
+// room for the kBarEvery tiles until the next check
+static_assert(kHigh > CSA2_PREFILL_MAX_K && kHigh + kBarEvery * kTile <= kCand, "compaction trigger");
 
 struct __align__(1024) PrefillSmem {
   uint8_t tiles[kPStages][kTileBytes];

@@ -357,12 +357,13 @@ __global__ void __launch_bounds__(kBlockSelectThreads, 1)
   const int b = blockIdx.x / L, l = blockIdx.x % L;
   const long long bl = static_cast<long long>(b) * L + l;
   const int n_keys = P * kBlock;
+  // The request's pool (block ids of the key groups), used by the emits
+  // after the select's barriers.  The scoring launch lets this one start only
+  // after its own wait for the pool's launch to complete, so the pool is read
+  // before this launch's wait.
+  for (int i = tid; i < P; i += kBlockSelectThreads) pool_ids[i] = pool[static_cast<long long>(b) * P + i];
   pdl_wait();                 // the keys and histograms of the scoring launch are complete
   pdl_launch_dependents();
-
-  // the request's pool (block ids of the key groups), read before the keys
-  // and used by the emits after the select's barriers
-  for (int i = tid; i < P; i += kBlockSelectThreads) pool_ids[i] = pool[static_cast<long long>(b) * P + i];
   // keys [tid*ITEMS, (tid+1)*ITEMS) in registers (groups of 4: n_keys is a multiple of 8)
   uint32_t k[ITEMS];
   const uint32_t* src = keys + bl * n_keys;

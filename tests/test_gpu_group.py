@@ -93,8 +93,13 @@ def _check_request(csa2, wl, cache, group, b, n, q_idx, w_idx, q_main, out, dev)
     for layer in range(len(wl.modes)):
         ot = ora["topk"][layer].astype(np.int32)
         ref = C.sparse_attention(q_main[layer][b].float().numpy(), full_c, full_s, ot, wl.scale)
-        qi = torch.tensor([b], dtype=torch.int32, device=dev)
-        g = csa2.sparse_attn(cache, torch.from_numpy(ot[None]).to(dev), q_main[layer][b:b + 1].to(dev), wl.scale,
+        # as many queries as the group's launch (all of them request b's): the
+        # number of queries per launch decides the key split, and with it the
+        # rounding of the merge
+        nq = wl.batch
+        qi = torch.full((nq,), b, dtype=torch.int32, device=dev)
+        g = csa2.sparse_attn(cache, torch.from_numpy(np.repeat(ot[None], nq, axis=0)).to(dev),
+                             q_main[layer][b:b + 1].repeat(nq, 1, 1).to(dev), wl.scale,
                              q_req=qi).float().cpu().numpy()[0]
         worst = max(worst, U.assert_attention_close(g, ref, f"attention layer {layer} b={b}"))
         if np.array_equal(group.topk[layer][b].cpu().numpy(), ot):

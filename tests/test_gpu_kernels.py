@@ -533,6 +533,37 @@ def test_sparse_attention_workspace_exchange_is_bit_identical(csa2, H, k, n_laye
     assert csa2.get_error(cache)[0] == csa2.OK
 
 
+@pytest.mark.parametrize("nq", [8, 13])
+def test_sparse_attention_key_splits(csa2, nq):
+    """Launches of more queries take 2 (up to 12 queries) or 1 (more) CTAs per
+    query instead of 4: parity with the oracle for every query, and the merge
+    through the caller's workspace equals the merge through shared memory."""
+    wl = W.scaled(W.WORKLOADS["group_64k_b8"], batch=3, ctx=5000, heads=64)
+    cache = U.build_cache(wl, csa2)
+    dev = cache.device
+    rng = np.random.default_rng(31 + nq)
+    q_req = (np.arange(nq) % 3).astype(np.int32)
+    topk = np.stack([np.sort(rng.choice(5000, 512, replace=False)) for _ in range(nq)]).astype(np.int32)
+    topk[1, 200:] = -1
+    topk[nq - 1] = rng.permutation(topk[nq - 1])
+    tq = torch.from_numpy(q_req).to(dev)
+    tk = torch.from_numpy(topk).to(dev)
+    qs = [W.main_query(wl, layer, rows=nq) for layer in range(2)]
+    out = csa2.sparse_attn(cache, tk, qs[0].to(dev), wl.scale, q_req=tq).float().cpu().numpy()
+    rows = {b: U.oracle_kv_rows(wl, b, np.arange(5000)) for b in range(3)}
+    for i in range(nq):
+        codes, scales = rows[int(q_req[i])]
+        ref = C.sparse_attention(qs[0][i].float().numpy(), codes, scales, topk[i], wl.scale)
+        U.assert_attention_close(out[i], ref, f"nq={nq} query {i}")
+    ws = torch.full((csa2.attn_workspace_bytes(2, nq, 64),), 0xFF, dtype=torch.uint8, device=dev)
+    via_smem = csa2.sparse_attn_layers(cache, tk, [q.to(dev) for q in qs], wl.scale, q_req=tq)
+    via_ws = csa2.sparse_attn_layers(cache, tk, [q.to(dev) for q in qs], wl.scale, q_req=tq, workspace=ws)
+    for layer in range(2):
+        assert torch.equal(via_ws[layer], via_smem[layer]), f"layer {layer}"
+    np.testing.assert_array_equal(via_smem[0].float().cpu().numpy(), out)
+    assert csa2.get_error(cache)[0] == csa2.OK
+
+
 def test_sparse_attention_empty_and_query_map(csa2):
     wl = W.scaled(W.WORKLOADS["full_4k_b1"], batch=2, heads=16, page_size=1024)
     cache = U.build_cache(wl, csa2, lengths=[2000, 3000])
