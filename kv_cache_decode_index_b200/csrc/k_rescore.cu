@@ -57,7 +57,6 @@ struct __align__(1024) ScoreSmemT {
   uint8_t qscale[kFp4 ? 1024 : 16];                         // FP4: the query heads' block scales
   uint8_t tscale[kFp4 ? kSMaxTiles : 1][kFp4 ? 1024 : 16];  // FP4: each tile's block scales
   float ws[kLayers][kIndexHeads];                           // w_h (FP4) or w_h * sigma^q_h (FP8) per layer
-  uint64_t blk_exp[kSMaxTiles * kSBlocksPerTile];
   int blk_row[kSMaxTiles * kSBlocksPerTile];
   int blk_id[kSMaxTiles * kSBlocksPerTile];
   uint64_t full[kSStages];
@@ -162,17 +161,16 @@ __global__ void __launch_bounds__(kSThreads, 2)
   const int n = max(n_raw, 0);
   const int n_work = n_raw < 0 ? 0 : n_tiles;   // tiles this CTA scores
 
-  // ---- this CTA's pool blocks: block id -> page -> row and exponent bytes ----
+  // ---- this CTA's pool blocks: block id -> page -> row (the exponent bytes
+  // are read by the epilogue while the codes are gathered) ----
   for (int i = tid; i < (n_raw < 0 ? 0 : nblk); i += kSThreads) {
     const int j = pool[static_cast<long long>(b) * P + slot0 + i];
     int row = -1;
-    uint64_t ex = 0x7F7F7F7F7F7F7F7Full;
     if (j >= 0 && static_cast<long long>(j) * kBlock < n) {
       const int t = j * kBlock;
       const int page = cache.page_table[static_cast<long long>(b) * cache.max_pages_per_req + t / cache.page_size];
       if (page >= 0 && page < cache.num_pages) {
         row = page * cache.page_size + t % cache.page_size;
-        if (!kFp4) ex = *reinterpret_cast<const uint64_t*>(cache.ik_exp + row);
       } else {
         report_error(cache.err_word, CSA2_ERR_DEVICE_BOUNDS, kKReindex, b, t);
       }
@@ -181,7 +179,6 @@ __global__ void __launch_bounds__(kSThreads, 2)
     }
     S.blk_row[i] = row;
     S.blk_id[i] = row >= 0 ? j : -1;
-    S.blk_exp[i] = ex;
   }
   if constexpr (kFp4) {
     // block scales of the CTA's blocks, moved into each tile's tensor-core
@@ -211,7 +208,7 @@ __global__ void __launch_bounds__(kSThreads, 2)
     }
     fence_proxy_async_smem();
   }
-  __syncthreads();   // the blocks' rows, ids and exponents; every layer's head weights
+  __syncthreads();   // the blocks' rows and ids; every layer's head weights
 
   if (n_work > 0) {
     if (warp == 0) {
@@ -295,7 +292,8 @@ __global__ void __launch_bounds__(kSThreads, 2)
         const int o = m % kBlock;
         const bool in_range = e < nblk;
         const bool valid = in_range && S.blk_row[e] >= 0 && S.blk_id[e] * kBlock + o < n;
-        const uint32_t e_byte = (!kFp4 && valid) ? static_cast<uint32_t>((S.blk_exp[e] >> (8 * o)) & 0xFFu) : 127u;
+        // issued before the wait for the accumulator: its latency overlaps the gather and the MMA
+        const uint32_t e_byte = (!kFp4 && valid) ? static_cast<uint32_t>(cache.ik_exp[S.blk_row[e] + o]) : 127u;
         if (!mbar_wait_warp(&S.acc_full[a], aph, wait_ns)) {
           if (lane == 0) {
             report_error(cache.err_word, CSA2_ERR_TIMEOUT, kKReindex, b, t);
