@@ -210,15 +210,17 @@ __device__ void block_topk(const uint32_t (&keys)[ITEMS], int K, BlockSelectSmem
   const int gt_before = before.x, eq_before = before.y;
   int take = max(0, min(need - eq_before, eq));   // ties this thread takes
   int r = gt_before + min(eq_before, need);
+  if (gt + take > 0) {   // most threads select none of their keys
 #pragma unroll
-  for (int i = 0; i < ITEMS; ++i) {
-    const uint32_t k = keys[i], km = k & mask;
-    const bool above = k != 0u && km > prefix;
-    const bool tie = k != 0u && km == prefix && take > 0;
-    if (above || tie) {
-      emit(tid * ITEMS + i, r);
-      ++r;
-      if (tie) --take;
+    for (int i = 0; i < ITEMS; ++i) {
+      const uint32_t k = keys[i], km = k & mask;
+      const bool above = k != 0u && km > prefix;
+      const bool tie = k != 0u && km == prefix && take > 0;
+      if (above || tie) {
+        emit(tid * ITEMS + i, r);
+        ++r;
+        if (tie) --take;
+      }
     }
   }
   const int sel_total = gt_total + min(eq_total, need);
