@@ -322,8 +322,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           // count the segments passed; group 0 keeps the codes two segments ahead
           for (int b = cur_b; b != it.b; b = next_request_with_tiles(S.prefix, B, b)) ++seg;
           cur_b = it.b;
-          if (group == 0)
-            while (prep_x <= seg + 2 && prep_b < B && S.prefix[prep_b] < t_end) prepare();
           load_head_weights(q + static_cast<long long>(cur_b) * kIndexHeads * kIndexDim, w + cur_b * kIndexHeads,
                             ws, lane);
           nb = cache.ctx_len[cur_b];
@@ -354,6 +352,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_arrive(&S.acc_empty[a]);
           mbar_arrive(&S.empty[s]);
         }
+        // Group 0 writes the codes of up to two segments ahead only after this
+        // unit's accumulator: the buffer it reuses held the previous segment,
+        // whose last unit may be group 1's and issued after group 0's previous
+        // accumulator.
+        if (group == 0)
+          while (prep_x <= seg + 2 && prep_b < B && S.prefix[prep_b] < t_end) prepare();
 
 #pragma unroll
         for (int h = 0; h < 2; ++h) {

@@ -324,8 +324,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (it.b != cur_b) {
           for (int b = cur_b; b != it.b; b = next_request_with_tiles(S.prefix, B, b)) ++seg;
           cur_b = it.b;
-          if (group == 0)
-            while (prep_x <= seg + 2 && prep_b < B && S.prefix[prep_b] < t_end) prepare();
           load_w(cur_b);
           nb = cache.ctx_len[cur_b];
         }
@@ -346,6 +344,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&S.acc_empty[a]);
+        // Group 0 writes the codes of up to two segments ahead only after this
+        // unit's accumulator: the buffer it reuses held the previous segment,
+        // whose last unit may be group 1's and issued after group 0's previous
+        // accumulator.
+        if (group == 0)
+          while (prep_x <= seg + 2 && prep_b < B && S.prefix[prep_b] < t_end) prepare();
 
 #pragma unroll
         for (int h = 0; h < 2; ++h) {

@@ -79,15 +79,21 @@ def _fp4_bound(q, w, codes, scales):
     return (ka @ qa.T) @ np.abs(w.astype(np.float64)) * 2.0 ** -20
 
 
-def test_index_full_fp4_scores_ragged(csa2):
-    wl = W.scaled(W.WORKLOADS["group_64k_b8"], batch=5, page_size=512, shuffle_pages=True)
-    lengths = [4096, 1, 1000, 9999, 128 * 37]
+# Many short requests: about four requests per CTA's range of units, so the
+# scan's query buffers rotate (segment x in buffer x % 3) inside a CTA.
+MANY_SHORT = [int(n) for n in np.random.default_rng(77).integers(1, 1100, size=600)]
+
+
+@pytest.mark.parametrize("lengths", [[4096, 1, 1000, 9999, 128 * 37], MANY_SHORT], ids=["five", "many_short"])
+def test_index_full_fp4_scores_ragged(csa2, lengths):
+    B = len(lengths)
+    wl = W.scaled(W.WORKLOADS["group_64k_b8"], batch=B, page_size=512, shuffle_pages=True)
     from kv_cache_decode_index_b200.fill import build_cache
     cache = build_cache(wl, csa2, lengths=lengths, fp4_indexer=True)
     q, w = W.index_query(wl, 0)
     dev = cache.device
-    bm = torch.full((5, cache.capacity // 8), float("nan"), device=dev)
-    sc = torch.full((5, cache.capacity), float("nan"), device=dev)
+    bm = torch.full((B, cache.capacity // 8), float("nan"), device=dev)
+    sc = torch.full((B, cache.capacity), float("nan"), device=dev)
     hist = csa2.pool_hist(cache)
     csa2.index_full_fp4(cache, cache.ik4, torch.from_numpy(q).to(dev), torch.from_numpy(w).to(dev), bm, sc, hist)
     assert csa2.get_error(cache)[0] == csa2.OK

@@ -190,14 +190,20 @@ def _score_bound(q, w, codes, exp):
     return sig * (absdot @ w64) * 2.0 ** -22 * 2, sig
 
 
-def test_index_full_scores_ragged(csa2):
-    wl = W.scaled(W.WORKLOADS["group_64k_b8"], batch=5, page_size=512, shuffle_pages=True)
-    lengths = [4096, 1, 1000, 9999, 128 * 37]
+# Many short requests: about four requests per CTA's range of units, so the
+# scan's query-code buffers rotate (segment x in buffer x % 3) inside a CTA.
+MANY_SHORT = [int(n) for n in np.random.default_rng(77).integers(1, 1100, size=600)]
+
+
+@pytest.mark.parametrize("lengths", [[4096, 1, 1000, 9999, 128 * 37], MANY_SHORT], ids=["five", "many_short"])
+def test_index_full_scores_ragged(csa2, lengths):
+    B = len(lengths)
+    wl = W.scaled(W.WORKLOADS["group_64k_b8"], batch=B, page_size=512, shuffle_pages=True)
     cache = U.build_cache(wl, csa2, lengths=lengths)
     q, w = W.index_query(wl, 0)
     dev = cache.device
-    bm = torch.full((5, cache.capacity // 8), float("nan"), device=dev)
-    sc = torch.full((5, cache.capacity), float("nan"), device=dev)
+    bm = torch.full((B, cache.capacity // 8), float("nan"), device=dev)
+    sc = torch.full((B, cache.capacity), float("nan"), device=dev)
     csa2.index_full(cache, torch.from_numpy(q).to(dev), torch.from_numpy(w).to(dev), bm, sc)
     bm, sc = bm.cpu().numpy(), sc.cpu().numpy()
     worst = 0.0
