@@ -13,19 +13,21 @@
 // tile's scales reach tensor memory with one bulk copy and two tcgen05.cp.
 //
 // index_full_fp4_kernel follows the FP8 scan (one persistent CTA per SM,
-// 256-position units split into contiguous CTA ranges, TMA producer warp, MMA
-// warp, two epilogue warpgroups on alternate units), with:
+// 256-position units split into contiguous CTA ranges, TMA producer warp, two
+// epilogue warpgroups on alternate units), with:
 //   * stages of two 128-row code tiles (64-byte rows, 64-byte swizzle, 8 KB
 //     each) and their two 1 KB scale blocks: with pages of whole units, one
 //     256-row TMA load and one 2 KB bulk copy per unit (else one of each per
 //     tile), issued from cache rows the producer warp resolved 32 units at a
 //     time (UnitRows);
-//   * the MMA: per 128-row tile, tcgen05.cp of its scales to tensor memory,
-//     then two tcgen05.mma kind::mxf4nvf4 (K = 64 each, E4M3 block scales,
-//     M = 128 positions, N = 32 heads) into the tile's accumulator;
+//   * two MMA-issuing threads, one per 128-row tile of every unit: tcgen05.cp
+//     of the tile's scales to tensor memory, then two tcgen05.mma
+//     kind::mxf4nvf4 (K = 64 each, E4M3 block scales, M = 128 positions,
+//     N = 32 heads) into the tile's accumulator, one commit per unit each;
+//     the epilogue frees the stage once the accumulator pair is complete;
 //   * epilogue group 0 quantises each request's query (32 heads) into FP4
-//     codes and scales; the MMA warp copies the query's scales to tensor
-//     memory once per request segment.
+//     codes and scales; each issuer copies the query's scales to its own
+//     tensor-memory columns once per request segment.
 // Every wait is bounded (CSA2_ERR_TIMEOUT, drain, free tensor memory, return).
 #include <cub/block/block_scan.cuh>
 
@@ -38,11 +40,13 @@ namespace csa2 {
 namespace {
 
 constexpr int kUnit = kScanUnit;
-constexpr int kStages = 8;
+constexpr int kStages = 10;
 constexpr int kAcc = 4;                    // accumulator pairs
 constexpr int kEpiGroups = 2;
 constexpr int kQBufs = 3;
-constexpr int kThreads = 64 + kEpiGroups * 128;
+constexpr int kIssuers = 2;                 // one per 128-row tile of a unit
+constexpr int kEpiWarp0 = 1 + kIssuers;    // first epilogue warp
+constexpr int kThreads = 32 * kEpiWarp0 + kEpiGroups * 128;
 constexpr int kMaxBatchScan = 1024;
 constexpr int kScanItems = (kMaxBatchScan + kThreads - 1) / kThreads;
 constexpr int kCodeBytes = CSA2_IK4_CODE_BYTES;          // 64 per row
@@ -68,7 +72,7 @@ struct __align__(1024) Fp4Smem {
   uint64_t acc_full[kAcc];
   uint64_t acc_empty[kAcc];
   uint64_t q_full[kQBufs];
-  uint64_t drain;
+  uint64_t drain[kIssuers];
   uint32_t tmem_base;
   volatile int abort_flag;
 };
@@ -115,11 +119,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&S.empty[s], 1);
     }
     for (int a = 0; a < kAcc; ++a) {
-      mbar_init(&S.acc_full[a], 1);
+      mbar_init(&S.acc_full[a], kIssuers);
       mbar_init(&S.acc_empty[a], 4);
     }
     for (int k = 0; k < kQBufs; ++k) mbar_init(&S.q_full[k], 4);
-    mbar_init(&S.drain, 1);
+    for (int k = 0; k < kIssuers; ++k) mbar_init(&S.drain[k], 1);
     S.abort_flag = 0;
     fence_barrier_init();
   }
@@ -206,26 +210,34 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i = issued > kStages ? issued - kStages : 0; i < issued; ++i)
           (void)mbar_wait(&S.full[i % kStages], (i / kStages) & 1, kWaitLimitNs / 2);
       }
-    } else if (warp == 1) {
-      // ================= MMA issuer =================
-      // (the FP8 scan's issue loop: descriptors from one base, the query's
-      // only when the request changes, a unit count instead of the walker)
+    } else if (warp < kEpiWarp0) {
+      // ================= MMA issuers (lane 0 of warps 1, 2) =================
+      // A tensor-core instruction (MMA, scale copy or commit) costs its issuing
+      // thread tens of cycles whatever its size, and one thread issuing a
+      // unit's ten set the scan's pace: each of two threads issues one
+      // 128-row tile of every unit (two scale copies, two MMAs, one commit to
+      // the accumulator barrier, which completes on both).  Both walk the same
+      // units and segments and keep their own copy of the query's scales in
+      // tensor memory.  The issue loop of the FP8 scan otherwise: descriptors
+      // from one base, the query's only when the request changes, a unit
+      // count instead of the walker.
       if (lane == 0) {
+        const int h = warp - 1;   // this thread's tile of every unit
         TileIter it;
         it.init(S.prefix, B, t_begin);
         int seg = 0, cur_b = it.b;
         int left = S.prefix[cur_b + 1] - S.prefix[cur_b] - it.j;
+        const uint32_t sfb0 = tmem + kSfbCol + h * (kQBufs * 8);
         bool ok = mbar_wait(&S.q_full[0], 0, wait_ns);
         if (ok) {
           tc_fence_after();
 #pragma unroll
-          for (int kh = 0; kh < 2; ++kh)
-            tmem_cp_scales(tmem + kSfbCol + kh * 4, smem_u32(S.qscales[0] + kh * 512));
+          for (int kh = 0; kh < 2; ++kh) tmem_cp_scales(sfb0 + kh * 4, smem_u32(S.qscales[0] + kh * 512));
         }
-        const uint64_t adesc0 = sw64_kmajor_desc(smem_u32(S.tiles[0][0]));
-        const uint32_t scales0 = smem_u32(S.scales[0][0]);
+        const uint64_t adesc0 = sw64_kmajor_desc(smem_u32(S.tiles[0][h]));
+        const uint32_t scales0 = smem_u32(S.scales[0][h]);
         uint64_t bdesc = sw64_kmajor_desc(smem_u32(S.q[0]));
-        uint32_t sfb = tmem + kSfbCol;
+        uint32_t sfb = sfb0;
         int s = 0, a = 0;
         uint32_t ph_s = 0, ph_a = 0;
         for (int i = 0; ok && i < n_tiles; ++i) {
@@ -235,7 +247,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             ++seg;
             if (!mbar_wait(&S.q_full[seg % kQBufs], (seg / kQBufs) & 1, wait_ns)) { ok = false; break; }
             tc_fence_after();
-            sfb = tmem + kSfbCol + (seg % kQBufs) * 8;
+            sfb = sfb0 + (seg % kQBufs) * 8;
 #pragma unroll
             for (int kh = 0; kh < 2; ++kh)
               tmem_cp_scales(sfb + kh * 4, smem_u32(S.qscales[seg % kQBufs] + kh * 512));
@@ -248,21 +260,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           if (S.abort_flag) break;
           tc_fence_after();
+          const uint32_t sfa = tmem + kSfaCol + (2 * a + h) * 8;
+          const uint32_t sc = scales0 + static_cast<uint32_t>(s * 2 * kTileScaleBytes);
 #pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const uint32_t sfa = tmem + kSfaCol + (2 * a + h) * 8;
-            const uint32_t sc = scales0 + static_cast<uint32_t>((2 * s + h) * kTileScaleBytes);
+          for (int kh = 0; kh < 2; ++kh) tmem_cp_scales(sfa + kh * 4, sc + kh * 512);
+          // start-address field: bits 0..13 of the descriptor (address / 16)
+          const uint64_t adesc = adesc0 + static_cast<uint64_t>((s * 2 * kTileCodeBytes) >> 4);
 #pragma unroll
-            for (int kh = 0; kh < 2; ++kh) tmem_cp_scales(sfa + kh * 4, sc + kh * 512);
-            // start-address field: bits 0..13 of the descriptor (address / 16)
-            const uint64_t adesc = adesc0 + static_cast<uint64_t>(((2 * s + h) * kTileCodeBytes) >> 4);
-#pragma unroll
-            for (int kh = 0; kh < 2; ++kh)
-              umma_mxf4nvf4(tmem + (2 * a + h) * kAccCols, adesc + 2 * kh, bdesc + 2 * kh, kIdesc, sfa + kh * 4,
-                            sfb + kh * 4, kh > 0 ? 1u : 0u);
-          }
-          umma_commit(&S.empty[s]);
-          umma_commit(&S.acc_full[a]);
+          for (int kh = 0; kh < 2; ++kh)
+            umma_mxf4nvf4(tmem + (2 * a + h) * kAccCols, adesc + 2 * kh, bdesc + 2 * kh, kIdesc, sfa + kh * 4,
+                          sfb + kh * 4, kh > 0 ? 1u : 0u);
+          umma_commit(&S.acc_full[a]);   // the epilogue releases the stage once both tiles' MMAs are done
           if (++s == kStages) {
             s = 0;
             ph_s ^= 1u;
@@ -276,13 +284,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           report_error(cache.err_word, CSA2_ERR_TIMEOUT, kKIndexFull, cur_b, -1);
           S.abort_flag = 1;
         }
-        umma_commit(&S.drain);
-        (void)mbar_wait(&S.drain, 0, kWaitLimitNs);
+        umma_commit(&S.drain[h]);
+        (void)mbar_wait(&S.drain[h], 0, kWaitLimitNs);
       }
     } else {
-      // ================= epilogue groups (warps 2..5, 6..9) =================
-      const int group = (warp - 2) >> 2;
-      const int ew = (warp - 2) & 3;
+      // ================= epilogue groups (warps 3..6, 7..10) =================
+      const int group = (warp - kEpiWarp0) >> 2;
+      const int ew = (warp - kEpiWarp0) & 3;
       const int quarter = warp & 3;
       const int toff = quarter * 32 + lane;
       auto timed_out = [&](int where) {
@@ -336,6 +344,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           timed_out(j);
           break;
         }
+        // both tiles' MMAs (and scale copies) are complete: the stage is free
+        if (ew == 0 && lane == 0) mbar_arrive(&S.empty[i % kStages]);
         tc_fence_after();
         uint32_t acc0[32], acc1[32];
         tmem_ld_32x32b_x32(tmem + (2 * a) * kAccCols + (static_cast<uint32_t>(quarter * 32) << 16), acc0);
@@ -431,6 +441,8 @@ __global__ void __launch_bounds__(256) append_ik4_kernel(csa2_cache cache, uint8
 
 }  // namespace
 
+static_assert(sizeof(Fp4Smem) + 1024 <= 225 * 1024, "the FP4 scan's shared memory (plus the prefix sum's) exceeds one SM");
+static_assert(kSfbCol + kIssuers * kQBufs * 8 <= kTmemCols, "the FP4 scan's tensor-memory columns");
 size_t index_full_fp4_smem_bytes() { return sizeof(Fp4Smem) + 1024; }
 
 cudaError_t launch_index_full_fp4(const csa2_cache& cache, const uint8_t* ik4_scales, const float* q, const float* w,
