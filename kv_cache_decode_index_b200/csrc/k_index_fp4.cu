@@ -13,8 +13,9 @@
 // tile's scales reach tensor memory with one bulk copy and two tcgen05.cp.
 //
 // index_full_fp4_kernel follows the FP8 scan (one persistent CTA per SM,
-// 256-position units split into contiguous CTA ranges, TMA producer warp, two
-// epilogue warpgroups on alternate units), with:
+// 256-position units split into contiguous CTA ranges, two epilogue
+// warpgroups on alternate units), with:
+//   * two TMA producer warps, one for the even and one for the odd units;
 //   * stages of two 128-row code tiles (64-byte rows, 64-byte swizzle, 8 KB
 //     each) and their two 1 KB scale blocks: with pages of whole units, one
 //     256-row TMA load and one 2 KB bulk copy per unit (else one of each per
@@ -45,7 +46,8 @@ constexpr int kAcc = 4;                    // accumulator pairs
 constexpr int kEpiGroups = 2;
 constexpr int kQBufs = 3;
 constexpr int kIssuers = 2;                 // one per 128-row tile of a unit
-constexpr int kEpiWarp0 = 1 + kIssuers;    // first epilogue warp
+constexpr int kProducers = 2;               // warps 0 and 3: even and odd units
+constexpr int kEpiWarp0 = kProducers + kIssuers;   // first epilogue warp
 constexpr int kThreads = 32 * kEpiWarp0 + kEpiGroups * 128;
 constexpr int kMaxBatchScan = 1024;
 constexpr int kScanItems = (kMaxBatchScan + kThreads - 1) / kThreads;
@@ -65,7 +67,7 @@ struct __align__(1024) Fp4Smem {
   uint8_t q[kQBufs][kQCodeBytes];
   uint8_t qscales[kQBufs][kTileScaleBytes];
   uint32_t hist[2][kPoolHistBins / 2];
-  int rowq[32][2];                     // cache rows of the producer's current 32 units (-1: none)
+  int rowq[kProducers][32][2];         // cache rows of each producer's current 32 units (-1: none)
   int prefix[kMaxBatchScan + 1];
   uint64_t full[kStages];
   uint64_t empty[kStages];
@@ -155,25 +157,30 @@ __global__ void __launch_bounds__(kThreads, 1)
   const bool hist_smem = n_tiles < 2048;
 
   if (n_tiles > 0) {
-    if (warp == 0) {
-      // ================= producer =================
+    if (warp == 0 || warp == 3) {
+      // ================= producers (warps 0, 3) =================
+      // Each copies every other unit (the stages alternate with them: an even
+      // number of stages), from cache rows its warp resolved 32 units at a
+      // time (one unit per lane, the next 32 units' page-table loads in flight
+      // while lane 0 issues).
+      const int pr = warp == 0 ? 0 : 1;
       const uint64_t policy = l2_policy_evict_first();
       UnitRows next;   // this lane's unit of the next 32
-      next.fetch(cache, S.prefix, B, t_begin + lane, lane < n_tiles, capacity, page_size);
-      int issued = 0;   // lane 0
+      next.fetch(cache, S.prefix, B, t_begin + pr + 2 * lane, pr + 2 * lane < n_tiles, capacity, page_size);
+      int issued = 0;   // lane 0: own units
       bool stop = false;
-      for (int i0 = 0; i0 < n_tiles && !stop; i0 += 32) {
+      for (int i0 = 0; i0 < n_tiles && !stop; i0 += 64) {
         int r[2];
         next.rows(cache, capacity, kKIndexFull, r);
-        S.rowq[lane][0] = r[0];
-        S.rowq[lane][1] = r[1];
-        // the next 32 units' page-table loads are in flight while lane 0 issues
-        next.fetch(cache, S.prefix, B, t_begin + i0 + 32 + lane, i0 + 32 + lane < n_tiles, capacity, page_size);
+        S.rowq[pr][lane][0] = r[0];
+        S.rowq[pr][lane][1] = r[1];
+        const int g1 = i0 + 64 + pr + 2 * lane;
+        next.fetch(cache, S.prefix, B, t_begin + g1, g1 < n_tiles, capacity, page_size);
         __syncwarp();
         if (lane == 0) {
-          const int n = min(32, n_tiles - i0);
-          for (int k = 0; k < n; ++k) {
-            const int i = i0 + k, s = i % kStages;
+          for (int k = 0; k < 32; ++k) {
+            const int i = i0 + pr + 2 * k, s = i % kStages;
+            if (i >= n_tiles) break;
             if (!mbar_wait(&S.empty[s], ((i / kStages) & 1) ^ 1, wait_ns)) {
               report_error(cache.err_word, CSA2_ERR_TIMEOUT, kKIndexFull, -1, i);
               S.abort_flag = 1;
@@ -182,7 +189,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               stop = true;
               break;
             }
-            const int r0 = S.rowq[k][0], r1 = S.rowq[k][1];
+            const int r0 = S.rowq[pr][k][0], r1 = S.rowq[pr][k][1];
             // a tile's scale block is 1 KB at (row / 128) KB: 16-byte aligned
             if (whole_units && r0 >= 0) {   // the unit's 256 rows and two scale blocks are consecutive
               mbar_arrive_expect_tx(&S.full[s], 2 * (kTileCodeBytes + kTileScaleBytes));
@@ -206,9 +213,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
       }
       if (lane == 0) {
-        // copies still in flight (only after an abort): wait for the last one of each stage
-        for (int i = issued > kStages ? issued - kStages : 0; i < issued; ++i)
+        // copies still in flight (only after an abort): wait for the last one of each own stage
+        for (int m = issued > kStages / 2 ? issued - kStages / 2 : 0; m < issued; ++m) {
+          const int i = pr + 2 * m;
           (void)mbar_wait(&S.full[i % kStages], (i / kStages) & 1, kWaitLimitNs / 2);
+        }
       }
     } else if (warp < kEpiWarp0) {
       // ================= MMA issuers (lane 0 of warps 1, 2) =================
@@ -288,7 +297,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         (void)mbar_wait(&S.drain[h], 0, kWaitLimitNs);
       }
     } else {
-      // ================= epilogue groups (warps 3..6, 7..10) =================
+      // ================= epilogue groups (warps 4..7, 8..11) =================
       const int group = (warp - kEpiWarp0) >> 2;
       const int ew = (warp - kEpiWarp0) & 3;
       const int quarter = warp & 3;
@@ -311,9 +320,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         prep_b = next_request_with_tiles(S.prefix, B, prep_b);
         ++prep_x;
       };
+      // This group's units: a counter walk over (request, unit) two units at
+      // a time; `seg` counts the request segments passed.
       TileIter it;
       it.init(S.prefix, B, t_begin);
-      int seg = 0, cur_b = it.b;
+      int seg = 0, cur_b = it.b, j = it.j;
+      int units_b = S.prefix[cur_b + 1] - S.prefix[cur_b];
+      auto step = [&](int d) {
+        j += d;
+        while (j >= units_b) {
+          j -= units_b;
+          cur_b = next_request_with_tiles(S.prefix, B, cur_b);
+          if (cur_b >= B) break;   // past this CTA's last unit
+          units_b = S.prefix[cur_b + 1] - S.prefix[cur_b];
+          ++seg;
+        }
+      };
       if (group == 0) {
         prep_b = cur_b;
         for (int k = 0; k < kQBufs && prep_b < B && S.prefix[prep_b] < t_end; ++k) prepare();
@@ -324,22 +346,16 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int h = 0; h < 32; ++h) ws[h] = __shfl_sync(0xffffffffu, wl, h);
       };
-      load_w(cur_b);
-      int nb = cache.ctx_len[cur_b];
-      if (group == 1) it.advance();
+      if (group == 1) step(1);
+      int w_b = -1, nb = 0;   // the request whose weights and length are loaded
 
       for (int i = group; i < n_tiles; i += kEpiGroups) {
-        if (it.b != cur_b) {
-          for (int b = cur_b; b != it.b; b = next_request_with_tiles(S.prefix, B, b)) ++seg;
-          cur_b = it.b;
+        if (cur_b != w_b) {
+          w_b = cur_b;
           load_w(cur_b);
           nb = cache.ctx_len[cur_b];
         }
         const int a = i % kAcc;
-        const int j = it.j;
-        TileIter nx = it;
-        nx.advance();
-        nx.advance();
         if (!mbar_wait_warp(&S.acc_full[a], (i / kAcc) & 1, wait_ns)) {
           timed_out(j);
           break;
@@ -361,31 +377,46 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (group == 0)
           while (prep_x <= seg + 2 && prep_b < B && S.prefix[prep_b] < t_end) prepare();
 
+        // both tiles' sums side by side (each in head order, as the re-score)
+        float sc[2] = {0.0f, 0.0f};
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const int p = j * kUnit + h * kTile + toff;
-          const bool valid = p < nb;
-          const uint32_t(&acc)[32] = h == 0 ? acc0 : acc1;
-          float sc = 0.0f;
+        for (int hh = 0; hh < 32; ++hh) {
+          sc[0] = fmaf(ws[hh], fmaxf(__uint_as_float(acc0[hh]), 0.0f), sc[0]);
+          sc[1] = fmaf(ws[hh], fmaxf(__uint_as_float(acc1[hh]), 0.0f), sc[1]);
+        }
+        const int p0 = j * kUnit + toff;
+        float bm[2];
 #pragma unroll
-          for (int hh = 0; hh < 32; ++hh) sc = fmaf(ws[hh], fmaxf(__uint_as_float(acc[hh]), 0.0f), sc);
-          float bm = valid ? sc : -INFINITY;
-          bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 1));
-          bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 2));
-          bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 4));
-          if ((lane & 7) == 0 && valid) {
-            blockmax[static_cast<long long>(cur_b) * (capacity / kBlock) + p / kBlock] = bm;
+        for (int h = 0; h < 2; ++h) bm[h] = p0 + h * kTile < nb ? sc[h] : -INFINITY;
+#pragma unroll
+        for (int d = 1; d < 8; d <<= 1) {
+          const float o0 = __shfl_xor_sync(0xffffffffu, bm[0], d);
+          const float o1 = __shfl_xor_sync(0xffffffffu, bm[1], d);
+          bm[0] = fmaxf(bm[0], o0);
+          bm[1] = fmaxf(bm[1], o1);
+        }
+        if ((lane & 7) == 0) {
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int p = p0 + h * kTile;
+            if (p >= nb) continue;
+            blockmax[static_cast<long long>(cur_b) * (capacity / kBlock) + p / kBlock] = bm[h];
             if (hist != nullptr) {
-              const uint32_t bin = order_key(bm) >> (32 - kPoolHistBits);
+              const uint32_t bin = order_key(bm[h]) >> (32 - kPoolHistBits);
               const int slot = cur_b - hist_b0;
               if (hist_smem && slot < 2) atomicAdd(&S.hist[slot][bin >> 1], 1u << (16 * (bin & 1)));
               else atomicAdd(&hist[static_cast<long long>(cur_b) * kPoolHistBins + bin], 1u);
             }
           }
-          if (scores != nullptr && valid) scores[static_cast<long long>(cur_b) * capacity + p] = sc;
         }
-        if (warp_flag(&S.abort_flag)) break;
-        it = nx;
+        if (scores != nullptr) {
+#pragma unroll
+          for (int h = 0; h < 2; ++h)
+            if (p0 + h * kTile < nb) scores[static_cast<long long>(cur_b) * capacity + p0 + h * kTile] = sc[h];
+        }
+        // another role's time-out (every 8th unit: the waits above are bounded anyway)
+        if ((i & (8 * kEpiGroups - 1)) < kEpiGroups && warp_flag(&S.abort_flag)) break;
+        step(kEpiGroups);
       }
     }
   }
@@ -441,6 +472,7 @@ __global__ void __launch_bounds__(256) append_ik4_kernel(csa2_cache cache, uint8
 
 }  // namespace
 
+static_assert(kStages % kProducers == 0, "each producer keeps to its own stages");
 static_assert(sizeof(Fp4Smem) + 1024 <= 225 * 1024, "the FP4 scan's shared memory (plus the prefix sum's) exceeds one SM");
 static_assert(kSfbCol + kIssuers * kQBufs * 8 <= kTmemCols, "the FP4 scan's tensor-memory columns");
 size_t index_full_fp4_smem_bytes() { return sizeof(Fp4Smem) + 1024; }
