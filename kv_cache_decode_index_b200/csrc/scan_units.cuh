@@ -56,6 +56,7 @@ struct UnitRows {
   int p0;        // first position of the unit
   int pidx;      // page index of tile 0
   int page[2];   // page-table entries (page[1] = -2: tile 1 is on tile 0's page, or absent)
+  int n;         // the request's visible positions (a page-table slot past them need not be valid)
 
   // Unit g (global index among all units; g < prefix[batch] or the slot is
   // empty).  Positions are below 2^31 (checked on the host): 32-bit
@@ -72,6 +73,7 @@ struct UnitRows {
       else hi = mid - 1;
     }
     b = lo;
+    n = cache.ctx_len[lo];   // in flight with the page-table loads
     p0 = (g - prefix[lo]) * kScanUnit;
     pidx = static_cast<int>(static_cast<uint32_t>(p0) / page_size);
     const int32_t* pt = cache.page_table + static_cast<long long>(lo) * cache.max_pages_per_req;
@@ -81,7 +83,8 @@ struct UnitRows {
                                                                                                       : -2;
   }
 
-  // r[h]: cache row of tile h, or -1 past the request's capacity.  A page id
+  // r[h]: cache row of tile h, or -1 when the tile starts past the request's
+  // visible positions (its page-table slot need not hold a page).  A page id
   // outside [0, num_pages) is reported (CSA2_ERR_DEVICE_BOUNDS) and replaced
   // by page 0, so that the copy stays in bounds; the results of that tile
   // are flagged invalid by the report.
@@ -91,7 +94,7 @@ struct UnitRows {
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
       const int p = p0 + h * kTile;
-      if (p >= capacity) continue;
+      if (p >= capacity || p >= n) continue;
       const bool own_page = h == 1 && page[1] != -2;
       int pg = own_page ? page[1] : page[0];
       if (pg < 0 || pg >= cache.num_pages) {

@@ -195,10 +195,15 @@ def _score_bound(q, w, codes, exp):
 MANY_SHORT = [int(n) for n in np.random.default_rng(77).integers(1, 1100, size=600)]
 
 
-@pytest.mark.parametrize("lengths", [[4096, 1, 1000, 9999, 128 * 37], MANY_SHORT], ids=["five", "many_short"])
-def test_index_full_scores_ragged(csa2, lengths):
+# Pages of 128 or 384 rows: a unit's two tiles on two pages (or the second
+# absent), copied tile by tile instead of in one 256-row box.
+@pytest.mark.parametrize("lengths,page_size", [([4096, 1, 1000, 9999, 128 * 37], 512), (MANY_SHORT, 512),
+                                               ([4096, 1, 1000, 9999, 128 * 37], 128),
+                                               ([4096, 1, 1000, 9999, 128 * 37], 384)],
+                         ids=["five", "many_short", "five_page128", "five_page384"])
+def test_index_full_scores_ragged(csa2, lengths, page_size):
     B = len(lengths)
-    wl = W.scaled(W.WORKLOADS["group_64k_b8"], batch=B, page_size=512, shuffle_pages=True)
+    wl = W.scaled(W.WORKLOADS["group_64k_b8"], batch=B, page_size=page_size, shuffle_pages=True)
     cache = U.build_cache(wl, csa2, lengths=lengths)
     q, w = W.index_query(wl, 0)
     dev = cache.device
