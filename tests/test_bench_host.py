@@ -1,6 +1,7 @@
 """Host-side logic of bench.py, on CPU: algorithmic bytes, I/O bytes, clock
 parsing, per-rank workloads, the max-over-ranks reduction across 2 gloo ranks,
-and the reference arm's JSON line on a small workload."""
+the reference arm's JSON line on a small workload, and the keying of the
+reported DRAM traffic to the scan's source."""
 import io
 import json
 import os
@@ -176,3 +177,38 @@ def test_fp4_oracle_sample_runs_small():
     assert bench.oracle_sample_fp4(wl, 0) > 0
     step, scan = bench.alg_bytes(wl, ik_row_bytes=bench.IK4_ROW_BYTES)
     assert scan == 72 * 8192 * wl.batch
+
+
+def _fake_tree(root, fp4):
+    """A copy of the scan's source files under `root` (for the source hash)."""
+    src = os.path.join(os.path.dirname(bench.__file__), "kv_cache_decode_index_b200", "csrc")
+    dst = os.path.join(root, "kv_cache_decode_index_b200", "csrc")
+    os.makedirs(dst, exist_ok=True)
+    names = ("k_index_fp4.cu", "fp4.cuh") if fp4 else ("k_index.cu", "index_common.cuh")
+    for name in names + ("scan_units.cuh", "common.cuh"):
+        with open(os.path.join(src, name), "rb") as f, open(os.path.join(dst, name), "wb") as g:
+            g.write(f.read())
+    os.makedirs(os.path.join(root, "profiles"), exist_ok=True)
+
+
+def test_scan_traffic_is_keyed_to_the_kernel_source(monkeypatch, tmp_path):
+    """The reported DRAM traffic comes from the committed ncu summary only
+    while the scan's sources hash to the value it was captured on, and only
+    for its workload: any edit of those sources (a comment too) drops it."""
+    for fp4 in (False, True):
+        root = str(tmp_path / ("fp4" if fp4 else "fp8"))
+        _fake_tree(root, fp4)
+        monkeypatch.setattr(bench, "ROOT", root)
+        name = "index_full_fp4_traffic.txt" if fp4 else "index_full_traffic.txt"
+        path = os.path.join(root, "profiles", name)
+        with open(path, "w") as f:
+            f.write(f"kernel_source_hash: {bench.scan_kernel_hash(fp4)}\nworkload: group_1m_b4\n"
+                    "dram_bytes_per_launch: 123456\n")
+        assert bench.scan_traffic_per_launch("group_1m_b4", fp4) == 123456.0
+        assert bench.scan_traffic_per_launch("group_64k_b8", fp4) is None
+        src = os.path.join(root, "kv_cache_decode_index_b200", "csrc", "scan_units.cuh")
+        with open(src, "a") as f:
+            f.write("// edited\n")
+        assert bench.scan_traffic_per_launch("group_1m_b4", fp4) is None
+        os.remove(path)
+        assert bench.scan_traffic_per_launch("group_1m_b4", fp4) is None
